@@ -1,0 +1,191 @@
+/*
+ * rtq.h -- C ABI of the B200 weight-only quantized projection GEMM.
+ *
+ * The operation (both RT-J quantized model cards, opening paragraph): a
+ * transformer-block projection Y[M,N] = X[M,K] * W[N,K]^T whose weights stay
+ * quantized in device memory and are dequantized inside the GEMM, so the only
+ * weight traffic is the quantized payload.  Two weight formats:
+ *
+ *   q4  ("RT-J -- int4 (Q4-style, mixed-precision) quantized checkpoints",
+ *       section "Quantization format"): uint4 codes in groups of 32 along the
+ *       input dimension K, packed two per byte with the LOW nibble holding the
+ *       EVEN index; one fp16 (scale, min) pair per group;
+ *       W[o,k] = code(o,k) * scale[o,k/32] + min[o,k/32].
+ *         Wq        uint8  [N, K/2], row-major
+ *         scale_min uint16 [N, K/32, 2], binary16 bits, element 0 = scale,
+ *                   element 1 = min (the pages give a "(scale, min) pair per
+ *                   group" in one companion tensor; the interleaved order is
+ *                   this library's reading)
+ *
+ *   q8  ("RT-J -- int8 (Q8_0-style) quantized checkpoints", section
+ *       "Quantization format"): int8 codes with one symmetric fp32 scale per
+ *       output row; W[o,k] = q[o,k] * scale[o], scale[o] = max|W[o,:]|/127.
+ *         Wq    int8  [N, K], row-major
+ *         scale float [N]
+ *
+ * Activations X are fp32 [M, K] row-major and results Y are fp32 [M, N]
+ * row-major.  There is no bias term (the cards keep biases in fp32 outside
+ * the quantized projections).
+ *
+ * Conventions for every GEMM entry point:
+ *   - Ownership: the caller allocates and owns every buffer.  The library
+ *     never allocates per call and never frees caller memory.
+ *   - Pointers: X, Wq, scale(_min) and Y are DEVICE pointers on the current
+ *     device; `stream` is a cudaStream_t (NULL = legacy default stream).
+ *   - Execution: stream-ordered and asynchronous.  RT_OK means "validated and
+ *     enqueued".  Errors raised later on the device (a bounded wait that gave
+ *     up) are latched in a device status word read by rt_device_status().
+ *   - Alignment: X, Y and Wq 16-byte aligned; scale_min 4-byte aligned; scale
+ *     4-byte aligned.  Otherwise RT_ERR_ALIGNMENT.
+ *   - Shapes: M >= 0 (M == 0 is a no-op), N >= 1, K >= 1; q4 needs K % 32 == 0
+ *     (the group size); q8 needs K % 16 == 0.  The tensor-core path also needs
+ *     K % 64 == 0; RT_PATH_AUTO falls back to the SIMT path otherwise and an
+ *     explicit RT_PATH_TC returns RT_ERR_UNSUPPORTED_SHAPE.
+ *   - Aliasing: Y must not overlap X, Wq or the scales (RT_ERR_INVALID_ARG).
+ *   - No C++ exception crosses this boundary.
+ *   - Precision: the SIMT path dequantizes to fp32 and accumulates in fp32
+ *     (max|Y - Y_exact| / max|Y_exact| <= 1e-5).  The tensor-core path rounds
+ *     X and the dequantized q4 weights (their fp32 value) to fp16 -- q8 codes
+ *     are exact, their row scale is applied in fp32 after the MMA -- and
+ *     accumulates in fp32 in TMEM (<= 4e-3; about 3e-4 on N(0,1) activations).
+ *     fp16 operands need |X| <= 65504 (larger activations become infinite);
+ *     RT_PATH_TC_BF16 runs the same kernels on bf16 operands, which keep the
+ *     fp32 range but only 8 significant bits (about 2e-3 to 5e-3).
+ */
+#ifndef RTQ_H
+#define RTQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum rt_status {
+    RT_OK = 0,
+    RT_ERR_INVALID_ARG = 1,       /* null pointer, negative size, overlap, bad n_grid */
+    RT_ERR_ALIGNMENT = 2,         /* a pointer misses the alignment stated above */
+    RT_ERR_UNSUPPORTED_SHAPE = 3, /* K not a multiple of the format's granule */
+    RT_ERR_CUDA = 4,              /* a CUDA runtime call failed (launch, no device) */
+    RT_ERR_DEVICE_TIMEOUT = 5,    /* a kernel's bounded wait expired (see rt_device_status) */
+    RT_ERR_VALUE_RANGE = 6        /* quantizer input not finite / outside binary16 range */
+} rt_status;
+
+typedef enum rt_path {
+    RT_PATH_AUTO = 0,   /* SIMT for M <= 8 or K % 64 != 0, else TC */
+    RT_PATH_SIMT = 1,   /* fp32 CUDA-core kernels */
+    RT_PATH_TC = 2,     /* tcgen05 tensor-core kernels, fp16 operands, fp32 accumulate in TMEM */
+    RT_PATH_TC_BF16 = 3 /* the same kernels with bf16 operands */
+} rt_path;
+
+/* Human-readable name of a status code; never NULL. */
+const char *rt_status_string(int status);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int rt_version(void);
+
+/*
+ * Y = X * dequant_q4(Wq, scale_min)^T.   (int4 card, "Quantization format")
+ * X [M,K] fp32, Wq [N,K/2] u8, scale_min [N,K/32,2] binary16, Y [M,N] fp32.
+ */
+rt_status rt_qgemm_q4(const float *X, const uint8_t *Wq, const uint16_t *scale_min, float *Y,
+                      int64_t M, int64_t N, int64_t K, int path, void *stream);
+
+/*
+ * Y = X * dequant_q8(Wq, scale)^T.   (int8 card, "Quantization format")
+ * X [M,K] fp32, Wq [N,K] i8, scale [N] fp32, Y [M,N] fp32.
+ */
+rt_status rt_qgemm_q8(const float *X, const int8_t *Wq, const float *scale, float *Y,
+                      int64_t M, int64_t N, int64_t K, int path, void *stream);
+
+/* Which path RT_PATH_AUTO takes for a q4 (fmt = 4) or q8 (fmt = 8) GEMM of
+ * this shape: RT_PATH_SIMT or RT_PATH_TC; -1 for an unsupported shape. */
+int rt_qgemm_auto_path(int fmt, int64_t M, int64_t N, int64_t K);
+
+/*
+ * One RT-J block's quantized projection set, following the mixed-precision
+ * recipe of the int4 card ("Quantization format": wq/wk/wv/wg and ffn.w1/w3
+ * in q4 g32, the residual-writing wo and ffn.w2 in q8 per-row):
+ *   qkvg : q4, N = 4*d_model, K = d_model  (rows wq | wk | wv | wg)
+ *   wo   : q8, N = d_model,   K = d_model
+ *   w13  : q4, N = 2*d_ff,    K = d_model  (rows w1 | w3)
+ *   w2   : q8, N = d_model,   K = d_ff
+ * All pointers are device pointers.  The four products are independent (each
+ * reads its own input) and are enqueued on `stream` in the order qkvg, wo,
+ * w13, w2.  Y_qkvg [M, 4*d_model], Y_o [M, d_model], Y_13 [M, 2*d_ff],
+ * Y_2 [M, d_model].  The same validation as rt_qgemm_q4/q8 applies to each.
+ */
+typedef struct rt_qblock {
+    const uint8_t *qkvg;   const uint16_t *qkvg_sm;
+    const int8_t *wo;      const float *wo_s;
+    const uint8_t *w13;    const uint16_t *w13_sm;
+    const int8_t *w2;      const float *w2_s;
+    int64_t d_model;
+    int64_t d_ff;
+} rt_qblock;
+
+rt_status rt_qblock_project(const rt_qblock *blk, int64_t M,
+                            const float *X_qkvg, const float *X_o, const float *X_ffn,
+                            const float *X_w2, float *Y_qkvg, float *Y_o, float *Y_13,
+                            float *Y_2, int path, void *stream);
+
+/*
+ * Host-side quantizers (HOST pointers, caller-allocated outputs, synchronous,
+ * deterministic, thread-safe; several threads may work inside one call).
+ *
+ * rt_quantize_q4_g32 (int4 card, "Quantization format": min-MSE clip search
+ * over the shrink grid 1.0 -> 0.8): for each row and group of 32, try the
+ * n_grid shrink factors s_j = 1 - 0.2*j/(n_grid-1) (n_grid = 0 selects 21),
+ * take (scale, min) = binary16((s_j*hi - s_j*lo)/15), binary16(s_j*lo) with
+ * lo/hi the group's min/max, codes = clamp(round-half-even((w - min)/scale),
+ * 0, 15) (all zero when the scale rounds to 0), keep the j of least squared
+ * reconstruction error (smallest j on ties), pack the codes.
+ * W fp32 [N,K] -> Wq u8 [N,K/2], scale_min binary16 [N,K/32,2].
+ * Errors: RT_ERR_INVALID_ARG (null, negative size, n_grid < 0),
+ * RT_ERR_UNSUPPORTED_SHAPE (K % 32), RT_ERR_VALUE_RANGE (a weight is not
+ * finite or |w| > 65504).
+ */
+rt_status rt_quantize_q4_g32(const float *W, int64_t N, int64_t K, int n_grid,
+                             uint8_t *Wq, uint16_t *scale_min);
+
+/*
+ * rt_quantize_q8_row (int8 card, "Quantization format"): scale[o] =
+ * max|W[o,:]| / 127 (one fp32 division), q = clamp(round-half-even(w /
+ * scale), -127, 127); a zero row gets scale 0 and zero codes.
+ * W fp32 [N,K] -> Wq i8 [N,K], scale fp32 [N].  Errors: RT_ERR_INVALID_ARG,
+ * RT_ERR_VALUE_RANGE (a weight is not finite).
+ */
+rt_status rt_quantize_q8_row(const float *W, int64_t N, int64_t K, int8_t *Wq, float *scale);
+
+/*
+ * Dequantization exports (device pointers, stream-ordered).  They run the
+ * same __device__ dequantization routines the GEMM kernels use, so tests can
+ * check them bit for bit:
+ *   *_f32  : W[o,k] rounded once to fp32 (the SIMT path's operand);
+ *   q4_f16 : the fp32 value rounded again to fp16, stored as uint16 bits (the
+ *            tensor-core path's q4 operand);
+ *   q4_bf16: the same rounded to bf16 (the RT_PATH_TC_BF16 operand).
+ * W_out is [N,K].  Same alignment and shape rules as the GEMMs.
+ */
+rt_status rt_dequant_q4_f32(const uint8_t *Wq, const uint16_t *scale_min, float *W_out,
+                            int64_t N, int64_t K, void *stream);
+rt_status rt_dequant_q8_f32(const int8_t *Wq, const float *scale, float *W_out,
+                            int64_t N, int64_t K, void *stream);
+rt_status rt_dequant_q4_f16(const uint8_t *Wq, const uint16_t *scale_min, uint16_t *W_out,
+                            int64_t N, int64_t K, void *stream);
+rt_status rt_dequant_q4_bf16(const uint8_t *Wq, const uint16_t *scale_min, uint16_t *W_out,
+                             int64_t N, int64_t K, void *stream);
+
+/*
+ * Synchronizes `stream`, then reads and clears the device status word that
+ * kernels latch when one of their bounded waits gives up.  *device_status
+ * receives RT_OK or RT_ERR_DEVICE_TIMEOUT.  Returns RT_ERR_CUDA if the
+ * synchronization itself fails.
+ */
+rt_status rt_device_status(void *stream, int *device_status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RTQ_H */

@@ -1,0 +1,303 @@
+"""Python binding of librtq.so, the B200 weight-only quantized projection GEMM.
+
+The functions named ``rt_*`` mirror the C ABI in include/rtq.h one to one and
+only marshal arguments (raw pointers and sizes).  The helpers without the
+prefix take torch tensors (device memory and streams are PyTorch's; every step
+of the computation runs in the library's CUDA kernels) or numpy arrays (the
+host quantizers) and raise :class:`RtqError` on any non-OK status.
+
+There is no fallback: if librtq.so is missing or fails to load, every call
+raises.  Build it with ``python -m int8_dequant_gemm_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import numpy as np
+
+__all__ = [
+    "RtqError", "lib", "PATHS", "OK", "qgemm_q4", "qgemm_q8", "qblock_project", "QBlock",
+    "quantize_q4_g32", "quantize_q8_row", "dequant_q4_f32", "dequant_q8_f32",
+    "dequant_q4_bf16", "dequant_q4_f16", "device_status", "auto_path", "status_string",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librtq.so")
+
+OK = 0
+RT_ERR_DEVICE_TIMEOUT = 5
+PATHS = {"auto": 0, "simt": 1, "tc": 2, "tc_bf16": 3}
+
+_p = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_i32 = ctypes.c_int
+_lib = None
+
+
+class RtqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class _QBlockC(ctypes.Structure):
+    _fields_ = [("qkvg", _p), ("qkvg_sm", _p), ("wo", _p), ("wo_s", _p), ("w13", _p),
+                ("w13_sm", _p), ("w2", _p), ("w2_s", _p), ("d_model", _i64), ("d_ff", _i64)]
+
+
+def lib() -> ctypes.CDLL:
+    """Loads librtq.so once; raises if it is not built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is not built; run `python -m int8_dequant_gemm_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    L.rt_status_string.restype = ctypes.c_char_p
+    L.rt_status_string.argtypes = [_i32]
+    L.rt_version.restype = _i32
+    L.rt_version.argtypes = []
+    for name in ("rt_qgemm_q4", "rt_qgemm_q8"):
+        f = getattr(L, name)
+        f.restype = _i32
+        f.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _i32, _p]
+    L.rt_qgemm_auto_path.restype = _i32
+    L.rt_qgemm_auto_path.argtypes = [_i32, _i64, _i64, _i64]
+    L.rt_qblock_project.restype = _i32
+    L.rt_qblock_project.argtypes = [ctypes.POINTER(_QBlockC), _i64, _p, _p, _p, _p, _p, _p, _p,
+                                    _p, _i32, _p]
+    L.rt_quantize_q4_g32.restype = _i32
+    L.rt_quantize_q4_g32.argtypes = [_p, _i64, _i64, _i32, _p, _p]
+    L.rt_quantize_q8_row.restype = _i32
+    L.rt_quantize_q8_row.argtypes = [_p, _i64, _i64, _p, _p]
+    for name in ("rt_dequant_q4_f32", "rt_dequant_q8_f32", "rt_dequant_q4_bf16",
+                 "rt_dequant_q4_f16"):
+        f = getattr(L, name)
+        f.restype = _i32
+        f.argtypes = [_p, _p, _p, _i64, _i64, _p]
+    L.rt_device_status.restype = _i32
+    L.rt_device_status.argtypes = [_p, ctypes.POINTER(_i32)]
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return lib().rt_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        raise RtqError(status, where)
+
+
+# ----------------------------------------------------------------- raw ABI
+def rt_qgemm_q4(X, Wq, scale_min, Y, M, N, K, path, stream) -> int:
+    return lib().rt_qgemm_q4(X, Wq, scale_min, Y, M, N, K, path, stream)
+
+
+def rt_qgemm_q8(X, Wq, scale, Y, M, N, K, path, stream) -> int:
+    return lib().rt_qgemm_q8(X, Wq, scale, Y, M, N, K, path, stream)
+
+
+def rt_qblock_project(blk, M, X_qkvg, X_o, X_ffn, X_w2, Y_qkvg, Y_o, Y_13, Y_2, path,
+                      stream) -> int:
+    return lib().rt_qblock_project(ctypes.byref(blk), M, X_qkvg, X_o, X_ffn, X_w2, Y_qkvg, Y_o,
+                                   Y_13, Y_2, path, stream)
+
+
+def rt_quantize_q4_g32(W, N, K, n_grid, Wq, scale_min) -> int:
+    return lib().rt_quantize_q4_g32(W, N, K, n_grid, Wq, scale_min)
+
+
+def rt_quantize_q8_row(W, N, K, Wq, scale) -> int:
+    return lib().rt_quantize_q8_row(W, N, K, Wq, scale)
+
+
+def rt_dequant_q4_f32(Wq, scale_min, W_out, N, K, stream) -> int:
+    return lib().rt_dequant_q4_f32(Wq, scale_min, W_out, N, K, stream)
+
+
+def rt_dequant_q8_f32(Wq, scale, W_out, N, K, stream) -> int:
+    return lib().rt_dequant_q8_f32(Wq, scale, W_out, N, K, stream)
+
+
+def rt_dequant_q4_bf16(Wq, scale_min, W_out, N, K, stream) -> int:
+    return lib().rt_dequant_q4_bf16(Wq, scale_min, W_out, N, K, stream)
+
+
+def rt_dequant_q4_f16(Wq, scale_min, W_out, N, K, stream) -> int:
+    return lib().rt_dequant_q4_f16(Wq, scale_min, W_out, N, K, stream)
+
+
+def rt_device_status(stream, out) -> int:
+    return lib().rt_device_status(stream, out)
+
+
+def rt_qgemm_auto_path(fmt, M, N, K) -> int:
+    return lib().rt_qgemm_auto_path(fmt, M, N, K)
+
+
+# ------------------------------------------------------- torch-level helpers
+def _stream_ptr(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev(t, dtype, name):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _path(path) -> int:
+    return PATHS[path] if isinstance(path, str) else int(path)
+
+
+def qgemm_q4(X, Wq, scale_min, Y=None, path="auto", stream=None):
+    """Y[M,N] = X[M,K] @ dequant_q4(Wq[N,K/2], scale_min[N,K/32,2])^T on the GPU."""
+    import torch
+    M, K = X.shape
+    N = Wq.shape[0]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float32, device=X.device)
+    st = rt_qgemm_q4(_dev(X, torch.float32, "X"), _dev(Wq, torch.uint8, "Wq"),
+                     _dev(scale_min, torch.uint16, "scale_min"), _dev(Y, torch.float32, "Y"),
+                     M, N, K, _path(path), _stream_ptr(stream))
+    _check(st, "rt_qgemm_q4")
+    return Y
+
+
+def qgemm_q8(X, Wq, scale, Y=None, path="auto", stream=None):
+    """Y[M,N] = X[M,K] @ (Wq[N,K] * scale[N,None])^T on the GPU."""
+    import torch
+    M, K = X.shape
+    N = Wq.shape[0]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float32, device=X.device)
+    st = rt_qgemm_q8(_dev(X, torch.float32, "X"), _dev(Wq, torch.int8, "Wq"),
+                     _dev(scale, torch.float32, "scale"), _dev(Y, torch.float32, "Y"),
+                     M, N, K, _path(path), _stream_ptr(stream))
+    _check(st, "rt_qgemm_q8")
+    return Y
+
+
+@dataclass
+class QBlock:
+    """Device tensors of one block's packed projections (see rt_qblock in rtq.h)."""
+    qkvg: object
+    qkvg_sm: object
+    wo: object
+    wo_s: object
+    w13: object
+    w13_sm: object
+    w2: object
+    w2_s: object
+    d_model: int = 512
+    d_ff: int = 2048
+
+    def as_c(self) -> _QBlockC:
+        import torch
+        return _QBlockC(_dev(self.qkvg, torch.uint8, "qkvg"),
+                        _dev(self.qkvg_sm, torch.uint16, "qkvg_sm"),
+                        _dev(self.wo, torch.int8, "wo"), _dev(self.wo_s, torch.float32, "wo_s"),
+                        _dev(self.w13, torch.uint8, "w13"),
+                        _dev(self.w13_sm, torch.uint16, "w13_sm"),
+                        _dev(self.w2, torch.int8, "w2"), _dev(self.w2_s, torch.float32, "w2_s"),
+                        self.d_model, self.d_ff)
+
+
+def qblock_project(block: QBlock, X_qkvg, X_o, X_ffn, X_w2, Y_qkvg, Y_o, Y_13, Y_2,
+                   path="auto", stream=None, block_c=None):
+    """Runs one block's four quantized projections (qkvg, wo, w13, w2)."""
+    import torch
+    M = X_qkvg.shape[0]
+    bc = block_c if block_c is not None else block.as_c()
+    args = [_dev(t, torch.float32, n) for t, n in
+            ((X_qkvg, "X_qkvg"), (X_o, "X_o"), (X_ffn, "X_ffn"), (X_w2, "X_w2"),
+             (Y_qkvg, "Y_qkvg"), (Y_o, "Y_o"), (Y_13, "Y_13"), (Y_2, "Y_2"))]
+    st = rt_qblock_project(bc, M, *args, _path(path), _stream_ptr(stream))
+    _check(st, "rt_qblock_project")
+
+
+def quantize_q4_g32(W: np.ndarray, n_grid: int = 21):
+    """Host min-MSE g32 quantizer: (Wq uint8 [N,K/2], scale_min uint16 [N,K/32,2])."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    Wq = np.empty((N, K // 2), dtype=np.uint8)
+    sm = np.empty((N, K // 32, 2), dtype=np.uint16)
+    st = rt_quantize_q4_g32(W.ctypes.data, N, K, n_grid, Wq.ctypes.data, sm.ctypes.data)
+    _check(st, "rt_quantize_q4_g32")
+    return Wq, sm
+
+
+def quantize_q8_row(W: np.ndarray):
+    """Host per-row int8 quantizer: (Wq int8 [N,K], scale float32 [N])."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    Wq = np.empty((N, K), dtype=np.int8)
+    sc = np.empty((N,), dtype=np.float32)
+    st = rt_quantize_q8_row(W.ctypes.data, N, K, Wq.ctypes.data, sc.ctypes.data)
+    _check(st, "rt_quantize_q8_row")
+    return Wq, sc
+
+
+def dequant_q4_f32(Wq, scale_min, stream=None):
+    import torch
+    N, K2 = Wq.shape
+    out = torch.empty((N, 2 * K2), dtype=torch.float32, device=Wq.device)
+    st = rt_dequant_q4_f32(_dev(Wq, torch.uint8, "Wq"), _dev(scale_min, torch.uint16, "scale_min"),
+                           _dev(out, torch.float32, "W_out"), N, 2 * K2, _stream_ptr(stream))
+    _check(st, "rt_dequant_q4_f32")
+    return out
+
+
+def dequant_q4_bf16(Wq, scale_min, stream=None):
+    """bf16 rendering of the q4 weights as uint16 bits [N, K]."""
+    import torch
+    N, K2 = Wq.shape
+    out = torch.empty((N, 2 * K2), dtype=torch.uint16, device=Wq.device)
+    st = rt_dequant_q4_bf16(_dev(Wq, torch.uint8, "Wq"), _dev(scale_min, torch.uint16, "scale_min"),
+                            _dev(out, torch.uint16, "W_out"), N, 2 * K2, _stream_ptr(stream))
+    _check(st, "rt_dequant_q4_bf16")
+    return out
+
+
+def dequant_q4_f16(Wq, scale_min, stream=None):
+    """fp16 rendering of the q4 weights (the tensor-core operand) as uint16 bits [N, K]."""
+    import torch
+    N, K2 = Wq.shape
+    out = torch.empty((N, 2 * K2), dtype=torch.uint16, device=Wq.device)
+    st = rt_dequant_q4_f16(_dev(Wq, torch.uint8, "Wq"), _dev(scale_min, torch.uint16, "scale_min"),
+                           _dev(out, torch.uint16, "W_out"), N, 2 * K2, _stream_ptr(stream))
+    _check(st, "rt_dequant_q4_f16")
+    return out
+
+
+def dequant_q8_f32(Wq, scale, stream=None):
+    import torch
+    N, K = Wq.shape
+    out = torch.empty((N, K), dtype=torch.float32, device=Wq.device)
+    st = rt_dequant_q8_f32(_dev(Wq, torch.int8, "Wq"), _dev(scale, torch.float32, "scale"),
+                           _dev(out, torch.float32, "W_out"), N, K, _stream_ptr(stream))
+    _check(st, "rt_dequant_q8_f32")
+    return out
+
+
+def device_status(stream=None) -> int:
+    """Synchronizes the stream and returns (and clears) the device status word."""
+    v = ctypes.c_int(0)
+    _check(rt_device_status(_stream_ptr(stream), ctypes.byref(v)), "rt_device_status")
+    return int(v.value)
+
+
+def auto_path(fmt: int, M: int, N: int, K: int) -> int:
+    return int(rt_qgemm_auto_path(fmt, M, N, K))

@@ -1,0 +1,32 @@
+// Launchers of the device kernels, called only by the C ABI layer (api.cu).
+#pragma once
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace rtq {
+
+// fp32 CUDA-core path: one thread per output row, MT activation rows per block.
+cudaError_t launch_simt_q4(const float *X, const uint8_t *Wq, const uint16_t *SM, float *Y,
+                           int M, int N, int K, cudaStream_t s);
+cudaError_t launch_simt_q8(const float *X, const int8_t *Wq, const float *S, float *Y, int M,
+                           int N, int K, cudaStream_t s);
+
+// tcgen05 path: 128 weight rows x BN activation rows per CTA, fp16 (or bf16)
+// operands in swizzled shared memory, fp32 accumulator in TMEM.
+cudaError_t launch_tc_q4(const float *X, const uint8_t *Wq, const uint16_t *SM, float *Y, int M,
+                         int N, int K, bool bf16, unsigned *status, cudaStream_t s);
+cudaError_t launch_tc_q8(const float *X, const int8_t *Wq, const float *S, float *Y, int M, int N,
+                         int K, bool bf16, unsigned *status, cudaStream_t s);
+
+// dequantization exports (same __device__ routines as the GEMMs)
+cudaError_t launch_dequant_q4_f32(const uint8_t *Wq, const uint16_t *SM, float *W, int N, int K,
+                                  cudaStream_t s);
+cudaError_t launch_dequant_q4_16(const uint8_t *Wq, const uint16_t *SM, uint16_t *W, int N,
+                                 int K, bool bf16, cudaStream_t s);
+cudaError_t launch_dequant_q8_f32(const int8_t *Wq, const float *S, float *W, int N, int K,
+                                  cudaStream_t s);
+
+// Largest M the SIMT path takes under RT_PATH_AUTO.
+constexpr int kAutoSimtMaxM = 8;
+
+}  // namespace rtq

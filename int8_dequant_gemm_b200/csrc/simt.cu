@@ -1,0 +1,275 @@
+// fp32 CUDA-core kernels: the exact-rounding path (weights dequantized to
+// fp32 with one rounding, fp32 FMA accumulation) and the small-M path.
+//
+// Layout of work: each thread owns one output row o of W and MT activation
+// rows, staged once per block in shared memory.  Inside the K loop every lane
+// of a warp reads the same activation address (a shared-memory broadcast), so
+// shared memory bandwidth is not the limit; the weight stream is one 16-byte
+// load per thread per step (a q4 group, or 16 q8 codes) that L1 completes to
+// full sectors on the following step.
+#include <algorithm>
+
+#include "dequant.cuh"
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace rtq {
+namespace {
+
+constexpr int kSimtThreads = 256;
+
+template <int MT>
+__device__ __forceinline__ void stage_x(const float *__restrict__ X, float4 *xs4, int m0, int mt,
+                                        int K) {
+    const int K4 = K / 4;
+    for (int i = threadIdx.x; i < MT * K4; i += blockDim.x) {
+        const int r = i / K4;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r < mt) v = ldg_f4(X + static_cast<size_t>(m0 + r) * K + (i - r * K4) * 4);
+        xs4[i] = v;
+    }
+}
+
+template <int MT>
+__global__ void __launch_bounds__(kSimtThreads)
+    simt_q4_kernel(const float *__restrict__ X, const uint8_t *__restrict__ Wq,
+                   const uint32_t *__restrict__ SM, float *__restrict__ Y, int M, int N, int K) {
+    extern __shared__ float4 xs4[];
+    const float *xs = reinterpret_cast<const float *>(xs4);
+    const int m0 = blockIdx.x * MT;
+    const int mt = min(MT, M - m0);
+    pdl_wait_prior_grid();
+    stage_x<MT>(X, xs4, m0, mt, K);
+    __syncthreads();
+    pdl_launch_dependents();
+
+    const int o = blockIdx.y * kSimtThreads + threadIdx.x;
+    if (o >= N) return;
+    float acc[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) acc[m] = 0.f;
+
+    const uint8_t *wrow = Wq + static_cast<size_t>(o) * (K / 2);
+    const uint32_t *srow = SM + static_cast<size_t>(o) * (K / 32);
+    const int G = K / 32;
+    for (int g = 0; g < G; ++g) {
+        const uint4 p = ldg_v4(wrow + g * 16);
+        float sc, mn;
+        q4_scale_min(__ldg(srow + g), sc, mn);
+        const uint32_t words[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            float w[8];
+            q4_word_f32(words[c], sc, mn, w);
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                const float4 *xr = reinterpret_cast<const float4 *>(xs + m * K + g * 32 + c * 8);
+                const float4 a = xr[0], b = xr[1];
+                float t = acc[m];
+                t = fmaf(a.x, w[0], t);
+                t = fmaf(a.y, w[1], t);
+                t = fmaf(a.z, w[2], t);
+                t = fmaf(a.w, w[3], t);
+                t = fmaf(b.x, w[4], t);
+                t = fmaf(b.y, w[5], t);
+                t = fmaf(b.z, w[6], t);
+                t = fmaf(b.w, w[7], t);
+                acc[m] = t;
+            }
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+        if (m < mt) Y[static_cast<size_t>(m0 + m) * N + o] = acc[m];
+}
+
+// q8: the row scale is factored out of the K sum, Y = scale[o] * sum_k x*q,
+// and applied once in fp32 at the end.
+template <int MT>
+__global__ void __launch_bounds__(kSimtThreads)
+    simt_q8_kernel(const float *__restrict__ X, const int8_t *__restrict__ Wq,
+                   const float *__restrict__ S, float *__restrict__ Y, int M, int N, int K) {
+    extern __shared__ float4 xs4[];
+    const float *xs = reinterpret_cast<const float *>(xs4);
+    const int m0 = blockIdx.x * MT;
+    const int mt = min(MT, M - m0);
+    pdl_wait_prior_grid();
+    stage_x<MT>(X, xs4, m0, mt, K);
+    __syncthreads();
+    pdl_launch_dependents();
+
+    const int o = blockIdx.y * kSimtThreads + threadIdx.x;
+    if (o >= N) return;
+    float acc[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) acc[m] = 0.f;
+    const int8_t *wrow = Wq + static_cast<size_t>(o) * K;
+    for (int k0 = 0; k0 < K; k0 += 16) {
+        const uint4 p = ldg_v4(wrow + k0);
+        const uint32_t words[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const float w0 = q8_byte_f32(words[c], 0), w1 = q8_byte_f32(words[c], 1);
+            const float w2 = q8_byte_f32(words[c], 2), w3 = q8_byte_f32(words[c], 3);
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                const float4 a = *reinterpret_cast<const float4 *>(xs + m * K + k0 + c * 4);
+                float t = acc[m];
+                t = fmaf(a.x, w0, t);
+                t = fmaf(a.y, w1, t);
+                t = fmaf(a.z, w2, t);
+                t = fmaf(a.w, w3, t);
+                acc[m] = t;
+            }
+        }
+    }
+    const float sc = __ldg(S + o);
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+        if (m < mt) Y[static_cast<size_t>(m0 + m) * N + o] = acc[m] * sc;
+}
+
+template <int MT>
+cudaError_t launch_simt_mt(bool q4, const float *X, const void *Wq, const void *S, float *Y,
+                           int M, int N, int K, cudaStream_t s) {
+    const size_t smem = static_cast<size_t>(MT) * K * sizeof(float);
+    void *fn = q4 ? reinterpret_cast<void *>(&simt_q4_kernel<MT>)
+                  : reinterpret_cast<void *>(&simt_q8_kernel<MT>);
+    if (smem > 48 * 1024) {
+        cudaError_t e =
+            cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((M + MT - 1) / MT, (N + kSimtThreads - 1) / kSimtThreads, 1);
+    cfg.blockDim = dim3(kSimtThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (q4)
+        return cudaLaunchKernelEx(&cfg, simt_q4_kernel<MT>, X,
+                                  static_cast<const uint8_t *>(Wq),
+                                  static_cast<const uint32_t *>(S), Y, M, N, K);
+    return cudaLaunchKernelEx(&cfg, simt_q8_kernel<MT>, X, static_cast<const int8_t *>(Wq),
+                              static_cast<const float *>(S), Y, M, N, K);
+}
+
+// Activation rows per block: as many as M needs up to 8, capped so the staged
+// activations stay within 128 KB of shared memory.
+cudaError_t launch_simt(bool q4, const float *X, const void *Wq, const void *S, float *Y, int M,
+                        int N, int K, cudaStream_t s) {
+    int mt = M >= 8 ? 8 : (M >= 4 ? 4 : (M >= 2 ? 2 : 1));
+    while (mt > 1 && static_cast<size_t>(mt) * K * sizeof(float) > 128 * 1024) mt /= 2;
+    switch (mt) {
+        case 8: return launch_simt_mt<8>(q4, X, Wq, S, Y, M, N, K, s);
+        case 4: return launch_simt_mt<4>(q4, X, Wq, S, Y, M, N, K, s);
+        case 2: return launch_simt_mt<2>(q4, X, Wq, S, Y, M, N, K, s);
+        default: return launch_simt_mt<1>(q4, X, Wq, S, Y, M, N, K, s);
+    }
+}
+
+// ----------------------------------------------------------- dequant exports
+__global__ void dequant_q4_f32_kernel(const uint8_t *__restrict__ Wq,
+                                      const uint32_t *__restrict__ SM, float *__restrict__ W,
+                                      int N, int K) {
+    const int G = K / 32;
+    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= static_cast<int64_t>(N) * G) return;
+    const int64_t o = idx / G, g = idx % G;
+    const uint4 p = ldg_nc_v4(Wq + o * (K / 2) + g * 16);
+    float sc, mn;
+    q4_scale_min(__ldg(SM + o * G + g), sc, mn);
+    const uint32_t words[4] = {p.x, p.y, p.z, p.w};
+    float *dst = W + o * K + g * 32;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        float w[8];
+        q4_word_f32(words[c], sc, mn, w);
+        reinterpret_cast<float4 *>(dst + c * 8)[0] = make_float4(w[0], w[1], w[2], w[3]);
+        reinterpret_cast<float4 *>(dst + c * 8)[1] = make_float4(w[4], w[5], w[6], w[7]);
+    }
+}
+
+template <Op16 OP>
+__global__ void dequant_q4_16_kernel(const uint8_t *__restrict__ Wq,
+                                       const uint32_t *__restrict__ SM, uint16_t *__restrict__ W,
+                                       int N, int K) {
+    const int G = K / 32;
+    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= static_cast<int64_t>(N) * G) return;
+    const int64_t o = idx / G, g = idx % G;
+    const uint4 p = ldg_nc_v4(Wq + o * (K / 2) + g * 16);
+    float sc, mn;
+    q4_scale_min(__ldg(SM + o * G + g), sc, mn);
+    const uint32_t words[4] = {p.x, p.y, p.z, p.w};
+    uint4 *dst = reinterpret_cast<uint4 *>(W + o * K + g * 32);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) dst[c] = q4_word_op<OP>(words[c], sc, mn);
+}
+
+__global__ void dequant_q8_f32_kernel(const int8_t *__restrict__ Wq, const float *__restrict__ S,
+                                      float *__restrict__ W, int N, int K) {
+    const int C = K / 16;
+    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= static_cast<int64_t>(N) * C) return;
+    const int64_t o = idx / C, c = idx % C;
+    const uint4 p = ldg_nc_v4(Wq + o * K + c * 16);
+    const float sc = __ldg(S + o);
+    const uint32_t words[4] = {p.x, p.y, p.z, p.w};
+    float *dst = W + o * K + c * 16;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        reinterpret_cast<float4 *>(dst)[j] =
+            make_float4(q8_byte_f32(words[j], 0) * sc, q8_byte_f32(words[j], 1) * sc,
+                        q8_byte_f32(words[j], 2) * sc, q8_byte_f32(words[j], 3) * sc);
+    }
+}
+
+inline unsigned blocks_for(int64_t n, int threads) {
+    return static_cast<unsigned>((n + threads - 1) / threads);
+}
+
+}  // namespace
+
+cudaError_t launch_simt_q4(const float *X, const uint8_t *Wq, const uint16_t *SM, float *Y,
+                           int M, int N, int K, cudaStream_t s) {
+    return launch_simt(true, X, Wq, SM, Y, M, N, K, s);
+}
+
+cudaError_t launch_simt_q8(const float *X, const int8_t *Wq, const float *S, float *Y, int M,
+                           int N, int K, cudaStream_t s) {
+    return launch_simt(false, X, Wq, S, Y, M, N, K, s);
+}
+
+cudaError_t launch_dequant_q4_f32(const uint8_t *Wq, const uint16_t *SM, float *W, int N, int K,
+                                  cudaStream_t s) {
+    const int64_t n = static_cast<int64_t>(N) * (K / 32);
+    dequant_q4_f32_kernel<<<blocks_for(n, 256), 256, 0, s>>>(
+        Wq, reinterpret_cast<const uint32_t *>(SM), W, N, K);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dequant_q4_16(const uint8_t *Wq, const uint16_t *SM, uint16_t *W, int N,
+                                 int K, bool bf16, cudaStream_t s) {
+    const int64_t n = static_cast<int64_t>(N) * (K / 32);
+    const uint32_t *sm = reinterpret_cast<const uint32_t *>(SM);
+    if (bf16)
+        dequant_q4_16_kernel<Op16::bf16><<<blocks_for(n, 256), 256, 0, s>>>(Wq, sm, W, N, K);
+    else
+        dequant_q4_16_kernel<Op16::f16><<<blocks_for(n, 256), 256, 0, s>>>(Wq, sm, W, N, K);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dequant_q8_f32(const int8_t *Wq, const float *S, float *W, int N, int K,
+                                  cudaStream_t s) {
+    const int64_t n = static_cast<int64_t>(N) * (K / 16);
+    dequant_q8_f32_kernel<<<blocks_for(n, 256), 256, 0, s>>>(Wq, S, W, N, K);
+    return cudaGetLastError();
+}
+
+}  // namespace rtq

@@ -65,6 +65,7 @@ def with_outliers(W: np.ndarray, seed: int, frac: float = 0.01, factor: float = 
     seeded element multiplied by `factor` (the outlier stress of the M sweep)."""
     W = np.array(W, dtype=np.float32, copy=True)
     N, K = W.shape
+    span = min(span, K)
     n_spans = K // span
     g = generator(seed + 7_919)
     cells = N * n_spans

@@ -1,0 +1,161 @@
+"""Host-side checks of the C ABI that need no GPU.
+
+- librtq.so loads and exports every function include/rtq.h declares.
+- Argument validation returns the documented status before any CUDA call
+  (the pointers below are never dereferenced).
+- The library's host quantizers match the oracle's bit for bit on the
+  workloads' weights, outliers included.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import int8_dequant_gemm_b200 as rtq
+from int8_dequant_gemm_b200 import build as rtq_build
+from int8_dequant_gemm_b200 import workloads as wl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+RT_OK, INVALID, ALIGN, SHAPE, CUDA, TIMEOUT, RANGE = 0, 1, 2, 3, 4, 5, 6
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    rtq_build.build()
+    return rtq.lib()
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "rtq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = set(re.findall(r"\b(rt_[a-z0-9_]+)\s*\(", src))
+    return sorted(names)
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for required in ("rt_qgemm_q4", "rt_qgemm_q8", "rt_qblock_project", "rt_quantize_q4_g32",
+                     "rt_quantize_q8_row", "rt_dequant_q4_f32", "rt_dequant_q8_f32",
+                     "rt_device_status", "rt_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = ctypes.CDLL(rtq.LIB_PATH)
+    missing = [n for n in _declared_functions() if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_status_strings_and_version():
+    for s in range(7):
+        assert rtq.status_string(s) and rtq.status_string(s) != "unknown status"
+    assert rtq.status_string(99) == "unknown status"
+    assert rtq.lib().rt_version() >= 100
+
+
+# fake, well-aligned, non-overlapping device addresses (never dereferenced)
+X, W, S, Y = 0x10000000, 0x20000000, 0x30000000, 0x40000000
+
+
+@pytest.mark.parametrize("fn", ["rt_qgemm_q4", "rt_qgemm_q8"])
+def test_validation_statuses(fn):
+    f = getattr(rtq, fn)
+    K = 64
+    assert f(None, W, S, Y, 4, 16, K, 0, None) == INVALID          # null X with M > 0
+    assert f(X, None, S, Y, 4, 16, K, 0, None) == INVALID          # null weights
+    assert f(X, W, S, Y, -1, 16, K, 0, None) == INVALID            # negative M
+    assert f(X, W, S, Y, 4, 0, K, 0, None) == INVALID              # N < 1
+    assert f(X + 4, W, S, Y, 4, 16, K, 0, None) == ALIGN           # X not 16-byte aligned
+    assert f(X, W + 8, S, Y, 4, 16, K, 0, None) == ALIGN           # Wq not 16-byte aligned
+    assert f(X, W, S + 2, Y, 4, 16, K, 0, None) == ALIGN           # scales not 4-byte aligned
+    assert f(X, W, S, Y + 8, 4, 16, K, 0, None) == ALIGN           # Y not 16-byte aligned
+    assert f(X, W, S, X, 4, 16, K, 0, None) == INVALID             # Y overlaps X
+    assert f(X, W, S, W, 4, 16, K, 0, None) == INVALID             # Y overlaps Wq
+    assert f(X, W, S, Y, 4, 16, K, 7, None) == INVALID             # unknown path
+    assert f(None, W, S, None, 0, 16, K, 0, None) == RT_OK         # M == 0 is a no-op
+    bad_k = 40 if fn == "rt_qgemm_q4" else 24
+    assert f(X, W, S, Y, 4, 16, bad_k, 0, None) == SHAPE           # K not a multiple of the granule
+    assert f(X, W, S, Y, 4, 16, 96, 2, None) == SHAPE              # forced TC needs K % 64
+
+
+def test_auto_path_dispatch():
+    assert rtq.auto_path(4, 1, 2048, 512) == 1
+    assert rtq.auto_path(4, 80, 2048, 512) == 2
+    assert rtq.auto_path(8, 65536, 512, 2048) == 2
+    assert rtq.auto_path(4, 80, 2048, 96) == 1      # K % 64 != 0 -> SIMT
+    assert rtq.auto_path(4, 80, 2048, 40) == -1     # not a q4 shape
+    assert rtq.auto_path(5, 80, 2048, 512) == -1
+
+
+def test_block_driver_validation():
+    blk = rtq._QBlockC(W, S, W, S, W, S, W, S, 0, 2048)
+    assert rtq.rt_qblock_project(blk, 4, X, X, X, X, Y, Y, Y, Y, 0, None) == INVALID
+    assert rtq.lib().rt_qblock_project(None, 4, X, X, X, X, Y, Y, Y, Y, 0, None) == INVALID
+
+
+def test_dequant_validation():
+    assert rtq.rt_dequant_q4_f32(W, S, Y, 4, 40, None) == SHAPE
+    assert rtq.rt_dequant_q4_f32(W + 1, S, Y, 4, 64, None) == ALIGN
+    assert rtq.rt_dequant_q8_f32(None, S, Y, 4, 64, None) == INVALID
+    assert rtq.rt_device_status(None, None) == INVALID
+
+
+# ---------------------------------------------------------------- quantizers
+def test_quantizer_statuses():
+    w = np.zeros((2, 40), dtype=np.float32)
+    Wq = np.empty((2, 20), dtype=np.uint8)
+    sm = np.empty((2, 2, 2), dtype=np.uint16)
+    assert rtq.rt_quantize_q4_g32(w.ctypes.data, 2, 40, 21, Wq.ctypes.data, sm.ctypes.data) == SHAPE
+    w = np.full((1, 32), np.nan, dtype=np.float32)
+    assert rtq.rt_quantize_q4_g32(w.ctypes.data, 1, 32, 21, Wq.ctypes.data, sm.ctypes.data) == RANGE
+    w = np.full((1, 32), 7e4, dtype=np.float32)
+    assert rtq.rt_quantize_q4_g32(w.ctypes.data, 1, 32, 21, Wq.ctypes.data, sm.ctypes.data) == RANGE
+    assert rtq.rt_quantize_q4_g32(w.ctypes.data, 1, 32, -1, Wq.ctypes.data, sm.ctypes.data) == INVALID
+    assert rtq.rt_quantize_q8_row(None, 1, 32, None, None) == INVALID
+    w = np.full((1, 16), np.inf, dtype=np.float32)
+    q = np.empty((1, 16), dtype=np.int8)
+    s = np.empty(1, dtype=np.float32)
+    assert rtq.rt_quantize_q8_row(w.ctypes.data, 1, 16, q.ctypes.data, s.ctypes.data) == RANGE
+
+
+@pytest.mark.parametrize("name,outliers", [("qkvg", False), ("w13", False), ("qkvg", True)])
+def test_q4_quantizer_matches_oracle_bit_for_bit(name, outliers):
+    W = wl.projection_weights(3, 0, name, outliers=outliers)
+    if not outliers:
+        W = W[:512]  # a slice keeps the single-threaded oracle fast
+    Wq, sm = rtq.quantize_q4_g32(W)
+    Wq_o, sm_o = oracle.quant_q4_g32(W)
+    assert np.array_equal(Wq, Wq_o)
+    assert np.array_equal(sm, sm_o)
+
+
+def test_q4_quantizer_grid_sizes_and_degenerate_rows():
+    W = wl.weights(48, 96, seed=31)
+    W[5] = 0.25   # constant rows
+    W[6] = 0.0
+    W[7, :32] = -3.0
+    for n_grid in (1, 2, 5, 21, 41):
+        Wq, sm = rtq.quantize_q4_g32(W, n_grid=n_grid)
+        Wq_o, sm_o = oracle.quant_q4_g32(W, n_grid=n_grid)
+        assert np.array_equal(Wq, Wq_o) and np.array_equal(sm, sm_o), n_grid
+
+
+@pytest.mark.parametrize("name,outliers", [("wo", False), ("w2", False), ("w2", True)])
+def test_q8_quantizer_matches_oracle_bit_for_bit(name, outliers):
+    W = wl.projection_weights(3, 0, name, outliers=outliers)
+    W[1] = 0.0
+    Wq, s = rtq.quantize_q8_row(W)
+    Wq_o, s_o = oracle.quant_q8_row(W)
+    assert np.array_equal(Wq, Wq_o)
+    assert np.array_equal(s.view(np.uint32), s_o.view(np.uint32))
+
+
+def test_empty_quantizer_inputs():
+    Wq, sm = rtq.quantize_q4_g32(np.zeros((0, 64), dtype=np.float32))
+    assert Wq.shape == (0, 32) and sm.shape == (0, 2, 2)
+    q, s = rtq.quantize_q8_row(np.zeros((0, 16), dtype=np.float32))
+    assert q.shape == (0, 16)

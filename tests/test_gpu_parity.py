@@ -1,0 +1,323 @@
+"""GPU parity of the CUDA path against the CPU oracle, called through the C ABI.
+
+Packed weights come from the ORACLE's quantizer (or are random bytes), inputs
+from the seeded workload generator, and expected values only from oracle/.
+
+Gates:
+  - dequantization exports: bit-exact (fp32 rendering = exact value rounded
+    once; fp16 / bf16 renderings = that fp32 rounded again to nearest-even);
+  - X = I turns the GEMM into W_hat^T: bit-exact on every path;
+  - SIMT GEMM: max|Y - Y_ref| / max|Y_ref| <= 1e-5;
+  - tensor-core GEMM (fp16 operands): <= 4e-3, and every output within the
+    first-order rounding bound of its operands (below);
+  - tensor-core GEMM with bf16 operands: the same elementwise bound with the
+    bf16 unit roundoff;
+  - no write outside Y (NaN guard bands), deterministic repeats, device
+    status word clear afterwards.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from int8_dequant_gemm_b200 import workloads as wl
+
+torch = pytest.importorskip("torch")
+
+pytestmark = pytest.mark.gpu
+
+SIMT_TOL = 1e-5
+TC_TOL = 4e-3
+# unit roundoff (2^-p) of the 16-bit operand types
+UNIT = {"tc": 2.0 ** -11, "tc_bf16": 2.0 ** -8}
+MAX_REL = {"simt": SIMT_TOL, "tc": TC_TOL, "auto": TC_TOL, "tc_bf16": 1e-2}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def rtq_lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from int8_dequant_gemm_b200 import build
+    build.build()
+    import int8_dequant_gemm_b200 as rtq
+    rtq.lib()
+    yield rtq
+    torch.cuda.synchronize()
+    assert rtq.device_status() == 0
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def rel_err(Y, Yref):
+    Y = np.asarray(Y, dtype=np.float64)
+    return float(np.max(np.abs(Y - Yref)) / max(np.max(np.abs(Yref)), 1e-300))
+
+
+def f16_round(x32: np.ndarray) -> np.ndarray:
+    """fp32 -> nearest-even fp16 (numpy's conversion), back as fp32 values."""
+    return np.asarray(x32, dtype=np.float32).astype(np.float16).astype(np.float32)
+
+
+def op_round(x32, path):
+    return f16_round(x32) if path == "tc" else bf16_round(x32)
+
+
+def assert_within_rounding_bound(Y, X, What, path):
+    """Elementwise first-order bound of the tensor-core path: each product
+    x*w carries the roundings of x and w to the operand type (relative u each,
+    w also its fp32 rounding) and the fp32 accumulation adds at most K*2^-23
+    relative to sum|x*w|; an fp16 subnormal operand (below 2^-14) is rounded
+    with an absolute error of at most 2^-25 instead."""
+    u = UNIT[path]
+    A = np.abs(X.astype(np.float64)) @ np.abs(What).T
+    K = X.shape[1]
+    slack = 0.0
+    if path == "tc":
+        slack = 2.0 ** -25 * (np.abs(What).sum(axis=1)[None, :] +
+                              np.abs(X.astype(np.float64)).sum(axis=1)[:, None])
+    bound = (2.0 * u + u * u + 2.0 ** -23 + K * 2.0 ** -23) * A + slack
+    ref = X.astype(np.float64) @ What.T
+    bad = np.abs(np.asarray(Y, np.float64) - ref) > bound
+    assert not bad.any(), f"{bad.sum()} outputs outside the rounding bound"
+
+
+def bf16_round(x32: np.ndarray) -> np.ndarray:
+    """fp32 -> nearest-even bf16 (as fp32 values), finite inputs."""
+    u = np.ascontiguousarray(x32, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32)
+
+
+def q4_weights(N, K, seed, outliers=False):
+    W = wl.weights(N, K, seed)
+    if outliers:
+        W = wl.with_outliers(W, seed)
+    return oracle.quant_q4_g32(W)
+
+
+def q8_weights(N, K, seed, outliers=False):
+    W = wl.weights(N, K, seed)
+    if outliers:
+        W = wl.with_outliers(W, seed)
+    return oracle.quant_q8_row(W)
+
+
+def random_q4(N, K, seed):
+    """Random payload bytes and random binary16 (scale, min), both signs."""
+    g = np.random.default_rng(seed)
+    Wq = g.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    sc = g.uniform(-0.05, 0.05, size=(N, K // 32)).astype(np.float16)
+    mn = g.uniform(-0.5, 0.5, size=(N, K // 32)).astype(np.float16)
+    sc[0, 0] = 0.0
+    sm = np.stack([sc.view(np.uint16), mn.view(np.uint16)], axis=-1)
+    return Wq, np.ascontiguousarray(sm)
+
+
+# ------------------------------------------------------------ dequantization
+@pytest.mark.parametrize("N,K", [(64, 32), (130, 512), (512, 2048)])
+def test_dequant_q4_exports_bit_exact(rtq_lib, N, K):
+    for Wq, sm in (q4_weights(N, K, seed=N + K, outliers=True), random_q4(N, K, seed=N)):
+        exact = oracle.dequant_q4(Wq, sm)
+        ref32 = exact.astype(np.float32)
+        got32 = rtq_lib.dequant_q4_f32(dev(Wq), dev(sm)).cpu().numpy()
+        assert np.array_equal(got32.view(np.uint32), ref32.view(np.uint32))
+        got16 = rtq_lib.dequant_q4_bf16(dev(Wq), dev(sm)).cpu().numpy()
+        ref16 = (bf16_round(ref32).view(np.uint32) >> 16).astype(np.uint16)
+        assert np.array_equal(got16, ref16)
+        goth = rtq_lib.dequant_q4_f16(dev(Wq), dev(sm)).cpu().numpy()
+        refh = ref32.astype(np.float16).view(np.uint16)
+        assert np.array_equal(goth, refh)
+
+
+@pytest.mark.parametrize("N,K", [(16, 16), (512, 512), (512, 2048)])
+def test_dequant_q8_export_bit_exact(rtq_lib, N, K):
+    Wq, s = q8_weights(N, K, seed=N * 3 + K, outliers=True)
+    Wq[0, 0] = -128  # representable in the format even if the quantizer never emits it
+    ref32 = oracle.dequant_q8(Wq, s).astype(np.float32)
+    got = rtq_lib.dequant_q8_f32(dev(Wq), dev(s)).cpu().numpy()
+    assert np.array_equal(got.view(np.uint32), ref32.view(np.uint32))
+
+
+# --------------------------------------------------- X = I: exact transposes
+@pytest.mark.parametrize("path", ["simt", "tc", "tc_bf16"])
+def test_identity_input_q4_bit_exact(rtq_lib, path):
+    N, K = 384, 512
+    Wq, sm = q4_weights(N, K, seed=77, outliers=True)
+    Y = rtq_lib.qgemm_q4(torch.eye(K, device="cuda"), dev(Wq), dev(sm), path=path)
+    ref32 = oracle.dequant_q4(Wq, sm).astype(np.float32).T
+    if path != "simt":
+        ref32 = op_round(ref32, path)
+    assert np.array_equal(Y.cpu().numpy(), ref32)
+
+
+@pytest.mark.parametrize("path", ["simt", "tc", "tc_bf16"])
+def test_identity_input_q8_bit_exact(rtq_lib, path):
+    N, K = 256, 512
+    Wq, s = q8_weights(N, K, seed=78, outliers=True)
+    Y = rtq_lib.qgemm_q8(torch.eye(K, device="cuda"), dev(Wq), dev(s), path=path)
+    ref32 = oracle.dequant_q8(Wq, s).astype(np.float32).T
+    assert np.array_equal(Y.cpu().numpy(), ref32)
+
+
+# ----------------------------------------------------------- GEMM parity
+SIMT_SHAPES = [(1, 2048, 512), (3, 130, 96), (17, 300, 128), (80, 2048, 512), (79, 512, 2048),
+               (129, 64, 64), (8, 1, 32)]
+TC_SHAPES = [(16, 256, 64), (80, 2048, 512), (80, 512, 2048), (81, 130, 128), (300, 512, 512),
+             (1, 128, 64), (256, 200, 192), (1000, 640, 512)]
+
+
+def _run_q4(rtq_lib, M, N, K, path, seed, outliers=False):
+    X = wl.activations(M, K, seed)
+    Wq, sm = q4_weights(N, K, seed + 1, outliers)
+    Y = rtq_lib.qgemm_q4(dev(X), dev(Wq), dev(sm), path=path).cpu().numpy()
+    if path in UNIT:
+        assert_within_rounding_bound(Y, X, oracle.dequant_q4(Wq, sm), path)
+    return Y, oracle.gemm_q4(X, Wq, sm)
+
+
+def _run_q8(rtq_lib, M, N, K, path, seed, outliers=False):
+    X = wl.activations(M, K, seed)
+    Wq, s = q8_weights(N, K, seed + 1, outliers)
+    Y = rtq_lib.qgemm_q8(dev(X), dev(Wq), dev(s), path=path).cpu().numpy()
+    if path in UNIT:
+        assert_within_rounding_bound(Y, X, oracle.dequant_q8(Wq, s), path)
+    return Y, oracle.gemm_q8(X, Wq, s)
+
+
+@pytest.mark.parametrize("M,N,K", SIMT_SHAPES)
+def test_simt_parity_q4(rtq_lib, M, N, K):
+    Y, ref = _run_q4(rtq_lib, M, N, K, "simt", seed=M + N + K, outliers=True)
+    assert rel_err(Y, ref) <= SIMT_TOL
+
+
+@pytest.mark.parametrize("M,N,K", [s for s in SIMT_SHAPES if s[2] % 16 == 0])
+def test_simt_parity_q8(rtq_lib, M, N, K):
+    Y, ref = _run_q8(rtq_lib, M, N, K, "simt", seed=M * 7 + N + K, outliers=True)
+    assert rel_err(Y, ref) <= SIMT_TOL
+
+
+@pytest.mark.parametrize("path", ["tc", "tc_bf16"])
+@pytest.mark.parametrize("M,N,K", TC_SHAPES)
+def test_tc_parity_q4(rtq_lib, M, N, K, path):
+    Y, ref = _run_q4(rtq_lib, M, N, K, path, seed=M + 3 * N + K, outliers=True)
+    assert rel_err(Y, ref) <= MAX_REL[path]
+
+
+@pytest.mark.parametrize("path", ["tc", "tc_bf16"])
+@pytest.mark.parametrize("M,N,K", TC_SHAPES)
+def test_tc_parity_q8(rtq_lib, M, N, K, path):
+    Y, ref = _run_q8(rtq_lib, M, N, K, path, seed=M + 5 * N + K, outliers=True)
+    assert rel_err(Y, ref) <= MAX_REL[path]
+
+
+def test_random_format_bytes_both_paths(rtq_lib):
+    M, N, K = 96, 256, 256
+    X = wl.activations(M, K, 5)
+    Wq, sm = random_q4(N, K, 6)
+    ref = oracle.gemm_q4(X, Wq, sm)
+    for path in ("simt", "tc", "tc_bf16"):
+        Y = rtq_lib.qgemm_q4(dev(X), dev(Wq), dev(sm), path=path).cpu().numpy()
+        assert rel_err(Y, ref) <= MAX_REL[path], path
+        if path in UNIT:
+            assert_within_rounding_bound(Y, X, oracle.dequant_q4(Wq, sm), path)
+
+
+# ------------------------------------------------------- edge cases, guards
+@pytest.mark.parametrize("path", ["simt", "tc"])
+@pytest.mark.parametrize("M", [1, 3, 17, 79, 81, 129])
+def test_guard_bands_and_ragged_sizes(rtq_lib, path, M):
+    N, K = 136, 128
+    X = wl.activations(M, K, M)
+    Wq, sm = q4_weights(N, K, 40 + M)
+    guard = 1024
+    nan_bits = torch.full((M * N + 2 * guard,), 0x7FC01234, dtype=torch.int32, device="cuda")
+    buf = nan_bits.view(torch.float32)
+    Y = buf[guard:guard + M * N].view(M, N)
+    rtq_lib.qgemm_q4(dev(X), dev(Wq), dev(sm), Y=Y, path=path)
+    host = nan_bits.cpu().numpy()
+    assert np.all(host[:guard] == 0x7FC01234) and np.all(host[guard + M * N:] == 0x7FC01234)
+    tol = SIMT_TOL if path == "simt" else TC_TOL
+    assert rel_err(Y.cpu().numpy(), oracle.gemm_q4(X, Wq, sm)) <= tol
+
+
+def test_zero_rows_is_a_no_op(rtq_lib):
+    Wq, sm = q4_weights(128, 64, 1)
+    X = torch.empty((0, 64), device="cuda")
+    Y = rtq_lib.qgemm_q4(X, dev(Wq), dev(sm))
+    assert Y.shape == (0, 128)
+
+
+@pytest.mark.parametrize("path", ["simt", "tc"])
+def test_deterministic_repeats_and_side_stream(rtq_lib, path):
+    M, N, K = 200, 512, 512
+    X = dev(wl.activations(M, K, 9))
+    Wq, sm = q4_weights(N, K, 10)
+    Wq, sm = dev(Wq), dev(sm)
+    a = rtq_lib.qgemm_q4(X, Wq, sm, path=path)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        b = rtq_lib.qgemm_q4(X, Wq, sm, path=path, stream=s)
+    s.synchronize()
+    assert torch.equal(a, b)
+
+
+# ------------------------------------------- full sizes, sampled outputs
+@pytest.mark.parametrize("fmt", ["q4", "q8"])
+def test_full_size_m65536_sampled_rows(rtq_lib, fmt):
+    """The M sweep's largest point (B=64, S=1024) with 1% x20 outlier groups,
+    on the AUTO path, checked on 256 seeded rows (rows are independent)."""
+    M = 65536
+    if fmt == "q4":
+        N, K = 2048, 512
+        W = wl.with_outliers(wl.weights(N, K, wl.seed_for(5, 0, "w1")), wl.seed_for(5, 0, "w1"))
+        Wq, sm = oracle.quant_q4_g32(W)
+    else:
+        N, K = 512, 2048
+        W = wl.with_outliers(wl.weights(N, K, wl.seed_for(5, 0, "w2")), wl.seed_for(5, 0, "w2"))
+        Wq, sm = oracle.quant_q8_row(W)
+    X = wl.activations(M, K, wl.seed_for(5, 0, "x_ffn"))
+    rows = wl.sample_rows(M, 256, seed=123)
+    fn = rtq_lib.qgemm_q4 if fmt == "q4" else rtq_lib.qgemm_q8
+    gemm = oracle.gemm_q4 if fmt == "q4" else oracle.gemm_q8
+    ref = gemm(X, Wq, sm, rows=rows)
+    Xd, Wd, Sd = dev(X), dev(Wq), dev(sm)
+    for path, tol in (("auto", TC_TOL), ("simt", SIMT_TOL)):
+        Y = fn(Xd, Wd, Sd, path=path)
+        assert rel_err(Y[torch.from_numpy(rows).cuda()].cpu().numpy(), ref) <= tol, path
+
+
+def _block_tensors(config, block, M, outliers=False):
+    host = {}
+    for name in ("qkvg", "wo", "w13", "w2"):
+        W = wl.projection_weights(config, block, name, outliers)
+        fmt = wl.BLOCK_PROJECTIONS[name]["fmt"]
+        host[name] = oracle.quant_q4_g32(W) if fmt == "q4" else oracle.quant_q8_row(W)
+        host["x_" + name] = wl.projection_input(config, block, name, M)
+    return host
+
+
+@pytest.mark.parametrize("M,n_check", [(80, None), (2048, 96), (4096, 64)])
+def test_block_driver_matches_oracle(rtq_lib, M, n_check):
+    """One RT-J block's projection set through rt_qblock_project (AUTO path,
+    the configuration the benchmark times); at M >= 2048 on sampled rows."""
+    h = _block_tensors(4 if M == 4096 else 3, 0, M)
+    blk = rtq_lib.QBlock(*(dev(a) for a in (*h["qkvg"], *h["wo"], *h["w13"], *h["w2"])))
+    X = {n: dev(h["x_" + n]) for n in ("qkvg", "wo", "w13", "w2")}
+    Y = {"qkvg": torch.empty((M, 2048), device="cuda"), "wo": torch.empty((M, 512), device="cuda"),
+         "w13": torch.empty((M, 4096), device="cuda"), "w2": torch.empty((M, 512), device="cuda")}
+    rtq_lib.qblock_project(blk, X["qkvg"], X["wo"], X["w13"], X["w2"],
+                           Y["qkvg"], Y["wo"], Y["w13"], Y["w2"])
+    rows = None if n_check is None else wl.sample_rows(M, n_check, seed=M)
+    for name in ("qkvg", "wo", "w13", "w2"):
+        fmt = wl.BLOCK_PROJECTIONS[name]["fmt"]
+        gemm = oracle.gemm_q4 if fmt == "q4" else oracle.gemm_q8
+        ref = gemm(h["x_" + name], *h[name], rows=rows)
+        got = Y[name].cpu().numpy() if rows is None else Y[name].cpu().numpy()[rows]
+        tol = TC_TOL if rtq_lib.auto_path(4 if fmt == "q4" else 8, M, 1, 512) == 2 else SIMT_TOL
+        assert rel_err(got, ref) <= tol, name
+
+
+def test_device_status_clear(rtq_lib):
+    torch.cuda.synchronize()
+    assert rtq_lib.device_status() == 0
