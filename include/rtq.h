@@ -45,8 +45,8 @@
  *   - No C++ exception crosses this boundary.
  *   - Precision: the SIMT path dequantizes to fp32 and accumulates in fp32
  *     (max|Y - Y_exact| / max|Y_exact| <= 1e-5).  The tensor-core path rounds
- *     X and the dequantized q4 weights (their fp32 value) to fp16 -- q8 codes
- *     are exact, their row scale is applied in fp32 after the MMA -- and
+ *     X and the exact dequantized q4 weights once to fp16 -- q8 codes are
+ *     exact, their row scale is applied in fp32 after the MMA -- and
  *     accumulates in fp32 in TMEM (<= 4e-3; about 3e-4 on N(0,1) activations).
  *     fp16 operands need |X| <= 65504 (larger activations become infinite);
  *     RT_PATH_TC_BF16 runs the same kernels on bf16 operands, which keep the
@@ -101,6 +101,22 @@ rt_status rt_qgemm_q8(const float *X, const int8_t *Wq, const float *scale, floa
 /* Which path RT_PATH_AUTO takes for a q4 (fmt = 4) or q8 (fmt = 8) GEMM of
  * this shape: RT_PATH_SIMT or RT_PATH_TC; -1 for an unsupported shape. */
 int rt_qgemm_auto_path(int fmt, int64_t M, int64_t N, int64_t K);
+
+/* Kernels behind the paths:
+ *   RT_KERNEL_SIMT            fp32 CUDA-core kernel, one thread per output row;
+ *   RT_KERNEL_TC_W_STATIONARY tcgen05, one 128-row weight tile x up to 128
+ *                             activation rows per CTA (small M, long K);
+ *   RT_KERNEL_TC_X_RESIDENT   tcgen05, persistent CTAs keep a 128-row block of
+ *                             activations in shared memory and stream weight
+ *                             tiles past it (M >= 256, K <= 512). */
+typedef enum rt_kernel {
+    RT_KERNEL_SIMT = 1,
+    RT_KERNEL_TC_W_STATIONARY = 2,
+    RT_KERNEL_TC_X_RESIDENT = 3
+} rt_kernel;
+
+/* The kernel a GEMM of this format, shape and path runs; -1 if rejected. */
+int rt_qgemm_plan(int fmt, int64_t M, int64_t N, int64_t K, int path);
 
 /*
  * One RT-J block's quantized projection set, following the mixed-precision
@@ -162,9 +178,10 @@ rt_status rt_quantize_q8_row(const float *W, int64_t N, int64_t K, int8_t *Wq, f
  * same __device__ dequantization routines the GEMM kernels use, so tests can
  * check them bit for bit:
  *   *_f32  : W[o,k] rounded once to fp32 (the SIMT path's operand);
- *   q4_f16 : the fp32 value rounded again to fp16, stored as uint16 bits (the
+ *   q4_f16 : the exact value rounded once to fp16, stored as uint16 bits (the
  *            tensor-core path's q4 operand);
- *   q4_bf16: the same rounded to bf16 (the RT_PATH_TC_BF16 operand).
+ *   q4_bf16: the fp32 value rounded again to bf16 (the RT_PATH_TC_BF16
+ *            operand).
  * W_out is [N,K].  Same alignment and shape rules as the GEMMs.
  */
 rt_status rt_dequant_q4_f32(const uint8_t *Wq, const uint16_t *scale_min, float *W_out,

@@ -65,6 +65,8 @@ def lib() -> ctypes.CDLL:
         f.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _i32, _p]
     L.rt_qgemm_auto_path.restype = _i32
     L.rt_qgemm_auto_path.argtypes = [_i32, _i64, _i64, _i64]
+    L.rt_qgemm_plan.restype = _i32
+    L.rt_qgemm_plan.argtypes = [_i32, _i64, _i64, _i64, _i32]
     L.rt_qblock_project.restype = _i32
     L.rt_qblock_project.argtypes = [ctypes.POINTER(_QBlockC), _i64, _p, _p, _p, _p, _p, _p, _p,
                                     _p, _i32, _p]
@@ -137,6 +139,10 @@ def rt_device_status(stream, out) -> int:
 
 def rt_qgemm_auto_path(fmt, M, N, K) -> int:
     return lib().rt_qgemm_auto_path(fmt, M, N, K)
+
+
+def rt_qgemm_plan(fmt, M, N, K, path) -> int:
+    return lib().rt_qgemm_plan(fmt, M, N, K, path)
 
 
 # ------------------------------------------------------- torch-level helpers
@@ -301,3 +307,12 @@ def device_status(stream=None) -> int:
 
 def auto_path(fmt: int, M: int, N: int, K: int) -> int:
     return int(rt_qgemm_auto_path(fmt, M, N, K))
+
+
+KERNELS = {1: "simt", 2: "tc_w_stationary", 3: "tc_x_resident"}
+
+
+def plan(fmt: int, M: int, N: int, K: int, path="auto") -> str:
+    """Name of the kernel a GEMM of this shape runs (see rt_qgemm_plan)."""
+    k = int(rt_qgemm_plan(fmt, M, N, K, _path(path)))
+    return KERNELS.get(k, "rejected")

@@ -100,6 +100,19 @@ int rt_qgemm_auto_path(int fmt, int64_t M, int64_t N, int64_t K) {
     return pick_path(M, K, RT_PATH_AUTO);
 }
 
+int rt_qgemm_plan(int fmt, int64_t M, int64_t N, int64_t K, int path) {
+    if ((fmt != 4 && fmt != 8) || M < 0 || N < 1 || K < 1 || M > kMaxDim || N > kMaxDim ||
+        K > kMaxDim)
+        return -1;
+    if (K % (fmt == 4 ? 32 : 16) != 0) return -1;
+    const int p = pick_path(M, K, path);
+    if (p < 0) return -1;
+    if (p == RT_PATH_SIMT) return RT_KERNEL_SIMT;
+    return rtq::xs_supported(static_cast<int>(M), static_cast<int>(N), static_cast<int>(K))
+               ? RT_KERNEL_TC_X_RESIDENT
+               : RT_KERNEL_TC_W_STATIONARY;
+}
+
 rt_status rt_qgemm_q4(const float *X, const uint8_t *Wq, const uint16_t *scale_min, float *Y,
                       int64_t M, int64_t N, int64_t K, int path, void *stream) {
     rt_status st = validate(X, Wq, scale_min, Y, M, N, K, N * (K / 2), N * (K / 32) * 4, 4, 32);
@@ -114,9 +127,11 @@ rt_status rt_qgemm_q4(const float *X, const uint8_t *Wq, const uint16_t *scale_m
                                              static_cast<int>(N), static_cast<int>(K), s));
     unsigned *status = nullptr;
     if ((st = status_word(&status)) != RT_OK) return st;
-    return from_cuda(rtq::launch_tc_q4(X, Wq, scale_min, Y, static_cast<int>(M),
-                                       static_cast<int>(N), static_cast<int>(K),
-                                       p == RT_PATH_TC_BF16, status, s));
+    const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
+    const bool bf16 = p == RT_PATH_TC_BF16;
+    if (rtq::xs_supported(m, n, k))
+        return from_cuda(rtq::launch_xs_q4(X, Wq, scale_min, Y, m, n, k, bf16, status, s));
+    return from_cuda(rtq::launch_tc_q4(X, Wq, scale_min, Y, m, n, k, bf16, status, s));
 }
 
 rt_status rt_qgemm_q8(const float *X, const int8_t *Wq, const float *scale, float *Y, int64_t M,
@@ -133,8 +148,11 @@ rt_status rt_qgemm_q8(const float *X, const int8_t *Wq, const float *scale, floa
                                              static_cast<int>(N), static_cast<int>(K), s));
     unsigned *status = nullptr;
     if ((st = status_word(&status)) != RT_OK) return st;
-    return from_cuda(rtq::launch_tc_q8(X, Wq, scale, Y, static_cast<int>(M), static_cast<int>(N),
-                                       static_cast<int>(K), p == RT_PATH_TC_BF16, status, s));
+    const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
+    const bool bf16 = p == RT_PATH_TC_BF16;
+    if (rtq::xs_supported(m, n, k))
+        return from_cuda(rtq::launch_xs_q8(X, Wq, scale, Y, m, n, k, bf16, status, s));
+    return from_cuda(rtq::launch_tc_q8(X, Wq, scale, Y, m, n, k, bf16, status, s));
 }
 
 rt_status rt_qblock_project(const rt_qblock *blk, int64_t M, const float *X_qkvg,

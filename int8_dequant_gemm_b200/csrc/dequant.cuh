@@ -40,6 +40,11 @@ __device__ __forceinline__ void q4_word_f32(uint32_t v, float scale, float mn, f
 // Tensor-core operand types: both MMA operands share one 16-bit type.
 enum class Op16 { f16 = 0, bf16 = 1 };
 
+// Tensor-core operand chunks hold 8 consecutive K elements in the pair order
+// [0,2 | 1,3 | 4,6 | 5,7] (one 32-bit word per pair).  Weights and
+// activations use the same order, so the MMA's dot products are unchanged;
+// the order lets each pair come from one byte pair of the packed codes and
+// from one float4 of the activations.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&h);
@@ -56,14 +61,46 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     return OP == Op16::f16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
 }
 
-// 8 codes of one payload word -> 8 16-bit weights (the fp32 value rounded to
-// the operand type), packed low element first into one 16-byte smem chunk.
+// 4 activations (k, k+1, k+2, k+3) -> the two pair words (k,k+2), (k+1,k+3).
 template <Op16 OP>
-__device__ __forceinline__ uint4 q4_word_op(uint32_t v, float scale, float mn) {
+__device__ __forceinline__ uint2 x4_op(float4 a) {
+    return make_uint2(pack2<OP>(a.x, a.z), pack2<OP>(a.y, a.w));
+}
+
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
+__device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2 *>(&u); }
+
+// q4, fp16 operands: 8 codes of one payload word -> one chunk.  fp16 0x6400
+// is 1024 with a unit last place, so OR-ing a code into the low mantissa bits
+// gives 1024 + code exactly; subtracting 1024 is exact; fma.rn.f16x2 then
+// rounds code*scale + min once.  s2 / m2 hold the group's scale / min in both
+// halves.
+__device__ __forceinline__ uint4 q4_word_f16(uint32_t v, uint32_t s2, uint32_t m2) {
+    const uint32_t x0 = __byte_perm(v, 0u, 0x4140);   // bytes b0, b1 -> half words 0, 1
+    const uint32_t x1 = __byte_perm(v, 0u, 0x4342);   // bytes b2, b3
+    const __half2 k1024 = bits_h2(0x64006400u), s = bits_h2(s2), m = bits_h2(m2);
+    const uint32_t c0 = (x0 & 0x000F000Fu) | 0x64006400u;         // codes 0, 2
+    const uint32_t c1 = ((x0 >> 4) & 0x000F000Fu) | 0x64006400u;  // codes 1, 3
+    const uint32_t c2 = (x1 & 0x000F000Fu) | 0x64006400u;         // codes 4, 6
+    const uint32_t c3 = ((x1 >> 4) & 0x000F000Fu) | 0x64006400u;  // codes 5, 7
+    return make_uint4(h2_bits(__hfma2(__hsub2(bits_h2(c0), k1024), s, m)),
+                      h2_bits(__hfma2(__hsub2(bits_h2(c1), k1024), s, m)),
+                      h2_bits(__hfma2(__hsub2(bits_h2(c2), k1024), s, m)),
+                      h2_bits(__hfma2(__hsub2(bits_h2(c3), k1024), s, m)));
+}
+
+// (scale, min) word -> (scale, scale) and (min, min).
+__device__ __forceinline__ void q4_scale_min_f16x2(uint32_t sm, uint32_t &s2, uint32_t &m2) {
+    s2 = __byte_perm(sm, 0u, 0x1010);
+    m2 = __byte_perm(sm, 0u, 0x3232);
+}
+
+// q4, bf16 operands: the fp32 value rounded to bf16, same chunk order.
+__device__ __forceinline__ uint4 q4_word_bf16(uint32_t v, float scale, float mn) {
     float w[8];
     q4_word_f32(v, scale, mn, w);
-    return make_uint4(pack2<OP>(w[0], w[1]), pack2<OP>(w[2], w[3]), pack2<OP>(w[4], w[5]),
-                      pack2<OP>(w[6], w[7]));
+    return make_uint4(pack_bf16x2(w[0], w[2]), pack_bf16x2(w[1], w[3]), pack_bf16x2(w[4], w[6]),
+                      pack_bf16x2(w[5], w[7]));
 }
 
 // int8 code (byte i of v, two's complement) -> fp32, exact.
@@ -73,15 +110,30 @@ __device__ __forceinline__ float q8_byte_f32(uint32_t v, int i) {
     return __fsub_rn(__uint_as_float(0x4B000000u | u), 8388736.0f);
 }
 
-// Two 32-bit words (8 int8 codes, lowest address first) -> 8 16-bit codes in
-// one 16-byte chunk.  Exact in both types: |q| <= 128 needs at most 8
-// significant bits.
-template <Op16 OP>
-__device__ __forceinline__ uint4 q8_words_op(uint32_t a, uint32_t b) {
-    return make_uint4(pack2<OP>(q8_byte_f32(a, 0), q8_byte_f32(a, 1)),
-                      pack2<OP>(q8_byte_f32(a, 2), q8_byte_f32(a, 3)),
-                      pack2<OP>(q8_byte_f32(b, 0), q8_byte_f32(b, 1)),
-                      pack2<OP>(q8_byte_f32(b, 2), q8_byte_f32(b, 3)));
+// q8, fp16 operands: two payload words (codes 0..3, 4..7) -> one chunk.  The
+// offset-binary byte q + 128 under an 0x64 high byte is fp16 1024 + q + 128;
+// subtracting 1152 leaves q exactly.
+__device__ __forceinline__ uint4 q8_words_f16(uint32_t a, uint32_t b) {
+    const uint32_t ua = a ^ 0x80808080u, ub = b ^ 0x80808080u;
+    const __half2 k1152 = bits_h2(0x64806480u);
+    return make_uint4(h2_bits(__hsub2(bits_h2(__byte_perm(ua, 0x64646464u, 0x4240)), k1152)),
+                      h2_bits(__hsub2(bits_h2(__byte_perm(ua, 0x64646464u, 0x4341)), k1152)),
+                      h2_bits(__hsub2(bits_h2(__byte_perm(ub, 0x64646464u, 0x4240)), k1152)),
+                      h2_bits(__hsub2(bits_h2(__byte_perm(ub, 0x64646464u, 0x4341)), k1152)));
+}
+
+// q8, bf16 operands (exact: |q| <= 128 has at most 8 significant bits).
+__device__ __forceinline__ uint4 q8_words_bf16(uint32_t a, uint32_t b) {
+    return make_uint4(pack_bf16x2(q8_byte_f32(a, 0), q8_byte_f32(a, 2)),
+                      pack_bf16x2(q8_byte_f32(a, 1), q8_byte_f32(a, 3)),
+                      pack_bf16x2(q8_byte_f32(b, 0), q8_byte_f32(b, 2)),
+                      pack_bf16x2(q8_byte_f32(b, 1), q8_byte_f32(b, 3)));
+}
+
+// Chunk in operand order -> natural order (for the dequantization exports).
+__device__ __forceinline__ uint4 chunk_to_natural(uint4 c) {
+    return make_uint4(__byte_perm(c.x, c.y, 0x5410), __byte_perm(c.x, c.y, 0x7632),
+                      __byte_perm(c.z, c.w, 0x5410), __byte_perm(c.z, c.w, 0x7632));
 }
 
 }  // namespace rtq

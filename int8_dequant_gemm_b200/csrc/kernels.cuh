@@ -18,6 +18,14 @@ cudaError_t launch_tc_q4(const float *X, const uint8_t *Wq, const uint16_t *SM, 
 cudaError_t launch_tc_q8(const float *X, const int8_t *Wq, const float *S, float *Y, int M, int N,
                          int K, bool bf16, unsigned *status, cudaStream_t s);
 
+// tcgen05 path with the activation block resident in shared memory and the
+// weights streaming (K <= 512, many activation rows); see xs.cu.
+bool xs_supported(int M, int N, int K);
+cudaError_t launch_xs_q4(const float *X, const uint8_t *Wq, const uint16_t *SM, float *Y, int M,
+                         int N, int K, bool bf16, unsigned *status, cudaStream_t s);
+cudaError_t launch_xs_q8(const float *X, const int8_t *Wq, const float *S, float *Y, int M, int N,
+                         int K, bool bf16, unsigned *status, cudaStream_t s);
+
 // dequantization exports (same __device__ routines as the GEMMs)
 cudaError_t launch_dequant_q4_f32(const uint8_t *Wq, const uint16_t *SM, float *W, int N, int K,
                                   cudaStream_t s);

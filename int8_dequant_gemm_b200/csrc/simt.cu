@@ -209,7 +209,17 @@ __global__ void dequant_q4_16_kernel(const uint8_t *__restrict__ Wq,
     const uint32_t words[4] = {p.x, p.y, p.z, p.w};
     uint4 *dst = reinterpret_cast<uint4 *>(W + o * K + g * 32);
 #pragma unroll
-    for (int c = 0; c < 4; ++c) dst[c] = q4_word_op<OP>(words[c], sc, mn);
+    for (int c = 0; c < 4; ++c) {
+        uint4 chunk;
+        if (OP == Op16::f16) {
+            uint32_t s2, m2;
+            q4_scale_min_f16x2(__ldg(SM + o * G + g), s2, m2);
+            chunk = q4_word_f16(words[c], s2, m2);
+        } else {
+            chunk = q4_word_bf16(words[c], sc, mn);
+        }
+        dst[c] = chunk_to_natural(chunk);
+    }
 }
 
 __global__ void dequant_q8_f32_kernel(const int8_t *__restrict__ Wq, const float *__restrict__ S,

@@ -8,19 +8,23 @@
 // the instruction at full height.  The fp32 accumulator lives in TMEM: lane i
 // holds weight row o0 + i, column j holds activation row m0 + j.
 //
-// Operands are fp16 by default (q4 weights rounded once from their fp32
-// value, q8 codes exact, activations rounded to nearest-even) or bf16 on
-// request; both use tcgen05.mma kind::f16 at the same rate.  fp16 keeps 11
-// significant bits against bf16's 8, at the price of the fp16 range
-// (|X| <= 65504).
+// Operands are fp16 by default (q4 weights: the exact code*scale+min rounded
+// once by fma.rn.f16x2; q8 codes exact; activations rounded to nearest-even)
+// or bf16 on request; both use tcgen05.mma kind::f16 at the same rate.  fp16
+// keeps 11 significant bits against bf16's 8, at the price of the fp16 range
+// (|X| <= 65504).  Within every 8-element K chunk both operands store their
+// pairs in the order [0,2 | 1,3 | 4,6 | 5,7] (see dequant.cuh).
 //
 // One CTA = 8 converter warps + 1 MMA warp.  Per 64-wide K step the converter
 // warps
-//   - read the packed weight slice (q4: 32 B of codes + one (scale, min) word
-//     per group and row; q8: 64 B of codes per row), dequantize it in
-//     registers and store 16-bit operands into the A stage,
-//   - read the fp32 activation slice, round it to the operand type and store it
-//     into the B stage,
+//   - issue every global load of the step at once -- the packed weight slice
+//     (q4: 32 B of codes + one (scale, min) word per group and row; q8: 64 B
+//     of codes per row) and the fp32 activation slice, 16 threads per row in
+//     contiguous 16-byte pieces -- one step ahead of
+//     the step they convert, so a step's loads are in flight while the
+//     previous one is converted (register double buffering);
+//   - dequantize / round in registers and store 16-bit operands into the A
+//     (weights) and B (activations) stages,
 // both in the K-major 128-byte-swizzle layout the MMA descriptors describe,
 // then fence the generic->async proxy and arrive on the stage's `full`
 // mbarrier.  One thread of the MMA warp waits on `full`, issues four
@@ -28,7 +32,9 @@
 // hands the stage back to the converters once the tensor core has read it.
 // After the last K step a final commit releases the epilogue: the converter
 // warps read TMEM (32x32b loads, one weight row per thread), apply the q8 row
-// scale in fp32 and store fp32 Y with 128-byte coalesced rows.
+// scale in fp32 and store fp32 Y with 128-byte coalesced rows.  Tiles of up to
+// 128 activation rows leave room for two CTAs per SM, so one CTA's epilogue
+// overlaps the other's main loop.
 //
 // Every mbarrier wait is bounded; a wait that gives up latches
 // RT_ERR_DEVICE_TIMEOUT in the device status word and the CTA winds down.
@@ -42,12 +48,13 @@ namespace rtq {
 namespace {
 
 constexpr int kTileO = 128;                      // weight rows per tile (MMA M)
-constexpr int kTileK = 64;                       // K per stage: one 128-byte bf16 row
+constexpr int kTileK = 64;                       // K per stage: one 128-byte 16-bit row
 constexpr int kConvWarps = 8;
 constexpr int kConvThreads = kConvWarps * 32;    // 256
 constexpr int kTcThreads = kConvThreads + 32;    // + MMA warp
 constexpr int kAStageBytes = kTileO * 128;       // 16 KB
 constexpr int kMaxSmem = 227 * 1024;
+constexpr int kTwoCtaSmem = 110 * 1024;          // budget that lets two CTAs share an SM
 constexpr unsigned kStatusTimeout = 5u;          // RT_ERR_DEVICE_TIMEOUT
 
 __host__ __device__ inline int tc_stage_bytes(int bn) { return kAStageBytes + bn * 128; }
@@ -67,66 +74,114 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
     return static_cast<uint32_t>(r * 128 + ((c ^ (r & 7)) << 4));
 }
 
-// A stage, q4: thread t handles row t/2 and group (t&1) of the 64-wide slice.
-template <Op16 OP>
-__device__ __forceinline__ void fill_a_q4(uint32_t sA, const uint8_t *__restrict__ Wq,
-                                          const uint32_t *__restrict__ SM, int o0, int k0, int N,
-                                          int K, int t) {
-    const int r = t >> 1, g = t & 1;
-    const int o = o0 + r;
-    uint4 p = make_uint4(0, 0, 0, 0);
-    float sc = 0.f, mn = 0.f;
-    if (o < N) {
-        p = ldg_nc_v4(Wq + static_cast<size_t>(o) * (K / 2) + k0 / 2 + g * 16);
-        q4_scale_min(ldg_nc_u32(SM + static_cast<size_t>(o) * (K / 32) + k0 / 32 + g), sc, mn);
-    }
-    sts_v4(sA + swz(r, 4 * g + 0), q4_word_op<OP>(p.x, sc, mn));
-    sts_v4(sA + swz(r, 4 * g + 1), q4_word_op<OP>(p.y, sc, mn));
-    sts_v4(sA + swz(r, 4 * g + 2), q4_word_op<OP>(p.z, sc, mn));
-    sts_v4(sA + swz(r, 4 * g + 3), q4_word_op<OP>(p.w, sc, mn));
+// Per-thread constants of the converter role.
+//   A (weights): thread t owns row t/2 of the 128-row tile and half h = t&1 of
+//   its 64-element K slice (q4: one group of 32 codes; q8: 32 codes).
+//   B (activations): 16 threads cover one row's 64 fp32 (256 contiguous
+//   bytes) as 16-byte pieces; thread t owns piece p = t&15 of rows
+//   t/16 + 16*i, i < PIECES.
+struct ConvThread {
+    int t, ra, h, p, rb0;
+    uint32_t a_off[4];   // smem byte offsets of the thread's 4 A chunks
+    uint32_t b_off0;     // smem byte offset of its first B piece (+2048 per i)
+};
+
+__device__ __forceinline__ ConvThread conv_thread(int t) {
+    ConvThread c;
+    c.t = t;
+    c.ra = t >> 1;
+    c.h = t & 1;
+    for (int j = 0; j < 4; ++j) c.a_off[j] = swz(c.ra, 4 * c.h + j);
+    c.p = t & 15;
+    c.rb0 = t >> 4;
+    c.b_off0 = swz(c.rb0, c.p >> 1) + (c.p & 1) * 8;
+    return c;
 }
 
-// A stage, q8: thread t handles row t/2 and 32-byte half (t&1) of the slice.
-// Codes go in as exact 16-bit integers; the row scale is applied after the MMA.
-template <Op16 OP>
-__device__ __forceinline__ void fill_a_q8(uint32_t sA, const int8_t *__restrict__ Wq, int o0,
-                                          int k0, int N, int K, int t) {
-    const int r = t >> 1, h = t & 1;
-    const int o = o0 + r;
-    uint4 p0 = make_uint4(0, 0, 0, 0), p1 = make_uint4(0, 0, 0, 0);
-    if (o < N) {
-        const int8_t *src = Wq + static_cast<size_t>(o) * K + k0 + h * 32;
-        p0 = ldg_nc_v4(src);
-        p1 = ldg_nc_v4(src + 16);
-    }
-    sts_v4(sA + swz(r, 4 * h + 0), q8_words_op<OP>(p0.x, p0.y));
-    sts_v4(sA + swz(r, 4 * h + 1), q8_words_op<OP>(p0.z, p0.w));
-    sts_v4(sA + swz(r, 4 * h + 2), q8_words_op<OP>(p1.x, p1.y));
-    sts_v4(sA + swz(r, 4 * h + 3), q8_words_op<OP>(p1.z, p1.w));
-}
+// Registers holding one K step's raw data for one converter thread.
+//   A: q4 -> a0 = 16 B of codes, a1.x = the group's (scale, min);
+//      q8 -> a0, a1 = 32 B of codes.
+//   B: PIECES float4 of activations.
+template <int PIECES>
+struct StageRegs {
+    uint4 a0, a1;
+    float4 b[PIECES];
+};
 
-// B stage: BN activation rows x 64 fp32 -> 16-bit, 8 values (one chunk) per unit.
-template <Op16 OP>
-__device__ __forceinline__ void fill_b(uint32_t sB, const float *__restrict__ X, int m0, int k0,
-                                       int M, int K, int BN, int t) {
-    const int units = BN * 8;
-#pragma unroll 4
-    for (int u = t; u < units; u += kConvThreads) {
-        const int r = u >> 3, c = u & 7;
-        const int m = m0 + r;
-        float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
-        if (m < M) {
-            const float *src = X + static_cast<size_t>(m) * K + k0 + c * 8;
-            a = ldg_f4(src);
-            b = ldg_f4(src + 4);
+template <int FMT, int PIECES>
+__device__ __forceinline__ void load_stage(StageRegs<PIECES> &R, const ConvThread &c,
+                                           const float *__restrict__ X,
+                                           const void *__restrict__ Wq,
+                                           const void *__restrict__ S, int o0, int m0, int k0,
+                                           int M, int N, int K, int BN) {
+    const int o = o0 + c.ra;
+    R.a0 = make_uint4(0, 0, 0, 0);
+    R.a1 = make_uint4(0, 0, 0, 0);
+    if (o < N) {
+        if (FMT == 4) {
+            R.a0 = ldg_nc_v4(static_cast<const uint8_t *>(Wq) + static_cast<size_t>(o) * (K / 2) +
+                             k0 / 2 + c.h * 16);
+            R.a1.x = ldg_nc_u32(static_cast<const uint32_t *>(S) +
+                                static_cast<size_t>(o) * (K / 32) + k0 / 32 + c.h);
+        } else {
+            const int8_t *src =
+                static_cast<const int8_t *>(Wq) + static_cast<size_t>(o) * K + k0 + c.h * 32;
+            R.a0 = ldg_nc_v4(src);
+            R.a1 = ldg_nc_v4(src + 16);
         }
-        sts_v4(sB + swz(r, c), make_uint4(pack2<OP>(a.x, a.y), pack2<OP>(a.z, a.w),
-                                          pack2<OP>(b.x, b.y), pack2<OP>(b.z, b.w)));
+    }
+    const float *xb = X + static_cast<size_t>(m0 + c.rb0) * K + k0 + c.p * 4;
+#pragma unroll
+    for (int i = 0; i < PIECES; ++i) {
+        const int rr = c.rb0 + 16 * i;
+        R.b[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (rr < BN && m0 + rr < M) R.b[i] = ldg_f4(xb + static_cast<size_t>(16 * i) * K);
     }
 }
 
-template <int FMT, Op16 OP>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__device__ __forceinline__ void sts_v2(uint32_t saddr, uint2 v) {
+    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(saddr), "r"(v.x), "r"(v.y) : "memory");
+}
+
+template <int FMT, Op16 OP, int PIECES>
+__device__ __forceinline__ void store_stage(const StageRegs<PIECES> &R, const ConvThread &c,
+                                            uint32_t sA, uint32_t sB, int BN) {
+    if (FMT == 4) {
+        if (OP == Op16::f16) {
+            uint32_t s2, m2;
+            q4_scale_min_f16x2(R.a1.x, s2, m2);
+            sts_v4(sA + c.a_off[0], q4_word_f16(R.a0.x, s2, m2));
+            sts_v4(sA + c.a_off[1], q4_word_f16(R.a0.y, s2, m2));
+            sts_v4(sA + c.a_off[2], q4_word_f16(R.a0.z, s2, m2));
+            sts_v4(sA + c.a_off[3], q4_word_f16(R.a0.w, s2, m2));
+        } else {
+            float sc, mn;
+            q4_scale_min(R.a1.x, sc, mn);
+            sts_v4(sA + c.a_off[0], q4_word_bf16(R.a0.x, sc, mn));
+            sts_v4(sA + c.a_off[1], q4_word_bf16(R.a0.y, sc, mn));
+            sts_v4(sA + c.a_off[2], q4_word_bf16(R.a0.z, sc, mn));
+            sts_v4(sA + c.a_off[3], q4_word_bf16(R.a0.w, sc, mn));
+        }
+    } else {
+        if (OP == Op16::f16) {
+            sts_v4(sA + c.a_off[0], q8_words_f16(R.a0.x, R.a0.y));
+            sts_v4(sA + c.a_off[1], q8_words_f16(R.a0.z, R.a0.w));
+            sts_v4(sA + c.a_off[2], q8_words_f16(R.a1.x, R.a1.y));
+            sts_v4(sA + c.a_off[3], q8_words_f16(R.a1.z, R.a1.w));
+        } else {
+            sts_v4(sA + c.a_off[0], q8_words_bf16(R.a0.x, R.a0.y));
+            sts_v4(sA + c.a_off[1], q8_words_bf16(R.a0.z, R.a0.w));
+            sts_v4(sA + c.a_off[2], q8_words_bf16(R.a1.x, R.a1.y));
+            sts_v4(sA + c.a_off[3], q8_words_bf16(R.a1.z, R.a1.w));
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < PIECES; ++i)
+        if (c.rb0 + 16 * i < BN) sts_v2(sB + c.b_off0 + 2048u * i, x4_op<OP>(R.b[i]));
+}
+
+template <int FMT, Op16 OP, int PIECES>
+__global__ void __launch_bounds__(kTcThreads, 2)
     tc_qgemm_kernel(const float *__restrict__ X, const void *__restrict__ Wq,
                     const void *__restrict__ S, float *__restrict__ Y, int M, int N, int K,
                     int BN, int stages, unsigned *status) {
@@ -167,23 +222,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     pdl_wait_prior_grid();
 
     if (warp < kConvWarps) {
-        const int t = threadIdx.x;
-        for (int ks = 0; ks < nk && ok; ++ks) {
+        const ConvThread ct = conv_thread(threadIdx.x);
+        StageRegs<PIECES> r0, r1;
+        // Converts the step held in R into stage ks % stages once the MMA has
+        // released that stage.
+        auto consume = [&](const StageRegs<PIECES> &R, int ks) -> bool {
             const int s = ks % stages;
-            if (ks >= stages && !mbar_wait(&empty[s], static_cast<uint32_t>((ks / stages) - 1) & 1u)) {
-                ok = false;
-                break;
-            }
+            if (ks >= stages &&
+                !mbar_wait(&empty[s], static_cast<uint32_t>((ks / stages) - 1) & 1u))
+                return false;
             const uint32_t sA = base + s * stage_bytes;
-            const uint32_t sB = sA + kAStageBytes;
-            if (FMT == 4)
-                fill_a_q4<OP>(sA, static_cast<const uint8_t *>(Wq), static_cast<const uint32_t *>(S),
-                          o0, ks * kTileK, N, K, t);
-            else
-                fill_a_q8<OP>(sA, static_cast<const int8_t *>(Wq), o0, ks * kTileK, N, K, t);
-            fill_b<OP>(sB, X, m0, ks * kTileK, M, K, BN, t);
+            store_stage<FMT, OP, PIECES>(R, ct, sA, sA + kAStageBytes, BN);
             fence_proxy_async_smem();
             mbar_arrive(&full[s]);
+            return true;
+        };
+        load_stage<FMT, PIECES>(r0, ct, X, Wq, S, o0, m0, 0, M, N, K, BN);
+        for (int ks = 0; ks < nk; ks += 2) {
+            if (ks + 1 < nk)
+                load_stage<FMT, PIECES>(r1, ct, X, Wq, S, o0, m0, (ks + 1) * kTileK, M, N, K, BN);
+            if (!(ok = consume(r0, ks))) break;
+            if (ks + 1 >= nk) break;
+            if (ks + 2 < nk)
+                load_stage<FMT, PIECES>(r0, ct, X, Wq, S, o0, m0, (ks + 2) * kTileK, M, N, K, BN);
+            if (!(ok = consume(r1, ks + 1))) break;
         }
         pdl_launch_dependents();
         // ---------------------------------------------------------- epilogue
@@ -198,17 +260,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int o = o0 + row;
             float sc = 1.f;
             if (FMT == 8 && o < N) sc = __ldg(static_cast<const float *>(S) + o);
-            const int ncol = BN / 2;
+            const int ncol = BN / 2;           // a multiple of 8
             const int c0 = half * ncol;
-            for (int c = c0; c < c0 + ncol; c += 8) {
-                uint32_t v[8];
-                tmem_ld_x8(tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(c), v);
+            const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16);
+            for (int c = c0; c < c0 + ncol; c += 16) {
+                uint32_t v0[8], v1[8];
+                const bool two = c + 8 < c0 + ncol;
+                tmem_ld_x8(tbase + static_cast<uint32_t>(c), v0);
+                if (two) tmem_ld_x8(tbase + static_cast<uint32_t>(c + 8), v1);
                 tmem_ld_wait();
                 if (o < N) {
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const int m = m0 + c + j;
-                        if (m < M) Y[static_cast<size_t>(m) * N + o] = __uint_as_float(v[j]) * sc;
+                        if (m < M) Y[static_cast<size_t>(m) * N + o] = __uint_as_float(v0[j]) * sc;
+                    }
+                    if (two) {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const int m = m0 + c + 8 + j;
+                            if (m < M)
+                                Y[static_cast<size_t>(m) * N + o] = __uint_as_float(v1[j]) * sc;
+                        }
                     }
                 }
             }
@@ -231,7 +304,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int kk = 0; kk < kTileK / 16; ++kk) {
                 // +32 bytes per 16-element K step -> +2 in the 16-byte address field
                 tc_mma_f16kind(tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc,
-                            (ks > 0 || kk > 0) ? 1u : 0u);
+                               (ks > 0 || kk > 0) ? 1u : 0u);
             }
             tc_commit(&empty[s]);
         }
@@ -247,23 +320,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
 }
 
-template <int FMT, Op16 OP>
-cudaError_t launch_tc(const float *X, const void *Wq, const void *S, float *Y, int M, int N,
-                      int K, unsigned *status, cudaStream_t st) {
+// Activation rows per tile: one tile when M <= 128; otherwise 128, halved
+// (down to 64) while the grid would not give every SM one tile.  Each halving
+// doubles how often the weight tile is dequantized, so it stops early.
+int pick_bn(int M, int N) {
+    if (M <= 128) return std::max(16, (M + 15) / 16 * 16);
+    const int n_o = (N + kTileO - 1) / kTileO;
+    int bn = 128;
+    while (bn > 64 && static_cast<long>(n_o) * ((M + bn - 1) / bn) < 148) bn /= 2;
+    return bn;
+}
+
+template <int FMT, Op16 OP, int PIECES>
+cudaError_t launch_tc_pieces(const float *X, const void *Wq, const void *S, float *Y, int M, int N,
+                            int K, int BN, unsigned *status, cudaStream_t st) {
     static bool attr_set[64] = {false};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 64 && !attr_set[dev]) {
-        e = cudaFuncSetAttribute(tc_qgemm_kernel<FMT, OP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kMaxSmem);
+        e = cudaFuncSetAttribute(tc_qgemm_kernel<FMT, OP, PIECES>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    const int BN = M <= 256 ? std::max(16, (M + 15) / 16 * 16) : 256;
     const int nk = K / kTileK;
-    int stages = (kMaxSmem - 1024 - 256) / tc_stage_bytes(BN);
-    stages = std::max(1, std::min({stages, 6, nk}));
+    const int budget = kTwoCtaSmem;
+    int stages = (budget - 1024 - 256) / tc_stage_bytes(BN);
+    stages = std::max(1, std::min({stages, 4, nk}));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((N + kTileO - 1) / kTileO, (M + BN - 1) / BN, 1);
     cfg.blockDim = dim3(kTcThreads, 1, 1);
@@ -274,8 +358,17 @@ cudaError_t launch_tc(const float *X, const void *Wq, const void *S, float *Y, i
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, tc_qgemm_kernel<FMT, OP>, X, Wq, S, Y, M, N, K, BN, stages,
-                              status);
+    return cudaLaunchKernelEx(&cfg, tc_qgemm_kernel<FMT, OP, PIECES>, X, Wq, S, Y, M, N, K, BN,
+                              stages, status);
+}
+
+template <int FMT, Op16 OP>
+cudaError_t launch_tc(const float *X, const void *Wq, const void *S, float *Y, int M, int N,
+                      int K, unsigned *status, cudaStream_t st) {
+    const int BN = pick_bn(M, N);
+    if (BN <= 32) return launch_tc_pieces<FMT, OP, 2>(X, Wq, S, Y, M, N, K, BN, status, st);
+    if (BN <= 64) return launch_tc_pieces<FMT, OP, 4>(X, Wq, S, Y, M, N, K, BN, status, st);
+    return launch_tc_pieces<FMT, OP, 8>(X, Wq, S, Y, M, N, K, BN, status, st);
 }
 
 }  // namespace

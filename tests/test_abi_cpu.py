@@ -91,6 +91,17 @@ def test_auto_path_dispatch():
     assert rtq.auto_path(5, 80, 2048, 512) == -1
 
 
+def test_kernel_plan():
+    assert rtq.plan(4, 4, 2048, 512) == "simt"
+    assert rtq.plan(4, 80, 2048, 512) == "tc_w_stationary"
+    assert rtq.plan(4, 4096, 4096, 512) == "tc_x_resident"
+    assert rtq.plan(4, 65536, 2048, 512) == "tc_x_resident"
+    assert rtq.plan(8, 4096, 512, 2048) == "tc_w_stationary"   # K > 512 does not fit resident
+    assert rtq.plan(4, 4096, 4096, 512, "simt") == "simt"
+    assert rtq.plan(4, 4096, 4096, 96, "tc") == "rejected"
+    assert rtq.plan(4, 4096, 4096, 40) == "rejected"
+
+
 def test_block_driver_validation():
     blk = rtq._QBlockC(W, S, W, S, W, S, W, S, 0, 2048)
     assert rtq.rt_qblock_project(blk, 4, X, X, X, X, Y, Y, Y, Y, 0, None) == INVALID

@@ -4,8 +4,8 @@ Packed weights come from the ORACLE's quantizer (or are random bytes), inputs
 from the seeded workload generator, and expected values only from oracle/.
 
 Gates:
-  - dequantization exports: bit-exact (fp32 rendering = exact value rounded
-    once; fp16 / bf16 renderings = that fp32 rounded again to nearest-even);
+  - dequantization exports: bit-exact (fp32 and fp16 renderings = the exact
+    value rounded once; bf16 rendering = the fp32 one rounded again);
   - X = I turns the GEMM into W_hat^T: bit-exact on every path;
   - SIMT GEMM: max|Y - Y_ref| / max|Y_ref| <= 1e-5;
   - tensor-core GEMM (fp16 operands): <= 4e-3, and every output within the
@@ -59,14 +59,10 @@ def f16_round(x32: np.ndarray) -> np.ndarray:
     return np.asarray(x32, dtype=np.float32).astype(np.float16).astype(np.float32)
 
 
-def op_round(x32, path):
-    return f16_round(x32) if path == "tc" else bf16_round(x32)
-
-
 def assert_within_rounding_bound(Y, X, What, path):
     """Elementwise first-order bound of the tensor-core path: each product
-    x*w carries the roundings of x and w to the operand type (relative u each,
-    w also its fp32 rounding) and the fp32 accumulation adds at most K*2^-23
+    x*w carries the roundings of x and w to the operand type (relative u each;
+    the bf16 weight also its fp32 rounding) and the fp32 accumulation adds at most K*2^-23
     relative to sum|x*w|; an fp16 subnormal operand (below 2^-14) is rounded
     with an absolute error of at most 2^-25 instead."""
     u = UNIT[path]
@@ -126,7 +122,7 @@ def test_dequant_q4_exports_bit_exact(rtq_lib, N, K):
         ref16 = (bf16_round(ref32).view(np.uint32) >> 16).astype(np.uint16)
         assert np.array_equal(got16, ref16)
         goth = rtq_lib.dequant_q4_f16(dev(Wq), dev(sm)).cpu().numpy()
-        refh = ref32.astype(np.float16).view(np.uint16)
+        refh = exact.astype(np.float16).view(np.uint16)
         assert np.array_equal(goth, refh)
 
 
@@ -145,9 +141,13 @@ def test_identity_input_q4_bit_exact(rtq_lib, path):
     N, K = 384, 512
     Wq, sm = q4_weights(N, K, seed=77, outliers=True)
     Y = rtq_lib.qgemm_q4(torch.eye(K, device="cuda"), dev(Wq), dev(sm), path=path)
-    ref32 = oracle.dequant_q4(Wq, sm).astype(np.float32).T
-    if path != "simt":
-        ref32 = op_round(ref32, path)
+    exact = oracle.dequant_q4(Wq, sm)
+    if path == "simt":
+        ref32 = exact.astype(np.float32).T
+    elif path == "tc":
+        ref32 = exact.astype(np.float16).astype(np.float32).T
+    else:
+        ref32 = bf16_round(exact.astype(np.float32)).T
     assert np.array_equal(Y.cpu().numpy(), ref32)
 
 
@@ -209,6 +209,56 @@ def test_tc_parity_q4(rtq_lib, M, N, K, path):
 def test_tc_parity_q8(rtq_lib, M, N, K, path):
     Y, ref = _run_q8(rtq_lib, M, N, K, path, seed=M + 5 * N + K, outliers=True)
     assert rel_err(Y, ref) <= MAX_REL[path]
+
+
+# shapes that the activation-resident kernel takes: ragged M and N, K from 64 to
+# 512, a CTA run that crosses activation blocks
+XS_SHAPES = [(2048, 1024, 512), (2000, 1000, 512), (1500, 2100, 256), (4096, 512, 512),
+             (2048, 2048, 128), (300, 6000, 128)]
+
+
+@pytest.mark.parametrize("path", ["tc", "tc_bf16"])
+@pytest.mark.parametrize("M,N,K", XS_SHAPES)
+def test_x_resident_parity_q4(rtq_lib, M, N, K, path):
+    assert rtq_lib.plan(4, M, N, K, path) == "tc_x_resident"
+    Y, ref = _run_q4(rtq_lib, M, N, K, path, seed=M + 7 * N + K, outliers=True)
+    assert rel_err(Y, ref) <= MAX_REL[path]
+
+
+@pytest.mark.parametrize("path", ["tc", "tc_bf16"])
+@pytest.mark.parametrize("M,N,K", XS_SHAPES)
+def test_x_resident_parity_q8(rtq_lib, M, N, K, path):
+    assert rtq_lib.plan(8, M, N, K, path) == "tc_x_resident"
+    Y, ref = _run_q8(rtq_lib, M, N, K, path, seed=M + 11 * N + K, outliers=True)
+    assert rel_err(Y, ref) <= MAX_REL[path]
+
+
+def test_x_resident_long_runs_every_tile(rtq_lib):
+    """Many weight tiles per CTA and several activation-block reloads per run
+    (M = 65536, N = 2048): every 128 x 128 output tile against the fp32 SIMT
+    path on the same inputs, twice.  This is the regime in which a packed-code
+    staging slot could be refilled before its reads completed."""
+    M, N, K = 65536, 2048, 512
+    X = dev(wl.activations(M, K, 5010))
+    Wq, sm = q4_weights(N, K, 5005, outliers=True)
+    Wd, Sd = dev(Wq), dev(sm)
+    assert rtq_lib.plan(4, M, N, K) == "tc_x_resident"
+    ys = rtq_lib.qgemm_q4(X, Wd, Sd, path="simt")
+    scale = ys.abs().max()
+    for _ in range(2):
+        yt = rtq_lib.qgemm_q4(X, Wd, Sd, path="tc")
+        tile_err = ((yt - ys).abs() / scale).view(M // 128, 128, N // 128, 128).amax(dim=(1, 3))
+        assert float(tile_err.max()) <= TC_TOL, int((tile_err > TC_TOL).sum())
+
+
+def test_x_resident_identity_bit_exact(rtq_lib):
+    """X = I over four activation blocks: every output is one rounded weight."""
+    N, K = 12800, 512
+    Wq, sm = q4_weights(N, K, seed=91, outliers=True)
+    assert rtq_lib.plan(4, K, N, K) == "tc_x_resident"
+    Y = rtq_lib.qgemm_q4(torch.eye(K, device="cuda"), dev(Wq), dev(sm)).cpu().numpy()
+    ref = oracle.dequant_q4(Wq, sm).astype(np.float16).astype(np.float32).T
+    assert np.array_equal(Y, ref)
 
 
 def test_random_format_bytes_both_paths(rtq_lib):
