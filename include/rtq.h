@@ -28,8 +28,9 @@
  * the quantized projections).
  *
  * Conventions for every GEMM entry point:
- *   - Ownership: the caller allocates and owns every buffer.  The library
- *     never allocates per call and never frees caller memory.
+ *   - Ownership: the caller allocates and owns every buffer it passes.  The
+ *     library's only allocation is the activation workspace described at
+ *     rt_workspace_bytes(); it never frees caller memory.
  *   - Pointers: X, Wq, scale(_min) and Y are DEVICE pointers on the current
  *     device; `stream` is a cudaStream_t (NULL = legacy default stream).
  *   - Execution: stream-ordered and asynchronous.  RT_OK means "validated and
@@ -68,7 +69,8 @@ typedef enum rt_status {
     RT_ERR_UNSUPPORTED_SHAPE = 3, /* K not a multiple of the format's granule */
     RT_ERR_CUDA = 4,              /* a CUDA runtime call failed (launch, no device) */
     RT_ERR_DEVICE_TIMEOUT = 5,    /* a kernel's bounded wait expired (see rt_device_status) */
-    RT_ERR_VALUE_RANGE = 6        /* quantizer input not finite / outside binary16 range */
+    RT_ERR_VALUE_RANGE = 6,       /* quantizer input not finite / outside binary16 range */
+    RT_ERR_WORKSPACE = 7          /* the workspace would have to grow inside a stream capture */
 } rt_status;
 
 typedef enum rt_path {
@@ -105,18 +107,42 @@ int rt_qgemm_auto_path(int fmt, int64_t M, int64_t N, int64_t K);
 /* Kernels behind the paths:
  *   RT_KERNEL_SIMT            fp32 CUDA-core kernel, one thread per output row;
  *   RT_KERNEL_TC_W_STATIONARY tcgen05, one 128-row weight tile x up to 128
- *                             activation rows per CTA (small M, long K);
+ *                             activation rows per CTA, converter warps load and
+ *                             convert both operands (M <= 128, or shapes the
+ *                             TMA kernels do not take);
  *   RT_KERNEL_TC_X_RESIDENT   tcgen05, persistent CTAs keep a 128-row block of
- *                             activations in shared memory and stream weight
- *                             tiles past it (M >= 256, K <= 512). */
+ *                             activations in shared memory and stream TMA-staged
+ *                             weight tiles past it (M >= 256, K a multiple of
+ *                             128 up to 512);
+ *   RT_KERNEL_TC_W_STREAMED   tcgen05, persistent 128 x 128 tiles with both
+ *                             operands TMA-staged (M > 128, other K).
+ * The last two run an activation pre-pass (X rounded once to the 16-bit
+ * operand type) into a per-(device, stream) workspace of M * K * 2 bytes. */
 typedef enum rt_kernel {
     RT_KERNEL_SIMT = 1,
     RT_KERNEL_TC_W_STATIONARY = 2,
-    RT_KERNEL_TC_X_RESIDENT = 3
+    RT_KERNEL_TC_X_RESIDENT = 3,
+    RT_KERNEL_TC_W_STREAMED = 4
 } rt_kernel;
 
 /* The kernel a GEMM of this format, shape and path runs; -1 if rejected. */
 int rt_qgemm_plan(int fmt, int64_t M, int64_t N, int64_t K, int path);
+
+/*
+ * Workspace.  The TMA-fed kernels stage the activations, rounded to the
+ * 16-bit operand type, in a device buffer the library keeps per (device,
+ * stream): rt_workspace_bytes() gives the size a GEMM needs (0 for the other
+ * kernels, -1 for a rejected shape).  The buffer grows on first need with
+ * cudaMalloc; growth synchronizes that stream.  It cannot grow while the
+ * stream is being captured into a CUDA graph -- such a call returns
+ * RT_ERR_WORKSPACE -- so reserve the largest size first with
+ * rt_workspace_reserve(bytes, stream).  rt_workspace_release() synchronizes
+ * the current device and frees its workspaces.  Calls that share a stream
+ * share its workspace in stream order.
+ */
+int64_t rt_workspace_bytes(int fmt, int64_t M, int64_t N, int64_t K, int path);
+rt_status rt_workspace_reserve(int64_t bytes, void *stream);
+rt_status rt_workspace_release(void);
 
 /*
  * One RT-J block's quantized projection set, following the mixed-precision

@@ -67,6 +67,12 @@ def lib() -> ctypes.CDLL:
     L.rt_qgemm_auto_path.argtypes = [_i32, _i64, _i64, _i64]
     L.rt_qgemm_plan.restype = _i32
     L.rt_qgemm_plan.argtypes = [_i32, _i64, _i64, _i64, _i32]
+    L.rt_workspace_bytes.restype = _i64
+    L.rt_workspace_bytes.argtypes = [_i32, _i64, _i64, _i64, _i32]
+    L.rt_workspace_reserve.restype = _i32
+    L.rt_workspace_reserve.argtypes = [_i64, _p]
+    L.rt_workspace_release.restype = _i32
+    L.rt_workspace_release.argtypes = []
     L.rt_qblock_project.restype = _i32
     L.rt_qblock_project.argtypes = [ctypes.POINTER(_QBlockC), _i64, _p, _p, _p, _p, _p, _p, _p,
                                     _p, _i32, _p]
@@ -143,6 +149,18 @@ def rt_qgemm_auto_path(fmt, M, N, K) -> int:
 
 def rt_qgemm_plan(fmt, M, N, K, path) -> int:
     return lib().rt_qgemm_plan(fmt, M, N, K, path)
+
+
+def rt_workspace_bytes(fmt, M, N, K, path) -> int:
+    return lib().rt_workspace_bytes(fmt, M, N, K, path)
+
+
+def rt_workspace_reserve(nbytes, stream) -> int:
+    return lib().rt_workspace_reserve(nbytes, stream)
+
+
+def rt_workspace_release() -> int:
+    return lib().rt_workspace_release()
 
 
 # ------------------------------------------------------- torch-level helpers
@@ -309,10 +327,22 @@ def auto_path(fmt: int, M: int, N: int, K: int) -> int:
     return int(rt_qgemm_auto_path(fmt, M, N, K))
 
 
-KERNELS = {1: "simt", 2: "tc_w_stationary", 3: "tc_x_resident"}
+KERNELS = {1: "simt", 2: "tc_w_stationary", 3: "tc_x_resident", 4: "tc_w_streamed"}
 
 
 def plan(fmt: int, M: int, N: int, K: int, path="auto") -> str:
     """Name of the kernel a GEMM of this shape runs (see rt_qgemm_plan)."""
     k = int(rt_qgemm_plan(fmt, M, N, K, _path(path)))
     return KERNELS.get(k, "rejected")
+
+
+def workspace_bytes(fmt: int, M: int, N: int, K: int, path="auto") -> int:
+    return int(rt_workspace_bytes(fmt, M, N, K, _path(path)))
+
+
+def workspace_reserve(nbytes: int, stream=None):
+    _check(rt_workspace_reserve(int(nbytes), _stream_ptr(stream)), "rt_workspace_reserve")
+
+
+def workspace_release():
+    _check(rt_workspace_release(), "rt_workspace_release")

@@ -6,6 +6,7 @@
 #include <atomic>
 #include <cstdint>
 #include <mutex>
+#include <vector>
 
 #include "../../include/rtq.h"
 #include "kernels.cuh"
@@ -30,6 +31,53 @@ rt_status status_word(unsigned **out) {
         g_status_ptr[dev] = static_cast<unsigned *>(p);
     }
     *out = g_status_ptr[dev];
+    return RT_OK;
+}
+
+// Per-(device, stream) workspace for the activation pre-pass of the TMA-fed
+// kernels: M * K 16-bit values.  Grown on demand (never during stream
+// capture) and kept until rt_workspace_release().
+struct WorkspaceEntry {
+    int dev;
+    cudaStream_t stream;
+    void *ptr;
+    size_t bytes;
+};
+std::mutex g_ws_mu;
+std::vector<WorkspaceEntry> g_ws;
+
+rt_status workspace(cudaStream_t s, size_t need, void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return RT_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_ws_mu);
+    WorkspaceEntry *e = nullptr;
+    for (auto &w : g_ws)
+        if (w.dev == dev && w.stream == s) e = &w;
+    if (e && e->bytes >= need) {
+        *out = e->ptr;
+        return RT_OK;
+    }
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cap) != cudaSuccess) return RT_ERR_CUDA;
+    if (cap != cudaStreamCaptureStatusNone) return RT_ERR_WORKSPACE;
+    const size_t gran = size_t(2) << 20;
+    const size_t bytes = (need + gran - 1) / gran * gran;
+    if (e) {
+        // the old buffer may still be read by queued work on this stream
+        if (cudaStreamSynchronize(s) != cudaSuccess || cudaFree(e->ptr) != cudaSuccess)
+            return RT_ERR_CUDA;
+        e->ptr = nullptr;
+        e->bytes = 0;
+    }
+    void *p = nullptr;
+    if (cudaMalloc(&p, bytes) != cudaSuccess) return RT_ERR_CUDA;
+    if (e) {
+        e->ptr = p;
+        e->bytes = bytes;
+    } else {
+        g_ws.push_back({dev, s, p, bytes});
+    }
+    *out = p;
     return RT_OK;
 }
 
@@ -65,6 +113,14 @@ rt_status validate(const float *X, const void *Wq, const void *S, const float *Y
     return RT_OK;
 }
 
+int pick_kernel(int fmt, int64_t M, int64_t N, int64_t K, int p) {
+    if (p == RT_PATH_SIMT) return RT_KERNEL_SIMT;
+    const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
+    if (rtq::xs_supported(m, n, k)) return RT_KERNEL_TC_X_RESIDENT;
+    if (rtq::ws_supported(fmt, m, n, k)) return RT_KERNEL_TC_W_STREAMED;
+    return RT_KERNEL_TC_W_STATIONARY;
+}
+
 int pick_path(int64_t M, int64_t K, int path) {
     const bool tc_ok = (K % 64) == 0;
     if (path == RT_PATH_TC || path == RT_PATH_TC_BF16) return tc_ok ? path : -1;
@@ -74,6 +130,42 @@ int pick_path(int64_t M, int64_t K, int path) {
 }
 
 inline rt_status from_cuda(cudaError_t e) { return e == cudaSuccess ? RT_OK : RT_ERR_CUDA; }
+
+// Runs a validated GEMM on the kernel the plan picks.
+rt_status run_gemm(int fmt, const float *X, const void *Wq, const void *S, float *Y, int64_t M,
+                   int64_t N, int64_t K, int path, void *stream) {
+    const int p = pick_path(M, K, path);
+    if (p == -1) return RT_ERR_UNSUPPORTED_SHAPE;
+    if (p < 0) return RT_ERR_INVALID_ARG;
+    if (M == 0) return RT_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
+    const int kern = pick_kernel(fmt, M, N, K, p);
+    const bool q4 = fmt == 4;
+    const auto *w4 = static_cast<const uint8_t *>(Wq);
+    const auto *w8 = static_cast<const int8_t *>(Wq);
+    const auto *s4 = static_cast<const uint16_t *>(S);
+    const auto *s8 = static_cast<const float *>(S);
+    if (kern == RT_KERNEL_SIMT)
+        return from_cuda(q4 ? rtq::launch_simt_q4(X, w4, s4, Y, m, n, k, s)
+                            : rtq::launch_simt_q8(X, w8, s8, Y, m, n, k, s));
+    unsigned *status = nullptr;
+    rt_status st = status_word(&status);
+    if (st != RT_OK) return st;
+    const bool bf16 = p == RT_PATH_TC_BF16;
+    if (kern == RT_KERNEL_TC_W_STATIONARY)
+        return from_cuda(q4 ? rtq::launch_tc_q4(X, w4, s4, Y, m, n, k, bf16, status, s)
+                            : rtq::launch_tc_q8(X, w8, s8, Y, m, n, k, bf16, status, s));
+    void *xh = nullptr;
+    if ((st = workspace(s, static_cast<size_t>(M) * K * 2, &xh)) != RT_OK) return st;
+    cudaError_t e = rtq::launch_cvt_x16(X, xh, M, K, bf16, s);
+    if (e != cudaSuccess) return RT_ERR_CUDA;
+    if (kern == RT_KERNEL_TC_X_RESIDENT)
+        return from_cuda(q4 ? rtq::launch_xs_q4(xh, w4, s4, Y, m, n, k, bf16, status, s)
+                            : rtq::launch_xs_q8(xh, w8, s8, Y, m, n, k, bf16, status, s));
+    return from_cuda(q4 ? rtq::launch_ws_q4(xh, w4, s4, Y, m, n, k, bf16, status, s)
+                        : rtq::launch_ws_q8(xh, w8, s8, Y, m, n, k, bf16, status, s));
+}
 
 }  // namespace
 
@@ -88,6 +180,7 @@ const char *rt_status_string(int status) {
         case RT_ERR_CUDA: return "CUDA runtime error";
         case RT_ERR_DEVICE_TIMEOUT: return "device wait timed out";
         case RT_ERR_VALUE_RANGE: return "value out of range";
+        case RT_ERR_WORKSPACE: return "workspace must grow during stream capture";
         default: return "unknown status";
     }
 }
@@ -107,52 +200,50 @@ int rt_qgemm_plan(int fmt, int64_t M, int64_t N, int64_t K, int path) {
     if (K % (fmt == 4 ? 32 : 16) != 0) return -1;
     const int p = pick_path(M, K, path);
     if (p < 0) return -1;
-    if (p == RT_PATH_SIMT) return RT_KERNEL_SIMT;
-    return rtq::xs_supported(static_cast<int>(M), static_cast<int>(N), static_cast<int>(K))
-               ? RT_KERNEL_TC_X_RESIDENT
-               : RT_KERNEL_TC_W_STATIONARY;
+    return pick_kernel(fmt, M, N, K, p);
 }
 
 rt_status rt_qgemm_q4(const float *X, const uint8_t *Wq, const uint16_t *scale_min, float *Y,
                       int64_t M, int64_t N, int64_t K, int path, void *stream) {
     rt_status st = validate(X, Wq, scale_min, Y, M, N, K, N * (K / 2), N * (K / 32) * 4, 4, 32);
     if (st != RT_OK) return st;
-    const int p = pick_path(M, K, path);
-    if (p == -1) return RT_ERR_UNSUPPORTED_SHAPE;
-    if (p < 0) return RT_ERR_INVALID_ARG;
-    if (M == 0) return RT_OK;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (p == RT_PATH_SIMT)
-        return from_cuda(rtq::launch_simt_q4(X, Wq, scale_min, Y, static_cast<int>(M),
-                                             static_cast<int>(N), static_cast<int>(K), s));
-    unsigned *status = nullptr;
-    if ((st = status_word(&status)) != RT_OK) return st;
-    const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
-    const bool bf16 = p == RT_PATH_TC_BF16;
-    if (rtq::xs_supported(m, n, k))
-        return from_cuda(rtq::launch_xs_q4(X, Wq, scale_min, Y, m, n, k, bf16, status, s));
-    return from_cuda(rtq::launch_tc_q4(X, Wq, scale_min, Y, m, n, k, bf16, status, s));
+    return run_gemm(4, X, Wq, scale_min, Y, M, N, K, path, stream);
 }
 
 rt_status rt_qgemm_q8(const float *X, const int8_t *Wq, const float *scale, float *Y, int64_t M,
                       int64_t N, int64_t K, int path, void *stream) {
     rt_status st = validate(X, Wq, scale, Y, M, N, K, N * K, N * 4, 4, 16);
     if (st != RT_OK) return st;
-    const int p = pick_path(M, K, path);
-    if (p == -1) return RT_ERR_UNSUPPORTED_SHAPE;
-    if (p < 0) return RT_ERR_INVALID_ARG;
-    if (M == 0) return RT_OK;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (p == RT_PATH_SIMT)
-        return from_cuda(rtq::launch_simt_q8(X, Wq, scale, Y, static_cast<int>(M),
-                                             static_cast<int>(N), static_cast<int>(K), s));
-    unsigned *status = nullptr;
-    if ((st = status_word(&status)) != RT_OK) return st;
-    const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
-    const bool bf16 = p == RT_PATH_TC_BF16;
-    if (rtq::xs_supported(m, n, k))
-        return from_cuda(rtq::launch_xs_q8(X, Wq, scale, Y, m, n, k, bf16, status, s));
-    return from_cuda(rtq::launch_tc_q8(X, Wq, scale, Y, m, n, k, bf16, status, s));
+    return run_gemm(8, X, Wq, scale, Y, M, N, K, path, stream);
+}
+
+int64_t rt_workspace_bytes(int fmt, int64_t M, int64_t N, int64_t K, int path) {
+    const int kern = rt_qgemm_plan(fmt, M, N, K, path);
+    if (kern < 0) return -1;
+    if (kern == RT_KERNEL_TC_X_RESIDENT || kern == RT_KERNEL_TC_W_STREAMED) return M * K * 2;
+    return 0;
+}
+
+rt_status rt_workspace_reserve(int64_t bytes, void *stream) {
+    if (bytes < 0) return RT_ERR_INVALID_ARG;
+    void *p = nullptr;
+    return workspace(static_cast<cudaStream_t>(stream), static_cast<size_t>(bytes), &p);
+}
+
+rt_status rt_workspace_release(void) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return RT_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_ws_mu);
+    if (cudaDeviceSynchronize() != cudaSuccess) return RT_ERR_CUDA;
+    for (auto it = g_ws.begin(); it != g_ws.end();) {
+        if (it->dev == dev) {
+            cudaFree(it->ptr);
+            it = g_ws.erase(it);
+        } else {
+            ++it;
+        }
+    }
+    return RT_OK;
 }
 
 rt_status rt_qblock_project(const rt_qblock *blk, int64_t M, const float *X_qkvg,

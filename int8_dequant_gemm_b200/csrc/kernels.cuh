@@ -18,12 +18,26 @@ cudaError_t launch_tc_q4(const float *X, const uint8_t *Wq, const uint16_t *SM, 
 cudaError_t launch_tc_q8(const float *X, const int8_t *Wq, const float *S, float *Y, int M, int N,
                          int K, bool bf16, unsigned *status, cudaStream_t s);
 
-// tcgen05 path with the activation block resident in shared memory and the
-// weights streaming (K <= 512, many activation rows); see xs.cu.
+// Activation pre-pass of the TMA-fed kernels (prep.cu): X fp32 [M, K] ->
+// 16-bit [M, K] in the operand chunk order, into Xh (M * K * 2 bytes).
+cudaError_t launch_cvt_x16(const float *X, void *Xh, int64_t M, int64_t K, bool bf16,
+                           cudaStream_t s);
+
+// tcgen05, activation block resident in shared memory, TMA-streamed weights
+// (K a multiple of 128 up to 512, many activation rows); see xs.cu.  Xh is the
+// pre-pass output.
 bool xs_supported(int M, int N, int K);
-cudaError_t launch_xs_q4(const float *X, const uint8_t *Wq, const uint16_t *SM, float *Y, int M,
+cudaError_t launch_xs_q4(const void *Xh, const uint8_t *Wq, const uint16_t *SM, float *Y, int M,
                          int N, int K, bool bf16, unsigned *status, cudaStream_t s);
-cudaError_t launch_xs_q8(const float *X, const int8_t *Wq, const float *S, float *Y, int M, int N,
+cudaError_t launch_xs_q8(const void *Xh, const int8_t *Wq, const float *S, float *Y, int M, int N,
+                         int K, bool bf16, unsigned *status, cudaStream_t s);
+
+// tcgen05, persistent weight-stationary tiles with both operands TMA-staged
+// (more than 128 activation rows, any K of the format's TMA granule); see ws.cu.
+bool ws_supported(int fmt, int M, int N, int K);
+cudaError_t launch_ws_q4(const void *Xh, const uint8_t *Wq, const uint16_t *SM, float *Y, int M,
+                         int N, int K, bool bf16, unsigned *status, cudaStream_t s);
+cudaError_t launch_ws_q8(const void *Xh, const int8_t *Wq, const float *S, float *Y, int M, int N,
                          int K, bool bf16, unsigned *status, cudaStream_t s);
 
 // dequantization exports (same __device__ routines as the GEMMs)

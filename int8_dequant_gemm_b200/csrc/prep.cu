@@ -1,0 +1,86 @@
+// Activation pre-pass of the TMA-fed tensor-core kernels, and the TMA map
+// encoder they share.
+//
+// The pre-pass rounds X (fp32 [M, K]) once to the 16-bit operand type and
+// stores it in the chunk order the MMA operands use (pairs [0,2 | 1,3 | 4,6 |
+// 5,7] within every 8 elements, see dequant.cuh).  The GEMM kernels then
+// load activation tiles with TMA straight into the 128-byte-swizzled
+// operand layout, with no conversion work and at half the bytes of fp32.
+// It is a pure streaming kernel: 4 bytes read and 2 written per element.
+#include <algorithm>
+#include <mutex>
+
+#include "kernels.cuh"
+#include "tmapipe.cuh"
+
+namespace rtq {
+namespace {
+
+template <Op16 OP>
+__global__ void __launch_bounds__(256)
+    cvt_x16_kernel(const float4 *__restrict__ X, uint4 *__restrict__ Xh, int64_t n_chunks) {
+    pdl_wait_prior_grid();
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_chunks;
+         i += stride) {
+        const float4 a = __ldcs(X + 2 * i), b = __ldcs(X + 2 * i + 1);
+        const uint2 lo = x4_op<OP>(a), hi = x4_op<OP>(b);
+        Xh[i] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+    }
+    pdl_launch_dependents();
+}
+
+}  // namespace
+
+cudaError_t launch_cvt_x16(const float *X, void *Xh, int64_t M, int64_t K, bool bf16,
+                           cudaStream_t s) {
+    const int64_t n_chunks = M * K / 8;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t want = (n_chunks + 255) / 256;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>(want, 8LL * sms)), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const float4 *x4 = reinterpret_cast<const float4 *>(X);
+    uint4 *h = static_cast<uint4 *>(Xh);
+    return bf16 ? cudaLaunchKernelEx(&cfg, cvt_x16_kernel<Op16::bf16>, x4, h, n_chunks)
+                : cudaLaunchKernelEx(&cfg, cvt_x16_kernel<Op16::f16>, x4, h, n_chunks);
+}
+
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+}  // namespace
+
+bool encode_tma_2d(CUtensorMap *map, CUtensorMapDataType dt, int esize, const void *ptr,
+                   uint64_t cols, uint64_t rows, uint32_t bcols, CUtensorMapSwizzle swizzle) {
+    auto enc = get_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * static_cast<uint64_t>(esize)};
+    cuuint32_t box[2] = {bcols, static_cast<cuuint32_t>(kTileRows)};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace rtq

@@ -96,10 +96,22 @@ def test_kernel_plan():
     assert rtq.plan(4, 80, 2048, 512) == "tc_w_stationary"
     assert rtq.plan(4, 4096, 4096, 512) == "tc_x_resident"
     assert rtq.plan(4, 65536, 2048, 512) == "tc_x_resident"
-    assert rtq.plan(8, 4096, 512, 2048) == "tc_w_stationary"   # K > 512 does not fit resident
+    assert rtq.plan(8, 4096, 512, 2048) == "tc_w_streamed"     # K > 512 does not fit resident
+    assert rtq.plan(4, 200, 512, 512) == "tc_w_streamed"       # too few tiles to keep X resident
+    assert rtq.plan(4, 300, 512, 192) == "tc_w_stationary"     # q4 TMA needs K % 128
+    assert rtq.plan(8, 4096, 512, 2048, "tc_bf16") == "tc_w_streamed"
     assert rtq.plan(4, 4096, 4096, 512, "simt") == "simt"
     assert rtq.plan(4, 4096, 4096, 96, "tc") == "rejected"
     assert rtq.plan(4, 4096, 4096, 40) == "rejected"
+
+
+def test_workspace_sizes():
+    assert rtq.workspace_bytes(4, 4096, 4096, 512) == 4096 * 512 * 2
+    assert rtq.workspace_bytes(8, 4096, 512, 2048) == 4096 * 2048 * 2
+    assert rtq.workspace_bytes(4, 80, 2048, 512) == 0
+    assert rtq.workspace_bytes(4, 4, 2048, 512) == 0
+    assert rtq.workspace_bytes(4, 80, 2048, 40) == -1
+    assert rtq.rt_workspace_reserve(-1, None) == INVALID
 
 
 def test_block_driver_validation():

@@ -233,6 +233,45 @@ def test_x_resident_parity_q8(rtq_lib, M, N, K, path):
     assert rel_err(Y, ref) <= MAX_REL[path]
 
 
+# shapes that the TMA-fed weight-streamed kernel takes: K above the resident
+# limit or too few tiles to keep activations resident; ragged M and N; q4
+# chunks of (scale, min) words that end inside a chunk (K = 640)
+WS_SHAPES = [(2048, 512, 2048), (300, 640, 1024), (200, 512, 512), (1000, 700, 2048),
+             (129, 256, 640)]
+
+
+@pytest.mark.parametrize("path", ["tc", "tc_bf16"])
+@pytest.mark.parametrize("M,N,K", WS_SHAPES)
+def test_w_streamed_parity_q4(rtq_lib, M, N, K, path):
+    assert rtq_lib.plan(4, M, N, K, path) == "tc_w_streamed"
+    Y, ref = _run_q4(rtq_lib, M, N, K, path, seed=M + 13 * N + K, outliers=True)
+    assert rel_err(Y, ref) <= MAX_REL[path]
+
+
+@pytest.mark.parametrize("path", ["tc", "tc_bf16"])
+@pytest.mark.parametrize("M,N,K", WS_SHAPES)
+def test_w_streamed_parity_q8(rtq_lib, M, N, K, path):
+    assert rtq_lib.plan(8, M, N, K, path) == "tc_w_streamed"
+    Y, ref = _run_q8(rtq_lib, M, N, K, path, seed=M + 17 * N + K, outliers=True)
+    assert rel_err(Y, ref) <= MAX_REL[path]
+
+
+def test_w_streamed_many_tiles_every_tile(rtq_lib):
+    """Several 128 x 128 tiles per persistent CTA (M = 32768, N = 1024, q8,
+    K = 2048): every tile against the fp32 SIMT path, twice."""
+    M, N, K = 32768, 1024, 2048
+    X = dev(wl.activations(M, K, 6010))
+    Wq, s = q8_weights(N, K, 6005, outliers=True)
+    Wd, Sd = dev(Wq), dev(s)
+    assert rtq_lib.plan(8, M, N, K) == "tc_w_streamed"
+    ys = rtq_lib.qgemm_q8(X, Wd, Sd, path="simt")
+    scale = ys.abs().max()
+    for _ in range(2):
+        yt = rtq_lib.qgemm_q8(X, Wd, Sd, path="tc")
+        tile_err = ((yt - ys).abs() / scale).view(M // 128, 128, N // 128, 128).amax(dim=(1, 3))
+        assert float(tile_err.max()) <= TC_TOL, int((tile_err > TC_TOL).sum())
+
+
 def test_x_resident_long_runs_every_tile(rtq_lib):
     """Many weight tiles per CTA and several activation-block reloads per run
     (M = 65536, N = 2048): every 128 x 128 output tile against the fp32 SIMT
