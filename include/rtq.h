@@ -70,7 +70,8 @@ typedef enum rt_status {
     RT_ERR_CUDA = 4,              /* a CUDA runtime call failed (launch, no device) */
     RT_ERR_DEVICE_TIMEOUT = 5,    /* a kernel's bounded wait expired (see rt_device_status) */
     RT_ERR_VALUE_RANGE = 6,       /* quantizer input not finite / outside binary16 range */
-    RT_ERR_WORKSPACE = 7          /* the workspace would have to grow inside a stream capture */
+    RT_ERR_WORKSPACE = 7,         /* the workspace would have to grow inside a stream capture */
+    RT_ERR_SCRATCH_LIMIT = 8      /* rt_qgemm_noalloc: M * K * 2 > RT_NOALLOC_SCRATCH_BYTES */
 } rt_status;
 
 typedef enum rt_path {
@@ -143,6 +144,38 @@ int rt_qgemm_plan(int fmt, int64_t M, int64_t N, int64_t K, int path);
 int64_t rt_workspace_bytes(int fmt, int64_t M, int64_t N, int64_t K, int path);
 rt_status rt_workspace_reserve(int64_t bytes, void *stream);
 rt_status rt_workspace_release(void);
+
+/*
+ * The same GEMM without any device allocation (the model cards have no
+ * counterpart; this is a library convenience).  For callers that cannot
+ * allocate device memory once they are running: a serving process whose own
+ * pool already holds nearly all of HBM, so a late cudaMalloc would fail, or a
+ * latency-bound loop that cannot take the stall of the workspace's growth
+ * sync or of cudaFree.
+ *
+ * fmt = 4: Wq/scales are the q4 tensors of rt_qgemm_q4; fmt = 8: those of
+ * rt_qgemm_q8.  X, Y, M, N, K, path and stream, validation and results are
+ * as for rt_qgemm_q4/q8, and the same kernel runs (rt_qgemm_plan).  The
+ * TMA-fed kernels stage the 16-bit activations in one file-scope device
+ * array of RT_NOALLOC_SCRATCH_BYTES (16 MiB) per device instead of the
+ * per-stream workspace; a problem whose M * K * 2 exceeds it returns
+ * RT_ERR_SCRATCH_LIMIT and launches nothing (for example M * K up to 8M
+ * elements, M = 4096 x K = 2048).
+ *
+ * Set-up: the first call on a device that passes validation looks up
+ * the array's device address, which may load the library's module; make
+ * that first call before any stream capture.  No call allocates: no
+ * cudaMalloc, cudaFree or allocating library routine.
+ *
+ * Sharing: every call on a device uses the same array, which keeps the last
+ * call's contents; each call writes all of the scratch it reads before
+ * reading it.  Calls in one stream are ordered; calls that can overlap on
+ * the GPU (different streams, or host threads without ordering) race on the
+ * array and give wrong results.
+ */
+#define RT_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+rt_status rt_qgemm_noalloc(int fmt, const float *X, const void *Wq, const void *scales, float *Y,
+                           int64_t M, int64_t N, int64_t K, int path, void *stream);
 
 /*
  * One RT-J block's quantized projection set, following the mixed-precision

@@ -28,6 +28,8 @@ LIB_PATH = os.path.join(_HERE, "librtq.so")
 
 OK = 0
 RT_ERR_DEVICE_TIMEOUT = 5
+RT_ERR_SCRATCH_LIMIT = 8
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024   # RT_NOALLOC_SCRATCH_BYTES in include/rtq.h
 PATHS = {"auto": 0, "simt": 1, "tc": 2, "tc_bf16": 3}
 
 _p = ctypes.c_void_p
@@ -63,6 +65,8 @@ def lib() -> ctypes.CDLL:
         f = getattr(L, name)
         f.restype = _i32
         f.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _i32, _p]
+    L.rt_qgemm_noalloc.restype = _i32
+    L.rt_qgemm_noalloc.argtypes = [_i32, _p, _p, _p, _p, _i64, _i64, _i64, _i32, _p]
     L.rt_qgemm_auto_path.restype = _i32
     L.rt_qgemm_auto_path.argtypes = [_i32, _i64, _i64, _i64]
     L.rt_qgemm_plan.restype = _i32
@@ -107,6 +111,10 @@ def rt_qgemm_q4(X, Wq, scale_min, Y, M, N, K, path, stream) -> int:
 
 def rt_qgemm_q8(X, Wq, scale, Y, M, N, K, path, stream) -> int:
     return lib().rt_qgemm_q8(X, Wq, scale, Y, M, N, K, path, stream)
+
+
+def rt_qgemm_noalloc(fmt, X, Wq, scales, Y, M, N, K, path, stream) -> int:
+    return lib().rt_qgemm_noalloc(fmt, X, Wq, scales, Y, M, N, K, path, stream)
 
 
 def rt_qblock_project(blk, M, X_qkvg, X_o, X_ffn, X_w2, Y_qkvg, Y_o, Y_13, Y_2, path,
@@ -211,6 +219,20 @@ def qgemm_q8(X, Wq, scale, Y=None, path="auto", stream=None):
                      _dev(scale, torch.float32, "scale"), _dev(Y, torch.float32, "Y"),
                      M, N, K, _path(path), _stream_ptr(stream))
     _check(st, "rt_qgemm_q8")
+    return Y
+
+
+def qgemm_noalloc(fmt, X, Wq, scales, Y, path="auto", stream=None):
+    """rt_qgemm_q4 (fmt 4) or rt_qgemm_q8 (fmt 8) into a caller-given Y, with the
+    activation scratch in the library's fixed device array: no allocation."""
+    import torch
+    M, K = X.shape
+    N = Wq.shape[0]
+    wdt, sdt = (torch.uint8, torch.uint16) if fmt == 4 else (torch.int8, torch.float32)
+    st = rt_qgemm_noalloc(fmt, _dev(X, torch.float32, "X"), _dev(Wq, wdt, "Wq"),
+                          _dev(scales, sdt, "scales"), _dev(Y, torch.float32, "Y"),
+                          M, N, K, _path(path), _stream_ptr(stream))
+    _check(st, "rt_qgemm_noalloc")
     return Y
 
 

@@ -169,6 +169,20 @@ rt_status run_gemm(int fmt, const float *X, const void *Wq, const void *S, float
 
 }  // namespace
 
+namespace rtq {
+
+// The checks rt_qgemm_q4 (fmt 4) and rt_qgemm_q8 (fmt 8) apply, for the
+// fixed-scratch entry point in noalloc.cu.
+rt_status check_gemm_args(int fmt, const float *X, const void *Wq, const void *S, const float *Y,
+                          int64_t M, int64_t N, int64_t K) {
+    return fmt == 4 ? validate(X, Wq, S, Y, M, N, K, N * (K / 2), N * (K / 32) * 4, 4, 32)
+                    : validate(X, Wq, S, Y, M, N, K, N * K, N * 4, 4, 16);
+}
+
+rt_status device_status_word(unsigned **out) { return status_word(out); }
+
+}  // namespace rtq
+
 extern "C" {
 
 const char *rt_status_string(int status) {
@@ -181,6 +195,7 @@ const char *rt_status_string(int status) {
         case RT_ERR_DEVICE_TIMEOUT: return "device wait timed out";
         case RT_ERR_VALUE_RANGE: return "value out of range";
         case RT_ERR_WORKSPACE: return "workspace must grow during stream capture";
+        case RT_ERR_SCRATCH_LIMIT: return "problem needs more than the fixed scratch array holds";
         default: return "unknown status";
     }
 }

@@ -3,6 +3,8 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
+#include "../../include/rtq.h"
+
 namespace rtq {
 
 // fp32 CUDA-core path: one thread per output row, MT activation rows per block.
@@ -47,6 +49,12 @@ cudaError_t launch_dequant_q4_16(const uint8_t *Wq, const uint16_t *SM, uint16_t
                                  int K, bool bf16, cudaStream_t s);
 cudaError_t launch_dequant_q8_f32(const int8_t *Wq, const float *S, float *W, int N, int K,
                                   cudaStream_t s);
+
+// Argument checks of rt_qgemm_q4 / rt_qgemm_q8 (fmt 4 / 8) and the device
+// status word the tensor-core kernels latch timeouts into (api.cu).
+rt_status check_gemm_args(int fmt, const float *X, const void *Wq, const void *S, const float *Y,
+                          int64_t M, int64_t N, int64_t K);
+rt_status device_status_word(unsigned **out);
 
 // Largest M the SIMT path takes under RT_PATH_AUTO.
 constexpr int kAutoSimtMaxM = 8;

@@ -51,7 +51,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings_and_version():
-    for s in range(7):
+    for s in range(9):
         assert rtq.status_string(s) and rtq.status_string(s) != "unknown status"
     assert rtq.status_string(99) == "unknown status"
     assert rtq.lib().rt_version() >= 100
@@ -112,6 +112,23 @@ def test_workspace_sizes():
     assert rtq.workspace_bytes(4, 4, 2048, 512) == 0
     assert rtq.workspace_bytes(4, 80, 2048, 40) == -1
     assert rtq.rt_workspace_reserve(-1, None) == INVALID
+
+
+def test_noalloc_validation_and_scratch_limit():
+    # every status below is decided before any CUDA call
+    f = rtq.rt_qgemm_noalloc
+    assert f(5, X, W, S, Y, 4, 16, 64, 0, None) == INVALID          # unknown format
+    assert f(4, X, W, S, Y, 4, 16, 40, 0, None) == SHAPE            # q4 K granule
+    assert f(8, X + 4, W, S, Y, 4, 16, 64, 0, None) == ALIGN        # X alignment
+    assert f(4, X, W, S, X, 4, 16, 64, 0, None) == INVALID          # Y overlaps X
+    assert f(4, X, W, S, Y, 4, 16, 64, 9, None) == INVALID          # unknown path
+    assert f(4, X, W, S, Y, 4096, 16, 96, 2, None) == SHAPE         # forced TC needs K % 64
+    # M * K * 2 bytes of scratch above the fixed array: rejected, nothing launched
+    limit = rtq.NOALLOC_SCRATCH_BYTES
+    assert rtq.plan(8, 4096, 512, 4096) == "tc_w_streamed" and 4096 * 4096 * 2 > limit
+    assert f(8, 0x100000000, W, S, 0x300000000, 4096, 512, 4096, 0, None) == 8
+    assert rtq.plan(4, 16384, 4096, 512) == "tc_x_resident" and 16384 * 512 * 2 == limit
+    assert rtq.status_string(8) != "unknown status"
 
 
 def test_block_driver_validation():
