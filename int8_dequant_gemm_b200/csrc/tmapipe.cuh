@@ -61,6 +61,20 @@ __device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, uint32_t (&r)[16]) {
         : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+        "%28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+}
+
 // Raw bytes of one weight row for one K step, as staged by TMA: q4 -> 32 B
 // of codes (row r at r*32) plus the two (scale, min) words of its groups;
 // q8 -> 64 B of codes (row r at r*64).  The read order is rotated with the
@@ -97,11 +111,10 @@ __device__ __forceinline__ RowRaw load_row_raw(uint32_t slot, int r, uint32_t sc
     return R;
 }
 
-// Dequantizes one row's 64 weights and writes them as 8 swizzled 16-byte
-// chunks of row r of an A stage (sa = stage base).
+// Dequantizes one row's 64 weights into 8 chunks of 8 16-bit operands (in the
+// operand chunk order).
 template <int FMT, Op16 OP>
-__device__ __forceinline__ void store_row_op(const RowRaw &R, uint32_t sa, int r) {
-    uint4 ch[8];
+__device__ __forceinline__ void row_chunks(const RowRaw &R, uint4 (&ch)[8]) {
     if (FMT == 4) {
         if (OP == Op16::f16) {
             uint32_t s0, m0, s1, m1;
@@ -149,10 +162,37 @@ __device__ __forceinline__ void store_row_op(const RowRaw &R, uint32_t sa, int r
             ch[7] = q8_words_bf16(R.p3.z, R.p3.w);
         }
     }
+}
+
+// Dequantizes one row's 64 weights and writes them as 8 swizzled 16-byte
+// chunks of row r of an A stage in shared memory (sa = stage base).
+template <int FMT, Op16 OP>
+__device__ __forceinline__ void store_row_op(const RowRaw &R, uint32_t sa, int r) {
+    uint4 ch[8];
+    row_chunks<FMT, OP>(R, ch);
     const uint32_t row = sa + static_cast<uint32_t>(r * 128);
     const int rsw = r & 7;
 #pragma unroll
     for (int c = 0; c < 8; ++c) sts_v4(row + ((c ^ rsw) << 4), ch[c]);
+}
+
+// Dequantizes one row's 64 weights into 32 TMEM columns of this thread's lane
+// (ta = the warp's lane base | first column): column 4c + i holds 32-bit word
+// i of chunk c, i.e. K values 8c + 2i and 8c + 2i + 1 of the operand order.
+// Must be reached by the whole warp (tcgen05.st is warp-collective).
+template <int FMT, Op16 OP>
+__device__ __forceinline__ void tmem_row_op(const RowRaw &R, uint32_t ta) {
+    uint4 ch[8];
+    row_chunks<FMT, OP>(R, ch);
+    uint32_t w[32];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        w[4 * c + 0] = ch[c].x;
+        w[4 * c + 1] = ch[c].y;
+        w[4 * c + 2] = ch[c].z;
+        w[4 * c + 3] = ch[c].w;
+    }
+    tmem_st_x32(ta, w);
 }
 
 // ---------------------------------------------------------------- host side

@@ -26,10 +26,13 @@
 //   warps 0-7   dequantizers, two groups of 128 threads taking alternate K
 //               steps; thread r owns row r of the weight tile: it reads its 32
 //               (q4) or 64 (q8) bytes of codes, dequantizes 64 weights and
-//               writes them into a 16 KB A stage in the K-major
-//               128-byte-swizzle layout.
+//               writes them with tcgen05.st into TMEM lane r of an A stage
+//               (32 columns).  The A operand never touches shared memory,
+//               which leaves its bandwidth to the MMA's activation reads and
+//               the TMA traffic.
 //   warp 8      MMA issuer (one thread): per weight tile, K/64 stages x 4
-//               tcgen05.mma (K = 16) into one of two TMEM accumulators.
+//               tcgen05.mma (K = 16, A from TMEM, B from shared memory) into
+//               one of two TMEM accumulators.
 //   warps 9-12  epilogue: TMEM -> registers (q8 row scale) -> fp32 Y with
 //               128-byte coalesced rows, overlapping the next tile's MMAs.
 //
@@ -55,22 +58,25 @@ constexpr int kWTmaWarp = kEpiWarp0 + 4;                 // 13
 constexpr int kXTmaWarp = kWTmaWarp + 1;                 // 14
 constexpr int kXsThreads = (kXTmaWarp + 1) * 32;         // 480
 constexpr int kXAtom = kXsTileM * 128;                   // 16 KB
-constexpr int kAStages = 3;
-constexpr int kRaw = 4;                                  // packed-code ring depth (steps)
+constexpr int kAStages = 4;                              // A stages in TMEM, 32 columns each
+constexpr int kRaw = 6;                                  // packed-code ring depth (steps)
 constexpr int kRawSlot = 8 * 1024;                       // 128 rows x 64 B (q8) or 32 B (q4)
 constexpr int kScaleSlot = 8 * 1024;                     // 128 rows x 16 (scale, min) words
-constexpr uint32_t kXsTmemCols = 256;                    // 2 accumulators x 128 columns
+constexpr uint32_t kAccCols = 2 * kXsTileM;              // 2 accumulators x 128 columns
+constexpr uint32_t kAStageCols = kAtomK / 2;             // 64 16-bit values per lane
+constexpr uint32_t kXsTmemCols = 512;                    // accumulators + A stages, pow2
 constexpr unsigned kStatusTimeout = 5u;
 
+static_assert(kAccCols + kAStages * kAStageCols <= kXsTmemCols, "TMEM budget");
+
 struct XsLayout {
-    int x_off, a_off, raw_off, sc_off, bar_off, total;
+    int x_off, raw_off, sc_off, bar_off, total;
 };
 
 __host__ __device__ inline XsLayout xs_layout(int K) {
     XsLayout L;
     L.x_off = 0;
-    L.a_off = (K / kAtomK) * kXAtom;
-    L.raw_off = L.a_off + kAStages * kOpStage;
+    L.raw_off = (K / kAtomK) * kXAtom;
     L.sc_off = L.raw_off + kRaw * kRawSlot;
     L.bar_off = L.sc_off + 2 * kScaleSlot;
     // raw_full/empty[kRaw], sc_full/empty[2], a_full/empty[kAStages],
@@ -216,6 +222,8 @@ __global__ void __launch_bounds__(kXsThreads, 1)
         // ============================================================ dequantizers
         const int g = warp >> 2;                     // group: K steps ks = g, g + 2, ...
         const int r = threadIdx.x & (kDeqThreads - 1);
+        // this warp's 32 TMEM lanes (warp % 4 selects the lane quadrant)
+        const uint32_t ta = tmem + kAccCols + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         for (ItemCursor it(first, last, n_o_tiles); it.valid() && ok; it.next()) {
             const int n_local = it.item - first;
             const int b = n_local & 1;
@@ -239,12 +247,15 @@ __global__ void __launch_bounds__(kXsThreads, 1)
                     ok = false;
                     break;
                 }
-                store_row_op<FMT, OP>(R, base + L.a_off + s * kOpStage, r);
-                fence_proxy_async_smem();
+                tc_fence_after_sync();
+                tmem_row_op<FMT, OP>(R, ta + static_cast<uint32_t>(s) * kAStageCols);
+                tmem_st_wait();
+                tc_fence_before_sync();
                 mbar_arrive(&a_full[s]);
                 // the raw slot goes back only after its contents were consumed
                 // above; the proxy fence orders those generic reads before the
                 // TMA that refills it
+                fence_proxy_async_smem();
                 mbar_arrive(&raw_empty[slot]);
             }
             if (!ok) break;
@@ -282,12 +293,12 @@ __global__ void __launch_bounds__(kXsThreads, 1)
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint64_t adesc = sw128_kmajor_desc(base + L.a_off + s * kOpStage);
+                    const uint32_t at = tmem + kAccCols + static_cast<uint32_t>(s) * kAStageCols;
                     const uint64_t bdesc = sw128_kmajor_desc(base + L.x_off + ks * kXAtom);
 #pragma unroll
                     for (int kk = 0; kk < kAtomK / 16; ++kk)
-                        tc_mma_f16kind(d, adesc + 2 * kk, bdesc + 2 * kk, idesc,
-                                       (ks > 0 || kk > 0) ? 1u : 0u);
+                        tc_mma_f16kind_ts(d, at + 8 * kk, bdesc + 2 * kk, idesc,
+                                          (ks > 0 || kk > 0) ? 1u : 0u);
                     tc_commit(&a_empty[s]);
                 }
                 if (!ok) break;
@@ -316,15 +327,21 @@ __global__ void __launch_bounds__(kXsThreads, 1)
             if (FMT == 8 && o < N) sc = __ldg(S8 + o);
             const int mlim = min(kXsTileM, M - m0);
             float *yo = Y + static_cast<size_t>(m0) * N + o;
-            for (int c = 0; c < kXsTileM; c += 16) {
-                uint32_t v[16];
-                tmem_ld_x16(tq + static_cast<uint32_t>(b * kXsTileM + c), v);
+            const size_t rs = static_cast<size_t>(N);
+            for (int c = 0; c < kXsTileM; c += 32) {
+                uint32_t v[32];
+                tmem_ld_x32(tq + static_cast<uint32_t>(b * kXsTileM + c), v);
                 tmem_ld_wait();
                 if (o < N) {
+                    float *p = yo + static_cast<size_t>(c) * rs;
+                    if (c + 32 <= mlim) {
 #pragma unroll
-                    for (int jj = 0; jj < 16; ++jj)
-                        if (c + jj < mlim)
-                            yo[static_cast<size_t>(c + jj) * N] = __uint_as_float(v[jj]) * sc;
+                        for (int jj = 0; jj < 32; ++jj) p[jj * rs] = __uint_as_float(v[jj]) * sc;
+                    } else {
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj)
+                            if (c + jj < mlim) p[jj * rs] = __uint_as_float(v[jj]) * sc;
+                    }
                 }
             }
             tc_fence_before_sync();
