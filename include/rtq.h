@@ -111,11 +111,11 @@ int rt_qgemm_auto_path(int fmt, int64_t M, int64_t N, int64_t K);
  *                             activation rows per CTA, converter warps load and
  *                             convert both operands (M <= 128, or shapes the
  *                             TMA kernels do not take);
- *   RT_KERNEL_TC_X_RESIDENT   tcgen05, persistent CTAs keep a 128-row block of
+ *   RT_KERNEL_TC_X_RESIDENT   tcgen05, persistent CTAs keep a 192-row block of
  *                             activations in shared memory and stream TMA-staged
- *                             weight tiles past it (M >= 256, K a multiple of
+ *                             weight tiles past it (M > 128, K a multiple of
  *                             128 up to 512);
- *   RT_KERNEL_TC_W_STREAMED   tcgen05, persistent 128 x 128 tiles with both
+ *   RT_KERNEL_TC_W_STREAMED   tcgen05, persistent 128 x 192 tiles with both
  *                             operands TMA-staged (M > 128, other K).
  * The last two run an activation pre-pass (X rounded once to the 16-bit
  * operand type) into a per-(device, stream) workspace of M * K * 2 bytes. */

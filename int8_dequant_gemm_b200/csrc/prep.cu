@@ -71,12 +71,13 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
 }  // namespace
 
 bool encode_tma_2d(CUtensorMap *map, CUtensorMapDataType dt, int esize, const void *ptr,
-                   uint64_t cols, uint64_t rows, uint32_t bcols, CUtensorMapSwizzle swizzle) {
+                   uint64_t cols, uint64_t rows, uint32_t bcols, CUtensorMapSwizzle swizzle,
+                   uint32_t brows) {
     auto enc = get_encoder();
     if (!enc) return false;
     cuuint64_t dims[2] = {cols, rows};
     cuuint64_t strides[1] = {cols * static_cast<uint64_t>(esize)};
-    cuuint32_t box[2] = {bcols, static_cast<cuuint32_t>(kTileRows)};
+    cuuint32_t box[2] = {bcols, brows};
     cuuint32_t estr[2] = {1, 1};
     return enc(map, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,

@@ -1,7 +1,7 @@
 // Device pieces shared by the TMA-fed tcgen05 kernels (xs.cu, ws.cu):
-// TMA loads and transaction barriers, shared-memory vector accesses, the
-// 32x32b.x16 TMEM load, and the per-row dequantization step of the weight
-// stream (one thread converts one 128-byte row of a 64-wide K slice).
+// TMA loads and transaction barriers, shared-memory vector accesses, TMEM
+// loads and stores, and the half-row dequantization step of the weight
+// stream (two threads per weight row and 64-wide K step).
 #pragma once
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -61,6 +61,16 @@ __device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, uint32_t (&r)[16]) {
         : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
+        "%10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
@@ -75,71 +85,61 @@ __device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr));
 }
 
-// Raw bytes of one weight row for one K step, as staged by TMA: q4 -> 32 B
-// of codes (row r at r*32) plus the two (scale, min) words of its groups;
-// q8 -> 64 B of codes (row r at r*64).  The read order is rotated with the
-// row so that 8 consecutive threads touch all 32 banks.
-struct RowRaw {
-    uint4 p0, p1, p2, p3;
-    uint2 smw;
+// ---------------------------------------------- half-row dequantization
+// The TMA-fed kernels split every K step between two threads per weight row:
+// thread (r, h) converts K values [32h, 32h + 32) of the 64-wide step of row r
+// into 16 TMEM columns.  Each step's A stage is then written by all dequant
+// threads at once, which halves the latency from "stage free" to "stage
+// full" -- the quantity that bounds a shallow ring of TMEM stages.
+
+// One thread's raw bytes for one step: q4 -> 16 B of codes (one 32-group)
+// plus that group's (scale, min) word; q8 -> 32 B of codes.
+struct HalfRaw {
+    uint4 p0, p1;
+    uint32_t smw;
 };
 
+// Row r's codes of a staged K step (q4: 32 B per row, q8: 64 B per row).
+// q8 reads its two 16-byte chunks in an order rotated with the row, which
+// halves the bank conflicts of the 64-byte row stride.
 template <int FMT>
-__device__ __forceinline__ RowRaw load_row_raw(uint32_t slot, int r, uint32_t sc_addr) {
-    RowRaw R;
+__device__ __forceinline__ HalfRaw load_half_raw(uint32_t slot, int r, int h, uint32_t smw) {
+    HalfRaw R;
     if (FMT == 4) {
-        const uint32_t h0 = ((r >> 2) & 1) * 16;
-        const uint4 u = lds_v4(slot + r * 32 + h0);
-        const uint4 w = lds_v4(slot + r * 32 + (16 - h0));
-        R.p0 = h0 ? w : u;
-        R.p1 = h0 ? u : w;
-        R.p2 = R.p3 = make_uint4(0, 0, 0, 0);
-        R.smw = lds_v2(sc_addr);
+        R.p0 = lds_v4(slot + r * 32 + h * 16);
+        R.p1 = make_uint4(0, 0, 0, 0);
+        R.smw = smw;
     } else {
-        const int rot = (r >> 1) & 3;
-        const uint4 u0 = lds_v4(slot + r * 64 + ((0 + rot) & 3) * 16);
-        const uint4 u1 = lds_v4(slot + r * 64 + ((1 + rot) & 3) * 16);
-        const uint4 u2 = lds_v4(slot + r * 64 + ((2 + rot) & 3) * 16);
-        const uint4 u3 = lds_v4(slot + r * 64 + ((3 + rot) & 3) * 16);
-        // chunk c was read at position (c - rot) & 3
-        R.p0 = rot == 0 ? u0 : rot == 1 ? u3 : rot == 2 ? u2 : u1;
-        R.p1 = rot == 0 ? u1 : rot == 1 ? u0 : rot == 2 ? u3 : u2;
-        R.p2 = rot == 0 ? u2 : rot == 1 ? u1 : rot == 2 ? u0 : u3;
-        R.p3 = rot == 0 ? u3 : rot == 1 ? u2 : rot == 2 ? u1 : u0;
-        R.smw = make_uint2(0, 0);
+        const int rot = (r >> 1) & 1;
+        const uint4 u = lds_v4(slot + r * 64 + h * 32 + rot * 16);
+        const uint4 w = lds_v4(slot + r * 64 + h * 32 + (rot ^ 1) * 16);
+        R.p0 = rot ? w : u;
+        R.p1 = rot ? u : w;
+        R.smw = 0;
     }
     return R;
 }
 
-// Dequantizes one row's 64 weights into 8 chunks of 8 16-bit operands (in the
-// operand chunk order).
+// 32 weights of a half step -> 16 32-bit operand words (4 chunks) -> TMEM
+// columns [ta, ta + 16) of this thread's lane.  Warp-collective.
 template <int FMT, Op16 OP>
-__device__ __forceinline__ void row_chunks(const RowRaw &R, uint4 (&ch)[8]) {
+__device__ __forceinline__ void tmem_half_op(const HalfRaw &R, uint32_t ta) {
+    uint4 ch[4];
     if (FMT == 4) {
         if (OP == Op16::f16) {
-            uint32_t s0, m0, s1, m1;
-            q4_scale_min_f16x2(R.smw.x, s0, m0);
-            q4_scale_min_f16x2(R.smw.y, s1, m1);
-            ch[0] = q4_word_f16(R.p0.x, s0, m0);
-            ch[1] = q4_word_f16(R.p0.y, s0, m0);
-            ch[2] = q4_word_f16(R.p0.z, s0, m0);
-            ch[3] = q4_word_f16(R.p0.w, s0, m0);
-            ch[4] = q4_word_f16(R.p1.x, s1, m1);
-            ch[5] = q4_word_f16(R.p1.y, s1, m1);
-            ch[6] = q4_word_f16(R.p1.z, s1, m1);
-            ch[7] = q4_word_f16(R.p1.w, s1, m1);
+            uint32_t s2, m2;
+            q4_scale_min_f16x2(R.smw, s2, m2);
+            ch[0] = q4_word_f16(R.p0.x, s2, m2);
+            ch[1] = q4_word_f16(R.p0.y, s2, m2);
+            ch[2] = q4_word_f16(R.p0.z, s2, m2);
+            ch[3] = q4_word_f16(R.p0.w, s2, m2);
         } else {
-            float sc0, mn0, sc1, mn1;
-            q4_scale_min(R.smw.x, sc0, mn0);
-            q4_scale_min(R.smw.y, sc1, mn1);
-            ch[0] = q4_word_bf16(R.p0.x, sc0, mn0);
-            ch[1] = q4_word_bf16(R.p0.y, sc0, mn0);
-            ch[2] = q4_word_bf16(R.p0.z, sc0, mn0);
-            ch[3] = q4_word_bf16(R.p0.w, sc0, mn0);
-            ch[4] = q4_word_bf16(R.p1.x, sc1, mn1);
-            ch[5] = q4_word_bf16(R.p1.y, sc1, mn1);
-            ch[6] = q4_word_bf16(R.p1.z, sc1, mn1);
-            ch[7] = q4_word_bf16(R.p1.w, sc1, mn1);
+            float sc, mn;
+            q4_scale_min(R.smw, sc, mn);
+            ch[0] = q4_word_bf16(R.p0.x, sc, mn);
+            ch[1] = q4_word_bf16(R.p0.y, sc, mn);
+            ch[2] = q4_word_bf16(R.p0.z, sc, mn);
+            ch[3] = q4_word_bf16(R.p0.w, sc, mn);
         }
     } else {
         if (OP == Op16::f16) {
@@ -147,59 +147,50 @@ __device__ __forceinline__ void row_chunks(const RowRaw &R, uint4 (&ch)[8]) {
             ch[1] = q8_words_f16(R.p0.z, R.p0.w);
             ch[2] = q8_words_f16(R.p1.x, R.p1.y);
             ch[3] = q8_words_f16(R.p1.z, R.p1.w);
-            ch[4] = q8_words_f16(R.p2.x, R.p2.y);
-            ch[5] = q8_words_f16(R.p2.z, R.p2.w);
-            ch[6] = q8_words_f16(R.p3.x, R.p3.y);
-            ch[7] = q8_words_f16(R.p3.z, R.p3.w);
         } else {
             ch[0] = q8_words_bf16(R.p0.x, R.p0.y);
             ch[1] = q8_words_bf16(R.p0.z, R.p0.w);
             ch[2] = q8_words_bf16(R.p1.x, R.p1.y);
             ch[3] = q8_words_bf16(R.p1.z, R.p1.w);
-            ch[4] = q8_words_bf16(R.p2.x, R.p2.y);
-            ch[5] = q8_words_bf16(R.p2.z, R.p2.w);
-            ch[6] = q8_words_bf16(R.p3.x, R.p3.y);
-            ch[7] = q8_words_bf16(R.p3.z, R.p3.w);
         }
     }
-}
-
-// Dequantizes one row's 64 weights and writes them as 8 swizzled 16-byte
-// chunks of row r of an A stage in shared memory (sa = stage base).
-template <int FMT, Op16 OP>
-__device__ __forceinline__ void store_row_op(const RowRaw &R, uint32_t sa, int r) {
-    uint4 ch[8];
-    row_chunks<FMT, OP>(R, ch);
-    const uint32_t row = sa + static_cast<uint32_t>(r * 128);
-    const int rsw = r & 7;
+    uint32_t w[16];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) sts_v4(row + ((c ^ rsw) << 4), ch[c]);
-}
-
-// Dequantizes one row's 64 weights into 32 TMEM columns of this thread's lane
-// (ta = the warp's lane base | first column): column 4c + i holds 32-bit word
-// i of chunk c, i.e. K values 8c + 2i and 8c + 2i + 1 of the operand order.
-// Must be reached by the whole warp (tcgen05.st is warp-collective).
-template <int FMT, Op16 OP>
-__device__ __forceinline__ void tmem_row_op(const RowRaw &R, uint32_t ta) {
-    uint4 ch[8];
-    row_chunks<FMT, OP>(R, ch);
-    uint32_t w[32];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < 4; ++c) {
         w[4 * c + 0] = ch[c].x;
         w[4 * c + 1] = ch[c].y;
         w[4 * c + 2] = ch[c].z;
         w[4 * c + 3] = ch[c].w;
     }
-    tmem_st_x32(ta, w);
+    tmem_st_x16(ta, w);
+}
+
+// The (scale, min) words of row r for 8 K steps: a 64-byte row of a staged
+// block (16 words, groups 0..15 of the block).  Thread (r, h) keeps word
+// 2i + h, the group of step i's half h.  The four 16-byte reads are rotated
+// with the row so that 8 consecutive rows hit 32 different banks.
+__device__ __forceinline__ void load_scale_words(uint32_t row, int r, int h, uint32_t (&sw)[8]) {
+    const int rot = (r >> 1) & 3;
+    uint4 u[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) u[c] = lds_v4(row + ((c + rot) & 3) * 16);
+    // u[c] holds chunk (c + rot) & 3; chunk k therefore sits at u[(k - rot) & 3]
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int i0 = (k - 0) & 3, i1 = (k - 1) & 3, i2 = (k - 2) & 3, i3 = (k - 3) & 3;
+        const uint4 v = rot == 0 ? u[i0] : rot == 1 ? u[i1] : rot == 2 ? u[i2] : u[i3];
+        // chunk k = words 4k .. 4k + 3 = steps 2k (words 4k, 4k + 1) and 2k + 1
+        sw[2 * k] = h ? v.y : v.x;
+        sw[2 * k + 1] = h ? v.w : v.z;
+    }
 }
 
 // ---------------------------------------------------------------- host side
 // Row-major 2-D tensor [rows, cols] of `esize`-byte elements as a TMA map
-// with box {bcols, 128}; swizzle as given.  Returns false if the driver
+// with box {bcols, brows}; swizzle as given.  Returns false if the driver
 // rejects it.
 bool encode_tma_2d(CUtensorMap *map, CUtensorMapDataType dt, int esize, const void *ptr,
-                   uint64_t cols, uint64_t rows, uint32_t bcols, CUtensorMapSwizzle swizzle);
+                   uint64_t cols, uint64_t rows, uint32_t bcols, CUtensorMapSwizzle swizzle,
+                   uint32_t brows = kTileRows);
 
 }  // namespace rtq

@@ -2,21 +2,25 @@
 // stationary, TMA streams both operands' raw data through a stage ring.
 //
 // Tile product as in tc.cu / xs.cu, D[o, m] = sum_k W_hat[o, k] * X[m, k],
-// 128 weight rows (MMA M) x 128 activation rows (MMA N), full K per tile.
+// 128 weight rows (MMA M) x 192 activation rows (MMA N), full K per tile.
 // A persistent CTA (one per SM) walks tiles t = blockIdx.x, + gridDim.x, ...
 // in weight-tile-fastest order, so concurrently running CTAs share activation
 // tiles in L2.
 //
 // Per 64-wide K step one stage holds
-//   A: the 128 x 64 dequantized weights (written by the dequantizers from
-//      TMA-staged packed codes, as in xs.cu), and
-//   B: the 128 x 64 16-bit activations, one TMA box from the pre-converted
-//      activations (prep.cu) in the 128-byte-swizzled operand layout.
-// Roles (15 warps): warps 0-7 dequantizers (two groups of 128 threads on
-// alternate K steps, thread = weight row), warp 8 MMA issuer, warps 9-12
-// epilogue (double-buffered TMEM accumulators), warp 13 weight TMA (codes and,
-// for q4, (scale, min) blocks of up to 16 words per row), warp 14 activation
-// TMA.
+//   A: the 128 x 64 dequantized weights in 32 TMEM columns (written with
+//      tcgen05.st by the dequantizers from TMA-staged packed codes, as in
+//      xs.cu), and
+//   B: the 128 x 64 16-bit activations in shared memory, one TMA box from the
+//      pre-converted activations (prep.cu) in the 128-byte-swizzled operand
+//      layout.
+// The A and B rings are separate: TMEM holds two 192-column accumulators and
+// four 32-column A stages (512 columns); shared memory holds six B stages.
+// Roles (19 warps): warps 0-7 dequantizers (thread (r, h) converts half h of
+// every K step of weight row r, as in xs.cu), warp 8 MMA issuer, warps 9-16
+// epilogue (two per TMEM lane quadrant, double-buffered accumulators), warp 17
+// weight TMA (codes and, for q4, (scale, min) blocks of up to 16 words per
+// row), warp 18 activation TMA.
 //
 // Every mbarrier wait is bounded; a wait that gives up latches
 // RT_ERR_DEVICE_TIMEOUT in the device status word and the CTA winds down.
@@ -28,24 +32,31 @@
 namespace rtq {
 namespace {
 
-constexpr int kWsTileM = 128;                 // activation rows per tile (MMA N)
-constexpr int kDeqGroups = 2;
+constexpr int kWsTileM = 192;                 // activation rows per tile (MMA N)
+constexpr int kDeqGroups = 2;                            // two K halves per step
 constexpr int kDeqThreads = kTileRows;                   // 128 per group
 constexpr int kDeqWarps = kDeqGroups * 4;                // 8
 constexpr int kMmaWarp = kDeqWarps;                      // 8
 constexpr int kEpiWarp0 = kMmaWarp + 1;                  // 9
-constexpr int kEpiThreads = 128;
-constexpr int kWTmaWarp = kEpiWarp0 + 4;                 // 13
-constexpr int kXTmaWarp = kWTmaWarp + 1;                 // 14
-constexpr int kWsThreads = (kXTmaWarp + 1) * 32;         // 480
-constexpr int kStages = 4;
-constexpr int kStageBytes = 2 * kOpStage;                // A + B, 32 KB
+constexpr int kEpiWarps = 8;                             // two per TMEM lane quadrant
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kEpiCols = kWsTileM / 2;
+constexpr int kWTmaWarp = kEpiWarp0 + kEpiWarps;         // 17
+constexpr int kXTmaWarp = kWTmaWarp + 1;                 // 18
+constexpr int kWsThreads = (kXTmaWarp + 1) * 32;         // 608
+constexpr int kStages = 6;                               // B stages (shared memory)
+constexpr int kStageBytes = kWsTileM * 128;              // 24 KB: 192 rows x 64 K
+constexpr int kAStages = 4;                              // A stages (TMEM)
 constexpr int kRaw = 6;
 constexpr int kRawSlot = 8 * 1024;
 constexpr int kScaleSlot = 8 * 1024;                     // 128 rows x 16 words
 constexpr int kScaleWords = 16;                          // (scale, min) words per chunk row
 constexpr int kChunkSteps = kScaleWords / 2;             // K steps covered by one chunk
-constexpr uint32_t kWsTmemCols = 256;
+constexpr uint32_t kAccCols = 2 * kWsTileM;              // 2 accumulators x 192 columns
+constexpr uint32_t kAStageCols = kAtomK / 2;
+constexpr uint32_t kWsTmemCols = 512;
+static_assert(kAccCols + kAStages * kAStageCols <= kWsTmemCols, "TMEM budget");
+static_assert(kEpiCols % 32 == 0, "epilogue reads 32 columns at a time");
 constexpr unsigned kStatusTimeout = 5u;
 
 struct WsLayout {
@@ -58,9 +69,9 @@ __host__ __device__ inline WsLayout ws_layout() {
     L.raw_off = kStages * kStageBytes;
     L.sc_off = L.raw_off + kRaw * kRawSlot;
     L.bar_off = L.sc_off + 2 * kScaleSlot;
-    // a_full/b_full/st_empty[kStages], raw_full/empty[kRaw], sc_full/empty[2],
-    // acc_full/empty[2], + TMEM address slot
-    L.total = L.bar_off + (3 * kStages + 2 * kRaw + 4 + 4) * 8 + 16;
+    // a_full/a_empty[kAStages], b_full/b_empty[kStages], raw_full/empty[kRaw],
+    // sc_full/empty[2], acc_full/empty[2], + TMEM address slot
+    L.total = L.bar_off + (2 * kAStages + 2 * kStages + 2 * kRaw + 4 + 4) * 8 + 16;
     return L;
 }
 
@@ -78,9 +89,10 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     const WsLayout L = ws_layout();
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bar_off);
     uint64_t *a_full = bars;
-    uint64_t *b_full = a_full + kStages;
-    uint64_t *st_empty = b_full + kStages;
-    uint64_t *raw_full = st_empty + kStages;
+    uint64_t *a_empty = a_full + kAStages;
+    uint64_t *b_full = a_empty + kAStages;
+    uint64_t *b_empty = b_full + kStages;
+    uint64_t *raw_full = b_empty + kStages;
     uint64_t *raw_empty = raw_full + kRaw;
     uint64_t *sc_full = raw_empty + kRaw;
     uint64_t *sc_empty = sc_full + 2;
@@ -95,14 +107,17 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     const uint32_t raw_bytes = kTileRows * (FMT == 4 ? 32 : 64);
 
     if (threadIdx.x == 0) {
+        for (int s = 0; s < kAStages; ++s) {
+            mbar_init(&a_full[s], kDeqGroups * kDeqThreads);
+            mbar_init(&a_empty[s], 1);
+        }
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&a_full[s], kDeqThreads);
             mbar_init(&b_full[s], 1);
-            mbar_init(&st_empty[s], 1);
+            mbar_init(&b_empty[s], 1);
         }
         for (int i = 0; i < kRaw; ++i) {
             mbar_init(&raw_full[i], 1);
-            mbar_init(&raw_empty[i], kDeqThreads);
+            mbar_init(&raw_empty[i], kDeqGroups * kDeqThreads);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sc_full[b], 1);
@@ -164,12 +179,12 @@ __global__ void __launch_bounds__(kWsThreads, 1)
                 for (int ks = 0; ks < nk; ++ks, ++j) {
                     const int s = j % kStages;
                     if (j >= kStages &&
-                        !mbar_wait(&st_empty[s], static_cast<uint32_t>((j / kStages) - 1) & 1u)) {
+                        !mbar_wait(&b_empty[s], static_cast<uint32_t>((j / kStages) - 1) & 1u)) {
                         ok = false;
                         break;
                     }
-                    mbar_expect_tx(&b_full[s], kWsTileM * 128);
-                    tma_load_2d(base + L.st_off + s * kStageBytes + kOpStage, &x_map,
+                    mbar_expect_tx(&b_full[s], kStageBytes);
+                    tma_load_2d(base + L.st_off + s * kStageBytes, &x_map,
                                 ks * kAtomK, m0, &b_full[s]);
                 }
             }
@@ -177,41 +192,52 @@ __global__ void __launch_bounds__(kWsThreads, 1)
         __syncwarp();
     } else if (warp < kDeqWarps) {
         // ============================================================ dequantizers
-        const int g = warp >> 2;
+        const int h = warp >> 2;                     // K half [32h, 32h + 32) of every step
         const int r = threadIdx.x & (kDeqThreads - 1);
+        const uint32_t ta = tmem + kAccCols + (static_cast<uint32_t>((warp & 3) * 32) << 16) +
+                            static_cast<uint32_t>(16 * h);
         int tile_local = 0;
         for (int t = blockIdx.x; t < n_tiles && ok; t += G, ++tile_local) {
             for (int c = 0; c < n_chunks && ok; ++c) {
                 const int q = tile_local * n_chunks + c;
                 const int b = q & 1;
-                if (FMT == 4 && !mbar_wait(&sc_full[b], static_cast<uint32_t>(q / 2) & 1u)) {
-                    ok = false;
-                    break;
+                uint32_t sw[kChunkSteps] = {};
+                if (FMT == 4) {
+                    if (!mbar_wait(&sc_full[b], static_cast<uint32_t>(q / 2) & 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    load_scale_words(base + L.sc_off + b * kScaleSlot + r * (kScaleWords * 4), r,
+                                     h, sw);
+                    fence_proxy_async_smem();       // sw depends on every word read
+                    mbar_arrive(&sc_empty[b]);
                 }
-                const uint32_t sc_row = base + L.sc_off + b * kScaleSlot + r * (kScaleWords * 4);
-                const int ks_end = min(nk, (c + 1) * kChunkSteps);
-                for (int ks = c * kChunkSteps + g; ks < ks_end; ks += kDeqGroups) {
+#pragma unroll
+                for (int i = 0; i < kChunkSteps; ++i) {
+                    const int ks = c * kChunkSteps + i;
+                    if (ks >= nk) break;
                     const int j = tile_local * nk + ks;
                     const int slot = j % kRaw;
                     if (!mbar_wait(&raw_full[slot], static_cast<uint32_t>(j / kRaw) & 1u)) {
                         ok = false;
                         break;
                     }
-                    const RowRaw R = load_row_raw<FMT>(base + L.raw_off + slot * kRawSlot, r,
-                                                       sc_row + (ks % kChunkSteps) * 8);
-                    const int s = j % kStages;
-                    if (j >= kStages &&
-                        !mbar_wait(&st_empty[s], static_cast<uint32_t>((j / kStages) - 1) & 1u)) {
+                    const HalfRaw R =
+                        load_half_raw<FMT>(base + L.raw_off + slot * kRawSlot, r, h, sw[i]);
+                    const int s = j % kAStages;
+                    if (j >= kAStages &&
+                        !mbar_wait(&a_empty[s], static_cast<uint32_t>((j / kAStages) - 1) & 1u)) {
                         ok = false;
                         break;
                     }
-                    store_row_op<FMT, OP>(R, base + L.st_off + s * kStageBytes, r);
-                    fence_proxy_async_smem();
+                    tc_fence_after_sync();
+                    tmem_half_op<FMT, OP>(R, ta + static_cast<uint32_t>(s) * kAStageCols);
+                    tmem_st_wait();
+                    tc_fence_before_sync();
                     mbar_arrive(&a_full[s]);
+                    fence_proxy_async_smem();
                     mbar_arrive(&raw_empty[slot]);   // after its contents were consumed
                 }
-                if (!ok) break;
-                if (FMT == 4) mbar_arrive(&sc_empty[b]);
             }
         }
     } else if (warp == kMmaWarp) {
@@ -219,6 +245,14 @@ __global__ void __launch_bounds__(kWsThreads, 1)
         if (lane == 0) {
             const uint32_t idesc =
                 idesc_f16kind_f32acc(kTileRows, kWsTileM, static_cast<uint32_t>(OP));
+            // As in xs.cu: the wait for step j + 1's stages sits between the
+            // second and third MMA of step j, so that it overlaps queued MMAs.
+            constexpr uint64_t kStageDesc = kStageBytes >> 4;   // descriptor step per B stage
+            const uint64_t bdesc0 = sw128_kmajor_desc(base + L.st_off);
+            auto ready = [&](int jj) {
+                return mbar_wait(&a_full[jj % kAStages], static_cast<uint32_t>(jj / kAStages) & 1u) &&
+                       mbar_wait(&b_full[jj % kStages], static_cast<uint32_t>(jj / kStages) & 1u);
+            };
             int j = 0, tile_local = 0;
             for (int t = blockIdx.x; t < n_tiles && ok; t += G, ++tile_local) {
                 const int b = tile_local & 1;
@@ -227,24 +261,25 @@ __global__ void __launch_bounds__(kWsThreads, 1)
                     ok = false;
                     break;
                 }
+                if (!ready(j)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after_sync();
                 const uint32_t d = tmem + static_cast<uint32_t>(b * kWsTileM);
                 for (int ks = 0; ks < nk; ++ks, ++j) {
-                    const int s = j % kStages;
-                    const uint32_t par = static_cast<uint32_t>(j / kStages) & 1u;
-                    if (!mbar_wait(&a_full[s], par) || !mbar_wait(&b_full[s], par)) {
-                        ok = false;
-                        break;
-                    }
+                    const int s = j % kAStages, sb = j % kStages;
+                    const uint32_t at = tmem + kAccCols + static_cast<uint32_t>(s) * kAStageCols;
+                    const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(sb) * kStageDesc;
+                    tc_mma_f16kind_ts(d, at, bdesc, idesc, ks > 0 ? 1u : 0u);
+                    tc_mma_f16kind_ts(d, at + 8, bdesc + 2, idesc, 1u);
+                    if (ks + 1 < nk && !ready(j + 1)) ok = false;
+                    tc_mma_f16kind_ts(d, at + 16, bdesc + 4, idesc, 1u);
+                    tc_mma_f16kind_ts(d, at + 24, bdesc + 6, idesc, 1u);
+                    tc_commit(&a_empty[s]);
+                    tc_commit(&b_empty[sb]);
+                    if (!ok) break;
                     tc_fence_after_sync();
-                    const uint32_t sa = base + L.st_off + s * kStageBytes;
-                    const uint64_t adesc = sw128_kmajor_desc(sa);
-                    const uint64_t bdesc = sw128_kmajor_desc(sa + kOpStage);
-#pragma unroll
-                    for (int kk = 0; kk < kAtomK / 16; ++kk)
-                        tc_mma_f16kind(d, adesc + 2 * kk, bdesc + 2 * kk, idesc,
-                                       (ks > 0 || kk > 0) ? 1u : 0u);
-                    tc_commit(&st_empty[s]);
                 }
                 if (!ok) break;
                 tc_commit(&acc_full[b]);
@@ -254,6 +289,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     } else {
         // ============================================================ epilogue
         const int qd = warp & 3;
+        const int c0 = ((warp - kEpiWarp0) >> 2) * kEpiCols;   // its half of the columns
         const int row = qd * 32 + lane;
         const uint32_t tq = tmem + (static_cast<uint32_t>(qd * 32) << 16);
         int tile_local = 0;
@@ -269,15 +305,21 @@ __global__ void __launch_bounds__(kWsThreads, 1)
             if (FMT == 8 && o < N) sc = __ldg(S8 + o);
             const int mlim = min(kWsTileM, M - m0);
             float *yo = Y + static_cast<size_t>(m0) * N + o;
-            for (int c = 0; c < kWsTileM; c += 16) {
-                uint32_t v[16];
-                tmem_ld_x16(tq + static_cast<uint32_t>(b * kWsTileM + c), v);
+            const size_t rs = static_cast<size_t>(N);
+            for (int c = c0; c < c0 + kEpiCols; c += 32) {
+                uint32_t v[32];
+                tmem_ld_x32(tq + static_cast<uint32_t>(b * kWsTileM + c), v);
                 tmem_ld_wait();
                 if (o < N) {
+                    float *p = yo + static_cast<size_t>(c) * rs;
+                    if (c + 32 <= mlim) {
 #pragma unroll
-                    for (int jj = 0; jj < 16; ++jj)
-                        if (c + jj < mlim)
-                            yo[static_cast<size_t>(c + jj) * N] = __uint_as_float(v[jj]) * sc;
+                        for (int jj = 0; jj < 32; ++jj) p[jj * rs] = __uint_as_float(v[jj]) * sc;
+                    } else {
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj)
+                            if (c + jj < mlim) p[jj * rs] = __uint_as_float(v[jj]) * sc;
+                    }
                 }
             }
             tc_fence_before_sync();
@@ -310,7 +352,7 @@ cudaError_t launch_ws(const void *Xh, const void *Wq, const void *S, float *Y, i
     CUtensorMap w_map, s_map, x_map;
     bool enc_ok = encode_tma_2d(&x_map, OP == Op16::f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                         : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                                2, Xh, K, M, kAtomK, CU_TENSOR_MAP_SWIZZLE_128B);
+                                2, Xh, K, M, kAtomK, CU_TENSOR_MAP_SWIZZLE_128B, kWsTileM);
     if (FMT == 4) {
         enc_ok = enc_ok &&
                  encode_tma_2d(&w_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Wq, K / 2, N, 32,
@@ -344,13 +386,12 @@ cudaError_t launch_ws(const void *Xh, const void *Wq, const void *S, float *Y, i
 
 }  // namespace
 
-// Shapes the TMA-fed weight-stationary kernel takes: more than one
-// 128-row activation tile, and K a multiple of 64 (q8) or 128 (q4: the
-// (scale, min) rows are TMA boxes whose global stride K/8 bytes must be a
-// multiple of 16).
+// Shapes the TMA-fed weight-streamed kernel takes: more than 128 activation
+// rows, and K a multiple of 64 (q8) or 128 (q4: the (scale, min) rows are TMA
+// boxes whose global stride K/8 bytes must be a multiple of 16).
 bool ws_supported(int fmt, int M, int N, int K) {
     (void)N;
-    if (M <= kWsTileM) return false;
+    if (M <= kTileRows) return false;
     return fmt == 4 ? K % 128 == 0 : K % 64 == 0;
 }
 

@@ -16,25 +16,27 @@
 // order, split into one contiguous run per CTA (one CTA per SM), so a CTA
 // changes activation block rarely.
 //
-// Roles (15 warps):
-//   warp 14     activation TMA (one thread): on every change of activation
+// Roles (19 warps):
+//   warp 18     activation TMA (one thread): on every change of activation
 //               block, once the MMAs on the previous block have completed,
 //               K/64 boxes into the resident tile, one transaction barrier.
-//   warp 13     weight TMA (one thread): per weight tile the (scale, min)
-//               block of its 128 rows (q4), and per 64-wide K step the
-//               128-row slice of packed codes, into rings kRaw steps deep.
-//   warps 0-7   dequantizers, two groups of 128 threads taking alternate K
-//               steps; thread r owns row r of the weight tile: it reads its 32
-//               (q4) or 64 (q8) bytes of codes, dequantizes 64 weights and
-//               writes them with tcgen05.st into TMEM lane r of an A stage
-//               (32 columns).  The A operand never touches shared memory,
+//   warp 17     weight TMA (one thread): per weight tile the (scale, min)
+//               words of its 128 rows (q4), and per 64-wide K step the
+//               128-row slice of packed codes, into a ring kRaw steps deep.
+//   warps 0-7   dequantizers: thread (r, h) converts K values [32h, 32h + 32)
+//               of every K step of weight row r (16 or 32 bytes of codes) and
+//               writes them with tcgen05.st into TMEM lane r of the step's A
+//               stage (16 of its 32 columns).  All 256 threads work on the
+//               same step, so a stage is refilled quickly once the MMAs that
+//               read it complete.  The A operand never touches shared memory,
 //               which leaves its bandwidth to the MMA's activation reads and
 //               the TMA traffic.
 //   warp 8      MMA issuer (one thread): per weight tile, K/64 stages x 4
 //               tcgen05.mma (K = 16, A from TMEM, B from shared memory) into
 //               one of two TMEM accumulators.
-//   warps 9-12  epilogue: TMEM -> registers (q8 row scale) -> fp32 Y with
-//               128-byte coalesced rows, overlapping the next tile's MMAs.
+//   warps 9-16  epilogue, two warps per TMEM lane quadrant: TMEM ->
+//               registers (q8 row scale) -> fp32 Y with 128-byte coalesced
+//               rows, overlapping the next tile's MMAs.
 //
 // Every mbarrier wait is bounded; a wait that gives up latches
 // RT_ERR_DEVICE_TIMEOUT in the device status word and the CTA winds down.
@@ -46,39 +48,53 @@
 namespace rtq {
 namespace {
 
-constexpr int kXsTileM = 128;                 // activation rows per block (MMA N)
+// MMA N.  An M = 128, K = 16 tcgen05.mma costs about the same time for any
+// N up to 192 and only a little more at 256, so the tile is as wide as TMEM
+// allows with two accumulators and the A stages: 2 x 192 + 4 x 32 = 512
+// columns.  192 resident rows of K = 512 also just fit in shared memory.
+constexpr int kXsTileM = 192;                 // activation rows per block (MMA N)
 constexpr int kXsMaxK = 512;
-constexpr int kDeqGroups = 2;
-constexpr int kDeqThreads = kTileRows;                   // 128 per group
+constexpr int kDeqGroups = 2;                            // two K halves per step
+constexpr int kDeqThreads = kTileRows;                   // 128 per half
 constexpr int kDeqWarps = kDeqGroups * 4;                // 8
 constexpr int kMmaWarp = kDeqWarps;                      // 8
 constexpr int kEpiWarp0 = kMmaWarp + 1;                  // 9
-constexpr int kEpiThreads = 128;
-constexpr int kWTmaWarp = kEpiWarp0 + 4;                 // 13
-constexpr int kXTmaWarp = kWTmaWarp + 1;                 // 14
-constexpr int kXsThreads = (kXTmaWarp + 1) * 32;         // 480
-constexpr int kXAtom = kXsTileM * 128;                   // 16 KB
+constexpr int kEpiWarps = 8;                             // two per TMEM lane quadrant
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kEpiCols = kXsTileM / 2;                   // columns per epilogue warp
+constexpr int kWTmaWarp = kEpiWarp0 + kEpiWarps;         // 17
+constexpr int kXTmaWarp = kWTmaWarp + 1;                 // 18
+constexpr int kXsThreads = (kXTmaWarp + 1) * 32;         // 608
+constexpr int kXAtom = kXsTileM * 128;                   // 24 KB: 192 rows x 64 K
 constexpr int kAStages = 4;                              // A stages in TMEM, 32 columns each
-constexpr int kRaw = 6;                                  // packed-code ring depth (steps)
-constexpr int kRawSlot = 8 * 1024;                       // 128 rows x 64 B (q8) or 32 B (q4)
-constexpr int kScaleSlot = 8 * 1024;                     // 128 rows x 16 (scale, min) words
-constexpr uint32_t kAccCols = 2 * kXsTileM;              // 2 accumulators x 128 columns
+constexpr int kRaw = 4;                                  // packed-code ring depth (steps)
+constexpr uint32_t kAccCols = 2 * kXsTileM;              // 2 accumulators x 192 columns
 constexpr uint32_t kAStageCols = kAtomK / 2;             // 64 16-bit values per lane
 constexpr uint32_t kXsTmemCols = 512;                    // accumulators + A stages, pow2
 constexpr unsigned kStatusTimeout = 5u;
 
 static_assert(kAccCols + kAStages * kAStageCols <= kXsTmemCols, "TMEM budget");
+static_assert(kEpiCols % 32 == 0, "epilogue reads 32 columns at a time");
+
+// Packed codes of one K step (128 rows x 32 B for q4, x 64 B for q8), and the
+// (scale, min) words of a weight tile (q4: 128 rows x 16 words, one box that
+// covers K = 512 and is zero-filled past the tensor for shorter K).
+constexpr int kScaleWords = 16;
+__host__ __device__ constexpr int raw_slot_bytes(int fmt) { return kTileRows * (fmt == 4 ? 32 : 64); }
+__host__ __device__ constexpr int scale_slot_bytes(int fmt, int K) {
+    return fmt == 4 ? kTileRows * kScaleWords * 4 + 0 * K : 0;
+}
 
 struct XsLayout {
     int x_off, raw_off, sc_off, bar_off, total;
 };
 
-__host__ __device__ inline XsLayout xs_layout(int K) {
+__host__ __device__ inline XsLayout xs_layout(int fmt, int K) {
     XsLayout L;
     L.x_off = 0;
     L.raw_off = (K / kAtomK) * kXAtom;
-    L.sc_off = L.raw_off + kRaw * kRawSlot;
-    L.bar_off = L.sc_off + 2 * kScaleSlot;
+    L.sc_off = L.raw_off + kRaw * raw_slot_bytes(fmt);
+    L.bar_off = L.sc_off + 2 * scale_slot_bytes(fmt, K);
     // raw_full/empty[kRaw], sc_full/empty[2], a_full/empty[kAStages],
     // x_full, x_empty, acc_full/empty[2], + TMEM address slot
     L.total = L.bar_off + (2 * kRaw + 4 + 2 * kAStages + 2 + 4) * 8 + 16;
@@ -113,7 +129,9 @@ __global__ void __launch_bounds__(kXsThreads, 1)
     const uint32_t raw_base = smem_addr(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;
     uint8_t *smem = smem_raw + (base - raw_base);
-    const XsLayout L = xs_layout(K);
+    const XsLayout L = xs_layout(FMT, K);
+    constexpr int kRawSlot = raw_slot_bytes(FMT);
+    const int kScaleSlot = scale_slot_bytes(FMT, K);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bar_off);
     uint64_t *raw_full = bars;
     uint64_t *raw_empty = raw_full + kRaw;
@@ -133,12 +151,12 @@ __global__ void __launch_bounds__(kXsThreads, 1)
     const int first = static_cast<int>((static_cast<long long>(blockIdx.x) * n_items) / G);
     const int last = static_cast<int>((static_cast<long long>(blockIdx.x + 1) * n_items) / G);
     const uint32_t raw_bytes = kTileRows * (FMT == 4 ? 32 : 64);
-    const uint32_t sc_bytes = kTileRows * (K / 8);
+    const uint32_t sc_bytes = kTileRows * kScaleWords * 4;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kRaw; ++i) {
             mbar_init(&raw_full[i], 1);
-            mbar_init(&raw_empty[i], kDeqThreads);
+            mbar_init(&raw_empty[i], kDeqGroups * kDeqThreads);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sc_full[b], 1);
@@ -147,7 +165,7 @@ __global__ void __launch_bounds__(kXsThreads, 1)
             mbar_init(&acc_empty[b], kEpiThreads);
         }
         for (int s = 0; s < kAStages; ++s) {
-            mbar_init(&a_full[s], kDeqThreads);
+            mbar_init(&a_full[s], kDeqGroups * kDeqThreads);
             mbar_init(&a_empty[s], 1);
         }
         mbar_init(x_full, 1);
@@ -220,27 +238,38 @@ __global__ void __launch_bounds__(kXsThreads, 1)
         __syncwarp();
     } else if (warp < kDeqWarps) {
         // ============================================================ dequantizers
-        const int g = warp >> 2;                     // group: K steps ks = g, g + 2, ...
+        const int h = warp >> 2;                     // K half [32h, 32h + 32) of every step
         const int r = threadIdx.x & (kDeqThreads - 1);
-        // this warp's 32 TMEM lanes (warp % 4 selects the lane quadrant)
-        const uint32_t ta = tmem + kAccCols + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        // this warp's 32 TMEM lanes (warp % 4 selects the lane quadrant) and
+        // its 16 columns of each 32-column A stage
+        const uint32_t ta = tmem + kAccCols + (static_cast<uint32_t>((warp & 3) * 32) << 16) +
+                            static_cast<uint32_t>(16 * h);
         for (ItemCursor it(first, last, n_o_tiles); it.valid() && ok; it.next()) {
             const int n_local = it.item - first;
             const int b = n_local & 1;
-            if (FMT == 4 && !mbar_wait(&sc_full[b], static_cast<uint32_t>(n_local / 2) & 1u)) {
-                ok = false;
-                break;
+            uint32_t sw[kScaleWords / 2] = {};
+            if (FMT == 4) {
+                if (!mbar_wait(&sc_full[b], static_cast<uint32_t>(n_local / 2) & 1u)) {
+                    ok = false;
+                    break;
+                }
+                load_scale_words(base + L.sc_off + b * kScaleSlot + r * (kScaleWords * 4), r, h,
+                                 sw);
+                // sw depends on every word read, so the reads have completed
+                fence_proxy_async_smem();
+                mbar_arrive(&sc_empty[b]);
             }
-            const uint32_t sc_row = base + L.sc_off + b * kScaleSlot + r * (K / 8);
-            for (int ks = g; ks < nk; ks += kDeqGroups) {
+#pragma unroll
+            for (int ks = 0; ks < kXsMaxK / kAtomK; ++ks) {
+                if (ks >= nk) break;
                 const int j = n_local * nk + ks;
                 const int slot = j % kRaw;
                 if (!mbar_wait(&raw_full[slot], static_cast<uint32_t>(j / kRaw) & 1u)) {
                     ok = false;
                     break;
                 }
-                const RowRaw R = load_row_raw<FMT>(base + L.raw_off + slot * kRawSlot, r,
-                                                   sc_row + ks * 8);
+                const HalfRaw R =
+                    load_half_raw<FMT>(base + L.raw_off + slot * kRawSlot, r, h, sw[ks]);
                 const int s = j % kAStages;
                 if (j >= kAStages &&
                     !mbar_wait(&a_empty[s], static_cast<uint32_t>((j / kAStages) - 1) & 1u)) {
@@ -248,7 +277,7 @@ __global__ void __launch_bounds__(kXsThreads, 1)
                     break;
                 }
                 tc_fence_after_sync();
-                tmem_row_op<FMT, OP>(R, ta + static_cast<uint32_t>(s) * kAStageCols);
+                tmem_half_op<FMT, OP>(R, ta + static_cast<uint32_t>(s) * kAStageCols);
                 tmem_st_wait();
                 tc_fence_before_sync();
                 mbar_arrive(&a_full[s]);
@@ -259,14 +288,22 @@ __global__ void __launch_bounds__(kXsThreads, 1)
                 mbar_arrive(&raw_empty[slot]);
             }
             if (!ok) break;
-            if (FMT == 4) mbar_arrive(&sc_empty[b]);
         }
     } else if (warp == kMmaWarp) {
         // ============================================================ MMA issuer
         if (lane == 0) {
             const uint32_t idesc =
                 idesc_f16kind_f32acc(kTileRows, kXsTileM, static_cast<uint32_t>(OP));
-            int cur_m = -1, x_loads = 0, j = 0;
+            static_assert(kXsTileM % 16 == 0 && kXsTileM <= 256, "MMA N for M = 128");
+            static_assert((kAStages & (kAStages - 1)) == 0, "A ring indexed with a mask");
+            // The tensor pipe queues about one MMA ahead of the issuing thread,
+            // so the bookkeeping between two K steps (commit, wait, fence) must
+            // overlap queued MMAs: the wait for step j + 1's A stage sits
+            // between the second and third MMA of step j.
+            constexpr uint64_t kXAtomDesc = kXAtom >> 4;   // descriptor step per X atom
+            const uint64_t bdesc0 = sw128_kmajor_desc(base + L.x_off);
+            int cur_m = -1, x_loads = 0;
+            uint32_t j = 0;                                 // K steps issued so far
             for (ItemCursor it(first, last, n_o_tiles); it.valid() && ok; it.next()) {
                 const int n_local = it.item - first;
                 const int b = n_local & 1;
@@ -284,22 +321,27 @@ __global__ void __launch_bounds__(kXsThreads, 1)
                     ok = false;
                     break;
                 }
+                if (!mbar_wait(&a_full[j & (kAStages - 1)], (j / kAStages) & 1u)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after_sync();
                 const uint32_t d = tmem + static_cast<uint32_t>(b * kXsTileM);
-                for (int ks = 0; ks < nk; ++ks, ++j) {
-                    const int s = j % kAStages;
-                    if (!mbar_wait(&a_full[s], static_cast<uint32_t>(j / kAStages) & 1u)) {
+                uint64_t bdesc = bdesc0;
+                for (int ks = 0; ks < nk; ++ks, ++j, bdesc += kXAtomDesc) {
+                    const uint32_t s = j & (kAStages - 1);
+                    const uint32_t at = tmem + kAccCols + s * kAStageCols;
+                    tc_mma_f16kind_ts(d, at, bdesc, idesc, ks > 0 ? 1u : 0u);
+                    tc_mma_f16kind_ts(d, at + 8, bdesc + 2, idesc, 1u);
+                    const uint32_t jn = j + 1;
+                    if (ks + 1 < nk &&
+                        !mbar_wait(&a_full[jn & (kAStages - 1)], (jn / kAStages) & 1u))
                         ok = false;
-                        break;
-                    }
-                    tc_fence_after_sync();
-                    const uint32_t at = tmem + kAccCols + static_cast<uint32_t>(s) * kAStageCols;
-                    const uint64_t bdesc = sw128_kmajor_desc(base + L.x_off + ks * kXAtom);
-#pragma unroll
-                    for (int kk = 0; kk < kAtomK / 16; ++kk)
-                        tc_mma_f16kind_ts(d, at + 8 * kk, bdesc + 2 * kk, idesc,
-                                          (ks > 0 || kk > 0) ? 1u : 0u);
+                    tc_mma_f16kind_ts(d, at + 16, bdesc + 4, idesc, 1u);
+                    tc_mma_f16kind_ts(d, at + 24, bdesc + 6, idesc, 1u);
                     tc_commit(&a_empty[s]);
+                    if (!ok) break;
+                    tc_fence_after_sync();
                 }
                 if (!ok) break;
                 tc_commit(&acc_full[b]);
@@ -312,6 +354,7 @@ __global__ void __launch_bounds__(kXsThreads, 1)
     } else {
         // ============================================================ epilogue
         const int q = warp & 3;                       // TMEM lane quadrant of this warp
+        const int c0 = ((warp - kEpiWarp0) >> 2) * kEpiCols;   // its half of the columns
         const int row = q * 32 + lane;
         const uint32_t tq = tmem + (static_cast<uint32_t>(q * 32) << 16);
         for (ItemCursor it(first, last, n_o_tiles); it.valid() && ok; it.next()) {
@@ -328,7 +371,7 @@ __global__ void __launch_bounds__(kXsThreads, 1)
             const int mlim = min(kXsTileM, M - m0);
             float *yo = Y + static_cast<size_t>(m0) * N + o;
             const size_t rs = static_cast<size_t>(N);
-            for (int c = 0; c < kXsTileM; c += 32) {
+            for (int c = c0; c < c0 + kEpiCols; c += 32) {
                 uint32_t v[32];
                 tmem_ld_x32(tq + static_cast<uint32_t>(b * kXsTileM + c), v);
                 tmem_ld_wait();
@@ -374,12 +417,12 @@ cudaError_t launch_xs(const void *Xh, const void *Wq, const void *S, float *Y, i
     CUtensorMap w_map, s_map, x_map;
     bool enc_ok = encode_tma_2d(&x_map, OP == Op16::f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                         : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                                2, Xh, K, M, kAtomK, CU_TENSOR_MAP_SWIZZLE_128B);
+                                2, Xh, K, M, kAtomK, CU_TENSOR_MAP_SWIZZLE_128B, kXsTileM);
     if (FMT == 4) {
         enc_ok = enc_ok &&
                  encode_tma_2d(&w_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Wq, K / 2, N, 32,
                                CU_TENSOR_MAP_SWIZZLE_NONE) &&
-                 encode_tma_2d(&s_map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, S, K / 32, N, K / 32,
+                 encode_tma_2d(&s_map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, S, K / 32, N, kScaleWords,
                                CU_TENSOR_MAP_SWIZZLE_NONE);
     } else {
         enc_ok = enc_ok && encode_tma_2d(&w_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Wq, K, N, 64,
@@ -395,7 +438,7 @@ cudaError_t launch_xs(const void *Xh, const void *Wq, const void *S, float *Y, i
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(std::min(items, sms), 1, 1);
     cfg.blockDim = dim3(kXsThreads, 1, 1);
-    cfg.dynamicSmemBytes = xs_layout(K).total + 1024;
+    cfg.dynamicSmemBytes = xs_layout(FMT, K).total + 1024;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -410,13 +453,11 @@ cudaError_t launch_xs(const void *Xh, const void *Wq, const void *S, float *Y, i
 
 // Shapes the activation-resident kernel takes: K a multiple of 128 up to 512
 // (the (scale, min) rows are TMA boxes, whose global stride K/8 bytes must be
-// a multiple of 16), at least two activation blocks, and enough work items
-// to give most SMs one.
+// a multiple of 16; 192 rows of K = 512 fill the shared memory) and more than
+// 128 activation rows (fewer go to the weight-stationary kernel).
 bool xs_supported(int M, int N, int K) {
-    if (K % 128 != 0 || K > kXsMaxK) return false;
-    const long items = static_cast<long>((N + kTileRows - 1) / kTileRows) *
-                       ((M + kXsTileM - 1) / kXsTileM);
-    return M >= 2 * kXsTileM && items >= 96;
+    (void)N;
+    return K % 128 == 0 && K <= kXsMaxK && M > kTileRows;
 }
 
 cudaError_t launch_xs_q4(const void *Xh, const uint8_t *Wq, const uint16_t *SM, float *Y, int M,

@@ -97,7 +97,9 @@ def test_kernel_plan():
     assert rtq.plan(4, 4096, 4096, 512) == "tc_x_resident"
     assert rtq.plan(4, 65536, 2048, 512) == "tc_x_resident"
     assert rtq.plan(8, 4096, 512, 2048) == "tc_w_streamed"     # K > 512 does not fit resident
-    assert rtq.plan(4, 200, 512, 512) == "tc_w_streamed"       # too few tiles to keep X resident
+    assert rtq.plan(4, 200, 512, 512) == "tc_x_resident"       # one full block and a tail
+    assert rtq.plan(4, 129, 512, 512) == "tc_x_resident"
+    assert rtq.plan(4, 200, 512, 768) == "tc_w_streamed"       # K above the resident limit
     assert rtq.plan(4, 300, 512, 192) == "tc_w_stationary"     # q4 TMA needs K % 128
     assert rtq.plan(8, 4096, 512, 2048, "tc_bf16") == "tc_w_streamed"
     assert rtq.plan(4, 4096, 4096, 512, "simt") == "simt"
