@@ -202,6 +202,23 @@ def build_host(workload, rank, use_oracle_quantizer=False):
     return cfg, nblocks, M, projs, blocks
 
 
+def reduce_max(x, world, device):
+    """Largest value of x over all ranks (x itself at world size 1): every
+    rank's timed region is the job's when the ranks run in lockstep."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world, flops_per_rank_step, ms_per_step):
+    """Whole-job TFLOP/s: every rank processes its own batch each step."""
+    return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
+
+
 def step_flops(M, nblocks, projs):
     return nblocks * sum(proj_flops(p, M) for p in projs)
 
@@ -329,11 +346,7 @@ def run_gpu(args, rank, world, local_rank):
             dist.barrier(device_ids=[local_rank])
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, world, dev)
 
     # ---- warm-up
     with torch.cuda.stream(stream):
@@ -389,7 +402,7 @@ def run_gpu(args, rank, world, local_rank):
         raise RuntimeError("device status word reports a timed-out wait")
 
     flops = step_flops(M, nblocks, projs)
-    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    value = job_value(world, flops, ms_per_step)
     wbytes = step_weight_bytes(nblocks, projs)
 
     # ---- roofline of the dominant kernel
@@ -449,7 +462,7 @@ def run_gpu(args, rank, world, local_rank):
         torch.cuda.synchronize(dev)
         barrier()
         ms_e2e = max_over_ranks(f0.elapsed_time(f1)) / n_e2e
-        e2e = {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": job_value(world, flops, ms_e2e), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
                "steps": n_e2e}
 
