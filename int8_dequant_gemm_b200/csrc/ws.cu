@@ -16,8 +16,9 @@
 //      layout.
 // The A and B rings are separate: TMEM holds two 192-column accumulators and
 // four 32-column A stages (512 columns); shared memory holds six B stages.
-// Roles (19 warps): warps 0-7 dequantizers (thread (r, h) converts half h of
-// every K step of weight row r, as in xs.cu), warp 8 MMA issuer, warps 9-16
+// Roles (20 warps): warps 0-7 dequantizers (thread (r, h) converts half h of
+// every K step of weight row r, as in xs.cu), warp 8 MMA issuer (fed by the
+// waiter, warp 19, through a named barrier, as in xs.cu), warps 9-16
 // epilogue (two per TMEM lane quadrant, double-buffered accumulators), warp 17
 // weight TMA (codes and, for q4, (scale, min) blocks of up to 16 words per
 // row), warp 18 activation TMA.
@@ -43,7 +44,9 @@ constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kEpiCols = kWsTileM / 2;
 constexpr int kWTmaWarp = kEpiWarp0 + kEpiWarps;         // 17
 constexpr int kXTmaWarp = kWTmaWarp + 1;                 // 18
-constexpr int kWsThreads = (kXTmaWarp + 1) * 32;         // 608
+constexpr int kWaitWarp = kXTmaWarp + 1;                 // 19
+constexpr int kWsThreads = (kWaitWarp + 1) * 32;         // 640
+constexpr uint32_t kMmaBar = 1;                          // named barrier: waiter <-> MMA warp
 constexpr int kStages = 6;                               // B stages (shared memory)
 constexpr int kStageBytes = kWsTileM * 128;              // 24 KB: 192 rows x 64 K
 constexpr int kAStages = 4;                              // A stages (TMEM)
@@ -99,6 +102,8 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     uint64_t *acc_full = sc_empty + 2;
     uint64_t *acc_empty = acc_full + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    // waiter -> MMA warp abort flags, one per K-step parity
+    volatile uint32_t *mma_abort = tmem_slot + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nk = K / kAtomK;
@@ -240,50 +245,64 @@ __global__ void __launch_bounds__(kWsThreads, 1)
                 }
             }
         }
+    } else if (warp == kWaitWarp) {
+        // ============================================================ MMA waiter
+        // As in xs.cu: the waits of the MMA issuer, handed over per K step
+        // through named barrier kMmaBar, so that the issuing thread never
+        // waits on an mbarrier after a tcgen05.commit.
+        int j = 0, tile_local = 0;
+        for (int t = blockIdx.x; t < n_tiles && ok; t += G, ++tile_local) {
+            const int b = tile_local & 1;
+            bool good = true;
+            if (lane == 0 && tile_local >= 2)
+                good = mbar_wait(&acc_empty[b], static_cast<uint32_t>((tile_local / 2) - 1) & 1u);
+            for (int ks = 0; ks < nk; ++ks, ++j) {
+                if (lane == 0) {
+                    if (good)
+                        good = mbar_wait(&a_full[j % kAStages],
+                                         static_cast<uint32_t>(j / kAStages) & 1u) &&
+                               mbar_wait(&b_full[j % kStages], static_cast<uint32_t>(j / kStages) & 1u);
+                    mma_abort[j & 1] = good ? 0u : 1u;
+                }
+                named_bar_sync(kMmaBar, 64);
+                if (__shfl_sync(0xffffffffu, good ? 1 : 0, 0) == 0) {
+                    ok = false;
+                    break;
+                }
+            }
+        }
     } else if (warp == kMmaWarp) {
         // ============================================================ MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc =
-                idesc_f16kind_f32acc(kTileRows, kWsTileM, static_cast<uint32_t>(OP));
-            // As in xs.cu: the wait for step j + 1's stages sits between the
-            // second and third MMA of step j, so that it overlaps queued MMAs.
-            constexpr uint64_t kStageDesc = kStageBytes >> 4;   // descriptor step per B stage
-            const uint64_t bdesc0 = sw128_kmajor_desc(base + L.st_off);
-            auto ready = [&](int jj) {
-                return mbar_wait(&a_full[jj % kAStages], static_cast<uint32_t>(jj / kAStages) & 1u) &&
-                       mbar_wait(&b_full[jj % kStages], static_cast<uint32_t>(jj / kStages) & 1u);
-            };
-            int j = 0, tile_local = 0;
-            for (int t = blockIdx.x; t < n_tiles && ok; t += G, ++tile_local) {
-                const int b = tile_local & 1;
-                if (tile_local >= 2 &&
-                    !mbar_wait(&acc_empty[b], static_cast<uint32_t>((tile_local / 2) - 1) & 1u)) {
-                    ok = false;
+        const uint32_t idesc =
+            idesc_f16kind_f32acc(kTileRows, kWsTileM, static_cast<uint32_t>(OP));
+        constexpr uint64_t kStageDesc = kStageBytes >> 4;   // descriptor step per B stage
+        const uint64_t bdesc0 = sw128_kmajor_desc(base + L.st_off);
+        int j = 0, tile_local = 0;
+        bool abort = false;
+        for (int t = blockIdx.x; t < n_tiles && !abort; t += G, ++tile_local) {
+            const int b = tile_local & 1;
+            const uint32_t d = tmem + static_cast<uint32_t>(b * kWsTileM);
+            for (int ks = 0; ks < nk; ++ks, ++j) {
+                named_bar_sync(kMmaBar, 64);           // the waiter saw step j's stages full
+                if (mma_abort[j & 1]) {
+                    abort = true;
                     break;
                 }
-                if (!ready(j)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after_sync();
-                const uint32_t d = tmem + static_cast<uint32_t>(b * kWsTileM);
-                for (int ks = 0; ks < nk; ++ks, ++j) {
+                if (lane == 0) {
+                    tc_fence_after_sync();
                     const int s = j % kAStages, sb = j % kStages;
                     const uint32_t at = tmem + kAccCols + static_cast<uint32_t>(s) * kAStageCols;
                     const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(sb) * kStageDesc;
-                    tc_mma_f16kind_ts(d, at, bdesc, idesc, ks > 0 ? 1u : 0u);
-                    tc_mma_f16kind_ts(d, at + 8, bdesc + 2, idesc, 1u);
-                    if (ks + 1 < nk && !ready(j + 1)) ok = false;
-                    tc_mma_f16kind_ts(d, at + 16, bdesc + 4, idesc, 1u);
-                    tc_mma_f16kind_ts(d, at + 24, bdesc + 6, idesc, 1u);
+#pragma unroll
+                    for (int kk = 0; kk < kAtomK / 16; ++kk)
+                        tc_mma_f16kind_ts(d, at + 8 * kk, bdesc + 2 * kk, idesc,
+                                          (ks > 0 || kk > 0) ? 1u : 0u);
                     tc_commit(&a_empty[s]);
                     tc_commit(&b_empty[sb]);
-                    if (!ok) break;
-                    tc_fence_after_sync();
                 }
-                if (!ok) break;
-                tc_commit(&acc_full[b]);
             }
+            if (abort) break;
+            if (lane == 0) tc_commit(&acc_full[b]);
         }
         __syncwarp();
     } else {

@@ -16,7 +16,7 @@
 // order, split into one contiguous run per CTA (one CTA per SM), so a CTA
 // changes activation block rarely.
 //
-// Roles (19 warps):
+// Roles (20 warps):
 //   warp 18     activation TMA (one thread): on every change of activation
 //               block, once the MMAs on the previous block have completed,
 //               K/64 boxes into the resident tile, one transaction barrier.
@@ -33,7 +33,10 @@
 //               the TMA traffic.
 //   warp 8      MMA issuer (one thread): per weight tile, K/64 stages x 4
 //               tcgen05.mma (K = 16, A from TMEM, B from shared memory) into
-//               one of two TMEM accumulators.
+//               one of two TMEM accumulators.  It waits on no mbarrier.
+//   warp 19     MMA waiter: waits for each stage (and the activation block
+//               and accumulator) and hands the step to the issuer through a
+//               named barrier.
 //   warps 9-16  epilogue, two warps per TMEM lane quadrant: TMEM ->
 //               registers (q8 row scale) -> fp32 Y with 128-byte coalesced
 //               rows, overlapping the next tile's MMAs.
@@ -64,7 +67,9 @@ constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kEpiCols = kXsTileM / 2;                   // columns per epilogue warp
 constexpr int kWTmaWarp = kEpiWarp0 + kEpiWarps;         // 17
 constexpr int kXTmaWarp = kWTmaWarp + 1;                 // 18
-constexpr int kXsThreads = (kXTmaWarp + 1) * 32;         // 608
+constexpr int kWaitWarp = kXTmaWarp + 1;                 // 19
+constexpr int kXsThreads = (kWaitWarp + 1) * 32;         // 640
+constexpr uint32_t kMmaBar = 1;                          // named barrier: waiter <-> MMA warp
 constexpr int kXAtom = kXsTileM * 128;                   // 24 KB: 192 rows x 64 K
 constexpr int kAStages = 4;                              // A stages in TMEM, 32 columns each
 constexpr int kRaw = 4;                                  // packed-code ring depth (steps)
@@ -144,6 +149,8 @@ __global__ void __launch_bounds__(kXsThreads, 1)
     uint64_t *acc_full = x_empty + 1;
     uint64_t *acc_empty = acc_full + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    // waiter -> MMA warp abort flags, one per K-step parity
+    volatile uint32_t *mma_abort = tmem_slot + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nk = K / kAtomK;
@@ -289,61 +296,73 @@ __global__ void __launch_bounds__(kXsThreads, 1)
             }
             if (!ok) break;
         }
+    } else if (warp == kWaitWarp) {
+        // ============================================================ MMA waiter
+        // Every mbarrier wait the MMA issuer needs happens here; each K step
+        // is handed over through named barrier kMmaBar.  A thread that waits
+        // on an mbarrier after issuing tcgen05.commit stalls until its
+        // queued MMAs drain, so the issuing thread itself never waits.
+        int cur_m = -1, x_loads = 0;
+        uint32_t j = 0;
+        for (ItemCursor it(first, last, n_o_tiles); it.valid() && ok; it.next()) {
+            const int n_local = it.item - first;
+            const int b = n_local & 1;
+            bool good = true;
+            if (lane == 0) {
+                if (it.m_tile != cur_m) good = mbar_wait(x_full, static_cast<uint32_t>(x_loads) & 1u);
+                // accumulator b must have been drained by the epilogue
+                if (good && n_local >= 2)
+                    good = mbar_wait(&acc_empty[b], static_cast<uint32_t>((n_local / 2) - 1) & 1u);
+            }
+            if (it.m_tile != cur_m) {
+                cur_m = it.m_tile;
+                ++x_loads;
+            }
+            for (int ks = 0; ks < nk; ++ks, ++j) {
+                if (lane == 0) {
+                    if (good) good = mbar_wait(&a_full[j & (kAStages - 1)], (j / kAStages) & 1u);
+                    mma_abort[j & 1] = good ? 0u : 1u;
+                }
+                named_bar_sync(kMmaBar, 64);
+                if (__shfl_sync(0xffffffffu, good ? 1 : 0, 0) == 0) {
+                    ok = false;
+                    break;
+                }
+            }
+        }
     } else if (warp == kMmaWarp) {
         // ============================================================ MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc =
-                idesc_f16kind_f32acc(kTileRows, kXsTileM, static_cast<uint32_t>(OP));
-            static_assert(kXsTileM % 16 == 0 && kXsTileM <= 256, "MMA N for M = 128");
-            static_assert((kAStages & (kAStages - 1)) == 0, "A ring indexed with a mask");
-            // The tensor pipe queues about one MMA ahead of the issuing thread,
-            // so the bookkeeping between two K steps (commit, wait, fence) must
-            // overlap queued MMAs: the wait for step j + 1's A stage sits
-            // between the second and third MMA of step j.
-            constexpr uint64_t kXAtomDesc = kXAtom >> 4;   // descriptor step per X atom
-            const uint64_t bdesc0 = sw128_kmajor_desc(base + L.x_off);
-            int cur_m = -1, x_loads = 0;
-            uint32_t j = 0;                                 // K steps issued so far
-            for (ItemCursor it(first, last, n_o_tiles); it.valid() && ok; it.next()) {
-                const int n_local = it.item - first;
-                const int b = n_local & 1;
-                if (it.m_tile != cur_m) {
-                    cur_m = it.m_tile;
-                    ++x_loads;
-                    if (!mbar_wait(x_full, static_cast<uint32_t>(x_loads - 1) & 1u)) {
-                        ok = false;
-                        break;
-                    }
-                }
-                // accumulator b must have been drained by the epilogue
-                if (n_local >= 2 &&
-                    !mbar_wait(&acc_empty[b], static_cast<uint32_t>((n_local / 2) - 1) & 1u)) {
-                    ok = false;
+        const uint32_t idesc =
+            idesc_f16kind_f32acc(kTileRows, kXsTileM, static_cast<uint32_t>(OP));
+        static_assert(kXsTileM % 16 == 0 && kXsTileM <= 256, "MMA N for M = 128");
+        static_assert((kAStages & (kAStages - 1)) == 0, "A ring indexed with a mask");
+        constexpr uint64_t kXAtomDesc = kXAtom >> 4;   // descriptor step per X atom
+        const uint64_t bdesc0 = sw128_kmajor_desc(base + L.x_off);
+        uint32_t j = 0;                                 // K steps issued so far
+        bool abort = false;
+        for (ItemCursor it(first, last, n_o_tiles); it.valid() && !abort; it.next()) {
+            const int n_local = it.item - first;
+            const int b = n_local & 1;
+            const uint32_t d = tmem + static_cast<uint32_t>(b * kXsTileM);
+            uint64_t bdesc = bdesc0;
+            for (int ks = 0; ks < nk; ++ks, ++j, bdesc += kXAtomDesc) {
+                named_bar_sync(kMmaBar, 64);           // the waiter saw step j's stage full
+                if (mma_abort[j & 1]) {
+                    abort = true;
                     break;
                 }
-                if (!mbar_wait(&a_full[j & (kAStages - 1)], (j / kAStages) & 1u)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after_sync();
-                const uint32_t d = tmem + static_cast<uint32_t>(b * kXsTileM);
-                uint64_t bdesc = bdesc0;
-                for (int ks = 0; ks < nk; ++ks, ++j, bdesc += kXAtomDesc) {
-                    const uint32_t s = j & (kAStages - 1);
-                    const uint32_t at = tmem + kAccCols + s * kAStageCols;
-                    tc_mma_f16kind_ts(d, at, bdesc, idesc, ks > 0 ? 1u : 0u);
-                    tc_mma_f16kind_ts(d, at + 8, bdesc + 2, idesc, 1u);
-                    const uint32_t jn = j + 1;
-                    if (ks + 1 < nk &&
-                        !mbar_wait(&a_full[jn & (kAStages - 1)], (jn / kAStages) & 1u))
-                        ok = false;
-                    tc_mma_f16kind_ts(d, at + 16, bdesc + 4, idesc, 1u);
-                    tc_mma_f16kind_ts(d, at + 24, bdesc + 6, idesc, 1u);
-                    tc_commit(&a_empty[s]);
-                    if (!ok) break;
+                if (lane == 0) {
                     tc_fence_after_sync();
+                    const uint32_t at = tmem + kAccCols + (j & (kAStages - 1)) * kAStageCols;
+#pragma unroll
+                    for (int kk = 0; kk < kAtomK / 16; ++kk)
+                        tc_mma_f16kind_ts(d, at + 8 * kk, bdesc + 2 * kk, idesc,
+                                          (ks > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(&a_empty[j & (kAStages - 1)]);
                 }
-                if (!ok) break;
+            }
+            if (abort) break;
+            if (lane == 0) {
                 tc_commit(&acc_full[b]);
                 // last item of this activation block with another block to
                 // follow: release the X tile once these MMAs have completed

@@ -214,7 +214,8 @@ def test_tc_parity_q8(rtq_lib, M, N, K, path):
 # shapes that the activation-resident kernel takes: ragged M and N, K from 64 to
 # 512, a CTA run that crosses activation blocks
 XS_SHAPES = [(2048, 1024, 512), (2000, 1000, 512), (1500, 2100, 256), (4096, 512, 512),
-             (2048, 2048, 128), (300, 6000, 128), (150, 640, 512), (200, 384, 256)]
+             (2048, 2048, 128), (300, 6000, 128), (150, 640, 512), (200, 384, 256),
+             (500, 1002, 256)]
 
 
 @pytest.mark.parametrize("path", ["tc", "tc_bf16"])
@@ -237,7 +238,7 @@ def test_x_resident_parity_q8(rtq_lib, M, N, K, path):
 # limit; ragged M and N; q4 chunks of (scale, min) words that end inside a
 # chunk (K = 640)
 WS_SHAPES = [(2048, 512, 2048), (300, 640, 1024), (200, 512, 768), (1000, 700, 2048),
-             (129, 256, 640)]
+             (129, 256, 640), (300, 1002, 768)]
 
 
 @pytest.mark.parametrize("path", ["tc", "tc_bf16"])
