@@ -58,6 +58,9 @@ WORKLOADS = {
     "w13_m4096": (4, 1, 4096, ("w13",)),
     "w2_m4096": (4, 1, 4096, ("w2",)),
     "qkvg_m4096": (4, 1, 4096, ("qkvg",)),
+    # outputs larger than L2, for full profiler captures of one launch
+    "w13_m16384": (4, 1, 16384, ("w13",)),
+    "w2_m16384": (4, 1, 16384, ("w2",)),
 }
 
 
