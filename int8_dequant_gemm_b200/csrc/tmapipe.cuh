@@ -120,6 +120,30 @@ __device__ __forceinline__ HalfRaw load_half_raw(uint32_t slot, int r, int h, ui
     return R;
 }
 
+// The same half-row read from a slot that holds two K steps per row, as one
+// TMA box in a swizzled layout: q4 rows of 64 bytes (SWIZZLE_64B: 16-byte
+// chunk c of row r sits at chunk c ^ ((r >> 1) & 3)), q8 rows of 128 bytes
+// (SWIZZLE_128B: chunk c at c ^ (r & 7)).  u selects the step within the
+// pair.  A TMA box costs about 3 cycles per row whatever its width, so two
+// steps per box halve the weight stream's TMA time per step; the swizzle
+// keeps 8 consecutive rows on 8 different bank groups.
+template <int FMT>
+__device__ __forceinline__ HalfRaw load_half_raw2(uint32_t slot, int r, int h, int u, uint32_t smw) {
+    HalfRaw R;
+    if (FMT == 4) {
+        const int c = (2 * u + h) ^ ((r >> 1) & 3);
+        R.p0 = lds_v4(slot + r * 64 + c * 16);
+        R.p1 = make_uint4(0, 0, 0, 0);
+        R.smw = smw;
+    } else {
+        const int c0 = 4 * u + 2 * h;
+        R.p0 = lds_v4(slot + r * 128 + ((c0 ^ (r & 7)) * 16));
+        R.p1 = lds_v4(slot + r * 128 + (((c0 + 1) ^ (r & 7)) * 16));
+        R.smw = 0;
+    }
+    return R;
+}
+
 // 32 weights of a half step -> 16 32-bit operand words (4 chunks) -> TMEM
 // columns [ta, ta + 16) of this thread's lane.  Warp-collective.
 template <int FMT, Op16 OP>

@@ -22,7 +22,9 @@
 //               K/64 boxes into the resident tile, one transaction barrier.
 //   warp 17     weight TMA (one thread): per weight tile the (scale, min)
 //               words of its 128 rows (q4), and per 64-wide K step the
-//               128-row slice of packed codes, into a ring kRaw steps deep.
+//               128-row slice of packed codes, two K steps per TMA box
+//               (a box costs about the same per row at any width up to 256
+//               bytes), into a ring of kRaw such pairs.
 //   warps 0-7   dequantizers: thread (r, h) converts K values [32h, 32h + 32)
 //               of every K step of weight row r (16 or 32 bytes of codes) and
 //               writes them with tcgen05.st into TMEM lane r of the step's A
@@ -57,6 +59,7 @@ namespace {
 // columns.  192 resident rows of K = 512 also just fit in shared memory.
 constexpr int kXsTileM = 192;                 // activation rows per block (MMA N)
 constexpr int kXsMaxK = 512;
+constexpr int kXAtoms = kXsMaxK / 64;                    // 64-wide K atoms of a resident block
 constexpr int kDeqGroups = 2;                            // two K halves per step
 constexpr int kDeqThreads = kTileRows;                   // 128 per half
 constexpr int kDeqWarps = kDeqGroups * 4;                // 8
@@ -72,7 +75,7 @@ constexpr int kXsThreads = (kWaitWarp + 1) * 32;         // 640
 constexpr uint32_t kMmaBar = 1;                          // named barrier: waiter <-> MMA warp
 constexpr int kXAtom = kXsTileM * 128;                   // 24 KB: 192 rows x 64 K
 constexpr int kAStages = 4;                              // A stages in TMEM, 32 columns each
-constexpr int kRaw = 4;                                  // packed-code ring depth (steps)
+constexpr int kRaw = 2;                                  // packed-code ring depth (step pairs)
 constexpr uint32_t kAccCols = 2 * kXsTileM;              // 2 accumulators x 192 columns
 constexpr uint32_t kAStageCols = kAtomK / 2;             // 64 16-bit values per lane
 constexpr uint32_t kXsTmemCols = 512;                    // accumulators + A stages, pow2
@@ -81,11 +84,11 @@ constexpr unsigned kStatusTimeout = 5u;
 static_assert(kAccCols + kAStages * kAStageCols <= kXsTmemCols, "TMEM budget");
 static_assert(kEpiCols % 32 == 0, "epilogue reads 32 columns at a time");
 
-// Packed codes of one K step (128 rows x 32 B for q4, x 64 B for q8), and the
+// Packed codes of two K steps (128 rows x 64 B for q4, x 128 B for q8), and the
 // (scale, min) words of a weight tile (q4: 128 rows x 16 words, one box that
 // covers K = 512 and is zero-filled past the tensor for shorter K).
 constexpr int kScaleWords = 16;
-__host__ __device__ constexpr int raw_slot_bytes(int fmt) { return kTileRows * (fmt == 4 ? 32 : 64); }
+__host__ __device__ constexpr int raw_slot_bytes(int fmt) { return kTileRows * (fmt == 4 ? 64 : 128); }
 __host__ __device__ constexpr int scale_slot_bytes(int fmt, int K) {
     return fmt == 4 ? kTileRows * kScaleWords * 4 + 0 * K : 0;
 }
@@ -101,8 +104,8 @@ __host__ __device__ inline XsLayout xs_layout(int fmt, int K) {
     L.sc_off = L.raw_off + kRaw * raw_slot_bytes(fmt);
     L.bar_off = L.sc_off + 2 * scale_slot_bytes(fmt, K);
     // raw_full/empty[kRaw], sc_full/empty[2], a_full/empty[kAStages],
-    // x_full, x_empty, acc_full/empty[2], + TMEM address slot
-    L.total = L.bar_off + (2 * kRaw + 4 + 2 * kAStages + 2 + 4) * 8 + 16;
+    // x_full[kXAtoms], x_empty, acc_full/empty[2], + TMEM address slot
+    L.total = L.bar_off + (2 * kRaw + 4 + 2 * kAStages + kXAtoms + 1 + 4) * 8 + 16;
     return L;
 }
 
@@ -144,8 +147,8 @@ __global__ void __launch_bounds__(kXsThreads, 1)
     uint64_t *sc_empty = sc_full + 2;
     uint64_t *a_full = sc_empty + 2;
     uint64_t *a_empty = a_full + kAStages;
-    uint64_t *x_full = a_empty + kAStages;
-    uint64_t *x_empty = x_full + 1;
+    uint64_t *x_full = a_empty + kAStages;                // one per K atom
+    uint64_t *x_empty = x_full + kXAtoms;
     uint64_t *acc_full = x_empty + 1;
     uint64_t *acc_empty = acc_full + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
@@ -157,7 +160,7 @@ __global__ void __launch_bounds__(kXsThreads, 1)
     const int G = gridDim.x;
     const int first = static_cast<int>((static_cast<long long>(blockIdx.x) * n_items) / G);
     const int last = static_cast<int>((static_cast<long long>(blockIdx.x + 1) * n_items) / G);
-    const uint32_t raw_bytes = kTileRows * (FMT == 4 ? 32 : 64);
+    const uint32_t raw_bytes = raw_slot_bytes(FMT);
     const uint32_t sc_bytes = kTileRows * kScaleWords * 4;
 
     if (threadIdx.x == 0) {
@@ -175,7 +178,7 @@ __global__ void __launch_bounds__(kXsThreads, 1)
             mbar_init(&a_full[s], kDeqGroups * kDeqThreads);
             mbar_init(&a_empty[s], 1);
         }
-        mbar_init(x_full, 1);
+        for (int a = 0; a < kXAtoms; ++a) mbar_init(&x_full[a], 1);
         mbar_init(x_empty, 1);
         fence_mbar_init();
     }
@@ -208,7 +211,7 @@ __global__ void __launch_bounds__(kXsThreads, 1)
                     mbar_expect_tx(&sc_full[b], sc_bytes);
                     tma_load_2d(base + L.sc_off + b * kScaleSlot, &s_map, 0, y0, &sc_full[b]);
                 }
-                for (int ks = 0; ks < nk; ++ks, ++j) {
+                for (int p = 0; p < nk / 2; ++p, ++j) {
                     const int slot = j % kRaw;
                     if (j >= kRaw &&
                         !mbar_wait(&raw_empty[slot], static_cast<uint32_t>((j / kRaw) - 1) & 1u)) {
@@ -217,7 +220,7 @@ __global__ void __launch_bounds__(kXsThreads, 1)
                     }
                     mbar_expect_tx(&raw_full[slot], raw_bytes);
                     tma_load_2d(base + L.raw_off + slot * kRawSlot, &w_map,
-                                ks * (FMT == 4 ? 32 : 64), y0, &raw_full[slot]);
+                                p * (FMT == 4 ? 64 : 128), y0, &raw_full[slot]);
                 }
             }
         }
@@ -235,10 +238,13 @@ __global__ void __launch_bounds__(kXsThreads, 1)
                     ok = false;
                     break;
                 }
-                mbar_expect_tx(x_full, static_cast<uint32_t>(nk * kXAtom));
-                for (int a = 0; a < nk; ++a)
+                // one barrier per atom: the first item's K steps start as
+                // their own atoms land instead of after the whole block
+                for (int a = 0; a < nk; ++a) {
+                    mbar_expect_tx(&x_full[a], static_cast<uint32_t>(kXAtom));
                     tma_load_2d(base + L.x_off + a * kXAtom, &x_map, a * kAtomK,
-                                cur_m * kXsTileM, x_full);
+                                cur_m * kXsTileM, &x_full[a]);
+                }
                 ++x_loads;
             }
         }
@@ -270,13 +276,15 @@ __global__ void __launch_bounds__(kXsThreads, 1)
             for (int ks = 0; ks < kXsMaxK / kAtomK; ++ks) {
                 if (ks >= nk) break;
                 const int j = n_local * nk + ks;
-                const int slot = j % kRaw;
-                if (!mbar_wait(&raw_full[slot], static_cast<uint32_t>(j / kRaw) & 1u)) {
+                const int jp = n_local * (nk / 2) + (ks >> 1);   // step pair of the raw ring
+                const int slot = jp % kRaw;
+                if ((ks & 1) == 0 &&
+                    !mbar_wait(&raw_full[slot], static_cast<uint32_t>(jp / kRaw) & 1u)) {
                     ok = false;
                     break;
                 }
-                const HalfRaw R =
-                    load_half_raw<FMT>(base + L.raw_off + slot * kRawSlot, r, h, sw[ks]);
+                const HalfRaw R = load_half_raw2<FMT>(base + L.raw_off + slot * kRawSlot, r, h,
+                                                      ks & 1, sw[ks]);
                 const int s = j % kAStages;
                 if (j >= kAStages &&
                     !mbar_wait(&a_empty[s], static_cast<uint32_t>((j / kAStages) - 1) & 1u)) {
@@ -288,11 +296,13 @@ __global__ void __launch_bounds__(kXsThreads, 1)
                 tmem_st_wait();
                 tc_fence_before_sync();
                 mbar_arrive(&a_full[s]);
-                // the raw slot goes back only after its contents were consumed
-                // above; the proxy fence orders those generic reads before the
-                // TMA that refills it
-                fence_proxy_async_smem();
-                mbar_arrive(&raw_empty[slot]);
+                // the raw slot goes back after the pair's second step has
+                // consumed its reads; the proxy fence orders those generic
+                // reads before the TMA that refills it
+                if (ks & 1) {
+                    fence_proxy_async_smem();
+                    mbar_arrive(&raw_empty[slot]);
+                }
             }
             if (!ok) break;
         }
@@ -308,18 +318,18 @@ __global__ void __launch_bounds__(kXsThreads, 1)
             const int n_local = it.item - first;
             const int b = n_local & 1;
             bool good = true;
-            if (lane == 0) {
-                if (it.m_tile != cur_m) good = mbar_wait(x_full, static_cast<uint32_t>(x_loads) & 1u);
-                // accumulator b must have been drained by the epilogue
-                if (good && n_local >= 2)
-                    good = mbar_wait(&acc_empty[b], static_cast<uint32_t>((n_local / 2) - 1) & 1u);
-            }
-            if (it.m_tile != cur_m) {
+            const bool fresh = it.m_tile != cur_m;          // first item of a new block
+            if (fresh) {
                 cur_m = it.m_tile;
                 ++x_loads;
             }
+            const uint32_t xpar = static_cast<uint32_t>(x_loads - 1) & 1u;
+            // accumulator b must have been drained by the epilogue
+            if (lane == 0 && n_local >= 2)
+                good = mbar_wait(&acc_empty[b], static_cast<uint32_t>((n_local / 2) - 1) & 1u);
             for (int ks = 0; ks < nk; ++ks, ++j) {
                 if (lane == 0) {
+                    if (good && fresh) good = mbar_wait(&x_full[ks], xpar);
                     if (good) good = mbar_wait(&a_full[j & (kAStages - 1)], (j / kAStages) & 1u);
                     mma_abort[j & 1] = good ? 0u : 1u;
                 }
@@ -439,13 +449,13 @@ cudaError_t launch_xs(const void *Xh, const void *Wq, const void *S, float *Y, i
                                 2, Xh, K, M, kAtomK, CU_TENSOR_MAP_SWIZZLE_128B, kXsTileM);
     if (FMT == 4) {
         enc_ok = enc_ok &&
-                 encode_tma_2d(&w_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Wq, K / 2, N, 32,
-                               CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                 encode_tma_2d(&w_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Wq, K / 2, N, 64,
+                               CU_TENSOR_MAP_SWIZZLE_64B) &&
                  encode_tma_2d(&s_map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, S, K / 32, N, kScaleWords,
                                CU_TENSOR_MAP_SWIZZLE_NONE);
     } else {
-        enc_ok = enc_ok && encode_tma_2d(&w_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Wq, K, N, 64,
-                                         CU_TENSOR_MAP_SWIZZLE_NONE);
+        enc_ok = enc_ok && encode_tma_2d(&w_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Wq, K, N, 128,
+                                         CU_TENSOR_MAP_SWIZZLE_128B);
         s_map = w_map;   // unused by the q8 kernel
     }
     if (!enc_ok) return cudaErrorInvalidValue;
