@@ -27,6 +27,7 @@ weights, rank-seeded activations, no data-path collective) -> weak scaling.
 from __future__ import annotations
 
 import argparse
+import math
 import ctypes
 import hashlib
 import json
@@ -58,6 +59,8 @@ WORKLOADS = {
     "w13_m4096": (4, 1, 4096, ("w13",)),
     "w2_m4096": (4, 1, 4096, ("w2",)),
     "qkvg_m4096": (4, 1, 4096, ("qkvg",)),
+    # small M as an aggregate weight stream (see run_small_m)
+    "rot_m80": (4, 0, 80, ("qkvg", "wo", "w13", "w2")),
     # outputs larger than L2, for full profiler captures of one launch
     "w13_m16384": (4, 1, 16384, ("w13",)),
     "w2_m16384": (4, 1, 16384, ("w2",)),
@@ -277,6 +280,132 @@ def run_reference(args, rank, world):
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------- small-M stream
+def run_small_m(args, rank, world, local_rank):
+    """Small-M projections measured as an aggregate weight stream.
+
+    One M = 80 projection moves well under a megabyte of weights, less than a
+    launch's latency worth, so the small-M rate is measured over many: the 12
+    blocks' quantized weights are copied into distinct device buffers until the
+    copies total about 4x L2, and one step runs every copy's block projection
+    set (qkvg, wo, w13, w2) at M = 80 through rt_qblock_project.  X and Y are
+    one buffer per projection shared by all copies (L2-resident, as the
+    activations of a real forward pass are).  The step is captured once as a
+    CUDA graph and replayed.  value = quantized weight bytes per step / time.
+    """
+    import torch
+    import torch.distributed as dist
+
+    import int8_dequant_gemm_b200 as rtq
+
+    rtq.lib()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.Stream(device=dev)
+    sptr = ctypes.c_void_p(stream.cuda_stream)
+    L = rtq.lib()
+    cfg, nblocks, M, projs = WORKLOADS[args.workload]
+    _, _, _, _, blocks = build_host("blocks12_m4096", rank)   # the 12 blocks' quantized weights
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    per_block = sum(weight_bytes(p) for p in projs)
+    copies = max(len(blocks), int(math.ceil(4 * l2 / per_block)))
+
+    def d(a):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    xs = {p: d(wl.activations(M, proj_dims(p)[2], wl.seed_for(cfg, 0, wl.BLOCK_PROJECTIONS[p]["x"])
+                                  + 100_000 * rank)) for p in projs}
+    ys = {p: torch.empty((M, proj_dims(p)[1]), dtype=torch.float32, device=dev) for p in projs}
+    dev_blocks, structs = [], []
+    for c in range(copies):
+        blk = blocks[c % len(blocks)]
+        db = {p: tuple(d(a) for a in blk[p]) for p in projs}   # fresh device copy each time
+        dev_blocks.append(db)
+        structs.append(rtq._QBlockC(*(t.data_ptr() for p in projs for t in db[p]),
+                                    wl.D_MODEL, wl.D_FF))
+    xptr = [xs[p].data_ptr() for p in projs]
+    yptr = [ys[p].data_ptr() for p in projs]
+
+    def step():
+        for c in structs:
+            st = L.rt_qblock_project(ctypes.byref(c), M, *xptr, *yptr, 0, sptr)
+            if st:
+                raise rtq.RtqError(st, "rt_qblock_project")
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            step()
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 1)):
+            graph.replay()
+    stream.synchronize()
+    if rtq.device_status(stream) != 0:
+        raise RuntimeError("device status word reports a timed-out wait during warm-up")
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+
+    gpu_id = local_rank
+    try:
+        gpu_id = str(torch.cuda.get_device_properties(dev).uuid)
+        gpu_id = gpu_id if gpu_id.startswith("GPU-") else "GPU-" + gpu_id
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    time.sleep(0.3)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    t0 = time.time()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    t1 = time.time()
+    barrier()
+    sampler.stop()
+    clocks = sampler.summary(t0, t1)
+    ms = reduce_max(e0.elapsed_time(e1), world, dev) / args.steps
+    if rtq.device_status(stream) != 0:
+        raise RuntimeError("device status word reports a timed-out wait")
+    del graph
+    wbytes = copies * per_block
+    gbs = world * wbytes / (ms * 1e-3) / 1e9
+    flops = copies * sum(proj_flops(p, M) for p in projs)
+    peaks = load_peaks()
+    kernels = sorted({rtq.plan(4 if proj_dims(p)[0] == "q4" else 8, M, *proj_dims(p)[1:])
+                      for p in projs})
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16", "accumulate": "f32",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "M": M, "projections": list(projs),
+                       "weight_copies": copies, "weight_bytes_per_step": wbytes,
+                       "l2_bytes": l2, "replay": "CUDA graph of all copies' block projection sets",
+                       "l2": f"weights rotate over {wbytes / 1e6:.0f} MB ({wbytes / l2:.1f}x L2); "
+                             f"X and Y fixed",
+                       "parallelism": f"replicas{world}" if world > 1 else "single"},
+            "tflops": world * flops / (ms * 1e-3) / 1e12,
+            "kernels": kernels, "clocks": clocks, "gpu_launches": args.steps * copies * len(projs),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                         "algorithmic_bytes_per_step": wbytes, "peak_source": peaks["source"]},
+            "e2e": None, "cpu_baseline": None,
+        }
+        print(json.dumps(line), flush=True)
 
 
 # ------------------------------------------------------------------- GPU
@@ -529,7 +658,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        run_gpu(args, rank, world, local_rank)
+        if args.workload == "rot_m80":
+            run_small_m(args, rank, world, local_rank)
+        else:
+            run_gpu(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -59,8 +59,16 @@ constexpr unsigned kStatusTimeout = 5u;          // RT_ERR_DEVICE_TIMEOUT
 
 __host__ __device__ inline int tc_stage_bytes(int bn) { return kAStageBytes + bn * 128; }
 
-__host__ __device__ inline int tc_smem_bytes(int bn, int stages) {
-    return 1024 + stages * tc_stage_bytes(bn) + (2 * stages + 1) * 8 + 16;
+// The stage ring, which with split K is reused for the CTA's fp32 partial
+// tile (BN columns of 128 rows).
+__host__ __device__ inline int tc_region_bytes(int bn, int stages, int ksplit) {
+    const int ring = stages * tc_stage_bytes(bn);
+    const int part = ksplit > 1 ? bn * kTileO * 4 : 0;
+    return ((ring > part ? ring : part) + 1023) / 1024 * 1024;
+}
+
+__host__ __device__ inline int tc_smem_bytes(int bn, int stages, int ksplit) {
+    return 1024 + tc_region_bytes(bn, stages, ksplit) + (2 * stages + 1) * 8 + 16;
 }
 
 __host__ __device__ inline uint32_t tmem_cols_for(int bn) {
@@ -184,13 +192,13 @@ template <int FMT, Op16 OP, int PIECES>
 __global__ void __launch_bounds__(kTcThreads, 2)
     tc_qgemm_kernel(const float *__restrict__ X, const void *__restrict__ Wq,
                     const void *__restrict__ S, float *__restrict__ Y, int M, int N, int K,
-                    int BN, int stages, unsigned *status) {
+                    int BN, int stages, int ksplit, unsigned *status) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *smem = smem_raw + (base - raw);
     const int stage_bytes = tc_stage_bytes(BN);
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + stages * stage_bytes);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + tc_region_bytes(BN, stages, ksplit));
     uint64_t *empty = full + stages;
     uint64_t *done = empty + stages;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
@@ -199,7 +207,9 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int o0 = blockIdx.x * kTileO;
     const int m0 = blockIdx.y * BN;
-    const int nk = K / kTileK;
+    // split K: CTA z of the cluster takes K steps [kz0, kz0 + nk)
+    const int nk = K / kTileK / ksplit;
+    const int kz0 = static_cast<int>(blockIdx.z) * nk;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
@@ -219,6 +229,22 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     const uint32_t tmem = *tmem_slot;
     bool ok = true;
 
+    if (warp < kConvWarps) {
+        // The weights do not depend on the previous kernel in the stream:
+        // start pulling this CTA's slice into L2 before waiting for it.
+        const int o = o0 + (static_cast<int>(threadIdx.x) >> 1);
+        if (o < N) {
+            for (int ks = 0; ks < nk; ++ks) {
+                const int k0 = (kz0 + ks) * kTileK;
+                if (FMT == 4)
+                    prefetch_l2(static_cast<const uint8_t *>(Wq) + static_cast<size_t>(o) * (K / 2) +
+                                k0 / 2);
+                else
+                    prefetch_l2(static_cast<const int8_t *>(Wq) + static_cast<size_t>(o) * K + k0 +
+                                (threadIdx.x & 1) * 32);
+            }
+        }
+    }
     pdl_wait_prior_grid();
 
     if (warp < kConvWarps) {
@@ -237,14 +263,17 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             mbar_arrive(&full[s]);
             return true;
         };
-        load_stage<FMT, PIECES>(r0, ct, X, Wq, S, o0, m0, 0, M, N, K, BN);
+        const int kb = kz0 * kTileK;
+        load_stage<FMT, PIECES>(r0, ct, X, Wq, S, o0, m0, kb, M, N, K, BN);
         for (int ks = 0; ks < nk; ks += 2) {
             if (ks + 1 < nk)
-                load_stage<FMT, PIECES>(r1, ct, X, Wq, S, o0, m0, (ks + 1) * kTileK, M, N, K, BN);
+                load_stage<FMT, PIECES>(r1, ct, X, Wq, S, o0, m0, kb + (ks + 1) * kTileK, M, N, K,
+                                        BN);
             if (!(ok = consume(r0, ks))) break;
             if (ks + 1 >= nk) break;
             if (ks + 2 < nk)
-                load_stage<FMT, PIECES>(r0, ct, X, Wq, S, o0, m0, (ks + 2) * kTileK, M, N, K, BN);
+                load_stage<FMT, PIECES>(r0, ct, X, Wq, S, o0, m0, kb + (ks + 2) * kTileK, M, N, K,
+                                        BN);
             if (!(ok = consume(r1, ks + 1))) break;
         }
         pdl_launch_dependents();
@@ -269,7 +298,18 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                 tmem_ld_x8(tbase + static_cast<uint32_t>(c), v0);
                 if (two) tmem_ld_x8(tbase + static_cast<uint32_t>(c + 8), v1);
                 tmem_ld_wait();
-                if (o < N) {
+                if (ksplit > 1) {
+                    // this CTA's partial sum, column-major [BN][128] in the
+                    // retired stage ring; reduced across the cluster below
+                    float *part = reinterpret_cast<float *>(smem);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) part[(c + j) * kTileO + row] = __uint_as_float(v0[j]);
+                    if (two) {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            part[(c + 8 + j) * kTileO + row] = __uint_as_float(v1[j]);
+                    }
+                } else if (o < N) {
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const int m = m0 + c + j;
@@ -314,6 +354,48 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     if (!ok) atomicOr(status, 1u << kStatusTimeout);
     tc_fence_before_sync();
     __syncthreads();
+    if (ksplit > 1) {
+        // Every CTA of the cluster reaches both barriers on every path (a
+        // timed-out wait only skips work), and a cluster's CTAs are resident
+        // together, so neither barrier can hang.
+        cluster_sync();                       // all partials written
+        if (warp < kConvWarps) {
+            // CTA rank r sums columns [r * BN/ksplit, (r + 1) * BN/ksplit) over
+            // the cluster's partials in rank order (deterministic) and stores Y.
+            const int cols = BN / ksplit;
+            const int mbeg = static_cast<int>(cluster_ctarank()) * cols;
+            for (int idx = threadIdx.x; idx < cols * (kTileO / 4); idx += kConvThreads) {
+                const int ml = mbeg + idx / (kTileO / 4), o4 = idx % (kTileO / 4);
+                const int m = m0 + ml, o = o0 + 4 * o4;
+                const uint32_t off = base + static_cast<uint32_t>((ml * kTileO + 4 * o4) * 4);
+                float4 acc = ld_cluster_f4(cluster_map(off, 0));
+                for (int r = 1; r < ksplit; ++r) {
+                    const float4 v = ld_cluster_f4(cluster_map(off, static_cast<uint32_t>(r)));
+                    acc.x += v.x;
+                    acc.y += v.y;
+                    acc.z += v.z;
+                    acc.w += v.w;
+                }
+                if (m < M && o < N) {
+                    float a[4] = {acc.x, acc.y, acc.z, acc.w};
+                    if (FMT == 8) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            if (o + e < N) a[e] *= __ldg(static_cast<const float *>(S) + o + e);
+                    }
+                    float *yp = Y + static_cast<size_t>(m) * N + o;
+                    if ((N & 3) == 0 && o + 3 < N) {
+                        *reinterpret_cast<float4 *>(yp) = make_float4(a[0], a[1], a[2], a[3]);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            if (o + e < N) yp[e] = a[e];
+                    }
+                }
+            }
+        }
+        cluster_sync();                       // peers are done reading this CTA's partial
+    }
     if (warp == 0) {
         tc_fence_after_sync();
         tmem_dealloc(tmem, tmem_cols);
@@ -331,6 +413,19 @@ int pick_bn(int M, int N) {
     return bn;
 }
 
+// K slices per output tile.  Small problems (one activation tile) have too
+// few 128-row weight tiles to occupy the GPU -- q8 w2 and wo have 4 -- so K is
+// split across a cluster of up to 8 CTAs, up to about two CTAs per SM.  The
+// slices' partial sums are reduced through distributed shared memory.
+int pick_ksplit(int M, int N, int K, int BN) {
+    if (M > BN) return 1;
+    const int nk = K / kTileK;
+    const long tiles = static_cast<long>((N + kTileO - 1) / kTileO);
+    int ks = 1;
+    while (ks < 8 && nk % (2 * ks) == 0 && tiles * ks * 2 <= 2 * 148) ks *= 2;
+    return ks;
+}
+
 template <int FMT, Op16 OP, int PIECES>
 cudaError_t launch_tc_pieces(const float *X, const void *Wq, const void *S, float *Y, int M, int N,
                             int K, int BN, unsigned *status, cudaStream_t st) {
@@ -344,22 +439,27 @@ cudaError_t launch_tc_pieces(const float *X, const void *Wq, const void *S, floa
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    const int nk = K / kTileK;
+    const int ksplit = pick_ksplit(M, N, K, BN);
+    const int nk = K / kTileK / ksplit;
     const int budget = kTwoCtaSmem;
     int stages = (budget - 1024 - 256) / tc_stage_bytes(BN);
     stages = std::max(1, std::min({stages, 4, nk}));
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((N + kTileO - 1) / kTileO, (M + BN - 1) / BN, 1);
+    cfg.gridDim = dim3((N + kTileO - 1) / kTileO, (M + BN - 1) / BN, ksplit);
     cfg.blockDim = dim3(kTcThreads, 1, 1);
-    cfg.dynamicSmemBytes = tc_smem_bytes(BN, stages);
+    cfg.dynamicSmemBytes = tc_smem_bytes(BN, stages, ksplit);
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 1;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = static_cast<unsigned>(ksplit);
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = ksplit > 1 ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, tc_qgemm_kernel<FMT, OP, PIECES>, X, Wq, S, Y, M, N, K, BN,
-                              stages, status);
+                              stages, ksplit, status);
 }
 
 template <int FMT, Op16 OP>
