@@ -61,6 +61,8 @@ WORKLOADS = {
     "qkvg_m4096": (4, 1, 4096, ("qkvg",)),
     # small M as an aggregate weight stream (see run_small_m)
     "rot_m80": (4, 0, 80, ("qkvg", "wo", "w13", "w2")),
+    # M in {1, 16, 80, 512, 4096, 65536} for the q4 512->2048 and q8 2048->512 shapes
+    "m_sweep": (5, 0, 0, ()),
     # outputs larger than L2, for full profiler captures of one launch
     "w13_m16384": (4, 1, 16384, ("w13",)),
     "w2_m16384": (4, 1, 16384, ("w2",)),
@@ -408,6 +410,97 @@ def run_small_m(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+# --------------------------------------------------------------- M sweep
+SWEEP_SHAPES = (("q4", 2048, 512), ("q8", 512, 2048))    # ffn.w1 and ffn.w2 shapes
+SWEEP_M = (1, 16, 80, 512, 4096, 65536)
+
+
+def run_sweep(args, rank, world, local_rank):
+    """M sweep of the q4 512->2048 and q8 2048->512 projections under
+    RT_PATH_AUTO (weights with a seeded 1 % of 32-groups holding a x20
+    outlier).  Each point is 20 calls captured in a CUDA graph, replayed
+    after warm-up; inputs stay in place between calls, so points whose data
+    fit in L2 (M <= 4096) run L2-warm.  value = TFLOP/s of the q4 shape at
+    M = 65536, the large-M gate; `sweep` lists every point and the kernel the
+    dispatcher chose."""
+    import torch
+
+    import int8_dequant_gemm_b200 as rtq
+
+    rtq.lib()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.Stream(device=dev)
+    sptr = ctypes.c_void_p(stream.cuda_stream)
+    L = rtq.lib()
+    reps = 20
+    points = []
+    for fmt, N, K in SWEEP_SHAPES:
+        seed = wl.seed_for(5, 0, 1 if fmt == "q4" else 3)
+        W = wl.with_outliers(wl.weights(N, K, seed), seed + 1)
+        Wq, S = rtq.quantize_q4_g32(W) if fmt == "q4" else rtq.quantize_q8_row(W)
+        Wd = torch.from_numpy(Wq).to(dev)
+        Sd = torch.from_numpy(S).to(dev)
+        fn = L.rt_qgemm_q4 if fmt == "q4" else L.rt_qgemm_q8
+        fcode = 4 if fmt == "q4" else 8
+        for M in SWEEP_M:
+            X = torch.from_numpy(wl.activations(M, K, seed + 2 + M)).to(dev)
+            Y = torch.empty((M, N), dtype=torch.float32, device=dev)
+            call_args = (X.data_ptr(), Wd.data_ptr(), Sd.data_ptr(), Y.data_ptr(), M, N, K, 0, sptr)
+
+            def calls():
+                for _ in range(reps):
+                    st = fn(*call_args)
+                    if st:
+                        raise rtq.RtqError(st, "rt_qgemm")
+
+            with torch.cuda.stream(stream):
+                calls()                      # grows the workspace outside the capture
+            stream.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                calls()
+            with torch.cuda.stream(stream):
+                for _ in range(max(args.warmup, 1)):
+                    g.replay()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            stream.synchronize()
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                for _ in range(args.steps):
+                    g.replay()
+                e1.record(stream)
+            stream.synchronize()
+            del g
+            us = e0.elapsed_time(e1) * 1e3 / (args.steps * reps)
+            wb = Wq.nbytes + S.nbytes
+            points.append({"shape": f"{fmt} {K}->{N}", "M": M, "kernel": rtq.plan(fcode, M, N, K),
+                           "us_per_call": us, "tflops": 2.0 * M * N * K / (us * 1e-6) / 1e12,
+                           "weight_gbs": wb / (us * 1e-6) / 1e9})
+            del X, Y
+    if rtq.device_status(stream) != 0:
+        raise RuntimeError("device status word reports a timed-out wait")
+    peaks = load_peaks()
+    head = next(p for p in points if p["shape"].startswith("q4") and p["M"] == SWEEP_M[-1])
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": head["tflops"], "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["us_per_call"] * 1e-3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+            "accumulate": "f32", "data": "synthetic",
+            "config": {"workload": "m_sweep", "shapes": [f"{f} {k}->{n}" for f, n, k in SWEEP_SHAPES],
+                       "M": list(SWEEP_M), "calls_per_graph": reps, "path": "auto",
+                       "l2": "inputs reused between calls: L2-warm for M <= 4096"},
+            "roofline": {"bound": "tensor", "achieved": head["tflops"],
+                         "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                         "frac": head["tflops"] / peaks["bf16_tflops_sustained"],
+                         "peak_source": peaks["source"]},
+            "sweep": points, "e2e": None, "cpu_baseline": None,
+        }
+        print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------- GPU
 def run_gpu(args, rank, world, local_rank):
     import torch
@@ -660,6 +753,8 @@ def main():
     try:
         if args.workload == "rot_m80":
             run_small_m(args, rank, world, local_rank)
+        elif args.workload == "m_sweep":
+            run_sweep(args, rank, world, local_rank)
         else:
             run_gpu(args, rank, world, local_rank)
     finally:

@@ -110,7 +110,10 @@ int rt_qgemm_auto_path(int fmt, int64_t M, int64_t N, int64_t K);
  *   RT_KERNEL_TC_W_STATIONARY tcgen05, one 128-row weight tile x up to 128
  *                             activation rows per CTA, converter warps load and
  *                             convert both operands (M <= 128, or shapes the
- *                             TMA kernels do not take);
+ *                             TMA kernels do not take); with one activation
+ *                             tile, K is split over a cluster of up to 8 CTAs
+ *                             whose partial sums are reduced in distributed
+ *                             shared memory (deterministic order);
  *   RT_KERNEL_TC_X_RESIDENT   tcgen05, persistent CTAs keep a 192-row block of
  *                             activations in shared memory and stream TMA-staged
  *                             weight tiles past it (M > 128, K a multiple of

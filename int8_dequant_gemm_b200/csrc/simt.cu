@@ -1,12 +1,19 @@
 // fp32 CUDA-core kernels: the exact-rounding path (weights dequantized to
-// fp32 with one rounding, fp32 FMA accumulation) and the small-M path.
+// fp32 with one rounding, fp32 FMA accumulation) and the path for M <= 8.
 //
 // Layout of work: each thread owns one output row o of W and MT activation
-// rows, staged once per block in shared memory.  Inside the K loop every lane
-// of a warp reads the same activation address (a shared-memory broadcast), so
+// rows, staged per CTA in shared memory.  Inside the K loop every lane of a
+// warp reads the same activation address (a shared-memory broadcast), so
 // shared memory bandwidth is not the limit; the weight stream is one 16-byte
 // load per thread per step (a q4 group, or 16 q8 codes) that L1 completes to
 // full sectors on the following step.
+//
+// One thread per row gives only N threads, too few to keep the weight stream
+// in flight (N = 512 for the q8 projections), so K is split across a cluster
+// of up to 8 CTAs: each stages and sums its K slice, writes its per-row
+// partials to shared memory, and after a cluster barrier CTA rank r sums a
+// 1/ksplit share of the (row, activation row) outputs over the cluster in rank
+// order (deterministic) and stores them.
 #include <algorithm>
 
 #include "dequant.cuh"
@@ -16,125 +23,163 @@
 namespace rtq {
 namespace {
 
-constexpr int kSimtThreads = 256;
+constexpr int kSimtThreads = 128;                 // weight rows per CTA
 
+// X rows m0 .. m0 + mt - 1, columns [k0, k0 + Ks), as MT x Ks floats.
 template <int MT>
 __device__ __forceinline__ void stage_x(const float *__restrict__ X, float4 *xs4, int m0, int mt,
-                                        int K) {
-    const int K4 = K / 4;
+                                        int K, int k0, int Ks) {
+    const int K4 = Ks / 4;
     for (int i = threadIdx.x; i < MT * K4; i += blockDim.x) {
         const int r = i / K4;
         float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (r < mt) v = ldg_f4(X + static_cast<size_t>(m0 + r) * K + (i - r * K4) * 4);
+        if (r < mt) v = ldg_f4(X + static_cast<size_t>(m0 + r) * K + k0 + (i - r * K4) * 4);
         xs4[i] = v;
     }
 }
 
-template <int MT>
-__global__ void __launch_bounds__(kSimtThreads)
-    simt_q4_kernel(const float *__restrict__ X, const uint8_t *__restrict__ Wq,
-                   const uint32_t *__restrict__ SM, float *__restrict__ Y, int M, int N, int K) {
-    extern __shared__ float4 xs4[];
-    const float *xs = reinterpret_cast<const float *>(xs4);
-    const int m0 = blockIdx.x * MT;
-    const int mt = min(MT, M - m0);
-    pdl_wait_prior_grid();
-    stage_x<MT>(X, xs4, m0, mt, K);
-    __syncthreads();
-    pdl_launch_dependents();
-
-    const int o = blockIdx.y * kSimtThreads + threadIdx.x;
-    if (o >= N) return;
-    float acc[MT];
+// Sum of the K slice [k0, k0 + Ks) of row o (valid: o < N) into acc[MT].
+template <int MT, int FMT>
+__device__ __forceinline__ void simt_slice(const float *xs, const void *__restrict__ Wq,
+                                           const void *__restrict__ S, int o, bool valid, int K,
+                                           int k0, int Ks, float (&acc)[MT]) {
 #pragma unroll
     for (int m = 0; m < MT; ++m) acc[m] = 0.f;
-
-    const uint8_t *wrow = Wq + static_cast<size_t>(o) * (K / 2);
-    const uint32_t *srow = SM + static_cast<size_t>(o) * (K / 32);
-    const int G = K / 32;
-    for (int g = 0; g < G; ++g) {
-        const uint4 p = ldg_v4(wrow + g * 16);
-        float sc, mn;
-        q4_scale_min(__ldg(srow + g), sc, mn);
-        const uint32_t words[4] = {p.x, p.y, p.z, p.w};
+    if (!valid) return;
+    if (FMT == 4) {
+        const uint8_t *wrow = static_cast<const uint8_t *>(Wq) + static_cast<size_t>(o) * (K / 2);
+        const uint32_t *srow = static_cast<const uint32_t *>(S) + static_cast<size_t>(o) * (K / 32);
+        for (int g = 0; g < Ks / 32; ++g) {
+            const int kg = k0 / 32 + g;
+            const uint4 p = ldg_v4(wrow + kg * 16);
+            float sc, mn;
+            q4_scale_min(__ldg(srow + kg), sc, mn);
+            const uint32_t words[4] = {p.x, p.y, p.z, p.w};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            float w[8];
-            q4_word_f32(words[c], sc, mn, w);
+            for (int c = 0; c < 4; ++c) {
+                float w[8];
+                q4_word_f32(words[c], sc, mn, w);
 #pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                const float4 *xr = reinterpret_cast<const float4 *>(xs + m * K + g * 32 + c * 8);
-                const float4 a = xr[0], b = xr[1];
-                float t = acc[m];
-                t = fmaf(a.x, w[0], t);
-                t = fmaf(a.y, w[1], t);
-                t = fmaf(a.z, w[2], t);
-                t = fmaf(a.w, w[3], t);
-                t = fmaf(b.x, w[4], t);
-                t = fmaf(b.y, w[5], t);
-                t = fmaf(b.z, w[6], t);
-                t = fmaf(b.w, w[7], t);
-                acc[m] = t;
+                for (int m = 0; m < MT; ++m) {
+                    const float4 *xr = reinterpret_cast<const float4 *>(xs + m * Ks + g * 32 + c * 8);
+                    const float4 a = xr[0], b = xr[1];
+                    float t = acc[m];
+                    t = fmaf(a.x, w[0], t);
+                    t = fmaf(a.y, w[1], t);
+                    t = fmaf(a.z, w[2], t);
+                    t = fmaf(a.w, w[3], t);
+                    t = fmaf(b.x, w[4], t);
+                    t = fmaf(b.y, w[5], t);
+                    t = fmaf(b.z, w[6], t);
+                    t = fmaf(b.w, w[7], t);
+                    acc[m] = t;
+                }
+            }
+        }
+    } else {
+        // q8: the row scale is factored out of the K sum and applied once at
+        // the end, Y = scale[o] * sum_k x * q.
+        const int8_t *wrow = static_cast<const int8_t *>(Wq) + static_cast<size_t>(o) * K + k0;
+        for (int kk = 0; kk < Ks; kk += 16) {
+            const uint4 p = ldg_v4(wrow + kk);
+            const uint32_t words[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float w0 = q8_byte_f32(words[c], 0), w1 = q8_byte_f32(words[c], 1);
+                const float w2 = q8_byte_f32(words[c], 2), w3 = q8_byte_f32(words[c], 3);
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    const float4 a = *reinterpret_cast<const float4 *>(xs + m * Ks + kk + c * 4);
+                    float t = acc[m];
+                    t = fmaf(a.x, w0, t);
+                    t = fmaf(a.y, w1, t);
+                    t = fmaf(a.z, w2, t);
+                    t = fmaf(a.w, w3, t);
+                    acc[m] = t;
+                }
             }
         }
     }
-#pragma unroll
-    for (int m = 0; m < MT; ++m)
-        if (m < mt) Y[static_cast<size_t>(m0 + m) * N + o] = acc[m];
 }
 
-// q8: the row scale is factored out of the K sum, Y = scale[o] * sum_k x*q,
-// and applied once in fp32 at the end.
-template <int MT>
+template <int MT, int FMT>
 __global__ void __launch_bounds__(kSimtThreads)
-    simt_q8_kernel(const float *__restrict__ X, const int8_t *__restrict__ Wq,
-                   const float *__restrict__ S, float *__restrict__ Y, int M, int N, int K) {
+    simt_kernel(const float *__restrict__ X, const void *__restrict__ Wq,
+                const void *__restrict__ S, float *__restrict__ Y, int M, int N, int K,
+                int ksplit) {
     extern __shared__ float4 xs4[];
     const float *xs = reinterpret_cast<const float *>(xs4);
+    const int Ks = K / ksplit;
+    const int k0 = static_cast<int>(blockIdx.z) * Ks;
     const int m0 = blockIdx.x * MT;
     const int mt = min(MT, M - m0);
+    const int o0 = blockIdx.y * kSimtThreads;
+    const int o = o0 + threadIdx.x;
+    const bool valid = o < N;
+    // the weights do not depend on the previous kernel in the stream
+    if (valid) {
+        const int step = FMT == 4 ? 256 : 128;   // one prefetch per 128-byte line
+        const char *w = static_cast<const char *>(Wq) +
+                        (FMT == 4 ? static_cast<size_t>(o) * (K / 2) + k0 / 2
+                                  : static_cast<size_t>(o) * K + k0);
+        for (int k = 0; k < Ks; k += step) prefetch_l2(w + (FMT == 4 ? k / 2 : k));
+    }
     pdl_wait_prior_grid();
-    stage_x<MT>(X, xs4, m0, mt, K);
+    stage_x<MT>(X, xs4, m0, mt, K, k0, Ks);
     __syncthreads();
     pdl_launch_dependents();
 
-    const int o = blockIdx.y * kSimtThreads + threadIdx.x;
-    if (o >= N) return;
     float acc[MT];
+    simt_slice<MT, FMT>(xs, Wq, S, o, valid, K, k0, Ks, acc);
+    const float sc = (FMT == 8 && valid) ? __ldg(static_cast<const float *>(S) + o) : 1.f;
+    if (ksplit == 1) {
+        if (valid) {
 #pragma unroll
-    for (int m = 0; m < MT; ++m) acc[m] = 0.f;
-    const int8_t *wrow = Wq + static_cast<size_t>(o) * K;
-    for (int k0 = 0; k0 < K; k0 += 16) {
-        const uint4 p = ldg_v4(wrow + k0);
-        const uint32_t words[4] = {p.x, p.y, p.z, p.w};
+            for (int m = 0; m < MT; ++m)
+                if (m < mt) Y[static_cast<size_t>(m0 + m) * N + o] = acc[m] * sc;
+        }
+        return;
+    }
+    // split K: partials [MT][kSimtThreads] after the staged activations
+    float *part = reinterpret_cast<float *>(xs4) + MT * Ks;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const float w0 = q8_byte_f32(words[c], 0), w1 = q8_byte_f32(words[c], 1);
-            const float w2 = q8_byte_f32(words[c], 2), w3 = q8_byte_f32(words[c], 3);
-#pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                const float4 a = *reinterpret_cast<const float4 *>(xs + m * K + k0 + c * 4);
-                float t = acc[m];
-                t = fmaf(a.x, w0, t);
-                t = fmaf(a.y, w1, t);
-                t = fmaf(a.z, w2, t);
-                t = fmaf(a.w, w3, t);
-                acc[m] = t;
-            }
+    for (int m = 0; m < MT; ++m) part[m * kSimtThreads + threadIdx.x] = acc[m];
+    cluster_sync();                           // all partials written
+    const int share = MT * kSimtThreads / ksplit;
+    const int beg = static_cast<int>(cluster_ctarank()) * share;
+    const uint32_t pbase = smem_addr(part);
+    for (int i = threadIdx.x; i < share; i += kSimtThreads) {
+        const int idx = beg + i, m = idx / kSimtThreads, row = idx % kSimtThreads;
+        const uint32_t off = pbase + static_cast<uint32_t>(idx * 4);
+        float v = ld_cluster_f32(cluster_map(off, 0));
+        for (int r = 1; r < ksplit; ++r) v += ld_cluster_f32(cluster_map(off, static_cast<uint32_t>(r)));
+        const int oo = o0 + row;
+        if (m < mt && oo < N) {
+            const float s8 = FMT == 8 ? __ldg(static_cast<const float *>(S) + oo) : 1.f;
+            Y[static_cast<size_t>(m0 + m) * N + oo] = v * s8;
         }
     }
-    const float sc = __ldg(S + o);
-#pragma unroll
-    for (int m = 0; m < MT; ++m)
-        if (m < mt) Y[static_cast<size_t>(m0 + m) * N + o] = acc[m] * sc;
+    cluster_sync();                           // peers are done reading this CTA's partials
+}
+
+// K slices: up to 8, while the grid stays within about four CTAs per SM and
+// each slice keeps whole q4 groups (32) and 16-byte q8 loads, at least 64
+// wide.
+int pick_simt_ksplit(int M, int N, int K, int MT) {
+    const long ctas = static_cast<long>((M + MT - 1) / MT) * ((N + kSimtThreads - 1) / kSimtThreads);
+    int ks = 1;
+    while (ks < 8 && K % (2 * ks * 64) == 0 && ctas * ks * 2 <= 4 * 148) ks *= 2;
+    return ks;
 }
 
 template <int MT>
 cudaError_t launch_simt_mt(bool q4, const float *X, const void *Wq, const void *S, float *Y,
                            int M, int N, int K, cudaStream_t s) {
-    const size_t smem = static_cast<size_t>(MT) * K * sizeof(float);
-    void *fn = q4 ? reinterpret_cast<void *>(&simt_q4_kernel<MT>)
-                  : reinterpret_cast<void *>(&simt_q8_kernel<MT>);
+    const int ksplit = pick_simt_ksplit(M, N, K, MT);
+    const size_t smem = static_cast<size_t>(MT) * (K / ksplit) * sizeof(float) +
+                        (ksplit > 1 ? static_cast<size_t>(MT) * kSimtThreads * sizeof(float) : 0);
+    void *fn = q4 ? reinterpret_cast<void *>(&simt_kernel<MT, 4>)
+                  : reinterpret_cast<void *>(&simt_kernel<MT, 8>);
     if (smem > 48 * 1024) {
         cudaError_t e =
             cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -142,21 +187,21 @@ cudaError_t launch_simt_mt(bool q4, const float *X, const void *Wq, const void *
         if (e != cudaSuccess) return e;
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((M + MT - 1) / MT, (N + kSimtThreads - 1) / kSimtThreads, 1);
+    cfg.gridDim = dim3((M + MT - 1) / MT, (N + kSimtThreads - 1) / kSimtThreads, ksplit);
     cfg.blockDim = dim3(kSimtThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 1;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = static_cast<unsigned>(ksplit);
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (q4)
-        return cudaLaunchKernelEx(&cfg, simt_q4_kernel<MT>, X,
-                                  static_cast<const uint8_t *>(Wq),
-                                  static_cast<const uint32_t *>(S), Y, M, N, K);
-    return cudaLaunchKernelEx(&cfg, simt_q8_kernel<MT>, X, static_cast<const int8_t *>(Wq),
-                              static_cast<const float *>(S), Y, M, N, K);
+    cfg.numAttrs = ksplit > 1 ? 2 : 1;
+    if (q4) return cudaLaunchKernelEx(&cfg, simt_kernel<MT, 4>, X, Wq, S, Y, M, N, K, ksplit);
+    return cudaLaunchKernelEx(&cfg, simt_kernel<MT, 8>, X, Wq, S, Y, M, N, K, ksplit);
 }
 
 // Activation rows per block: as many as M needs up to 8, capped so the staged

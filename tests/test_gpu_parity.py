@@ -163,8 +163,12 @@ def test_identity_input_q8_bit_exact(rtq_lib, path):
 # ----------------------------------------------------------- GEMM parity
 SIMT_SHAPES = [(1, 2048, 512), (3, 130, 96), (17, 300, 128), (80, 2048, 512), (79, 512, 2048),
                (129, 64, 64), (8, 1, 32)]
+# one activation tile splits K over a cluster of 2, 4 or 8 CTAs: (81, 130, 128)
+# -> 2, (64, 5120, 256) -> 4, (80, 2048, 512) and (80, 512, 2048) -> 8; (48,
+# 1001, 512) reduces into an odd N, (5, 640, 1024) leaves 2 columns per CTA
 TC_SHAPES = [(16, 256, 64), (80, 2048, 512), (80, 512, 2048), (81, 130, 128), (300, 512, 512),
-             (1, 128, 64), (256, 200, 192), (1000, 640, 512)]
+             (1, 128, 64), (256, 200, 192), (1000, 640, 512), (64, 5120, 256), (48, 1001, 512),
+             (5, 640, 1024)]
 
 
 def _run_q4(rtq_lib, M, N, K, path, seed, outliers=False):
