@@ -144,10 +144,9 @@ __device__ __forceinline__ HalfRaw load_half_raw2(uint32_t slot, int r, int h, i
     return R;
 }
 
-// 32 weights of a half step -> 16 32-bit operand words (4 chunks) -> TMEM
-// columns [ta, ta + 16) of this thread's lane.  Warp-collective.
+// 32 weights of a half step -> 16 32-bit operand words (4 chunks).
 template <int FMT, Op16 OP>
-__device__ __forceinline__ void tmem_half_op(const HalfRaw &R, uint32_t ta) {
+__device__ __forceinline__ void half_words(const HalfRaw &R, uint32_t (&w)[16]) {
     uint4 ch[4];
     if (FMT == 4) {
         if (OP == Op16::f16) {
@@ -178,7 +177,6 @@ __device__ __forceinline__ void tmem_half_op(const HalfRaw &R, uint32_t ta) {
             ch[3] = q8_words_bf16(R.p1.z, R.p1.w);
         }
     }
-    uint32_t w[16];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
         w[4 * c + 0] = ch[c].x;
@@ -186,7 +184,6 @@ __device__ __forceinline__ void tmem_half_op(const HalfRaw &R, uint32_t ta) {
         w[4 * c + 2] = ch[c].z;
         w[4 * c + 3] = ch[c].w;
     }
-    tmem_st_x16(ta, w);
 }
 
 // The (scale, min) words of row r for 8 K steps: a 64-byte row of a staged

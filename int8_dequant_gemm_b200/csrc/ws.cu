@@ -229,6 +229,8 @@ __global__ void __launch_bounds__(kWsThreads, 1)
                     }
                     const HalfRaw R =
                         load_half_raw<FMT>(base + L.raw_off + slot * kRawSlot, r, h, sw[i]);
+                    uint32_t w[16];
+                    half_words<FMT, OP>(R, w);          // before the stage wait, as in xs.cu
                     const int s = j % kAStages;
                     if (j >= kAStages &&
                         !mbar_wait(&a_empty[s], static_cast<uint32_t>((j / kAStages) - 1) & 1u)) {
@@ -236,7 +238,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
                         break;
                     }
                     tc_fence_after_sync();
-                    tmem_half_op<FMT, OP>(R, ta + static_cast<uint32_t>(s) * kAStageCols);
+                    tmem_st_x16(ta + static_cast<uint32_t>(s) * kAStageCols, w);
                     tmem_st_wait();
                     tc_fence_before_sync();
                     mbar_arrive(&a_full[s]);

@@ -285,6 +285,10 @@ __global__ void __launch_bounds__(kXsThreads, 1)
                 }
                 const HalfRaw R = load_half_raw2<FMT>(base + L.raw_off + slot * kRawSlot, r, h,
                                                       ks & 1, sw[ks]);
+                // convert before waiting: only the TMEM store needs the stage
+                // free, which keeps the arithmetic off the stage's round trip
+                uint32_t w[16];
+                half_words<FMT, OP>(R, w);
                 const int s = j % kAStages;
                 if (j >= kAStages &&
                     !mbar_wait(&a_empty[s], static_cast<uint32_t>((j / kAStages) - 1) & 1u)) {
@@ -292,7 +296,7 @@ __global__ void __launch_bounds__(kXsThreads, 1)
                     break;
                 }
                 tc_fence_after_sync();
-                tmem_half_op<FMT, OP>(R, ta + static_cast<uint32_t>(s) * kAStageCols);
+                tmem_st_x16(ta + static_cast<uint32_t>(s) * kAStageCols, w);
                 tmem_st_wait();
                 tc_fence_before_sync();
                 mbar_arrive(&a_full[s]);
