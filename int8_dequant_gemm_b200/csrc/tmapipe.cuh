@@ -13,12 +13,6 @@ namespace rtq {
 
 constexpr int kTileRows = 128;      // MMA M (weight rows) and TMA box height
 constexpr int kAtomK = 64;          // K per stage: one 128-byte row of 16-bit operands
-constexpr int kOpStage = kTileRows * 128;   // 16 KB: one 128 x 64 16-bit operand tile
-
-__device__ __forceinline__ uint32_t swz128(int r, int c) {
-    return static_cast<uint32_t>(r * 128 + ((c ^ (r & 7)) << 4));
-}
-
 __device__ __forceinline__ uint4 lds_v4(uint32_t a) {
     uint4 v;
     asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -99,28 +93,7 @@ struct HalfRaw {
     uint32_t smw;
 };
 
-// Row r's codes of a staged K step (q4: 32 B per row, q8: 64 B per row).
-// q8 reads its two 16-byte chunks in an order rotated with the row, which
-// halves the bank conflicts of the 64-byte row stride.
-template <int FMT>
-__device__ __forceinline__ HalfRaw load_half_raw(uint32_t slot, int r, int h, uint32_t smw) {
-    HalfRaw R;
-    if (FMT == 4) {
-        R.p0 = lds_v4(slot + r * 32 + h * 16);
-        R.p1 = make_uint4(0, 0, 0, 0);
-        R.smw = smw;
-    } else {
-        const int rot = (r >> 1) & 1;
-        const uint4 u = lds_v4(slot + r * 64 + h * 32 + rot * 16);
-        const uint4 w = lds_v4(slot + r * 64 + h * 32 + (rot ^ 1) * 16);
-        R.p0 = rot ? w : u;
-        R.p1 = rot ? u : w;
-        R.smw = 0;
-    }
-    return R;
-}
-
-// The same half-row read from a slot that holds two K steps per row, as one
+// A half-row read from a slot that holds two K steps per row, as one
 // TMA box in a swizzled layout: q4 rows of 64 bytes (SWIZZLE_64B: 16-byte
 // chunk c of row r sits at chunk c ^ ((r >> 1) & 3)), q8 rows of 128 bytes
 // (SWIZZLE_128B: chunk c at c ^ (r & 7)).  u selects the step within the

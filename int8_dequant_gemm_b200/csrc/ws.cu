@@ -50,8 +50,10 @@ constexpr uint32_t kMmaBar = 1;                          // named barrier: waite
 constexpr int kStages = 6;                               // B stages (shared memory)
 constexpr int kStageBytes = kWsTileM * 128;              // 24 KB: 192 rows x 64 K
 constexpr int kAStages = 4;                              // A stages (TMEM)
-constexpr int kRaw = 6;
-constexpr int kRawSlot = 8 * 1024;
+constexpr int kRaw = 3;                                  // packed-code ring depth (step pairs)
+// Two K steps of packed codes per TMA box (128 rows x 64 B for q4, x 128 B for
+// q8, swizzled), as in xs.cu: a box costs about the same per row at any width.
+__host__ __device__ constexpr int raw_slot_bytes(int fmt) { return kTileRows * (fmt == 4 ? 64 : 128); }
 constexpr int kScaleSlot = 8 * 1024;                     // 128 rows x 16 words
 constexpr int kScaleWords = 16;                          // (scale, min) words per chunk row
 constexpr int kChunkSteps = kScaleWords / 2;             // K steps covered by one chunk
@@ -70,7 +72,7 @@ __host__ __device__ inline WsLayout ws_layout() {
     WsLayout L;
     L.st_off = 0;
     L.raw_off = kStages * kStageBytes;
-    L.sc_off = L.raw_off + kRaw * kRawSlot;
+    L.sc_off = L.raw_off + kRaw * raw_slot_bytes(8);   // sized for the larger q8 slots
     L.bar_off = L.sc_off + 2 * kScaleSlot;
     // a_full/a_empty[kAStages], b_full/b_empty[kStages], raw_full/empty[kRaw],
     // sc_full/empty[2], acc_full/empty[2], + TMEM address slot
@@ -109,7 +111,9 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     const int nk = K / kAtomK;
     const int n_chunks = (nk + kChunkSteps - 1) / kChunkSteps;
     const int G = gridDim.x;
-    const uint32_t raw_bytes = kTileRows * (FMT == 4 ? 32 : 64);
+    constexpr int kRawSlot = raw_slot_bytes(FMT);
+    const uint32_t raw_bytes = kRawSlot;
+    const int npairs = (nk + 1) / 2;                 // step pairs per tile (q8 K may be odd)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kAStages; ++s) {
@@ -148,7 +152,8 @@ __global__ void __launch_bounds__(kWsThreads, 1)
             int j = 0, q = 0;
             for (int t = blockIdx.x; t < n_tiles && ok; t += G) {
                 const int y0 = (t % n_o_tiles) * kTileRows;
-                for (int ks = 0; ks < nk; ++ks, ++j) {
+                for (int p = 0; p < npairs; ++p, ++j) {
+                    const int ks = 2 * p;
                     if (FMT == 4 && ks % kChunkSteps == 0) {
                         const int b = q & 1;
                         if (q >= 2 &&
@@ -169,7 +174,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
                     }
                     mbar_expect_tx(&raw_full[slot], raw_bytes);
                     tma_load_2d(base + L.raw_off + slot * kRawSlot, &w_map,
-                                ks * (FMT == 4 ? 32 : 64), y0, &raw_full[slot]);
+                                p * (FMT == 4 ? 64 : 128), y0, &raw_full[slot]);
                 }
             }
         }
@@ -222,13 +227,15 @@ __global__ void __launch_bounds__(kWsThreads, 1)
                     const int ks = c * kChunkSteps + i;
                     if (ks >= nk) break;
                     const int j = tile_local * nk + ks;
-                    const int slot = j % kRaw;
-                    if (!mbar_wait(&raw_full[slot], static_cast<uint32_t>(j / kRaw) & 1u)) {
+                    const int jp = tile_local * npairs + (ks >> 1);   // step pair of the raw ring
+                    const int slot = jp % kRaw;
+                    if ((ks & 1) == 0 &&
+                        !mbar_wait(&raw_full[slot], static_cast<uint32_t>(jp / kRaw) & 1u)) {
                         ok = false;
                         break;
                     }
-                    const HalfRaw R =
-                        load_half_raw<FMT>(base + L.raw_off + slot * kRawSlot, r, h, sw[i]);
+                    const HalfRaw R = load_half_raw2<FMT>(base + L.raw_off + slot * kRawSlot, r, h,
+                                                          ks & 1, sw[i]);
                     uint32_t w[16];
                     half_words<FMT, OP>(R, w);          // before the stage wait, as in xs.cu
                     const int s = j % kAStages;
@@ -242,8 +249,10 @@ __global__ void __launch_bounds__(kWsThreads, 1)
                     tmem_st_wait();
                     tc_fence_before_sync();
                     mbar_arrive(&a_full[s]);
-                    fence_proxy_async_smem();
-                    mbar_arrive(&raw_empty[slot]);   // after its contents were consumed
+                    if ((ks & 1) || ks == nk - 1) {   // the pair's last step has consumed it
+                        fence_proxy_async_smem();
+                        mbar_arrive(&raw_empty[slot]);
+                    }
                 }
             }
         }
@@ -376,13 +385,13 @@ cudaError_t launch_ws(const void *Xh, const void *Wq, const void *S, float *Y, i
                                 2, Xh, K, M, kAtomK, CU_TENSOR_MAP_SWIZZLE_128B, kWsTileM);
     if (FMT == 4) {
         enc_ok = enc_ok &&
-                 encode_tma_2d(&w_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Wq, K / 2, N, 32,
-                               CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                 encode_tma_2d(&w_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Wq, K / 2, N, 64,
+                               CU_TENSOR_MAP_SWIZZLE_64B) &&
                  encode_tma_2d(&s_map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, S, K / 32, N,
                                kScaleWords, CU_TENSOR_MAP_SWIZZLE_NONE);
     } else {
-        enc_ok = enc_ok && encode_tma_2d(&w_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Wq, K, N, 64,
-                                         CU_TENSOR_MAP_SWIZZLE_NONE);
+        enc_ok = enc_ok && encode_tma_2d(&w_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Wq, K, N, 128,
+                                         CU_TENSOR_MAP_SWIZZLE_128B);
         s_map = w_map;   // unused by the q8 kernel
     }
     if (!enc_ok) return cudaErrorInvalidValue;

@@ -261,6 +261,16 @@ def test_w_streamed_parity_q8(rtq_lib, M, N, K, path):
     assert rel_err(Y, ref) <= MAX_REL[path]
 
 
+@pytest.mark.parametrize("path", ["tc", "tc_bf16"])
+def test_w_streamed_odd_step_count_q8(rtq_lib, path):
+    """q8 with K = 576: nine 64-wide K steps, so the last two-step box of
+    packed codes is half past the end of each row (zero-filled by TMA)."""
+    M, N, K = 700, 384, 576
+    assert rtq_lib.plan(8, M, N, K, path) == "tc_w_streamed"
+    Y, ref = _run_q8(rtq_lib, M, N, K, path, seed=4242, outliers=True)
+    assert rel_err(Y, ref) <= MAX_REL[path]
+
+
 def test_w_streamed_many_tiles_every_tile(rtq_lib):
     """Several 128 x 128 tiles per persistent CTA (M = 32768, N = 1024, q8,
     K = 2048): every tile against the fp32 SIMT path, twice."""
