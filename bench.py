@@ -21,6 +21,17 @@ Printed as one JSON line (rank 0):
 `--impl reference` times the CPU oracle itself (rank 0 only) on the same
 workload, metric and unit, one bounded row sample per step.
 
+Other workloads (`--workload`), each printing one line of the same form:
+  rot_m80      small M as an aggregate weight stream: the 12 blocks' weights in
+               rotating device copies totalling ~4x L2, every copy's projection
+               set at M = 80, replayed from a CUDA graph; value in GB/s of
+               quantized weights.
+  m_sweep      M in {1, 16, 80, 512, 4096, 65536} for the q4 512->2048 and q8
+               2048->512 shapes under the automatic dispatch; value = TFLOP/s
+               of the q4 shape at M = 65536, every point under `sweep`.
+  w13_m4096, w2_m4096, qkvg_m4096, w13_m16384, w2_m16384
+               single projections, sized for profiler captures.
+
 Multi-GPU (torchrun): every rank runs the same step on its own batch (replica
 weights, rank-seeded activations, no data-path collective) -> weak scaling.
 """
@@ -256,6 +267,11 @@ def cpu_oracle_sample(blocks, M, projs, rows_per_proj, seed):
 def run_reference(args, rank, world):
     """The CPU oracle, timed on this host's cores, on the same workload."""
     if rank != 0:
+        return
+    if WORKLOADS[args.workload][1] == 0:
+        print(json.dumps({"impl": "reference", "unavailable":
+                          f"the oracle arm times the block workloads; {args.workload} has none"}),
+              flush=True)
         return
     cfg, nblocks, M, projs, blocks = build_host(args.workload, 0, use_oracle_quantizer=True)
     rows = args.ref_rows
