@@ -404,6 +404,10 @@ def run_small_m(args, rank, world, local_rank):
     peaks = load_peaks()
     kernels = sorted({rtq.plan(4 if proj_dims(p)[0] == "q4" else 8, M, *proj_dims(p)[1:])
                       for p in projs})
+    fused = rtq.block_fused(M, wl.D_MODEL, wl.D_FF) == 1
+    launches_per_copy = 1 if fused else sum(
+        2 if rtq.plan(4 if proj_dims(p)[0] == "q4" else 8, M, *proj_dims(p)[1:])
+        in ("tc_x_resident", "tc_w_streamed") else 1 for p in projs)
     if rank == 0:
         line = {
             "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -417,7 +421,8 @@ def run_small_m(args, rank, world, local_rank):
                              f"X and Y fixed",
                        "parallelism": f"replicas{world}" if world > 1 else "single"},
             "tflops": world * flops / (ms * 1e-3) / 1e12,
-            "kernels": kernels, "clocks": clocks, "gpu_launches": args.steps * copies * len(projs),
+            "kernels": kernels, "block_launch": "grouped" if fused else "per projection",
+            "clocks": clocks, "gpu_launches": args.steps * copies * launches_per_copy,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm_gbs"], "traffic": None,
                          "algorithmic_bytes_per_step": wbytes, "peak_source": peaks["source"]},
@@ -576,11 +581,15 @@ def run_gpu(args, rank, world, local_rank):
                 if st:
                     raise rtq.RtqError(st, "rt_qgemm")
 
-    # the TMA-fed kernels add an activation pre-pass launch
-    launches_per_step = sum(
-        2 if rtq.plan(4 if proj_dims(name)[0] == "q4" else 8, M, *proj_dims(name)[1:])
-        in ("tc_x_resident", "tc_w_streamed") else 1
-        for name, _, _ in calls)
+    # the TMA-fed kernels add an activation pre-pass launch; the block driver
+    # runs a small-M block as one grouped launch
+    if full_block and rtq.block_fused(M, wl.D_MODEL, wl.D_FF) == 1:
+        launches_per_step = nblocks
+    else:
+        launches_per_step = sum(
+            2 if rtq.plan(4 if proj_dims(name)[0] == "q4" else 8, M, *proj_dims(name)[1:])
+            in ("tc_x_resident", "tc_w_streamed") else 1
+            for name, _, _ in calls)
 
     def barrier():
         if world > 1:

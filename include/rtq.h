@@ -189,9 +189,22 @@ rt_status rt_qgemm_noalloc(int fmt, const float *X, const void *Wq, const void *
  *   w13  : q4, N = 2*d_ff,    K = d_model  (rows w1 | w3)
  *   w2   : q8, N = d_model,   K = d_ff
  * All pointers are device pointers.  The four products are independent (each
- * reads its own input) and are enqueued on `stream` in the order qkvg, wo,
- * w13, w2.  Y_qkvg [M, 4*d_model], Y_o [M, d_model], Y_13 [M, 2*d_ff],
- * Y_2 [M, d_model].  The same validation as rt_qgemm_q4/q8 applies to each.
+ * reads its own input; two inputs may be the same buffer).  Y_qkvg
+ * [M, 4*d_model], Y_o [M, d_model], Y_13 [M, 2*d_ff], Y_2 [M, d_model].
+ *
+ * Launches: where all four products take RT_KERNEL_TC_W_STATIONARY with one
+ * activation tile (1 <= M <= 128 on a tensor-core path: RT_PATH_AUTO above
+ * the SIMT range, RT_PATH_TC, RT_PATH_TC_BF16), one grouped launch of that
+ * kernel computes all four: each CTA takes a 128-row weight tile of one of
+ * the projections, and K is split over a cluster by one factor for the
+ * whole group.  Otherwise the four run one after another on `stream` in the
+ * order qkvg, wo, w13, w2, each as rt_qgemm_q4/q8 would.
+ *
+ * Validation: each product as in rt_qgemm_q4/q8; in addition no output may
+ * overlap another projection's output, activations, codes or scales
+ * (RT_ERR_INVALID_ARG), since the products may run concurrently.  All four
+ * are checked before anything is enqueued, so an error status means nothing
+ * was launched.
  */
 typedef struct rt_qblock {
     const uint8_t *qkvg;   const uint16_t *qkvg_sm;
@@ -206,6 +219,11 @@ rt_status rt_qblock_project(const rt_qblock *blk, int64_t M,
                             const float *X_qkvg, const float *X_o, const float *X_ffn,
                             const float *X_w2, float *Y_qkvg, float *Y_o, float *Y_13,
                             float *Y_2, int path, void *stream);
+
+/* 1 if rt_qblock_project runs a block of these sizes as one grouped launch,
+ * 0 if it makes one call per projection, -1 if it rejects the sizes or path.
+ * Host-only; touches no device. */
+int rt_qblock_fused(int64_t M, int64_t d_model, int64_t d_ff, int path);
 
 /*
  * Host-side quantizers (HOST pointers, caller-allocated outputs, synchronous,

@@ -80,6 +80,8 @@ def lib() -> ctypes.CDLL:
     L.rt_qblock_project.restype = _i32
     L.rt_qblock_project.argtypes = [ctypes.POINTER(_QBlockC), _i64, _p, _p, _p, _p, _p, _p, _p,
                                     _p, _i32, _p]
+    L.rt_qblock_fused.restype = _i32
+    L.rt_qblock_fused.argtypes = [_i64, _i64, _i64, _i32]
     L.rt_quantize_q4_g32.restype = _i32
     L.rt_quantize_q4_g32.argtypes = [_p, _i64, _i64, _i32, _p, _p]
     L.rt_quantize_q8_row.restype = _i32
@@ -121,6 +123,10 @@ def rt_qblock_project(blk, M, X_qkvg, X_o, X_ffn, X_w2, Y_qkvg, Y_o, Y_13, Y_2, 
                       stream) -> int:
     return lib().rt_qblock_project(ctypes.byref(blk), M, X_qkvg, X_o, X_ffn, X_w2, Y_qkvg, Y_o,
                                    Y_13, Y_2, path, stream)
+
+
+def rt_qblock_fused(M, d_model, d_ff, path) -> int:
+    return lib().rt_qblock_fused(M, d_model, d_ff, path)
 
 
 def rt_quantize_q4_g32(W, N, K, n_grid, Wq, scale_min) -> int:
@@ -356,6 +362,12 @@ def plan(fmt: int, M: int, N: int, K: int, path="auto") -> str:
     """Name of the kernel a GEMM of this shape runs (see rt_qgemm_plan)."""
     k = int(rt_qgemm_plan(fmt, M, N, K, _path(path)))
     return KERNELS.get(k, "rejected")
+
+
+def block_fused(M: int, d_model: int, d_ff: int, path="auto") -> int:
+    """1 if rt_qblock_project runs the block as one grouped launch, 0 if one
+    call per projection, -1 if it rejects the sizes (see rt_qblock_fused)."""
+    return int(rt_qblock_fused(M, d_model, d_ff, _path(path)))
 
 
 def workspace_bytes(fmt: int, M: int, N: int, K: int, path="auto") -> int:

@@ -261,22 +261,76 @@ rt_status rt_workspace_release(void) {
     return RT_OK;
 }
 
+int rt_qblock_fused(int64_t M, int64_t d_model, int64_t d_ff, int path) {
+    if (d_model < 1 || d_ff < 1 || d_model > kMaxDim / 4 || d_ff > kMaxDim / 2) return -1;
+    const int64_t shapes[4][3] = {{4, 4 * d_model, d_model}, {8, d_model, d_model},
+                                  {4, 2 * d_ff, d_model}, {8, d_model, d_ff}};
+    bool fused = M >= 1 && M <= 128;
+    for (const auto &sh : shapes) {
+        const int kern = rt_qgemm_plan(static_cast<int>(sh[0]), M, sh[1], sh[2], path);
+        if (kern < 0) return -1;
+        fused = fused && kern == RT_KERNEL_TC_W_STATIONARY;
+    }
+    return fused ? 1 : 0;
+}
+
 rt_status rt_qblock_project(const rt_qblock *blk, int64_t M, const float *X_qkvg,
                             const float *X_o, const float *X_ffn, const float *X_w2,
                             float *Y_qkvg, float *Y_o, float *Y_13, float *Y_2, int path,
                             void *stream) {
     if (!blk || blk->d_model < 1 || blk->d_ff < 1) return RT_ERR_INVALID_ARG;
     const int64_t d = blk->d_model, f = blk->d_ff;
+    struct Proj {
+        int fmt;
+        const float *X;
+        const void *W, *S;
+        float *Y;
+        int64_t N, K;
+    };
+    const Proj p[4] = {{4, X_qkvg, blk->qkvg, blk->qkvg_sm, Y_qkvg, 4 * d, d},
+                       {8, X_o, blk->wo, blk->wo_s, Y_o, d, d},
+                       {4, X_ffn, blk->w13, blk->w13_sm, Y_13, 2 * f, d},
+                       {8, X_w2, blk->w2, blk->w2_s, Y_2, d, f}};
+    // Every projection is checked before any is enqueued.
     rt_status st;
-    if ((st = rt_qgemm_q4(X_qkvg, blk->qkvg, blk->qkvg_sm, Y_qkvg, M, 4 * d, d, path, stream)) !=
-        RT_OK)
-        return st;
-    if ((st = rt_qgemm_q8(X_o, blk->wo, blk->wo_s, Y_o, M, d, d, path, stream)) != RT_OK)
-        return st;
-    if ((st = rt_qgemm_q4(X_ffn, blk->w13, blk->w13_sm, Y_13, M, 2 * f, d, path, stream)) !=
-        RT_OK)
-        return st;
-    return rt_qgemm_q8(X_w2, blk->w2, blk->w2_s, Y_2, M, d, f, path, stream);
+    for (const Proj &q : p) {
+        if ((st = rtq::check_gemm_args(q.fmt, q.X, q.W, q.S, q.Y, M, q.N, q.K)) != RT_OK)
+            return st;
+        const int pp = pick_path(M, q.K, path);
+        if (pp == -1) return RT_ERR_UNSUPPORTED_SHAPE;
+        if (pp < 0) return RT_ERR_INVALID_ARG;
+    }
+    // The four products may run concurrently: no output may overlap another
+    // projection's output or inputs.
+    if (M > 0) {
+        for (int i = 0; i < 4; ++i) {
+            const int64_t yb = M * p[i].N * 4;
+            for (int j = 0; j < 4; ++j) {
+                if (j == i) continue;
+                const int64_t wb = p[j].fmt == 4 ? p[j].N * (p[j].K / 2) : p[j].N * p[j].K;
+                const int64_t sb = p[j].fmt == 4 ? p[j].N * (p[j].K / 32) * 4 : p[j].N * 4;
+                if (overlap(p[i].Y, yb, p[j].Y, M * p[j].N * 4) ||
+                    overlap(p[i].Y, yb, p[j].X, M * p[j].K * 4) || overlap(p[i].Y, yb, p[j].W, wb) ||
+                    overlap(p[i].Y, yb, p[j].S, sb))
+                    return RT_ERR_INVALID_ARG;
+            }
+        }
+    }
+    if (rt_qblock_fused(M, d, f, path) == 1) {
+        unsigned *status = nullptr;
+        if ((st = status_word(&status)) != RT_OK) return st;
+        rtq::GroupProblem g[4];
+        for (int i = 0; i < 4; ++i)
+            g[i] = {p[i].X, p[i].W, p[i].S, p[i].Y, static_cast<int>(p[i].N),
+                    static_cast<int>(p[i].K), p[i].fmt};
+        return from_cuda(rtq::launch_tc_group(g, 4, static_cast<int>(M),
+                                              pick_path(M, d, path) == RT_PATH_TC_BF16, status,
+                                              static_cast<cudaStream_t>(stream)));
+    }
+    for (const Proj &q : p)
+        if ((st = run_gemm(q.fmt, q.X, q.W, q.S, q.Y, M, q.N, q.K, path, stream)) != RT_OK)
+            return st;
+    return RT_OK;
 }
 
 static rt_status validate_dequant(const void *Wq, const void *S, const void *W, int64_t N,

@@ -20,6 +20,21 @@ cudaError_t launch_tc_q4(const float *X, const uint8_t *Wq, const uint16_t *SM, 
 cudaError_t launch_tc_q8(const float *X, const int8_t *Wq, const float *S, float *Y, int M, int N,
                          int K, bool bf16, unsigned *status, cudaStream_t s);
 
+// Up to kMaxGroup independent projections with the same M (1..128) in one
+// launch of the same tcgen05 tile code: X [M, K] fp32, Wq/S as for
+// rt_qgemm_q4 (fmt 4) or rt_qgemm_q8 (fmt 8), Y [M, N] fp32; K a multiple of
+// 64.  Arguments are validated by the caller.
+constexpr int kMaxGroup = 4;
+struct GroupProblem {
+    const float *X;
+    const void *Wq;
+    const void *S;
+    float *Y;
+    int N, K, fmt;
+};
+cudaError_t launch_tc_group(const GroupProblem *probs, int count, int M, bool bf16,
+                            unsigned *status, cudaStream_t s);
+
 // Activation pre-pass of the TMA-fed kernels (prep.cu): X fp32 [M, K] ->
 // 16-bit [M, K] in the operand chunk order, into Xh (M * K * 2 bytes).
 cudaError_t launch_cvt_x16(const float *X, void *Xh, int64_t M, int64_t K, bool bf16,

@@ -38,6 +38,12 @@
 //
 // Every mbarrier wait is bounded; a wait that gives up latches
 // RT_ERR_DEVICE_TIMEOUT in the device status word and the CTA winds down.
+//
+// The same tile code also runs as a grouped launch (tc_group_kernel): up to
+// four independent projections with one activation tile each, e.g. a block's
+// qkvg, wo, w13 and w2 at M = 80.  Each CTA takes a weight tile of one of
+// them, so the four dependency chains of load -> MMA -> reduction -> store
+// overlap in one launch instead of following one another.
 #include <algorithm>
 
 #include "dequant.cuh"
@@ -55,6 +61,8 @@ constexpr int kTcThreads = kConvThreads + 32;    // + MMA warp
 constexpr int kAStageBytes = kTileO * 128;       // 16 KB
 constexpr int kMaxSmem = 227 * 1024;
 constexpr int kTwoCtaSmem = 110 * 1024;          // budget that lets two CTAs share an SM
+constexpr int kSmemPerSm = 228 * 1024;           // shared memory of one SM
+constexpr int kSmemReserve = 1024;               // the runtime's reservation per CTA
 constexpr unsigned kStatusTimeout = 5u;          // RT_ERR_DEVICE_TIMEOUT
 
 __host__ __device__ inline int tc_stage_bytes(int bn) { return kAStageBytes + bn * 128; }
@@ -75,6 +83,20 @@ __host__ __device__ inline uint32_t tmem_cols_for(int bn) {
     uint32_t c = 32;
     while (c < static_cast<uint32_t>(bn)) c <<= 1;
     return c;
+}
+
+// Dynamic shared memory of a launch, raised where needed so that no more CTAs
+// fit on an SM than its 512 TMEM columns serve.  tcgen05.alloc blocks until
+// columns are free, and a CTA holding columns may wait in a cluster barrier
+// for a peer that is blocked in its allocation on another SM, so residency
+// must never ask for more columns than an SM has.  (Registers already hold
+// the kernel to two CTAs per SM; this keeps the guarantee independent of
+// register allocation.)
+inline int tc_launch_smem(int bn, int stages, int ksplit) {
+    const int need = tc_smem_bytes(bn, stages, ksplit);
+    const int max_ctas = 512 / static_cast<int>(tmem_cols_for(bn));
+    const int floor_bytes = kSmemPerSm / (max_ctas + 1) - kSmemReserve + 1;
+    return std::max(need, (floor_bytes + 127) / 128 * 128);
 }
 
 // Byte offset of 16-byte chunk `c` (0..7) of row `r` in a 128B-swizzled tile.
@@ -188,12 +210,14 @@ __device__ __forceinline__ void store_stage(const StageRegs<PIECES> &R, const Co
         if (c.rb0 + 16 * i < BN) sts_v2(sB + c.b_off0 + 2048u * i, x4_op<OP>(R.b[i]));
 }
 
+// One CTA's work: the output tile of weight rows [o0, o0 + 128) and
+// activation rows [m0, m0 + BN), over K slice blockIdx.z of `ksplit`.
 template <int FMT, Op16 OP, int PIECES>
-__global__ void __launch_bounds__(kTcThreads, 2)
-    tc_qgemm_kernel(const float *__restrict__ X, const void *__restrict__ Wq,
-                    const void *__restrict__ S, float *__restrict__ Y, int M, int N, int K,
-                    int BN, int stages, int ksplit, unsigned *status) {
-    extern __shared__ uint8_t smem_raw[];
+__device__ __forceinline__ void tc_tile(uint8_t *smem_raw, const float *__restrict__ X,
+                                        const void *__restrict__ Wq, const void *__restrict__ S,
+                                        float *__restrict__ Y, int M, int N, int K, int BN,
+                                        int stages, int ksplit, int o0, int m0,
+                                        unsigned *status) {
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *smem = smem_raw + (base - raw);
@@ -205,8 +229,6 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     const uint32_t tmem_cols = tmem_cols_for(BN);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int o0 = blockIdx.x * kTileO;
-    const int m0 = blockIdx.y * BN;
     // split K: CTA z of the cluster takes K steps [kz0, kz0 + nk)
     const int nk = K / kTileK / ksplit;
     const int kz0 = static_cast<int>(blockIdx.z) * nk;
@@ -402,6 +424,52 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     }
 }
 
+template <int FMT, Op16 OP, int PIECES>
+__global__ void __launch_bounds__(kTcThreads, 2)
+    tc_qgemm_kernel(const float *__restrict__ X, const void *__restrict__ Wq,
+                    const void *__restrict__ S, float *__restrict__ Y, int M, int N, int K,
+                    int BN, int stages, int ksplit, unsigned *status) {
+    extern __shared__ uint8_t smem_raw[];
+    tc_tile<FMT, OP, PIECES>(smem_raw, X, Wq, S, Y, M, N, K, BN, stages, ksplit,
+                             static_cast<int>(blockIdx.x) * kTileO,
+                             static_cast<int>(blockIdx.y) * BN, status);
+}
+
+// Several independent projections that share M (<= BN, one activation tile)
+// in one launch.  Problem i owns the CTAs whose blockIdx.x lies in
+// [tile0[i], tile0[i + 1]); each of them is a weight tile of that problem, so
+// every CTA of a split-K cluster (same x) works on the same problem.
+struct TcProblem {
+    const float *X;
+    const void *Wq;
+    const void *S;
+    float *Y;
+    int N, K, fmt, tile0;
+};
+
+struct TcGroup {
+    TcProblem p[kMaxGroup];
+    int count;
+};
+
+template <Op16 OP, int PIECES>
+__global__ void __launch_bounds__(kTcThreads, 2)
+    tc_group_kernel(const __grid_constant__ TcGroup g, int M, int BN, int stages, int ksplit,
+                    unsigned *status) {
+    extern __shared__ uint8_t smem_raw[];
+    const int bx = static_cast<int>(blockIdx.x);
+    int i = 0;
+    while (i + 1 < g.count && bx >= g.p[i + 1].tile0) ++i;
+    const TcProblem &p = g.p[i];
+    const int o0 = (bx - p.tile0) * kTileO;
+    if (p.fmt == 4)
+        tc_tile<4, OP, PIECES>(smem_raw, p.X, p.Wq, p.S, p.Y, M, p.N, p.K, BN, stages, ksplit,
+                               o0, 0, status);
+    else
+        tc_tile<8, OP, PIECES>(smem_raw, p.X, p.Wq, p.S, p.Y, M, p.N, p.K, BN, stages, ksplit,
+                               o0, 0, status);
+}
+
 // Activation rows per tile: one tile when M <= 128; otherwise 128, halved
 // (down to 64) while the grid would not give every SM one tile.  Each halving
 // doubles how often the weight tile is dequantized, so it stops early.
@@ -447,7 +515,7 @@ cudaError_t launch_tc_pieces(const float *X, const void *Wq, const void *S, floa
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((N + kTileO - 1) / kTileO, (M + BN - 1) / BN, ksplit);
     cfg.blockDim = dim3(kTcThreads, 1, 1);
-    cfg.dynamicSmemBytes = tc_smem_bytes(BN, stages, ksplit);
+    cfg.dynamicSmemBytes = tc_launch_smem(BN, stages, ksplit);
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -471,7 +539,82 @@ cudaError_t launch_tc(const float *X, const void *Wq, const void *S, float *Y, i
     return launch_tc_pieces<FMT, OP, 8>(X, Wq, S, Y, M, N, K, BN, status, st);
 }
 
+// K slices for a group: the single-problem rule applied to the group's
+// total tile count, with every problem's K step count divisible by the split.
+int pick_group_ksplit(const TcGroup &g, int total_tiles) {
+    int ks = 1;
+    while (ks < 8 && static_cast<long>(total_tiles) * ks * 2 <= 2 * 148) {
+        bool divides = true;
+        for (int i = 0; i < g.count; ++i) divides = divides && (g.p[i].K / kTileK) % (2 * ks) == 0;
+        if (!divides) break;
+        ks *= 2;
+    }
+    return ks;
+}
+
+template <Op16 OP, int PIECES>
+cudaError_t launch_group_pieces(const TcGroup &g, int total_tiles, int M, int BN,
+                                unsigned *status, cudaStream_t st) {
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 64 && !attr_set[dev]) {
+        e = cudaFuncSetAttribute(tc_group_kernel<OP, PIECES>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    const int ksplit = pick_group_ksplit(g, total_tiles);
+    int max_nk = 1;
+    for (int i = 0; i < g.count; ++i) max_nk = std::max(max_nk, g.p[i].K / kTileK / ksplit);
+    int stages = (kTwoCtaSmem - 1024 - 256) / tc_stage_bytes(BN);
+    stages = std::max(1, std::min({stages, 4, max_nk}));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(total_tiles), 1, static_cast<unsigned>(ksplit));
+    cfg.blockDim = dim3(kTcThreads, 1, 1);
+    cfg.dynamicSmemBytes = tc_launch_smem(BN, stages, ksplit);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 1;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = static_cast<unsigned>(ksplit);
+    cfg.attrs = attr;
+    cfg.numAttrs = ksplit > 1 ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, tc_group_kernel<OP, PIECES>, g, M, BN, stages, ksplit,
+                              status);
+}
+
+template <Op16 OP>
+cudaError_t launch_group(const TcGroup &g, int total_tiles, int M, unsigned *status,
+                         cudaStream_t st) {
+    const int BN = pick_bn(M, 0);
+    if (BN <= 32) return launch_group_pieces<OP, 2>(g, total_tiles, M, BN, status, st);
+    if (BN <= 64) return launch_group_pieces<OP, 4>(g, total_tiles, M, BN, status, st);
+    return launch_group_pieces<OP, 8>(g, total_tiles, M, BN, status, st);
+}
+
 }  // namespace
+
+cudaError_t launch_tc_group(const GroupProblem *probs, int count, int M, bool bf16,
+                            unsigned *status, cudaStream_t s) {
+    if (count < 1 || count > kMaxGroup || M < 1 || M > kTileO) return cudaErrorInvalidValue;
+    TcGroup g = {};
+    g.count = count;
+    int tiles = 0;
+    for (int i = 0; i < count; ++i) {
+        const GroupProblem &q = probs[i];
+        if ((q.fmt != 4 && q.fmt != 8) || q.N < 1 || q.K < kTileK || q.K % kTileK != 0)
+            return cudaErrorInvalidValue;
+        g.p[i] = {q.X, q.Wq, q.S, q.Y, q.N, q.K, q.fmt, tiles};
+        tiles += (q.N + kTileO - 1) / kTileO;
+    }
+    return bf16 ? launch_group<Op16::bf16>(g, tiles, M, status, s)
+                : launch_group<Op16::f16>(g, tiles, M, status, s);
+}
 
 cudaError_t launch_tc_q4(const float *X, const uint8_t *Wq, const uint16_t *SM, float *Y, int M,
                          int N, int K, bool bf16, unsigned *status, cudaStream_t s) {

@@ -139,6 +139,49 @@ def test_block_driver_validation():
     assert rtq.lib().rt_qblock_project(None, 4, X, X, X, X, Y, Y, Y, Y, 0, None) == INVALID
 
 
+def test_block_grouped_launch_plan():
+    # one grouped launch exactly where all four projections take the
+    # weight-stationary kernel with a single activation tile
+    assert rtq.block_fused(80, 512, 2048) == 1
+    assert rtq.block_fused(9, 512, 2048) == 1 and rtq.block_fused(128, 512, 2048) == 1
+    assert rtq.block_fused(8, 512, 2048) == 0             # AUTO takes SIMT at M <= 8
+    assert rtq.block_fused(8, 512, 2048, "tc") == 1
+    assert rtq.block_fused(1, 512, 2048, "tc_bf16") == 1
+    assert rtq.block_fused(129, 512, 2048) == 0           # the TMA-fed kernels
+    assert rtq.block_fused(80, 512, 2048, "simt") == 0
+    assert rtq.block_fused(0, 512, 2048) == 0
+    assert rtq.block_fused(80, 512, 2000) == 0            # w2's K % 64 != 0: SIMT under AUTO
+    assert rtq.block_fused(80, 512, 2000, "tc") == -1     # and rejected on forced TC
+    assert rtq.block_fused(80, 0, 2048) == -1
+    assert rtq.block_fused(80, 512, 2048, 9) == -1
+
+
+def test_block_driver_rejects_overlapping_outputs():
+    # distinct fake regions 16 MB apart: X_i at 0x1i000000, codes at 0x2i..,
+    # scales at 0x3i.., Y_i at 0x4i..; every status is decided before any
+    # CUDA call, and an error means nothing was enqueued
+    Xs = [0x11000000, 0x12000000, 0x13000000, 0x14000000]
+    Ws = [0x21000000, 0x22000000, 0x23000000, 0x24000000]
+    Ss = [0x31000000, 0x32000000, 0x33000000, 0x34000000]
+    Ys = [0x41000000, 0x42000000, 0x43000000, 0x44000000]
+    blk = rtq._QBlockC(Ws[0], Ss[0], Ws[1], Ss[1], Ws[2], Ss[2], Ws[3], Ss[3], 512, 2048)
+    f = rtq.rt_qblock_project
+
+    def call(M, xs, ys, path=0):
+        return f(blk, M, *xs, *ys, path, None)
+
+    assert call(0, Xs, Ys) == RT_OK                                   # M == 0: no-op
+    assert call(80, Xs, [Ys[0], Ys[1], Ys[0] + 4096, Ys[3]]) == INVALID  # Y_13 inside Y_qkvg
+    assert call(80, Xs, [Ys[0], Xs[2], Ys[2], Ys[3]]) == INVALID      # Y_o is w13's input
+    assert call(80, Xs, [Ys[0], Ys[1], Ys[2], Ws[0]]) == INVALID      # Y_2 on qkvg's codes
+    assert call(80, Xs, [Ys[0], Ys[1], Ss[1], Ys[3]]) == INVALID      # Y_13 on wo's scales
+    # the rule holds on the one-call-per-projection route too: at M = 4096,
+    # Y_qkvg (32 MB) runs into Y_o
+    assert rtq.block_fused(4096, 512, 2048) == 0
+    assert call(4096, Xs, Ys) == INVALID
+    assert call(80, Xs, Ys, path=9) == INVALID                        # unknown path
+
+
 def test_dequant_validation():
     assert rtq.rt_dequant_q4_f32(W, S, Y, 4, 40, None) == SHAPE
     assert rtq.rt_dequant_q4_f32(W + 1, S, Y, 4, 64, None) == ALIGN

@@ -422,6 +422,91 @@ def test_block_driver_matches_oracle(rtq_lib, M, n_check):
         assert rel_err(got, ref) <= tol, name
 
 
+def _sized_block(d_model, d_ff, M, seed):
+    """A seeded block of any size: weights ~ N(0, 0.02^2) quantized by the
+    oracle, activations ~ N(0, 1)."""
+    shapes = {"qkvg": ("q4", 4 * d_model, d_model), "wo": ("q8", d_model, d_model),
+              "w13": ("q4", 2 * d_ff, d_model), "w2": ("q8", d_model, d_ff)}
+    host = {}
+    for i, (name, (fmt, N, K)) in enumerate(shapes.items()):
+        W = wl.weights(N, K, seed + i)
+        host[name] = oracle.quant_q4_g32(W) if fmt == "q4" else oracle.quant_q8_row(W)
+        host["x_" + name] = wl.activations(M, K, seed + 10 + i)
+    return host, shapes
+
+
+def _guarded_outputs(M, shapes, guard=64):
+    """The four Y buffers as views of one NaN-filled allocation, separated by
+    `guard` floats that the kernels must not write."""
+    sizes = [M * shapes[n][1] for n in ("qkvg", "wo", "w13", "w2")]
+    flat = torch.full((sum(sizes) + 5 * guard,), float("nan"), device="cuda")
+    views, off = {}, guard
+    for n, sz in zip(("qkvg", "wo", "w13", "w2"), sizes):
+        views[n] = flat[off:off + sz].view(M, shapes[n][1])
+        off += sz + guard
+    return flat, views, sizes
+
+
+# (M, d_model, d_ff, path): the weight tiles of the four projections and the
+# common split-K factor the grouped launch picks for them are in the comments
+FUSED_CASES = [
+    (80, 512, 2048, "auto"),      # RT-J block at the small-M config: 56 tiles, K split by 4
+    (16, 512, 2048, "auto"),      # 16-column activation tile
+    (48, 512, 2048, "auto"),
+    (128, 512, 2048, "auto"),     # largest single activation tile
+    (1, 512, 2048, "tc"),         # one row, tensor cores forced
+    (80, 512, 2048, "tc_bf16"),
+    (100, 256, 1024, "auto"),     # 28 tiles, K split by 4 (one step per CTA at K = 256)
+    (37, 1024, 4096, "auto"),     # 112 tiles, K split by 2
+    (16, 2048, 8192, "auto"),     # 224 tiles, no split: 128 K steps per w2 CTA
+]
+
+
+@pytest.mark.parametrize("M,d_model,d_ff,path", FUSED_CASES)
+def test_block_driver_grouped_launch_matches_oracle(rtq_lib, M, d_model, d_ff, path):
+    """rt_qblock_project at M <= 128 runs the four projections as one grouped
+    tcgen05 launch; every output element against the oracle, nothing written
+    outside the outputs, and a repeat gives the same bits."""
+    assert rtq_lib.block_fused(M, d_model, d_ff, path) == 1
+    h, shapes = _sized_block(d_model, d_ff, M, seed=1000 + M + d_model)
+    blk = rtq_lib.QBlock(*(dev(a) for a in (*h["qkvg"], *h["wo"], *h["w13"], *h["w2"])),
+                         d_model=d_model, d_ff=d_ff)
+    X = {n: dev(h["x_" + n]) for n in ("qkvg", "wo", "w13", "w2")}
+    flat, Y, sizes = _guarded_outputs(M, shapes)
+    rtq_lib.qblock_project(blk, X["qkvg"], X["wo"], X["w13"], X["w2"],
+                           Y["qkvg"], Y["wo"], Y["w13"], Y["w2"], path=path)
+    first = {n: Y[n].cpu().numpy().copy() for n in Y}
+    for n in ("qkvg", "wo", "w13", "w2"):
+        gemm = oracle.gemm_q4 if shapes[n][0] == "q4" else oracle.gemm_q8
+        ref = gemm(h["x_" + n], *h[n])
+        assert rel_err(first[n], ref) <= MAX_REL[path], n
+    guard = torch.ones_like(flat, dtype=torch.bool)
+    off = 64
+    for sz in sizes:
+        guard[off:off + sz] = False
+        off += sz + 64
+    assert torch.isnan(flat[guard]).all()
+    rtq_lib.qblock_project(blk, X["qkvg"], X["wo"], X["w13"], X["w2"],
+                           Y["qkvg"], Y["wo"], Y["w13"], Y["w2"], path=path)
+    for n in Y:
+        assert np.array_equal(Y[n].cpu().numpy(), first[n]), n
+
+
+def test_block_driver_grouped_launch_shared_input(rtq_lib):
+    """qkvg, wo and w13 read one activation buffer (allowed: inputs are only
+    read) in the grouped launch."""
+    M = 64
+    h, shapes = _sized_block(512, 2048, M, seed=77)
+    Xs = dev(h["x_qkvg"])
+    blk = rtq_lib.QBlock(*(dev(a) for a in (*h["qkvg"], *h["wo"], *h["w13"], *h["w2"])))
+    Y = {n: torch.empty((M, shapes[n][1]), device="cuda") for n in shapes}
+    rtq_lib.qblock_project(blk, Xs, Xs, Xs, dev(h["x_w2"]), Y["qkvg"], Y["wo"], Y["w13"], Y["w2"])
+    for n in ("qkvg", "wo", "w13"):
+        gemm = oracle.gemm_q4 if shapes[n][0] == "q4" else oracle.gemm_q8
+        assert rel_err(Y[n].cpu().numpy(), gemm(h["x_qkvg"], *h[n])) <= TC_TOL, n
+    assert rel_err(Y["w2"].cpu().numpy(), oracle.gemm_q8(h["x_w2"], *h["w2"])) <= TC_TOL
+
+
 def test_device_status_clear(rtq_lib):
     torch.cuda.synchronize()
     assert rtq_lib.device_status() == 0
