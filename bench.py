@@ -583,7 +583,8 @@ def run_gpu(args, rank, world, local_rank):
 
     # the TMA-fed kernels add an activation pre-pass launch; the block driver
     # runs a small-M block as one grouped launch
-    if full_block and rtq.block_fused(M, wl.D_MODEL, wl.D_FF) == 1:
+    fused_block = full_block and rtq.block_fused(M, wl.D_MODEL, wl.D_FF) == 1
+    if fused_block:
         launches_per_step = nblocks
     else:
         launches_per_step = sum(
@@ -632,10 +633,22 @@ def run_gpu(args, rank, world, local_rank):
     ms_total = max_over_ranks(e0.elapsed_time(e1))
     ms_per_step = ms_total / args.steps
 
-    # ---- per-kernel durations: every launch bracketed by events, K steps
-    evs = {name: [] for name in projs}
+    # ---- per-kernel durations: every launch bracketed by events, K steps.
+    # A block run as one grouped launch is timed as that launch.
+    evs = {"block": []} if fused_block else {name: [] for name in projs}
     with torch.cuda.stream(stream):
         for _ in range(args.steps):
+            if fused_block:
+                for c, ptrs in block_args:
+                    s0 = torch.cuda.Event(enable_timing=True)
+                    s1 = torch.cuda.Event(enable_timing=True)
+                    s0.record(stream)
+                    st = L.rt_qblock_project(ctypes.byref(c), M, *ptrs, 0, sptr)
+                    s1.record(stream)
+                    if st:
+                        raise rtq.RtqError(st, "rt_qblock_project")
+                    evs["block"].append((s0, s1))
+                continue
             for name, fn, a in calls:
                 s0 = torch.cuda.Event(enable_timing=True)
                 s1 = torch.cuda.Event(enable_timing=True)
@@ -657,15 +670,23 @@ def run_gpu(args, rank, world, local_rank):
 
     # ---- roofline of the dominant kernel
     peaks = load_peaks()
-    share = {n: kern_us[n] * nblocks for n in projs}
-    dom = max(share, key=share.get)
-    fmt, N, K = proj_dims(dom)
-    path = "tc" if rtq.auto_path(4 if fmt == "q4" else 8, M, N, K) == 2 else "simt"
+    if fused_block:
+        # one launch per block: its bytes and flops are the four projections'
+        share = {"block": kern_us["block"] * nblocks}
+        dom, path = "block", "tc"
+        b_alg = sum(proj_bytes(p, M) for p in projs)
+        f_alg = sum(proj_flops(p, M) for p in projs)
+        kernel_key = f"block_grouped_tc_M{M}"
+    else:
+        share = {n: kern_us[n] * nblocks for n in projs}
+        dom = max(share, key=share.get)
+        fmt, N, K = proj_dims(dom)
+        path = "tc" if rtq.auto_path(4 if fmt == "q4" else 8, M, N, K) == 2 else "simt"
+        b_alg, f_alg = proj_bytes(dom, M), proj_flops(dom, M)
+        kernel_key = f"{dom}_{fmt}_{path}_M{M}"
     t_s = kern_us[dom] * 1e-6
-    b_alg, f_alg = proj_bytes(dom, M), proj_flops(dom, M)
     t_hbm = b_alg / (peaks["hbm_gbs"] * 1e9)
     t_tc = f_alg / (peaks["bf16_tflops_sustained"] * 1e12)
-    kernel_key = f"{dom}_{fmt}_{path}_M{M}"
     traffic = recorded_traffic(kernel_key)
     if t_hbm >= t_tc or path == "simt":
         roof = {"bound": "hbm", "achieved": b_alg / t_s / 1e9, "peak": peaks["hbm_gbs"],
