@@ -196,9 +196,11 @@ rt_status rt_qgemm_noalloc(int fmt, const float *X, const void *Wq, const void *
  * activation tile (1 <= M <= 128 on a tensor-core path: RT_PATH_AUTO above
  * the SIMT range, RT_PATH_TC, RT_PATH_TC_BF16), one grouped launch of that
  * kernel computes all four: each CTA takes a 128-row weight tile of one of
- * the projections, and K is split over a cluster by one factor for the
- * whole group.  Otherwise the four run one after another on `stream` in the
- * order qkvg, wo, w13, w2, each as rt_qgemm_q4/q8 would.
+ * the projections and a slice of its K; each projection splits K by its own
+ * factor (so w2, with four times the K of the others, splits four times as
+ * far) and reduces the slices in distributed shared memory in a fixed order.
+ * Otherwise the four run one after another on `stream` in the order qkvg,
+ * wo, w13, w2, each as rt_qgemm_q4/q8 would.
  *
  * Validation: each product as in rt_qgemm_q4/q8; in addition no output may
  * overlap another projection's output, activations, codes or scales

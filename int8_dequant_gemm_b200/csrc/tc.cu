@@ -211,13 +211,17 @@ __device__ __forceinline__ void store_stage(const StageRegs<PIECES> &R, const Co
 }
 
 // One CTA's work: the output tile of weight rows [o0, o0 + 128) and
-// activation rows [m0, m0 + BN), over K slice blockIdx.z of `ksplit`.
+// activation rows [m0, m0 + BN), over K slice `kslice` of `ksplit`.  With
+// ksplit > 1 the tile's slices are the cluster's CTAs of ranks
+// [kbase, kbase + ksplit), which reduce their partial sums among themselves;
+// every CTA of the cluster must have the same ksplit (each reaches the
+// cluster barriers exactly when ksplit > 1).
 template <int FMT, Op16 OP, int PIECES>
 __device__ __forceinline__ void tc_tile(uint8_t *smem_raw, const float *__restrict__ X,
                                         const void *__restrict__ Wq, const void *__restrict__ S,
                                         float *__restrict__ Y, int M, int N, int K, int BN,
-                                        int stages, int ksplit, int o0, int m0,
-                                        unsigned *status) {
+                                        int stages, int ksplit, int o0, int m0, int kslice,
+                                        int kbase, unsigned *status) {
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *smem = smem_raw + (base - raw);
@@ -229,9 +233,9 @@ __device__ __forceinline__ void tc_tile(uint8_t *smem_raw, const float *__restri
     const uint32_t tmem_cols = tmem_cols_for(BN);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // split K: CTA z of the cluster takes K steps [kz0, kz0 + nk)
+    // split K: slice `kslice` takes K steps [kz0, kz0 + nk)
     const int nk = K / kTileK / ksplit;
-    const int kz0 = static_cast<int>(blockIdx.z) * nk;
+    const int kz0 = kslice * nk;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
@@ -382,17 +386,18 @@ __device__ __forceinline__ void tc_tile(uint8_t *smem_raw, const float *__restri
         // together, so neither barrier can hang.
         cluster_sync();                       // all partials written
         if (warp < kConvWarps) {
-            // CTA rank r sums columns [r * BN/ksplit, (r + 1) * BN/ksplit) over
-            // the cluster's partials in rank order (deterministic) and stores Y.
+            // Slice s sums columns [s * BN/ksplit, (s + 1) * BN/ksplit) over
+            // the tile's partials in rank order (deterministic) and stores Y.
             const int cols = BN / ksplit;
-            const int mbeg = static_cast<int>(cluster_ctarank()) * cols;
+            const int mbeg = kslice * cols;
             for (int idx = threadIdx.x; idx < cols * (kTileO / 4); idx += kConvThreads) {
                 const int ml = mbeg + idx / (kTileO / 4), o4 = idx % (kTileO / 4);
                 const int m = m0 + ml, o = o0 + 4 * o4;
                 const uint32_t off = base + static_cast<uint32_t>((ml * kTileO + 4 * o4) * 4);
-                float4 acc = ld_cluster_f4(cluster_map(off, 0));
+                float4 acc = ld_cluster_f4(cluster_map(off, static_cast<uint32_t>(kbase)));
                 for (int r = 1; r < ksplit; ++r) {
-                    const float4 v = ld_cluster_f4(cluster_map(off, static_cast<uint32_t>(r)));
+                    const float4 v =
+                        ld_cluster_f4(cluster_map(off, static_cast<uint32_t>(kbase + r)));
                     acc.x += v.x;
                     acc.y += v.y;
                     acc.z += v.z;
@@ -432,19 +437,24 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     extern __shared__ uint8_t smem_raw[];
     tc_tile<FMT, OP, PIECES>(smem_raw, X, Wq, S, Y, M, N, K, BN, stages, ksplit,
                              static_cast<int>(blockIdx.x) * kTileO,
-                             static_cast<int>(blockIdx.y) * BN, status);
+                             static_cast<int>(blockIdx.y) * BN, static_cast<int>(blockIdx.z), 0,
+                             status);
 }
 
 // Several independent projections that share M (<= BN, one activation tile)
-// in one launch.  Problem i owns the CTAs whose blockIdx.x lies in
-// [tile0[i], tile0[i + 1]); each of them is a weight tile of that problem, so
-// every CTA of a split-K cluster (same x) works on the same problem.
+// in one launch.  The launch's clusters have `csize` CTAs along z; problem i
+// owns the clusters whose blockIdx.x lies in [cl0[i], cl0[i + 1]) and splits K
+// by its own factor ks (a divisor of csize), so one cluster holds csize / ks of
+// its 128-row weight tiles: CTA rank r works on tile r / ks of the cluster's
+// run, K slice r % ks.  Every CTA of a cluster belongs to one problem.  Tiles
+// past the problem's last one (a partly filled last cluster) compute zeros
+// and store nothing.
 struct TcProblem {
     const float *X;
     const void *Wq;
     const void *S;
     float *Y;
-    int N, K, fmt, tile0;
+    int N, K, fmt, cl0, ks;
 };
 
 struct TcGroup {
@@ -454,20 +464,23 @@ struct TcGroup {
 
 template <Op16 OP, int PIECES>
 __global__ void __launch_bounds__(kTcThreads, 2)
-    tc_group_kernel(const __grid_constant__ TcGroup g, int M, int BN, int stages, int ksplit,
+    tc_group_kernel(const __grid_constant__ TcGroup g, int M, int BN, int stages, int csize,
                     unsigned *status) {
     extern __shared__ uint8_t smem_raw[];
     const int bx = static_cast<int>(blockIdx.x);
     int i = 0;
-    while (i + 1 < g.count && bx >= g.p[i + 1].tile0) ++i;
+    while (i + 1 < g.count && bx >= g.p[i + 1].cl0) ++i;
     const TcProblem &p = g.p[i];
-    const int o0 = (bx - p.tile0) * kTileO;
+    const int r = static_cast<int>(blockIdx.z);          // rank in the cluster
+    const int tile = (bx - p.cl0) * (csize / p.ks) + r / p.ks;
+    const int o0 = tile * kTileO;
+    const int kslice = r % p.ks, kbase = r - kslice;
     if (p.fmt == 4)
-        tc_tile<4, OP, PIECES>(smem_raw, p.X, p.Wq, p.S, p.Y, M, p.N, p.K, BN, stages, ksplit,
-                               o0, 0, status);
+        tc_tile<4, OP, PIECES>(smem_raw, p.X, p.Wq, p.S, p.Y, M, p.N, p.K, BN, stages, p.ks, o0,
+                               0, kslice, kbase, status);
     else
-        tc_tile<8, OP, PIECES>(smem_raw, p.X, p.Wq, p.S, p.Y, M, p.N, p.K, BN, stages, ksplit,
-                               o0, 0, status);
+        tc_tile<8, OP, PIECES>(smem_raw, p.X, p.Wq, p.S, p.Y, M, p.N, p.K, BN, stages, p.ks, o0,
+                               0, kslice, kbase, status);
 }
 
 // Activation rows per tile: one tile when M <= 128; otherwise 128, halved
@@ -539,22 +552,42 @@ cudaError_t launch_tc(const float *X, const void *Wq, const void *S, float *Y, i
     return launch_tc_pieces<FMT, OP, 8>(X, Wq, S, Y, M, N, K, BN, status, st);
 }
 
-// K slices for a group: the single-problem rule applied to the group's
-// total tile count, with every problem's K step count divisible by the split.
-int pick_group_ksplit(const TcGroup &g, int total_tiles) {
-    int ks = 1;
-    while (ks < 8 && static_cast<long>(total_tiles) * ks * 2 <= 2 * 148) {
-        bool divides = true;
-        for (int i = 0; i < g.count; ++i) divides = divides && (g.p[i].K / kTileK) % (2 * ks) == 0;
-        if (!divides) break;
-        ks *= 2;
+// K splits for a group.  A launch lasts as long as its longest chain of K
+// steps, and the projections' K differ (the RT-J block has 8 K steps in qkvg,
+// wo and w13 but 32 in w2), so each projection gets its own split: the
+// smallest power of two (up to 8, dividing its step count) that brings it to
+// at most T steps per CTA.  T starts at the longest projection's steps / 8 and
+// doubles until the launch fits one wave of two CTAs per SM.  The cluster size
+// is the largest split.  Fills g.p[i].ks and .cl0; returns the cluster size
+// and the cluster count in *nclusters.
+int plan_group(TcGroup &g, int *nclusters) {
+    int max_nk = 1;
+    for (int i = 0; i < g.count; ++i) max_nk = std::max(max_nk, g.p[i].K / kTileK);
+    for (int T = std::max(1, (max_nk + 7) / 8);; T *= 2) {
+        int csize = 1;
+        for (int i = 0; i < g.count; ++i) {
+            const int nk = g.p[i].K / kTileK;
+            int ks = 1;
+            while (ks < 8 && nk / ks > T && nk % (2 * ks) == 0) ks *= 2;
+            g.p[i].ks = ks;
+            csize = std::max(csize, ks);
+        }
+        int clusters = 0;
+        for (int i = 0; i < g.count; ++i) {
+            const int per = csize / g.p[i].ks;        // weight tiles per cluster
+            const int tiles = (g.p[i].N + kTileO - 1) / kTileO;
+            g.p[i].cl0 = clusters;
+            clusters += (tiles + per - 1) / per;
+        }
+        if (static_cast<long>(clusters) * csize <= 2 * 148 || T >= max_nk) {
+            *nclusters = clusters;
+            return csize;
+        }
     }
-    return ks;
 }
 
 template <Op16 OP, int PIECES>
-cudaError_t launch_group_pieces(const TcGroup &g, int total_tiles, int M, int BN,
-                                unsigned *status, cudaStream_t st) {
+cudaError_t launch_group_pieces(TcGroup g, int M, int BN, unsigned *status, cudaStream_t st) {
     static bool attr_set[64] = {false};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -565,15 +598,17 @@ cudaError_t launch_group_pieces(const TcGroup &g, int total_tiles, int M, int BN
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    const int ksplit = pick_group_ksplit(g, total_tiles);
+    int nclusters = 0;
+    const int csize = plan_group(g, &nclusters);
     int max_nk = 1;
-    for (int i = 0; i < g.count; ++i) max_nk = std::max(max_nk, g.p[i].K / kTileK / ksplit);
+    for (int i = 0; i < g.count; ++i) max_nk = std::max(max_nk, g.p[i].K / kTileK / g.p[i].ks);
     int stages = (kTwoCtaSmem - 1024 - 256) / tc_stage_bytes(BN);
     stages = std::max(1, std::min({stages, 4, max_nk}));
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(total_tiles), 1, static_cast<unsigned>(ksplit));
+    cfg.gridDim = dim3(static_cast<unsigned>(nclusters), 1, static_cast<unsigned>(csize));
     cfg.blockDim = dim3(kTcThreads, 1, 1);
-    cfg.dynamicSmemBytes = tc_launch_smem(BN, stages, ksplit);
+    // the partial-sum region is sized whenever some projection splits K
+    cfg.dynamicSmemBytes = tc_launch_smem(BN, stages, csize);
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -581,20 +616,19 @@ cudaError_t launch_group_pieces(const TcGroup &g, int total_tiles, int M, int BN
     attr[1].id = cudaLaunchAttributeClusterDimension;
     attr[1].val.clusterDim.x = 1;
     attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = static_cast<unsigned>(ksplit);
+    attr[1].val.clusterDim.z = static_cast<unsigned>(csize);
     cfg.attrs = attr;
-    cfg.numAttrs = ksplit > 1 ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, tc_group_kernel<OP, PIECES>, g, M, BN, stages, ksplit,
+    cfg.numAttrs = csize > 1 ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, tc_group_kernel<OP, PIECES>, g, M, BN, stages, csize,
                               status);
 }
 
 template <Op16 OP>
-cudaError_t launch_group(const TcGroup &g, int total_tiles, int M, unsigned *status,
-                         cudaStream_t st) {
+cudaError_t launch_group(const TcGroup &g, int M, unsigned *status, cudaStream_t st) {
     const int BN = pick_bn(M, 0);
-    if (BN <= 32) return launch_group_pieces<OP, 2>(g, total_tiles, M, BN, status, st);
-    if (BN <= 64) return launch_group_pieces<OP, 4>(g, total_tiles, M, BN, status, st);
-    return launch_group_pieces<OP, 8>(g, total_tiles, M, BN, status, st);
+    if (BN <= 32) return launch_group_pieces<OP, 2>(g, M, BN, status, st);
+    if (BN <= 64) return launch_group_pieces<OP, 4>(g, M, BN, status, st);
+    return launch_group_pieces<OP, 8>(g, M, BN, status, st);
 }
 
 }  // namespace
@@ -604,16 +638,14 @@ cudaError_t launch_tc_group(const GroupProblem *probs, int count, int M, bool bf
     if (count < 1 || count > kMaxGroup || M < 1 || M > kTileO) return cudaErrorInvalidValue;
     TcGroup g = {};
     g.count = count;
-    int tiles = 0;
     for (int i = 0; i < count; ++i) {
         const GroupProblem &q = probs[i];
         if ((q.fmt != 4 && q.fmt != 8) || q.N < 1 || q.K < kTileK || q.K % kTileK != 0)
             return cudaErrorInvalidValue;
-        g.p[i] = {q.X, q.Wq, q.S, q.Y, q.N, q.K, q.fmt, tiles};
-        tiles += (q.N + kTileO - 1) / kTileO;
+        g.p[i] = {q.X, q.Wq, q.S, q.Y, q.N, q.K, q.fmt, 0, 1};
     }
-    return bf16 ? launch_group<Op16::bf16>(g, tiles, M, status, s)
-                : launch_group<Op16::f16>(g, tiles, M, status, s);
+    return bf16 ? launch_group<Op16::bf16>(g, M, status, s)
+                : launch_group<Op16::f16>(g, M, status, s);
 }
 
 cudaError_t launch_tc_q4(const float *X, const uint8_t *Wq, const uint16_t *SM, float *Y, int M,

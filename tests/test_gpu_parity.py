@@ -447,18 +447,19 @@ def _guarded_outputs(M, shapes, guard=64):
     return flat, views, sizes
 
 
-# (M, d_model, d_ff, path): the weight tiles of the four projections and the
-# common split-K factor the grouped launch picks for them are in the comments
+# (M, d_model, d_ff, path).  The grouped launch splits each projection's K by
+# its own factor inside clusters of a common size; the comments give the plan.
 FUSED_CASES = [
-    (80, 512, 2048, "auto"),      # RT-J block at the small-M config: 56 tiles, K split by 4
+    (80, 512, 2048, "auto"),      # RT-J block at the small-M config: qkvg, wo, w13 split by 2
+                                  # (4 tiles per cluster of 8), w2 by 8; 136 CTAs of 4 K steps
     (16, 512, 2048, "auto"),      # 16-column activation tile
     (48, 512, 2048, "auto"),
     (128, 512, 2048, "auto"),     # largest single activation tile
     (1, 512, 2048, "tc"),         # one row, tensor cores forced
     (80, 512, 2048, "tc_bf16"),
-    (100, 256, 1024, "auto"),     # 28 tiles, K split by 4 (one step per CTA at K = 256)
-    (37, 1024, 4096, "auto"),     # 112 tiles, K split by 2
-    (16, 2048, 8192, "auto"),     # 224 tiles, no split: 128 K steps per w2 CTA
+    (100, 256, 1024, "auto"),     # wo's 2 tiles half-fill a cluster: 2 CTA pairs store nothing
+    (37, 1024, 4096, "auto"),     # 272 CTAs of 8 K steps
+    (16, 2048, 8192, "auto"),     # clusters of 4: w2 split by 4, the others unsplit
 ]
 
 
