@@ -21,6 +21,7 @@ __all__ = [
     "RtqError", "lib", "PATHS", "OK", "qgemm_q4", "qgemm_q8", "qblock_project", "QBlock",
     "quantize_q4_g32", "quantize_q8_row", "dequant_q4_f32", "dequant_q8_f32",
     "dequant_q4_bf16", "dequant_q4_f16", "device_status", "auto_path", "status_string",
+    "qgemm_noalloc", "plan", "block_fused", "workspace_bytes",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -200,11 +201,38 @@ def _path(path) -> int:
     return PATHS[path] if isinstance(path, str) else int(path)
 
 
+def _shape(t, shape, name):
+    """The C layer sees only pointers and sizes, so a tensor whose shape does
+    not match the sizes would be read or written out of bounds: reject it."""
+    got = tuple(t.shape)
+    if got != tuple(shape):
+        raise ValueError(f"{name} has shape {got}, expected {tuple(shape)}")
+
+
+def _packed_shapes(fmt: int, N: int, K: int):
+    """Shapes of the codes and the scales of an N x K weight in format q4 / q8."""
+    if fmt == 4:
+        return (N, K // 2), (N, K // 32, 2)
+    return (N, K), (N,)
+
+
+def _check_gemm_shapes(fmt, X, Wq, scales, Y):
+    if X.dim() != 2:
+        raise ValueError(f"X must be 2-D [M, K], got shape {tuple(X.shape)}")
+    M, K = X.shape
+    N = Wq.shape[0]
+    wshape, sshape = _packed_shapes(fmt, N, K)
+    _shape(Wq, wshape, "Wq")
+    _shape(scales, sshape, "scale_min" if fmt == 4 else "scale")
+    if Y is not None:
+        _shape(Y, (M, N), "Y")
+    return M, N, K
+
+
 def qgemm_q4(X, Wq, scale_min, Y=None, path="auto", stream=None):
     """Y[M,N] = X[M,K] @ dequant_q4(Wq[N,K/2], scale_min[N,K/32,2])^T on the GPU."""
     import torch
-    M, K = X.shape
-    N = Wq.shape[0]
+    M, N, K = _check_gemm_shapes(4, X, Wq, scale_min, Y)
     if Y is None:
         Y = torch.empty((M, N), dtype=torch.float32, device=X.device)
     st = rt_qgemm_q4(_dev(X, torch.float32, "X"), _dev(Wq, torch.uint8, "Wq"),
@@ -217,8 +245,7 @@ def qgemm_q4(X, Wq, scale_min, Y=None, path="auto", stream=None):
 def qgemm_q8(X, Wq, scale, Y=None, path="auto", stream=None):
     """Y[M,N] = X[M,K] @ (Wq[N,K] * scale[N,None])^T on the GPU."""
     import torch
-    M, K = X.shape
-    N = Wq.shape[0]
+    M, N, K = _check_gemm_shapes(8, X, Wq, scale, Y)
     if Y is None:
         Y = torch.empty((M, N), dtype=torch.float32, device=X.device)
     st = rt_qgemm_q8(_dev(X, torch.float32, "X"), _dev(Wq, torch.int8, "Wq"),
@@ -232,8 +259,9 @@ def qgemm_noalloc(fmt, X, Wq, scales, Y, path="auto", stream=None):
     """rt_qgemm_q4 (fmt 4) or rt_qgemm_q8 (fmt 8) into a caller-given Y, with the
     activation scratch in the library's fixed device array: no allocation."""
     import torch
-    M, K = X.shape
-    N = Wq.shape[0]
+    if fmt not in (4, 8):
+        raise ValueError(f"fmt must be 4 or 8, got {fmt}")
+    M, N, K = _check_gemm_shapes(fmt, X, Wq, scales, Y)
     wdt, sdt = (torch.uint8, torch.uint16) if fmt == 4 else (torch.int8, torch.float32)
     st = rt_qgemm_noalloc(fmt, _dev(X, torch.float32, "X"), _dev(Wq, wdt, "Wq"),
                           _dev(scales, sdt, "scales"), _dev(Y, torch.float32, "Y"),
@@ -258,6 +286,13 @@ class QBlock:
 
     def as_c(self) -> _QBlockC:
         import torch
+        d, f = self.d_model, self.d_ff
+        for (name, fmt, N, K) in (("qkvg", 4, 4 * d, d), ("wo", 8, d, d), ("w13", 4, 2 * f, d),
+                                  ("w2", 8, d, f)):
+            wshape, sshape = _packed_shapes(fmt, N, K)
+            _shape(getattr(self, name), wshape, name)
+            sname = name + ("_sm" if fmt == 4 else "_s")
+            _shape(getattr(self, sname), sshape, sname)
         return _QBlockC(_dev(self.qkvg, torch.uint8, "qkvg"),
                         _dev(self.qkvg_sm, torch.uint16, "qkvg_sm"),
                         _dev(self.wo, torch.int8, "wo"), _dev(self.wo_s, torch.float32, "wo_s"),
@@ -272,6 +307,12 @@ def qblock_project(block: QBlock, X_qkvg, X_o, X_ffn, X_w2, Y_qkvg, Y_o, Y_13, Y
     """Runs one block's four quantized projections (qkvg, wo, w13, w2)."""
     import torch
     M = X_qkvg.shape[0]
+    d, f = block.d_model, block.d_ff
+    for t, shape, name in ((X_qkvg, (M, d), "X_qkvg"), (X_o, (M, d), "X_o"),
+                           (X_ffn, (M, d), "X_ffn"), (X_w2, (M, f), "X_w2"),
+                           (Y_qkvg, (M, 4 * d), "Y_qkvg"), (Y_o, (M, d), "Y_o"),
+                           (Y_13, (M, 2 * f), "Y_13"), (Y_2, (M, d), "Y_2")):
+        _shape(t, shape, name)
     bc = block_c if block_c is not None else block.as_c()
     args = [_dev(t, torch.float32, n) for t, n in
             ((X_qkvg, "X_qkvg"), (X_o, "X_o"), (X_ffn, "X_ffn"), (X_w2, "X_w2"),
@@ -305,6 +346,7 @@ def quantize_q8_row(W: np.ndarray):
 def dequant_q4_f32(Wq, scale_min, stream=None):
     import torch
     N, K2 = Wq.shape
+    _shape(scale_min, _packed_shapes(4, N, 2 * K2)[1], "scale_min")
     out = torch.empty((N, 2 * K2), dtype=torch.float32, device=Wq.device)
     st = rt_dequant_q4_f32(_dev(Wq, torch.uint8, "Wq"), _dev(scale_min, torch.uint16, "scale_min"),
                            _dev(out, torch.float32, "W_out"), N, 2 * K2, _stream_ptr(stream))
@@ -316,6 +358,7 @@ def dequant_q4_bf16(Wq, scale_min, stream=None):
     """bf16 rendering of the q4 weights as uint16 bits [N, K]."""
     import torch
     N, K2 = Wq.shape
+    _shape(scale_min, _packed_shapes(4, N, 2 * K2)[1], "scale_min")
     out = torch.empty((N, 2 * K2), dtype=torch.uint16, device=Wq.device)
     st = rt_dequant_q4_bf16(_dev(Wq, torch.uint8, "Wq"), _dev(scale_min, torch.uint16, "scale_min"),
                             _dev(out, torch.uint16, "W_out"), N, 2 * K2, _stream_ptr(stream))
@@ -327,6 +370,7 @@ def dequant_q4_f16(Wq, scale_min, stream=None):
     """fp16 rendering of the q4 weights (the tensor-core operand) as uint16 bits [N, K]."""
     import torch
     N, K2 = Wq.shape
+    _shape(scale_min, _packed_shapes(4, N, 2 * K2)[1], "scale_min")
     out = torch.empty((N, 2 * K2), dtype=torch.uint16, device=Wq.device)
     st = rt_dequant_q4_f16(_dev(Wq, torch.uint8, "Wq"), _dev(scale_min, torch.uint16, "scale_min"),
                            _dev(out, torch.uint16, "W_out"), N, 2 * K2, _stream_ptr(stream))
@@ -337,6 +381,7 @@ def dequant_q4_f16(Wq, scale_min, stream=None):
 def dequant_q8_f32(Wq, scale, stream=None):
     import torch
     N, K = Wq.shape
+    _shape(scale, (N,), "scale")
     out = torch.empty((N, K), dtype=torch.float32, device=Wq.device)
     st = rt_dequant_q8_f32(_dev(Wq, torch.int8, "Wq"), _dev(scale, torch.float32, "scale"),
                            _dev(out, torch.float32, "W_out"), N, K, _stream_ptr(stream))

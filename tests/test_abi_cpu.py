@@ -182,6 +182,61 @@ def test_block_driver_rejects_overlapping_outputs():
     assert call(80, Xs, Ys, path=9) == INVALID                        # unknown path
 
 
+def test_binding_rejects_mismatched_shapes_before_any_launch():
+    """The C layer sees pointers and sizes only, so the torch-level helpers
+    check every tensor's shape against M, N and K first (host tensors with the
+    right shapes get as far as the CUDA-tensor check)."""
+    torch = pytest.importorskip("torch")
+    M, N, K = 4, 16, 64
+    X = torch.zeros((M, K))
+    Wq4 = torch.zeros((N, K // 2), dtype=torch.uint8)
+    sm = torch.zeros((N, K // 32, 2), dtype=torch.uint16)
+    Wq8 = torch.zeros((N, K), dtype=torch.int8)
+    s8 = torch.zeros((N,))
+    with pytest.raises(ValueError, match="Wq"):
+        rtq.qgemm_q4(X, Wq4[:, :16], sm)                 # codes of a K = 32 weight
+    with pytest.raises(ValueError, match="scale_min"):
+        rtq.qgemm_q4(X, Wq4, sm[:, :1])
+    with pytest.raises(ValueError, match="Y"):
+        rtq.qgemm_q4(X, Wq4, sm, Y=torch.zeros((M, N // 2)))
+    with pytest.raises(ValueError, match="X"):
+        rtq.qgemm_q4(X.view(-1), Wq4, sm)
+    with pytest.raises(TypeError, match="CUDA"):
+        rtq.qgemm_q4(X, Wq4, sm)                         # shapes fine, host memory
+    with pytest.raises(ValueError, match="scale"):
+        rtq.qgemm_q8(X, Wq8, s8[:8])
+    with pytest.raises(ValueError, match="Wq"):
+        rtq.qgemm_q8(X, Wq8[:, :32], s8)
+    with pytest.raises(ValueError, match="fmt"):
+        rtq.qgemm_noalloc(5, X, Wq8, s8, torch.zeros((M, N)))
+    with pytest.raises(ValueError, match="scale_min"):
+        rtq.dequant_q4_f32(Wq4, sm[:, :1])
+    with pytest.raises(ValueError, match="scale"):
+        rtq.dequant_q8_f32(Wq8, s8[:1])
+
+    d, f = 64, 128
+    blk = rtq.QBlock(torch.zeros((4 * d, d // 2), dtype=torch.uint8),
+                     torch.zeros((4 * d, d // 32, 2), dtype=torch.uint16),
+                     torch.zeros((d, d), dtype=torch.int8), torch.zeros((d,)),
+                     torch.zeros((2 * f, d // 2), dtype=torch.uint8),
+                     torch.zeros((2 * f, d // 32, 2), dtype=torch.uint16),
+                     torch.zeros((d, f), dtype=torch.int8), torch.zeros((d,)), d_model=d, d_ff=f)
+    Xs = [torch.zeros((M, d)), torch.zeros((M, d)), torch.zeros((M, d)), torch.zeros((M, f))]
+    Ys = [torch.zeros((M, 4 * d)), torch.zeros((M, d)), torch.zeros((M, 2 * f)),
+          torch.zeros((M, d))]
+    with pytest.raises(ValueError, match="Y_13"):
+        rtq.qblock_project(blk, *Xs, Ys[0], Ys[1], torch.zeros((M, f)), Ys[3])
+    with pytest.raises(ValueError, match="X_w2"):
+        rtq.qblock_project(blk, Xs[0], Xs[1], Xs[2], torch.zeros((M, d)), *Ys)
+    with pytest.raises(TypeError, match="CUDA"):
+        rtq.qblock_project(blk, *Xs, *Ys)                # shapes fine, host memory
+    bad = rtq.QBlock(*(getattr(blk, n) for n in ("qkvg", "qkvg_sm", "wo", "wo_s", "w13",
+                                                 "w13_sm")),
+                     torch.zeros((d, d), dtype=torch.int8), blk.w2_s, d_model=d, d_ff=f)
+    with pytest.raises(ValueError, match="w2"):
+        bad.as_c()
+
+
 def test_dequant_validation():
     assert rtq.rt_dequant_q4_f32(W, S, Y, 4, 40, None) == SHAPE
     assert rtq.rt_dequant_q4_f32(W + 1, S, Y, 4, 64, None) == ALIGN
