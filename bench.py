@@ -811,6 +811,8 @@ def main():
     ap.add_argument("--eager", action="store_true",
                     help="issue the timed steps call by call instead of replaying a CUDA graph")
     args = ap.parse_args()
+    if args.cpu_rows < 2 or args.ref_rows < 2:
+        ap.error("--cpu-rows and --ref-rows take at least 2 (rows 0 and M-1 are always sampled)")
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -101,6 +101,8 @@ def sample_rows(M: int, n: int, seed: int) -> np.ndarray:
     """Sorted seeded subset of n row indices of [0, M) that always holds 0 and M-1."""
     if M <= n:
         return np.arange(M, dtype=np.int64)
+    if n < 2:
+        raise ValueError(f"a row sample holds rows 0 and M-1, so n >= 2 (got n = {n})")
     g = generator(seed)
     inner = g.choice(np.arange(1, M - 1), size=n - 2, replace=False)
     return np.sort(np.concatenate([[0, M - 1], inner]).astype(np.int64))
