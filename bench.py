@@ -24,6 +24,9 @@ Printed as one JSON line (rank 0):
 workload, metric and unit, one bounded row sample per step.
 
 Other workloads (`--workload`), each printing one line of the same form:
+  block_m80, block_m2048
+               one block's projection set at M = 80 (one grouped launch; the
+               roofline object then describes that launch) and at M = 2048.
   rot_m80      small M as an aggregate weight stream: the 12 blocks' weights in
                rotating device copies totalling ~4x L2, every copy's projection
                set at M = 80, replayed from a CUDA graph; value in GB/s of
