@@ -252,19 +252,33 @@ def step_weight_bytes(nblocks, projs):
 
 
 # ---------------------------------------------------------- CPU baseline
-def cpu_oracle_sample(blocks, M, projs, rows_per_proj, seed):
-    """Runs the oracle on `rows_per_proj` seeded rows of every projection;
-    returns (seconds, flops)."""
+def host_threads():
+    """Host cores this process may run on."""
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return max(1, os.cpu_count() or 1)
+
+
+def cpu_oracle_sample(blocks, M, projs, rows_per_proj, seed, threads=1):
+    """Runs the oracle on `rows_per_proj` seeded rows of every projection,
+    the rows split over `threads` host threads (the oracle's C call releases
+    the interpreter lock, so the threads run on separate cores); returns
+    (seconds, flops)."""
+    from concurrent.futures import ThreadPoolExecutor
+
     import oracle
     rows = wl.sample_rows(M, rows_per_proj, seed)
+    parts = [p for p in np.array_split(rows, max(1, min(threads, len(rows)))) if len(p)]
     flops = 0
     t0 = time.perf_counter()
-    for blk in blocks:
-        for name in projs:
-            fmt, N, K = proj_dims(name)
-            g = oracle.gemm_q4 if fmt == "q4" else oracle.gemm_q8
-            g(blk["x_" + name], *blk[name], rows=rows)
-            flops += 2 * len(rows) * N * K
+    with ThreadPoolExecutor(max_workers=len(parts)) as pool:
+        for blk in blocks:
+            for name in projs:
+                fmt, N, K = proj_dims(name)
+                g = oracle.gemm_q4 if fmt == "q4" else oracle.gemm_q8
+                list(pool.map(lambda r: g(blk["x_" + name], *blk[name], rows=r), parts))
+                flops += 2 * len(rows) * N * K
     return time.perf_counter() - t0, flops
 
 
@@ -279,17 +293,18 @@ def run_reference(args, rank, world):
               flush=True)
         return
     cfg, nblocks, M, projs, blocks = build_host(args.workload, 0, use_oracle_quantizer=True)
-    rows = args.ref_rows
+    threads = host_threads()
+    rows = max(args.ref_rows, 2 * threads)
     for i in range(args.warmup):
-        cpu_oracle_sample(blocks, M, projs, rows, seed=i)
+        cpu_oracle_sample(blocks, M, projs, rows, seed=i, threads=threads)
     secs, flops = 0.0, 0
     for i in range(args.steps):
-        s, f = cpu_oracle_sample(blocks, M, projs, rows, seed=1000 + i)
+        s, f = cpu_oracle_sample(blocks, M, projs, rows, seed=1000 + i, threads=threads)
         secs += s
         flops += f
     value = flops / secs / 1e12
     sample = (f"{rows} seeded rows of M={M} per projection, {nblocks} block(s) x "
-              f"{len(projs)} projections per step")
+              f"{len(projs)} projections per step, rows split over {threads} threads")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -297,7 +312,7 @@ def run_reference(args, rank, world):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": args.workload, "blocks": nblocks, "M": M,
                    "projections": list(projs), "rows_sampled_per_step": rows},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -305,8 +320,70 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------ timing helpers
+def gpu_uuid(dev, local_rank):
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return local_rank
+
+
+def graph_time_us(stream, fn, reps, steps, warmup):
+    """Device time of one call of fn(): `reps` back-to-back calls captured in
+    one CUDA graph, `steps` replays between CUDA events on `stream` (after
+    `warmup` replays); the first call runs outside the capture."""
+    import torch
+    with torch.cuda.stream(stream):
+        fn()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(reps):
+            fn()
+    with torch.cuda.stream(stream):
+        for _ in range(max(warmup, 1)):
+            g.replay()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    stream.synchronize()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(steps):
+            g.replay()
+        e1.record(stream)
+    stream.synchronize()
+    del g
+    return e0.elapsed_time(e1) * 1e3 / (steps * reps)
+
+
+def roofline(flops, nbytes, seconds, peaks, sustained=False):
+    """Roofline object of work that moves `nbytes` of algorithmic HBM traffic
+    and does `flops` in `seconds`.  The bound is the binding side of
+    min(tensor peak, flops/byte x HBM peak): "hbm" reports GB/s against the
+    measured copy bandwidth, "tensor" TFLOP/s against the measured dense peak
+    (the fp16 MMA runs at the bf16 rate, nominal ratio 1; the burst figure for
+    work timed in short windows, the sustained one for seconds-long loops)."""
+    tc = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    hbm = peaks["hbm_gbs"]
+    intensity = flops / nbytes
+    attainable = min(tc, intensity * hbm / 1e3)             # TFLOP/s
+    if intensity * hbm / 1e3 <= tc:
+        r = {"bound": "hbm", "achieved": nbytes / seconds / 1e9, "peak": hbm, "unit": "GB/s"}
+    else:
+        r = {"bound": "tensor", "achieved": flops / seconds / 1e12, "peak": tc, "unit": "TFLOP/s"}
+    r["frac"] = r["achieved"] / r["peak"]
+    r.update({"algorithmic_flops": flops, "algorithmic_bytes": nbytes,
+              "flop_per_byte": intensity, "attainable_tflops": attainable,
+              "tflops": flops / seconds / 1e12,
+              "tensor_peak": "sustained" if sustained else "burst",
+              "peak_source": peaks["source"]})
+    return r
+
+
 # --------------------------------------------------------- small-M stream
-def run_small_m(args, rank, world, local_rank):
+def measure_small_m(args, rank, world, local_rank, dev, stream, blocks=None):
     """Small-M projections measured as an aggregate weight stream.
 
     One M = 80 projection moves well under a megabyte of weights, less than a
@@ -316,21 +393,19 @@ def run_small_m(args, rank, world, local_rank):
     set (qkvg, wo, w13, w2) at M = 80 through rt_qblock_project.  X and Y are
     one buffer per projection shared by all copies (L2-resident, as the
     activations of a real forward pass are).  The step is captured once as a
-    CUDA graph and replayed.  value = quantized weight bytes per step / time.
-    """
+    CUDA graph and replayed.  Returns the measurement (value = quantized
+    weight bytes per step / time, GB/s)."""
     import torch
     import torch.distributed as dist
 
     import int8_dequant_gemm_b200 as rtq
 
-    rtq.lib()
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    stream = torch.cuda.Stream(device=dev)
-    sptr = ctypes.c_void_p(stream.cuda_stream)
     L = rtq.lib()
-    cfg, nblocks, M, projs = WORKLOADS[args.workload]
-    _, _, _, _, blocks = build_host("blocks12_m4096", rank)   # the 12 blocks' quantized weights
+    sptr = ctypes.c_void_p(stream.cuda_stream)
+    M, projs = 80, ("qkvg", "wo", "w13", "w2")
+    cfg = 4
+    if blocks is None:
+        _, _, _, _, blocks = build_host("blocks12_m4096", rank)   # the 12 blocks' weights
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     per_block = sum(weight_bytes(p) for p in projs)
     copies = max(len(blocks), int(math.ceil(4 * l2 / per_block)))
@@ -369,24 +444,15 @@ def run_small_m(args, rank, world, local_rank):
             graph.replay()
     stream.synchronize()
     if rtq.device_status(stream) != 0:
-        raise RuntimeError("device status word reports a timed-out wait during warm-up")
+        raise RuntimeError("device status word reports a fault during the small-M warm-up")
 
-    def barrier():
-        if world > 1:
-            dist.barrier(device_ids=[local_rank])
-
-    gpu_id = local_rank
-    try:
-        gpu_id = str(torch.cuda.get_device_properties(dev).uuid)
-        gpu_id = gpu_id if gpu_id.startswith("GPU-") else "GPU-" + gpu_id
-    except Exception:
-        pass
-    sampler = ClockSampler(gpu_id)
+    sampler = ClockSampler(gpu_uuid(dev, local_rank))
     sampler.start()
     time.sleep(0.3)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    barrier()
+    if world > 1:
+        dist.barrier(device_ids=[local_rank])
     torch.cuda.synchronize(dev)
     t0 = time.time()
     with torch.cuda.stream(stream):
@@ -396,59 +462,139 @@ def run_small_m(args, rank, world, local_rank):
         e1.record(stream)
     torch.cuda.synchronize(dev)
     t1 = time.time()
-    barrier()
+    if world > 1:
+        dist.barrier(device_ids=[local_rank])
     sampler.stop()
-    clocks = sampler.summary(t0, t1)
     ms = reduce_max(e0.elapsed_time(e1), world, dev) / args.steps
     if rtq.device_status(stream) != 0:
-        raise RuntimeError("device status word reports a timed-out wait")
+        raise RuntimeError("device status word reports a fault in the small-M stream")
     del graph
     wbytes = copies * per_block
-    gbs = world * wbytes / (ms * 1e-3) / 1e9
     flops = copies * sum(proj_flops(p, M) for p in projs)
+    abytes = copies * sum(proj_bytes(p, M) for p in projs)
     peaks = load_peaks()
-    kernels = sorted({rtq.plan(4 if proj_dims(p)[0] == "q4" else 8, M, *proj_dims(p)[1:])
-                      for p in projs})
+    gbs = world * wbytes / (ms * 1e-3) / 1e9
     fused = rtq.block_fused(M, wl.D_MODEL, wl.D_FF) == 1
     launches_per_copy = 1 if fused else sum(
         2 if rtq.plan(4 if proj_dims(p)[0] == "q4" else 8, M, *proj_dims(p)[1:])
         in ("tc_x_resident", "tc_w_streamed") else 1 for p in projs)
+    return {
+        "metric": "quantized weight GB/s at M = 80 (aggregate stream)", "value": gbs,
+        "unit": "GB/s", "ms_per_step": ms, "steps": args.steps,
+        "frac_of_hbm": gbs / world / peaks["hbm_gbs"], "hbm_peak_gbs": peaks["hbm_gbs"],
+        "tflops": world * flops / (ms * 1e-3) / 1e12,
+        "config": {"workload": "rot_m80", "M": M, "projections": list(projs),
+                   "weight_copies": copies, "weight_bytes_per_step": wbytes,
+                   "l2": f"weights rotate over {wbytes / 1e6:.0f} MB ({wbytes / l2:.1f}x L2); "
+                         f"X and Y fixed (L2-resident)",
+                   "block_launch": "grouped" if fused else "per projection",
+                   "replay": "CUDA graph of all copies' block projection sets"},
+        "gpu_launches": args.steps * copies * launches_per_copy,
+        "roofline_weights_only": {"bound": "hbm", "achieved": gbs / world,
+                                  "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                  "frac": gbs / world / peaks["hbm_gbs"],
+                                  "peak_source": peaks["source"]},
+        "roofline": roofline(flops, abytes, ms * 1e-3, peaks),
+        "clocks": sampler.summary(t0, t1),
+    }
+
+
+def run_small_m(args, rank, world, local_rank):
+    """The rot_m80 workload on its own, printed as one JSON line."""
+    import torch
+    import int8_dequant_gemm_b200 as rtq
+    rtq.lib()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.Stream(device=dev)
+    r = measure_small_m(args, rank, world, local_rank, dev, stream)
     if rank == 0:
         line = {
-            "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f16", "accumulate": "f32",
-            "data": "synthetic",
-            "config": {"workload": args.workload, "M": M, "projections": list(projs),
-                       "weight_copies": copies, "weight_bytes_per_step": wbytes,
-                       "l2_bytes": l2, "replay": "CUDA graph of all copies' block projection sets",
-                       "l2": f"weights rotate over {wbytes / 1e6:.0f} MB ({wbytes / l2:.1f}x L2); "
-                             f"X and Y fixed",
-                       "parallelism": f"replicas{world}" if world > 1 else "single"},
-            "tflops": world * flops / (ms * 1e-3) / 1e12,
-            "kernels": kernels, "block_launch": "grouped" if fused else "per projection",
-            "clocks": clocks, "gpu_launches": args.steps * copies * launches_per_copy,
-            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / peaks["hbm_gbs"], "traffic": None,
-                         "algorithmic_bytes_per_step": wbytes, "peak_source": peaks["source"]},
-            "e2e": None, "cpu_baseline": None,
+            "metric": METRIC, "value": r["value"], "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+            "accumulate": "f32", "data": "synthetic",
+            "config": dict(r["config"],
+                           parallelism=f"replicas{world}" if world > 1 else "single"),
+            "tflops": r["tflops"], "clocks": r["clocks"], "gpu_launches": r["gpu_launches"],
+            "roofline": dict(r["roofline_weights_only"], traffic=None),
+            "roofline_all_bytes": r["roofline"], "e2e": None, "cpu_baseline": None,
         }
         print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------ large M gate
+def measure_large_m(args, rank, world, local_rank, dev, stream):
+    """The large-M gate: q4 512->2048 (the ffn.w1 shape) at M = 65536 (B = 64,
+    S = 1024) with a seeded 1 % of groups holding a x20 outlier, RT_PATH_AUTO,
+    five calls per CUDA graph.  X (128 MiB) and Y (512 MiB) exceed L2."""
+    import torch
+    import torch.distributed as dist
+
+    import int8_dequant_gemm_b200 as rtq
+
+    L = rtq.lib()
+    sptr = ctypes.c_void_p(stream.cuda_stream)
+    M, N, K = 65536, 2048, 512
+    seed = wl.seed_for(5, 0, 1)
+    W = wl.with_outliers(wl.weights(N, K, seed), seed + 1)
+    Wq, S = rtq.quantize_q4_g32(W)
+    Wd = torch.from_numpy(Wq).to(dev)
+    Sd = torch.from_numpy(S).to(dev)
+    X = torch.from_numpy(wl.activations(M, K, seed + 2 + M + 100_000 * rank)).to(dev)
+    Y = torch.empty((M, N), dtype=torch.float32, device=dev)
+    a = (X.data_ptr(), Wd.data_ptr(), Sd.data_ptr(), Y.data_ptr(), M, N, K, 0, sptr)
+
+    def call():
+        st = L.rt_qgemm_q4(*a)
+        if st:
+            raise rtq.RtqError(st, "rt_qgemm_q4")
+
+    sampler = ClockSampler(gpu_uuid(dev, local_rank))
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier(device_ids=[local_rank])
+    t0 = time.time()
+    us = graph_time_us(stream, call, reps=5, steps=max(2, args.steps // 2), warmup=args.warmup)
+    t1 = time.time()
+    sampler.stop()
+    us = reduce_max(us, world, dev)
+    if rtq.device_status(stream) != 0:
+        raise RuntimeError("device status word reports a fault in the large-M gate")
+    flops = 2 * M * N * K
+    nbytes = Wq.nbytes + S.nbytes + 4 * M * K + 4 * M * N
+    peaks = load_peaks()
+    r = roofline(flops, nbytes, us * 1e-6, peaks)
+    del X, Y
+    torch.cuda.empty_cache()
+    return {
+        "metric": "TFLOP/s of q4 512->2048 at M = 65536", "value": world * flops / (us * 1e-6) / 1e12,
+        "unit": "TFLOP/s", "us_per_call": us,
+        "frac_of_dense_peak": flops / (us * 1e-6) / 1e12 / peaks["bf16_tflops"],
+        "dense_peak_tflops": peaks["bf16_tflops"], "kernel": rtq.plan(4, M, N, K),
+        "launches_per_call": 2,
+        "config": {"shape": "q4 512->2048", "M": M, "path": "auto", "calls_per_graph": 5,
+                   "outliers": "1% of groups x20", "l2": "X 128 MiB + Y 512 MiB > L2"},
+        "roofline": r, "clocks": sampler.summary(t0, t1),
+    }
 
 
 # --------------------------------------------------------------- M sweep
 SWEEP_SHAPES = (("q4", 2048, 512), ("q8", 512, 2048))    # ffn.w1 and ffn.w2 shapes
 SWEEP_M = (1, 16, 80, 512, 4096, 65536)
+SWEEP_SIMT_MAX_M = 4096      # the fp32 SIMT path is timed up to here
 
 
 def run_sweep(args, rank, world, local_rank):
-    """M sweep of the q4 512->2048 and q8 2048->512 projections under
-    RT_PATH_AUTO (weights with a seeded 1 % of 32-groups holding a x20
-    outlier).  Each point is 20 calls captured in a CUDA graph, replayed
-    after warm-up; inputs stay in place between calls, so points whose data
-    fit in L2 (M <= 4096) run L2-warm.  value = TFLOP/s of the q4 shape at
-    M = 65536, the large-M gate; `sweep` lists every point and the kernel the
-    dispatcher chose."""
+    """M sweep of the q4 512->2048 and q8 2048->512 projections (weights with a
+    seeded 1 % of 32-groups holding a x20 outlier) on the SIMT path, the
+    tensor-core path and RT_PATH_AUTO.  Every point streams from HBM: the
+    weights, activations and outputs are held in as many copies as make at
+    least 2x L2, and successive calls use successive copies (a CUDA graph of
+    max(copies, 20) calls).  `crossover` gives, per shape, the smallest M at
+    which the tensor-core path beats the SIMT path; value = TFLOP/s of the q4
+    shape at M = 65536 (AUTO), the large-M gate."""
     import torch
 
     import int8_dequant_gemm_b200 as rtq
@@ -459,56 +605,65 @@ def run_sweep(args, rank, world, local_rank):
     stream = torch.cuda.Stream(device=dev)
     sptr = ctypes.c_void_p(stream.cuda_stream)
     L = rtq.lib()
-    reps = 20
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    peaks = load_peaks()
     points = []
     for fmt, N, K in SWEEP_SHAPES:
         seed = wl.seed_for(5, 0, 1 if fmt == "q4" else 3)
         W = wl.with_outliers(wl.weights(N, K, seed), seed + 1)
         Wq, S = rtq.quantize_q4_g32(W) if fmt == "q4" else rtq.quantize_q8_row(W)
-        Wd = torch.from_numpy(Wq).to(dev)
-        Sd = torch.from_numpy(S).to(dev)
         fn = L.rt_qgemm_q4 if fmt == "q4" else L.rt_qgemm_q8
         fcode = 4 if fmt == "q4" else 8
+        wb = Wq.nbytes + S.nbytes
         for M in SWEEP_M:
-            X = torch.from_numpy(wl.activations(M, K, seed + 2 + M)).to(dev)
-            Y = torch.empty((M, N), dtype=torch.float32, device=dev)
-            call_args = (X.data_ptr(), Wd.data_ptr(), Sd.data_ptr(), Y.data_ptr(), M, N, K, 0, sptr)
+            per_copy = wb + 4 * M * K + 4 * M * N
+            copies = max(1, min(1000, int(math.ceil(2 * l2 / per_copy))))
+            X0 = wl.activations(M, K, seed + 2 + M)
+            bufs = []
+            for _ in range(copies):
+                bufs.append((torch.from_numpy(X0).to(dev), torch.from_numpy(Wq).to(dev),
+                             torch.from_numpy(S).to(dev),
+                             torch.empty((M, N), dtype=torch.float32, device=dev)))
+            reps = max(copies, 20)
+            for path, pcode in (("simt", 1), ("tc", 2), ("auto", 0)):
+                if path == "simt" and M > SWEEP_SIMT_MAX_M:
+                    continue
+                args_list = [(x.data_ptr(), w.data_ptr(), sc.data_ptr(), y.data_ptr(), M, N, K,
+                              pcode, sptr) for x, w, sc, y in bufs]
+                state = {"i": 0}
 
-            def calls():
-                for _ in range(reps):
-                    st = fn(*call_args)
+                def call():
+                    st = fn(*args_list[state["i"] % copies])
+                    state["i"] += 1
                     if st:
                         raise rtq.RtqError(st, "rt_qgemm")
 
-            with torch.cuda.stream(stream):
-                calls()                      # grows the workspace outside the capture
-            stream.synchronize()
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                calls()
-            with torch.cuda.stream(stream):
-                for _ in range(max(args.warmup, 1)):
-                    g.replay()
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            stream.synchronize()
-            with torch.cuda.stream(stream):
-                e0.record(stream)
-                for _ in range(args.steps):
-                    g.replay()
-                e1.record(stream)
-            stream.synchronize()
-            del g
-            us = e0.elapsed_time(e1) * 1e3 / (args.steps * reps)
-            wb = Wq.nbytes + S.nbytes
-            points.append({"shape": f"{fmt} {K}->{N}", "M": M, "kernel": rtq.plan(fcode, M, N, K),
-                           "us_per_call": us, "tflops": 2.0 * M * N * K / (us * 1e-6) / 1e12,
-                           "weight_gbs": wb / (us * 1e-6) / 1e9})
-            del X, Y
+                us = graph_time_us(stream, call, reps=reps, steps=args.steps, warmup=args.warmup)
+                points.append({
+                    "shape": f"{fmt} {K}->{N}", "M": M, "path": path,
+                    "kernel": rtq.plan(fcode, M, N, K, path), "us_per_call": us,
+                    "tflops": 2.0 * M * N * K / (us * 1e-6) / 1e12,
+                    "weight_gbs": wb / (us * 1e-6) / 1e9,
+                    "roofline": roofline(2.0 * M * N * K, per_copy, us * 1e-6, peaks),
+                    "copies": copies})
+            del bufs
+            torch.cuda.empty_cache()
     if rtq.device_status(stream) != 0:
-        raise RuntimeError("device status word reports a timed-out wait")
-    peaks = load_peaks()
-    head = next(p for p in points if p["shape"].startswith("q4") and p["M"] == SWEEP_M[-1])
+        raise RuntimeError("device status word reports a fault")
+    crossover = {}
+    for fmt, N, K in SWEEP_SHAPES:
+        name = f"{fmt} {K}->{N}"
+        won = [M for M in SWEEP_M
+               if any(p["shape"] == name and p["M"] == M and p["path"] == "simt" for p in points)
+               and next(p for p in points if p["shape"] == name and p["M"] == M
+                        and p["path"] == "tc")["us_per_call"]
+               < next(p for p in points if p["shape"] == name and p["M"] == M
+                      and p["path"] == "simt")["us_per_call"]]
+        crossover[name] = {"tc_faster_from_M": min(won) if won else None,
+                           "auto_simt_max_M": max(M for M in range(1, 129)
+                                                  if rtq.auto_path(fmt == "q4" and 4 or 8, M, N, K) == 1)}
+    head = next(p for p in points if p["shape"].startswith("q4") and p["M"] == SWEEP_M[-1]
+                and p["path"] == "auto")
     if rank == 0:
         line = {
             "metric": METRIC, "value": head["tflops"], "unit": "TFLOP/s", "n_gpus": 1,
@@ -516,13 +671,11 @@ def run_sweep(args, rank, world, local_rank):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
             "accumulate": "f32", "data": "synthetic",
             "config": {"workload": "m_sweep", "shapes": [f"{f} {k}->{n}" for f, n, k in SWEEP_SHAPES],
-                       "M": list(SWEEP_M), "calls_per_graph": reps, "path": "auto",
-                       "l2": "inputs reused between calls: L2-warm for M <= 4096"},
-            "roofline": {"bound": "tensor", "achieved": head["tflops"],
-                         "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                         "frac": head["tflops"] / peaks["bf16_tflops_sustained"],
-                         "peak_source": peaks["source"]},
-            "sweep": points, "e2e": None, "cpu_baseline": None,
+                       "M": list(SWEEP_M), "paths": ["simt", "tc", "auto"],
+                       "simt_max_M": SWEEP_SIMT_MAX_M,
+                       "l2": "weights, X and Y in >= 2x L2 of rotating copies"},
+            "roofline": dict(head["roofline"], traffic=None),
+            "crossover": crossover, "sweep": points, "e2e": None, "cpu_baseline": None,
         }
         print(json.dumps(line), flush=True)
 
@@ -574,12 +727,16 @@ def run_gpu(args, rank, world, local_rank):
             block_args.append((c, [db[n][2].data_ptr() for n in projs] +
                                [db[n][3].data_ptr() for n in projs]))
 
+    def run_block(i):
+        c, ptrs = block_args[i]
+        st = L.rt_qblock_project(ctypes.byref(c), M, *ptrs, 0, sptr)
+        if st:
+            raise rtq.RtqError(st, "rt_qblock_project")
+
     def step():
         if full_block:
-            for c, ptrs in block_args:
-                st = L.rt_qblock_project(ctypes.byref(c), M, *ptrs, 0, sptr)
-                if st:
-                    raise rtq.RtqError(st, "rt_qblock_project")
+            for i in range(len(block_args)):
+                run_block(i)
         else:
             for _, fn, a in calls:
                 st = fn(*a)
@@ -610,7 +767,7 @@ def run_gpu(args, rank, world, local_rank):
             step()
     stream.synchronize()
     if rtq.device_status(stream) != 0:
-        raise RuntimeError("device status word reports a timed-out wait during warm-up")
+        raise RuntimeError("device status word reports a fault during warm-up")
 
     # ---- the step captured once as a CUDA graph, so that the host's cost of
     # issuing 96 launches stays out of the timed region; if the capture is
@@ -625,7 +782,7 @@ def run_gpu(args, rank, world, local_rank):
                 g.replay()
             stream.synchronize()
             if rtq.device_status(stream) != 0:
-                raise RuntimeError("timed-out wait in the captured step")
+                raise RuntimeError("fault in the captured step")
             graph, issue = g, "cuda_graph"
         except Exception as exc:   # fall back to eager issue, recorded in the line
             torch.cuda.synchronize(dev)
@@ -638,13 +795,7 @@ def run_gpu(args, rank, world, local_rank):
             step()
 
     # ---- timed region: K steps through the block driver
-    gpu_id = local_rank
-    try:
-        gpu_id = str(torch.cuda.get_device_properties(dev).uuid)
-        gpu_id = gpu_id if gpu_id.startswith("GPU-") else "GPU-" + gpu_id
-    except Exception:
-        pass
-    sampler = ClockSampler(gpu_id)
+    sampler = ClockSampler(gpu_uuid(dev, local_rank))
     sampler.start()
     time.sleep(0.3)
     e0 = torch.cuda.Event(enable_timing=True)
@@ -660,74 +811,61 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     t_wall1 = time.time()
     barrier()
+    sampler.stop()
+    clocks = sampler.summary(t_wall0, t_wall1)
     ms_total = max_over_ranks(e0.elapsed_time(e1))
     ms_per_step = ms_total / args.steps
+    del graph
 
-    # ---- per-kernel durations: every launch bracketed by events, K steps.
-    # A block run as one grouped launch is timed as that launch.
-    evs = {"block": []} if fused_block else {name: [] for name in projs}
-    with torch.cuda.stream(stream):
-        for _ in range(args.steps):
-            if fused_block:
-                for c, ptrs in block_args:
-                    s0 = torch.cuda.Event(enable_timing=True)
-                    s1 = torch.cuda.Event(enable_timing=True)
-                    s0.record(stream)
-                    st = L.rt_qblock_project(ctypes.byref(c), M, *ptrs, 0, sptr)
-                    s1.record(stream)
-                    if st:
-                        raise rtq.RtqError(st, "rt_qblock_project")
-                    evs["block"].append((s0, s1))
-                continue
-            for name, fn, a in calls:
-                s0 = torch.cuda.Event(enable_timing=True)
-                s1 = torch.cuda.Event(enable_timing=True)
-                s0.record(stream)
-                fn(*a)
-                s1.record(stream)
-                evs[name].append((s0, s1))
-    torch.cuda.synchronize(dev)
-    t_wall2 = time.time()
-    sampler.stop()
-    clocks = sampler.summary(t_wall0, t_wall2)
-    kern_us = {n: 1e3 * statistics.mean(a.elapsed_time(b) for a, b in v) for n, v in evs.items()}
+    # ---- per-call device time, each call of block 0 in its own CUDA graph of
+    # 20 back-to-back calls (a block run as one grouped launch is timed as
+    # that launch); the sum over the step is checked against ms_per_step
+    reps = 20
+    if fused_block:
+        kern_us = {"block": graph_time_us(stream, lambda: run_block(0), reps, args.steps,
+                                          args.warmup)}
+    else:
+        kern_us = {}
+        for name, fn, a in calls[:len(projs)]:
+            def one(fn=fn, a=a):
+                st = fn(*a)
+                if st:
+                    raise rtq.RtqError(st, "rt_qgemm")
+            kern_us[name] = graph_time_us(stream, one, reps, args.steps, args.warmup)
     if rtq.device_status(stream) != 0:
-        raise RuntimeError("device status word reports a timed-out wait")
+        raise RuntimeError("device status word reports a fault")
 
     flops = step_flops(M, nblocks, projs)
     value = job_value(world, flops, ms_per_step)
     wbytes = step_weight_bytes(nblocks, projs)
 
-    # ---- roofline of the dominant kernel
+    # ---- roofline of the dominant call
     peaks = load_peaks()
     if fused_block:
-        # one launch per block: its bytes and flops are the four projections'
         share = {"block": kern_us["block"] * nblocks}
         dom, path = "block", "tc"
         b_alg = sum(proj_bytes(p, M) for p in projs)
         f_alg = sum(proj_flops(p, M) for p in projs)
         kernel_key = f"block_grouped_tc_M{M}"
+        call_launches = 1
     else:
         share = {n: kern_us[n] * nblocks for n in projs}
         dom = max(share, key=share.get)
         fmt, N, K = proj_dims(dom)
-        path = "tc" if rtq.auto_path(4 if fmt == "q4" else 8, M, N, K) == 2 else "simt"
+        fcode = 4 if fmt == "q4" else 8
+        path = "tc" if rtq.auto_path(fcode, M, N, K) == 2 else "simt"
         b_alg, f_alg = proj_bytes(dom, M), proj_flops(dom, M)
         kernel_key = f"{dom}_{fmt}_{path}_M{M}"
-    t_s = kern_us[dom] * 1e-6
-    t_hbm = b_alg / (peaks["hbm_gbs"] * 1e9)
-    t_tc = f_alg / (peaks["bf16_tflops_sustained"] * 1e12)
-    traffic = recorded_traffic(kernel_key)
-    if t_hbm >= t_tc or path == "simt":
-        roof = {"bound": "hbm", "achieved": b_alg / t_s / 1e9, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s"}
-    else:
-        roof = {"bound": "tensor", "achieved": f_alg / t_s / 1e12,
-                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s"}
-    roof.update({"frac": roof["achieved"] / roof["peak"], "traffic": traffic,
-                 "kernel": kernel_key, "algorithmic_bytes": b_alg, "algorithmic_flops": f_alg,
-                 "avg_launch_us": kern_us[dom], "peak_source": peaks["source"],
+        call_launches = 2 if rtq.plan(fcode, M, N, K) in ("tc_x_resident", "tc_w_streamed") else 1
+    roof = roofline(f_alg, b_alg, kern_us[dom] * 1e-6, peaks)
+    roof.update({"traffic": recorded_traffic(kernel_key), "kernel": kernel_key,
+                 "kernel_plan": (rtq.plan(4 if proj_dims(dom)[0] == "q4" else 8, M,
+                                          *proj_dims(dom)[1:]) if dom != "block"
+                                 else "tc_w_stationary (grouped)"),
+                 "launches_per_call": call_launches, "avg_call_us": kern_us[dom],
+                 "timed_as": "one call, 20 per CUDA graph, mean over replays",
                  "share_of_step": share[dom] / sum(share.values())})
+    calls_sum_ms = sum(share.values()) * 1e-3
 
     # ---- end to end: pinned host inputs in, results out, inside the timed region
     e2e = None
@@ -766,15 +904,29 @@ def run_gpu(args, rank, world, local_rank):
         e2e = {"value": job_value(world, flops, ms_e2e), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
                "steps": n_e2e}
+        del hx, hy
+
+    # ---- the two gates of the metric, measured in the same run on the
+    # default workload: small M (aggregate weight stream) and M = 65536
+    small_m = large_m = None
+    if args.workload == "blocks12_m4096" and not args.no_gates:
+        del dblocks, calls, block_args
+        torch.cuda.empty_cache()
+        small_m = measure_small_m(args, rank, world, local_rank, dev, stream, blocks=blocks)
+        torch.cuda.empty_cache()
+        large_m = measure_large_m(args, rank, world, local_rank, dev, stream)
 
     # ---- CPU oracle baseline on a bounded sample (rank 0, single GPU only)
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        secs, cflops = cpu_oracle_sample(blocks, M, projs, args.cpu_rows, seed=7)
-        cpu = {"value": cflops / secs / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-               "sample": f"{args.cpu_rows} seeded rows of M={M} for each of the "
+        threads = host_threads()
+        rows = max(args.cpu_rows, 16 * threads)
+        secs, cflops = cpu_oracle_sample(blocks, M, projs, rows, seed=7, threads=threads)
+        cpu = {"value": cflops / secs / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"{rows} seeded rows of M={M} for each of the "
                          f"{nblocks * len(projs)} projections ({cflops / 1e9:.2f} GFLOP, "
-                         f"{secs:.1f} s, single-threaded double-precision oracle)"}
+                         f"{secs:.1f} s, double-precision oracle, rows split over {threads} "
+                         f"host threads)"}
 
     if rank == 0:
         bytes_act = sum(4 * M * (proj_dims(p)[1] + proj_dims(p)[2]) for p in projs) * nblocks
@@ -790,9 +942,10 @@ def run_gpu(args, rank, world, local_rank):
                              f"step), no flush",
                        "issue": issue},
             "weight_gbs": world * wbytes / (ms_per_step * 1e-3) / 1e9,
-            "kernel_us": kern_us,
+            "call_us": kern_us, "calls_sum_ms_per_step": calls_sum_ms,
             "clocks": clocks, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
             "roofline": roof, "cpu_baseline": cpu,
+            "small_m": small_m, "large_m": large_m,
         }
         print(json.dumps(line), flush=True)
 
@@ -813,6 +966,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true",
                     help="issue the timed steps call by call instead of replaying a CUDA graph")
+    ap.add_argument("--no-gates", action="store_true",
+                    help="skip the small-M and M = 65536 measurements of the default workload")
     args = ap.parse_args()
     if args.cpu_rows < 2 or args.ref_rows < 2:
         ap.error("--cpu-rows and --ref-rows take at least 2 (rows 0 and M-1 are always sampled)")

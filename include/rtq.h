@@ -34,8 +34,9 @@
  *   - Pointers: X, Wq, scale(_min) and Y are DEVICE pointers on the current
  *     device; `stream` is a cudaStream_t (NULL = legacy default stream).
  *   - Execution: stream-ordered and asynchronous.  RT_OK means "validated and
- *     enqueued".  Errors raised later on the device (a bounded wait that gave
- *     up) are latched in a device status word read by rt_device_status().
+ *     enqueued".  Conditions found later on the device (a bounded wait that
+ *     gave up, an activation outside the fp16 range) are latched in a device
+ *     status word read by rt_device_status().
  *   - Alignment: X, Y and Wq 16-byte aligned; scale_min 4-byte aligned; scale
  *     4-byte aligned.  Otherwise RT_ERR_ALIGNMENT.
  *   - Shapes: M >= 0 (M == 0 is a no-op), N >= 1, K >= 1; q4 needs K % 32 == 0
@@ -49,9 +50,10 @@
  *     X and the exact dequantized q4 weights once to fp16 -- q8 codes are
  *     exact, their row scale is applied in fp32 after the MMA -- and
  *     accumulates in fp32 in TMEM (<= 4e-3; about 3e-4 on N(0,1) activations).
- *     fp16 operands need |X| <= 65504 (larger activations become infinite);
- *     RT_PATH_TC_BF16 runs the same kernels on bf16 operands, which keep the
- *     fp32 range but only 8 significant bits (about 2e-3 to 5e-3).
+ *     fp16 operands hold |x| < 65520: an activation that rounds to infinity
+ *     or is not finite makes the affected outputs infinite or NaN and latches
+ *     RT_ERR_OPERAND_RANGE for rt_device_status(); such activations need the
+ *     SIMT path.
  */
 #ifndef RTQ_H
 #define RTQ_H
@@ -71,15 +73,16 @@ typedef enum rt_status {
     RT_ERR_DEVICE_TIMEOUT = 5,    /* a kernel's bounded wait expired (see rt_device_status) */
     RT_ERR_VALUE_RANGE = 6,       /* quantizer input not finite / outside binary16 range */
     RT_ERR_WORKSPACE = 7,         /* the workspace would have to grow inside a stream capture */
-    RT_ERR_SCRATCH_LIMIT = 8      /* rt_qgemm_noalloc: M * K * 2 > RT_NOALLOC_SCRATCH_BYTES */
+    RT_ERR_SCRATCH_LIMIT = 8,     /* rt_qgemm_noalloc: M * K * 2 > RT_NOALLOC_SCRATCH_BYTES */
+    RT_ERR_OPERAND_RANGE = 9,     /* an activation was not a finite fp16 value (rt_device_status) */
+    RT_ERR_UNSUPPORTED_DEVICE = 10 /* current device index >= 64, the library's per-device limit */
 } rt_status;
 
 typedef enum rt_path {
     RT_PATH_AUTO = 0,   /* SIMT for M <= 8 or K % 64 != 0, else TC */
     RT_PATH_SIMT = 1,   /* fp32 CUDA-core kernels */
-    RT_PATH_TC = 2,     /* tcgen05 tensor-core kernels, fp16 operands, fp32 accumulate in TMEM */
-    RT_PATH_TC_BF16 = 3 /* the same kernels with bf16 operands */
-} rt_path;
+    RT_PATH_TC = 2      /* tcgen05 tensor-core kernels, fp16 operands, fp32 accumulate in TMEM */
+} rt_path;            /* any other value: RT_ERR_INVALID_ARG */
 
 /* Human-readable name of a status code; never NULL. */
 const char *rt_status_string(int status);
@@ -120,8 +123,8 @@ int rt_qgemm_auto_path(int fmt, int64_t M, int64_t N, int64_t K);
  *                             128 up to 512);
  *   RT_KERNEL_TC_W_STREAMED   tcgen05, persistent 128 x 192 tiles with both
  *                             operands TMA-staged (M > 128, other K).
- * The last two run an activation pre-pass (X rounded once to the 16-bit
- * operand type) into a per-(device, stream) workspace of M * K * 2 bytes. */
+ * The last two run an activation pre-pass (X rounded once to fp16) into a
+ * per-(device, stream) workspace of M * K * 2 bytes. */
 typedef enum rt_kernel {
     RT_KERNEL_SIMT = 1,
     RT_KERNEL_TC_W_STATIONARY = 2,
@@ -133,8 +136,8 @@ typedef enum rt_kernel {
 int rt_qgemm_plan(int fmt, int64_t M, int64_t N, int64_t K, int path);
 
 /*
- * Workspace.  The TMA-fed kernels stage the activations, rounded to the
- * 16-bit operand type, in a device buffer the library keeps per (device,
+ * Workspace.  The TMA-fed kernels stage the activations, rounded to fp16,
+ * in a device buffer the library keeps per (device,
  * stream): rt_workspace_bytes() gives the size a GEMM needs (0 for the other
  * kernels, -1 for a rejected shape).  The buffer grows on first need with
  * cudaMalloc; growth synchronizes that stream.  It cannot grow while the
@@ -159,7 +162,7 @@ rt_status rt_workspace_release(void);
  * fmt = 4: Wq/scales are the q4 tensors of rt_qgemm_q4; fmt = 8: those of
  * rt_qgemm_q8.  X, Y, M, N, K, path and stream, validation and results are
  * as for rt_qgemm_q4/q8, and the same kernel runs (rt_qgemm_plan).  The
- * TMA-fed kernels stage the 16-bit activations in one file-scope device
+ * TMA-fed kernels stage the fp16 activations in one file-scope device
  * array of RT_NOALLOC_SCRATCH_BYTES (16 MiB) per device instead of the
  * per-stream workspace; a problem whose M * K * 2 exceeds it returns
  * RT_ERR_SCRATCH_LIMIT and launches nothing (for example M * K up to 8M
@@ -193,8 +196,8 @@ rt_status rt_qgemm_noalloc(int fmt, const float *X, const void *Wq, const void *
  * [M, 4*d_model], Y_o [M, d_model], Y_13 [M, 2*d_ff], Y_2 [M, d_model].
  *
  * Launches: where all four products take RT_KERNEL_TC_W_STATIONARY with one
- * activation tile (1 <= M <= 128 on a tensor-core path: RT_PATH_AUTO above
- * the SIMT range, RT_PATH_TC, RT_PATH_TC_BF16), one grouped launch of that
+ * activation tile (1 <= M <= 128 on the tensor-core path: RT_PATH_AUTO above
+ * the SIMT range, or RT_PATH_TC), one grouped launch of that
  * kernel computes all four: each CTA takes a 128-row weight tile of one of
  * the projections and a slice of its K; each projection splits K by its own
  * factor (so w2, with four times the K of the others, splits four times as
@@ -261,9 +264,7 @@ rt_status rt_quantize_q8_row(const float *W, int64_t N, int64_t K, int8_t *Wq, f
  * check them bit for bit:
  *   *_f32  : W[o,k] rounded once to fp32 (the SIMT path's operand);
  *   q4_f16 : the exact value rounded once to fp16, stored as uint16 bits (the
- *            tensor-core path's q4 operand);
- *   q4_bf16: the fp32 value rounded again to bf16 (the RT_PATH_TC_BF16
- *            operand).
+ *            tensor-core path's q4 operand).
  * W_out is [N,K].  Same alignment and shape rules as the GEMMs.
  */
 rt_status rt_dequant_q4_f32(const uint8_t *Wq, const uint16_t *scale_min, float *W_out,
@@ -272,16 +273,33 @@ rt_status rt_dequant_q8_f32(const int8_t *Wq, const float *scale, float *W_out,
                             int64_t N, int64_t K, void *stream);
 rt_status rt_dequant_q4_f16(const uint8_t *Wq, const uint16_t *scale_min, uint16_t *W_out,
                             int64_t N, int64_t K, void *stream);
-rt_status rt_dequant_q4_bf16(const uint8_t *Wq, const uint16_t *scale_min, uint16_t *W_out,
-                             int64_t N, int64_t K, void *stream);
 
 /*
- * Synchronizes `stream`, then reads and clears the device status word that
- * kernels latch when one of their bounded waits gives up.  *device_status
- * receives RT_OK or RT_ERR_DEVICE_TIMEOUT.  Returns RT_ERR_CUDA if the
+ * Synchronizes `stream`, then reads and clears the current device's status
+ * word, which the tensor-core kernels latch when one of their bounded waits
+ * gives up (RT_ERR_DEVICE_TIMEOUT; outputs of that launch are undefined) or
+ * when an activation is not a finite fp16 value after rounding
+ * (RT_ERR_OPERAND_RANGE).  *device_status receives RT_OK or one of those two
+ * (the timeout when both were latched).  Returns RT_ERR_CUDA if the
  * synchronization itself fails.
  */
 rt_status rt_device_status(void *stream, int *device_status);
+
+/*
+ * Test hook for the device-side failure path (not for production use; the
+ * model cards have no counterpart).  Synchronizes the current device, then
+ * sets how its tensor-core kernels launched from now on behave:
+ *   mode 0: normal operation;
+ *   mode 1: in every CTA the first producer arrival is left out (a converter
+ *           thread skips its arrival on the first stage, or the weight TMA
+ *           thread never requests its first box), so a consumer's bounded
+ *           wait runs out, the kernel winds down and latches
+ *           RT_ERR_DEVICE_TIMEOUT.
+ * wait_ns: bound of every mbarrier wait in nanoseconds; 0 restores the
+ * default of 2 s.  RT_ERR_INVALID_ARG for another mode or a negative bound.
+ * Restore rt_debug_inject(0, 0) before normal use.
+ */
+rt_status rt_debug_inject(int mode, int64_t wait_ns);
 
 #ifdef __cplusplus
 }

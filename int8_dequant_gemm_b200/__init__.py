@@ -20,18 +20,20 @@ import numpy as np
 __all__ = [
     "RtqError", "lib", "PATHS", "OK", "qgemm_q4", "qgemm_q8", "qblock_project", "QBlock",
     "quantize_q4_g32", "quantize_q8_row", "dequant_q4_f32", "dequant_q8_f32",
-    "dequant_q4_bf16", "dequant_q4_f16", "device_status", "auto_path", "status_string",
-    "qgemm_noalloc", "plan", "block_fused", "workspace_bytes",
+    "dequant_q4_f16", "device_status", "auto_path", "status_string",
+    "qgemm_noalloc", "plan", "block_fused", "workspace_bytes", "debug_inject",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "librtq.so")
 
 OK = 0
+RT_ERR_INVALID_ARG = 1
 RT_ERR_DEVICE_TIMEOUT = 5
 RT_ERR_SCRATCH_LIMIT = 8
+RT_ERR_OPERAND_RANGE = 9
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024   # RT_NOALLOC_SCRATCH_BYTES in include/rtq.h
-PATHS = {"auto": 0, "simt": 1, "tc": 2, "tc_bf16": 3}
+PATHS = {"auto": 0, "simt": 1, "tc": 2}
 
 _p = ctypes.c_void_p
 _i64 = ctypes.c_int64
@@ -87,13 +89,14 @@ def lib() -> ctypes.CDLL:
     L.rt_quantize_q4_g32.argtypes = [_p, _i64, _i64, _i32, _p, _p]
     L.rt_quantize_q8_row.restype = _i32
     L.rt_quantize_q8_row.argtypes = [_p, _i64, _i64, _p, _p]
-    for name in ("rt_dequant_q4_f32", "rt_dequant_q8_f32", "rt_dequant_q4_bf16",
-                 "rt_dequant_q4_f16"):
+    for name in ("rt_dequant_q4_f32", "rt_dequant_q8_f32", "rt_dequant_q4_f16"):
         f = getattr(L, name)
         f.restype = _i32
         f.argtypes = [_p, _p, _p, _i64, _i64, _p]
     L.rt_device_status.restype = _i32
     L.rt_device_status.argtypes = [_p, ctypes.POINTER(_i32)]
+    L.rt_debug_inject.restype = _i32
+    L.rt_debug_inject.argtypes = [_i32, _i64]
     _lib = L
     return L
 
@@ -146,16 +149,16 @@ def rt_dequant_q8_f32(Wq, scale, W_out, N, K, stream) -> int:
     return lib().rt_dequant_q8_f32(Wq, scale, W_out, N, K, stream)
 
 
-def rt_dequant_q4_bf16(Wq, scale_min, W_out, N, K, stream) -> int:
-    return lib().rt_dequant_q4_bf16(Wq, scale_min, W_out, N, K, stream)
-
-
 def rt_dequant_q4_f16(Wq, scale_min, W_out, N, K, stream) -> int:
     return lib().rt_dequant_q4_f16(Wq, scale_min, W_out, N, K, stream)
 
 
 def rt_device_status(stream, out) -> int:
     return lib().rt_device_status(stream, out)
+
+
+def rt_debug_inject(mode, wait_ns) -> int:
+    return lib().rt_debug_inject(mode, wait_ns)
 
 
 def rt_qgemm_auto_path(fmt, M, N, K) -> int:
@@ -354,18 +357,6 @@ def dequant_q4_f32(Wq, scale_min, stream=None):
     return out
 
 
-def dequant_q4_bf16(Wq, scale_min, stream=None):
-    """bf16 rendering of the q4 weights as uint16 bits [N, K]."""
-    import torch
-    N, K2 = Wq.shape
-    _shape(scale_min, _packed_shapes(4, N, 2 * K2)[1], "scale_min")
-    out = torch.empty((N, 2 * K2), dtype=torch.uint16, device=Wq.device)
-    st = rt_dequant_q4_bf16(_dev(Wq, torch.uint8, "Wq"), _dev(scale_min, torch.uint16, "scale_min"),
-                            _dev(out, torch.uint16, "W_out"), N, 2 * K2, _stream_ptr(stream))
-    _check(st, "rt_dequant_q4_bf16")
-    return out
-
-
 def dequant_q4_f16(Wq, scale_min, stream=None):
     """fp16 rendering of the q4 weights (the tensor-core operand) as uint16 bits [N, K]."""
     import torch
@@ -390,10 +381,18 @@ def dequant_q8_f32(Wq, scale, stream=None):
 
 
 def device_status(stream=None) -> int:
-    """Synchronizes the stream and returns (and clears) the device status word."""
+    """Synchronizes the stream and returns (and clears) the device status word:
+    OK, RT_ERR_DEVICE_TIMEOUT or RT_ERR_OPERAND_RANGE."""
     v = ctypes.c_int(0)
     _check(rt_device_status(_stream_ptr(stream), ctypes.byref(v)), "rt_device_status")
     return int(v.value)
+
+
+def debug_inject(mode: int, wait_ns: int = 0):
+    """Test hook of the device failure path (see rt_debug_inject): mode 1 makes
+    the first producer arrival of every CTA go missing, with every bounded wait
+    limited to wait_ns; debug_inject(0) restores normal operation."""
+    _check(rt_debug_inject(int(mode), int(wait_ns)), "rt_debug_inject")
 
 
 def auto_path(fmt: int, M: int, N: int, K: int) -> int:

@@ -1,6 +1,7 @@
 // C ABI of the library (declared in include/rtq.h): argument validation, the
 // M-based choice between the SIMT and tensor-core kernels, the per-block
-// projection driver and the device status word.
+// projection driver and the per-device control block (status bits, the wait
+// bound and the fault-injection test hook).
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -10,27 +11,30 @@
 
 #include "../../include/rtq.h"
 #include "kernels.cuh"
+#include "ptx.cuh"
 
-// Latched by kernels whose bounded waits gave up (bit RT_ERR_DEVICE_TIMEOUT).
-__device__ unsigned int g_rtq_device_status;
+// The control block every tensor-core kernel reads (see rtq::DevCtl).
+__device__ rtq::DevCtl g_rtq_ctl = {0u, 0u, rtq::kWaitLimitNs};
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::mutex g_status_mu;
-unsigned *g_status_ptr[kMaxDevices] = {nullptr};
+using rtq::DevCtl;
+using rtq::kMaxDevices;
+std::mutex g_ctl_mu;
+DevCtl *g_ctl_ptr[kMaxDevices] = {nullptr};
 
-// Device address of the status word on the current device (looked up once).
-rt_status status_word(unsigned **out) {
+// Device address of the control block on the current device (looked up once).
+rt_status ctl_block(DevCtl **out) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RT_ERR_CUDA;
-    std::lock_guard<std::mutex> lk(g_status_mu);
-    if (!g_status_ptr[dev]) {
+    if (cudaGetDevice(&dev) != cudaSuccess) return RT_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return RT_ERR_UNSUPPORTED_DEVICE;
+    std::lock_guard<std::mutex> lk(g_ctl_mu);
+    if (!g_ctl_ptr[dev]) {
         void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_rtq_device_status) != cudaSuccess) return RT_ERR_CUDA;
-        g_status_ptr[dev] = static_cast<unsigned *>(p);
+        if (cudaGetSymbolAddress(&p, g_rtq_ctl) != cudaSuccess) return RT_ERR_CUDA;
+        g_ctl_ptr[dev] = static_cast<DevCtl *>(p);
     }
-    *out = g_status_ptr[dev];
+    *out = g_ctl_ptr[dev];
     return RT_OK;
 }
 
@@ -123,7 +127,7 @@ int pick_kernel(int fmt, int64_t M, int64_t N, int64_t K, int p) {
 
 int pick_path(int64_t M, int64_t K, int path) {
     const bool tc_ok = (K % 64) == 0;
-    if (path == RT_PATH_TC || path == RT_PATH_TC_BF16) return tc_ok ? path : -1;
+    if (path == RT_PATH_TC) return tc_ok ? path : -1;
     if (path == RT_PATH_SIMT) return RT_PATH_SIMT;
     if (path != RT_PATH_AUTO) return -2;
     return (M <= rtq::kAutoSimtMaxM || !tc_ok) ? RT_PATH_SIMT : RT_PATH_TC;
@@ -149,22 +153,21 @@ rt_status run_gemm(int fmt, const float *X, const void *Wq, const void *S, float
     if (kern == RT_KERNEL_SIMT)
         return from_cuda(q4 ? rtq::launch_simt_q4(X, w4, s4, Y, m, n, k, s)
                             : rtq::launch_simt_q8(X, w8, s8, Y, m, n, k, s));
-    unsigned *status = nullptr;
-    rt_status st = status_word(&status);
+    DevCtl *ctl = nullptr;
+    rt_status st = ctl_block(&ctl);
     if (st != RT_OK) return st;
-    const bool bf16 = p == RT_PATH_TC_BF16;
     if (kern == RT_KERNEL_TC_W_STATIONARY)
-        return from_cuda(q4 ? rtq::launch_tc_q4(X, w4, s4, Y, m, n, k, bf16, status, s)
-                            : rtq::launch_tc_q8(X, w8, s8, Y, m, n, k, bf16, status, s));
+        return from_cuda(q4 ? rtq::launch_tc_q4(X, w4, s4, Y, m, n, k, ctl, s)
+                            : rtq::launch_tc_q8(X, w8, s8, Y, m, n, k, ctl, s));
     void *xh = nullptr;
     if ((st = workspace(s, static_cast<size_t>(M) * K * 2, &xh)) != RT_OK) return st;
-    cudaError_t e = rtq::launch_cvt_x16(X, xh, M, K, bf16, s);
+    cudaError_t e = rtq::launch_cvt_x16(X, xh, M, K, ctl, s);
     if (e != cudaSuccess) return RT_ERR_CUDA;
     if (kern == RT_KERNEL_TC_X_RESIDENT)
-        return from_cuda(q4 ? rtq::launch_xs_q4(xh, w4, s4, Y, m, n, k, bf16, status, s)
-                            : rtq::launch_xs_q8(xh, w8, s8, Y, m, n, k, bf16, status, s));
-    return from_cuda(q4 ? rtq::launch_ws_q4(xh, w4, s4, Y, m, n, k, bf16, status, s)
-                        : rtq::launch_ws_q8(xh, w8, s8, Y, m, n, k, bf16, status, s));
+        return from_cuda(q4 ? rtq::launch_xs_q4(xh, w4, s4, Y, m, n, k, ctl, s)
+                            : rtq::launch_xs_q8(xh, w8, s8, Y, m, n, k, ctl, s));
+    return from_cuda(q4 ? rtq::launch_ws_q4(xh, w4, s4, Y, m, n, k, ctl, s)
+                        : rtq::launch_ws_q8(xh, w8, s8, Y, m, n, k, ctl, s));
 }
 
 }  // namespace
@@ -179,7 +182,7 @@ rt_status check_gemm_args(int fmt, const float *X, const void *Wq, const void *S
                     : validate(X, Wq, S, Y, M, N, K, N * K, N * 4, 4, 16);
 }
 
-rt_status device_status_word(unsigned **out) { return status_word(out); }
+rt_status device_ctl(DevCtl **out) { return ctl_block(out); }
 
 }  // namespace rtq
 
@@ -196,11 +199,13 @@ const char *rt_status_string(int status) {
         case RT_ERR_VALUE_RANGE: return "value out of range";
         case RT_ERR_WORKSPACE: return "workspace must grow during stream capture";
         case RT_ERR_SCRATCH_LIMIT: return "problem needs more than the fixed scratch array holds";
+        case RT_ERR_OPERAND_RANGE: return "an activation is not a finite fp16 value";
+        case RT_ERR_UNSUPPORTED_DEVICE: return "device index beyond the library's limit";
         default: return "unknown status";
     }
 }
 
-int rt_version(void) { return 100; }
+int rt_version(void) { return 200; }
 
 int rt_qgemm_auto_path(int fmt, int64_t M, int64_t N, int64_t K) {
     if ((fmt != 4 && fmt != 8) || M < 0 || N < 1 || K < 1) return -1;
@@ -317,14 +322,13 @@ rt_status rt_qblock_project(const rt_qblock *blk, int64_t M, const float *X_qkvg
         }
     }
     if (rt_qblock_fused(M, d, f, path) == 1) {
-        unsigned *status = nullptr;
-        if ((st = status_word(&status)) != RT_OK) return st;
+        DevCtl *ctl = nullptr;
+        if ((st = ctl_block(&ctl)) != RT_OK) return st;
         rtq::GroupProblem g[4];
         for (int i = 0; i < 4; ++i)
             g[i] = {p[i].X, p[i].W, p[i].S, p[i].Y, static_cast<int>(p[i].N),
                     static_cast<int>(p[i].K), p[i].fmt};
-        return from_cuda(rtq::launch_tc_group(g, 4, static_cast<int>(M),
-                                              pick_path(M, d, path) == RT_PATH_TC_BF16, status,
+        return from_cuda(rtq::launch_tc_group(g, 4, static_cast<int>(M), ctl,
                                               static_cast<cudaStream_t>(stream)));
     }
     for (const Proj &q : p)
@@ -360,39 +364,48 @@ rt_status rt_dequant_q8_f32(const int8_t *Wq, const float *scale, float *W_out, 
                                                 static_cast<cudaStream_t>(stream)));
 }
 
-rt_status rt_dequant_q4_bf16(const uint8_t *Wq, const uint16_t *scale_min, uint16_t *W_out,
-                             int64_t N, int64_t K, void *stream) {
-    rt_status st = validate_dequant(Wq, scale_min, W_out, N, K, 32, 4);
-    if (st != RT_OK) return st;
-    return from_cuda(rtq::launch_dequant_q4_16(Wq, scale_min, W_out, static_cast<int>(N),
-                                               static_cast<int>(K), true,
-                                               static_cast<cudaStream_t>(stream)));
-}
-
 rt_status rt_dequant_q4_f16(const uint8_t *Wq, const uint16_t *scale_min, uint16_t *W_out,
                             int64_t N, int64_t K, void *stream) {
     rt_status st = validate_dequant(Wq, scale_min, W_out, N, K, 32, 4);
     if (st != RT_OK) return st;
-    return from_cuda(rtq::launch_dequant_q4_16(Wq, scale_min, W_out, static_cast<int>(N),
-                                               static_cast<int>(K), false,
-                                               static_cast<cudaStream_t>(stream)));
+    return from_cuda(rtq::launch_dequant_q4_f16(Wq, scale_min, W_out, static_cast<int>(N),
+                                                static_cast<int>(K),
+                                                static_cast<cudaStream_t>(stream)));
 }
 
 rt_status rt_device_status(void *stream, int *device_status) {
     if (!device_status) return RT_ERR_INVALID_ARG;
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return RT_ERR_CUDA;
-    unsigned *p = nullptr;
-    rt_status st = status_word(&p);
+    DevCtl *ctl = nullptr;
+    rt_status st = ctl_block(&ctl);
     if (st != RT_OK) return st;
     unsigned v = 0;
-    if (cudaMemcpy(&v, p, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return RT_ERR_CUDA;
+    if (cudaMemcpy(&v, &ctl->status, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return RT_ERR_CUDA;
     if (v != 0) {
         const unsigned zero = 0;
-        if (cudaMemcpy(p, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess)
+        if (cudaMemcpy(&ctl->status, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess)
             return RT_ERR_CUDA;
     }
-    *device_status = v ? RT_ERR_DEVICE_TIMEOUT : RT_OK;
+    *device_status = (v & (1u << rtq::kStatusTimeout))  ? RT_ERR_DEVICE_TIMEOUT
+                     : (v & (1u << rtq::kStatusRange)) ? RT_ERR_OPERAND_RANGE
+                                                       : RT_OK;
+    return RT_OK;
+}
+
+rt_status rt_debug_inject(int mode, int64_t wait_ns) {
+    if (mode < 0 || mode > 1 || wait_ns < 0) return RT_ERR_INVALID_ARG;
+    DevCtl *ctl = nullptr;
+    rt_status st = ctl_block(&ctl);
+    if (st != RT_OK) return st;
+    if (cudaDeviceSynchronize() != cudaSuccess) return RT_ERR_CUDA;
+    const unsigned inject = static_cast<unsigned>(mode);
+    const unsigned long long ns =
+        wait_ns == 0 ? rtq::kWaitLimitNs : static_cast<unsigned long long>(wait_ns);
+    if (cudaMemcpy(&ctl->inject, &inject, sizeof inject, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(&ctl->wait_ns, &ns, sizeof ns, cudaMemcpyHostToDevice) != cudaSuccess)
+        return RT_ERR_CUDA;
     return RT_OK;
 }
 

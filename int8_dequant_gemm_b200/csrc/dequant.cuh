@@ -10,9 +10,8 @@
 //   times 11-bit significands), so one fmaf yields the exact value rounded
 //   once to fp32.
 // q8 ("RT-J -- int8 ... quantized checkpoints", "Quantization format"):
-//   W = q * scale[o]; q (|q| <= 127) is exact in fp32 and in bf16.
+//   W = q * scale[o]; q (|q| <= 127) is exact in fp32 and in fp16.
 #pragma once
-#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cstdint>
 
@@ -37,34 +36,27 @@ __device__ __forceinline__ void q4_word_f32(uint32_t v, float scale, float mn, f
     for (int i = 0; i < 8; ++i) w[i] = fmaf(small_uint_to_f32((v >> (4 * i)) & 0xFu), scale, mn);
 }
 
-// Tensor-core operand types: both MMA operands share one 16-bit type.
-enum class Op16 { f16 = 0, bf16 = 1 };
-
 // Tensor-core operand chunks hold 8 consecutive K elements in the pair order
 // [0,2 | 1,3 | 4,6 | 5,7] (one 32-bit word per pair).  Weights and
 // activations use the same order, so the MMA's dot products are unchanged;
 // the order lets each pair come from one byte pair of the packed codes and
-// from one float4 of the activations.
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t *>(&h);
-}
-
+// from one float4 of the activations.  Both operands are fp16.
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
-// Two fp32 values -> two 16-bit operands (round to nearest-even), low first.
-template <Op16 OP>
-__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
-    return OP == Op16::f16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
+// 4 activations (k, k+1, k+2, k+3) -> the two fp16 pair words (k,k+2),
+// (k+1,k+3), rounded to nearest-even.
+__device__ __forceinline__ uint2 x4_f16(float4 a) {
+    return make_uint2(pack_f16x2(a.x, a.z), pack_f16x2(a.y, a.w));
 }
 
-// 4 activations (k, k+1, k+2, k+3) -> the two pair words (k,k+2), (k+1,k+3).
-template <Op16 OP>
-__device__ __forceinline__ uint2 x4_op(float4 a) {
-    return make_uint2(pack2<OP>(a.x, a.z), pack2<OP>(a.y, a.w));
+// Non-zero where a half of an fp16 pair word is infinite or NaN (exponent
+// field all ones): an activation that fp16 cannot hold (|x| >= 65520 rounds
+// to infinity) or that was not finite to begin with.
+__device__ __forceinline__ uint32_t f16x2_nonfinite(uint2 w) {
+    return __vcmpeq2(w.x & 0x7C007C00u, 0x7C007C00u) | __vcmpeq2(w.y & 0x7C007C00u, 0x7C007C00u);
 }
 
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
@@ -95,14 +87,6 @@ __device__ __forceinline__ void q4_scale_min_f16x2(uint32_t sm, uint32_t &s2, ui
     m2 = __byte_perm(sm, 0u, 0x3232);
 }
 
-// q4, bf16 operands: the fp32 value rounded to bf16, same chunk order.
-__device__ __forceinline__ uint4 q4_word_bf16(uint32_t v, float scale, float mn) {
-    float w[8];
-    q4_word_f32(v, scale, mn, w);
-    return make_uint4(pack_bf16x2(w[0], w[2]), pack_bf16x2(w[1], w[3]), pack_bf16x2(w[4], w[6]),
-                      pack_bf16x2(w[5], w[7]));
-}
-
 // int8 code (byte i of v, two's complement) -> fp32, exact.
 __device__ __forceinline__ float q8_byte_f32(uint32_t v, int i) {
     // offset-binary byte (q + 128) in 0..255, then remove 2^23 + 128 exactly
@@ -120,14 +104,6 @@ __device__ __forceinline__ uint4 q8_words_f16(uint32_t a, uint32_t b) {
                       h2_bits(__hsub2(bits_h2(__byte_perm(ua, 0x64646464u, 0x4341)), k1152)),
                       h2_bits(__hsub2(bits_h2(__byte_perm(ub, 0x64646464u, 0x4240)), k1152)),
                       h2_bits(__hsub2(bits_h2(__byte_perm(ub, 0x64646464u, 0x4341)), k1152)));
-}
-
-// q8, bf16 operands (exact: |q| <= 128 has at most 8 significant bits).
-__device__ __forceinline__ uint4 q8_words_bf16(uint32_t a, uint32_t b) {
-    return make_uint4(pack_bf16x2(q8_byte_f32(a, 0), q8_byte_f32(a, 2)),
-                      pack_bf16x2(q8_byte_f32(a, 1), q8_byte_f32(a, 3)),
-                      pack_bf16x2(q8_byte_f32(b, 0), q8_byte_f32(b, 2)),
-                      pack_bf16x2(q8_byte_f32(b, 1), q8_byte_f32(b, 3)));
 }
 
 // Chunk in operand order -> natural order (for the dequantization exports).

@@ -1,11 +1,47 @@
-// Launchers of the device kernels, called only by the C ABI layer (api.cu).
+// Launchers of the device kernels, called only by the C ABI layer (api.cu,
+// noalloc.cu), and the per-device control block the tensor-core kernels read.
 #pragma once
 #include <cuda_runtime.h>
+
+#include <atomic>
 #include <cstdint>
 
 #include "../../include/rtq.h"
 
 namespace rtq {
+
+constexpr int kMaxDevices = 64;
+
+// Per-device control block, one __device__ instance (api.cu).  Every
+// tensor-core kernel reads `wait_ns` and `inject` at its start and ORs status
+// bits into `status`; rt_device_status() reads and clears the bits.
+//   status  bit kStatusTimeout: a bounded mbarrier wait gave up;
+//           bit kStatusRange:   an activation was not a finite fp16 value
+//                               after rounding (|x| >= 65520, inf or NaN).
+//   inject  test hook (rt_debug_inject): 1 makes the first producer arrival
+//           of every CTA go missing, so a consumer's bounded wait runs out;
+//           0 in normal operation.
+//   wait_ns bound of every mbarrier wait (default kWaitLimitNs, 2 s).
+struct DevCtl {
+    unsigned status;
+    unsigned inject;
+    unsigned long long wait_ns;
+};
+constexpr unsigned kStatusTimeout = 5u;
+constexpr unsigned kStatusRange = 6u;
+
+// Raises `kernel`'s dynamic shared-memory limit to `bytes` on device `dev`,
+// once per device.  cudaFuncSetAttribute is idempotent, so two host threads
+// that both see the flag clear only repeat the call.
+template <typename Kernel>
+cudaError_t smem_attr_once(Kernel kernel, int bytes, int dev, std::atomic<bool> (&done)[kMaxDevices]) {
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    const cudaError_t e =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done[dev].store(true, std::memory_order_release);
+    return e;
+}
 
 // fp32 CUDA-core path: one thread per output row, MT activation rows per block.
 cudaError_t launch_simt_q4(const float *X, const uint8_t *Wq, const uint16_t *SM, float *Y,
@@ -13,12 +49,12 @@ cudaError_t launch_simt_q4(const float *X, const uint8_t *Wq, const uint16_t *SM
 cudaError_t launch_simt_q8(const float *X, const int8_t *Wq, const float *S, float *Y, int M,
                            int N, int K, cudaStream_t s);
 
-// tcgen05 path: 128 weight rows x BN activation rows per CTA, fp16 (or bf16)
-// operands in swizzled shared memory, fp32 accumulator in TMEM.
+// tcgen05 path: 128 weight rows x BN activation rows per CTA, fp16 operands
+// in swizzled shared memory, fp32 accumulator in TMEM.
 cudaError_t launch_tc_q4(const float *X, const uint8_t *Wq, const uint16_t *SM, float *Y, int M,
-                         int N, int K, bool bf16, unsigned *status, cudaStream_t s);
+                         int N, int K, DevCtl *ctl, cudaStream_t s);
 cudaError_t launch_tc_q8(const float *X, const int8_t *Wq, const float *S, float *Y, int M, int N,
-                         int K, bool bf16, unsigned *status, cudaStream_t s);
+                         int K, DevCtl *ctl, cudaStream_t s);
 
 // Up to kMaxGroup independent projections with the same M (1..128) in one
 // launch of the same tcgen05 tile code: X [M, K] fp32, Wq/S as for
@@ -32,12 +68,13 @@ struct GroupProblem {
     float *Y;
     int N, K, fmt;
 };
-cudaError_t launch_tc_group(const GroupProblem *probs, int count, int M, bool bf16,
-                            unsigned *status, cudaStream_t s);
+cudaError_t launch_tc_group(const GroupProblem *probs, int count, int M, DevCtl *ctl,
+                            cudaStream_t s);
 
 // Activation pre-pass of the TMA-fed kernels (prep.cu): X fp32 [M, K] ->
-// 16-bit [M, K] in the operand chunk order, into Xh (M * K * 2 bytes).
-cudaError_t launch_cvt_x16(const float *X, void *Xh, int64_t M, int64_t K, bool bf16,
+// fp16 [M, K] in the operand chunk order, into Xh (M * K * 2 bytes); latches
+// kStatusRange for an activation fp16 cannot hold.
+cudaError_t launch_cvt_x16(const float *X, void *Xh, int64_t M, int64_t K, DevCtl *ctl,
                            cudaStream_t s);
 
 // tcgen05, activation block resident in shared memory, TMA-streamed weights
@@ -45,31 +82,31 @@ cudaError_t launch_cvt_x16(const float *X, void *Xh, int64_t M, int64_t K, bool 
 // pre-pass output.
 bool xs_supported(int M, int N, int K);
 cudaError_t launch_xs_q4(const void *Xh, const uint8_t *Wq, const uint16_t *SM, float *Y, int M,
-                         int N, int K, bool bf16, unsigned *status, cudaStream_t s);
+                         int N, int K, DevCtl *ctl, cudaStream_t s);
 cudaError_t launch_xs_q8(const void *Xh, const int8_t *Wq, const float *S, float *Y, int M, int N,
-                         int K, bool bf16, unsigned *status, cudaStream_t s);
+                         int K, DevCtl *ctl, cudaStream_t s);
 
 // tcgen05, persistent weight-stationary tiles with both operands TMA-staged
 // (more than 128 activation rows, any K of the format's TMA granule); see ws.cu.
 bool ws_supported(int fmt, int M, int N, int K);
 cudaError_t launch_ws_q4(const void *Xh, const uint8_t *Wq, const uint16_t *SM, float *Y, int M,
-                         int N, int K, bool bf16, unsigned *status, cudaStream_t s);
+                         int N, int K, DevCtl *ctl, cudaStream_t s);
 cudaError_t launch_ws_q8(const void *Xh, const int8_t *Wq, const float *S, float *Y, int M, int N,
-                         int K, bool bf16, unsigned *status, cudaStream_t s);
+                         int K, DevCtl *ctl, cudaStream_t s);
 
 // dequantization exports (same __device__ routines as the GEMMs)
 cudaError_t launch_dequant_q4_f32(const uint8_t *Wq, const uint16_t *SM, float *W, int N, int K,
                                   cudaStream_t s);
-cudaError_t launch_dequant_q4_16(const uint8_t *Wq, const uint16_t *SM, uint16_t *W, int N,
-                                 int K, bool bf16, cudaStream_t s);
+cudaError_t launch_dequant_q4_f16(const uint8_t *Wq, const uint16_t *SM, uint16_t *W, int N,
+                                  int K, cudaStream_t s);
 cudaError_t launch_dequant_q8_f32(const int8_t *Wq, const float *S, float *W, int N, int K,
                                   cudaStream_t s);
 
-// Argument checks of rt_qgemm_q4 / rt_qgemm_q8 (fmt 4 / 8) and the device
-// status word the tensor-core kernels latch timeouts into (api.cu).
+// Argument checks of rt_qgemm_q4 / rt_qgemm_q8 (fmt 4 / 8) and the control
+// block of the current device (api.cu).
 rt_status check_gemm_args(int fmt, const float *X, const void *Wq, const void *S, const float *Y,
                           int64_t M, int64_t N, int64_t K);
-rt_status device_status_word(unsigned **out);
+rt_status device_ctl(DevCtl **out);
 
 // Largest M the SIMT path takes under RT_PATH_AUTO.
 constexpr int kAutoSimtMaxM = 8;

@@ -24,7 +24,7 @@ static __device__ __align__(256) unsigned char g_rtq_noalloc_scratch[RT_NOALLOC_
 
 namespace {
 
-constexpr int kMaxDevices = 64;
+using rtq::kMaxDevices;
 std::mutex g_scratch_mu;
 void *g_scratch_ptr[kMaxDevices] = {nullptr};
 
@@ -33,7 +33,8 @@ void *g_scratch_ptr[kMaxDevices] = {nullptr};
 // come before any stream capture.
 rt_status scratch_ptr(void **out) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RT_ERR_CUDA;
+    if (cudaGetDevice(&dev) != cudaSuccess) return RT_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return RT_ERR_UNSUPPORTED_DEVICE;
     std::lock_guard<std::mutex> lk(g_scratch_mu);
     if (!g_scratch_ptr[dev]) {
         void *p = nullptr;
@@ -54,7 +55,7 @@ extern "C" rt_status rt_qgemm_noalloc(int fmt, const float *X, const void *Wq, c
     if (fmt != 4 && fmt != 8) return RT_ERR_INVALID_ARG;
     rt_status st = rtq::check_gemm_args(fmt, X, Wq, scales, Y, M, N, K);
     if (st != RT_OK) return st;
-    if (path < RT_PATH_AUTO || path > RT_PATH_TC_BF16) return RT_ERR_INVALID_ARG;
+    if (path < RT_PATH_AUTO || path > RT_PATH_TC) return RT_ERR_INVALID_ARG;
     const int kern = rt_qgemm_plan(fmt, M, N, K, path);
     if (kern < 0) return RT_ERR_UNSUPPORTED_SHAPE;
     const bool staged = kern == RT_KERNEL_TC_X_RESIDENT || kern == RT_KERNEL_TC_W_STREAMED;
@@ -74,16 +75,15 @@ extern "C" rt_status rt_qgemm_noalloc(int fmt, const float *X, const void *Wq, c
     if (kern == RT_KERNEL_SIMT)
         return from_cuda(q4 ? rtq::launch_simt_q4(X, w4, s4, Y, m, n, k, s)
                             : rtq::launch_simt_q8(X, w8, s8, Y, m, n, k, s));
-    unsigned *status = nullptr;
-    if ((st = rtq::device_status_word(&status)) != RT_OK) return st;
-    const bool bf16 = path == RT_PATH_TC_BF16;
+    rtq::DevCtl *ctl = nullptr;
+    if ((st = rtq::device_ctl(&ctl)) != RT_OK) return st;
     if (kern == RT_KERNEL_TC_W_STATIONARY)
-        return from_cuda(q4 ? rtq::launch_tc_q4(X, w4, s4, Y, m, n, k, bf16, status, s)
-                            : rtq::launch_tc_q8(X, w8, s8, Y, m, n, k, bf16, status, s));
-    if (rtq::launch_cvt_x16(X, xh, M, K, bf16, s) != cudaSuccess) return RT_ERR_CUDA;
+        return from_cuda(q4 ? rtq::launch_tc_q4(X, w4, s4, Y, m, n, k, ctl, s)
+                            : rtq::launch_tc_q8(X, w8, s8, Y, m, n, k, ctl, s));
+    if (rtq::launch_cvt_x16(X, xh, M, K, ctl, s) != cudaSuccess) return RT_ERR_CUDA;
     if (kern == RT_KERNEL_TC_X_RESIDENT)
-        return from_cuda(q4 ? rtq::launch_xs_q4(xh, w4, s4, Y, m, n, k, bf16, status, s)
-                            : rtq::launch_xs_q8(xh, w8, s8, Y, m, n, k, bf16, status, s));
-    return from_cuda(q4 ? rtq::launch_ws_q4(xh, w4, s4, Y, m, n, k, bf16, status, s)
-                        : rtq::launch_ws_q8(xh, w8, s8, Y, m, n, k, bf16, status, s));
+        return from_cuda(q4 ? rtq::launch_xs_q4(xh, w4, s4, Y, m, n, k, ctl, s)
+                            : rtq::launch_xs_q8(xh, w8, s8, Y, m, n, k, ctl, s));
+    return from_cuda(q4 ? rtq::launch_ws_q4(xh, w4, s4, Y, m, n, k, ctl, s)
+                        : rtq::launch_ws_q8(xh, w8, s8, Y, m, n, k, ctl, s));
 }

@@ -1,12 +1,13 @@
 // Activation pre-pass of the TMA-fed tensor-core kernels, and the TMA map
 // encoder they share.
 //
-// The pre-pass rounds X (fp32 [M, K]) once to the 16-bit operand type and
-// stores it in the chunk order the MMA operands use (pairs [0,2 | 1,3 | 4,6 |
-// 5,7] within every 8 elements, see dequant.cuh).  The GEMM kernels then
-// load activation tiles with TMA straight into the 128-byte-swizzled
-// operand layout, with no conversion work and at half the bytes of fp32.
-// It is a pure streaming kernel: 4 bytes read and 2 written per element.
+// The pre-pass rounds X (fp32 [M, K]) once to fp16 and stores it in the chunk
+// order the MMA operands use (pairs [0,2 | 1,3 | 4,6 | 5,7] within every 8
+// elements, see dequant.cuh).  The GEMM kernels then load activation tiles
+// with TMA straight into the 128-byte-swizzled operand layout, with no
+// conversion work and at half the bytes of fp32.  It is a pure streaming
+// kernel: 4 bytes read and 2 written per element.  An activation that is not
+// a finite fp16 value after rounding latches kStatusRange.
 #include <algorithm>
 #include <mutex>
 
@@ -16,23 +17,27 @@
 namespace rtq {
 namespace {
 
-template <Op16 OP>
 __global__ void __launch_bounds__(256)
-    cvt_x16_kernel(const float4 *__restrict__ X, uint4 *__restrict__ Xh, int64_t n_chunks) {
+    cvt_x16_kernel(const float4 *__restrict__ X, uint4 *__restrict__ Xh, int64_t n_chunks,
+                   DevCtl *ctl) {
     pdl_wait_prior_grid();
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    uint32_t bad = 0;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_chunks;
          i += stride) {
         const float4 a = __ldcs(X + 2 * i), b = __ldcs(X + 2 * i + 1);
-        const uint2 lo = x4_op<OP>(a), hi = x4_op<OP>(b);
+        const uint2 lo = x4_f16(a), hi = x4_f16(b);
+        bad |= f16x2_nonfinite(lo) | f16x2_nonfinite(hi);
         Xh[i] = make_uint4(lo.x, lo.y, hi.x, hi.y);
     }
+    if (__any_sync(0xffffffffu, bad != 0) && (threadIdx.x & 31) == 0)
+        atomicOr(&ctl->status, 1u << kStatusRange);
     pdl_launch_dependents();
 }
 
 }  // namespace
 
-cudaError_t launch_cvt_x16(const float *X, void *Xh, int64_t M, int64_t K, bool bf16,
+cudaError_t launch_cvt_x16(const float *X, void *Xh, int64_t M, int64_t K, DevCtl *ctl,
                            cudaStream_t s) {
     const int64_t n_chunks = M * K / 8;
     int dev = 0, sms = 148;
@@ -50,8 +55,7 @@ cudaError_t launch_cvt_x16(const float *X, void *Xh, int64_t M, int64_t K, bool 
     cfg.numAttrs = 1;
     const float4 *x4 = reinterpret_cast<const float4 *>(X);
     uint4 *h = static_cast<uint4 *>(Xh);
-    return bf16 ? cudaLaunchKernelEx(&cfg, cvt_x16_kernel<Op16::bf16>, x4, h, n_chunks)
-                : cudaLaunchKernelEx(&cfg, cvt_x16_kernel<Op16::f16>, x4, h, n_chunks);
+    return cudaLaunchKernelEx(&cfg, cvt_x16_kernel, x4, h, n_chunks, ctl);
 }
 
 namespace {

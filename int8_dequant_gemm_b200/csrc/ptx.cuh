@@ -6,8 +6,10 @@
 
 namespace rtq {
 
-// A bounded wait gives up after this many nanoseconds of %globaltimer and the
-// kernel latches RT_ERR_DEVICE_TIMEOUT instead of hanging the GPU.
+// Default bound of every mbarrier wait: a wait gives up after this many
+// nanoseconds of %globaltimer and the kernel latches RT_ERR_DEVICE_TIMEOUT
+// instead of hanging the GPU.  Kernels read the bound in force from the
+// device control block (DevCtl::wait_ns).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
@@ -50,14 +52,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Returns false when
-// kWaitLimitNs elapse first.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+// *limit_ns nanoseconds elapse first (read only once the first try fails, so
+// the bound occupies no register on the fast path).
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
+                                          const unsigned long long *limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
+    const uint64_t limit = *limit_ns;
     uint32_t n = 0;
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((++n & 255u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) return false;
+        if ((++n & 255u) == 0 && global_timer_ns() - t0 > limit) return false;
     }
 }
 
@@ -92,6 +97,12 @@ __device__ __forceinline__ float4 ld_cluster_f4(uint32_t caddr) {
                  : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
                  : "r"(caddr)
                  : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t caddr) {
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(caddr) : "memory");
     return v;
 }
 
@@ -194,7 +205,7 @@ __device__ __forceinline__ void tmem_ld_wait() {
 }
 
 // Shared-memory matrix descriptor for a K-major operand tile stored in the
-// 128-byte swizzle layout: rows of 128 bytes (64 bf16), 8-row groups of 1024
+// 128-byte swizzle layout: rows of 128 bytes (64 fp16), 8-row groups of 1024
 // bytes laid out back to back (stride-dimension offset 1024 B), leading
 // offset unused for this layout (encoded as 1), descriptor version 1 (sm_100),
 // layout type 2 = SWIZZLE_128B.  The tile base must be 1024-byte aligned; a K
@@ -211,12 +222,11 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
 }
 
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator, A and B
-// of the same 16-bit type (ab_format 0 = f16, 1 = bf16), both K-major, no
-// negation, shape M x N.
-__host__ __device__ constexpr uint32_t idesc_f16kind_f32acc(int M, int N, uint32_t ab_format) {
+// both f16 (type field 0), both K-major, no negation, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_f16_f32acc(int M, int N) {
     return (1u << 4)                                   // D: f32
-           | (ab_format << 7)                          // A type
-           | (ab_format << 10)                         // B type
+           | (0u << 7)                                 // A type: f16
+           | (0u << 10)                                // B type: f16
            | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
            | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }

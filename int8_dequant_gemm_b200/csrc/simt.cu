@@ -24,6 +24,7 @@ namespace rtq {
 namespace {
 
 constexpr int kSimtThreads = 128;                 // weight rows per CTA
+constexpr int kSimtMaxSmem = 160 * 1024;          // activations (<= 128 KB) + partials
 
 // X rows m0 .. m0 + mt - 1, columns [k0, k0 + Ks), as MT x Ks floats.
 template <int MT>
@@ -178,14 +179,16 @@ cudaError_t launch_simt_mt(bool q4, const float *X, const void *Wq, const void *
     const int ksplit = pick_simt_ksplit(M, N, K, MT);
     const size_t smem = static_cast<size_t>(MT) * (K / ksplit) * sizeof(float) +
                         (ksplit > 1 ? static_cast<size_t>(MT) * kSimtThreads * sizeof(float) : 0);
-    void *fn = q4 ? reinterpret_cast<void *>(&simt_kernel<MT, 4>)
-                  : reinterpret_cast<void *>(&simt_kernel<MT, 8>);
-    if (smem > 48 * 1024) {
-        cudaError_t e =
-            cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem));
-        if (e != cudaSuccess) return e;
-    }
+    // The limit is raised once per device to the largest size any call asks
+    // for (staged activations of at most 128 KB plus the partials), so calls
+    // from several host threads never lower it under one another.
+    static std::atomic<bool> attr_done[2][kMaxDevices];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = q4 ? smem_attr_once(simt_kernel<MT, 4>, kSimtMaxSmem, dev, attr_done[0])
+           : smem_attr_once(simt_kernel<MT, 8>, kSimtMaxSmem, dev, attr_done[1]);
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((M + MT - 1) / MT, (N + kSimtThreads - 1) / kSimtThreads, ksplit);
     cfg.blockDim = dim3(kSimtThreads, 1, 1);
@@ -240,31 +243,20 @@ __global__ void dequant_q4_f32_kernel(const uint8_t *__restrict__ Wq,
     }
 }
 
-template <Op16 OP>
-__global__ void dequant_q4_16_kernel(const uint8_t *__restrict__ Wq,
-                                       const uint32_t *__restrict__ SM, uint16_t *__restrict__ W,
-                                       int N, int K) {
+__global__ void dequant_q4_f16_kernel(const uint8_t *__restrict__ Wq,
+                                      const uint32_t *__restrict__ SM, uint16_t *__restrict__ W,
+                                      int N, int K) {
     const int G = K / 32;
     const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (idx >= static_cast<int64_t>(N) * G) return;
     const int64_t o = idx / G, g = idx % G;
     const uint4 p = ldg_nc_v4(Wq + o * (K / 2) + g * 16);
-    float sc, mn;
-    q4_scale_min(__ldg(SM + o * G + g), sc, mn);
+    uint32_t s2, m2;
+    q4_scale_min_f16x2(__ldg(SM + o * G + g), s2, m2);
     const uint32_t words[4] = {p.x, p.y, p.z, p.w};
     uint4 *dst = reinterpret_cast<uint4 *>(W + o * K + g * 32);
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        uint4 chunk;
-        if (OP == Op16::f16) {
-            uint32_t s2, m2;
-            q4_scale_min_f16x2(__ldg(SM + o * G + g), s2, m2);
-            chunk = q4_word_f16(words[c], s2, m2);
-        } else {
-            chunk = q4_word_bf16(words[c], sc, mn);
-        }
-        dst[c] = chunk_to_natural(chunk);
-    }
+    for (int c = 0; c < 4; ++c) dst[c] = chunk_to_natural(q4_word_f16(words[c], s2, m2));
 }
 
 __global__ void dequant_q8_f32_kernel(const int8_t *__restrict__ Wq, const float *__restrict__ S,
@@ -309,14 +301,11 @@ cudaError_t launch_dequant_q4_f32(const uint8_t *Wq, const uint16_t *SM, float *
     return cudaGetLastError();
 }
 
-cudaError_t launch_dequant_q4_16(const uint8_t *Wq, const uint16_t *SM, uint16_t *W, int N,
-                                 int K, bool bf16, cudaStream_t s) {
+cudaError_t launch_dequant_q4_f16(const uint8_t *Wq, const uint16_t *SM, uint16_t *W, int N,
+                                  int K, cudaStream_t s) {
     const int64_t n = static_cast<int64_t>(N) * (K / 32);
     const uint32_t *sm = reinterpret_cast<const uint32_t *>(SM);
-    if (bf16)
-        dequant_q4_16_kernel<Op16::bf16><<<blocks_for(n, 256), 256, 0, s>>>(Wq, sm, W, N, K);
-    else
-        dequant_q4_16_kernel<Op16::f16><<<blocks_for(n, 256), 256, 0, s>>>(Wq, sm, W, N, K);
+    dequant_q4_f16_kernel<<<blocks_for(n, 256), 256, 0, s>>>(Wq, sm, W, N, K);
     return cudaGetLastError();
 }
 

@@ -8,12 +8,15 @@
 // the instruction at full height.  The fp32 accumulator lives in TMEM: lane i
 // holds weight row o0 + i, column j holds activation row m0 + j.
 //
-// Operands are fp16 by default (q4 weights: the exact code*scale+min rounded
-// once by fma.rn.f16x2; q8 codes exact; activations rounded to nearest-even)
-// or bf16 on request; both use tcgen05.mma kind::f16 at the same rate.  fp16
-// keeps 11 significant bits against bf16's 8, at the price of the fp16 range
-// (|X| <= 65504).  Within every 8-element K chunk both operands store their
-// pairs in the order [0,2 | 1,3 | 4,6 | 5,7] (see dequant.cuh).
+// Operands are fp16 (q4 weights: the exact code*scale+min rounded once by
+// fma.rn.f16x2; q8 codes exact; activations rounded to nearest-even) in
+// tcgen05.mma kind::f16.  fp16 keeps 11 significant bits, at the price of the
+// fp16 range: an activation that rounds to infinity (|x| >= 65520) or is not
+// finite makes its outputs infinite or NaN, and the epilogue latches
+// kStatusRange in the device control block for any output that is not finite
+// (finite fp16 operands cannot overflow an fp32 sum of K <= 2^20 products).  Within every
+// 8-element K chunk both operands store their pairs in the order
+// [0,2 | 1,3 | 4,6 | 5,7] (see dequant.cuh).
 //
 // One CTA = 8 converter warps + 1 MMA warp.  Per 64-wide K step the converter
 // warps
@@ -37,7 +40,10 @@
 // overlaps the other's main loop.
 //
 // Every mbarrier wait is bounded; a wait that gives up latches
-// RT_ERR_DEVICE_TIMEOUT in the device status word and the CTA winds down.
+// RT_ERR_DEVICE_TIMEOUT in the device status word and the CTA winds down: the
+// MMA thread waits (bounded) for the MMAs it issued before TMEM is released,
+// and with split K no CTA of the cluster stores a tile that any of its CTAs
+// failed to finish.
 //
 // The same tile code also runs as a grouped launch (tc_group_kernel): up to
 // four independent projections with one activation tile each, e.g. a block's
@@ -63,7 +69,6 @@ constexpr int kMaxSmem = 227 * 1024;
 constexpr int kTwoCtaSmem = 110 * 1024;          // budget that lets two CTAs share an SM
 constexpr int kSmemPerSm = 228 * 1024;           // shared memory of one SM
 constexpr int kSmemReserve = 1024;               // the runtime's reservation per CTA
-constexpr unsigned kStatusTimeout = 5u;          // RT_ERR_DEVICE_TIMEOUT
 
 __host__ __device__ inline int tc_stage_bytes(int bn) { return kAStageBytes + bn * 128; }
 
@@ -76,7 +81,8 @@ __host__ __device__ inline int tc_region_bytes(int bn, int stages, int ksplit) {
 }
 
 __host__ __device__ inline int tc_smem_bytes(int bn, int stages, int ksplit) {
-    return 1024 + tc_region_bytes(bn, stages, ksplit) + (2 * stages + 1) * 8 + 16;
+    // full/empty per stage, done, drain, TMEM address + CTA-ok flag
+    return 1024 + tc_region_bytes(bn, stages, ksplit) + (2 * stages + 2) * 8 + 16;
 }
 
 __host__ __device__ inline uint32_t tmem_cols_for(int bn) {
@@ -173,41 +179,32 @@ __device__ __forceinline__ void sts_v2(uint32_t saddr, uint2 v) {
     asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(saddr), "r"(v.x), "r"(v.y) : "memory");
 }
 
-template <int FMT, Op16 OP, int PIECES>
+// Converts one K step held in R and stores it into the stage at sA (weights)
+// and sB (activations).
+template <int FMT, int PIECES>
 __device__ __forceinline__ void store_stage(const StageRegs<PIECES> &R, const ConvThread &c,
                                             uint32_t sA, uint32_t sB, int BN) {
     if (FMT == 4) {
-        if (OP == Op16::f16) {
-            uint32_t s2, m2;
-            q4_scale_min_f16x2(R.a1.x, s2, m2);
-            sts_v4(sA + c.a_off[0], q4_word_f16(R.a0.x, s2, m2));
-            sts_v4(sA + c.a_off[1], q4_word_f16(R.a0.y, s2, m2));
-            sts_v4(sA + c.a_off[2], q4_word_f16(R.a0.z, s2, m2));
-            sts_v4(sA + c.a_off[3], q4_word_f16(R.a0.w, s2, m2));
-        } else {
-            float sc, mn;
-            q4_scale_min(R.a1.x, sc, mn);
-            sts_v4(sA + c.a_off[0], q4_word_bf16(R.a0.x, sc, mn));
-            sts_v4(sA + c.a_off[1], q4_word_bf16(R.a0.y, sc, mn));
-            sts_v4(sA + c.a_off[2], q4_word_bf16(R.a0.z, sc, mn));
-            sts_v4(sA + c.a_off[3], q4_word_bf16(R.a0.w, sc, mn));
-        }
+        uint32_t s2, m2;
+        q4_scale_min_f16x2(R.a1.x, s2, m2);
+        sts_v4(sA + c.a_off[0], q4_word_f16(R.a0.x, s2, m2));
+        sts_v4(sA + c.a_off[1], q4_word_f16(R.a0.y, s2, m2));
+        sts_v4(sA + c.a_off[2], q4_word_f16(R.a0.z, s2, m2));
+        sts_v4(sA + c.a_off[3], q4_word_f16(R.a0.w, s2, m2));
     } else {
-        if (OP == Op16::f16) {
-            sts_v4(sA + c.a_off[0], q8_words_f16(R.a0.x, R.a0.y));
-            sts_v4(sA + c.a_off[1], q8_words_f16(R.a0.z, R.a0.w));
-            sts_v4(sA + c.a_off[2], q8_words_f16(R.a1.x, R.a1.y));
-            sts_v4(sA + c.a_off[3], q8_words_f16(R.a1.z, R.a1.w));
-        } else {
-            sts_v4(sA + c.a_off[0], q8_words_bf16(R.a0.x, R.a0.y));
-            sts_v4(sA + c.a_off[1], q8_words_bf16(R.a0.z, R.a0.w));
-            sts_v4(sA + c.a_off[2], q8_words_bf16(R.a1.x, R.a1.y));
-            sts_v4(sA + c.a_off[3], q8_words_bf16(R.a1.z, R.a1.w));
-        }
+        sts_v4(sA + c.a_off[0], q8_words_f16(R.a0.x, R.a0.y));
+        sts_v4(sA + c.a_off[1], q8_words_f16(R.a0.z, R.a0.w));
+        sts_v4(sA + c.a_off[2], q8_words_f16(R.a1.x, R.a1.y));
+        sts_v4(sA + c.a_off[3], q8_words_f16(R.a1.z, R.a1.w));
     }
 #pragma unroll
     for (int i = 0; i < PIECES; ++i)
-        if (c.rb0 + 16 * i < BN) sts_v2(sB + c.b_off0 + 2048u * i, x4_op<OP>(R.b[i]));
+        if (c.rb0 + 16 * i < BN) sts_v2(sB + c.b_off0 + 2048u * i, x4_f16(R.b[i]));
+}
+
+// True for an infinite or NaN fp32 value.
+__device__ __forceinline__ bool nonfinite(float v) {
+    return (__float_as_uint(v) & 0x7F800000u) == 0x7F800000u;
 }
 
 // One CTA's work: the output tile of weight rows [o0, o0 + 128) and
@@ -216,12 +213,12 @@ __device__ __forceinline__ void store_stage(const StageRegs<PIECES> &R, const Co
 // [kbase, kbase + ksplit), which reduce their partial sums among themselves;
 // every CTA of the cluster must have the same ksplit (each reaches the
 // cluster barriers exactly when ksplit > 1).
-template <int FMT, Op16 OP, int PIECES>
+template <int FMT, int PIECES>
 __device__ __forceinline__ void tc_tile(uint8_t *smem_raw, const float *__restrict__ X,
                                         const void *__restrict__ Wq, const void *__restrict__ S,
                                         float *__restrict__ Y, int M, int N, int K, int BN,
                                         int stages, int ksplit, int o0, int m0, int kslice,
-                                        int kbase, unsigned *status) {
+                                        int kbase, DevCtl *ctl) {
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *smem = smem_raw + (base - raw);
@@ -229,8 +226,11 @@ __device__ __forceinline__ void tc_tile(uint8_t *smem_raw, const float *__restri
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + tc_region_bytes(BN, stages, ksplit));
     uint64_t *empty = full + stages;
     uint64_t *done = empty + stages;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
+    uint64_t *drain = done + 1;       // the MMA thread's own completion wait on a failed tile
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    uint32_t *cta_ok = tmem_slot + 1; // read by cluster peers before they store the tile
     const uint32_t tmem_cols = tmem_cols_for(BN);
+    const unsigned long long *lim = &ctl->wait_ns;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // split K: slice `kslice` takes K steps [kz0, kz0 + nk)
@@ -243,6 +243,7 @@ __device__ __forceinline__ void tc_tile(uint8_t *smem_raw, const float *__restri
             mbar_init(&empty[s], 1);
         }
         mbar_init(done, 1);
+        mbar_init(drain, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -277,16 +278,17 @@ __device__ __forceinline__ void tc_tile(uint8_t *smem_raw, const float *__restri
         const ConvThread ct = conv_thread(threadIdx.x);
         StageRegs<PIECES> r0, r1;
         // Converts the step held in R into stage ks % stages once the MMA has
-        // released that stage.
+        // released that stage.  (Test hook: with `inject`, thread 0 leaves out
+        // its arrival for the first step, so the MMA thread's wait runs out.)
         auto consume = [&](const StageRegs<PIECES> &R, int ks) -> bool {
             const int s = ks % stages;
             if (ks >= stages &&
-                !mbar_wait(&empty[s], static_cast<uint32_t>((ks / stages) - 1) & 1u))
+                !mbar_wait(&empty[s], static_cast<uint32_t>((ks / stages) - 1) & 1u, lim))
                 return false;
             const uint32_t sA = base + s * stage_bytes;
-            store_stage<FMT, OP, PIECES>(R, ct, sA, sA + kAStageBytes, BN);
+            store_stage<FMT, PIECES>(R, ct, sA, sA + kAStageBytes, BN);
             fence_proxy_async_smem();
-            mbar_arrive(&full[s]);
+            if (!(ks == 0 && threadIdx.x == 0 && ctl->inject)) mbar_arrive(&full[s]);
             return true;
         };
         const int kb = kz0 * kTileK;
@@ -304,9 +306,10 @@ __device__ __forceinline__ void tc_tile(uint8_t *smem_raw, const float *__restri
         }
         pdl_launch_dependents();
         // ---------------------------------------------------------- epilogue
-        if (ok) ok = mbar_wait(done, 0);
+        if (ok) ok = mbar_wait(done, 0, lim);
         // tcgen05.ld is warp-collective: the whole warp takes the epilogue or none of it
         ok = __all_sync(0xffffffffu, ok);
+        bool ybad = false;                     // an output that is not finite
         if (ok) {
             tc_fence_after_sync();
             const int q = warp & 3;            // TMEM lane quadrant of this warp
@@ -339,25 +342,33 @@ __device__ __forceinline__ void tc_tile(uint8_t *smem_raw, const float *__restri
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const int m = m0 + c + j;
-                        if (m < M) Y[static_cast<size_t>(m) * N + o] = __uint_as_float(v0[j]) * sc;
+                        if (m < M) {
+                            const float y = __uint_as_float(v0[j]) * sc;
+                            ybad |= nonfinite(y);
+                            Y[static_cast<size_t>(m) * N + o] = y;
+                        }
                     }
                     if (two) {
 #pragma unroll
                         for (int j = 0; j < 8; ++j) {
                             const int m = m0 + c + 8 + j;
-                            if (m < M)
-                                Y[static_cast<size_t>(m) * N + o] = __uint_as_float(v1[j]) * sc;
+                            if (m < M) {
+                                const float y = __uint_as_float(v1[j]) * sc;
+                                ybad |= nonfinite(y);
+                                Y[static_cast<size_t>(m) * N + o] = y;
+                            }
                         }
                     }
                 }
             }
         }
+        if (__any_sync(0xffffffffu, ybad) && lane == 0) atomicOr(&ctl->status, 1u << kStatusRange);
     } else if (lane == 0) {
         // -------------------------------------------------------- MMA issuer
-        const uint32_t idesc = idesc_f16kind_f32acc(kTileO, BN, static_cast<uint32_t>(OP));
+        const uint32_t idesc = idesc_f16_f32acc(kTileO, BN);
         for (int ks = 0; ks < nk; ++ks) {
             const int s = ks % stages;
-            if (!mbar_wait(&full[s], static_cast<uint32_t>(ks / stages) & 1u)) {
+            if (!mbar_wait(&full[s], static_cast<uint32_t>(ks / stages) & 1u, lim)) {
                 ok = false;
                 break;
             }
@@ -374,18 +385,32 @@ __device__ __forceinline__ void tc_tile(uint8_t *smem_raw, const float *__restri
             }
             tc_commit(&empty[s]);
         }
-        if (ok) tc_commit(done);
+        if (ok) {
+            tc_commit(done);
+        } else {
+            // MMAs already issued may still read the stage ring and write
+            // TMEM: wait (bounded) for them before the CTA releases either.
+            tc_commit(drain);
+            mbar_wait(drain, 0, lim);
+        }
     }
     __syncwarp();
-    if (!ok) atomicOr(status, 1u << kStatusTimeout);
+    if (!ok) atomicOr(&ctl->status, 1u << kStatusTimeout);
     tc_fence_before_sync();
-    __syncthreads();
+    const int all_ok = __syncthreads_and(ok ? 1 : 0);
     if (ksplit > 1) {
         // Every CTA of the cluster reaches both barriers on every path (a
         // timed-out wait only skips work), and a cluster's CTAs are resident
-        // together, so neither barrier can hang.
-        cluster_sync();                       // all partials written
-        if (warp < kConvWarps) {
+        // together, so neither barrier can hang.  A tile is stored only if
+        // every CTA of its K slices finished.
+        if (threadIdx.x == 0) *cta_ok = static_cast<uint32_t>(all_ok);
+        cluster_sync();                       // all partials and flags written
+        bool tile_ok = true;
+        for (int r = 0; r < ksplit; ++r)
+            tile_ok = tile_ok && ld_cluster_u32(cluster_map(smem_addr(cta_ok),
+                                                            static_cast<uint32_t>(kbase + r))) != 0;
+        if (warp < kConvWarps && tile_ok) {
+            bool ybad = false;
             // Slice s sums columns [s * BN/ksplit, (s + 1) * BN/ksplit) over
             // the tile's partials in rank order (deterministic) and stores Y.
             const int cols = BN / ksplit;
@@ -410,6 +435,8 @@ __device__ __forceinline__ void tc_tile(uint8_t *smem_raw, const float *__restri
                         for (int e = 0; e < 4; ++e)
                             if (o + e < N) a[e] *= __ldg(static_cast<const float *>(S) + o + e);
                     }
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) ybad |= o + e < N && nonfinite(a[e]);
                     float *yp = Y + static_cast<size_t>(m) * N + o;
                     if ((N & 3) == 0 && o + 3 < N) {
                         *reinterpret_cast<float4 *>(yp) = make_float4(a[0], a[1], a[2], a[3]);
@@ -420,6 +447,8 @@ __device__ __forceinline__ void tc_tile(uint8_t *smem_raw, const float *__restri
                     }
                 }
             }
+            if (__any_sync(0xffffffffu, ybad) && lane == 0)
+                atomicOr(&ctl->status, 1u << kStatusRange);
         }
         cluster_sync();                       // peers are done reading this CTA's partial
     }
@@ -429,16 +458,15 @@ __device__ __forceinline__ void tc_tile(uint8_t *smem_raw, const float *__restri
     }
 }
 
-template <int FMT, Op16 OP, int PIECES>
+template <int FMT, int PIECES>
 __global__ void __launch_bounds__(kTcThreads, 2)
     tc_qgemm_kernel(const float *__restrict__ X, const void *__restrict__ Wq,
                     const void *__restrict__ S, float *__restrict__ Y, int M, int N, int K,
-                    int BN, int stages, int ksplit, unsigned *status) {
+                    int BN, int stages, int ksplit, DevCtl *ctl) {
     extern __shared__ uint8_t smem_raw[];
-    tc_tile<FMT, OP, PIECES>(smem_raw, X, Wq, S, Y, M, N, K, BN, stages, ksplit,
-                             static_cast<int>(blockIdx.x) * kTileO,
-                             static_cast<int>(blockIdx.y) * BN, static_cast<int>(blockIdx.z), 0,
-                             status);
+    tc_tile<FMT, PIECES>(smem_raw, X, Wq, S, Y, M, N, K, BN, stages, ksplit,
+                         static_cast<int>(blockIdx.x) * kTileO, static_cast<int>(blockIdx.y) * BN,
+                         static_cast<int>(blockIdx.z), 0, ctl);
 }
 
 // Several independent projections that share M (<= BN, one activation tile)
@@ -462,10 +490,10 @@ struct TcGroup {
     int count;
 };
 
-template <Op16 OP, int PIECES>
+template <int PIECES>
 __global__ void __launch_bounds__(kTcThreads, 2)
     tc_group_kernel(const __grid_constant__ TcGroup g, int M, int BN, int stages, int csize,
-                    unsigned *status) {
+                    DevCtl *ctl) {
     extern __shared__ uint8_t smem_raw[];
     const int bx = static_cast<int>(blockIdx.x);
     int i = 0;
@@ -476,11 +504,11 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     const int o0 = tile * kTileO;
     const int kslice = r % p.ks, kbase = r - kslice;
     if (p.fmt == 4)
-        tc_tile<4, OP, PIECES>(smem_raw, p.X, p.Wq, p.S, p.Y, M, p.N, p.K, BN, stages, p.ks, o0,
-                               0, kslice, kbase, status);
+        tc_tile<4, PIECES>(smem_raw, p.X, p.Wq, p.S, p.Y, M, p.N, p.K, BN, stages, p.ks, o0, 0,
+                           kslice, kbase, ctl);
     else
-        tc_tile<8, OP, PIECES>(smem_raw, p.X, p.Wq, p.S, p.Y, M, p.N, p.K, BN, stages, p.ks, o0,
-                               0, kslice, kbase, status);
+        tc_tile<8, PIECES>(smem_raw, p.X, p.Wq, p.S, p.Y, M, p.N, p.K, BN, stages, p.ks, o0, 0,
+                           kslice, kbase, ctl);
 }
 
 // Activation rows per tile: one tile when M <= 128; otherwise 128, halved
@@ -507,19 +535,15 @@ int pick_ksplit(int M, int N, int K, int BN) {
     return ks;
 }
 
-template <int FMT, Op16 OP, int PIECES>
+template <int FMT, int PIECES>
 cudaError_t launch_tc_pieces(const float *X, const void *Wq, const void *S, float *Y, int M, int N,
-                            int K, int BN, unsigned *status, cudaStream_t st) {
-    static bool attr_set[64] = {false};
+                            int K, int BN, DevCtl *ctl, cudaStream_t st) {
+    static std::atomic<bool> attr_done[kMaxDevices];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 64 && !attr_set[dev]) {
-        e = cudaFuncSetAttribute(tc_qgemm_kernel<FMT, OP, PIECES>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
-        if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
-    }
+    if ((e = smem_attr_once(tc_qgemm_kernel<FMT, PIECES>, kMaxSmem, dev, attr_done)) != cudaSuccess)
+        return e;
     const int ksplit = pick_ksplit(M, N, K, BN);
     const int nk = K / kTileK / ksplit;
     const int budget = kTwoCtaSmem;
@@ -539,17 +563,17 @@ cudaError_t launch_tc_pieces(const float *X, const void *Wq, const void *S, floa
     attr[1].val.clusterDim.z = static_cast<unsigned>(ksplit);
     cfg.attrs = attr;
     cfg.numAttrs = ksplit > 1 ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, tc_qgemm_kernel<FMT, OP, PIECES>, X, Wq, S, Y, M, N, K, BN,
-                              stages, ksplit, status);
+    return cudaLaunchKernelEx(&cfg, tc_qgemm_kernel<FMT, PIECES>, X, Wq, S, Y, M, N, K, BN,
+                              stages, ksplit, ctl);
 }
 
-template <int FMT, Op16 OP>
+template <int FMT>
 cudaError_t launch_tc(const float *X, const void *Wq, const void *S, float *Y, int M, int N,
-                      int K, unsigned *status, cudaStream_t st) {
+                      int K, DevCtl *ctl, cudaStream_t st) {
     const int BN = pick_bn(M, N);
-    if (BN <= 32) return launch_tc_pieces<FMT, OP, 2>(X, Wq, S, Y, M, N, K, BN, status, st);
-    if (BN <= 64) return launch_tc_pieces<FMT, OP, 4>(X, Wq, S, Y, M, N, K, BN, status, st);
-    return launch_tc_pieces<FMT, OP, 8>(X, Wq, S, Y, M, N, K, BN, status, st);
+    if (BN <= 32) return launch_tc_pieces<FMT, 2>(X, Wq, S, Y, M, N, K, BN, ctl, st);
+    if (BN <= 64) return launch_tc_pieces<FMT, 4>(X, Wq, S, Y, M, N, K, BN, ctl, st);
+    return launch_tc_pieces<FMT, 8>(X, Wq, S, Y, M, N, K, BN, ctl, st);
 }
 
 // K splits for a group.  A launch lasts as long as its longest chain of K
@@ -586,18 +610,14 @@ int plan_group(TcGroup &g, int *nclusters) {
     }
 }
 
-template <Op16 OP, int PIECES>
-cudaError_t launch_group_pieces(TcGroup g, int M, int BN, unsigned *status, cudaStream_t st) {
-    static bool attr_set[64] = {false};
+template <int PIECES>
+cudaError_t launch_group_pieces(TcGroup g, int M, int BN, DevCtl *ctl, cudaStream_t st) {
+    static std::atomic<bool> attr_done[kMaxDevices];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 64 && !attr_set[dev]) {
-        e = cudaFuncSetAttribute(tc_group_kernel<OP, PIECES>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
-        if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
-    }
+    if ((e = smem_attr_once(tc_group_kernel<PIECES>, kMaxSmem, dev, attr_done)) != cudaSuccess)
+        return e;
     int nclusters = 0;
     const int csize = plan_group(g, &nclusters);
     int max_nk = 1;
@@ -619,22 +639,20 @@ cudaError_t launch_group_pieces(TcGroup g, int M, int BN, unsigned *status, cuda
     attr[1].val.clusterDim.z = static_cast<unsigned>(csize);
     cfg.attrs = attr;
     cfg.numAttrs = csize > 1 ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, tc_group_kernel<OP, PIECES>, g, M, BN, stages, csize,
-                              status);
+    return cudaLaunchKernelEx(&cfg, tc_group_kernel<PIECES>, g, M, BN, stages, csize, ctl);
 }
 
-template <Op16 OP>
-cudaError_t launch_group(const TcGroup &g, int M, unsigned *status, cudaStream_t st) {
+cudaError_t launch_group(const TcGroup &g, int M, DevCtl *ctl, cudaStream_t st) {
     const int BN = pick_bn(M, 0);
-    if (BN <= 32) return launch_group_pieces<OP, 2>(g, M, BN, status, st);
-    if (BN <= 64) return launch_group_pieces<OP, 4>(g, M, BN, status, st);
-    return launch_group_pieces<OP, 8>(g, M, BN, status, st);
+    if (BN <= 32) return launch_group_pieces<2>(g, M, BN, ctl, st);
+    if (BN <= 64) return launch_group_pieces<4>(g, M, BN, ctl, st);
+    return launch_group_pieces<8>(g, M, BN, ctl, st);
 }
 
 }  // namespace
 
-cudaError_t launch_tc_group(const GroupProblem *probs, int count, int M, bool bf16,
-                            unsigned *status, cudaStream_t s) {
+cudaError_t launch_tc_group(const GroupProblem *probs, int count, int M, DevCtl *ctl,
+                            cudaStream_t s) {
     if (count < 1 || count > kMaxGroup || M < 1 || M > kTileO) return cudaErrorInvalidValue;
     TcGroup g = {};
     g.count = count;
@@ -644,20 +662,17 @@ cudaError_t launch_tc_group(const GroupProblem *probs, int count, int M, bool bf
             return cudaErrorInvalidValue;
         g.p[i] = {q.X, q.Wq, q.S, q.Y, q.N, q.K, q.fmt, 0, 1};
     }
-    return bf16 ? launch_group<Op16::bf16>(g, M, status, s)
-                : launch_group<Op16::f16>(g, M, status, s);
+    return launch_group(g, M, ctl, s);
 }
 
 cudaError_t launch_tc_q4(const float *X, const uint8_t *Wq, const uint16_t *SM, float *Y, int M,
-                         int N, int K, bool bf16, unsigned *status, cudaStream_t s) {
-    return bf16 ? launch_tc<4, Op16::bf16>(X, Wq, SM, Y, M, N, K, status, s)
-                : launch_tc<4, Op16::f16>(X, Wq, SM, Y, M, N, K, status, s);
+                         int N, int K, DevCtl *ctl, cudaStream_t s) {
+    return launch_tc<4>(X, Wq, SM, Y, M, N, K, ctl, s);
 }
 
 cudaError_t launch_tc_q8(const float *X, const int8_t *Wq, const float *S, float *Y, int M, int N,
-                         int K, bool bf16, unsigned *status, cudaStream_t s) {
-    return bf16 ? launch_tc<8, Op16::bf16>(X, Wq, S, Y, M, N, K, status, s)
-                : launch_tc<8, Op16::f16>(X, Wq, S, Y, M, N, K, status, s);
+                         int K, DevCtl *ctl, cudaStream_t s) {
+    return launch_tc<8>(X, Wq, S, Y, M, N, K, ctl, s);
 }
 
 }  // namespace rtq

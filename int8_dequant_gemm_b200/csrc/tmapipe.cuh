@@ -117,38 +117,22 @@ __device__ __forceinline__ HalfRaw load_half_raw2(uint32_t slot, int r, int h, i
     return R;
 }
 
-// 32 weights of a half step -> 16 32-bit operand words (4 chunks).
-template <int FMT, Op16 OP>
+// 32 weights of a half step -> 16 32-bit fp16 operand words (4 chunks).
+template <int FMT>
 __device__ __forceinline__ void half_words(const HalfRaw &R, uint32_t (&w)[16]) {
     uint4 ch[4];
     if (FMT == 4) {
-        if (OP == Op16::f16) {
-            uint32_t s2, m2;
-            q4_scale_min_f16x2(R.smw, s2, m2);
-            ch[0] = q4_word_f16(R.p0.x, s2, m2);
-            ch[1] = q4_word_f16(R.p0.y, s2, m2);
-            ch[2] = q4_word_f16(R.p0.z, s2, m2);
-            ch[3] = q4_word_f16(R.p0.w, s2, m2);
-        } else {
-            float sc, mn;
-            q4_scale_min(R.smw, sc, mn);
-            ch[0] = q4_word_bf16(R.p0.x, sc, mn);
-            ch[1] = q4_word_bf16(R.p0.y, sc, mn);
-            ch[2] = q4_word_bf16(R.p0.z, sc, mn);
-            ch[3] = q4_word_bf16(R.p0.w, sc, mn);
-        }
+        uint32_t s2, m2;
+        q4_scale_min_f16x2(R.smw, s2, m2);
+        ch[0] = q4_word_f16(R.p0.x, s2, m2);
+        ch[1] = q4_word_f16(R.p0.y, s2, m2);
+        ch[2] = q4_word_f16(R.p0.z, s2, m2);
+        ch[3] = q4_word_f16(R.p0.w, s2, m2);
     } else {
-        if (OP == Op16::f16) {
-            ch[0] = q8_words_f16(R.p0.x, R.p0.y);
-            ch[1] = q8_words_f16(R.p0.z, R.p0.w);
-            ch[2] = q8_words_f16(R.p1.x, R.p1.y);
-            ch[3] = q8_words_f16(R.p1.z, R.p1.w);
-        } else {
-            ch[0] = q8_words_bf16(R.p0.x, R.p0.y);
-            ch[1] = q8_words_bf16(R.p0.z, R.p0.w);
-            ch[2] = q8_words_bf16(R.p1.x, R.p1.y);
-            ch[3] = q8_words_bf16(R.p1.z, R.p1.w);
-        }
+        ch[0] = q8_words_f16(R.p0.x, R.p0.y);
+        ch[1] = q8_words_f16(R.p0.z, R.p0.w);
+        ch[2] = q8_words_f16(R.p1.x, R.p1.y);
+        ch[3] = q8_words_f16(R.p1.z, R.p1.w);
     }
 #pragma unroll
     for (int c = 0; c < 4; ++c) {

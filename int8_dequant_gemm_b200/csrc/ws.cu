@@ -11,7 +11,7 @@
 //   A: the 128 x 64 dequantized weights in 32 TMEM columns (written with
 //      tcgen05.st by the dequantizers from TMA-staged packed codes, as in
 //      xs.cu), and
-//   B: the 128 x 64 16-bit activations in shared memory, one TMA box from the
+//   B: the 192 x 64 fp16 activations in shared memory, one TMA box from the
 //      pre-converted activations (prep.cu) in the 128-byte-swizzled operand
 //      layout.
 // The A and B rings are separate: TMEM holds two 192-column accumulators and
@@ -24,7 +24,9 @@
 // row), warp 18 activation TMA.
 //
 // Every mbarrier wait is bounded; a wait that gives up latches
-// RT_ERR_DEVICE_TIMEOUT in the device status word and the CTA winds down.
+// RT_ERR_DEVICE_TIMEOUT in the device status word and the CTA winds down: the
+// TMA threads wait (bounded) for the copies they issued, the MMA thread for the
+// MMAs it issued, before the CTA releases its shared memory and TMEM.
 #include <algorithm>
 
 #include "kernels.cuh"
@@ -62,7 +64,6 @@ constexpr uint32_t kAStageCols = kAtomK / 2;
 constexpr uint32_t kWsTmemCols = 512;
 static_assert(kAccCols + kAStages * kAStageCols <= kWsTmemCols, "TMEM budget");
 static_assert(kEpiCols % 32 == 0, "epilogue reads 32 columns at a time");
-constexpr unsigned kStatusTimeout = 5u;
 
 struct WsLayout {
     int st_off, raw_off, sc_off, bar_off, total;
@@ -75,18 +76,18 @@ __host__ __device__ inline WsLayout ws_layout() {
     L.sc_off = L.raw_off + kRaw * raw_slot_bytes(8);   // sized for the larger q8 slots
     L.bar_off = L.sc_off + 2 * kScaleSlot;
     // a_full/a_empty[kAStages], b_full/b_empty[kStages], raw_full/empty[kRaw],
-    // sc_full/empty[2], acc_full/empty[2], + TMEM address slot
-    L.total = L.bar_off + (2 * kAStages + 2 * kStages + 2 * kRaw + 4 + 4) * 8 + 16;
+    // sc_full/empty[2], acc_full/empty[2], drain, + TMEM address slot
+    L.total = L.bar_off + (2 * kAStages + 2 * kStages + 2 * kRaw + 4 + 4 + 1) * 8 + 16;
     return L;
 }
 
-template <int FMT, Op16 OP>
+template <int FMT>
 __global__ void __launch_bounds__(kWsThreads, 1)
     ws_qgemm_kernel(const __grid_constant__ CUtensorMap w_map,
                     const __grid_constant__ CUtensorMap s_map,
                     const __grid_constant__ CUtensorMap x_map, const float *__restrict__ S8,
                     float *__restrict__ Y, int M, int N, int K, int n_o_tiles, int n_tiles,
-                    unsigned *status) {
+                    DevCtl *ctl) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_addr(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;
@@ -103,9 +104,11 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     uint64_t *sc_empty = sc_full + 2;
     uint64_t *acc_full = sc_empty + 2;
     uint64_t *acc_empty = acc_full + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    uint64_t *drain = acc_empty + 2;          // MMA thread's completion wait after an abort
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     // waiter -> MMA warp abort flags, one per K-step parity
     volatile uint32_t *mma_abort = tmem_slot + 1;
+    const unsigned long long *lim = &ctl->wait_ns;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nk = K / kAtomK;
@@ -134,6 +137,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
             mbar_init(&acc_full[b], 1);
             mbar_init(&acc_empty[b], kEpiThreads);
         }
+        mbar_init(drain, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -148,6 +152,8 @@ __global__ void __launch_bounds__(kWsThreads, 1)
 
     if (warp == kWTmaWarp) {
         // ============================================================ weight TMA
+        // (Test hook: with `inject` the first packed-code box is never
+        // requested, so the dequantizers' wait for it runs out.)
         if (lane == 0) {
             int j = 0, q = 0;
             for (int t = blockIdx.x; t < n_tiles && ok; t += G) {
@@ -157,7 +163,8 @@ __global__ void __launch_bounds__(kWsThreads, 1)
                     if (FMT == 4 && ks % kChunkSteps == 0) {
                         const int b = q & 1;
                         if (q >= 2 &&
-                            !mbar_wait(&sc_empty[b], static_cast<uint32_t>((q / 2) - 1) & 1u)) {
+                            !mbar_wait(&sc_empty[b], static_cast<uint32_t>((q / 2) - 1) & 1u,
+                                       lim)) {
                             ok = false;
                             break;
                         }
@@ -168,14 +175,28 @@ __global__ void __launch_bounds__(kWsThreads, 1)
                     }
                     const int slot = j % kRaw;
                     if (j >= kRaw &&
-                        !mbar_wait(&raw_empty[slot], static_cast<uint32_t>((j / kRaw) - 1) & 1u)) {
+                        !mbar_wait(&raw_empty[slot], static_cast<uint32_t>((j / kRaw) - 1) & 1u,
+                                   lim)) {
                         ok = false;
                         break;
                     }
+                    if (j == 0 && ctl->inject) continue;
                     mbar_expect_tx(&raw_full[slot], raw_bytes);
                     tma_load_2d(base + L.raw_off + slot * kRawSlot, &w_map,
                                 p * (FMT == 4 ? 64 : 128), y0, &raw_full[slot]);
                 }
+            }
+            // Before the CTA may exit, every box this thread requested has
+            // landed (immediate unless a consumer gave up).  Load number i of
+            // a ring slot completes that slot's phase i.
+            for (int i = 0; i < kRaw && i < j; ++i) {
+                const int last_j = i + ((j - 1 - i) / kRaw) * kRaw;
+                if (!(last_j == 0 && ctl->inject))
+                    mbar_wait(&raw_full[i], static_cast<uint32_t>(last_j / kRaw) & 1u, lim);
+            }
+            for (int i = 0; i < 2 && i < q; ++i) {
+                const int last_q = i + ((q - 1 - i) / 2) * 2;
+                mbar_wait(&sc_full[i], static_cast<uint32_t>(last_q / 2) & 1u, lim);
             }
         }
         __syncwarp();
@@ -189,7 +210,8 @@ __global__ void __launch_bounds__(kWsThreads, 1)
                 for (int ks = 0; ks < nk; ++ks, ++j) {
                     const int s = j % kStages;
                     if (j >= kStages &&
-                        !mbar_wait(&b_empty[s], static_cast<uint32_t>((j / kStages) - 1) & 1u)) {
+                        !mbar_wait(&b_empty[s], static_cast<uint32_t>((j / kStages) - 1) & 1u,
+                                   lim)) {
                         ok = false;
                         break;
                     }
@@ -197,6 +219,11 @@ __global__ void __launch_bounds__(kWsThreads, 1)
                     tma_load_2d(base + L.st_off + s * kStageBytes, &x_map,
                                 ks * kAtomK, m0, &b_full[s]);
                 }
+            }
+            // every requested activation box has landed before the CTA exits
+            for (int i = 0; i < kStages && i < j; ++i) {
+                const int last_j = i + ((j - 1 - i) / kStages) * kStages;
+                mbar_wait(&b_full[i], static_cast<uint32_t>(last_j / kStages) & 1u, lim);
             }
         }
         __syncwarp();
@@ -213,7 +240,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
                 const int b = q & 1;
                 uint32_t sw[kChunkSteps] = {};
                 if (FMT == 4) {
-                    if (!mbar_wait(&sc_full[b], static_cast<uint32_t>(q / 2) & 1u)) {
+                    if (!mbar_wait(&sc_full[b], static_cast<uint32_t>(q / 2) & 1u, lim)) {
                         ok = false;
                         break;
                     }
@@ -230,17 +257,18 @@ __global__ void __launch_bounds__(kWsThreads, 1)
                     const int jp = tile_local * npairs + (ks >> 1);   // step pair of the raw ring
                     const int slot = jp % kRaw;
                     if ((ks & 1) == 0 &&
-                        !mbar_wait(&raw_full[slot], static_cast<uint32_t>(jp / kRaw) & 1u)) {
+                        !mbar_wait(&raw_full[slot], static_cast<uint32_t>(jp / kRaw) & 1u, lim)) {
                         ok = false;
                         break;
                     }
                     const HalfRaw R = load_half_raw2<FMT>(base + L.raw_off + slot * kRawSlot, r, h,
                                                           ks & 1, sw[i]);
                     uint32_t w[16];
-                    half_words<FMT, OP>(R, w);          // before the stage wait, as in xs.cu
+                    half_words<FMT>(R, w);          // before the stage wait, as in xs.cu
                     const int s = j % kAStages;
                     if (j >= kAStages &&
-                        !mbar_wait(&a_empty[s], static_cast<uint32_t>((j / kAStages) - 1) & 1u)) {
+                        !mbar_wait(&a_empty[s], static_cast<uint32_t>((j / kAStages) - 1) & 1u,
+                                   lim)) {
                         ok = false;
                         break;
                     }
@@ -266,13 +294,15 @@ __global__ void __launch_bounds__(kWsThreads, 1)
             const int b = tile_local & 1;
             bool good = true;
             if (lane == 0 && tile_local >= 2)
-                good = mbar_wait(&acc_empty[b], static_cast<uint32_t>((tile_local / 2) - 1) & 1u);
+                good = mbar_wait(&acc_empty[b],
+                                 static_cast<uint32_t>((tile_local / 2) - 1) & 1u, lim);
             for (int ks = 0; ks < nk; ++ks, ++j) {
                 if (lane == 0) {
                     if (good)
                         good = mbar_wait(&a_full[j % kAStages],
-                                         static_cast<uint32_t>(j / kAStages) & 1u) &&
-                               mbar_wait(&b_full[j % kStages], static_cast<uint32_t>(j / kStages) & 1u);
+                                         static_cast<uint32_t>(j / kAStages) & 1u, lim) &&
+                               mbar_wait(&b_full[j % kStages],
+                                         static_cast<uint32_t>(j / kStages) & 1u, lim);
                     mma_abort[j & 1] = good ? 0u : 1u;
                 }
                 named_bar_sync(kMmaBar, 64);
@@ -284,8 +314,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
         }
     } else if (warp == kMmaWarp) {
         // ============================================================ MMA issuer
-        const uint32_t idesc =
-            idesc_f16kind_f32acc(kTileRows, kWsTileM, static_cast<uint32_t>(OP));
+        const uint32_t idesc = idesc_f16_f32acc(kTileRows, kWsTileM);
         constexpr uint64_t kStageDesc = kStageBytes >> 4;   // descriptor step per B stage
         const uint64_t bdesc0 = sw128_kmajor_desc(base + L.st_off);
         int j = 0, tile_local = 0;
@@ -315,6 +344,12 @@ __global__ void __launch_bounds__(kWsThreads, 1)
             if (abort) break;
             if (lane == 0) tc_commit(&acc_full[b]);
         }
+        if (abort && lane == 0) {
+            // MMAs already issued may still read shared memory and write
+            // TMEM: wait (bounded) for them before the CTA releases either
+            tc_commit(drain);
+            mbar_wait(drain, 0, lim);
+        }
         __syncwarp();
     } else {
         // ============================================================ epilogue
@@ -325,7 +360,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
         int tile_local = 0;
         for (int t = blockIdx.x; t < n_tiles && ok; t += G, ++tile_local) {
             const int b = tile_local & 1;
-            ok = mbar_wait(&acc_full[b], static_cast<uint32_t>(tile_local / 2) & 1u);
+            ok = mbar_wait(&acc_full[b], static_cast<uint32_t>(tile_local / 2) & 1u, lim);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after_sync();
@@ -357,7 +392,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
         }
         pdl_launch_dependents();
     }
-    if (!ok) atomicOr(status, 1u << kStatusTimeout);
+    if (!ok) atomicOr(&ctl->status, 1u << kStatusTimeout);
     tc_fence_before_sync();
     __syncthreads();
     if (warp == 0) {
@@ -366,23 +401,18 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     }
 }
 
-template <int FMT, Op16 OP>
+template <int FMT>
 cudaError_t launch_ws(const void *Xh, const void *Wq, const void *S, float *Y, int M, int N,
-                      int K, unsigned *status, cudaStream_t st) {
-    static bool attr_set[64] = {false};
+                      int K, DevCtl *ctl, cudaStream_t st) {
+    static std::atomic<bool> attr_done[kMaxDevices];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 64 && !attr_set[dev]) {
-        e = cudaFuncSetAttribute(ws_qgemm_kernel<FMT, OP>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-        if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
-    }
+    if ((e = smem_attr_once(ws_qgemm_kernel<FMT>, 227 * 1024, dev, attr_done)) != cudaSuccess)
+        return e;
     CUtensorMap w_map, s_map, x_map;
-    bool enc_ok = encode_tma_2d(&x_map, OP == Op16::f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
-                                                        : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                                2, Xh, K, M, kAtomK, CU_TENSOR_MAP_SWIZZLE_128B, kWsTileM);
+    bool enc_ok = encode_tma_2d(&x_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, Xh, K, M, kAtomK,
+                                CU_TENSOR_MAP_SWIZZLE_128B, kWsTileM);
     if (FMT == 4) {
         enc_ok = enc_ok &&
                  encode_tma_2d(&w_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Wq, K / 2, N, 64,
@@ -410,8 +440,8 @@ cudaError_t launch_ws(const void *Xh, const void *Wq, const void *S, float *Y, i
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, ws_qgemm_kernel<FMT, OP>, w_map, s_map, x_map,
-                              static_cast<const float *>(S), Y, M, N, K, n_o, tiles, status);
+    return cudaLaunchKernelEx(&cfg, ws_qgemm_kernel<FMT>, w_map, s_map, x_map,
+                              static_cast<const float *>(S), Y, M, N, K, n_o, tiles, ctl);
 }
 
 }  // namespace
@@ -426,15 +456,13 @@ bool ws_supported(int fmt, int M, int N, int K) {
 }
 
 cudaError_t launch_ws_q4(const void *Xh, const uint8_t *Wq, const uint16_t *SM, float *Y, int M,
-                         int N, int K, bool bf16, unsigned *status, cudaStream_t s) {
-    return bf16 ? launch_ws<4, Op16::bf16>(Xh, Wq, SM, Y, M, N, K, status, s)
-                : launch_ws<4, Op16::f16>(Xh, Wq, SM, Y, M, N, K, status, s);
+                         int N, int K, DevCtl *ctl, cudaStream_t s) {
+    return launch_ws<4>(Xh, Wq, SM, Y, M, N, K, ctl, s);
 }
 
 cudaError_t launch_ws_q8(const void *Xh, const int8_t *Wq, const float *S, float *Y, int M, int N,
-                         int K, bool bf16, unsigned *status, cudaStream_t s) {
-    return bf16 ? launch_ws<8, Op16::bf16>(Xh, Wq, S, Y, M, N, K, status, s)
-                : launch_ws<8, Op16::f16>(Xh, Wq, S, Y, M, N, K, status, s);
+                         int K, DevCtl *ctl, cudaStream_t s) {
+    return launch_ws<8>(Xh, Wq, S, Y, M, N, K, ctl, s);
 }
 
 }  // namespace rtq

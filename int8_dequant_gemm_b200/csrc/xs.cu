@@ -3,10 +3,10 @@
 //
 // The tile product is the same transposed one as in tc.cu,
 //   D[o, m] = sum_k W_hat[o, k] * X[m, k],
-// with 128 weight rows as the MMA's M dimension and 128 activation rows as its
-// N dimension, but the operands swap roles in memory: a CTA loads one 128-row
-// block of the activations (already rounded to 16 bits by the pre-pass in
-// prep.cu) ONCE -- all of K, 128 x K x 2 bytes of shared memory, as K/64
+// with 128 weight rows as the MMA's M dimension and 192 activation rows as its
+// N dimension, but the operands swap roles in memory: a CTA loads one 192-row
+// block of the activations (already rounded to fp16 by the pre-pass in
+// prep.cu) ONCE -- all of K, 192 x K x 2 bytes of shared memory, as K/64
 // TMA boxes in the 128-byte-swizzled operand layout -- and then walks a run of
 // weight tiles against it.  Each activation byte crosses L2 once per CTA
 // rather than once per 128-row weight tile; the weights (0.6 to 1.3 MB per
@@ -44,7 +44,9 @@
 //               rows, overlapping the next tile's MMAs.
 //
 // Every mbarrier wait is bounded; a wait that gives up latches
-// RT_ERR_DEVICE_TIMEOUT in the device status word and the CTA winds down.
+// RT_ERR_DEVICE_TIMEOUT in the device status word and the CTA winds down: the
+// TMA threads wait (bounded) for the copies they issued, the MMA thread for the
+// MMAs it issued, before the CTA releases its shared memory and TMEM.
 #include <algorithm>
 
 #include "kernels.cuh"
@@ -79,7 +81,6 @@ constexpr int kRaw = 2;                                  // packed-code ring dep
 constexpr uint32_t kAccCols = 2 * kXsTileM;              // 2 accumulators x 192 columns
 constexpr uint32_t kAStageCols = kAtomK / 2;             // 64 16-bit values per lane
 constexpr uint32_t kXsTmemCols = 512;                    // accumulators + A stages, pow2
-constexpr unsigned kStatusTimeout = 5u;
 
 static_assert(kAccCols + kAStages * kAStageCols <= kXsTmemCols, "TMEM budget");
 static_assert(kEpiCols % 32 == 0, "epilogue reads 32 columns at a time");
@@ -104,8 +105,8 @@ __host__ __device__ inline XsLayout xs_layout(int fmt, int K) {
     L.sc_off = L.raw_off + kRaw * raw_slot_bytes(fmt);
     L.bar_off = L.sc_off + 2 * scale_slot_bytes(fmt, K);
     // raw_full/empty[kRaw], sc_full/empty[2], a_full/empty[kAStages],
-    // x_full[kXAtoms], x_empty, acc_full/empty[2], + TMEM address slot
-    L.total = L.bar_off + (2 * kRaw + 4 + 2 * kAStages + kXAtoms + 1 + 4) * 8 + 16;
+    // x_full[kXAtoms], x_empty, acc_full/empty[2], drain, + TMEM address slot
+    L.total = L.bar_off + (2 * kRaw + 4 + 2 * kAStages + kXAtoms + 1 + 4 + 1) * 8 + 16;
     return L;
 }
 
@@ -126,13 +127,13 @@ struct ItemCursor {
     }
 };
 
-template <int FMT, Op16 OP>
+template <int FMT>
 __global__ void __launch_bounds__(kXsThreads, 1)
     xs_qgemm_kernel(const __grid_constant__ CUtensorMap w_map,
                     const __grid_constant__ CUtensorMap s_map,
                     const __grid_constant__ CUtensorMap x_map, const float *__restrict__ S8,
                     float *__restrict__ Y, int M, int N, int K, int n_o_tiles, int n_items,
-                    unsigned *status) {
+                    DevCtl *ctl) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_addr(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;
@@ -151,9 +152,11 @@ __global__ void __launch_bounds__(kXsThreads, 1)
     uint64_t *x_empty = x_full + kXAtoms;
     uint64_t *acc_full = x_empty + 1;
     uint64_t *acc_empty = acc_full + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    uint64_t *drain = acc_empty + 2;          // MMA thread's completion wait after an abort
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     // waiter -> MMA warp abort flags, one per K-step parity
     volatile uint32_t *mma_abort = tmem_slot + 1;
+    const unsigned long long *lim = &ctl->wait_ns;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nk = K / kAtomK;
@@ -180,6 +183,7 @@ __global__ void __launch_bounds__(kXsThreads, 1)
         }
         for (int a = 0; a < kXAtoms; ++a) mbar_init(&x_full[a], 1);
         mbar_init(x_empty, 1);
+        mbar_init(drain, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -195,33 +199,51 @@ __global__ void __launch_bounds__(kXsThreads, 1)
     if (warp == kWTmaWarp) {
         // ============================================================ weight TMA
         // Packed weights do not depend on the previous kernel in the stream,
-        // so this role starts before the dependency wait.
+        // so this role starts before the dependency wait.  (Test hook: with
+        // `inject` the first packed-code box is never requested, so the
+        // dequantizers' wait for it runs out.)
         if (lane == 0) {
-            int j = 0;
+            int j = 0, n_sc = 0;
             for (ItemCursor it(first, last, n_o_tiles); it.valid() && ok; it.next()) {
                 const int n_local = it.item - first;
                 const int y0 = it.o_tile * kTileRows;
                 if (FMT == 4) {
                     const int b = n_local & 1;
                     if (n_local >= 2 &&
-                        !mbar_wait(&sc_empty[b], static_cast<uint32_t>((n_local / 2) - 1) & 1u)) {
+                        !mbar_wait(&sc_empty[b], static_cast<uint32_t>((n_local / 2) - 1) & 1u,
+                                   lim)) {
                         ok = false;
                         break;
                     }
                     mbar_expect_tx(&sc_full[b], sc_bytes);
                     tma_load_2d(base + L.sc_off + b * kScaleSlot, &s_map, 0, y0, &sc_full[b]);
+                    ++n_sc;
                 }
                 for (int p = 0; p < nk / 2; ++p, ++j) {
                     const int slot = j % kRaw;
                     if (j >= kRaw &&
-                        !mbar_wait(&raw_empty[slot], static_cast<uint32_t>((j / kRaw) - 1) & 1u)) {
+                        !mbar_wait(&raw_empty[slot], static_cast<uint32_t>((j / kRaw) - 1) & 1u,
+                                   lim)) {
                         ok = false;
                         break;
                     }
+                    if (j == 0 && ctl->inject) continue;
                     mbar_expect_tx(&raw_full[slot], raw_bytes);
                     tma_load_2d(base + L.raw_off + slot * kRawSlot, &w_map,
                                 p * (FMT == 4 ? 64 : 128), y0, &raw_full[slot]);
                 }
+            }
+            // Before the CTA may exit, every box this thread requested has
+            // landed (immediate unless a consumer gave up).  Load number i of
+            // a ring slot completes that slot's phase i.
+            for (int i = 0; i < kRaw && i < j; ++i) {
+                const int last_j = i + ((j - 1 - i) / kRaw) * kRaw;   // last load of slot i
+                if (!(last_j == 0 && ctl->inject))
+                    mbar_wait(&raw_full[i], static_cast<uint32_t>(last_j / kRaw) & 1u, lim);
+            }
+            for (int i = 0; i < 2 && i < n_sc; ++i) {
+                const int last_q = i + ((n_sc - 1 - i) / 2) * 2;
+                mbar_wait(&sc_full[i], static_cast<uint32_t>(last_q / 2) & 1u, lim);
             }
         }
         __syncwarp();
@@ -234,7 +256,7 @@ __global__ void __launch_bounds__(kXsThreads, 1)
                 if (it.m_tile == cur_m) continue;
                 cur_m = it.m_tile;
                 if (x_loads > 0 &&
-                    !mbar_wait(x_empty, static_cast<uint32_t>(x_loads - 1) & 1u)) {
+                    !mbar_wait(x_empty, static_cast<uint32_t>(x_loads - 1) & 1u, lim)) {
                     ok = false;
                     break;
                 }
@@ -247,6 +269,10 @@ __global__ void __launch_bounds__(kXsThreads, 1)
                 }
                 ++x_loads;
             }
+            // every requested activation box has landed before the CTA exits
+            if (x_loads > 0)
+                for (int a = 0; a < nk; ++a)
+                    mbar_wait(&x_full[a], static_cast<uint32_t>(x_loads - 1) & 1u, lim);
         }
         __syncwarp();
     } else if (warp < kDeqWarps) {
@@ -262,7 +288,7 @@ __global__ void __launch_bounds__(kXsThreads, 1)
             const int b = n_local & 1;
             uint32_t sw[kScaleWords / 2] = {};
             if (FMT == 4) {
-                if (!mbar_wait(&sc_full[b], static_cast<uint32_t>(n_local / 2) & 1u)) {
+                if (!mbar_wait(&sc_full[b], static_cast<uint32_t>(n_local / 2) & 1u, lim)) {
                     ok = false;
                     break;
                 }
@@ -279,7 +305,7 @@ __global__ void __launch_bounds__(kXsThreads, 1)
                 const int jp = n_local * (nk / 2) + (ks >> 1);   // step pair of the raw ring
                 const int slot = jp % kRaw;
                 if ((ks & 1) == 0 &&
-                    !mbar_wait(&raw_full[slot], static_cast<uint32_t>(jp / kRaw) & 1u)) {
+                    !mbar_wait(&raw_full[slot], static_cast<uint32_t>(jp / kRaw) & 1u, lim)) {
                     ok = false;
                     break;
                 }
@@ -288,10 +314,11 @@ __global__ void __launch_bounds__(kXsThreads, 1)
                 // convert before waiting: only the TMEM store needs the stage
                 // free, which keeps the arithmetic off the stage's round trip
                 uint32_t w[16];
-                half_words<FMT, OP>(R, w);
+                half_words<FMT>(R, w);
                 const int s = j % kAStages;
                 if (j >= kAStages &&
-                    !mbar_wait(&a_empty[s], static_cast<uint32_t>((j / kAStages) - 1) & 1u)) {
+                    !mbar_wait(&a_empty[s], static_cast<uint32_t>((j / kAStages) - 1) & 1u,
+                               lim)) {
                     ok = false;
                     break;
                 }
@@ -330,11 +357,13 @@ __global__ void __launch_bounds__(kXsThreads, 1)
             const uint32_t xpar = static_cast<uint32_t>(x_loads - 1) & 1u;
             // accumulator b must have been drained by the epilogue
             if (lane == 0 && n_local >= 2)
-                good = mbar_wait(&acc_empty[b], static_cast<uint32_t>((n_local / 2) - 1) & 1u);
+                good = mbar_wait(&acc_empty[b], static_cast<uint32_t>((n_local / 2) - 1) & 1u,
+                                 lim);
             for (int ks = 0; ks < nk; ++ks, ++j) {
                 if (lane == 0) {
-                    if (good && fresh) good = mbar_wait(&x_full[ks], xpar);
-                    if (good) good = mbar_wait(&a_full[j & (kAStages - 1)], (j / kAStages) & 1u);
+                    if (good && fresh) good = mbar_wait(&x_full[ks], xpar, lim);
+                    if (good)
+                        good = mbar_wait(&a_full[j & (kAStages - 1)], (j / kAStages) & 1u, lim);
                     mma_abort[j & 1] = good ? 0u : 1u;
                 }
                 named_bar_sync(kMmaBar, 64);
@@ -346,8 +375,7 @@ __global__ void __launch_bounds__(kXsThreads, 1)
         }
     } else if (warp == kMmaWarp) {
         // ============================================================ MMA issuer
-        const uint32_t idesc =
-            idesc_f16kind_f32acc(kTileRows, kXsTileM, static_cast<uint32_t>(OP));
+        const uint32_t idesc = idesc_f16_f32acc(kTileRows, kXsTileM);
         static_assert(kXsTileM % 16 == 0 && kXsTileM <= 256, "MMA N for M = 128");
         static_assert((kAStages & (kAStages - 1)) == 0, "A ring indexed with a mask");
         constexpr uint64_t kXAtomDesc = kXAtom >> 4;   // descriptor step per X atom
@@ -383,6 +411,12 @@ __global__ void __launch_bounds__(kXsThreads, 1)
                 if (it.item + 1 < last && it.o_tile + 1 == n_o_tiles) tc_commit(x_empty);
             }
         }
+        if (abort && lane == 0) {
+            // MMAs already issued may still read shared memory and write
+            // TMEM: wait (bounded) for them before the CTA releases either
+            tc_commit(drain);
+            mbar_wait(drain, 0, lim);
+        }
         __syncwarp();
     } else {
         // ============================================================ epilogue
@@ -393,7 +427,7 @@ __global__ void __launch_bounds__(kXsThreads, 1)
         for (ItemCursor it(first, last, n_o_tiles); it.valid() && ok; it.next()) {
             const int n_local = it.item - first;
             const int b = n_local & 1;
-            ok = mbar_wait(&acc_full[b], static_cast<uint32_t>(n_local / 2) & 1u);
+            ok = mbar_wait(&acc_full[b], static_cast<uint32_t>(n_local / 2) & 1u, lim);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after_sync();
@@ -425,7 +459,7 @@ __global__ void __launch_bounds__(kXsThreads, 1)
         }
         pdl_launch_dependents();
     }
-    if (!ok) atomicOr(status, 1u << kStatusTimeout);
+    if (!ok) atomicOr(&ctl->status, 1u << kStatusTimeout);
     tc_fence_before_sync();
     __syncthreads();
     if (warp == 0) {
@@ -434,23 +468,18 @@ __global__ void __launch_bounds__(kXsThreads, 1)
     }
 }
 
-template <int FMT, Op16 OP>
+template <int FMT>
 cudaError_t launch_xs(const void *Xh, const void *Wq, const void *S, float *Y, int M, int N,
-                      int K, unsigned *status, cudaStream_t st) {
-    static bool attr_set[64] = {false};
+                      int K, DevCtl *ctl, cudaStream_t st) {
+    static std::atomic<bool> attr_done[kMaxDevices];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 64 && !attr_set[dev]) {
-        e = cudaFuncSetAttribute(xs_qgemm_kernel<FMT, OP>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-        if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
-    }
+    if ((e = smem_attr_once(xs_qgemm_kernel<FMT>, 227 * 1024, dev, attr_done)) != cudaSuccess)
+        return e;
     CUtensorMap w_map, s_map, x_map;
-    bool enc_ok = encode_tma_2d(&x_map, OP == Op16::f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
-                                                        : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                                2, Xh, K, M, kAtomK, CU_TENSOR_MAP_SWIZZLE_128B, kXsTileM);
+    bool enc_ok = encode_tma_2d(&x_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, Xh, K, M, kAtomK,
+                                CU_TENSOR_MAP_SWIZZLE_128B, kXsTileM);
     if (FMT == 4) {
         enc_ok = enc_ok &&
                  encode_tma_2d(&w_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Wq, K / 2, N, 64,
@@ -478,8 +507,8 @@ cudaError_t launch_xs(const void *Xh, const void *Wq, const void *S, float *Y, i
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, xs_qgemm_kernel<FMT, OP>, w_map, s_map, x_map,
-                              static_cast<const float *>(S), Y, M, N, K, n_o, items, status);
+    return cudaLaunchKernelEx(&cfg, xs_qgemm_kernel<FMT>, w_map, s_map, x_map,
+                              static_cast<const float *>(S), Y, M, N, K, n_o, items, ctl);
 }
 
 }  // namespace
@@ -494,15 +523,13 @@ bool xs_supported(int M, int N, int K) {
 }
 
 cudaError_t launch_xs_q4(const void *Xh, const uint8_t *Wq, const uint16_t *SM, float *Y, int M,
-                         int N, int K, bool bf16, unsigned *status, cudaStream_t s) {
-    return bf16 ? launch_xs<4, Op16::bf16>(Xh, Wq, SM, Y, M, N, K, status, s)
-                : launch_xs<4, Op16::f16>(Xh, Wq, SM, Y, M, N, K, status, s);
+                         int N, int K, DevCtl *ctl, cudaStream_t s) {
+    return launch_xs<4>(Xh, Wq, SM, Y, M, N, K, ctl, s);
 }
 
 cudaError_t launch_xs_q8(const void *Xh, const int8_t *Wq, const float *S, float *Y, int M, int N,
-                         int K, bool bf16, unsigned *status, cudaStream_t s) {
-    return bf16 ? launch_xs<8, Op16::bf16>(Xh, Wq, S, Y, M, N, K, status, s)
-                : launch_xs<8, Op16::f16>(Xh, Wq, S, Y, M, N, K, status, s);
+                         int K, DevCtl *ctl, cudaStream_t s) {
+    return launch_xs<8>(Xh, Wq, S, Y, M, N, K, ctl, s);
 }
 
 }  // namespace rtq

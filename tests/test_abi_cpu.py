@@ -51,7 +51,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings_and_version():
-    for s in range(9):
+    for s in range(11):
         assert rtq.status_string(s) and rtq.status_string(s) != "unknown status"
     assert rtq.status_string(99) == "unknown status"
     assert rtq.lib().rt_version() >= 100
@@ -76,6 +76,7 @@ def test_validation_statuses(fn):
     assert f(X, W, S, X, 4, 16, K, 0, None) == INVALID             # Y overlaps X
     assert f(X, W, S, W, 4, 16, K, 0, None) == INVALID             # Y overlaps Wq
     assert f(X, W, S, Y, 4, 16, K, 7, None) == INVALID             # unknown path
+    assert f(X, W, S, Y, 4, 16, K, 3, None) == INVALID             # path 3 no longer exists
     assert f(None, W, S, None, 0, 16, K, 0, None) == RT_OK         # M == 0 is a no-op
     bad_k = 40 if fn == "rt_qgemm_q4" else 24
     assert f(X, W, S, Y, 4, 16, bad_k, 0, None) == SHAPE           # K not a multiple of the granule
@@ -101,7 +102,8 @@ def test_kernel_plan():
     assert rtq.plan(4, 129, 512, 512) == "tc_x_resident"
     assert rtq.plan(4, 200, 512, 768) == "tc_w_streamed"       # K above the resident limit
     assert rtq.plan(4, 300, 512, 192) == "tc_w_stationary"     # q4 TMA needs K % 128
-    assert rtq.plan(8, 4096, 512, 2048, "tc_bf16") == "tc_w_streamed"
+    assert rtq.plan(8, 4096, 512, 2048, "tc") == "tc_w_streamed"
+    assert rtq.plan(8, 4096, 512, 2048, 3) == "rejected"       # no path 3 (bf16 operands removed)
     assert rtq.plan(4, 4096, 4096, 512, "simt") == "simt"
     assert rtq.plan(4, 4096, 4096, 96, "tc") == "rejected"
     assert rtq.plan(4, 4096, 4096, 40) == "rejected"
@@ -146,7 +148,8 @@ def test_block_grouped_launch_plan():
     assert rtq.block_fused(9, 512, 2048) == 1 and rtq.block_fused(128, 512, 2048) == 1
     assert rtq.block_fused(8, 512, 2048) == 0             # AUTO takes SIMT at M <= 8
     assert rtq.block_fused(8, 512, 2048, "tc") == 1
-    assert rtq.block_fused(1, 512, 2048, "tc_bf16") == 1
+    assert rtq.block_fused(1, 512, 2048, "tc") == 1
+    assert rtq.block_fused(1, 512, 2048, 3) == -1
     assert rtq.block_fused(129, 512, 2048) == 0           # the TMA-fed kernels
     assert rtq.block_fused(80, 512, 2048, "simt") == 0
     assert rtq.block_fused(0, 512, 2048) == 0
@@ -242,6 +245,13 @@ def test_dequant_validation():
     assert rtq.rt_dequant_q4_f32(W + 1, S, Y, 4, 64, None) == ALIGN
     assert rtq.rt_dequant_q8_f32(None, S, Y, 4, 64, None) == INVALID
     assert rtq.rt_device_status(None, None) == INVALID
+
+
+def test_debug_inject_rejects_bad_arguments():
+    # checked before any CUDA call
+    assert rtq.rt_debug_inject(2, 0) == INVALID
+    assert rtq.rt_debug_inject(-1, 0) == INVALID
+    assert rtq.rt_debug_inject(1, -5) == INVALID
 
 
 # ---------------------------------------------------------------- quantizers

@@ -69,3 +69,23 @@ def test_row_sample_holds_both_ends():
     assert np.array_equal(wl.sample_rows(5, 8, seed=3), np.arange(5))
     with pytest.raises(ValueError):
         wl.sample_rows(4096, 1, seed=3)
+
+
+def test_roofline_bound_and_fraction_follow_from_their_inputs():
+    import bench
+    peaks = {"hbm_gbs": 6540.0, "bf16_tflops": 1683.8, "bf16_tflops_sustained": 1391.3,
+             "source": "measured"}
+    # w13 at M = 4096: 224 flop/B, so the HBM side binds (224 * 6.54 < 1683.8)
+    flops = 2 * 4096 * 4096 * 512
+    nbytes = 4096 * 256 + 4096 * 16 * 4 + 4 * 4096 * 512 + 4 * 4096 * 4096
+    r = bench.roofline(flops, nbytes, 33.12e-6, peaks)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["peak"] == 6540.0
+    assert r["achieved"] == pytest.approx(nbytes / 33.12e-6 / 1e9)
+    assert r["frac"] == pytest.approx(r["achieved"] / 6540.0)
+    assert r["attainable_tflops"] == pytest.approx(flops / nbytes * 6.540)
+    assert r["tensor_peak"] == "burst"
+    # a high-intensity call binds on the tensor side, against the burst peak
+    r = bench.roofline(1e12, 1e8, 1e-3, peaks)
+    assert r["bound"] == "tensor" and r["peak"] == 1683.8
+    assert r["frac"] == pytest.approx(1000.0 / 1683.8)
+    assert bench.roofline(1e12, 1e8, 1e-3, peaks, sustained=True)["peak"] == 1391.3

@@ -5,13 +5,11 @@ from the seeded workload generator, and expected values only from oracle/.
 
 Gates:
   - dequantization exports: bit-exact (fp32 and fp16 renderings = the exact
-    value rounded once; bf16 rendering = the fp32 one rounded again);
+    value rounded once);
   - X = I turns the GEMM into W_hat^T: bit-exact on every path;
   - SIMT GEMM: max|Y - Y_ref| / max|Y_ref| <= 1e-5;
   - tensor-core GEMM (fp16 operands): <= 4e-3, and every output within the
     first-order rounding bound of its operands (below);
-  - tensor-core GEMM with bf16 operands: the same elementwise bound with the
-    bf16 unit roundoff;
   - no write outside Y (NaN guard bands), deterministic repeats, device
     status word clear afterwards.
 """
@@ -27,9 +25,9 @@ pytestmark = pytest.mark.gpu
 
 SIMT_TOL = 1e-5
 TC_TOL = 4e-3
-# unit roundoff (2^-p) of the 16-bit operand types
-UNIT = {"tc": 2.0 ** -11, "tc_bf16": 2.0 ** -8}
-MAX_REL = {"simt": SIMT_TOL, "tc": TC_TOL, "auto": TC_TOL, "tc_bf16": 1e-2}
+# unit roundoff (2^-11) of the fp16 operands of the tensor-core path
+UNIT = {"tc": 2.0 ** -11}
+MAX_REL = {"simt": SIMT_TOL, "tc": TC_TOL, "auto": TC_TOL}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -61,28 +59,19 @@ def f16_round(x32: np.ndarray) -> np.ndarray:
 
 def assert_within_rounding_bound(Y, X, What, path):
     """Elementwise first-order bound of the tensor-core path: each product
-    x*w carries the roundings of x and w to the operand type (relative u each;
-    the bf16 weight also its fp32 rounding) and the fp32 accumulation adds at most K*2^-23
-    relative to sum|x*w|; an fp16 subnormal operand (below 2^-14) is rounded
-    with an absolute error of at most 2^-25 instead."""
+    x*w carries the roundings of x and w to fp16 (relative u each) and the
+    fp32 accumulation adds at most K*2^-23 relative to sum|x*w|; an fp16
+    subnormal operand (below 2^-14) is rounded with an absolute error of at
+    most 2^-25 instead."""
     u = UNIT[path]
     A = np.abs(X.astype(np.float64)) @ np.abs(What).T
     K = X.shape[1]
-    slack = 0.0
-    if path == "tc":
-        slack = 2.0 ** -25 * (np.abs(What).sum(axis=1)[None, :] +
-                              np.abs(X.astype(np.float64)).sum(axis=1)[:, None])
+    slack = 2.0 ** -25 * (np.abs(What).sum(axis=1)[None, :] +
+                          np.abs(X.astype(np.float64)).sum(axis=1)[:, None])
     bound = (2.0 * u + u * u + 2.0 ** -23 + K * 2.0 ** -23) * A + slack
     ref = X.astype(np.float64) @ What.T
     bad = np.abs(np.asarray(Y, np.float64) - ref) > bound
     assert not bad.any(), f"{bad.sum()} outputs outside the rounding bound"
-
-
-def bf16_round(x32: np.ndarray) -> np.ndarray:
-    """fp32 -> nearest-even bf16 (as fp32 values), finite inputs."""
-    u = np.ascontiguousarray(x32, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
-    return r.astype(np.uint32).view(np.float32)
 
 
 def q4_weights(N, K, seed, outliers=False):
@@ -118,9 +107,6 @@ def test_dequant_q4_exports_bit_exact(rtq_lib, N, K):
         ref32 = exact.astype(np.float32)
         got32 = rtq_lib.dequant_q4_f32(dev(Wq), dev(sm)).cpu().numpy()
         assert np.array_equal(got32.view(np.uint32), ref32.view(np.uint32))
-        got16 = rtq_lib.dequant_q4_bf16(dev(Wq), dev(sm)).cpu().numpy()
-        ref16 = (bf16_round(ref32).view(np.uint32) >> 16).astype(np.uint16)
-        assert np.array_equal(got16, ref16)
         goth = rtq_lib.dequant_q4_f16(dev(Wq), dev(sm)).cpu().numpy()
         refh = exact.astype(np.float16).view(np.uint16)
         assert np.array_equal(goth, refh)
@@ -136,7 +122,7 @@ def test_dequant_q8_export_bit_exact(rtq_lib, N, K):
 
 
 # --------------------------------------------------- X = I: exact transposes
-@pytest.mark.parametrize("path", ["simt", "tc", "tc_bf16"])
+@pytest.mark.parametrize("path", ["simt", "tc"])
 def test_identity_input_q4_bit_exact(rtq_lib, path):
     N, K = 384, 512
     Wq, sm = q4_weights(N, K, seed=77, outliers=True)
@@ -144,14 +130,12 @@ def test_identity_input_q4_bit_exact(rtq_lib, path):
     exact = oracle.dequant_q4(Wq, sm)
     if path == "simt":
         ref32 = exact.astype(np.float32).T
-    elif path == "tc":
-        ref32 = exact.astype(np.float16).astype(np.float32).T
     else:
-        ref32 = bf16_round(exact.astype(np.float32)).T
+        ref32 = exact.astype(np.float16).astype(np.float32).T
     assert np.array_equal(Y.cpu().numpy(), ref32)
 
 
-@pytest.mark.parametrize("path", ["simt", "tc", "tc_bf16"])
+@pytest.mark.parametrize("path", ["simt", "tc"])
 def test_identity_input_q8_bit_exact(rtq_lib, path):
     N, K = 256, 512
     Wq, s = q8_weights(N, K, seed=78, outliers=True)
@@ -201,16 +185,14 @@ def test_simt_parity_q8(rtq_lib, M, N, K):
     assert rel_err(Y, ref) <= SIMT_TOL
 
 
-@pytest.mark.parametrize("path", ["tc", "tc_bf16"])
 @pytest.mark.parametrize("M,N,K", TC_SHAPES)
-def test_tc_parity_q4(rtq_lib, M, N, K, path):
+def test_tc_parity_q4(rtq_lib, M, N, K, path="tc"):
     Y, ref = _run_q4(rtq_lib, M, N, K, path, seed=M + 3 * N + K, outliers=True)
     assert rel_err(Y, ref) <= MAX_REL[path]
 
 
-@pytest.mark.parametrize("path", ["tc", "tc_bf16"])
 @pytest.mark.parametrize("M,N,K", TC_SHAPES)
-def test_tc_parity_q8(rtq_lib, M, N, K, path):
+def test_tc_parity_q8(rtq_lib, M, N, K, path="tc"):
     Y, ref = _run_q8(rtq_lib, M, N, K, path, seed=M + 5 * N + K, outliers=True)
     assert rel_err(Y, ref) <= MAX_REL[path]
 
@@ -222,17 +204,15 @@ XS_SHAPES = [(2048, 1024, 512), (2000, 1000, 512), (1500, 2100, 256), (4096, 512
              (500, 1002, 256)]
 
 
-@pytest.mark.parametrize("path", ["tc", "tc_bf16"])
 @pytest.mark.parametrize("M,N,K", XS_SHAPES)
-def test_x_resident_parity_q4(rtq_lib, M, N, K, path):
+def test_x_resident_parity_q4(rtq_lib, M, N, K, path="tc"):
     assert rtq_lib.plan(4, M, N, K, path) == "tc_x_resident"
     Y, ref = _run_q4(rtq_lib, M, N, K, path, seed=M + 7 * N + K, outliers=True)
     assert rel_err(Y, ref) <= MAX_REL[path]
 
 
-@pytest.mark.parametrize("path", ["tc", "tc_bf16"])
 @pytest.mark.parametrize("M,N,K", XS_SHAPES)
-def test_x_resident_parity_q8(rtq_lib, M, N, K, path):
+def test_x_resident_parity_q8(rtq_lib, M, N, K, path="tc"):
     assert rtq_lib.plan(8, M, N, K, path) == "tc_x_resident"
     Y, ref = _run_q8(rtq_lib, M, N, K, path, seed=M + 11 * N + K, outliers=True)
     assert rel_err(Y, ref) <= MAX_REL[path]
@@ -245,24 +225,21 @@ WS_SHAPES = [(2048, 512, 2048), (300, 640, 1024), (200, 512, 768), (1000, 700, 2
              (129, 256, 640), (300, 1002, 768)]
 
 
-@pytest.mark.parametrize("path", ["tc", "tc_bf16"])
 @pytest.mark.parametrize("M,N,K", WS_SHAPES)
-def test_w_streamed_parity_q4(rtq_lib, M, N, K, path):
+def test_w_streamed_parity_q4(rtq_lib, M, N, K, path="tc"):
     assert rtq_lib.plan(4, M, N, K, path) == "tc_w_streamed"
     Y, ref = _run_q4(rtq_lib, M, N, K, path, seed=M + 13 * N + K, outliers=True)
     assert rel_err(Y, ref) <= MAX_REL[path]
 
 
-@pytest.mark.parametrize("path", ["tc", "tc_bf16"])
 @pytest.mark.parametrize("M,N,K", WS_SHAPES)
-def test_w_streamed_parity_q8(rtq_lib, M, N, K, path):
+def test_w_streamed_parity_q8(rtq_lib, M, N, K, path="tc"):
     assert rtq_lib.plan(8, M, N, K, path) == "tc_w_streamed"
     Y, ref = _run_q8(rtq_lib, M, N, K, path, seed=M + 17 * N + K, outliers=True)
     assert rel_err(Y, ref) <= MAX_REL[path]
 
 
-@pytest.mark.parametrize("path", ["tc", "tc_bf16"])
-def test_w_streamed_odd_step_count_q8(rtq_lib, path):
+def test_w_streamed_odd_step_count_q8(rtq_lib, path="tc"):
     """q8 with K = 576: nine 64-wide K steps, so the last two-step box of
     packed codes is half past the end of each row (zero-filled by TMA)."""
     M, N, K = 700, 384, 576
@@ -320,7 +297,7 @@ def test_random_format_bytes_both_paths(rtq_lib):
     X = wl.activations(M, K, 5)
     Wq, sm = random_q4(N, K, 6)
     ref = oracle.gemm_q4(X, Wq, sm)
-    for path in ("simt", "tc", "tc_bf16"):
+    for path in ("simt", "tc"):
         Y = rtq_lib.qgemm_q4(dev(X), dev(Wq), dev(sm), path=path).cpu().numpy()
         assert rel_err(Y, ref) <= MAX_REL[path], path
         if path in UNIT:
@@ -456,7 +433,7 @@ FUSED_CASES = [
     (48, 512, 2048, "auto"),
     (128, 512, 2048, "auto"),     # largest single activation tile
     (1, 512, 2048, "tc"),         # one row, tensor cores forced
-    (80, 512, 2048, "tc_bf16"),
+    (80, 512, 2048, "tc"),
     (100, 256, 1024, "auto"),     # wo's 2 tiles half-fill a cluster: 2 CTA pairs store nothing
     (37, 1024, 4096, "auto"),     # 272 CTAs of 8 K steps
     (16, 2048, 8192, "auto"),     # clusters of 4: w2 split by 4, the others unsplit
