@@ -388,13 +388,17 @@ def measure_small_m(args, rank, world, local_rank, dev, stream, blocks=None):
 
     One M = 80 projection moves well under a megabyte of weights, less than a
     launch's latency worth, so the small-M rate is measured over many: the 12
-    blocks' quantized weights are copied into distinct device buffers until the
-    copies total about 4x L2, and one step runs every copy's block projection
-    set (qkvg, wo, w13, w2) at M = 80 through rt_qblock_project.  X and Y are
-    one buffer per projection shared by all copies (L2-resident, as the
-    activations of a real forward pass are).  The step is captured once as a
-    CUDA graph and replayed.  Returns the measurement (value = quantized
-    weight bytes per step / time, GB/s)."""
+    blocks' quantized weights are copied into distinct device buffers until
+    the copies total about 4x L2, and one step runs every copy's block
+    projection set (qkvg, wo, w13, w2) at M = 80.  The projections go through
+    rt_qgemm_batch, `copies_per_call` block copies (4 entries each) per call:
+    within a call every entry has its own Y, and the calls reuse one set of
+    Y buffers and one X buffer per projection (L2-resident, as the
+    activations of a real forward pass are), so the weights are the only
+    stream from HBM.  The step is captured once as a CUDA graph and replayed.
+    The same copies are also run one rt_qblock_project call per copy (the
+    block driver's grouped launch) for comparison.  Returns the measurement
+    (value = quantized weight bytes per step / time, GB/s)."""
     import torch
     import torch.distributed as dist
 
@@ -404,98 +408,127 @@ def measure_small_m(args, rank, world, local_rank, dev, stream, blocks=None):
     sptr = ctypes.c_void_p(stream.cuda_stream)
     M, projs = 80, ("qkvg", "wo", "w13", "w2")
     cfg = 4
+    per_call = args.copies_per_call
     if blocks is None:
         _, _, _, _, blocks = build_host("blocks12_m4096", rank)   # the 12 blocks' weights
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     per_block = sum(weight_bytes(p) for p in projs)
     copies = max(len(blocks), int(math.ceil(4 * l2 / per_block)))
+    copies = (copies + per_call - 1) // per_call * per_call
 
     def d(a):
         return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
 
     xs = {p: d(wl.activations(M, proj_dims(p)[2], wl.seed_for(cfg, 0, wl.BLOCK_PROJECTIONS[p]["x"])
                                   + 100_000 * rank)) for p in projs}
-    ys = {p: torch.empty((M, proj_dims(p)[1]), dtype=torch.float32, device=dev) for p in projs}
-    dev_blocks, structs = [], []
+    ys = [{p: torch.empty((M, proj_dims(p)[1]), dtype=torch.float32, device=dev) for p in projs}
+          for _ in range(per_call)]
+    dev_blocks = []
     for c in range(copies):
         blk = blocks[c % len(blocks)]
-        db = {p: tuple(d(a) for a in blk[p]) for p in projs}   # fresh device copy each time
-        dev_blocks.append(db)
-        structs.append(rtq._QBlockC(*(t.data_ptr() for p in projs for t in db[p]),
-                                    wl.D_MODEL, wl.D_FF))
+        dev_blocks.append({p: tuple(d(a) for a in blk[p]) for p in projs})   # distinct copies
+    # one rt_qproj array per call: per_call copies x 4 projections
+    arrays = []
+    for c0 in range(0, copies, per_call):
+        arr = (rtq._QProjC * (4 * per_call))()
+        for j in range(per_call):
+            db = dev_blocks[c0 + j]
+            for k, p in enumerate(projs):
+                N, K = proj_dims(p)[1:]
+                arr[4 * j + k] = rtq._QProjC(4 if proj_dims(p)[0] == "q4" else 8, 0,
+                                             xs[p].data_ptr(), db[p][0].data_ptr(),
+                                             db[p][1].data_ptr(), ys[j][p].data_ptr(), N, K)
+        arrays.append(arr)
+    route = rtq.KERNELS.get(L.rt_qgemm_batch_plan(arrays[0], 4 * per_call, M, 0), "per call")
+    structs = [rtq._QBlockC(*(t.data_ptr() for p in projs for t in db[p]), wl.D_MODEL, wl.D_FF)
+               for db in dev_blocks]
     xptr = [xs[p].data_ptr() for p in projs]
-    yptr = [ys[p].data_ptr() for p in projs]
+    yptr = [ys[0][p].data_ptr() for p in projs]
 
-    def step():
+    def step_batch():
+        for arr in arrays:
+            st = L.rt_qgemm_batch(arr, 4 * per_call, M, 0, sptr)
+            if st:
+                raise rtq.RtqError(st, "rt_qgemm_batch")
+
+    def step_blocks():
         for c in structs:
             st = L.rt_qblock_project(ctypes.byref(c), M, *xptr, *yptr, 0, sptr)
             if st:
                 raise rtq.RtqError(st, "rt_qblock_project")
 
-    with torch.cuda.stream(stream):
-        for _ in range(2):
+    def timed(step, sample_clocks):
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                step()
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
             step()
-    stream.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        step()
-    with torch.cuda.stream(stream):
-        for _ in range(max(args.warmup, 1)):
-            graph.replay()
-    stream.synchronize()
-    if rtq.device_status(stream) != 0:
-        raise RuntimeError("device status word reports a fault during the small-M warm-up")
+        with torch.cuda.stream(stream):
+            for _ in range(max(args.warmup, 1)):
+                graph.replay()
+        stream.synchronize()
+        if rtq.device_status(stream) != 0:
+            raise RuntimeError("device status word reports a fault during the small-M warm-up")
+        sampler = ClockSampler(gpu_uuid(dev, local_rank)) if sample_clocks else None
+        if sampler:
+            sampler.start()
+            time.sleep(0.3)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+        torch.cuda.synchronize(dev)
+        t0 = time.time()
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.steps):
+                graph.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        t1 = time.time()
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+        clocks = None
+        if sampler:
+            sampler.stop()
+            clocks = sampler.summary(t0, t1)
+        ms = reduce_max(e0.elapsed_time(e1), world, dev) / args.steps
+        if rtq.device_status(stream) != 0:
+            raise RuntimeError("device status word reports a fault in the small-M stream")
+        del graph
+        return ms, clocks
 
-    sampler = ClockSampler(gpu_uuid(dev, local_rank))
-    sampler.start()
-    time.sleep(0.3)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier(device_ids=[local_rank])
-    torch.cuda.synchronize(dev)
-    t0 = time.time()
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(args.steps):
-            graph.replay()
-        e1.record(stream)
-    torch.cuda.synchronize(dev)
-    t1 = time.time()
-    if world > 1:
-        dist.barrier(device_ids=[local_rank])
-    sampler.stop()
-    ms = reduce_max(e0.elapsed_time(e1), world, dev) / args.steps
-    if rtq.device_status(stream) != 0:
-        raise RuntimeError("device status word reports a fault in the small-M stream")
-    del graph
+    ms, clocks = timed(step_batch, True)
+    ms_blocks, _ = timed(step_blocks, False)
     wbytes = copies * per_block
     flops = copies * sum(proj_flops(p, M) for p in projs)
     abytes = copies * sum(proj_bytes(p, M) for p in projs)
     peaks = load_peaks()
     gbs = world * wbytes / (ms * 1e-3) / 1e9
-    fused = rtq.block_fused(M, wl.D_MODEL, wl.D_FF) == 1
-    launches_per_copy = 1 if fused else sum(
-        2 if rtq.plan(4 if proj_dims(p)[0] == "q4" else 8, M, *proj_dims(p)[1:])
-        in ("tc_x_resident", "tc_w_streamed") else 1 for p in projs)
+    n_calls = len(arrays)
+    launches_per_call = (1 + int(math.ceil(4 * per_call / 256))) if route == "tc_list" else None
     return {
         "metric": "quantized weight GB/s at M = 80 (aggregate stream)", "value": gbs,
         "unit": "GB/s", "ms_per_step": ms, "steps": args.steps,
         "frac_of_hbm": gbs / world / peaks["hbm_gbs"], "hbm_peak_gbs": peaks["hbm_gbs"],
         "tflops": world * flops / (ms * 1e-3) / 1e12,
         "config": {"workload": "rot_m80", "M": M, "projections": list(projs),
-                   "weight_copies": copies, "weight_bytes_per_step": wbytes,
+                   "weight_copies": copies, "copies_per_call": per_call,
+                   "calls_per_step": n_calls, "weight_bytes_per_step": wbytes,
+                   "route": route,
                    "l2": f"weights rotate over {wbytes / 1e6:.0f} MB ({wbytes / l2:.1f}x L2); "
-                         f"X and Y fixed (L2-resident)",
-                   "block_launch": "grouped" if fused else "per projection",
-                   "replay": "CUDA graph of all copies' block projection sets"},
-        "gpu_launches": args.steps * copies * launches_per_copy,
+                         f"X and Y reused by every call (L2-resident)",
+                   "replay": "CUDA graph of the step's rt_qgemm_batch calls"},
+        "gpu_launches": args.steps * n_calls * launches_per_call if launches_per_call else None,
+        "grouped_block_launch_gbs": world * wbytes / (ms_blocks * 1e-3) / 1e9,
         "roofline_weights_only": {"bound": "hbm", "achieved": gbs / world,
                                   "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                   "frac": gbs / world / peaks["hbm_gbs"],
                                   "peak_source": peaks["source"]},
         "roofline": roofline(flops, abytes, ms * 1e-3, peaks),
-        "clocks": sampler.summary(t0, t1),
+        "clocks": clocks,
     }
 
 
@@ -966,6 +999,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true",
                     help="issue the timed steps call by call instead of replaying a CUDA graph")
+    ap.add_argument("--copies-per-call", type=int, default=16,
+                    help="block copies per rt_qgemm_batch call in the small-M stream")
     ap.add_argument("--no-gates", action="store_true",
                     help="skip the small-M and M = 65536 measurements of the default workload")
     args = ap.parse_args()

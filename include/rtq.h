@@ -122,14 +122,18 @@ int rt_qgemm_auto_path(int fmt, int64_t M, int64_t N, int64_t K);
  *                             weight tiles past it (M > 128, K a multiple of
  *                             128 up to 512);
  *   RT_KERNEL_TC_W_STREAMED   tcgen05, persistent 128 x 192 tiles with both
- *                             operands TMA-staged (M > 128, other K).
- * The last two run an activation pre-pass (X rounded once to fp16) into a
- * per-(device, stream) workspace of M * K * 2 bytes. */
+ *                             operands TMA-staged (M > 128, other K);
+ *   RT_KERNEL_TC_LIST         tcgen05, rt_qgemm_batch only: persistent CTAs
+ *                             stream the weights of a whole list of
+ *                             projections with the same M <= 128.
+ * The TMA-fed kernels run an activation pre-pass (X rounded once to fp16)
+ * into a per-(device, stream) workspace of M * K * 2 bytes. */
 typedef enum rt_kernel {
     RT_KERNEL_SIMT = 1,
     RT_KERNEL_TC_W_STATIONARY = 2,
     RT_KERNEL_TC_X_RESIDENT = 3,
-    RT_KERNEL_TC_W_STREAMED = 4
+    RT_KERNEL_TC_W_STREAMED = 4,
+    RT_KERNEL_TC_LIST = 5
 } rt_kernel;
 
 /* The kernel a GEMM of this format, shape and path runs; -1 if rejected. */
@@ -184,6 +188,56 @@ rt_status rt_qgemm_noalloc(int fmt, const float *X, const void *Wq, const void *
                            int64_t M, int64_t N, int64_t K, int path, void *stream);
 
 /*
+ * A list of independent projections with the same M in one call.  The model
+ * cards have no such call: it batches the projection they define (each entry
+ * is exactly rt_qgemm_q4 or rt_qgemm_q8 on its own buffers) so that many
+ * small-M projections -- the weight-bandwidth-bound regime, where a single
+ * projection's weights stream in less time than a launch takes -- overlap
+ * their weight streams instead of paying one launch and one dependency chain
+ * each.
+ *
+ *   fmt       4: Wq/scales are q4 tensors as for rt_qgemm_q4;
+ *             8: q8 tensors as for rt_qgemm_q8.
+ *   reserved  must be 0.
+ *   X, Y      fp32 [M, K] / [M, N] device buffers of this projection.
+ *
+ * Validation: every entry as for rt_qgemm_q4/q8 (the same statuses); in
+ * addition no entry's Y may overlap any other entry's X, Wq, scales or Y
+ * (RT_ERR_INVALID_ARG), since the entries may run concurrently; X, Wq and
+ * scales may be shared between entries.  All entries are checked before
+ * anything is enqueued.  count == 0 or M == 0 is a no-op.
+ *
+ * Route (rt_qgemm_batch_plan): with 1 <= M <= 128 on the tensor-core path
+ * (RT_PATH_AUTO above the SIMT range, or RT_PATH_TC), every entry's K a
+ * multiple of 128 (q4) or 64 (q8) and every q4 scale_min 16-byte aligned, the
+ * list runs as RT_KERNEL_TC_LIST: one
+ * pre-pass launch rounds each distinct (X, K) once to fp16 into the
+ * stream's workspace (rt_workspace_reserve applies; M rounded up to 16, times
+ * K, times 2 bytes per distinct X), then persistent launches of up to 256
+ * entries each stream the entries' weights through every SM.  Under
+ * RT_PATH_AUTO this happens only when the entries hold at least as many
+ * 128-row weight tiles as the GPU has SMs.  Otherwise the entries run one
+ * after another as rt_qgemm_q4/q8 calls.  Results are those of the
+ * tensor-core path (<= 4e-3) and do not depend on the entries' order.
+ */
+typedef struct rt_qproj {
+    int32_t fmt;
+    int32_t reserved;
+    const float *X;
+    const void *Wq;
+    const void *scales;
+    float *Y;
+    int64_t N;
+    int64_t K;
+} rt_qproj;
+
+rt_status rt_qgemm_batch(const rt_qproj *list, int count, int64_t M, int path, void *stream);
+
+/* RT_KERNEL_TC_LIST if rt_qgemm_batch runs this list as list launches, 0 if
+ * it makes one call per entry, -1 if it rejects the list.  Host-only. */
+int rt_qgemm_batch_plan(const rt_qproj *list, int count, int64_t M, int path);
+
+/*
  * One RT-J block's quantized projection set, following the mixed-precision
  * recipe of the int4 card ("Quantization format": wq/wk/wv/wg and ffn.w1/w3
  * in q4 g32, the residual-writing wo and ffn.w2 in q8 per-row):
@@ -229,6 +283,41 @@ rt_status rt_qblock_project(const rt_qblock *blk, int64_t M,
  * 0 if it makes one call per projection, -1 if it rejects the sizes or path.
  * Host-only; touches no device. */
 int rt_qblock_fused(int64_t M, int64_t d_model, int64_t d_ff, int path);
+
+/*
+ * The same block projection set with each projection's format chosen by the
+ * caller, e.g. the int8 card's all-int8 (Q8_0-style) recipe ("RT-J -- int8
+ * (Q8_0-style) quantized checkpoints", section "Quantization format": every
+ * block projection wq/wk/wv/wg, wo, ffn.w1/w2/w3 stored as I8 with a
+ * per-output-row fp32 scale), where qkvg is a q8 [4*d_model, d_model] tensor
+ * and w13 a q8 [2*d_ff, d_model] tensor.
+ *   fmt       4: Wq u8 [N, K/2] and scales binary16 [N, K/32, 2] (q4);
+ *             8: Wq i8 [N, K] and scales fp32 [N] (q8);
+ *   reserved  must be 0.
+ * Shapes, outputs, launches, validation and errors are those of
+ * rt_qblock_project; rt_qblock_project is this call with the int4 card's
+ * mixed recipe (qkvg and w13 q4, wo and w2 q8).
+ */
+typedef struct rt_qweight {
+    int32_t fmt;
+    int32_t reserved;
+    const void *Wq;
+    const void *scales;
+} rt_qweight;
+
+typedef struct rt_qblock_fmt {
+    rt_qweight qkvg, wo, w13, w2;
+    int64_t d_model;
+    int64_t d_ff;
+} rt_qblock_fmt;
+
+rt_status rt_qblock_project_fmt(const rt_qblock_fmt *blk, int64_t M,
+                                const float *X_qkvg, const float *X_o, const float *X_ffn,
+                                const float *X_w2, float *Y_qkvg, float *Y_o, float *Y_13,
+                                float *Y_2, int path, void *stream);
+
+/* As rt_qblock_fused for a block with the formats of `blk` (host-only). */
+int rt_qblock_fused_fmt(const rt_qblock_fmt *blk, int64_t M, int path);
 
 /*
  * Host-side quantizers (HOST pointers, caller-allocated outputs, synchronous,

@@ -22,6 +22,7 @@ __all__ = [
     "quantize_q4_g32", "quantize_q8_row", "dequant_q4_f32", "dequant_q8_f32",
     "dequant_q4_f16", "device_status", "auto_path", "status_string",
     "qgemm_noalloc", "plan", "block_fused", "workspace_bytes", "debug_inject",
+    "qgemm_batch", "batch_plan", "Proj", "QBlockFmt", "qblock_project_fmt", "block_fused_fmt",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -45,6 +46,20 @@ class RtqError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = int(status)
         super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class _QProjC(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("reserved", ctypes.c_int32), ("X", _p), ("Wq", _p),
+                ("scales", _p), ("Y", _p), ("N", _i64), ("K", _i64)]
+
+
+class _QWeightC(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("reserved", ctypes.c_int32), ("Wq", _p), ("scales", _p)]
+
+
+class _QBlockFmtC(ctypes.Structure):
+    _fields_ = [("qkvg", _QWeightC), ("wo", _QWeightC), ("w13", _QWeightC), ("w2", _QWeightC),
+                ("d_model", _i64), ("d_ff", _i64)]
 
 
 class _QBlockC(ctypes.Structure):
@@ -85,6 +100,11 @@ def lib() -> ctypes.CDLL:
                                     _p, _i32, _p]
     L.rt_qblock_fused.restype = _i32
     L.rt_qblock_fused.argtypes = [_i64, _i64, _i64, _i32]
+    L.rt_qblock_project_fmt.restype = _i32
+    L.rt_qblock_project_fmt.argtypes = [ctypes.POINTER(_QBlockFmtC), _i64, _p, _p, _p, _p, _p, _p,
+                                        _p, _p, _i32, _p]
+    L.rt_qblock_fused_fmt.restype = _i32
+    L.rt_qblock_fused_fmt.argtypes = [ctypes.POINTER(_QBlockFmtC), _i64, _i32]
     L.rt_quantize_q4_g32.restype = _i32
     L.rt_quantize_q4_g32.argtypes = [_p, _i64, _i64, _i32, _p, _p]
     L.rt_quantize_q8_row.restype = _i32
@@ -97,6 +117,10 @@ def lib() -> ctypes.CDLL:
     L.rt_device_status.argtypes = [_p, ctypes.POINTER(_i32)]
     L.rt_debug_inject.restype = _i32
     L.rt_debug_inject.argtypes = [_i32, _i64]
+    L.rt_qgemm_batch.restype = _i32
+    L.rt_qgemm_batch.argtypes = [ctypes.POINTER(_QProjC), _i32, _i64, _i32, _p]
+    L.rt_qgemm_batch_plan.restype = _i32
+    L.rt_qgemm_batch_plan.argtypes = [ctypes.POINTER(_QProjC), _i32, _i64, _i32]
     _lib = L
     return L
 
@@ -133,6 +157,16 @@ def rt_qblock_fused(M, d_model, d_ff, path) -> int:
     return lib().rt_qblock_fused(M, d_model, d_ff, path)
 
 
+def rt_qblock_project_fmt(blk, M, X_qkvg, X_o, X_ffn, X_w2, Y_qkvg, Y_o, Y_13, Y_2, path,
+                          stream) -> int:
+    return lib().rt_qblock_project_fmt(ctypes.byref(blk), M, X_qkvg, X_o, X_ffn, X_w2, Y_qkvg,
+                                       Y_o, Y_13, Y_2, path, stream)
+
+
+def rt_qblock_fused_fmt(blk, M, path) -> int:
+    return lib().rt_qblock_fused_fmt(ctypes.byref(blk), M, path)
+
+
 def rt_quantize_q4_g32(W, N, K, n_grid, Wq, scale_min) -> int:
     return lib().rt_quantize_q4_g32(W, N, K, n_grid, Wq, scale_min)
 
@@ -159,6 +193,14 @@ def rt_device_status(stream, out) -> int:
 
 def rt_debug_inject(mode, wait_ns) -> int:
     return lib().rt_debug_inject(mode, wait_ns)
+
+
+def rt_qgemm_batch(projs, count, M, path, stream) -> int:
+    return lib().rt_qgemm_batch(projs, count, M, path, stream)
+
+
+def rt_qgemm_batch_plan(projs, count, M, path) -> int:
+    return lib().rt_qgemm_batch_plan(projs, count, M, path)
 
 
 def rt_qgemm_auto_path(fmt, M, N, K) -> int:
@@ -274,6 +316,49 @@ def qgemm_noalloc(fmt, X, Wq, scales, Y, path="auto", stream=None):
 
 
 @dataclass
+class Proj:
+    """One entry of a projection list (see rt_qproj in rtq.h): fmt 4 or 8, the
+    device tensors X [M, K], Wq and scales in that format, Y [M, N]."""
+    fmt: int
+    X: object
+    Wq: object
+    scales: object
+    Y: object
+
+
+def _batch_array(projs, M):
+    import torch
+    arr = (_QProjC * max(1, len(projs)))()
+    for i, q in enumerate(projs):
+        if q.fmt not in (4, 8):
+            raise ValueError(f"entry {i}: fmt must be 4 or 8, got {q.fmt}")
+        if q.X.dim() != 2 or q.X.shape[0] != M:
+            raise ValueError(f"entry {i}: X must be [M={M}, K], got {tuple(q.X.shape)}")
+        _, N, K = _check_gemm_shapes(q.fmt, q.X, q.Wq, q.scales, q.Y)
+        wdt, sdt = (torch.uint8, torch.uint16) if q.fmt == 4 else (torch.int8, torch.float32)
+        arr[i] = _QProjC(q.fmt, 0, _dev(q.X, torch.float32, "X"), _dev(q.Wq, wdt, "Wq"),
+                         _dev(q.scales, sdt, "scales"), _dev(q.Y, torch.float32, "Y"), N, K)
+    return arr
+
+
+def qgemm_batch(projs, M=None, path="auto", stream=None):
+    """Runs a list of independent projections with the same M (rt_qgemm_batch)."""
+    if M is None:
+        M = projs[0].X.shape[0] if projs else 0
+    arr = _batch_array(projs, M)
+    _check(rt_qgemm_batch(arr, len(projs), M, _path(path), _stream_ptr(stream)), "rt_qgemm_batch")
+
+
+def batch_plan(projs, M=None, path="auto") -> str:
+    """'tc_list' if rt_qgemm_batch runs the list as list launches, 'per_call'
+    for one call per entry, 'rejected' otherwise."""
+    if M is None:
+        M = projs[0].X.shape[0] if projs else 0
+    r = int(rt_qgemm_batch_plan(_batch_array(projs, M), len(projs), M, _path(path)))
+    return {5: "tc_list", 0: "per_call"}.get(r, "rejected")
+
+
+@dataclass
 class QBlock:
     """Device tensors of one block's packed projections (see rt_qblock in rtq.h)."""
     qkvg: object
@@ -322,6 +407,60 @@ def qblock_project(block: QBlock, X_qkvg, X_o, X_ffn, X_w2, Y_qkvg, Y_o, Y_13, Y
              (Y_qkvg, "Y_qkvg"), (Y_o, "Y_o"), (Y_13, "Y_13"), (Y_2, "Y_2"))]
     st = rt_qblock_project(bc, M, *args, _path(path), _stream_ptr(stream))
     _check(st, "rt_qblock_project")
+
+
+@dataclass
+class QBlockFmt:
+    """A block's four projections, each (fmt, Wq, scales) with fmt 4 (q4) or
+    8 (q8), as device tensors (see rt_qblock_fmt in rtq.h).  All four q8 is
+    the int8 card's all-int8 recipe."""
+    qkvg: tuple
+    wo: tuple
+    w13: tuple
+    w2: tuple
+    d_model: int = 512
+    d_ff: int = 2048
+
+    def as_c(self) -> _QBlockFmtC:
+        import torch
+        d, f = self.d_model, self.d_ff
+        ws = []
+        for name, N, K in (("qkvg", 4 * d, d), ("wo", d, d), ("w13", 2 * f, d), ("w2", d, f)):
+            fmt, Wq, S = getattr(self, name)
+            if fmt not in (4, 8):
+                raise ValueError(f"{name}: fmt must be 4 or 8, got {fmt}")
+            wshape, sshape = _packed_shapes(fmt, N, K)
+            _shape(Wq, wshape, name)
+            _shape(S, sshape, name + " scales")
+            wdt, sdt = (torch.uint8, torch.uint16) if fmt == 4 else (torch.int8, torch.float32)
+            ws.append(_QWeightC(fmt, 0, _dev(Wq, wdt, name), _dev(S, sdt, name + " scales")))
+        return _QBlockFmtC(*ws, d, f)
+
+
+def _block_io(d, f, X_qkvg, X_o, X_ffn, X_w2, Y_qkvg, Y_o, Y_13, Y_2):
+    import torch
+    M = X_qkvg.shape[0]
+    for t, shape, name in ((X_qkvg, (M, d), "X_qkvg"), (X_o, (M, d), "X_o"),
+                           (X_ffn, (M, d), "X_ffn"), (X_w2, (M, f), "X_w2"),
+                           (Y_qkvg, (M, 4 * d), "Y_qkvg"), (Y_o, (M, d), "Y_o"),
+                           (Y_13, (M, 2 * f), "Y_13"), (Y_2, (M, d), "Y_2")):
+        _shape(t, shape, name)
+    return M, [_dev(t, torch.float32, n) for t, n in
+               ((X_qkvg, "X_qkvg"), (X_o, "X_o"), (X_ffn, "X_ffn"), (X_w2, "X_w2"),
+                (Y_qkvg, "Y_qkvg"), (Y_o, "Y_o"), (Y_13, "Y_13"), (Y_2, "Y_2"))]
+
+
+def qblock_project_fmt(block: QBlockFmt, X_qkvg, X_o, X_ffn, X_w2, Y_qkvg, Y_o, Y_13, Y_2,
+                       path="auto", stream=None):
+    """Runs one block's four projections with per-projection formats."""
+    M, args = _block_io(block.d_model, block.d_ff, X_qkvg, X_o, X_ffn, X_w2, Y_qkvg, Y_o, Y_13,
+                        Y_2)
+    st = rt_qblock_project_fmt(block.as_c(), M, *args, _path(path), _stream_ptr(stream))
+    _check(st, "rt_qblock_project_fmt")
+
+
+def block_fused_fmt(block: QBlockFmt, M: int, path="auto") -> int:
+    return int(rt_qblock_fused_fmt(block.as_c(), M, _path(path)))
 
 
 def quantize_q4_g32(W: np.ndarray, n_grid: int = 21):
@@ -399,7 +538,7 @@ def auto_path(fmt: int, M: int, N: int, K: int) -> int:
     return int(rt_qgemm_auto_path(fmt, M, N, K))
 
 
-KERNELS = {1: "simt", 2: "tc_w_stationary", 3: "tc_x_resident", 4: "tc_w_streamed"}
+KERNELS = {1: "simt", 2: "tc_w_stationary", 3: "tc_x_resident", 4: "tc_w_streamed", 5: "tc_list"}
 
 
 def plan(fmt: int, M: int, N: int, K: int, path="auto") -> str:

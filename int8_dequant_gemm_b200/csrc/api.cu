@@ -4,6 +4,7 @@
 // bound and the fault-injection test hook).
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <mutex>
@@ -266,39 +267,43 @@ rt_status rt_workspace_release(void) {
     return RT_OK;
 }
 
-int rt_qblock_fused(int64_t M, int64_t d_model, int64_t d_ff, int path) {
-    if (d_model < 1 || d_ff < 1 || d_model > kMaxDim / 4 || d_ff > kMaxDim / 2) return -1;
-    const int64_t shapes[4][3] = {{4, 4 * d_model, d_model}, {8, d_model, d_model},
-                                  {4, 2 * d_ff, d_model}, {8, d_model, d_ff}};
+}  // extern "C"
+
+namespace {
+
+// One projection of a block: format, activations, packed weights, output.
+struct BlockProj {
+    int fmt;
+    const float *X;
+    const void *W, *S;
+    float *Y;
+    int64_t N, K;
+};
+
+// 1 if the block's four projections run as one grouped launch, 0 if one call
+// each, -1 if a format or size is rejected (shapes only; no pointers).
+int block_route(const int fmt[4], int64_t M, int64_t d, int64_t f, int path) {
+    if (d < 1 || f < 1 || d > kMaxDim / 4 || f > kMaxDim / 2) return -1;
+    const int64_t NK[4][2] = {{4 * d, d}, {d, d}, {2 * f, d}, {d, f}};
     bool fused = M >= 1 && M <= 128;
-    for (const auto &sh : shapes) {
-        const int kern = rt_qgemm_plan(static_cast<int>(sh[0]), M, sh[1], sh[2], path);
+    for (int i = 0; i < 4; ++i) {
+        if (fmt[i] != 4 && fmt[i] != 8) return -1;
+        const int kern = rt_qgemm_plan(fmt[i], M, NK[i][0], NK[i][1], path);
         if (kern < 0) return -1;
         fused = fused && kern == RT_KERNEL_TC_W_STATIONARY;
     }
     return fused ? 1 : 0;
 }
 
-rt_status rt_qblock_project(const rt_qblock *blk, int64_t M, const float *X_qkvg,
-                            const float *X_o, const float *X_ffn, const float *X_w2,
-                            float *Y_qkvg, float *Y_o, float *Y_13, float *Y_2, int path,
-                            void *stream) {
-    if (!blk || blk->d_model < 1 || blk->d_ff < 1) return RT_ERR_INVALID_ARG;
-    const int64_t d = blk->d_model, f = blk->d_ff;
-    struct Proj {
-        int fmt;
-        const float *X;
-        const void *W, *S;
-        float *Y;
-        int64_t N, K;
-    };
-    const Proj p[4] = {{4, X_qkvg, blk->qkvg, blk->qkvg_sm, Y_qkvg, 4 * d, d},
-                       {8, X_o, blk->wo, blk->wo_s, Y_o, d, d},
-                       {4, X_ffn, blk->w13, blk->w13_sm, Y_13, 2 * f, d},
-                       {8, X_w2, blk->w2, blk->w2_s, Y_2, d, f}};
+rt_status block_run(const BlockProj p[4], int64_t M, int64_t d, int64_t f, int path,
+                    void *stream) {
     // Every projection is checked before any is enqueued.
     rt_status st;
-    for (const Proj &q : p) {
+    int fmts[4];
+    for (int i = 0; i < 4; ++i) {
+        const BlockProj &q = p[i];
+        if (q.fmt != 4 && q.fmt != 8) return RT_ERR_INVALID_ARG;
+        fmts[i] = q.fmt;
         if ((st = rtq::check_gemm_args(q.fmt, q.X, q.W, q.S, q.Y, M, q.N, q.K)) != RT_OK)
             return st;
         const int pp = pick_path(M, q.K, path);
@@ -321,7 +326,7 @@ rt_status rt_qblock_project(const rt_qblock *blk, int64_t M, const float *X_qkvg
             }
         }
     }
-    if (rt_qblock_fused(M, d, f, path) == 1) {
+    if (block_route(fmts, M, d, f, path) == 1) {
         DevCtl *ctl = nullptr;
         if ((st = ctl_block(&ctl)) != RT_OK) return st;
         rtq::GroupProblem g[4];
@@ -331,11 +336,140 @@ rt_status rt_qblock_project(const rt_qblock *blk, int64_t M, const float *X_qkvg
         return from_cuda(rtq::launch_tc_group(g, 4, static_cast<int>(M), ctl,
                                               static_cast<cudaStream_t>(stream)));
     }
-    for (const Proj &q : p)
+    for (int i = 0; i < 4; ++i) {
+        const BlockProj &q = p[i];
         if ((st = run_gemm(q.fmt, q.X, q.W, q.S, q.Y, M, q.N, q.K, path, stream)) != RT_OK)
             return st;
+    }
     return RT_OK;
 }
+
+// The int4 card's mixed recipe: qkvg and w13 in q4, wo and w2 in q8.
+constexpr int kMixedFmt[4] = {4, 8, 4, 8};
+
+}  // namespace
+
+extern "C" {
+
+int rt_qblock_fused(int64_t M, int64_t d_model, int64_t d_ff, int path) {
+    return block_route(kMixedFmt, M, d_model, d_ff, path);
+}
+
+rt_status rt_qblock_project(const rt_qblock *blk, int64_t M, const float *X_qkvg,
+                            const float *X_o, const float *X_ffn, const float *X_w2,
+                            float *Y_qkvg, float *Y_o, float *Y_13, float *Y_2, int path,
+                            void *stream) {
+    if (!blk || blk->d_model < 1 || blk->d_ff < 1) return RT_ERR_INVALID_ARG;
+    const int64_t d = blk->d_model, f = blk->d_ff;
+    const BlockProj p[4] = {{4, X_qkvg, blk->qkvg, blk->qkvg_sm, Y_qkvg, 4 * d, d},
+                            {8, X_o, blk->wo, blk->wo_s, Y_o, d, d},
+                            {4, X_ffn, blk->w13, blk->w13_sm, Y_13, 2 * f, d},
+                            {8, X_w2, blk->w2, blk->w2_s, Y_2, d, f}};
+    return block_run(p, M, d, f, path, stream);
+}
+
+int rt_qblock_fused_fmt(const rt_qblock_fmt *blk, int64_t M, int path) {
+    if (!blk) return -1;
+    const rt_qweight *w[4] = {&blk->qkvg, &blk->wo, &blk->w13, &blk->w2};
+    int fmts[4];
+    for (int i = 0; i < 4; ++i) {
+        if (w[i]->reserved != 0) return -1;
+        fmts[i] = w[i]->fmt;
+    }
+    return block_route(fmts, M, blk->d_model, blk->d_ff, path);
+}
+
+rt_status rt_qblock_project_fmt(const rt_qblock_fmt *blk, int64_t M, const float *X_qkvg,
+                                const float *X_o, const float *X_ffn, const float *X_w2,
+                                float *Y_qkvg, float *Y_o, float *Y_13, float *Y_2, int path,
+                                void *stream) {
+    if (!blk || blk->d_model < 1 || blk->d_ff < 1) return RT_ERR_INVALID_ARG;
+    const rt_qweight *w[4] = {&blk->qkvg, &blk->wo, &blk->w13, &blk->w2};
+    for (int i = 0; i < 4; ++i)
+        if (w[i]->reserved != 0) return RT_ERR_INVALID_ARG;
+    const int64_t d = blk->d_model, f = blk->d_ff;
+    const BlockProj p[4] = {{blk->qkvg.fmt, X_qkvg, blk->qkvg.Wq, blk->qkvg.scales, Y_qkvg, 4 * d, d},
+                            {blk->wo.fmt, X_o, blk->wo.Wq, blk->wo.scales, Y_o, d, d},
+                            {blk->w13.fmt, X_ffn, blk->w13.Wq, blk->w13.scales, Y_13, 2 * f, d},
+                            {blk->w2.fmt, X_w2, blk->w2.Wq, blk->w2.scales, Y_2, d, f}};
+    return block_run(p, M, d, f, path, stream);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- batches
+namespace {
+
+int sm_count() {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms;
+}
+
+// Checks a list and returns the route it takes: RT_KERNEL_TC_LIST, 0 for one
+// call per projection, or a negative rt_status for a rejected list.
+int batch_route(const rt_qproj *list, int count, int64_t M, int path) {
+    if (count < 0 || (count > 0 && !list) || M < 0 || M > kMaxDim) return -RT_ERR_INVALID_ARG;
+    if (path != RT_PATH_AUTO && path != RT_PATH_SIMT && path != RT_PATH_TC)
+        return -RT_ERR_INVALID_ARG;
+    bool tc_all = true, list_ok = M >= 1 && M <= 128;
+    int64_t tiles = 0;
+    for (int i = 0; i < count; ++i) {
+        const rt_qproj &q = list[i];
+        if ((q.fmt != 4 && q.fmt != 8) || q.reserved != 0) return -RT_ERR_INVALID_ARG;
+        const rt_status st = rtq::check_gemm_args(q.fmt, q.X, q.Wq, q.scales, q.Y, M, q.N, q.K);
+        if (st != RT_OK) return -st;
+        const int p = pick_path(M, q.K, path);
+        if (p == -1) return -RT_ERR_UNSUPPORTED_SHAPE;
+        tc_all = tc_all && p == RT_PATH_TC;
+        // the list kernel copies q4 (scale, min) rows in 16-byte pieces
+        list_ok = list_ok && rtq::pl_supported(q.fmt, static_cast<int>(M), static_cast<int>(q.K)) &&
+                  (q.fmt != 4 || aligned(q.scales, 16));
+        tiles += (q.N + 127) / 128;
+    }
+    // the projections may run concurrently: no output may overlap another
+    // projection's output or inputs (sorted sweep over the address ranges)
+    if (M > 0 && count > 1) {
+        struct Range {
+            uintptr_t lo, hi;
+            bool out;
+        };
+        std::vector<Range> r;
+        r.reserve(static_cast<size_t>(count) * 4);
+        for (int i = 0; i < count; ++i) {
+            const rt_qproj &q = list[i];
+            const int64_t wb = q.fmt == 4 ? q.N * (q.K / 2) : q.N * q.K;
+            const int64_t sb = q.fmt == 4 ? q.N * (q.K / 32) * 4 : q.N * 4;
+            auto add = [&](const void *p, int64_t n, bool out) {
+                const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+                r.push_back({a, a + static_cast<uintptr_t>(n), out});
+            };
+            add(q.Y, M * q.N * 4, true);
+            add(q.X, M * q.K * 4, false);
+            add(q.Wq, wb, false);
+            add(q.scales, sb, false);
+        }
+        std::sort(r.begin(), r.end(), [](const Range &a, const Range &b) { return a.lo < b.lo; });
+        // In address order, each range is checked against the furthest end
+        // reached so far: an output against every earlier range, an input
+        // against earlier outputs.  (Overlaps within one projection are
+        // already rejected above, and inputs may share memory.)
+        uintptr_t end_any = 0, end_out = 0;
+        for (const Range &x : r) {
+            if (x.out ? end_any > x.lo : end_out > x.lo) return -RT_ERR_INVALID_ARG;
+            end_any = std::max(end_any, x.hi);
+            if (x.out) end_out = std::max(end_out, x.hi);
+        }
+    }
+    if (!tc_all || !list_ok || count == 0) return 0;
+    if (path == RT_PATH_AUTO && tiles < sm_count()) return 0;
+    return RT_KERNEL_TC_LIST;
+}
+
+}  // namespace
+
+extern "C" {
 
 static rt_status validate_dequant(const void *Wq, const void *S, const void *W, int64_t N,
                                   int64_t K, int64_t granule, uintptr_t salign) {
@@ -371,6 +505,39 @@ rt_status rt_dequant_q4_f16(const uint8_t *Wq, const uint16_t *scale_min, uint16
     return from_cuda(rtq::launch_dequant_q4_f16(Wq, scale_min, W_out, static_cast<int>(N),
                                                 static_cast<int>(K),
                                                 static_cast<cudaStream_t>(stream)));
+}
+
+int rt_qgemm_batch_plan(const rt_qproj *list, int count, int64_t M, int path) {
+    const int r = batch_route(list, count, M, path);
+    return r < 0 ? -1 : r;
+}
+
+rt_status rt_qgemm_batch(const rt_qproj *list, int count, int64_t M, int path, void *stream) {
+    const int route = batch_route(list, count, M, path);
+    if (route < 0) return static_cast<rt_status>(-route);
+    if (M == 0 || count == 0) return RT_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (route != RT_KERNEL_TC_LIST) {
+        rt_status st;
+        for (int i = 0; i < count; ++i) {
+            const rt_qproj &q = list[i];
+            if ((st = run_gemm(q.fmt, q.X, q.Wq, q.scales, q.Y, M, q.N, q.K, path, stream)) != RT_OK)
+                return st;
+        }
+        return RT_OK;
+    }
+    DevCtl *ctl = nullptr;
+    rt_status st = ctl_block(&ctl);
+    if (st != RT_OK) return st;
+    std::vector<rtq::PlInput> in(static_cast<size_t>(count));
+    for (int i = 0; i < count; ++i) {
+        const rt_qproj &q = list[i];
+        in[i] = {q.fmt, q.X, q.Wq, q.scales, q.Y, static_cast<int>(q.N), static_cast<int>(q.K)};
+    }
+    void *ws = nullptr;
+    const size_t need = rtq::pl_workspace_bytes(in.data(), count, static_cast<int>(M));
+    if ((st = workspace(s, need, &ws)) != RT_OK) return st;
+    return from_cuda(rtq::launch_pl_batch(in.data(), count, static_cast<int>(M), ws, ctl, s));
 }
 
 rt_status rt_device_status(void *stream, int *device_status) {

@@ -94,6 +94,25 @@ cudaError_t launch_ws_q4(const void *Xh, const uint8_t *Wq, const uint16_t *SM, 
 cudaError_t launch_ws_q8(const void *Xh, const int8_t *Wq, const float *S, float *Y, int M, int N,
                          int K, DevCtl *ctl, cudaStream_t s);
 
+// tcgen05, a list of independent projections with the same M (1..128) in
+// persistent launches that stream every projection's weights back to back;
+// see pl.cu.  pl_supported: the shapes it takes; pl_workspace_bytes: bytes of
+// the fp16 activation images (one per distinct (X, K)); launch_pl_batch runs
+// the image pre-pass and the list launches.  Arguments are validated by the
+// caller.
+struct PlInput {
+    int fmt;
+    const float *X;
+    const void *Wq;
+    const void *S;
+    float *Y;
+    int N, K;
+};
+bool pl_supported(int fmt, int M, int K);
+size_t pl_workspace_bytes(const PlInput *in, int count, int M);
+cudaError_t launch_pl_batch(const PlInput *in, int count, int M, void *ws, DevCtl *ctl,
+                            cudaStream_t s);
+
 // dequantization exports (same __device__ routines as the GEMMs)
 cudaError_t launch_dequant_q4_f32(const uint8_t *Wq, const uint16_t *SM, float *W, int N, int K,
                                   cudaStream_t s);

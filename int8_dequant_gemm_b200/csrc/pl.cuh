@@ -1,0 +1,51 @@
+// Parameters of the projection-list kernel (pl.cu): the projections, the work
+// items cut from them and each CTA's share, passed by value as one
+// __grid_constant__ kernel parameter (under the 32 KB parameter limit).
+#pragma once
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace rtq {
+
+constexpr int kPlMaxProj = 256;     // projections per launch
+constexpr int kPlMaxItems = 2048;   // work items per launch
+constexpr int kPlMaxCtas = 160;     // >= the SM count of one B200
+constexpr int kPlMaxAcc = 8;        // accumulators in the TMEM ring
+
+struct PlProj {
+    const uint8_t *Xh;   // fp16 image of the projection's activations (pre-pass output)
+    const void *Wq;      // q4: u8 [N, K/2]; q8: i8 [N, K]
+    const void *S;       // q4: binary16 (scale, min) [N, K/32, 2]; q8: fp32 [N]
+    float *Y;            // fp32 [M, N]
+    int N, K, fmt, xid;  // xid: index of the distinct activation image
+};
+
+struct PlItem {
+    uint32_t tile0;      // first 128-row weight tile
+    uint16_t proj;       // index into PlParams::proj
+    uint16_t ntiles;
+};
+
+struct PlParams {
+    int M, bnp, nslots, nacc;
+    int cta_items[kPlMaxCtas + 1];   // CTA b runs items [cta_items[b], cta_items[b + 1])
+    PlProj proj[kPlMaxProj];
+    PlItem items[kPlMaxItems];
+};
+
+struct PlPrepImage {
+    const float *X;      // fp32 [M, K]
+    uint8_t *Xh;         // fp16 image, pl_image_bytes(M, K) bytes
+    int K, pad;
+};
+
+struct PlPrep {
+    int M, bnp;
+    PlPrepImage img[kPlMaxProj];
+};
+
+static_assert(sizeof(PlParams) + 8 <= 32764, "kernel parameter limit");
+static_assert(sizeof(PlPrep) + 8 <= 32764, "kernel parameter limit");
+
+}  // namespace rtq

@@ -309,3 +309,79 @@ def test_empty_quantizer_inputs():
     assert Wq.shape == (0, 32) and sm.shape == (0, 2, 2)
     q, s = rtq.quantize_q8_row(np.zeros((0, 16), dtype=np.float32))
     assert q.shape == (0, 16)
+
+
+# ------------------------------------------------------------ projection lists
+def _qproj_array(entries):
+    arr = (rtq._QProjC * len(entries))()
+    for i, e in enumerate(entries):
+        arr[i] = rtq._QProjC(*e)
+    return arr
+
+
+def test_batch_validation_and_routes():
+    # (fmt, reserved, X, Wq, scales, Y, N, K) at fake, aligned, disjoint addresses
+    GB = 1 << 30
+    def entry(i, fmt=4, N=2048, K=512, X=None, Y=None):
+        return (fmt, 0, X or (1 * GB + i * 16 * 2 ** 20), 2 * GB + i * 16 * 2 ** 20,
+                3 * GB + i * 16 * 2 ** 20, Y or (4 * GB + i * 16 * 2 ** 20), N, K)
+    plan, run = rtq.lib().rt_qgemm_batch_plan, rtq.lib().rt_qgemm_batch
+    TC_LIST = 5
+    ok = _qproj_array([entry(i) for i in range(12)])          # 12 x 16 tiles = 192 >= SMs
+    assert plan(ok, 12, 80, 0) == TC_LIST
+    assert plan(ok, 12, 80, 2) == TC_LIST
+    assert plan(ok, 12, 80, 1) == 0                           # SIMT: one call per entry
+    assert plan(ok, 12, 4, 0) == 0                            # AUTO takes SIMT at M <= 8
+    assert plan(ok, 12, 200, 2) == 0                          # M > 128: per call
+    assert plan(ok, 2, 80, 0) == 0                            # 32 tiles < SMs under AUTO
+    assert plan(ok, 2, 80, 2) == TC_LIST                      # forced
+    # shared activations are allowed
+    shared = _qproj_array([entry(i, X=1 * GB) for i in range(3)])
+    assert plan(shared, 3, 80, 2) == TC_LIST
+    # q4 K % 128 != 0 runs per call; K % 64 != 0 needs SIMT under AUTO
+    assert plan(_qproj_array([entry(0, K=192), entry(1)]), 2, 80, 2) == 0
+    assert plan(_qproj_array([entry(0, K=96)]), 1, 80, 2) == -1
+    # rejections, all before any CUDA call
+    assert run(None, 1, 80, 0, None) == INVALID
+    assert run(ok, -1, 80, 0, None) == INVALID
+    assert run(ok, 12, -1, 0, None) == INVALID
+    assert run(ok, 12, 80, 3, None) == INVALID                # no path 3
+    assert run(_qproj_array([entry(0, fmt=5)]), 1, 80, 0, None) == INVALID
+    bad = list(entry(0)); bad[1] = 1                           # reserved must be 0
+    assert run(_qproj_array([tuple(bad)]), 1, 80, 0, None) == INVALID
+    bad = list(entry(0)); bad[2] += 4                          # X misaligned
+    assert run(_qproj_array([tuple(bad)]), 1, 80, 0, None) == ALIGN
+    assert run(_qproj_array([entry(0, K=40)]), 1, 80, 0, None) == SHAPE
+    # outputs may not overlap another entry's output or inputs
+    assert run(_qproj_array([entry(0), entry(1, Y=4 * GB + 4096)]), 2, 80, 0, None) == INVALID
+    assert run(_qproj_array([entry(0), entry(1, Y=2 * GB)]), 2, 80, 0, None) == INVALID
+    assert run(_qproj_array([entry(0), entry(1, X=4 * GB + 64)]), 2, 80, 0, None) == INVALID
+    # no-ops
+    assert run(ok, 0, 80, 0, None) == RT_OK
+    assert run(ok, 12, 0, 0, None) == RT_OK
+
+
+def test_block_fmt_validation_and_routes():
+    GB = 1 << 30
+    def blk(fmts, reserved=0, d=512, f=2048):
+        ws = [rtq._QWeightC(fm, reserved, (2 + i) * GB, (6 + i) * GB) for i, fm in enumerate(fmts)]
+        return rtq._QBlockFmtC(*ws, d, f)
+    fused = rtq.lib().rt_qblock_fused_fmt
+    run = rtq.lib().rt_qblock_project_fmt
+    import ctypes as C
+    q8 = blk((8, 8, 8, 8))
+    assert fused(C.byref(q8), 80, 0) == 1                  # one grouped launch
+    assert fused(C.byref(q8), 2048, 0) == 0                # one call per projection
+    assert fused(C.byref(q8), 4, 0) == 0                   # SIMT under AUTO
+    mixed = blk((4, 8, 4, 8))
+    assert fused(C.byref(mixed), 80, 0) == rtq.block_fused(80, 512, 2048) == 1
+    assert fused(C.byref(blk((8, 8, 5, 8))), 80, 0) == -1  # unknown format
+    assert fused(C.byref(blk((8, 8, 8, 8), reserved=1)), 80, 0) == -1
+    X = [10 * GB + i * GB // 4 for i in range(4)]
+    Y = [20 * GB + i * GB // 4 for i in range(4)]
+    assert run(C.byref(blk((8, 8, 9, 8))), 80, *X, *Y, 0, None) == INVALID
+    assert run(C.byref(blk((8, 8, 8, 8), reserved=2)), 80, *X, *Y, 0, None) == INVALID
+    assert run(None, 80, *X, *Y, 0, None) == INVALID
+    Ybad = list(Y); Ybad[1] = Y[0] + 64                    # outputs overlap
+    assert run(C.byref(q8), 80, *X, *Ybad, 0, None) == INVALID
+    assert run(C.byref(q8), 0, *X, *Y, 0, None) == RT_OK   # M == 0: no-op

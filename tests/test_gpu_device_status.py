@@ -140,3 +140,35 @@ def test_activation_outside_fp16_range_is_reported(rtq_lib, M, kernel):
     X[M // 2, 3] = 1.0
     rtq_lib.qgemm_q8(dev(X), Wd, Sd, path="tc")
     assert rtq_lib.device_status() == rtq_lib.OK
+
+
+def test_injected_timeout_in_list_kernel(rtq_lib):
+    """The projection-list kernel: the first weight slot of every CTA never
+    completes, so its dequantizers' waits run out; the weight producers
+    still drain their copies and the CTA releases TMEM."""
+    M = 80
+    shapes = [(4, 2048, 512), (8, 512, 2048), (4, 1024, 512)]
+    host = [_problem(f, M, n, k, seed=990 + i) for i, (f, n, k) in enumerate(shapes)]
+    projs = [rtq_lib.Proj(f, dev(X), dev(q[0]), dev(q[1]), torch.full((M, n), 7.0, device="cuda"))
+             for (f, n, k), (X, q, _) in zip(shapes, host)]
+    assert rtq_lib.batch_plan(projs, path="tc") == "tc_list"
+    rtq_lib.debug_inject(1, WAIT_NS)
+    try:
+        rtq_lib.qgemm_batch(projs, path="tc")
+        assert rtq_lib.device_status() == rtq_lib.RT_ERR_DEVICE_TIMEOUT
+    finally:
+        rtq_lib.debug_inject(0, 0)
+    rtq_lib.qgemm_batch(projs, path="tc")
+    assert rtq_lib.device_status() == rtq_lib.OK
+    for p, (_, _, ref) in zip(projs, host):
+        assert rel_err(p.Y.cpu().numpy(), ref) <= TC_TOL
+
+
+def test_activation_outside_fp16_range_in_list_kernel(rtq_lib):
+    M = 48
+    X, q, _ = _problem(4, M, 1024, 512, seed=995)
+    X[5, 100] = -7.0e4
+    Y = torch.empty((M, 1024), device="cuda")
+    rtq_lib.qgemm_batch([rtq_lib.Proj(4, dev(X), dev(q[0]), dev(q[1]), Y)], path="tc")
+    assert rtq_lib.device_status() == rtq_lib.RT_ERR_OPERAND_RANGE
+    assert not bool(torch.isfinite(Y[5]).all()) and bool(torch.isfinite(Y[6:]).all())
