@@ -68,6 +68,15 @@ def lib() -> ctypes.CDLL:
         L.oracle_gemm_q4.argtypes = [_p, _p, _p, _i64, _i64, _i64, _p, _i64, _p, _p]
         L.oracle_gemm_q8.restype = ctypes.c_int
         L.oracle_gemm_q8.argtypes = [_p, _p, _p, _i64, _i64, _i64, _p, _i64, _p, _p]
+        L.oracle_e4m3_to_double.restype = ctypes.c_double
+        L.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_from_double.restype = ctypes.c_int
+        L.oracle_e4m3_from_double.argtypes = [ctypes.c_double, ctypes.POINTER(ctypes.c_uint8)]
+        L.oracle_quant_e4m3.restype = ctypes.c_int
+        L.oracle_quant_e4m3.argtypes = [_p, _i64, _p]
+        L.oracle_dequant_e4m3.argtypes = [_p, _i64, _i64, _p]
+        L.oracle_gemm_e4m3.restype = ctypes.c_int
+        L.oracle_gemm_e4m3.argtypes = [_p, _p, _i64, _i64, _i64, _p, _i64, _p, _p]
         _lib = L
     return _lib
 
@@ -211,4 +220,48 @@ def gemm_q8(X: np.ndarray, Wq: np.ndarray, scale: np.ndarray, rows=None) -> np.n
     wrow = np.empty(max(K, 1), dtype=np.float64)
     lib().oracle_gemm_q8(_ptr(X), _ptr(Wq), _ptr(scale), M, N, K, _ptr(rows), n,
                          _ptr(Y), _ptr(wrow))
+    return Y
+
+
+# --------------------------------------------------------------------------
+# FP8 E4M3 (the FP8 card's float8_e4m3fn weights, no scale)
+# --------------------------------------------------------------------------
+def e4m3_to_double(b: int) -> float:
+    return float(lib().oracle_e4m3_to_double(int(b) & 0xFF))
+
+
+def e4m3_from_double(x: float):
+    """Code of the nearest E4M3 value (ties to the even code); None if out of range."""
+    out = ctypes.c_uint8()
+    rc = lib().oracle_e4m3_from_double(float(x), ctypes.byref(out))
+    return None if rc != 0 else int(out.value)
+
+
+def quant_e4m3(W: np.ndarray) -> np.ndarray:
+    """uint8 [N, K] of E4M3 codes; ValueError if a weight is out of range."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    out = np.empty(W.shape, dtype=np.uint8)
+    if lib().oracle_quant_e4m3(_ptr(W), W.size, _ptr(out)) != 0:
+        raise ValueError("oracle_quant_e4m3: a weight is NaN or beyond 464 in magnitude")
+    return out
+
+
+def dequant_e4m3(Wq: np.ndarray) -> np.ndarray:
+    Wq = np.ascontiguousarray(Wq, dtype=np.uint8)
+    N, K = Wq.shape
+    out = np.empty((N, K), dtype=np.float64)
+    lib().oracle_dequant_e4m3(_ptr(Wq), N, K, _ptr(out))
+    return out
+
+
+def gemm_e4m3(X: np.ndarray, Wq: np.ndarray, rows=None) -> np.ndarray:
+    X = np.ascontiguousarray(X, dtype=np.float32)
+    Wq = np.ascontiguousarray(Wq, dtype=np.uint8)
+    M, K = X.shape
+    N = Wq.shape[0]
+    assert Wq.shape == (N, K)
+    rows, n = _rows_arg(rows, M)
+    Y = np.empty((n, N), dtype=np.float64)
+    wrow = np.empty(max(K, 1), dtype=np.float64)
+    lib().oracle_gemm_e4m3(_ptr(X), _ptr(Wq), M, N, K, _ptr(rows), n, _ptr(Y), _ptr(wrow))
     return Y

@@ -16,6 +16,9 @@
  *   [Q8]  "RT-J -- int8 (Q8_0-style) quantized checkpoints", section
  *         "Quantization format": int8 codes with one symmetric fp32 scale per
  *         output row, W[o,i] ~= q[o,i] * scale[o], scale[o] = max|W[o,:]|/127.
+ *   [F8]  "RT-J -- FP8 E4M3 checkpoints", section "FP8 Format": every
+ *         two-dimensional matrix weight is stored directly as PyTorch
+ *         float8_e4m3fn (no scale).
  *   [GEMM] Both cards, opening paragraph: the engine dequantizes inside the
  *         GEMM; the projection computes Y = X * W^T with W indexed [out, in].
  *
@@ -26,7 +29,9 @@
  * dequantization will use, codes round half-to-even and clamp to [0,15], ties
  * between grid points keep the smallest j, a group whose fp16 scale is zero
  * stores all-zero codes, the companion tensor is [N, K/32, 2] with scale
- * first, and the int8 codes round half-to-even and clamp to [-127, 127].
+ * first, the int8 codes round half-to-even and clamp to [-127, 127], and an
+ * FP8 weight is the nearest E4M3 value (ties to the even code) with magnitudes
+ * above 464, which would round past the largest finite value 448, out of range.
  *
  * Every function below states the step of the pages it follows.  All
  * arithmetic on weights is in IEEE double; dequantized values are exact in
@@ -241,6 +246,61 @@ void oracle_dequant_q8(const int8_t *Wq, const float *scale, int64_t N, int64_t 
 }
 
 /* ---------------------------------------------------------------------------
+ * FP8 E4M3 ([F8]).  float8_e4m3fn is the finite-only 8-bit E4M3 format: one
+ * sign bit, four exponent bits with bias 7, three mantissa bits.  Exponent
+ * field e = 0 holds the subnormals m * 2^-9; e = 1..15 hold (1 + m/8) *
+ * 2^(e-7), except that S.1111.111 is NaN; there is no infinity, and the
+ * largest finite magnitude is 1.75 * 2^8 = 448.
+ * ------------------------------------------------------------------------- */
+double oracle_e4m3_to_double(uint8_t b)
+{
+    const int sign = (b >> 7) & 1, e = (b >> 3) & 0xF, m = b & 7;
+    double v;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        v = (double)m * ldexp(1.0, -9);
+    else
+        v = (1.0 + (double)m / 8.0) * ldexp(1.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* The nearest finite E4M3 value to x, by search over the 127 non-negative
+ * finite codes; of two equally near codes the even one (mantissa bit 0
+ * clear).  Returns -1 for NaN and for |x| > 464 (half way between 448 and the
+ * next step 480, which the format does not have); 0 otherwise. */
+int oracle_e4m3_from_double(double x, uint8_t *out)
+{
+    if (isnan(x) || fabs(x) > 464.0) return -1;
+    const double a = fabs(x);
+    int best = 0;
+    double best_d = a;                       /* distance to code 0 (zero) */
+    for (int c = 1; c <= 0x7E; ++c) {
+        const double d = fabs(a - oracle_e4m3_to_double((uint8_t)c));
+        if (d < best_d || (d == best_d && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            best_d = d;
+        }
+    }
+    *out = (uint8_t)(best | (signbit(x) ? 0x80 : 0));
+    return 0;
+}
+
+/* [F8]: each weight stored directly as its E4M3 rounding.  Returns -1 (and
+ * leaves the rest of `out` unspecified) at the first weight out of range. */
+int oracle_quant_e4m3(const float *W, int64_t n, uint8_t *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        if (oracle_e4m3_from_double((double)W[i], &out[i]) != 0) return -1;
+    return 0;
+}
+
+void oracle_dequant_e4m3(const uint8_t *Wq, int64_t N, int64_t K, double *W)
+{
+    for (int64_t i = 0; i < N * K; ++i) W[i] = oracle_e4m3_to_double(Wq[i]);
+}
+
+/* ---------------------------------------------------------------------------
  * The projection ([GEMM]): Y[m,o] = sum_k X[m,k] * W[o,k], summed over k in
  * ascending order in double.  `rows` (may be NULL for all rows 0..M-1) lists
  * which rows of X to compute; Y is [n_rows, N].  wrow is caller scratch of K
@@ -277,6 +337,17 @@ int oracle_gemm_q8(const float *X, const int8_t *Wq, const float *scale,
     if (!rows) n_rows = M;
     for (int64_t o = 0; o < N; ++o) {
         oracle_dequant_q8(Wq + o * K, scale + o, 1, K, wrow);
+        gemm_rows(X, K, wrow, o, N, rows, n_rows, Y);
+    }
+    return 0;
+}
+
+int oracle_gemm_e4m3(const float *X, const uint8_t *Wq, int64_t M, int64_t N, int64_t K,
+                     const int64_t *rows, int64_t n_rows, double *Y, double *wrow)
+{
+    if (!rows) n_rows = M;
+    for (int64_t o = 0; o < N; ++o) {
+        oracle_dequant_e4m3(Wq + o * K, 1, K, wrow);
         gemm_rows(X, K, wrow, o, N, rows, n_rows, Y);
     }
     return 0;

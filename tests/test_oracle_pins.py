@@ -331,3 +331,64 @@ def test_quantizer_rejects_bad_input():
         oracle.quant_q4_g32(np.full((1, 32), np.inf, dtype=np.float32))
     with pytest.raises(ValueError):
         oracle.quant_q4_g32(np.full((1, 32), 1e5, dtype=np.float32))
+
+
+# ---------------------------------------------------------------- FP8 E4M3
+torch = pytest.importorskip("torch")
+
+
+def test_e6_e4m3_hand_worked(golden):
+    g = golden("e6_e4m3.txt")
+    codes = [int(c, 16) for c in g["codes"].split()]
+    values = [float(v) for v in g["values"].split()]
+    assert [oracle.e4m3_to_double(c) for c in codes] == values
+    ins = [float(v) for v in g["encode_in"].split()]
+    outs = [int(c, 16) for c in g["encode_out"].split()]
+    assert [oracle.e4m3_from_double(x) for x in ins] == outs
+
+
+def test_e4m3_decode_all_codes_match_torch():
+    """Every one of the 256 codes against PyTorch's own float8_e4m3fn decoding."""
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    got = np.array([oracle.e4m3_to_double(b) for b in range(256)])
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+    assert np.isnan(got).sum() == 2          # 0x7F and 0xFF
+
+
+def test_e4m3_encode_matches_torch_rounding():
+    """The nearest-value search against PyTorch's float -> float8_e4m3fn cast on
+    every finite value, every midpoint (ties), random values across the
+    binades and the subnormals, and the edge up to 464."""
+    finite = np.array([oracle.e4m3_to_double(b) for b in range(0x7F)])
+    mids = (finite[:-1] + finite[1:]) / 2
+    g = np.random.default_rng(11)
+    rnd = np.concatenate([g.uniform(-448, 448, 2000), g.normal(0, 0.02, 2000),
+                          g.uniform(-2 ** -6, 2 ** -6, 1000), np.linspace(440, 464, 97)])
+    xs = np.concatenate([finite, -finite, mids, -mids, rnd]).astype(np.float32)
+    ref = torch.from_numpy(xs).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_from_double(float(x)) for x in xs], dtype=np.uint8)
+    assert np.array_equal(got, ref)
+
+
+def test_e4m3_out_of_range_is_rejected():
+    for x in (464.0001, -500.0, 1e30, float("nan"), float("inf")):
+        assert oracle.e4m3_from_double(x) is None
+    with pytest.raises(ValueError):
+        oracle.quant_e4m3(np.array([[0.1, 600.0]], dtype=np.float32))
+
+
+def test_gemm_e4m3_identity_and_bruteforce():
+    W = wl.weights(24, 32, 5)
+    Wq = oracle.quant_e4m3(W)
+    What = oracle.dequant_e4m3(Wq)
+    # X = I gives the dequantized weights transposed, exactly
+    assert np.array_equal(oracle.gemm_e4m3(np.eye(32, dtype=np.float32), Wq), What.T)
+    # a tiny product against exact rational arithmetic
+    X = wl.activations(3, 32, 6)
+    Y = oracle.gemm_e4m3(X, Wq)
+    for m in range(3):
+        for o in range(0, 24, 5):
+            exact = sum(Fraction(float(X[m, k])) * Fraction(What[o, k]) for k in range(32))
+            assert abs(Fraction(Y[m, o]) - exact) <= abs(exact) * Fraction(1, 2 ** 48) + Fraction(1, 2 ** 80)
