@@ -23,6 +23,13 @@
  *         Wq    int8  [N, K], row-major
  *         scale float [N]
  *
+ *   e4m3 ("RT-J -- FP8 E4M3 checkpoints", section "FP8 Format"): every weight
+ *       stored directly as PyTorch float8_e4m3fn, no scale: sign, 4 exponent
+ *       bits (bias 7), 3 mantissa bits, subnormals m * 2^-9, largest 448; the
+ *       codes S.1111.111 are NaN in the format and are not weights (the GEMM
+ *       kernels read them as +-480).
+ *         W     uint8 [N, K], row-major
+ *
  * Activations X are fp32 [M, K] row-major and results Y are fp32 [M, N]
  * row-major.  There is no bias term (the cards keep biases in fp32 outside
  * the quantized projections).
@@ -78,6 +85,13 @@ typedef enum rt_status {
     RT_ERR_UNSUPPORTED_DEVICE = 10 /* current device index >= 64, the library's per-device limit */
 } rt_status;
 
+/* Weight formats, where an entry point takes a `fmt` argument. */
+typedef enum rt_format {
+    RT_FMT_E4M3 = 3,    /* FP8 E4M3 codes [N, K], no scales (scales pointer unused, may be NULL) */
+    RT_FMT_Q4 = 4,      /* q4 g32 codes [N, K/2] + binary16 (scale, min) [N, K/32, 2] */
+    RT_FMT_Q8 = 8       /* q8 codes [N, K] + fp32 row scales [N] */
+} rt_format;
+
 typedef enum rt_path {
     RT_PATH_AUTO = 0,   /* SIMT for M <= 8 or K % 64 != 0, else TC */
     RT_PATH_SIMT = 1,   /* fp32 CUDA-core kernels */
@@ -104,7 +118,18 @@ rt_status rt_qgemm_q4(const float *X, const uint8_t *Wq, const uint16_t *scale_m
 rt_status rt_qgemm_q8(const float *X, const int8_t *Wq, const float *scale, float *Y,
                       int64_t M, int64_t N, int64_t K, int path, void *stream);
 
-/* Which path RT_PATH_AUTO takes for a q4 (fmt = 4) or q8 (fmt = 8) GEMM of
+/*
+ * Y = X * W^T with W the FP8 E4M3 weights, converted exactly to the operand
+ * type inside the GEMM.   (FP8 card, "FP8 Format")
+ * X [M,K] fp32, W [N,K] uint8 float8_e4m3fn codes, Y [M,N] fp32.  K % 16 == 0;
+ * everything else as for rt_qgemm_q8 (paths, kernels, precision: the SIMT
+ * path is exact up to fp32 accumulation, the tensor-core path rounds X to
+ * fp16 and keeps the weights exact).
+ */
+rt_status rt_gemm_e4m3(const float *X, const uint8_t *W, float *Y, int64_t M, int64_t N,
+                       int64_t K, int path, void *stream);
+
+/* Which path RT_PATH_AUTO takes for a GEMM of format fmt (rt_format) and
  * this shape: RT_PATH_SIMT or RT_PATH_TC; -1 for an unsupported shape. */
 int rt_qgemm_auto_path(int fmt, int64_t M, int64_t N, int64_t K);
 
@@ -197,7 +222,8 @@ rt_status rt_qgemm_noalloc(int fmt, const float *X, const void *Wq, const void *
  * each.
  *
  *   fmt       4: Wq/scales are q4 tensors as for rt_qgemm_q4;
- *             8: q8 tensors as for rt_qgemm_q8.
+ *             8: q8 tensors as for rt_qgemm_q8;
+ *             3: Wq are e4m3 codes as for rt_gemm_e4m3 (scales unused).
  *   reserved  must be 0.
  *   X, Y      fp32 [M, K] / [M, N] device buffers of this projection.
  *
@@ -293,6 +319,8 @@ int rt_qblock_fused(int64_t M, int64_t d_model, int64_t d_ff, int path);
  * and w13 a q8 [2*d_ff, d_model] tensor.
  *   fmt       4: Wq u8 [N, K/2] and scales binary16 [N, K/32, 2] (q4);
  *             8: Wq i8 [N, K] and scales fp32 [N] (q8);
+ *             3: Wq u8 [N, K] float8_e4m3fn codes, scales unused (the FP8
+ *                card's recipe: every block projection in e4m3);
  *   reserved  must be 0.
  * Shapes, outputs, launches, validation and errors are those of
  * rt_qblock_project; rt_qblock_project is this call with the int4 card's
@@ -348,6 +376,16 @@ rt_status rt_quantize_q4_g32(const float *W, int64_t N, int64_t K, int n_grid,
 rt_status rt_quantize_q8_row(const float *W, int64_t N, int64_t K, int8_t *Wq, float *scale);
 
 /*
+ * rt_quantize_e4m3 (FP8 card, "FP8 Format": weights stored directly as
+ * float8_e4m3fn): each of the n weights to the nearest E4M3 value, ties to
+ * the even code, the same rounding as PyTorch's float8_e4m3fn cast.  W fp32
+ * [n] -> codes uint8 [n].  Errors: RT_ERR_INVALID_ARG, RT_ERR_VALUE_RANGE (a
+ * weight is NaN or |w| > 464, which would round past 448; out is then
+ * incomplete).
+ */
+rt_status rt_quantize_e4m3(const float *W, int64_t n, uint8_t *out);
+
+/*
  * Dequantization exports (device pointers, stream-ordered).  They run the
  * same __device__ dequantization routines the GEMM kernels use, so tests can
  * check them bit for bit:
@@ -362,6 +400,12 @@ rt_status rt_dequant_q8_f32(const int8_t *Wq, const float *scale, float *W_out,
                             int64_t N, int64_t K, void *stream);
 rt_status rt_dequant_q4_f16(const uint8_t *Wq, const uint16_t *scale_min, uint16_t *W_out,
                             int64_t N, int64_t K, void *stream);
+/* e4m3 codes -> their exact values in fp32 / in fp16 bits (the tensor-core
+ * operand); K % 16 == 0, Wq and W_out 16-byte aligned. */
+rt_status rt_dequant_e4m3_f32(const uint8_t *Wq, float *W_out, int64_t N, int64_t K,
+                              void *stream);
+rt_status rt_dequant_e4m3_f16(const uint8_t *Wq, uint16_t *W_out, int64_t N, int64_t K,
+                              void *stream);
 
 /*
  * Synchronizes `stream`, then reads and clears the current device's status

@@ -23,6 +23,7 @@ __all__ = [
     "dequant_q4_f16", "device_status", "auto_path", "status_string",
     "qgemm_noalloc", "plan", "block_fused", "workspace_bytes", "debug_inject",
     "qgemm_batch", "batch_plan", "Proj", "QBlockFmt", "qblock_project_fmt", "block_fused_fmt",
+    "gemm_e4m3", "quantize_e4m3", "dequant_e4m3_f32", "dequant_e4m3_f16", "FMT_E4M3",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -35,6 +36,7 @@ RT_ERR_SCRATCH_LIMIT = 8
 RT_ERR_OPERAND_RANGE = 9
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024   # RT_NOALLOC_SCRATCH_BYTES in include/rtq.h
 PATHS = {"auto": 0, "simt": 1, "tc": 2}
+FMT_E4M3, FMT_Q4, FMT_Q8 = 3, 4, 8     # rt_format
 
 _p = ctypes.c_void_p
 _i64 = ctypes.c_int64
@@ -83,6 +85,14 @@ def lib() -> ctypes.CDLL:
         f = getattr(L, name)
         f.restype = _i32
         f.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _i32, _p]
+    L.rt_gemm_e4m3.restype = _i32
+    L.rt_gemm_e4m3.argtypes = [_p, _p, _p, _i64, _i64, _i64, _i32, _p]
+    L.rt_quantize_e4m3.restype = _i32
+    L.rt_quantize_e4m3.argtypes = [_p, _i64, _p]
+    for name in ("rt_dequant_e4m3_f32", "rt_dequant_e4m3_f16"):
+        f = getattr(L, name)
+        f.restype = _i32
+        f.argtypes = [_p, _p, _i64, _i64, _p]
     L.rt_qgemm_noalloc.restype = _i32
     L.rt_qgemm_noalloc.argtypes = [_i32, _p, _p, _p, _p, _i64, _i64, _i64, _i32, _p]
     L.rt_qgemm_auto_path.restype = _i32
@@ -141,6 +151,22 @@ def rt_qgemm_q4(X, Wq, scale_min, Y, M, N, K, path, stream) -> int:
 
 def rt_qgemm_q8(X, Wq, scale, Y, M, N, K, path, stream) -> int:
     return lib().rt_qgemm_q8(X, Wq, scale, Y, M, N, K, path, stream)
+
+
+def rt_gemm_e4m3(X, W, Y, M, N, K, path, stream) -> int:
+    return lib().rt_gemm_e4m3(X, W, Y, M, N, K, path, stream)
+
+
+def rt_quantize_e4m3(W, n, out) -> int:
+    return lib().rt_quantize_e4m3(W, n, out)
+
+
+def rt_dequant_e4m3_f32(Wq, W_out, N, K, stream) -> int:
+    return lib().rt_dequant_e4m3_f32(Wq, W_out, N, K, stream)
+
+
+def rt_dequant_e4m3_f16(Wq, W_out, N, K, stream) -> int:
+    return lib().rt_dequant_e4m3_f16(Wq, W_out, N, K, stream)
 
 
 def rt_qgemm_noalloc(fmt, X, Wq, scales, Y, M, N, K, path, stream) -> int:
@@ -255,10 +281,26 @@ def _shape(t, shape, name):
 
 
 def _packed_shapes(fmt: int, N: int, K: int):
-    """Shapes of the codes and the scales of an N x K weight in format q4 / q8."""
+    """Shapes of the codes and the scales of an N x K weight in format q4 / q8
+    (e4m3 has no scales: None)."""
     if fmt == 4:
         return (N, K // 2), (N, K // 32, 2)
+    if fmt == FMT_E4M3:
+        return (N, K), None
     return (N, K), (N,)
+
+
+_DTYPES = {4: ("uint8", "uint16"), 8: ("int8", "float32"), FMT_E4M3: ("uint8", None)}
+
+
+def _weight_ptrs(fmt, Wq, scales, name):
+    """(codes, scales) pointers of one weight, dtypes checked (scales None for e4m3)."""
+    import torch
+    wdt, sdt = _DTYPES[fmt]
+    w = _dev(Wq, getattr(torch, wdt), name)
+    if sdt is None:
+        return w, None
+    return w, _dev(scales, getattr(torch, sdt), name + " scales")
 
 
 def _check_gemm_shapes(fmt, X, Wq, scales, Y):
@@ -268,7 +310,8 @@ def _check_gemm_shapes(fmt, X, Wq, scales, Y):
     N = Wq.shape[0]
     wshape, sshape = _packed_shapes(fmt, N, K)
     _shape(Wq, wshape, "Wq")
-    _shape(scales, sshape, "scale_min" if fmt == 4 else "scale")
+    if sshape is not None:
+        _shape(scales, sshape, "scale_min" if fmt == 4 else "scale")
     if Y is not None:
         _shape(Y, (M, N), "Y")
     return M, N, K
@@ -297,6 +340,18 @@ def qgemm_q8(X, Wq, scale, Y=None, path="auto", stream=None):
                      _dev(scale, torch.float32, "scale"), _dev(Y, torch.float32, "Y"),
                      M, N, K, _path(path), _stream_ptr(stream))
     _check(st, "rt_qgemm_q8")
+    return Y
+
+
+def gemm_e4m3(X, W, Y=None, path="auto", stream=None):
+    """Y[M,N] = X[M,K] @ e4m3(W[N,K])^T on the GPU (W: uint8 float8_e4m3fn codes)."""
+    import torch
+    M, N, K = _check_gemm_shapes(FMT_E4M3, X, W, None, Y)
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float32, device=X.device)
+    st = rt_gemm_e4m3(_dev(X, torch.float32, "X"), _dev(W, torch.uint8, "W"),
+                      _dev(Y, torch.float32, "Y"), M, N, K, _path(path), _stream_ptr(stream))
+    _check(st, "rt_gemm_e4m3")
     return Y
 
 
@@ -330,14 +385,14 @@ def _batch_array(projs, M):
     import torch
     arr = (_QProjC * max(1, len(projs)))()
     for i, q in enumerate(projs):
-        if q.fmt not in (4, 8):
-            raise ValueError(f"entry {i}: fmt must be 4 or 8, got {q.fmt}")
+        if q.fmt not in _DTYPES:
+            raise ValueError(f"entry {i}: fmt must be 4, 8 or 3 (e4m3), got {q.fmt}")
         if q.X.dim() != 2 or q.X.shape[0] != M:
             raise ValueError(f"entry {i}: X must be [M={M}, K], got {tuple(q.X.shape)}")
         _, N, K = _check_gemm_shapes(q.fmt, q.X, q.Wq, q.scales, q.Y)
-        wdt, sdt = (torch.uint8, torch.uint16) if q.fmt == 4 else (torch.int8, torch.float32)
-        arr[i] = _QProjC(q.fmt, 0, _dev(q.X, torch.float32, "X"), _dev(q.Wq, wdt, "Wq"),
-                         _dev(q.scales, sdt, "scales"), _dev(q.Y, torch.float32, "Y"), N, K)
+        w, sc = _weight_ptrs(q.fmt, q.Wq, q.scales, f"entry {i} Wq")
+        arr[i] = _QProjC(q.fmt, 0, _dev(q.X, torch.float32, "X"), w, sc,
+                         _dev(q.Y, torch.float32, "Y"), N, K)
     return arr
 
 
@@ -427,13 +482,13 @@ class QBlockFmt:
         ws = []
         for name, N, K in (("qkvg", 4 * d, d), ("wo", d, d), ("w13", 2 * f, d), ("w2", d, f)):
             fmt, Wq, S = getattr(self, name)
-            if fmt not in (4, 8):
-                raise ValueError(f"{name}: fmt must be 4 or 8, got {fmt}")
+            if fmt not in _DTYPES:
+                raise ValueError(f"{name}: fmt must be 4, 8 or 3 (e4m3), got {fmt}")
             wshape, sshape = _packed_shapes(fmt, N, K)
             _shape(Wq, wshape, name)
-            _shape(S, sshape, name + " scales")
-            wdt, sdt = (torch.uint8, torch.uint16) if fmt == 4 else (torch.int8, torch.float32)
-            ws.append(_QWeightC(fmt, 0, _dev(Wq, wdt, name), _dev(S, sdt, name + " scales")))
+            if sshape is not None:
+                _shape(S, sshape, name + " scales")
+            ws.append(_QWeightC(fmt, 0, *_weight_ptrs(fmt, Wq, S, name)))
         return _QBlockFmtC(*ws, d, f)
 
 
@@ -472,6 +527,33 @@ def quantize_q4_g32(W: np.ndarray, n_grid: int = 21):
     st = rt_quantize_q4_g32(W.ctypes.data, N, K, n_grid, Wq.ctypes.data, sm.ctypes.data)
     _check(st, "rt_quantize_q4_g32")
     return Wq, sm
+
+
+def quantize_e4m3(W: np.ndarray) -> np.ndarray:
+    """Host FP8 quantizer: float8_e4m3fn codes (uint8, same shape as W)."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    out = np.empty(W.shape, dtype=np.uint8)
+    _check(rt_quantize_e4m3(W.ctypes.data, W.size, out.ctypes.data), "rt_quantize_e4m3")
+    return out
+
+
+def dequant_e4m3_f32(Wq, stream=None):
+    import torch
+    N, K = Wq.shape
+    out = torch.empty((N, K), dtype=torch.float32, device=Wq.device)
+    _check(rt_dequant_e4m3_f32(_dev(Wq, torch.uint8, "Wq"), _dev(out, torch.float32, "W_out"),
+                               N, K, _stream_ptr(stream)), "rt_dequant_e4m3_f32")
+    return out
+
+
+def dequant_e4m3_f16(Wq, stream=None):
+    """The tensor-core operand of e4m3 weights, as fp16 bits (uint16) [N, K]."""
+    import torch
+    N, K = Wq.shape
+    out = torch.empty((N, K), dtype=torch.uint16, device=Wq.device)
+    _check(rt_dequant_e4m3_f16(_dev(Wq, torch.uint8, "Wq"), _dev(out, torch.uint16, "W_out"),
+                               N, K, _stream_ptr(stream)), "rt_dequant_e4m3_f16")
+    return out
 
 
 def quantize_q8_row(W: np.ndarray):

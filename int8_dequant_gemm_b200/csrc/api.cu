@@ -97,25 +97,32 @@ inline bool overlap(const void *a, int64_t abytes, const void *b, int64_t bbytes
 
 constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
 
-// Validation shared by both formats.  wbytes/sbytes: sizes of the payload and
-// the scale tensor; walign/salign: their required alignment.
+// Validation shared by the formats.  wbytes/sbytes: sizes of the payload and
+// the scale tensor (sbytes 0: the format has none and S is not read);
+// salign: the scales' required alignment.
 rt_status validate(const float *X, const void *Wq, const void *S, const float *Y, int64_t M,
                    int64_t N, int64_t K, int64_t wbytes, int64_t sbytes, uintptr_t salign,
                    int64_t k_granule) {
     if (M < 0 || N < 1 || K < 1 || M > kMaxDim || N > kMaxDim || K > kMaxDim)
         return RT_ERR_INVALID_ARG;
     if (K % k_granule != 0) return RT_ERR_UNSUPPORTED_SHAPE;
-    if (!Wq || !S) return RT_ERR_INVALID_ARG;
+    if (!Wq || (sbytes > 0 && !S)) return RT_ERR_INVALID_ARG;
     if (M > 0 && (!X || !Y)) return RT_ERR_INVALID_ARG;
-    if (!aligned(Wq, 16) || !aligned(S, salign)) return RT_ERR_ALIGNMENT;
+    if (!aligned(Wq, 16) || (sbytes > 0 && !aligned(S, salign))) return RT_ERR_ALIGNMENT;
     if (M > 0 && (!aligned(X, 16) || !aligned(Y, 16))) return RT_ERR_ALIGNMENT;
     if (M > 0) {
         const int64_t ybytes = M * N * 4;
         if (overlap(Y, ybytes, X, M * K * 4) || overlap(Y, ybytes, Wq, wbytes) ||
-            overlap(Y, ybytes, S, sbytes))
+            (sbytes > 0 && overlap(Y, ybytes, S, sbytes)))
             return RT_ERR_INVALID_ARG;
     }
     return RT_OK;
+}
+
+// Bytes of the packed codes and of the scales of an N x K weight.
+int64_t code_bytes(int fmt, int64_t N, int64_t K) { return fmt == 4 ? N * (K / 2) : N * K; }
+int64_t scale_bytes(int fmt, int64_t N, int64_t K) {
+    return fmt == 4 ? N * (K / 32) * 4 : (fmt == 8 ? N * 4 : 0);
 }
 
 int pick_kernel(int fmt, int64_t M, int64_t N, int64_t K, int p) {
@@ -146,41 +153,32 @@ rt_status run_gemm(int fmt, const float *X, const void *Wq, const void *S, float
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
     const int kern = pick_kernel(fmt, M, N, K, p);
-    const bool q4 = fmt == 4;
-    const auto *w4 = static_cast<const uint8_t *>(Wq);
-    const auto *w8 = static_cast<const int8_t *>(Wq);
-    const auto *s4 = static_cast<const uint16_t *>(S);
-    const auto *s8 = static_cast<const float *>(S);
-    if (kern == RT_KERNEL_SIMT)
-        return from_cuda(q4 ? rtq::launch_simt_q4(X, w4, s4, Y, m, n, k, s)
-                            : rtq::launch_simt_q8(X, w8, s8, Y, m, n, k, s));
+    if (kern == RT_KERNEL_SIMT) return from_cuda(rtq::launch_simt(fmt, X, Wq, S, Y, m, n, k, s));
     DevCtl *ctl = nullptr;
     rt_status st = ctl_block(&ctl);
     if (st != RT_OK) return st;
     if (kern == RT_KERNEL_TC_W_STATIONARY)
-        return from_cuda(q4 ? rtq::launch_tc_q4(X, w4, s4, Y, m, n, k, ctl, s)
-                            : rtq::launch_tc_q8(X, w8, s8, Y, m, n, k, ctl, s));
+        return from_cuda(rtq::launch_tc(fmt, X, Wq, S, Y, m, n, k, ctl, s));
     void *xh = nullptr;
     if ((st = workspace(s, static_cast<size_t>(M) * K * 2, &xh)) != RT_OK) return st;
     cudaError_t e = rtq::launch_cvt_x16(X, xh, M, K, ctl, s);
     if (e != cudaSuccess) return RT_ERR_CUDA;
     if (kern == RT_KERNEL_TC_X_RESIDENT)
-        return from_cuda(q4 ? rtq::launch_xs_q4(xh, w4, s4, Y, m, n, k, ctl, s)
-                            : rtq::launch_xs_q8(xh, w8, s8, Y, m, n, k, ctl, s));
-    return from_cuda(q4 ? rtq::launch_ws_q4(xh, w4, s4, Y, m, n, k, ctl, s)
-                        : rtq::launch_ws_q8(xh, w8, s8, Y, m, n, k, ctl, s));
+        return from_cuda(rtq::launch_xs(fmt, xh, Wq, S, Y, m, n, k, ctl, s));
+    return from_cuda(rtq::launch_ws(fmt, xh, Wq, S, Y, m, n, k, ctl, s));
 }
 
 }  // namespace
 
 namespace rtq {
 
-// The checks rt_qgemm_q4 (fmt 4) and rt_qgemm_q8 (fmt 8) apply, for the
-// fixed-scratch entry point in noalloc.cu.
+// The checks rt_qgemm_q4 (fmt 4), rt_qgemm_q8 (fmt 8) and rt_gemm_e4m3
+// (fmt 3) apply; also used by the fixed-scratch entry point in noalloc.cu.
 rt_status check_gemm_args(int fmt, const float *X, const void *Wq, const void *S, const float *Y,
                           int64_t M, int64_t N, int64_t K) {
-    return fmt == 4 ? validate(X, Wq, S, Y, M, N, K, N * (K / 2), N * (K / 32) * 4, 4, 32)
-                    : validate(X, Wq, S, Y, M, N, K, N * K, N * 4, 4, 16);
+    if (!rtq::fmt_valid(fmt)) return RT_ERR_INVALID_ARG;
+    return validate(X, Wq, S, Y, M, N, K, code_bytes(fmt, N, K), scale_bytes(fmt, N, K), 4,
+                    fmt == 4 ? 32 : 16);
 }
 
 rt_status device_ctl(DevCtl **out) { return ctl_block(out); }
@@ -209,13 +207,13 @@ const char *rt_status_string(int status) {
 int rt_version(void) { return 200; }
 
 int rt_qgemm_auto_path(int fmt, int64_t M, int64_t N, int64_t K) {
-    if ((fmt != 4 && fmt != 8) || M < 0 || N < 1 || K < 1) return -1;
+    if (!rtq::fmt_valid(fmt) || M < 0 || N < 1 || K < 1) return -1;
     if (K % (fmt == 4 ? 32 : 16) != 0) return -1;
     return pick_path(M, K, RT_PATH_AUTO);
 }
 
 int rt_qgemm_plan(int fmt, int64_t M, int64_t N, int64_t K, int path) {
-    if ((fmt != 4 && fmt != 8) || M < 0 || N < 1 || K < 1 || M > kMaxDim || N > kMaxDim ||
+    if (!rtq::fmt_valid(fmt) || M < 0 || N < 1 || K < 1 || M > kMaxDim || N > kMaxDim ||
         K > kMaxDim)
         return -1;
     if (K % (fmt == 4 ? 32 : 16) != 0) return -1;
@@ -236,6 +234,13 @@ rt_status rt_qgemm_q8(const float *X, const int8_t *Wq, const float *scale, floa
     rt_status st = validate(X, Wq, scale, Y, M, N, K, N * K, N * 4, 4, 16);
     if (st != RT_OK) return st;
     return run_gemm(8, X, Wq, scale, Y, M, N, K, path, stream);
+}
+
+rt_status rt_gemm_e4m3(const float *X, const uint8_t *W, float *Y, int64_t M, int64_t N,
+                       int64_t K, int path, void *stream) {
+    rt_status st = rtq::check_gemm_args(rtq::kFmtE4M3, X, W, nullptr, Y, M, N, K);
+    if (st != RT_OK) return st;
+    return run_gemm(rtq::kFmtE4M3, X, W, nullptr, Y, M, N, K, path, stream);
 }
 
 int64_t rt_workspace_bytes(int fmt, int64_t M, int64_t N, int64_t K, int path) {
@@ -287,7 +292,7 @@ int block_route(const int fmt[4], int64_t M, int64_t d, int64_t f, int path) {
     const int64_t NK[4][2] = {{4 * d, d}, {d, d}, {2 * f, d}, {d, f}};
     bool fused = M >= 1 && M <= 128;
     for (int i = 0; i < 4; ++i) {
-        if (fmt[i] != 4 && fmt[i] != 8) return -1;
+        if (!rtq::fmt_valid(fmt[i])) return -1;
         const int kern = rt_qgemm_plan(fmt[i], M, NK[i][0], NK[i][1], path);
         if (kern < 0) return -1;
         fused = fused && kern == RT_KERNEL_TC_W_STATIONARY;
@@ -302,7 +307,7 @@ rt_status block_run(const BlockProj p[4], int64_t M, int64_t d, int64_t f, int p
     int fmts[4];
     for (int i = 0; i < 4; ++i) {
         const BlockProj &q = p[i];
-        if (q.fmt != 4 && q.fmt != 8) return RT_ERR_INVALID_ARG;
+        if (!rtq::fmt_valid(q.fmt)) return RT_ERR_INVALID_ARG;
         fmts[i] = q.fmt;
         if ((st = rtq::check_gemm_args(q.fmt, q.X, q.W, q.S, q.Y, M, q.N, q.K)) != RT_OK)
             return st;
@@ -317,11 +322,11 @@ rt_status block_run(const BlockProj p[4], int64_t M, int64_t d, int64_t f, int p
             const int64_t yb = M * p[i].N * 4;
             for (int j = 0; j < 4; ++j) {
                 if (j == i) continue;
-                const int64_t wb = p[j].fmt == 4 ? p[j].N * (p[j].K / 2) : p[j].N * p[j].K;
-                const int64_t sb = p[j].fmt == 4 ? p[j].N * (p[j].K / 32) * 4 : p[j].N * 4;
+                const int64_t wb = code_bytes(p[j].fmt, p[j].N, p[j].K);
+                const int64_t sb = scale_bytes(p[j].fmt, p[j].N, p[j].K);
                 if (overlap(p[i].Y, yb, p[j].Y, M * p[j].N * 4) ||
                     overlap(p[i].Y, yb, p[j].X, M * p[j].K * 4) || overlap(p[i].Y, yb, p[j].W, wb) ||
-                    overlap(p[i].Y, yb, p[j].S, sb))
+                    (sb > 0 && overlap(p[i].Y, yb, p[j].S, sb)))
                     return RT_ERR_INVALID_ARG;
             }
         }
@@ -417,7 +422,7 @@ int batch_route(const rt_qproj *list, int count, int64_t M, int path) {
     int64_t tiles = 0;
     for (int i = 0; i < count; ++i) {
         const rt_qproj &q = list[i];
-        if ((q.fmt != 4 && q.fmt != 8) || q.reserved != 0) return -RT_ERR_INVALID_ARG;
+        if (!rtq::fmt_valid(q.fmt) || q.reserved != 0) return -RT_ERR_INVALID_ARG;
         const rt_status st = rtq::check_gemm_args(q.fmt, q.X, q.Wq, q.scales, q.Y, M, q.N, q.K);
         if (st != RT_OK) return -st;
         const int p = pick_path(M, q.K, path);
@@ -439,8 +444,8 @@ int batch_route(const rt_qproj *list, int count, int64_t M, int path) {
         r.reserve(static_cast<size_t>(count) * 4);
         for (int i = 0; i < count; ++i) {
             const rt_qproj &q = list[i];
-            const int64_t wb = q.fmt == 4 ? q.N * (q.K / 2) : q.N * q.K;
-            const int64_t sb = q.fmt == 4 ? q.N * (q.K / 32) * 4 : q.N * 4;
+            const int64_t wb = code_bytes(q.fmt, q.N, q.K);
+            const int64_t sb = scale_bytes(q.fmt, q.N, q.K);
             auto add = [&](const void *p, int64_t n, bool out) {
                 const uintptr_t a = reinterpret_cast<uintptr_t>(p);
                 r.push_back({a, a + static_cast<uintptr_t>(n), out});
@@ -448,7 +453,7 @@ int batch_route(const rt_qproj *list, int count, int64_t M, int path) {
             add(q.Y, M * q.N * 4, true);
             add(q.X, M * q.K * 4, false);
             add(q.Wq, wb, false);
-            add(q.scales, sb, false);
+            if (sb > 0) add(q.scales, sb, false);
         }
         std::sort(r.begin(), r.end(), [](const Range &a, const Range &b) { return a.lo < b.lo; });
         // In address order, each range is checked against the furthest end
@@ -496,6 +501,22 @@ rt_status rt_dequant_q8_f32(const int8_t *Wq, const float *scale, float *W_out, 
     return from_cuda(rtq::launch_dequant_q8_f32(Wq, scale, W_out, static_cast<int>(N),
                                                 static_cast<int>(K),
                                                 static_cast<cudaStream_t>(stream)));
+}
+
+rt_status rt_dequant_e4m3_f32(const uint8_t *Wq, float *W_out, int64_t N, int64_t K,
+                              void *stream) {
+    rt_status st = validate_dequant(Wq, W_out, W_out, N, K, 16, 4);
+    if (st != RT_OK) return st;
+    return from_cuda(rtq::launch_dequant_e4m3(Wq, W_out, static_cast<int>(N), static_cast<int>(K),
+                                              false, static_cast<cudaStream_t>(stream)));
+}
+
+rt_status rt_dequant_e4m3_f16(const uint8_t *Wq, uint16_t *W_out, int64_t N, int64_t K,
+                              void *stream) {
+    rt_status st = validate_dequant(Wq, W_out, W_out, N, K, 16, 4);
+    if (st != RT_OK) return st;
+    return from_cuda(rtq::launch_dequant_e4m3(Wq, W_out, static_cast<int>(N), static_cast<int>(K),
+                                              true, static_cast<cudaStream_t>(stream)));
 }
 
 rt_status rt_dequant_q4_f16(const uint8_t *Wq, const uint16_t *scale_min, uint16_t *W_out,

@@ -106,6 +106,37 @@ __device__ __forceinline__ uint4 q8_words_f16(uint32_t a, uint32_t b) {
                       h2_bits(__hsub2(bits_h2(__byte_perm(ub, 0x64646464u, 0x4341)), k1152)));
 }
 
+// FP8 E4M3 ("RT-J -- FP8 E4M3 checkpoints", "FP8 Format": weights stored
+// directly as float8_e4m3fn, no scale).  A code b = S EEEE MMM reads as
+// (1 + M/8) * 2^(E-7), or M * 2^-9 when E = 0.  Its low seven bits shifted left
+// by 7 are an fp16 pattern worth exactly that value times 2^-8 (exponent bias
+// 15 instead of 7; the E = 0 codes land on fp16 subnormals with the same
+// factor), so one exact fp16 multiplication by 256 finishes the conversion.
+// The two NaN codes S.1111.111 are not weights; they read as +-480.
+__device__ __forceinline__ uint32_t e4m3_pair_f16(uint32_t x) {
+    // x holds two codes in the low bytes of its 16-bit halves
+    const uint32_t h = ((x & 0x007F007Fu) << 7) | ((x & 0x00800080u) << 8);
+    return h2_bits(__hmul2(bits_h2(h), bits_h2(0x5C005C00u)));   // x 256, exact
+}
+
+// e4m3, fp16 operands: two payload words (codes 0..3, 4..7) -> one chunk.
+__device__ __forceinline__ uint4 e4m3_words_f16(uint32_t a, uint32_t b) {
+    return make_uint4(e4m3_pair_f16(__byte_perm(a, 0u, 0x4240)),
+                      e4m3_pair_f16(__byte_perm(a, 0u, 0x4341)),
+                      e4m3_pair_f16(__byte_perm(b, 0u, 0x4240)),
+                      e4m3_pair_f16(__byte_perm(b, 0u, 0x4341)));
+}
+
+// e4m3 code (byte i of v) -> fp32, exact: the integer (8 + M) << (E - 1), or
+// M for E = 0, times 2^-9.
+__device__ __forceinline__ float e4m3_byte_f32(uint32_t v, int i) {
+    const uint32_t b = (v >> (8 * i)) & 0xFFu;
+    const uint32_t e = (b >> 3) & 0xFu, m = b & 7u;
+    const uint32_t mag = e == 0 ? m : (8u + m) << (e - 1);
+    const float f = static_cast<float>(mag) * 0.001953125f;   // 2^-9
+    return (b & 0x80u) ? -f : f;
+}
+
 // Chunk in operand order -> natural order (for the dequantization exports).
 __device__ __forceinline__ uint4 chunk_to_natural(uint4 c) {
     return make_uint4(__byte_perm(c.x, c.y, 0x5410), __byte_perm(c.x, c.y, 0x7632),

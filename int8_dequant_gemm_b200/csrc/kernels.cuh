@@ -12,6 +12,15 @@ namespace rtq {
 
 constexpr int kMaxDevices = 64;
 
+// Weight formats (the `fmt` arguments): q4 g32 with (scale, min), q8 with a
+// row scale, FP8 E4M3 without scale.  The e4m3 payload has the q8 layout
+// (one byte per weight, [N, K]); kernels treat it as q8 with another byte
+// conversion and no scale.
+constexpr int kFmtQ4 = 4;
+constexpr int kFmtQ8 = 8;
+constexpr int kFmtE4M3 = 3;
+inline bool fmt_valid(int f) { return f == kFmtQ4 || f == kFmtQ8 || f == kFmtE4M3; }
+
 // Per-device control block, one __device__ instance (api.cu).  Every
 // tensor-core kernel reads `wait_ns` and `inject` at its start and ORs status
 // bits into `status`; rt_device_status() reads and clears the bits.
@@ -44,17 +53,13 @@ cudaError_t smem_attr_once(Kernel kernel, int bytes, int dev, std::atomic<bool> 
 }
 
 // fp32 CUDA-core path: one thread per output row, MT activation rows per block.
-cudaError_t launch_simt_q4(const float *X, const uint8_t *Wq, const uint16_t *SM, float *Y,
-                           int M, int N, int K, cudaStream_t s);
-cudaError_t launch_simt_q8(const float *X, const int8_t *Wq, const float *S, float *Y, int M,
-                           int N, int K, cudaStream_t s);
+cudaError_t launch_simt(int fmt, const float *X, const void *Wq, const void *S, float *Y, int M,
+                        int N, int K, cudaStream_t s);
 
 // tcgen05 path: 128 weight rows x BN activation rows per CTA, fp16 operands
 // in swizzled shared memory, fp32 accumulator in TMEM.
-cudaError_t launch_tc_q4(const float *X, const uint8_t *Wq, const uint16_t *SM, float *Y, int M,
-                         int N, int K, DevCtl *ctl, cudaStream_t s);
-cudaError_t launch_tc_q8(const float *X, const int8_t *Wq, const float *S, float *Y, int M, int N,
-                         int K, DevCtl *ctl, cudaStream_t s);
+cudaError_t launch_tc(int fmt, const float *X, const void *Wq, const void *S, float *Y, int M,
+                      int N, int K, DevCtl *ctl, cudaStream_t s);
 
 // Up to kMaxGroup independent projections with the same M (1..128) in one
 // launch of the same tcgen05 tile code: X [M, K] fp32, Wq/S as for
@@ -81,18 +86,14 @@ cudaError_t launch_cvt_x16(const float *X, void *Xh, int64_t M, int64_t K, DevCt
 // (K a multiple of 128 up to 512, many activation rows); see xs.cu.  Xh is the
 // pre-pass output.
 bool xs_supported(int M, int N, int K);
-cudaError_t launch_xs_q4(const void *Xh, const uint8_t *Wq, const uint16_t *SM, float *Y, int M,
-                         int N, int K, DevCtl *ctl, cudaStream_t s);
-cudaError_t launch_xs_q8(const void *Xh, const int8_t *Wq, const float *S, float *Y, int M, int N,
-                         int K, DevCtl *ctl, cudaStream_t s);
+cudaError_t launch_xs(int fmt, const void *Xh, const void *Wq, const void *S, float *Y, int M,
+                      int N, int K, DevCtl *ctl, cudaStream_t s);
 
 // tcgen05, persistent weight-stationary tiles with both operands TMA-staged
 // (more than 128 activation rows, any K of the format's TMA granule); see ws.cu.
 bool ws_supported(int fmt, int M, int N, int K);
-cudaError_t launch_ws_q4(const void *Xh, const uint8_t *Wq, const uint16_t *SM, float *Y, int M,
-                         int N, int K, DevCtl *ctl, cudaStream_t s);
-cudaError_t launch_ws_q8(const void *Xh, const int8_t *Wq, const float *S, float *Y, int M, int N,
-                         int K, DevCtl *ctl, cudaStream_t s);
+cudaError_t launch_ws(int fmt, const void *Xh, const void *Wq, const void *S, float *Y, int M,
+                      int N, int K, DevCtl *ctl, cudaStream_t s);
 
 // tcgen05, a list of independent projections with the same M (1..128) in
 // persistent launches that stream every projection's weights back to back;
@@ -120,9 +121,12 @@ cudaError_t launch_dequant_q4_f16(const uint8_t *Wq, const uint16_t *SM, uint16_
                                   int K, cudaStream_t s);
 cudaError_t launch_dequant_q8_f32(const int8_t *Wq, const float *S, float *W, int N, int K,
                                   cudaStream_t s);
+cudaError_t launch_dequant_e4m3(const uint8_t *Wq, void *W, int N, int K, bool f16,
+                                cudaStream_t s);
 
-// Argument checks of rt_qgemm_q4 / rt_qgemm_q8 (fmt 4 / 8) and the control
-// block of the current device (api.cu).
+// Argument checks of rt_qgemm_q4 / rt_qgemm_q8 / rt_gemm_e4m3 (fmt 4 / 8 / 3;
+// S is unused and may be null for e4m3) and the control block of the current
+// device (api.cu).
 rt_status check_gemm_args(int fmt, const float *X, const void *Wq, const void *S, const float *Y,
                           int64_t M, int64_t N, int64_t K);
 rt_status device_ctl(DevCtl **out);

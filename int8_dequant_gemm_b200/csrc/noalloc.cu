@@ -67,23 +67,14 @@ extern "C" rt_status rt_qgemm_noalloc(int fmt, const float *X, const void *Wq, c
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
-    const bool q4 = fmt == 4;
-    const auto *w4 = static_cast<const uint8_t *>(Wq);
-    const auto *w8 = static_cast<const int8_t *>(Wq);
-    const auto *s4 = static_cast<const uint16_t *>(scales);
-    const auto *s8 = static_cast<const float *>(scales);
     if (kern == RT_KERNEL_SIMT)
-        return from_cuda(q4 ? rtq::launch_simt_q4(X, w4, s4, Y, m, n, k, s)
-                            : rtq::launch_simt_q8(X, w8, s8, Y, m, n, k, s));
+        return from_cuda(rtq::launch_simt(fmt, X, Wq, scales, Y, m, n, k, s));
     rtq::DevCtl *ctl = nullptr;
     if ((st = rtq::device_ctl(&ctl)) != RT_OK) return st;
     if (kern == RT_KERNEL_TC_W_STATIONARY)
-        return from_cuda(q4 ? rtq::launch_tc_q4(X, w4, s4, Y, m, n, k, ctl, s)
-                            : rtq::launch_tc_q8(X, w8, s8, Y, m, n, k, ctl, s));
+        return from_cuda(rtq::launch_tc(fmt, X, Wq, scales, Y, m, n, k, ctl, s));
     if (rtq::launch_cvt_x16(X, xh, M, K, ctl, s) != cudaSuccess) return RT_ERR_CUDA;
     if (kern == RT_KERNEL_TC_X_RESIDENT)
-        return from_cuda(q4 ? rtq::launch_xs_q4(xh, w4, s4, Y, m, n, k, ctl, s)
-                            : rtq::launch_xs_q8(xh, w8, s8, Y, m, n, k, ctl, s));
-    return from_cuda(q4 ? rtq::launch_ws_q4(xh, w4, s4, Y, m, n, k, ctl, s)
-                        : rtq::launch_ws_q8(xh, w8, s8, Y, m, n, k, ctl, s));
+        return from_cuda(rtq::launch_xs(fmt, xh, Wq, scales, Y, m, n, k, ctl, s));
+    return from_cuda(rtq::launch_ws(fmt, xh, Wq, scales, Y, m, n, k, ctl, s));
 }

@@ -170,11 +170,11 @@ __device__ __forceinline__ void dequant_slot(uint32_t wslot, uint32_t sslot, int
         const int wi = (2 * s + h) & 3;
         R.smw = wi == 0 ? sc.x : wi == 1 ? sc.y : wi == 2 ? sc.z : sc.w;
         half_words<4>(R, w);
-    } else {
+    } else {   // q8 and e4m3: one byte per weight
         R.p0 = lds_v4(wslot + r * 256 + wswz(4 * s + 2 * h, r) * 16);
         R.p1 = lds_v4(wslot + r * 256 + wswz(4 * s + 2 * h + 1, r) * 16);
         R.smw = 0;
-        half_words<8>(R, w);
+        half_words<FMT>(R, w);
     }
 }
 
@@ -345,10 +345,12 @@ __global__ void __launch_bounds__(kPlThreads, 1)
                         const uint32_t sslot = base + L.s_off + slot * kScaleBytes;
                         for (int s = 0; s < nsteps; ++s, ++ja) {
                             uint32_t wv[16];
-                            if (p.fmt == 4)
-                                dequant_slot<4>(wslot, sslot, r, h, s, wv);
+                            if (p.fmt == kFmtQ4)
+                                dequant_slot<kFmtQ4>(wslot, sslot, r, h, s, wv);
+                            else if (p.fmt == kFmtQ8)
+                                dequant_slot<kFmtQ8>(wslot, sslot, r, h, s, wv);
                             else
-                                dequant_slot<8>(wslot, sslot, r, h, s, wv);
+                                dequant_slot<kFmtE4M3>(wslot, sslot, r, h, s, wv);
                             const int st = ja % kAStages;
                             if (ja >= kAStages &&
                                 !mbar_wait(&a_empty[st], static_cast<uint32_t>((ja / kAStages) - 1) & 1u,

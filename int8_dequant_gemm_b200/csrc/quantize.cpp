@@ -6,6 +6,8 @@
 //   a min-MSE clip search over the shrink grid 1.0 -> 0.8.
 // q8 per-row: "RT-J -- int8 (Q8_0-style) quantized checkpoints", section
 //   "Quantization format" -- scale[o] = max|W[o,:]|/127, W ~= q*scale[o].
+// e4m3: "RT-J -- FP8 E4M3 checkpoints", section "FP8 Format" -- every weight
+//   stored directly as float8_e4m3fn, no scale.
 //
 // The grid, rounding and tie rules are spelled out in include/rtq.h.  All
 // weight arithmetic is IEEE double with no contraction (this file is built
@@ -152,5 +154,39 @@ extern "C" rt_status rt_quantize_q8_row(const float *W, int64_t N, int64_t K, in
     for (int64_t i = 0; i < N * K; ++i)
         if (!std::isfinite(W[i])) return RT_ERR_VALUE_RANGE;
     parallel_rows(N, K, [&](int64_t a, int64_t b) { q8_rows(W, a, b, K, Wq, scale); });
+    return RT_OK;
+}
+
+namespace {
+
+// One weight to its float8_e4m3fn code: round to nearest, ties to even, from
+// the binade of |w|.  Below 2^-6 the step is 2^-9 (subnormal codes 0..7; a
+// rounded 8 is the smallest normal code 0x08); from 2^-6 on, |w| = f * 2^E
+// with f in [1, 2) takes code ((E + 7) << 3) + round(8 (f - 1)), where a
+// rounded 8 carries into the exponent field.  Returns false for NaN and for
+// |w| > 464, which would round past the largest finite value 448.
+inline bool e4m3_code(float w, uint8_t *out) {
+    const double a = std::fabs(static_cast<double>(w));
+    if (std::isnan(w) || a > 464.0) return false;
+    int code;
+    if (a < 0.015625) {
+        code = static_cast<int>(std::nearbyint(a * 512.0));
+    } else {
+        int E = 0;
+        const double f = 2.0 * std::frexp(a, &E);   // a = f * 2^(E - 1), f in [1, 2)
+        code = ((E - 1 + 7) << 3) + static_cast<int>(std::nearbyint((f - 1.0) * 8.0));
+    }
+    *out = static_cast<uint8_t>(code | (std::signbit(w) ? 0x80 : 0));
+    return true;
+}
+
+}  // namespace
+
+extern "C" rt_status rt_quantize_e4m3(const float *W, int64_t n, uint8_t *out) {
+    if (n < 0) return RT_ERR_INVALID_ARG;
+    if (n == 0) return RT_OK;
+    if (!W || !out) return RT_ERR_INVALID_ARG;
+    for (int64_t i = 0; i < n; ++i)
+        if (!e4m3_code(W[i], &out[i])) return RT_ERR_VALUE_RANGE;
     return RT_OK;
 }

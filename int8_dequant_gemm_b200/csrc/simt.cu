@@ -1,5 +1,6 @@
 // fp32 CUDA-core kernels: the exact-rounding path (weights dequantized to
-// fp32 with one rounding, fp32 FMA accumulation) and the path for M <= 8.
+// fp32 with one rounding -- exactly, for q8 codes and e4m3 values -- fp32 FMA
+// accumulation) and the path for M <= 8.
 //
 // Layout of work: each thread owns one output row o of W and MT activation
 // rows, staged per CTA in shared memory.  Inside the K loop every lane of a
@@ -79,15 +80,26 @@ __device__ __forceinline__ void simt_slice(const float *xs, const void *__restri
         }
     } else {
         // q8: the row scale is factored out of the K sum and applied once at
-        // the end, Y = scale[o] * sum_k x * q.
+        // the end, Y = scale[o] * sum_k x * q.  e4m3: the same loop over one
+        // byte per weight, values exact in fp32, no scale.
         const int8_t *wrow = static_cast<const int8_t *>(Wq) + static_cast<size_t>(o) * K + k0;
         for (int kk = 0; kk < Ks; kk += 16) {
             const uint4 p = ldg_v4(wrow + kk);
             const uint32_t words[4] = {p.x, p.y, p.z, p.w};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                const float w0 = q8_byte_f32(words[c], 0), w1 = q8_byte_f32(words[c], 1);
-                const float w2 = q8_byte_f32(words[c], 2), w3 = q8_byte_f32(words[c], 3);
+                float w0, w1, w2, w3;
+                if (FMT == kFmtE4M3) {
+                    w0 = e4m3_byte_f32(words[c], 0);
+                    w1 = e4m3_byte_f32(words[c], 1);
+                    w2 = e4m3_byte_f32(words[c], 2);
+                    w3 = e4m3_byte_f32(words[c], 3);
+                } else {
+                    w0 = q8_byte_f32(words[c], 0);
+                    w1 = q8_byte_f32(words[c], 1);
+                    w2 = q8_byte_f32(words[c], 2);
+                    w3 = q8_byte_f32(words[c], 3);
+                }
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
                     const float4 a = *reinterpret_cast<const float4 *>(xs + m * Ks + kk + c * 4);
@@ -173,22 +185,21 @@ int pick_simt_ksplit(int M, int N, int K, int MT) {
     return ks;
 }
 
-template <int MT>
-cudaError_t launch_simt_mt(bool q4, const float *X, const void *Wq, const void *S, float *Y,
-                           int M, int N, int K, cudaStream_t s) {
+template <int MT, int FMT>
+cudaError_t launch_simt_mt(const float *X, const void *Wq, const void *S, float *Y, int M, int N,
+                           int K, cudaStream_t s) {
     const int ksplit = pick_simt_ksplit(M, N, K, MT);
     const size_t smem = static_cast<size_t>(MT) * (K / ksplit) * sizeof(float) +
                         (ksplit > 1 ? static_cast<size_t>(MT) * kSimtThreads * sizeof(float) : 0);
     // The limit is raised once per device to the largest size any call asks
     // for (staged activations of at most 128 KB plus the partials), so calls
     // from several host threads never lower it under one another.
-    static std::atomic<bool> attr_done[2][kMaxDevices];
+    static std::atomic<bool> attr_done[kMaxDevices];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    e = q4 ? smem_attr_once(simt_kernel<MT, 4>, kSimtMaxSmem, dev, attr_done[0])
-           : smem_attr_once(simt_kernel<MT, 8>, kSimtMaxSmem, dev, attr_done[1]);
-    if (e != cudaSuccess) return e;
+    if ((e = smem_attr_once(simt_kernel<MT, FMT>, kSimtMaxSmem, dev, attr_done)) != cudaSuccess)
+        return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((M + MT - 1) / MT, (N + kSimtThreads - 1) / kSimtThreads, ksplit);
     cfg.blockDim = dim3(kSimtThreads, 1, 1);
@@ -203,23 +214,34 @@ cudaError_t launch_simt_mt(bool q4, const float *X, const void *Wq, const void *
     attr[1].val.clusterDim.z = static_cast<unsigned>(ksplit);
     cfg.attrs = attr;
     cfg.numAttrs = ksplit > 1 ? 2 : 1;
-    if (q4) return cudaLaunchKernelEx(&cfg, simt_kernel<MT, 4>, X, Wq, S, Y, M, N, K, ksplit);
-    return cudaLaunchKernelEx(&cfg, simt_kernel<MT, 8>, X, Wq, S, Y, M, N, K, ksplit);
+    return cudaLaunchKernelEx(&cfg, simt_kernel<MT, FMT>, X, Wq, S, Y, M, N, K, ksplit);
 }
+
+template <int MT>
+cudaError_t launch_simt_fmt(int fmt, const float *X, const void *Wq, const void *S, float *Y,
+                            int M, int N, int K, cudaStream_t s) {
+    if (fmt == kFmtQ4) return launch_simt_mt<MT, kFmtQ4>(X, Wq, S, Y, M, N, K, s);
+    if (fmt == kFmtQ8) return launch_simt_mt<MT, kFmtQ8>(X, Wq, S, Y, M, N, K, s);
+    return launch_simt_mt<MT, kFmtE4M3>(X, Wq, S, Y, M, N, K, s);
+}
+
+}  // namespace
 
 // Activation rows per block: as many as M needs up to 8, capped so the staged
 // activations stay within 128 KB of shared memory.
-cudaError_t launch_simt(bool q4, const float *X, const void *Wq, const void *S, float *Y, int M,
+cudaError_t launch_simt(int fmt, const float *X, const void *Wq, const void *S, float *Y, int M,
                         int N, int K, cudaStream_t s) {
     int mt = M >= 8 ? 8 : (M >= 4 ? 4 : (M >= 2 ? 2 : 1));
     while (mt > 1 && static_cast<size_t>(mt) * K * sizeof(float) > 128 * 1024) mt /= 2;
     switch (mt) {
-        case 8: return launch_simt_mt<8>(q4, X, Wq, S, Y, M, N, K, s);
-        case 4: return launch_simt_mt<4>(q4, X, Wq, S, Y, M, N, K, s);
-        case 2: return launch_simt_mt<2>(q4, X, Wq, S, Y, M, N, K, s);
-        default: return launch_simt_mt<1>(q4, X, Wq, S, Y, M, N, K, s);
+        case 8: return launch_simt_fmt<8>(fmt, X, Wq, S, Y, M, N, K, s);
+        case 4: return launch_simt_fmt<4>(fmt, X, Wq, S, Y, M, N, K, s);
+        case 2: return launch_simt_fmt<2>(fmt, X, Wq, S, Y, M, N, K, s);
+        default: return launch_simt_fmt<1>(fmt, X, Wq, S, Y, M, N, K, s);
     }
 }
+
+namespace {
 
 // ----------------------------------------------------------- dequant exports
 __global__ void dequant_q4_f32_kernel(const uint8_t *__restrict__ Wq,
@@ -277,21 +299,35 @@ __global__ void dequant_q8_f32_kernel(const int8_t *__restrict__ Wq, const float
     }
 }
 
+// e4m3 codes -> fp32 (f16 = false) or fp16 bits (f16 = true, the tensor-core
+// operand), natural order, 16 codes per thread.
+__global__ void dequant_e4m3_kernel(const uint8_t *__restrict__ Wq, void *__restrict__ W, int N,
+                                    int K, bool f16) {
+    const int C = K / 16;
+    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= static_cast<int64_t>(N) * C) return;
+    const int64_t o = idx / C, c = idx % C;
+    const uint4 p = ldg_nc_v4(Wq + o * K + c * 16);
+    const uint32_t words[4] = {p.x, p.y, p.z, p.w};
+    if (f16) {
+        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(W) + o * K + c * 16);
+        dst[0] = chunk_to_natural(e4m3_words_f16(words[0], words[1]));
+        dst[1] = chunk_to_natural(e4m3_words_f16(words[2], words[3]));
+    } else {
+        float *dst = static_cast<float *>(W) + o * K + c * 16;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            reinterpret_cast<float4 *>(dst)[j] =
+                make_float4(e4m3_byte_f32(words[j], 0), e4m3_byte_f32(words[j], 1),
+                            e4m3_byte_f32(words[j], 2), e4m3_byte_f32(words[j], 3));
+    }
+}
+
 inline unsigned blocks_for(int64_t n, int threads) {
     return static_cast<unsigned>((n + threads - 1) / threads);
 }
 
 }  // namespace
-
-cudaError_t launch_simt_q4(const float *X, const uint8_t *Wq, const uint16_t *SM, float *Y,
-                           int M, int N, int K, cudaStream_t s) {
-    return launch_simt(true, X, Wq, SM, Y, M, N, K, s);
-}
-
-cudaError_t launch_simt_q8(const float *X, const int8_t *Wq, const float *S, float *Y, int M,
-                           int N, int K, cudaStream_t s) {
-    return launch_simt(false, X, Wq, S, Y, M, N, K, s);
-}
 
 cudaError_t launch_dequant_q4_f32(const uint8_t *Wq, const uint16_t *SM, float *W, int N, int K,
                                   cudaStream_t s) {
@@ -313,6 +349,13 @@ cudaError_t launch_dequant_q8_f32(const int8_t *Wq, const float *S, float *W, in
                                   cudaStream_t s) {
     const int64_t n = static_cast<int64_t>(N) * (K / 16);
     dequant_q8_f32_kernel<<<blocks_for(n, 256), 256, 0, s>>>(Wq, S, W, N, K);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dequant_e4m3(const uint8_t *Wq, void *W, int N, int K, bool f16,
+                                cudaStream_t s) {
+    const int64_t n = static_cast<int64_t>(N) * (K / 16);
+    dequant_e4m3_kernel<<<blocks_for(n, 256), 256, 0, s>>>(Wq, W, N, K, f16);
     return cudaGetLastError();
 }
 

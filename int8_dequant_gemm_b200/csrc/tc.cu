@@ -191,11 +191,16 @@ __device__ __forceinline__ void store_stage(const StageRegs<PIECES> &R, const Co
         sts_v4(sA + c.a_off[1], q4_word_f16(R.a0.y, s2, m2));
         sts_v4(sA + c.a_off[2], q4_word_f16(R.a0.z, s2, m2));
         sts_v4(sA + c.a_off[3], q4_word_f16(R.a0.w, s2, m2));
-    } else {
+    } else if (FMT == 8) {
         sts_v4(sA + c.a_off[0], q8_words_f16(R.a0.x, R.a0.y));
         sts_v4(sA + c.a_off[1], q8_words_f16(R.a0.z, R.a0.w));
         sts_v4(sA + c.a_off[2], q8_words_f16(R.a1.x, R.a1.y));
         sts_v4(sA + c.a_off[3], q8_words_f16(R.a1.z, R.a1.w));
+    } else {   // e4m3: one byte per weight like q8, no scale
+        sts_v4(sA + c.a_off[0], e4m3_words_f16(R.a0.x, R.a0.y));
+        sts_v4(sA + c.a_off[1], e4m3_words_f16(R.a0.z, R.a0.w));
+        sts_v4(sA + c.a_off[2], e4m3_words_f16(R.a1.x, R.a1.y));
+        sts_v4(sA + c.a_off[3], e4m3_words_f16(R.a1.z, R.a1.w));
     }
 #pragma unroll
     for (int i = 0; i < PIECES; ++i)
@@ -503,12 +508,15 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     const int tile = (bx - p.cl0) * (csize / p.ks) + r / p.ks;
     const int o0 = tile * kTileO;
     const int kslice = r % p.ks, kbase = r - kslice;
-    if (p.fmt == 4)
-        tc_tile<4, PIECES>(smem_raw, p.X, p.Wq, p.S, p.Y, M, p.N, p.K, BN, stages, p.ks, o0, 0,
-                           kslice, kbase, ctl);
+    if (p.fmt == kFmtQ4)
+        tc_tile<kFmtQ4, PIECES>(smem_raw, p.X, p.Wq, p.S, p.Y, M, p.N, p.K, BN, stages, p.ks, o0,
+                                0, kslice, kbase, ctl);
+    else if (p.fmt == kFmtQ8)
+        tc_tile<kFmtQ8, PIECES>(smem_raw, p.X, p.Wq, p.S, p.Y, M, p.N, p.K, BN, stages, p.ks, o0,
+                                0, kslice, kbase, ctl);
     else
-        tc_tile<8, PIECES>(smem_raw, p.X, p.Wq, p.S, p.Y, M, p.N, p.K, BN, stages, p.ks, o0, 0,
-                           kslice, kbase, ctl);
+        tc_tile<kFmtE4M3, PIECES>(smem_raw, p.X, p.Wq, p.S, p.Y, M, p.N, p.K, BN, stages, p.ks,
+                                  o0, 0, kslice, kbase, ctl);
 }
 
 // Activation rows per tile: one tile when M <= 128; otherwise 128, halved
@@ -568,8 +576,8 @@ cudaError_t launch_tc_pieces(const float *X, const void *Wq, const void *S, floa
 }
 
 template <int FMT>
-cudaError_t launch_tc(const float *X, const void *Wq, const void *S, float *Y, int M, int N,
-                      int K, DevCtl *ctl, cudaStream_t st) {
+cudaError_t launch_tc_fmt(const float *X, const void *Wq, const void *S, float *Y, int M, int N,
+                          int K, DevCtl *ctl, cudaStream_t st) {
     const int BN = pick_bn(M, N);
     if (BN <= 32) return launch_tc_pieces<FMT, 2>(X, Wq, S, Y, M, N, K, BN, ctl, st);
     if (BN <= 64) return launch_tc_pieces<FMT, 4>(X, Wq, S, Y, M, N, K, BN, ctl, st);
@@ -658,21 +666,18 @@ cudaError_t launch_tc_group(const GroupProblem *probs, int count, int M, DevCtl 
     g.count = count;
     for (int i = 0; i < count; ++i) {
         const GroupProblem &q = probs[i];
-        if ((q.fmt != 4 && q.fmt != 8) || q.N < 1 || q.K < kTileK || q.K % kTileK != 0)
+        if (!fmt_valid(q.fmt) || q.N < 1 || q.K < kTileK || q.K % kTileK != 0)
             return cudaErrorInvalidValue;
         g.p[i] = {q.X, q.Wq, q.S, q.Y, q.N, q.K, q.fmt, 0, 1};
     }
     return launch_group(g, M, ctl, s);
 }
 
-cudaError_t launch_tc_q4(const float *X, const uint8_t *Wq, const uint16_t *SM, float *Y, int M,
-                         int N, int K, DevCtl *ctl, cudaStream_t s) {
-    return launch_tc<4>(X, Wq, SM, Y, M, N, K, ctl, s);
-}
-
-cudaError_t launch_tc_q8(const float *X, const int8_t *Wq, const float *S, float *Y, int M, int N,
-                         int K, DevCtl *ctl, cudaStream_t s) {
-    return launch_tc<8>(X, Wq, S, Y, M, N, K, ctl, s);
+cudaError_t launch_tc(int fmt, const float *X, const void *Wq, const void *S, float *Y, int M,
+                      int N, int K, DevCtl *ctl, cudaStream_t s) {
+    if (fmt == kFmtQ4) return launch_tc_fmt<kFmtQ4>(X, Wq, S, Y, M, N, K, ctl, s);
+    if (fmt == kFmtQ8) return launch_tc_fmt<kFmtQ8>(X, Wq, S, Y, M, N, K, ctl, s);
+    return launch_tc_fmt<kFmtE4M3>(X, Wq, S, Y, M, N, K, ctl, s);
 }
 
 }  // namespace rtq

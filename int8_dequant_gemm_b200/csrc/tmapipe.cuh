@@ -128,11 +128,16 @@ __device__ __forceinline__ void half_words(const HalfRaw &R, uint32_t (&w)[16]) 
         ch[1] = q4_word_f16(R.p0.y, s2, m2);
         ch[2] = q4_word_f16(R.p0.z, s2, m2);
         ch[3] = q4_word_f16(R.p0.w, s2, m2);
-    } else {
+    } else if (FMT == 8) {
         ch[0] = q8_words_f16(R.p0.x, R.p0.y);
         ch[1] = q8_words_f16(R.p0.z, R.p0.w);
         ch[2] = q8_words_f16(R.p1.x, R.p1.y);
         ch[3] = q8_words_f16(R.p1.z, R.p1.w);
+    } else {   // e4m3: the q8 byte layout, another conversion
+        ch[0] = e4m3_words_f16(R.p0.x, R.p0.y);
+        ch[1] = e4m3_words_f16(R.p0.z, R.p0.w);
+        ch[2] = e4m3_words_f16(R.p1.x, R.p1.y);
+        ch[3] = e4m3_words_f16(R.p1.z, R.p1.w);
     }
 #pragma unroll
     for (int c = 0; c < 4; ++c) {

@@ -402,8 +402,8 @@ __global__ void __launch_bounds__(kWsThreads, 1)
 }
 
 template <int FMT>
-cudaError_t launch_ws(const void *Xh, const void *Wq, const void *S, float *Y, int M, int N,
-                      int K, DevCtl *ctl, cudaStream_t st) {
+cudaError_t launch_ws_fmt(const void *Xh, const void *Wq, const void *S, float *Y, int M, int N,
+                          int K, DevCtl *ctl, cudaStream_t st) {
     static std::atomic<bool> attr_done[kMaxDevices];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -455,14 +455,11 @@ bool ws_supported(int fmt, int M, int N, int K) {
     return fmt == 4 ? K % 128 == 0 : K % 64 == 0;
 }
 
-cudaError_t launch_ws_q4(const void *Xh, const uint8_t *Wq, const uint16_t *SM, float *Y, int M,
-                         int N, int K, DevCtl *ctl, cudaStream_t s) {
-    return launch_ws<4>(Xh, Wq, SM, Y, M, N, K, ctl, s);
-}
-
-cudaError_t launch_ws_q8(const void *Xh, const int8_t *Wq, const float *S, float *Y, int M, int N,
-                         int K, DevCtl *ctl, cudaStream_t s) {
-    return launch_ws<8>(Xh, Wq, S, Y, M, N, K, ctl, s);
+cudaError_t launch_ws(int fmt, const void *Xh, const void *Wq, const void *S, float *Y, int M,
+                      int N, int K, DevCtl *ctl, cudaStream_t s) {
+    if (fmt == kFmtQ4) return launch_ws_fmt<kFmtQ4>(Xh, Wq, S, Y, M, N, K, ctl, s);
+    if (fmt == kFmtQ8) return launch_ws_fmt<kFmtQ8>(Xh, Wq, S, Y, M, N, K, ctl, s);
+    return launch_ws_fmt<kFmtE4M3>(Xh, Wq, S, Y, M, N, K, ctl, s);
 }
 
 }  // namespace rtq

@@ -469,8 +469,8 @@ __global__ void __launch_bounds__(kXsThreads, 1)
 }
 
 template <int FMT>
-cudaError_t launch_xs(const void *Xh, const void *Wq, const void *S, float *Y, int M, int N,
-                      int K, DevCtl *ctl, cudaStream_t st) {
+cudaError_t launch_xs_fmt(const void *Xh, const void *Wq, const void *S, float *Y, int M, int N,
+                          int K, DevCtl *ctl, cudaStream_t st) {
     static std::atomic<bool> attr_done[kMaxDevices];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -522,14 +522,11 @@ bool xs_supported(int M, int N, int K) {
     return K % 128 == 0 && K <= kXsMaxK && M > kTileRows;
 }
 
-cudaError_t launch_xs_q4(const void *Xh, const uint8_t *Wq, const uint16_t *SM, float *Y, int M,
-                         int N, int K, DevCtl *ctl, cudaStream_t s) {
-    return launch_xs<4>(Xh, Wq, SM, Y, M, N, K, ctl, s);
-}
-
-cudaError_t launch_xs_q8(const void *Xh, const int8_t *Wq, const float *S, float *Y, int M, int N,
-                         int K, DevCtl *ctl, cudaStream_t s) {
-    return launch_xs<8>(Xh, Wq, S, Y, M, N, K, ctl, s);
+cudaError_t launch_xs(int fmt, const void *Xh, const void *Wq, const void *S, float *Y, int M,
+                      int N, int K, DevCtl *ctl, cudaStream_t s) {
+    if (fmt == kFmtQ4) return launch_xs_fmt<kFmtQ4>(Xh, Wq, S, Y, M, N, K, ctl, s);
+    if (fmt == kFmtQ8) return launch_xs_fmt<kFmtQ8>(Xh, Wq, S, Y, M, N, K, ctl, s);
+    return launch_xs_fmt<kFmtE4M3>(Xh, Wq, S, Y, M, N, K, ctl, s);
 }
 
 }  // namespace rtq

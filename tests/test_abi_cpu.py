@@ -385,3 +385,46 @@ def test_block_fmt_validation_and_routes():
     Ybad = list(Y); Ybad[1] = Y[0] + 64                    # outputs overlap
     assert run(C.byref(q8), 80, *X, *Ybad, 0, None) == INVALID
     assert run(C.byref(q8), 0, *X, *Y, 0, None) == RT_OK   # M == 0: no-op
+
+
+# --------------------------------------------------------------- FP8 E4M3
+@pytest.mark.parametrize("outliers", [False, True])
+def test_e4m3_quantizer_matches_oracle_bit_for_bit(outliers):
+    W = wl.weights(256, 512, 4242)
+    if outliers:
+        W = wl.with_outliers(W, 4243)
+    assert np.array_equal(rtq.quantize_e4m3(W), oracle.quant_e4m3(W))
+
+
+def test_e4m3_quantizer_edges_match_oracle():
+    finite = np.array([oracle.e4m3_to_double(b) for b in range(0x7F)])
+    mids = (finite[:-1] + finite[1:]) / 2
+    edge = np.array([464.0, 463.99997, 448.0, 2 ** -10, 2 ** -6, 2 ** -6 - 2 ** -12, 0.0, -0.0])
+    W = np.concatenate([finite, -finite, mids, -mids, edge]).astype(np.float32)[None, :]
+    assert np.array_equal(rtq.quantize_e4m3(W), oracle.quant_e4m3(W))
+    for bad in (464.01, -1e6, np.nan, np.inf):
+        with pytest.raises(rtq.RtqError) as e:
+            rtq.quantize_e4m3(np.array([[0.5, bad]], dtype=np.float32))
+        assert e.value.status == RANGE
+    assert rtq.rt_quantize_e4m3(None, 4, None) == INVALID
+    assert rtq.rt_quantize_e4m3(None, 0, None) == RT_OK
+
+
+def test_e4m3_gemm_validation_and_plan():
+    f = rtq.rt_gemm_e4m3
+    assert f(None, W, Y, 4, 16, 64, 0, None) == INVALID           # null X with M > 0
+    assert f(X, None, Y, 4, 16, 64, 0, None) == INVALID           # null weights
+    assert f(X, W + 8, Y, 4, 16, 64, 0, None) == ALIGN            # W not 16-byte aligned
+    assert f(X, W, X, 4, 16, 64, 0, None) == INVALID              # Y overlaps X
+    assert f(X, W, Y, 4, 16, 24, 0, None) == SHAPE                # K % 16
+    assert f(X, W, Y, 4, 16, 96, 2, None) == SHAPE                # forced TC needs K % 64
+    assert f(None, W, None, 0, 16, 64, 0, None) == RT_OK          # M == 0
+    assert rtq.plan(3, 80, 512, 2048) == "tc_w_stationary"
+    assert rtq.plan(3, 4096, 512, 512) == "tc_x_resident"
+    assert rtq.plan(3, 4096, 512, 2048) == "tc_w_streamed"
+    assert rtq.plan(3, 4, 512, 2048) == "simt"
+    assert rtq.auto_path(3, 80, 512, 48) == 1                     # K % 64 != 0 -> SIMT
+    assert rtq.workspace_bytes(3, 4096, 512, 2048) == 4096 * 2048 * 2
+    # a batch entry in e4m3 carries no scales
+    arr = _qproj_array([(3, 0, X, W, 0, Y, 2048, 512)] * 1)
+    assert rtq.lib().rt_qgemm_batch_plan(arr, 1, 80, 2) == 5
