@@ -82,7 +82,10 @@ typedef enum rt_status {
     RT_ERR_WORKSPACE = 7,         /* the workspace would have to grow inside a stream capture */
     RT_ERR_SCRATCH_LIMIT = 8,     /* rt_qgemm_noalloc: M * K * 2 > RT_NOALLOC_SCRATCH_BYTES */
     RT_ERR_OPERAND_RANGE = 9,     /* an activation was not a finite fp16 value (rt_device_status) */
-    RT_ERR_UNSUPPORTED_DEVICE = 10 /* current device index >= 64, the library's per-device limit */
+    RT_ERR_UNSUPPORTED_DEVICE = 10, /* current device index >= 64, the library's per-device limit */
+    RT_ERR_IO = 11,               /* a checkpoint file cannot be opened or mapped */
+    RT_ERR_FORMAT = 12,           /* a checkpoint file or tensor is malformed */
+    RT_ERR_NOT_FOUND = 13         /* a checkpoint has no tensor (or companion) of that name */
 } rt_status;
 
 /* Weight formats, where an entry point takes a `fmt` argument. */
@@ -433,6 +436,50 @@ rt_status rt_device_status(void *stream, int *device_status);
  * Restore rt_debug_inject(0, 0) before normal use.
  */
 rt_status rt_debug_inject(int mode, int64_t wait_ns);
+
+/*
+ * Quantized checkpoints.  Both quantized cards ship plain safetensors files
+ * ("Plain safetensors -- no custom container") that the engine's loader takes
+ * directly, "the format is auto-detected from the tensor dtypes"; the FP8 card
+ * stores float8_e4m3fn weights the same way.  These calls read such a file
+ * on the host (the model cards have no other interface to match):
+ *
+ *   rt_st_open          maps the file read-only and parses its header;
+ *                       RT_ERR_IO if it cannot be opened or mapped,
+ *                       RT_ERR_FORMAT if the header, a dtype, a shape or an
+ *                       offset is malformed.  *out is NULL on error.
+ *   rt_st_count         number of tensors in the file (-1 for NULL).
+ *   rt_st_weight_find   the projection weight `name`, its format detected:
+ *                         U8 [N, K/2] + "<name>.q4_scale" F16 [N, K/32, 2]
+ *                           (or [N, K/16])                      -> RT_FMT_Q4
+ *                         I8 [N, K] + "<name>.q_scale" F32 [N] (or [N, 1])
+ *                                                               -> RT_FMT_Q8
+ *                         F8_E4M3 [N, K]                        -> RT_FMT_E4M3
+ *                       Pointers are HOST pointers into the mapping, valid
+ *                       until rt_st_close, with no alignment guarantee (copy
+ *                       them to device memory for the GEMMs); scales is NULL
+ *                       for e4m3.  RT_ERR_NOT_FOUND if `name` or its
+ *                       companion is missing, RT_ERR_FORMAT for another dtype
+ *                       or inconsistent shapes, RT_ERR_UNSUPPORTED_SHAPE if the
+ *                       weight is not a non-empty 2-D tensor.
+ *   rt_st_close         unmaps the file (NULL is a no-op).
+ * Files are only read; calls on distinct files may run concurrently.
+ */
+typedef struct rt_st_file rt_st_file;
+
+typedef struct rt_st_weight {
+    int32_t fmt;            /* rt_format */
+    int32_t reserved;
+    int64_t N, K;
+    const void *codes;      /* code_bytes bytes */
+    const void *scales;     /* scale_bytes bytes; NULL for e4m3 */
+    int64_t code_bytes, scale_bytes;
+} rt_st_weight;
+
+rt_status rt_st_open(const char *path, rt_st_file **out);
+int64_t rt_st_count(const rt_st_file *f);
+rt_status rt_st_weight_find(const rt_st_file *f, const char *name, rt_st_weight *out);
+void rt_st_close(rt_st_file *f);
 
 #ifdef __cplusplus
 }

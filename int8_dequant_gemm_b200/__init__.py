@@ -24,6 +24,7 @@ __all__ = [
     "qgemm_noalloc", "plan", "block_fused", "workspace_bytes", "debug_inject",
     "qgemm_batch", "batch_plan", "Proj", "QBlockFmt", "qblock_project_fmt", "block_fused_fmt",
     "gemm_e4m3", "quantize_e4m3", "dequant_e4m3_f32", "dequant_e4m3_f16", "FMT_E4M3",
+    "Checkpoint",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -64,6 +65,11 @@ class _QBlockFmtC(ctypes.Structure):
                 ("d_model", _i64), ("d_ff", _i64)]
 
 
+class _StWeightC(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("reserved", ctypes.c_int32), ("N", _i64), ("K", _i64),
+                ("codes", _p), ("scales", _p), ("code_bytes", _i64), ("scale_bytes", _i64)]
+
+
 class _QBlockC(ctypes.Structure):
     _fields_ = [("qkvg", _p), ("qkvg_sm", _p), ("wo", _p), ("wo_s", _p), ("w13", _p),
                 ("w13_sm", _p), ("w2", _p), ("w2_s", _p), ("d_model", _i64), ("d_ff", _i64)]
@@ -93,6 +99,14 @@ def lib() -> ctypes.CDLL:
         f = getattr(L, name)
         f.restype = _i32
         f.argtypes = [_p, _p, _i64, _i64, _p]
+    L.rt_st_open.restype = _i32
+    L.rt_st_open.argtypes = [ctypes.c_char_p, ctypes.POINTER(_p)]
+    L.rt_st_count.restype = _i64
+    L.rt_st_count.argtypes = [_p]
+    L.rt_st_weight_find.restype = _i32
+    L.rt_st_weight_find.argtypes = [_p, ctypes.c_char_p, ctypes.POINTER(_StWeightC)]
+    L.rt_st_close.restype = None
+    L.rt_st_close.argtypes = [_p]
     L.rt_qgemm_noalloc.restype = _i32
     L.rt_qgemm_noalloc.argtypes = [_i32, _p, _p, _p, _p, _i64, _i64, _i64, _i32, _p]
     L.rt_qgemm_auto_path.restype = _i32
@@ -645,3 +659,49 @@ def workspace_reserve(nbytes: int, stream=None):
 
 def workspace_release():
     _check(rt_workspace_release(), "rt_workspace_release")
+
+
+class Checkpoint:
+    """A quantized checkpoint file (plain safetensors) read through rt_st_*:
+    ``weight(name)`` returns (fmt, codes, scales) as host numpy arrays in the
+    layouts the GEMMs take (q4: uint8 [N, K/2] + uint16 [N, K/32, 2]; q8:
+    int8 [N, K] + float32 [N]; e4m3: uint8 [N, K] + None), the format detected
+    from the dtypes."""
+
+    def __init__(self, path):
+        self._h = ctypes.c_void_p()
+        _check(lib().rt_st_open(os.fsencode(path), ctypes.byref(self._h)), "rt_st_open")
+
+    def __len__(self):
+        return int(lib().rt_st_count(self._h))
+
+    def weight(self, name: str):
+        w = _StWeightC()
+        _check(lib().rt_st_weight_find(self._h, name.encode(), ctypes.byref(w)),
+               f"rt_st_weight_find({name})")
+        N, K, fmt = int(w.N), int(w.K), int(w.fmt)
+        codes = np.frombuffer(ctypes.string_at(w.codes, w.code_bytes), dtype=np.uint8)
+        if fmt == FMT_Q4:
+            sc = np.frombuffer(ctypes.string_at(w.scales, w.scale_bytes), dtype=np.uint16)
+            return fmt, codes.reshape(N, K // 2).copy(), sc.reshape(N, K // 32, 2).copy()
+        if fmt == FMT_Q8:
+            sc = np.frombuffer(ctypes.string_at(w.scales, w.scale_bytes), dtype=np.float32)
+            return fmt, codes.view(np.int8).reshape(N, K).copy(), sc.copy()
+        return fmt, codes.reshape(N, K).copy(), None
+
+    def close(self):
+        if self._h:
+            lib().rt_st_close(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

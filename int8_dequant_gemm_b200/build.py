@@ -20,7 +20,7 @@ LIB = os.path.join(HERE, "librtq.so")
 HEADER = os.path.join(ROOT, "include", "rtq.h")
 
 CU_SOURCES = ["api.cu", "simt.cu", "tc.cu", "xs.cu", "ws.cu", "prep.cu", "pl.cu", "noalloc.cu"]
-CPP_SOURCES = ["quantize.cpp"]
+CPP_SOURCES = ["quantize.cpp", "st_loader.cpp"]
 NVCC = os.environ.get("NVCC", "nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2",

@@ -200,6 +200,9 @@ const char *rt_status_string(int status) {
         case RT_ERR_SCRATCH_LIMIT: return "problem needs more than the fixed scratch array holds";
         case RT_ERR_OPERAND_RANGE: return "an activation is not a finite fp16 value";
         case RT_ERR_UNSUPPORTED_DEVICE: return "device index beyond the library's limit";
+        case RT_ERR_IO: return "file cannot be opened or mapped";
+        case RT_ERR_FORMAT: return "malformed checkpoint file or tensor";
+        case RT_ERR_NOT_FOUND: return "no tensor of that name";
         default: return "unknown status";
     }
 }
