@@ -437,7 +437,7 @@ def measure_small_m(args, rank, world, local_rank, dev, stream, blocks=None):
                 N, K = proj_dims(p)[1:]
                 arr[4 * j + k] = rtq._QProjC(4 if proj_dims(p)[0] == "q4" else 8, 0,
                                              xs[p].data_ptr(), db[p][0].data_ptr(),
-                                             db[p][1].data_ptr(), ys[j][p].data_ptr(), N, K)
+                                             db[p][1].data_ptr(), None, ys[j][p].data_ptr(), N, K)
         arrays.append(arr)
     route = rtq.KERNELS.get(L.rt_qgemm_batch_plan(arrays[0], 4 * per_call, M, 0), "per call")
     structs = [rtq._QBlockC(*(t.data_ptr() for p in projs for t in db[p]), wl.D_MODEL, wl.D_FF)

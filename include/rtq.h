@@ -122,6 +122,20 @@ rt_status rt_qgemm_q8(const float *X, const int8_t *Wq, const float *scale, floa
                       int64_t M, int64_t N, int64_t K, int path, void *stream);
 
 /*
+ * Y = X * dequant(Wq, scales)^T + bias, any weight format, with an optional
+ * fp32 bias fused into the epilogue (the cards keep biases in fp32 next to
+ * the quantized weights: int4 card, "Quantization format").
+ *   fmt     rt_format (scales unused for RT_FMT_E4M3 and may be NULL);
+ *   bias    NULL, or fp32 [N] device memory, 4-byte aligned, not overlapping
+ *           Y (RT_ERR_ALIGNMENT / RT_ERR_INVALID_ARG);
+ * each output is fma(sum, row scale, bias[o]) rounded once (row scale 1
+ * for q4 and e4m3).  Everything else as for rt_qgemm_q4 / rt_qgemm_q8 /
+ * rt_gemm_e4m3, which are this call with bias NULL.
+ */
+rt_status rt_qgemm(int fmt, const float *X, const void *Wq, const void *scales, const float *bias,
+                   float *Y, int64_t M, int64_t N, int64_t K, int path, void *stream);
+
+/*
  * Y = X * W^T with W the FP8 E4M3 weights, converted exactly to the operand
  * type inside the GEMM.   (FP8 card, "FP8 Format")
  * X [M,K] fp32, W [N,K] uint8 float8_e4m3fn codes, Y [M,N] fp32.  K % 16 == 0;
@@ -228,10 +242,11 @@ rt_status rt_qgemm_noalloc(int fmt, const float *X, const void *Wq, const void *
  *             8: q8 tensors as for rt_qgemm_q8;
  *             3: Wq are e4m3 codes as for rt_gemm_e4m3 (scales unused).
  *   reserved  must be 0.
+ *   bias      NULL, or an fp32 [N] bias added in the epilogue (rt_qgemm).
  *   X, Y      fp32 [M, K] / [M, N] device buffers of this projection.
  *
  * Validation: every entry as for rt_qgemm_q4/q8 (the same statuses); in
- * addition no entry's Y may overlap any other entry's X, Wq, scales or Y
+ * addition no entry's Y may overlap any other entry's X, Wq, scales, bias or Y
  * (RT_ERR_INVALID_ARG), since the entries may run concurrently; X, Wq and
  * scales may be shared between entries.  All entries are checked before
  * anything is enqueued.  count == 0 or M == 0 is a no-op.
@@ -255,6 +270,7 @@ typedef struct rt_qproj {
     const float *X;
     const void *Wq;
     const void *scales;
+    const float *bias;
     float *Y;
     int64_t N;
     int64_t K;
@@ -324,7 +340,9 @@ int rt_qblock_fused(int64_t M, int64_t d_model, int64_t d_ff, int path);
  *             8: Wq i8 [N, K] and scales fp32 [N] (q8);
  *             3: Wq u8 [N, K] float8_e4m3fn codes, scales unused (the FP8
  *                card's recipe: every block projection in e4m3);
- *   reserved  must be 0.
+ *   reserved  must be 0;
+ *   bias      NULL, or the projection's fp32 [N] bias, added in the
+ *             epilogue as in rt_qgemm.
  * Shapes, outputs, launches, validation and errors are those of
  * rt_qblock_project; rt_qblock_project is this call with the int4 card's
  * mixed recipe (qkvg and w13 q4, wo and w2 q8).
@@ -334,6 +352,7 @@ typedef struct rt_qweight {
     int32_t reserved;
     const void *Wq;
     const void *scales;
+    const float *bias;
 } rt_qweight;
 
 typedef struct rt_qblock_fmt {

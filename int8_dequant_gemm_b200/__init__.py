@@ -24,7 +24,7 @@ __all__ = [
     "qgemm_noalloc", "plan", "block_fused", "workspace_bytes", "debug_inject",
     "qgemm_batch", "batch_plan", "Proj", "QBlockFmt", "qblock_project_fmt", "block_fused_fmt",
     "gemm_e4m3", "quantize_e4m3", "dequant_e4m3_f32", "dequant_e4m3_f16", "FMT_E4M3",
-    "Checkpoint",
+    "Checkpoint", "qgemm",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -53,11 +53,12 @@ class RtqError(RuntimeError):
 
 class _QProjC(ctypes.Structure):
     _fields_ = [("fmt", ctypes.c_int32), ("reserved", ctypes.c_int32), ("X", _p), ("Wq", _p),
-                ("scales", _p), ("Y", _p), ("N", _i64), ("K", _i64)]
+                ("scales", _p), ("bias", _p), ("Y", _p), ("N", _i64), ("K", _i64)]
 
 
 class _QWeightC(ctypes.Structure):
-    _fields_ = [("fmt", ctypes.c_int32), ("reserved", ctypes.c_int32), ("Wq", _p), ("scales", _p)]
+    _fields_ = [("fmt", ctypes.c_int32), ("reserved", ctypes.c_int32), ("Wq", _p), ("scales", _p),
+                ("bias", _p)]
 
 
 class _QBlockFmtC(ctypes.Structure):
@@ -91,6 +92,8 @@ def lib() -> ctypes.CDLL:
         f = getattr(L, name)
         f.restype = _i32
         f.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _i32, _p]
+    L.rt_qgemm.restype = _i32
+    L.rt_qgemm.argtypes = [_i32, _p, _p, _p, _p, _p, _i64, _i64, _i64, _i32, _p]
     L.rt_gemm_e4m3.restype = _i32
     L.rt_gemm_e4m3.argtypes = [_p, _p, _p, _i64, _i64, _i64, _i32, _p]
     L.rt_quantize_e4m3.restype = _i32
@@ -165,6 +168,10 @@ def rt_qgemm_q4(X, Wq, scale_min, Y, M, N, K, path, stream) -> int:
 
 def rt_qgemm_q8(X, Wq, scale, Y, M, N, K, path, stream) -> int:
     return lib().rt_qgemm_q8(X, Wq, scale, Y, M, N, K, path, stream)
+
+
+def rt_qgemm(fmt, X, Wq, scales, bias, Y, M, N, K, path, stream) -> int:
+    return lib().rt_qgemm(fmt, X, Wq, scales, bias, Y, M, N, K, path, stream)
 
 
 def rt_gemm_e4m3(X, W, Y, M, N, K, path, stream) -> int:
@@ -357,6 +364,24 @@ def qgemm_q8(X, Wq, scale, Y=None, path="auto", stream=None):
     return Y
 
 
+def qgemm(fmt, X, Wq, scales=None, bias=None, Y=None, path="auto", stream=None):
+    """Y[M,N] = X[M,K] @ dequant(Wq, scales)^T + bias on the GPU, any format
+    (4: q4, 8: q8, 3: e4m3 with scales None); bias: None or fp32 [N]."""
+    import torch
+    M, N, K = _check_gemm_shapes(fmt, X, Wq, scales, Y)
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float32, device=X.device)
+    b = None
+    if bias is not None:
+        _shape(bias, (N,), "bias")
+        b = _dev(bias, torch.float32, "bias")
+    w, sc = _weight_ptrs(fmt, Wq, scales, "Wq")
+    st = rt_qgemm(fmt, _dev(X, torch.float32, "X"), w, sc, b, _dev(Y, torch.float32, "Y"),
+                  M, N, K, _path(path), _stream_ptr(stream))
+    _check(st, "rt_qgemm")
+    return Y
+
+
 def gemm_e4m3(X, W, Y=None, path="auto", stream=None):
     """Y[M,N] = X[M,K] @ e4m3(W[N,K])^T on the GPU (W: uint8 float8_e4m3fn codes)."""
     import torch
@@ -386,13 +411,15 @@ def qgemm_noalloc(fmt, X, Wq, scales, Y, path="auto", stream=None):
 
 @dataclass
 class Proj:
-    """One entry of a projection list (see rt_qproj in rtq.h): fmt 4 or 8, the
-    device tensors X [M, K], Wq and scales in that format, Y [M, N]."""
+    """One entry of a projection list (see rt_qproj in rtq.h): fmt 4, 8 or 3,
+    the device tensors X [M, K], Wq and scales in that format, Y [M, N], and
+    an optional fp32 bias [N]."""
     fmt: int
     X: object
     Wq: object
     scales: object
     Y: object
+    bias: object = None
 
 
 def _batch_array(projs, M):
@@ -405,7 +432,11 @@ def _batch_array(projs, M):
             raise ValueError(f"entry {i}: X must be [M={M}, K], got {tuple(q.X.shape)}")
         _, N, K = _check_gemm_shapes(q.fmt, q.X, q.Wq, q.scales, q.Y)
         w, sc = _weight_ptrs(q.fmt, q.Wq, q.scales, f"entry {i} Wq")
-        arr[i] = _QProjC(q.fmt, 0, _dev(q.X, torch.float32, "X"), w, sc,
+        b = None
+        if q.bias is not None:
+            _shape(q.bias, (N,), f"entry {i} bias")
+            b = _dev(q.bias, torch.float32, "bias")
+        arr[i] = _QProjC(q.fmt, 0, _dev(q.X, torch.float32, "X"), w, sc, b,
                          _dev(q.Y, torch.float32, "Y"), N, K)
     return arr
 
@@ -480,9 +511,10 @@ def qblock_project(block: QBlock, X_qkvg, X_o, X_ffn, X_w2, Y_qkvg, Y_o, Y_13, Y
 
 @dataclass
 class QBlockFmt:
-    """A block's four projections, each (fmt, Wq, scales) with fmt 4 (q4) or
-    8 (q8), as device tensors (see rt_qblock_fmt in rtq.h).  All four q8 is
-    the int8 card's all-int8 recipe."""
+    """A block's four projections, each (fmt, Wq, scales) or (fmt, Wq, scales,
+    bias) with fmt 4 (q4), 8 (q8) or 3 (e4m3, scales None), as device tensors
+    (see rt_qblock_fmt in rtq.h).  All four q8 is the int8 card's all-int8
+    recipe."""
     qkvg: tuple
     wo: tuple
     w13: tuple
@@ -495,14 +527,19 @@ class QBlockFmt:
         d, f = self.d_model, self.d_ff
         ws = []
         for name, N, K in (("qkvg", 4 * d, d), ("wo", d, d), ("w13", 2 * f, d), ("w2", d, f)):
-            fmt, Wq, S = getattr(self, name)
+            fmt, Wq, S, *rest = getattr(self, name)
+            bias = rest[0] if rest else None
             if fmt not in _DTYPES:
                 raise ValueError(f"{name}: fmt must be 4, 8 or 3 (e4m3), got {fmt}")
             wshape, sshape = _packed_shapes(fmt, N, K)
             _shape(Wq, wshape, name)
             if sshape is not None:
                 _shape(S, sshape, name + " scales")
-            ws.append(_QWeightC(fmt, 0, *_weight_ptrs(fmt, Wq, S, name)))
+            b = None
+            if bias is not None:
+                _shape(bias, (N,), name + " bias")
+                b = _dev(bias, torch.float32, name + " bias")
+            ws.append(_QWeightC(fmt, 0, *_weight_ptrs(fmt, Wq, S, name), b))
         return _QBlockFmtC(*ws, d, f)
 
 

@@ -119,6 +119,14 @@ rt_status validate(const float *X, const void *Wq, const void *S, const float *Y
     return RT_OK;
 }
 
+// The optional fp32 bias of a GEMM: 4-byte aligned, not overlapping Y.
+rt_status check_bias(const float *bias, const float *Y, int64_t M, int64_t N) {
+    if (!bias) return RT_OK;
+    if (!aligned(bias, 4)) return RT_ERR_ALIGNMENT;
+    if (M > 0 && overlap(Y, M * N * 4, bias, N * 4)) return RT_ERR_INVALID_ARG;
+    return RT_OK;
+}
+
 // Bytes of the packed codes and of the scales of an N x K weight.
 int64_t code_bytes(int fmt, int64_t N, int64_t K) { return fmt == 4 ? N * (K / 2) : N * K; }
 int64_t scale_bytes(int fmt, int64_t N, int64_t K) {
@@ -144,7 +152,8 @@ int pick_path(int64_t M, int64_t K, int path) {
 inline rt_status from_cuda(cudaError_t e) { return e == cudaSuccess ? RT_OK : RT_ERR_CUDA; }
 
 // Runs a validated GEMM on the kernel the plan picks.
-rt_status run_gemm(int fmt, const float *X, const void *Wq, const void *S, float *Y, int64_t M,
+rt_status run_gemm(int fmt, const float *X, const void *Wq, const void *S, const float *bias,
+                   float *Y, int64_t M,
                    int64_t N, int64_t K, int path, void *stream) {
     const int p = pick_path(M, K, path);
     if (p == -1) return RT_ERR_UNSUPPORTED_SHAPE;
@@ -153,19 +162,19 @@ rt_status run_gemm(int fmt, const float *X, const void *Wq, const void *S, float
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
     const int kern = pick_kernel(fmt, M, N, K, p);
-    if (kern == RT_KERNEL_SIMT) return from_cuda(rtq::launch_simt(fmt, X, Wq, S, Y, m, n, k, s));
+    if (kern == RT_KERNEL_SIMT) return from_cuda(rtq::launch_simt(fmt, X, Wq, S, bias, Y, m, n, k, s));
     DevCtl *ctl = nullptr;
     rt_status st = ctl_block(&ctl);
     if (st != RT_OK) return st;
     if (kern == RT_KERNEL_TC_W_STATIONARY)
-        return from_cuda(rtq::launch_tc(fmt, X, Wq, S, Y, m, n, k, ctl, s));
+        return from_cuda(rtq::launch_tc(fmt, X, Wq, S, bias, Y, m, n, k, ctl, s));
     void *xh = nullptr;
     if ((st = workspace(s, static_cast<size_t>(M) * K * 2, &xh)) != RT_OK) return st;
     cudaError_t e = rtq::launch_cvt_x16(X, xh, M, K, ctl, s);
     if (e != cudaSuccess) return RT_ERR_CUDA;
     if (kern == RT_KERNEL_TC_X_RESIDENT)
-        return from_cuda(rtq::launch_xs(fmt, xh, Wq, S, Y, m, n, k, ctl, s));
-    return from_cuda(rtq::launch_ws(fmt, xh, Wq, S, Y, m, n, k, ctl, s));
+        return from_cuda(rtq::launch_xs(fmt, xh, Wq, S, bias, Y, m, n, k, ctl, s));
+    return from_cuda(rtq::launch_ws(fmt, xh, Wq, S, bias, Y, m, n, k, ctl, s));
 }
 
 }  // namespace
@@ -229,21 +238,29 @@ rt_status rt_qgemm_q4(const float *X, const uint8_t *Wq, const uint16_t *scale_m
                       int64_t M, int64_t N, int64_t K, int path, void *stream) {
     rt_status st = validate(X, Wq, scale_min, Y, M, N, K, N * (K / 2), N * (K / 32) * 4, 4, 32);
     if (st != RT_OK) return st;
-    return run_gemm(4, X, Wq, scale_min, Y, M, N, K, path, stream);
+    return run_gemm(4, X, Wq, scale_min, nullptr, Y, M, N, K, path, stream);
 }
 
 rt_status rt_qgemm_q8(const float *X, const int8_t *Wq, const float *scale, float *Y, int64_t M,
                       int64_t N, int64_t K, int path, void *stream) {
     rt_status st = validate(X, Wq, scale, Y, M, N, K, N * K, N * 4, 4, 16);
     if (st != RT_OK) return st;
-    return run_gemm(8, X, Wq, scale, Y, M, N, K, path, stream);
+    return run_gemm(8, X, Wq, scale, nullptr, Y, M, N, K, path, stream);
+}
+
+rt_status rt_qgemm(int fmt, const float *X, const void *Wq, const void *scales, const float *bias,
+                   float *Y, int64_t M, int64_t N, int64_t K, int path, void *stream) {
+    rt_status st = rtq::check_gemm_args(fmt, X, Wq, scales, Y, M, N, K);
+    if (st == RT_OK) st = check_bias(bias, Y, M, N);
+    if (st != RT_OK) return st;
+    return run_gemm(fmt, X, Wq, scales, bias, Y, M, N, K, path, stream);
 }
 
 rt_status rt_gemm_e4m3(const float *X, const uint8_t *W, float *Y, int64_t M, int64_t N,
                        int64_t K, int path, void *stream) {
     rt_status st = rtq::check_gemm_args(rtq::kFmtE4M3, X, W, nullptr, Y, M, N, K);
     if (st != RT_OK) return st;
-    return run_gemm(rtq::kFmtE4M3, X, W, nullptr, Y, M, N, K, path, stream);
+    return run_gemm(rtq::kFmtE4M3, X, W, nullptr, nullptr, Y, M, N, K, path, stream);
 }
 
 int64_t rt_workspace_bytes(int fmt, int64_t M, int64_t N, int64_t K, int path) {
@@ -284,6 +301,7 @@ struct BlockProj {
     int fmt;
     const float *X;
     const void *W, *S;
+    const float *bias;
     float *Y;
     int64_t N, K;
 };
@@ -312,7 +330,8 @@ rt_status block_run(const BlockProj p[4], int64_t M, int64_t d, int64_t f, int p
         const BlockProj &q = p[i];
         if (!rtq::fmt_valid(q.fmt)) return RT_ERR_INVALID_ARG;
         fmts[i] = q.fmt;
-        if ((st = rtq::check_gemm_args(q.fmt, q.X, q.W, q.S, q.Y, M, q.N, q.K)) != RT_OK)
+        if ((st = rtq::check_gemm_args(q.fmt, q.X, q.W, q.S, q.Y, M, q.N, q.K)) != RT_OK ||
+            (st = check_bias(q.bias, q.Y, M, q.N)) != RT_OK)
             return st;
         const int pp = pick_path(M, q.K, path);
         if (pp == -1) return RT_ERR_UNSUPPORTED_SHAPE;
@@ -329,7 +348,8 @@ rt_status block_run(const BlockProj p[4], int64_t M, int64_t d, int64_t f, int p
                 const int64_t sb = scale_bytes(p[j].fmt, p[j].N, p[j].K);
                 if (overlap(p[i].Y, yb, p[j].Y, M * p[j].N * 4) ||
                     overlap(p[i].Y, yb, p[j].X, M * p[j].K * 4) || overlap(p[i].Y, yb, p[j].W, wb) ||
-                    (sb > 0 && overlap(p[i].Y, yb, p[j].S, sb)))
+                    (sb > 0 && overlap(p[i].Y, yb, p[j].S, sb)) ||
+                    (p[j].bias && overlap(p[i].Y, yb, p[j].bias, p[j].N * 4)))
                     return RT_ERR_INVALID_ARG;
             }
         }
@@ -339,14 +359,14 @@ rt_status block_run(const BlockProj p[4], int64_t M, int64_t d, int64_t f, int p
         if ((st = ctl_block(&ctl)) != RT_OK) return st;
         rtq::GroupProblem g[4];
         for (int i = 0; i < 4; ++i)
-            g[i] = {p[i].X, p[i].W, p[i].S, p[i].Y, static_cast<int>(p[i].N),
+            g[i] = {p[i].X, p[i].W, p[i].S, p[i].bias, p[i].Y, static_cast<int>(p[i].N),
                     static_cast<int>(p[i].K), p[i].fmt};
         return from_cuda(rtq::launch_tc_group(g, 4, static_cast<int>(M), ctl,
                                               static_cast<cudaStream_t>(stream)));
     }
     for (int i = 0; i < 4; ++i) {
         const BlockProj &q = p[i];
-        if ((st = run_gemm(q.fmt, q.X, q.W, q.S, q.Y, M, q.N, q.K, path, stream)) != RT_OK)
+        if ((st = run_gemm(q.fmt, q.X, q.W, q.S, q.bias, q.Y, M, q.N, q.K, path, stream)) != RT_OK)
             return st;
     }
     return RT_OK;
@@ -369,10 +389,10 @@ rt_status rt_qblock_project(const rt_qblock *blk, int64_t M, const float *X_qkvg
                             void *stream) {
     if (!blk || blk->d_model < 1 || blk->d_ff < 1) return RT_ERR_INVALID_ARG;
     const int64_t d = blk->d_model, f = blk->d_ff;
-    const BlockProj p[4] = {{4, X_qkvg, blk->qkvg, blk->qkvg_sm, Y_qkvg, 4 * d, d},
-                            {8, X_o, blk->wo, blk->wo_s, Y_o, d, d},
-                            {4, X_ffn, blk->w13, blk->w13_sm, Y_13, 2 * f, d},
-                            {8, X_w2, blk->w2, blk->w2_s, Y_2, d, f}};
+    const BlockProj p[4] = {{4, X_qkvg, blk->qkvg, blk->qkvg_sm, nullptr, Y_qkvg, 4 * d, d},
+                            {8, X_o, blk->wo, blk->wo_s, nullptr, Y_o, d, d},
+                            {4, X_ffn, blk->w13, blk->w13_sm, nullptr, Y_13, 2 * f, d},
+                            {8, X_w2, blk->w2, blk->w2_s, nullptr, Y_2, d, f}};
     return block_run(p, M, d, f, path, stream);
 }
 
@@ -396,10 +416,11 @@ rt_status rt_qblock_project_fmt(const rt_qblock_fmt *blk, int64_t M, const float
     for (int i = 0; i < 4; ++i)
         if (w[i]->reserved != 0) return RT_ERR_INVALID_ARG;
     const int64_t d = blk->d_model, f = blk->d_ff;
-    const BlockProj p[4] = {{blk->qkvg.fmt, X_qkvg, blk->qkvg.Wq, blk->qkvg.scales, Y_qkvg, 4 * d, d},
-                            {blk->wo.fmt, X_o, blk->wo.Wq, blk->wo.scales, Y_o, d, d},
-                            {blk->w13.fmt, X_ffn, blk->w13.Wq, blk->w13.scales, Y_13, 2 * f, d},
-                            {blk->w2.fmt, X_w2, blk->w2.Wq, blk->w2.scales, Y_2, d, f}};
+    const rt_qweight &a = blk->qkvg, &b = blk->wo, &c = blk->w13, &e = blk->w2;
+    const BlockProj p[4] = {{a.fmt, X_qkvg, a.Wq, a.scales, a.bias, Y_qkvg, 4 * d, d},
+                            {b.fmt, X_o, b.Wq, b.scales, b.bias, Y_o, d, d},
+                            {c.fmt, X_ffn, c.Wq, c.scales, c.bias, Y_13, 2 * f, d},
+                            {e.fmt, X_w2, e.Wq, e.scales, e.bias, Y_2, d, f}};
     return block_run(p, M, d, f, path, stream);
 }
 
@@ -426,7 +447,8 @@ int batch_route(const rt_qproj *list, int count, int64_t M, int path) {
     for (int i = 0; i < count; ++i) {
         const rt_qproj &q = list[i];
         if (!rtq::fmt_valid(q.fmt) || q.reserved != 0) return -RT_ERR_INVALID_ARG;
-        const rt_status st = rtq::check_gemm_args(q.fmt, q.X, q.Wq, q.scales, q.Y, M, q.N, q.K);
+        rt_status st = rtq::check_gemm_args(q.fmt, q.X, q.Wq, q.scales, q.Y, M, q.N, q.K);
+        if (st == RT_OK) st = check_bias(q.bias, q.Y, M, q.N);
         if (st != RT_OK) return -st;
         const int p = pick_path(M, q.K, path);
         if (p == -1) return -RT_ERR_UNSUPPORTED_SHAPE;
@@ -457,6 +479,7 @@ int batch_route(const rt_qproj *list, int count, int64_t M, int path) {
             add(q.X, M * q.K * 4, false);
             add(q.Wq, wb, false);
             if (sb > 0) add(q.scales, sb, false);
+            if (q.bias) add(q.bias, q.N * 4, false);
         }
         std::sort(r.begin(), r.end(), [](const Range &a, const Range &b) { return a.lo < b.lo; });
         // In address order, each range is checked against the furthest end
@@ -545,7 +568,8 @@ rt_status rt_qgemm_batch(const rt_qproj *list, int count, int64_t M, int path, v
         rt_status st;
         for (int i = 0; i < count; ++i) {
             const rt_qproj &q = list[i];
-            if ((st = run_gemm(q.fmt, q.X, q.Wq, q.scales, q.Y, M, q.N, q.K, path, stream)) != RT_OK)
+            if ((st = run_gemm(q.fmt, q.X, q.Wq, q.scales, q.bias, q.Y, M, q.N, q.K, path,
+                               stream)) != RT_OK)
                 return st;
         }
         return RT_OK;
@@ -556,7 +580,8 @@ rt_status rt_qgemm_batch(const rt_qproj *list, int count, int64_t M, int path, v
     std::vector<rtq::PlInput> in(static_cast<size_t>(count));
     for (int i = 0; i < count; ++i) {
         const rt_qproj &q = list[i];
-        in[i] = {q.fmt, q.X, q.Wq, q.scales, q.Y, static_cast<int>(q.N), static_cast<int>(q.K)};
+        in[i] = {q.fmt, q.X, q.Wq, q.scales, q.bias, q.Y, static_cast<int>(q.N),
+                 static_cast<int>(q.K)};
     }
     void *ws = nullptr;
     const size_t need = rtq::pl_workspace_bytes(in.data(), count, static_cast<int>(M));

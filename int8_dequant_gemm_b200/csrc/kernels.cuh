@@ -53,13 +53,16 @@ cudaError_t smem_attr_once(Kernel kernel, int bytes, int dev, std::atomic<bool> 
 }
 
 // fp32 CUDA-core path: one thread per output row, MT activation rows per block.
-cudaError_t launch_simt(int fmt, const float *X, const void *Wq, const void *S, float *Y, int M,
-                        int N, int K, cudaStream_t s);
+// Every GEMM launcher takes `bias`: NULL, or fp32 [N] added to each output
+// row in the epilogue (Y = X * W^T + bias, one fused multiply-add with the
+// q8 row scale).
+cudaError_t launch_simt(int fmt, const float *X, const void *Wq, const void *S, const float *bias,
+                        float *Y, int M, int N, int K, cudaStream_t s);
 
 // tcgen05 path: 128 weight rows x BN activation rows per CTA, fp16 operands
 // in swizzled shared memory, fp32 accumulator in TMEM.
-cudaError_t launch_tc(int fmt, const float *X, const void *Wq, const void *S, float *Y, int M,
-                      int N, int K, DevCtl *ctl, cudaStream_t s);
+cudaError_t launch_tc(int fmt, const float *X, const void *Wq, const void *S, const float *bias,
+                      float *Y, int M, int N, int K, DevCtl *ctl, cudaStream_t s);
 
 // Up to kMaxGroup independent projections with the same M (1..128) in one
 // launch of the same tcgen05 tile code: X [M, K] fp32, Wq/S as for
@@ -70,6 +73,7 @@ struct GroupProblem {
     const float *X;
     const void *Wq;
     const void *S;
+    const float *bias;
     float *Y;
     int N, K, fmt;
 };
@@ -86,14 +90,14 @@ cudaError_t launch_cvt_x16(const float *X, void *Xh, int64_t M, int64_t K, DevCt
 // (K a multiple of 128 up to 512, many activation rows); see xs.cu.  Xh is the
 // pre-pass output.
 bool xs_supported(int M, int N, int K);
-cudaError_t launch_xs(int fmt, const void *Xh, const void *Wq, const void *S, float *Y, int M,
-                      int N, int K, DevCtl *ctl, cudaStream_t s);
+cudaError_t launch_xs(int fmt, const void *Xh, const void *Wq, const void *S, const float *bias,
+                      float *Y, int M, int N, int K, DevCtl *ctl, cudaStream_t s);
 
 // tcgen05, persistent weight-stationary tiles with both operands TMA-staged
 // (more than 128 activation rows, any K of the format's TMA granule); see ws.cu.
 bool ws_supported(int fmt, int M, int N, int K);
-cudaError_t launch_ws(int fmt, const void *Xh, const void *Wq, const void *S, float *Y, int M,
-                      int N, int K, DevCtl *ctl, cudaStream_t s);
+cudaError_t launch_ws(int fmt, const void *Xh, const void *Wq, const void *S, const float *bias,
+                      float *Y, int M, int N, int K, DevCtl *ctl, cudaStream_t s);
 
 // tcgen05, a list of independent projections with the same M (1..128) in
 // persistent launches that stream every projection's weights back to back;
@@ -106,6 +110,7 @@ struct PlInput {
     const float *X;
     const void *Wq;
     const void *S;
+    const float *bias;
     float *Y;
     int N, K;
 };

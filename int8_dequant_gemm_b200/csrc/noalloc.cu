@@ -68,13 +68,13 @@ extern "C" rt_status rt_qgemm_noalloc(int fmt, const float *X, const void *Wq, c
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
     if (kern == RT_KERNEL_SIMT)
-        return from_cuda(rtq::launch_simt(fmt, X, Wq, scales, Y, m, n, k, s));
+        return from_cuda(rtq::launch_simt(fmt, X, Wq, scales, nullptr, Y, m, n, k, s));
     rtq::DevCtl *ctl = nullptr;
     if ((st = rtq::device_ctl(&ctl)) != RT_OK) return st;
     if (kern == RT_KERNEL_TC_W_STATIONARY)
-        return from_cuda(rtq::launch_tc(fmt, X, Wq, scales, Y, m, n, k, ctl, s));
+        return from_cuda(rtq::launch_tc(fmt, X, Wq, scales, nullptr, Y, m, n, k, ctl, s));
     if (rtq::launch_cvt_x16(X, xh, M, K, ctl, s) != cudaSuccess) return RT_ERR_CUDA;
     if (kern == RT_KERNEL_TC_X_RESIDENT)
-        return from_cuda(rtq::launch_xs(fmt, xh, Wq, scales, Y, m, n, k, ctl, s));
-    return from_cuda(rtq::launch_ws(fmt, xh, Wq, scales, Y, m, n, k, ctl, s));
+        return from_cuda(rtq::launch_xs(fmt, xh, Wq, scales, nullptr, Y, m, n, k, ctl, s));
+    return from_cuda(rtq::launch_ws(fmt, xh, Wq, scales, nullptr, Y, m, n, k, ctl, s));
 }

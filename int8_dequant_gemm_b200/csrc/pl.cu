@@ -502,8 +502,9 @@ __global__ void __launch_bounds__(kPlThreads, 1)
                 if (!ok) break;
                 tc_fence_after_sync();
                 const int o = (it.tile0 + tt) * 128 + q * 32 + lane;
-                float sc = 1.f;
+                float sc = 1.f, b = 0.f;
                 if (p.fmt == 8 && o < p.N) sc = __ldg(static_cast<const float *>(p.S) + o);
+                if (p.bias && o < p.N) b = __ldg(p.bias + o);
                 const uint32_t tacc = tq + static_cast<uint32_t>(slot * BNp + c0);
                 float *yo = p.Y + o;
                 const size_t rs = static_cast<size_t>(p.N);
@@ -515,7 +516,7 @@ __global__ void __launch_bounds__(kPlThreads, 1)
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
                             const int m = c0 + cc + e;
-                            if (m < M) yo[static_cast<size_t>(m) * rs] = __uint_as_float(v[e]) * sc;
+                            if (m < M) yo[static_cast<size_t>(m) * rs] = fmaf(__uint_as_float(v[e]), sc, b);
                         }
                     }
                 }
@@ -705,8 +706,8 @@ cudaError_t launch_pl_batch(const PlInput *in, int count, int M, void *ws, DevCt
             const int per = q.K > kXChunk ? nacc : 4;    // tiles per item
             const int n_items = (tiles + per - 1) / per;
             if (np > 0 && items.size() + n_items > static_cast<size_t>(kPlMaxItems)) break;
-            P.proj[np] = {wsb + im.off[im.xid[order[pos]]], q.Wq, q.S, q.Y, q.N, q.K, q.fmt,
-                          im.xid[order[pos]]};
+            P.proj[np] = {wsb + im.off[im.xid[order[pos]]], q.Wq, q.S, q.bias, q.Y, q.N, q.K,
+                          q.fmt, im.xid[order[pos]]};
             for (int t = 0; t < tiles; t += per) {
                 const int nt = std::min(per, tiles - t);
                 items.push_back({static_cast<uint32_t>(t), static_cast<uint16_t>(np),

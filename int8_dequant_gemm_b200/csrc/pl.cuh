@@ -17,6 +17,7 @@ struct PlProj {
     const uint8_t *Xh;   // fp16 image of the projection's activations (pre-pass output)
     const void *Wq;      // q4: u8 [N, K/2]; q8: i8 [N, K]
     const void *S;       // q4: binary16 (scale, min) [N, K/32, 2]; q8: fp32 [N]
+    const float *bias;   // fp32 [N] or null
     float *Y;            // fp32 [M, N]
     int N, K, fmt, xid;  // xid: index of the distinct activation image
 };

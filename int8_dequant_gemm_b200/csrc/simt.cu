@@ -118,8 +118,8 @@ __device__ __forceinline__ void simt_slice(const float *xs, const void *__restri
 template <int MT, int FMT>
 __global__ void __launch_bounds__(kSimtThreads)
     simt_kernel(const float *__restrict__ X, const void *__restrict__ Wq,
-                const void *__restrict__ S, float *__restrict__ Y, int M, int N, int K,
-                int ksplit) {
+                const void *__restrict__ S, const float *__restrict__ bias, float *__restrict__ Y,
+                int M, int N, int K, int ksplit) {
     extern __shared__ float4 xs4[];
     const float *xs = reinterpret_cast<const float *>(xs4);
     const int Ks = K / ksplit;
@@ -145,11 +145,12 @@ __global__ void __launch_bounds__(kSimtThreads)
     float acc[MT];
     simt_slice<MT, FMT>(xs, Wq, S, o, valid, K, k0, Ks, acc);
     const float sc = (FMT == 8 && valid) ? __ldg(static_cast<const float *>(S) + o) : 1.f;
+    const float b = (bias && valid) ? __ldg(bias + o) : 0.f;
     if (ksplit == 1) {
         if (valid) {
 #pragma unroll
             for (int m = 0; m < MT; ++m)
-                if (m < mt) Y[static_cast<size_t>(m0 + m) * N + o] = acc[m] * sc;
+                if (m < mt) Y[static_cast<size_t>(m0 + m) * N + o] = fmaf(acc[m], sc, b);
         }
         return;
     }
@@ -169,7 +170,8 @@ __global__ void __launch_bounds__(kSimtThreads)
         const int oo = o0 + row;
         if (m < mt && oo < N) {
             const float s8 = FMT == 8 ? __ldg(static_cast<const float *>(S) + oo) : 1.f;
-            Y[static_cast<size_t>(m0 + m) * N + oo] = v * s8;
+            const float bb = bias ? __ldg(bias + oo) : 0.f;
+            Y[static_cast<size_t>(m0 + m) * N + oo] = fmaf(v, s8, bb);
         }
     }
     cluster_sync();                           // peers are done reading this CTA's partials
@@ -186,8 +188,8 @@ int pick_simt_ksplit(int M, int N, int K, int MT) {
 }
 
 template <int MT, int FMT>
-cudaError_t launch_simt_mt(const float *X, const void *Wq, const void *S, float *Y, int M, int N,
-                           int K, cudaStream_t s) {
+cudaError_t launch_simt_mt(const float *X, const void *Wq, const void *S, const float *bias,
+                           float *Y, int M, int N, int K, cudaStream_t s) {
     const int ksplit = pick_simt_ksplit(M, N, K, MT);
     const size_t smem = static_cast<size_t>(MT) * (K / ksplit) * sizeof(float) +
                         (ksplit > 1 ? static_cast<size_t>(MT) * kSimtThreads * sizeof(float) : 0);
@@ -214,30 +216,30 @@ cudaError_t launch_simt_mt(const float *X, const void *Wq, const void *S, float 
     attr[1].val.clusterDim.z = static_cast<unsigned>(ksplit);
     cfg.attrs = attr;
     cfg.numAttrs = ksplit > 1 ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, simt_kernel<MT, FMT>, X, Wq, S, Y, M, N, K, ksplit);
+    return cudaLaunchKernelEx(&cfg, simt_kernel<MT, FMT>, X, Wq, S, bias, Y, M, N, K, ksplit);
 }
 
 template <int MT>
-cudaError_t launch_simt_fmt(int fmt, const float *X, const void *Wq, const void *S, float *Y,
-                            int M, int N, int K, cudaStream_t s) {
-    if (fmt == kFmtQ4) return launch_simt_mt<MT, kFmtQ4>(X, Wq, S, Y, M, N, K, s);
-    if (fmt == kFmtQ8) return launch_simt_mt<MT, kFmtQ8>(X, Wq, S, Y, M, N, K, s);
-    return launch_simt_mt<MT, kFmtE4M3>(X, Wq, S, Y, M, N, K, s);
+cudaError_t launch_simt_fmt(int fmt, const float *X, const void *Wq, const void *S,
+                            const float *bias, float *Y, int M, int N, int K, cudaStream_t s) {
+    if (fmt == kFmtQ4) return launch_simt_mt<MT, kFmtQ4>(X, Wq, S, bias, Y, M, N, K, s);
+    if (fmt == kFmtQ8) return launch_simt_mt<MT, kFmtQ8>(X, Wq, S, bias, Y, M, N, K, s);
+    return launch_simt_mt<MT, kFmtE4M3>(X, Wq, S, bias, Y, M, N, K, s);
 }
 
 }  // namespace
 
 // Activation rows per block: as many as M needs up to 8, capped so the staged
 // activations stay within 128 KB of shared memory.
-cudaError_t launch_simt(int fmt, const float *X, const void *Wq, const void *S, float *Y, int M,
-                        int N, int K, cudaStream_t s) {
+cudaError_t launch_simt(int fmt, const float *X, const void *Wq, const void *S, const float *bias,
+                        float *Y, int M, int N, int K, cudaStream_t s) {
     int mt = M >= 8 ? 8 : (M >= 4 ? 4 : (M >= 2 ? 2 : 1));
     while (mt > 1 && static_cast<size_t>(mt) * K * sizeof(float) > 128 * 1024) mt /= 2;
     switch (mt) {
-        case 8: return launch_simt_fmt<8>(fmt, X, Wq, S, Y, M, N, K, s);
-        case 4: return launch_simt_fmt<4>(fmt, X, Wq, S, Y, M, N, K, s);
-        case 2: return launch_simt_fmt<2>(fmt, X, Wq, S, Y, M, N, K, s);
-        default: return launch_simt_fmt<1>(fmt, X, Wq, S, Y, M, N, K, s);
+        case 8: return launch_simt_fmt<8>(fmt, X, Wq, S, bias, Y, M, N, K, s);
+        case 4: return launch_simt_fmt<4>(fmt, X, Wq, S, bias, Y, M, N, K, s);
+        case 2: return launch_simt_fmt<2>(fmt, X, Wq, S, bias, Y, M, N, K, s);
+        default: return launch_simt_fmt<1>(fmt, X, Wq, S, bias, Y, M, N, K, s);
     }
 }
 

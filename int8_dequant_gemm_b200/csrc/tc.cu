@@ -221,9 +221,9 @@ __device__ __forceinline__ bool nonfinite(float v) {
 template <int FMT, int PIECES>
 __device__ __forceinline__ void tc_tile(uint8_t *smem_raw, const float *__restrict__ X,
                                         const void *__restrict__ Wq, const void *__restrict__ S,
-                                        float *__restrict__ Y, int M, int N, int K, int BN,
-                                        int stages, int ksplit, int o0, int m0, int kslice,
-                                        int kbase, DevCtl *ctl) {
+                                        const float *__restrict__ bias, float *__restrict__ Y,
+                                        int M, int N, int K, int BN, int stages, int ksplit,
+                                        int o0, int m0, int kslice, int kbase, DevCtl *ctl) {
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *smem = smem_raw + (base - raw);
@@ -321,8 +321,9 @@ __device__ __forceinline__ void tc_tile(uint8_t *smem_raw, const float *__restri
             const int half = warp >> 2;        // which half of the columns
             const int row = q * 32 + lane;
             const int o = o0 + row;
-            float sc = 1.f;
+            float sc = 1.f, b = 0.f;
             if (FMT == 8 && o < N) sc = __ldg(static_cast<const float *>(S) + o);
+            if (bias && o < N) b = __ldg(bias + o);
             const int ncol = BN / 2;           // a multiple of 8
             const int c0 = half * ncol;
             const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16);
@@ -348,7 +349,7 @@ __device__ __forceinline__ void tc_tile(uint8_t *smem_raw, const float *__restri
                     for (int j = 0; j < 8; ++j) {
                         const int m = m0 + c + j;
                         if (m < M) {
-                            const float y = __uint_as_float(v0[j]) * sc;
+                            const float y = fmaf(__uint_as_float(v0[j]), sc, b);
                             ybad |= nonfinite(y);
                             Y[static_cast<size_t>(m) * N + o] = y;
                         }
@@ -358,7 +359,7 @@ __device__ __forceinline__ void tc_tile(uint8_t *smem_raw, const float *__restri
                         for (int j = 0; j < 8; ++j) {
                             const int m = m0 + c + 8 + j;
                             if (m < M) {
-                                const float y = __uint_as_float(v1[j]) * sc;
+                                const float y = fmaf(__uint_as_float(v1[j]), sc, b);
                                 ybad |= nonfinite(y);
                                 Y[static_cast<size_t>(m) * N + o] = y;
                             }
@@ -435,10 +436,13 @@ __device__ __forceinline__ void tc_tile(uint8_t *smem_raw, const float *__restri
                 }
                 if (m < M && o < N) {
                     float a[4] = {acc.x, acc.y, acc.z, acc.w};
-                    if (FMT == 8) {
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            if (o + e < N) a[e] *= __ldg(static_cast<const float *>(S) + o + e);
+                    for (int e = 0; e < 4; ++e) {
+                        if (o + e < N) {
+                            const float s = FMT == 8 ? __ldg(static_cast<const float *>(S) + o + e)
+                                                     : 1.f;
+                            a[e] = fmaf(a[e], s, bias ? __ldg(bias + o + e) : 0.f);
+                        }
                     }
 #pragma unroll
                     for (int e = 0; e < 4; ++e) ybad |= o + e < N && nonfinite(a[e]);
@@ -466,10 +470,11 @@ __device__ __forceinline__ void tc_tile(uint8_t *smem_raw, const float *__restri
 template <int FMT, int PIECES>
 __global__ void __launch_bounds__(kTcThreads, 2)
     tc_qgemm_kernel(const float *__restrict__ X, const void *__restrict__ Wq,
-                    const void *__restrict__ S, float *__restrict__ Y, int M, int N, int K,
-                    int BN, int stages, int ksplit, DevCtl *ctl) {
+                    const void *__restrict__ S, const float *__restrict__ bias,
+                    float *__restrict__ Y, int M, int N, int K, int BN, int stages, int ksplit,
+                    DevCtl *ctl) {
     extern __shared__ uint8_t smem_raw[];
-    tc_tile<FMT, PIECES>(smem_raw, X, Wq, S, Y, M, N, K, BN, stages, ksplit,
+    tc_tile<FMT, PIECES>(smem_raw, X, Wq, S, bias, Y, M, N, K, BN, stages, ksplit,
                          static_cast<int>(blockIdx.x) * kTileO, static_cast<int>(blockIdx.y) * BN,
                          static_cast<int>(blockIdx.z), 0, ctl);
 }
@@ -486,6 +491,7 @@ struct TcProblem {
     const float *X;
     const void *Wq;
     const void *S;
+    const float *bias;
     float *Y;
     int N, K, fmt, cl0, ks;
 };
@@ -509,14 +515,14 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     const int o0 = tile * kTileO;
     const int kslice = r % p.ks, kbase = r - kslice;
     if (p.fmt == kFmtQ4)
-        tc_tile<kFmtQ4, PIECES>(smem_raw, p.X, p.Wq, p.S, p.Y, M, p.N, p.K, BN, stages, p.ks, o0,
-                                0, kslice, kbase, ctl);
+        tc_tile<kFmtQ4, PIECES>(smem_raw, p.X, p.Wq, p.S, p.bias, p.Y, M, p.N, p.K, BN, stages,
+                                p.ks, o0, 0, kslice, kbase, ctl);
     else if (p.fmt == kFmtQ8)
-        tc_tile<kFmtQ8, PIECES>(smem_raw, p.X, p.Wq, p.S, p.Y, M, p.N, p.K, BN, stages, p.ks, o0,
-                                0, kslice, kbase, ctl);
+        tc_tile<kFmtQ8, PIECES>(smem_raw, p.X, p.Wq, p.S, p.bias, p.Y, M, p.N, p.K, BN, stages,
+                                p.ks, o0, 0, kslice, kbase, ctl);
     else
-        tc_tile<kFmtE4M3, PIECES>(smem_raw, p.X, p.Wq, p.S, p.Y, M, p.N, p.K, BN, stages, p.ks,
-                                  o0, 0, kslice, kbase, ctl);
+        tc_tile<kFmtE4M3, PIECES>(smem_raw, p.X, p.Wq, p.S, p.bias, p.Y, M, p.N, p.K, BN, stages,
+                                  p.ks, o0, 0, kslice, kbase, ctl);
 }
 
 // Activation rows per tile: one tile when M <= 128; otherwise 128, halved
@@ -544,8 +550,8 @@ int pick_ksplit(int M, int N, int K, int BN) {
 }
 
 template <int FMT, int PIECES>
-cudaError_t launch_tc_pieces(const float *X, const void *Wq, const void *S, float *Y, int M, int N,
-                            int K, int BN, DevCtl *ctl, cudaStream_t st) {
+cudaError_t launch_tc_pieces(const float *X, const void *Wq, const void *S, const float *bias,
+                             float *Y, int M, int N, int K, int BN, DevCtl *ctl, cudaStream_t st) {
     static std::atomic<bool> attr_done[kMaxDevices];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -571,17 +577,17 @@ cudaError_t launch_tc_pieces(const float *X, const void *Wq, const void *S, floa
     attr[1].val.clusterDim.z = static_cast<unsigned>(ksplit);
     cfg.attrs = attr;
     cfg.numAttrs = ksplit > 1 ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, tc_qgemm_kernel<FMT, PIECES>, X, Wq, S, Y, M, N, K, BN,
-                              stages, ksplit, ctl);
+    return cudaLaunchKernelEx(&cfg, tc_qgemm_kernel<FMT, PIECES>, X, Wq, S, bias, Y, M, N, K,
+                              BN, stages, ksplit, ctl);
 }
 
 template <int FMT>
-cudaError_t launch_tc_fmt(const float *X, const void *Wq, const void *S, float *Y, int M, int N,
-                          int K, DevCtl *ctl, cudaStream_t st) {
+cudaError_t launch_tc_fmt(const float *X, const void *Wq, const void *S, const float *bias,
+                          float *Y, int M, int N, int K, DevCtl *ctl, cudaStream_t st) {
     const int BN = pick_bn(M, N);
-    if (BN <= 32) return launch_tc_pieces<FMT, 2>(X, Wq, S, Y, M, N, K, BN, ctl, st);
-    if (BN <= 64) return launch_tc_pieces<FMT, 4>(X, Wq, S, Y, M, N, K, BN, ctl, st);
-    return launch_tc_pieces<FMT, 8>(X, Wq, S, Y, M, N, K, BN, ctl, st);
+    if (BN <= 32) return launch_tc_pieces<FMT, 2>(X, Wq, S, bias, Y, M, N, K, BN, ctl, st);
+    if (BN <= 64) return launch_tc_pieces<FMT, 4>(X, Wq, S, bias, Y, M, N, K, BN, ctl, st);
+    return launch_tc_pieces<FMT, 8>(X, Wq, S, bias, Y, M, N, K, BN, ctl, st);
 }
 
 // K splits for a group.  A launch lasts as long as its longest chain of K
@@ -668,16 +674,16 @@ cudaError_t launch_tc_group(const GroupProblem *probs, int count, int M, DevCtl 
         const GroupProblem &q = probs[i];
         if (!fmt_valid(q.fmt) || q.N < 1 || q.K < kTileK || q.K % kTileK != 0)
             return cudaErrorInvalidValue;
-        g.p[i] = {q.X, q.Wq, q.S, q.Y, q.N, q.K, q.fmt, 0, 1};
+        g.p[i] = {q.X, q.Wq, q.S, q.bias, q.Y, q.N, q.K, q.fmt, 0, 1};
     }
     return launch_group(g, M, ctl, s);
 }
 
-cudaError_t launch_tc(int fmt, const float *X, const void *Wq, const void *S, float *Y, int M,
-                      int N, int K, DevCtl *ctl, cudaStream_t s) {
-    if (fmt == kFmtQ4) return launch_tc_fmt<kFmtQ4>(X, Wq, S, Y, M, N, K, ctl, s);
-    if (fmt == kFmtQ8) return launch_tc_fmt<kFmtQ8>(X, Wq, S, Y, M, N, K, ctl, s);
-    return launch_tc_fmt<kFmtE4M3>(X, Wq, S, Y, M, N, K, ctl, s);
+cudaError_t launch_tc(int fmt, const float *X, const void *Wq, const void *S, const float *bias,
+                      float *Y, int M, int N, int K, DevCtl *ctl, cudaStream_t s) {
+    if (fmt == kFmtQ4) return launch_tc_fmt<kFmtQ4>(X, Wq, S, bias, Y, M, N, K, ctl, s);
+    if (fmt == kFmtQ8) return launch_tc_fmt<kFmtQ8>(X, Wq, S, bias, Y, M, N, K, ctl, s);
+    return launch_tc_fmt<kFmtE4M3>(X, Wq, S, bias, Y, M, N, K, ctl, s);
 }
 
 }  // namespace rtq

@@ -86,8 +86,8 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     ws_qgemm_kernel(const __grid_constant__ CUtensorMap w_map,
                     const __grid_constant__ CUtensorMap s_map,
                     const __grid_constant__ CUtensorMap x_map, const float *__restrict__ S8,
-                    float *__restrict__ Y, int M, int N, int K, int n_o_tiles, int n_tiles,
-                    DevCtl *ctl) {
+                    const float *__restrict__ bias, float *__restrict__ Y, int M, int N, int K,
+                    int n_o_tiles, int n_tiles, DevCtl *ctl) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_addr(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;
@@ -366,8 +366,9 @@ __global__ void __launch_bounds__(kWsThreads, 1)
             tc_fence_after_sync();
             const int m0 = (t / n_o_tiles) * kWsTileM;
             const int o = (t % n_o_tiles) * kTileRows + row;
-            float sc = 1.f;
+            float sc = 1.f, bo = 0.f;
             if (FMT == 8 && o < N) sc = __ldg(S8 + o);
+            if (bias && o < N) bo = __ldg(bias + o);
             const int mlim = min(kWsTileM, M - m0);
             float *yo = Y + static_cast<size_t>(m0) * N + o;
             const size_t rs = static_cast<size_t>(N);
@@ -379,11 +380,11 @@ __global__ void __launch_bounds__(kWsThreads, 1)
                     float *p = yo + static_cast<size_t>(c) * rs;
                     if (c + 32 <= mlim) {
 #pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) p[jj * rs] = __uint_as_float(v[jj]) * sc;
+                        for (int jj = 0; jj < 32; ++jj) p[jj * rs] = fmaf(__uint_as_float(v[jj]), sc, bo);
                     } else {
 #pragma unroll
                         for (int jj = 0; jj < 32; ++jj)
-                            if (c + jj < mlim) p[jj * rs] = __uint_as_float(v[jj]) * sc;
+                            if (c + jj < mlim) p[jj * rs] = fmaf(__uint_as_float(v[jj]), sc, bo);
                     }
                 }
             }
@@ -402,8 +403,8 @@ __global__ void __launch_bounds__(kWsThreads, 1)
 }
 
 template <int FMT>
-cudaError_t launch_ws_fmt(const void *Xh, const void *Wq, const void *S, float *Y, int M, int N,
-                          int K, DevCtl *ctl, cudaStream_t st) {
+cudaError_t launch_ws_fmt(const void *Xh, const void *Wq, const void *S, const float *bias,
+                          float *Y, int M, int N, int K, DevCtl *ctl, cudaStream_t st) {
     static std::atomic<bool> attr_done[kMaxDevices];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -441,7 +442,7 @@ cudaError_t launch_ws_fmt(const void *Xh, const void *Wq, const void *S, float *
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, ws_qgemm_kernel<FMT>, w_map, s_map, x_map,
-                              static_cast<const float *>(S), Y, M, N, K, n_o, tiles, ctl);
+                              static_cast<const float *>(S), bias, Y, M, N, K, n_o, tiles, ctl);
 }
 
 }  // namespace
@@ -455,11 +456,11 @@ bool ws_supported(int fmt, int M, int N, int K) {
     return fmt == 4 ? K % 128 == 0 : K % 64 == 0;
 }
 
-cudaError_t launch_ws(int fmt, const void *Xh, const void *Wq, const void *S, float *Y, int M,
-                      int N, int K, DevCtl *ctl, cudaStream_t s) {
-    if (fmt == kFmtQ4) return launch_ws_fmt<kFmtQ4>(Xh, Wq, S, Y, M, N, K, ctl, s);
-    if (fmt == kFmtQ8) return launch_ws_fmt<kFmtQ8>(Xh, Wq, S, Y, M, N, K, ctl, s);
-    return launch_ws_fmt<kFmtE4M3>(Xh, Wq, S, Y, M, N, K, ctl, s);
+cudaError_t launch_ws(int fmt, const void *Xh, const void *Wq, const void *S, const float *bias,
+                      float *Y, int M, int N, int K, DevCtl *ctl, cudaStream_t s) {
+    if (fmt == kFmtQ4) return launch_ws_fmt<kFmtQ4>(Xh, Wq, S, bias, Y, M, N, K, ctl, s);
+    if (fmt == kFmtQ8) return launch_ws_fmt<kFmtQ8>(Xh, Wq, S, bias, Y, M, N, K, ctl, s);
+    return launch_ws_fmt<kFmtE4M3>(Xh, Wq, S, bias, Y, M, N, K, ctl, s);
 }
 
 }  // namespace rtq

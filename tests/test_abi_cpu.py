@@ -320,11 +320,11 @@ def _qproj_array(entries):
 
 
 def test_batch_validation_and_routes():
-    # (fmt, reserved, X, Wq, scales, Y, N, K) at fake, aligned, disjoint addresses
+    # (fmt, reserved, X, Wq, scales, bias, Y, N, K) at fake, aligned, disjoint addresses
     GB = 1 << 30
     def entry(i, fmt=4, N=2048, K=512, X=None, Y=None):
         return (fmt, 0, X or (1 * GB + i * 16 * 2 ** 20), 2 * GB + i * 16 * 2 ** 20,
-                3 * GB + i * 16 * 2 ** 20, Y or (4 * GB + i * 16 * 2 ** 20), N, K)
+                3 * GB + i * 16 * 2 ** 20, None, Y or (4 * GB + i * 16 * 2 ** 20), N, K)
     plan, run = rtq.lib().rt_qgemm_batch_plan, rtq.lib().rt_qgemm_batch
     TC_LIST = 5
     ok = _qproj_array([entry(i) for i in range(12)])          # 12 x 16 tiles = 192 >= SMs
@@ -426,5 +426,19 @@ def test_e4m3_gemm_validation_and_plan():
     assert rtq.auto_path(3, 80, 512, 48) == 1                     # K % 64 != 0 -> SIMT
     assert rtq.workspace_bytes(3, 4096, 512, 2048) == 4096 * 2048 * 2
     # a batch entry in e4m3 carries no scales
-    arr = _qproj_array([(3, 0, X, W, 0, Y, 2048, 512)] * 1)
+    arr = _qproj_array([(3, 0, X, W, 0, None, Y, 2048, 512)] * 1)
     assert rtq.lib().rt_qgemm_batch_plan(arr, 1, 80, 2) == 5
+
+
+def test_bias_validation():
+    f = rtq.lib().rt_qgemm
+    GB = 1 << 30
+    B = 5 * GB
+    assert f(4, X, W, S, B + 2, Y, 4, 16, 64, 0, None) == ALIGN        # bias not 4-byte aligned
+    assert f(4, X, W, S, Y + 64, Y, 4, 16, 64, 0, None) == INVALID     # bias overlaps Y
+    assert f(9, X, W, S, B, Y, 4, 16, 64, 0, None) == INVALID          # unknown format
+    assert f(3, X, W, None, B, Y, 4, 16, 24, 0, None) == SHAPE         # e4m3 K % 16
+    assert f(4, None, W, S, None, None, 0, 16, 64, 0, None) == RT_OK   # M == 0
+    # a list entry's output may not overlap another entry's bias
+    arr = _qproj_array([(4, 0, X, W, S, B, Y, 16, 64), (4, 0, X, W, S, None, B, 16, 64)])
+    assert rtq.lib().rt_qgemm_batch(arr, 2, 4, 0, None) == INVALID

@@ -77,21 +77,20 @@ class Entry:
 
 
 def device_list(rtq, entries, M, Xd=None, guard=64):
-    """Device tensors of the entries; every Y is a view of one NaN-filled
-    buffer with `guard` floats between outputs."""
+    """Device tensors of the entries; every Y is a 16-byte aligned view of one
+    NaN-filled buffer with at least `guard` floats between outputs."""
     sizes = [M * e.N for e in entries]
-    flat = torch.full((sum(sizes) + guard * (len(sizes) + 1),), float("nan"), device="cuda")
-    projs, off = [], guard
-    for i, (e, sz) in enumerate(zip(entries, sizes)):
-        X = Xd[i] if Xd is not None else dev(e.X)
-        Y = flat[off:off + sz].view(M, e.N)
-        off += sz + guard
-        projs.append(rtq.Proj(e.fmt, X, dev(e.q[0]), dev(e.q[1]), Y))
-    mask = torch.ones_like(flat, dtype=torch.bool)
-    off = guard
+    offs, off = [], guard
     for sz in sizes:
-        mask[off:off + sz] = False
-        off += sz + guard
+        offs.append(off)
+        off = (off + sz + guard + 3) // 4 * 4
+    flat = torch.full((off,), float("nan"), device="cuda")
+    projs = []
+    mask = torch.ones_like(flat, dtype=torch.bool)
+    for i, (e, sz, o) in enumerate(zip(entries, sizes, offs)):
+        X = Xd[i] if Xd is not None else dev(e.X)
+        projs.append(rtq.Proj(e.fmt, X, dev(e.q[0]), dev(e.q[1]), flat[o:o + sz].view(M, e.N)))
+        mask[o:o + sz] = False
     return projs, flat, mask
 
 
@@ -197,7 +196,7 @@ def test_routes_and_rejections(rtq_lib):
     check(entries, projs, flat, mask)
     # an output overlapping another entry's output is rejected before any launch
     bad = [projs[0], rtq_lib.Proj(projs[1].fmt, projs[1].X, projs[1].Wq, projs[1].scales,
-                                  flat[64:64 + M * 512].view(M, 512))]
+                                  flat[64:64 + M * 512].view(M, 512))]   # entry 0's output
     with pytest.raises(rtq_lib.RtqError) as e:
         rtq_lib.qgemm_batch(bad, path="tc")
     assert e.value.status == rtq_lib.RT_ERR_INVALID_ARG
