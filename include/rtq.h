@@ -253,12 +253,16 @@ rt_status rt_qgemm_noalloc(int fmt, const float *X, const void *Wq, const void *
  *
  * Route (rt_qgemm_batch_plan): with 1 <= M <= 128 on the tensor-core path
  * (RT_PATH_AUTO above the SIMT range, or RT_PATH_TC), every entry's K a
- * multiple of 128 (q4) or 64 (q8) and every q4 scale_min 16-byte aligned, the
- * list runs as RT_KERNEL_TC_LIST: one
- * pre-pass launch rounds each distinct (X, K) once to fp16 into the
- * stream's workspace (rt_workspace_reserve applies; M rounded up to 16, times
- * K, times 2 bytes per distinct X), then persistent launches of up to 256
- * entries each stream the entries' weights through every SM.  Under
+ * multiple of 128 (q4) or 64 (q8 and e4m3) and every q4 scale_min 16-byte
+ * aligned, the list runs as RT_KERNEL_TC_LIST: one pre-pass launch rounds
+ * each distinct (X, K) once to fp16 into the stream's workspace, then
+ * persistent launches of up to 256 entries each stream the entries' weights
+ * through every SM.  An entry with K > 512 is computed in 512-wide K chunks
+ * whose fp32 partial tiles are summed in chunk order (deterministically) by
+ * whichever chunk finishes last.  Workspace (rt_workspace_reserve applies):
+ * per distinct (X, K) M16 * K * 2 bytes, plus for the entries with K > 512
+ * ceil(N / 128) * ceil(K / 512) * M16 * 512 bytes of partials, with M16 = M
+ * rounded up to 16 (a few more bytes for counters and alignment).  Under
  * RT_PATH_AUTO this happens only when the entries hold at least as many
  * 128-row weight tiles as the GPU has SMs.  Otherwise the entries run one
  * after another as rt_qgemm_q4/q8 calls.  Results are those of the

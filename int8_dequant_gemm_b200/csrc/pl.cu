@@ -74,7 +74,8 @@ constexpr int kXWarp = 20;
 constexpr int kPlThreads = (kXWarp + 1) * 32;        // 672
 constexpr int kProdThreads = kProdWarps * 32;        // 64
 constexpr int kEpiThreads = kEpiWarps * 32;          // 256
-constexpr uint32_t kMmaBar = 1;
+constexpr uint32_t kMmaBar = 1;                      // named barrier: waiter <-> issuer
+constexpr uint32_t kEpiBar = 2;                      // named barrier: the epilogue warps
 constexpr int kSlotBytes = 32 * 1024;                // 128 rows x 256 bytes of codes
 constexpr int kScaleBytes = 8 * 1024;                // 128 rows x 16 (scale, min) words
 constexpr int kMaxSlots = 4;
@@ -96,8 +97,9 @@ __host__ __device__ inline PlLayout pl_layout(int bnp, int nslots) {
     L.w_off = bnp * kXChunk * 2;
     L.s_off = L.w_off + nslots * kSlotBytes;
     L.bar_off = L.s_off + nslots * kScaleBytes;
-    // slot full/empty, A full/empty, x full/empty, acc full/empty, drain, TMEM slot
-    L.total = L.bar_off + (2 * kMaxSlots + 2 * kAStages + 2 + 2 * kPlMaxAcc + 1) * 8 + 16;
+    // slot full/empty, A full/empty, x full/empty, acc full/empty, drain, then
+    // 8 words: TMEM address, 2 issuer abort flags, the epilogue's flags
+    L.total = L.bar_off + (2 * kMaxSlots + 2 * kAStages + 2 + 2 * kPlMaxAcc + 1) * 8 + 32;
     return L;
 }
 
@@ -130,11 +132,12 @@ __device__ __forceinline__ int wswz(int c, int r) { return (c & 8) | ((c & 7) ^ 
 // Physical 16-byte chunk of logical scale chunk c (0..3) of row r.
 __device__ __forceinline__ int sswz(int c, int r) { return c ^ ((r >> 1) & 3); }
 
-// The walk every role takes through a CTA's items: item -> K chunk -> tile ->
-// weight slot -> 64-wide K step.  Each role advances it at its own grain.
+// The walk every role takes through a CTA's items: item (one K chunk of a
+// few tiles) -> tile -> weight slot -> 64-wide K step.  Each role advances it
+// at its own grain.
 struct Item {
     const PlProj *p;
-    int tile0, ntiles, nchunks;
+    int tile0, ntiles, chunk, nchunks;
 };
 
 __device__ __forceinline__ Item item_at(const PlParams &P, int i) {
@@ -143,6 +146,7 @@ __device__ __forceinline__ Item item_at(const PlParams &P, int i) {
     r.p = &P.proj[it.proj];
     r.tile0 = static_cast<int>(it.tile0);
     r.ntiles = it.ntiles;
+    r.chunk = it.chunk;
     r.nchunks = (r.p->K + kXChunk - 1) / kXChunk;
     return r;
 }
@@ -243,52 +247,46 @@ __global__ void __launch_bounds__(kPlThreads, 1)
         for (int i = i_first; i < i_last && ok; ++i) {
             const Item it = item_at(P, i);
             const PlProj &p = *it.p;
-            const int fmt = p.fmt;
+            const int fmt = p.fmt, c = it.chunk;
             const size_t row_stride = fmt == 4 ? static_cast<size_t>(p.K / 2) : static_cast<size_t>(p.K);
-            for (int c = 0; c < it.nchunks && ok; ++c) {
-                const int nw = slots_in_chunk(p, c);
-                for (int tt = 0; tt < it.ntiles && ok; ++tt) {
-                    const int o0 = (it.tile0 + tt) * 128;
-                    const int rows = min(128, p.N - o0);
-                    for (int w = 0; w < nw; ++w, ++j) {
-                        const int slot = j % NS;
-                        if (j >= NS &&
-                            !mbar_wait(&slot_empty[slot], static_cast<uint32_t>((j / NS) - 1) & 1u,
-                                       lim)) {
-                            ok = false;
-                            break;
-                        }
-                        int k0;
-                        const int klen = slot_len(p, c, w, k0);
-                        const int row_chunks = (fmt == 4 ? klen / 2 : klen) / 16;
-                        const uint8_t *src = static_cast<const uint8_t *>(p.Wq) +
-                                             static_cast<size_t>(o0) * row_stride +
-                                             (fmt == 4 ? k0 / 2 : k0);
-                        const uint32_t dst = base + L.w_off + slot * kSlotBytes;
-                        for (int e = t; e < 128 * 16; e += kProdThreads) {
-                            const int r = e >> 4, ch = e & 15;
-                            if (r < rows && ch < row_chunks)
-                                cp_async_16(dst + r * 256 + wswz(ch, r) * 16,
-                                            src + static_cast<size_t>(r) * row_stride + ch * 16);
-                        }
-                        if (fmt == 4) {
-                            // (scale, min) words of the slot's groups: klen / 32
-                            // words per row, 16-byte chunks of 4 words
-                            const int schunks = klen / 128;
-                            const uint8_t *ssrc = static_cast<const uint8_t *>(p.S) +
-                                                  static_cast<size_t>(o0) * (p.K / 32) * 4 +
-                                                  (k0 / 32) * 4;
-                            const uint32_t sdst = base + L.s_off + slot * kScaleBytes;
-                            for (int e = t; e < 128 * 4; e += kProdThreads) {
-                                const int r = e >> 2, ch = e & 3;
-                                if (r < rows && ch < schunks)
-                                    cp_async_16(sdst + r * 64 + sswz(ch, r) * 16,
-                                                ssrc + static_cast<size_t>(r) * (p.K / 32) * 4 +
-                                                    ch * 16);
-                            }
-                        }
-                        if (!(j == 0 && t == 0 && ctl->inject)) cp_async_arrive(&slot_full[slot]);
+            const int nw = slots_in_chunk(p, c);
+            for (int tt = 0; tt < it.ntiles && ok; ++tt) {
+                const int o0 = (it.tile0 + tt) * 128;
+                const int rows = min(128, p.N - o0);
+                for (int w = 0; w < nw; ++w, ++j) {
+                    const int slot = j % NS;
+                    if (j >= NS &&
+                        !mbar_wait(&slot_empty[slot], static_cast<uint32_t>((j / NS) - 1) & 1u, lim)) {
+                        ok = false;
+                        break;
                     }
+                    int k0;
+                    const int klen = slot_len(p, c, w, k0);
+                    const int row_chunks = (fmt == 4 ? klen / 2 : klen) / 16;
+                    const uint8_t *src = static_cast<const uint8_t *>(p.Wq) +
+                                         static_cast<size_t>(o0) * row_stride + (fmt == 4 ? k0 / 2 : k0);
+                    const uint32_t dst = base + L.w_off + slot * kSlotBytes;
+                    for (int e = t; e < 128 * 16; e += kProdThreads) {
+                        const int r = e >> 4, ch = e & 15;
+                        if (r < rows && ch < row_chunks)
+                            cp_async_16(dst + r * 256 + wswz(ch, r) * 16,
+                                        src + static_cast<size_t>(r) * row_stride + ch * 16);
+                    }
+                    if (fmt == 4) {
+                        // (scale, min) words of the slot's groups: klen / 32
+                        // words per row, 16-byte chunks of 4 words
+                        const int schunks = klen / 128;
+                        const uint8_t *ssrc = static_cast<const uint8_t *>(p.S) +
+                                              static_cast<size_t>(o0) * (p.K / 32) * 4 + (k0 / 32) * 4;
+                        const uint32_t sdst = base + L.s_off + slot * kScaleBytes;
+                        for (int e = t; e < 128 * 4; e += kProdThreads) {
+                            const int r = e >> 2, ch = e & 3;
+                            if (r < rows && ch < schunks)
+                                cp_async_16(sdst + r * 64 + sswz(ch, r) * 16,
+                                            ssrc + static_cast<size_t>(r) * (p.K / 32) * 4 + ch * 16);
+                        }
+                    }
+                    if (!(j == 0 && t == 0 && ctl->inject)) cp_async_arrive(&slot_full[slot]);
                 }
             }
         }
@@ -301,21 +299,19 @@ __global__ void __launch_bounds__(kPlThreads, 1)
             for (int i = i_first; i < i_last && ok; ++i) {
                 const Item it = item_at(P, i);
                 const PlProj &p = *it.p;
-                for (int c = 0; c < it.nchunks; ++c) {
-                    if (p.xid == cur_x && c == cur_c) continue;
-                    if (nx > 0 && !mbar_wait(x_empty, static_cast<uint32_t>(nx - 1) & 1u, lim)) {
-                        ok = false;
-                        break;
-                    }
-                    const int atoms = (min(kXChunk, p.K - c * kXChunk)) / 64;
-                    const uint32_t bytes = static_cast<uint32_t>(atoms * BNp * 128);
-                    mbar_expect_tx(x_full, bytes);
-                    bulk_load(base + L.x_off, p.Xh + static_cast<size_t>(c) * BNp * 1024, bytes,
-                              x_full);
-                    cur_x = p.xid;
-                    cur_c = c;
-                    ++nx;
+                const int c = it.chunk;
+                if (p.xid == cur_x && c == cur_c) continue;
+                if (nx > 0 && !mbar_wait(x_empty, static_cast<uint32_t>(nx - 1) & 1u, lim)) {
+                    ok = false;
+                    break;
                 }
+                const int atoms = (min(kXChunk, p.K - c * kXChunk)) / 64;
+                const uint32_t bytes = static_cast<uint32_t>(atoms * BNp * 128);
+                mbar_expect_tx(x_full, bytes);
+                bulk_load(base + L.x_off, p.Xh + static_cast<size_t>(c) * BNp * 1024, bytes, x_full);
+                cur_x = p.xid;
+                cur_c = c;
+                ++nx;
             }
             if (nx > 0) mbar_wait(x_full, static_cast<uint32_t>(nx - 1) & 1u, lim);
         }
@@ -330,44 +326,43 @@ __global__ void __launch_bounds__(kPlThreads, 1)
         for (int i = i_first; i < i_last && ok; ++i) {
             const Item it = item_at(P, i);
             const PlProj &p = *it.p;
-            for (int c = 0; c < it.nchunks && ok; ++c) {
-                const int nw = slots_in_chunk(p, c);
-                for (int tt = 0; tt < it.ntiles && ok; ++tt) {
-                    for (int w = 0; w < nw; ++w, ++j) {
-                        const int slot = j % NS;
-                        if (!mbar_wait(&slot_full[slot], static_cast<uint32_t>(j / NS) & 1u, lim)) {
+            const int c = it.chunk;
+            const int nw = slots_in_chunk(p, c);
+            for (int tt = 0; tt < it.ntiles && ok; ++tt) {
+                for (int w = 0; w < nw; ++w, ++j) {
+                    const int slot = j % NS;
+                    if (!mbar_wait(&slot_full[slot], static_cast<uint32_t>(j / NS) & 1u, lim)) {
+                        ok = false;
+                        break;
+                    }
+                    int k0;
+                    const int nsteps = slot_len(p, c, w, k0) / 64;
+                    const uint32_t wslot = base + L.w_off + slot * kSlotBytes;
+                    const uint32_t sslot = base + L.s_off + slot * kScaleBytes;
+                    for (int s = 0; s < nsteps; ++s, ++ja) {
+                        uint32_t wv[16];
+                        if (p.fmt == kFmtQ4)
+                            dequant_slot<kFmtQ4>(wslot, sslot, r, h, s, wv);
+                        else if (p.fmt == kFmtQ8)
+                            dequant_slot<kFmtQ8>(wslot, sslot, r, h, s, wv);
+                        else
+                            dequant_slot<kFmtE4M3>(wslot, sslot, r, h, s, wv);
+                        const int st = ja % kAStages;
+                        if (ja >= kAStages &&
+                            !mbar_wait(&a_empty[st], static_cast<uint32_t>((ja / kAStages) - 1) & 1u,
+                                       lim)) {
                             ok = false;
                             break;
                         }
-                        int k0;
-                        const int nsteps = slot_len(p, c, w, k0) / 64;
-                        const uint32_t wslot = base + L.w_off + slot * kSlotBytes;
-                        const uint32_t sslot = base + L.s_off + slot * kScaleBytes;
-                        for (int s = 0; s < nsteps; ++s, ++ja) {
-                            uint32_t wv[16];
-                            if (p.fmt == kFmtQ4)
-                                dequant_slot<kFmtQ4>(wslot, sslot, r, h, s, wv);
-                            else if (p.fmt == kFmtQ8)
-                                dequant_slot<kFmtQ8>(wslot, sslot, r, h, s, wv);
-                            else
-                                dequant_slot<kFmtE4M3>(wslot, sslot, r, h, s, wv);
-                            const int st = ja % kAStages;
-                            if (ja >= kAStages &&
-                                !mbar_wait(&a_empty[st], static_cast<uint32_t>((ja / kAStages) - 1) & 1u,
-                                           lim)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after_sync();
-                            tmem_st_x16(ta + static_cast<uint32_t>(st) * kAStageCols, wv);
-                            tmem_st_wait();
-                            tc_fence_before_sync();
-                            mbar_arrive(&a_full[st]);
-                        }
-                        if (!ok) break;
-                        // every read of the slot has been consumed by a store above
-                        mbar_arrive(&slot_empty[slot]);
+                        tc_fence_after_sync();
+                        tmem_st_x16(ta + static_cast<uint32_t>(st) * kAStageCols, wv);
+                        tmem_st_wait();
+                        tc_fence_before_sync();
+                        mbar_arrive(&a_full[st]);
                     }
+                    if (!ok) break;
+                    // every read of the slot has been consumed by a store above
+                    mbar_arrive(&slot_empty[slot]);
                 }
             }
         }
@@ -380,37 +375,36 @@ __global__ void __launch_bounds__(kPlThreads, 1)
         for (int i = i_first; i < i_last && ok; ++i) {
             const Item it = item_at(P, i);
             const PlProj &p = *it.p;
-            for (int c = 0; c < it.nchunks && ok; ++c) {
-                bool good = true;
-                const bool fresh = !(p.xid == cur_x && c == cur_c);
-                if (fresh) {
-                    cur_x = p.xid;
-                    cur_c = c;
-                    ++nx;
-                }
-                const int nw = slots_in_chunk(p, c);
-                for (int tt = 0; tt < it.ntiles && ok; ++tt) {
-                    const int n_acc = ntile + tt;                 // accumulator of this tile
-                    for (int w = 0; w < nw && ok; ++w) {
-                        int k0;
-                        const int nsteps = slot_len(p, c, w, k0) / 64;
-                        for (int s = 0; s < nsteps; ++s, ++ja) {
-                            if (lane == 0) {
-                                if (good && fresh && tt == 0 && w == 0 && s == 0)
-                                    good = mbar_wait(x_full, static_cast<uint32_t>(nx - 1) & 1u, lim);
-                                if (good && c == 0 && w == 0 && s == 0 && n_acc >= R)
-                                    good = mbar_wait(&acc_empty[n_acc % R],
-                                                     static_cast<uint32_t>((n_acc / R) - 1) & 1u, lim);
-                                if (good)
-                                    good = mbar_wait(&a_full[ja % kAStages],
-                                                     static_cast<uint32_t>(ja / kAStages) & 1u, lim);
-                                mma_abort[ja & 1] = good ? 0u : 1u;
-                            }
-                            named_bar_sync(kMmaBar, 64);
-                            if (__shfl_sync(0xffffffffu, good ? 1 : 0, 0) == 0) {
-                                ok = false;
-                                break;
-                            }
+            const int c = it.chunk;
+            bool good = true;
+            const bool fresh = !(p.xid == cur_x && c == cur_c);
+            if (fresh) {
+                cur_x = p.xid;
+                cur_c = c;
+                ++nx;
+            }
+            const int nw = slots_in_chunk(p, c);
+            for (int tt = 0; tt < it.ntiles && ok; ++tt) {
+                const int n_acc = ntile + tt;                 // accumulator of this tile
+                for (int w = 0; w < nw && ok; ++w) {
+                    int k0;
+                    const int nsteps = slot_len(p, c, w, k0) / 64;
+                    for (int s = 0; s < nsteps; ++s, ++ja) {
+                        if (lane == 0) {
+                            if (good && fresh && tt == 0 && w == 0 && s == 0)
+                                good = mbar_wait(x_full, static_cast<uint32_t>(nx - 1) & 1u, lim);
+                            if (good && w == 0 && s == 0 && n_acc >= R)
+                                good = mbar_wait(&acc_empty[n_acc % R],
+                                                 static_cast<uint32_t>((n_acc / R) - 1) & 1u, lim);
+                            if (good)
+                                good = mbar_wait(&a_full[ja % kAStages],
+                                                 static_cast<uint32_t>(ja / kAStages) & 1u, lim);
+                            mma_abort[ja & 1] = good ? 0u : 1u;
+                        }
+                        named_bar_sync(kMmaBar, 64);
+                        if (__shfl_sync(0xffffffffu, good ? 1 : 0, 0) == 0) {
+                            ok = false;
+                            break;
                         }
                     }
                 }
@@ -422,57 +416,47 @@ __global__ void __launch_bounds__(kPlThreads, 1)
         const uint32_t idesc = idesc_f16_f32acc(128, BNp);
         const uint64_t xdesc0 = sw128_kmajor_desc(base + L.x_off);
         const uint64_t atom_desc = static_cast<uint64_t>(BNp * 128) >> 4;
-        int cur_x = -1, cur_c = -1, ja = 0, ntile = 0;
+        int ja = 0, ntile = 0;
         bool abort = false;
         for (int i = i_first; i < i_last && !abort; ++i) {
             const Item it = item_at(P, i);
             const PlProj &p = *it.p;
-            for (int c = 0; c < it.nchunks && !abort; ++c) {
-                cur_x = p.xid;
-                cur_c = c;
-                const int nw = slots_in_chunk(p, c);
-                for (int tt = 0; tt < it.ntiles && !abort; ++tt) {
-                    const int n_acc = ntile + tt;
-                    const uint32_t d = tmem + static_cast<uint32_t>((n_acc % R) * BNp);
-                    for (int w = 0; w < nw && !abort; ++w) {
-                        int k0;
-                        const int nsteps = slot_len(p, c, w, k0) / 64;
-                        const int atom0 = (k0 - c * kXChunk) / 64;
-                        for (int s = 0; s < nsteps; ++s, ++ja) {
-                            named_bar_sync(kMmaBar, 64);
-                            if (mma_abort[ja & 1]) {
-                                abort = true;
-                                break;
-                            }
-                            if (lane == 0) {
-                                tc_fence_after_sync();
-                                const uint32_t a =
-                                    tmem + kAOff + static_cast<uint32_t>(ja % kAStages) * kAStageCols;
-                                const uint64_t bdesc = xdesc0 + static_cast<uint64_t>(atom0 + s) * atom_desc;
-                                const bool first = c == 0 && w == 0 && s == 0;
+            const int c = it.chunk;
+            const int nw = slots_in_chunk(p, c);
+            for (int tt = 0; tt < it.ntiles && !abort; ++tt) {
+                const int n_acc = ntile + tt;
+                const uint32_t d = tmem + static_cast<uint32_t>((n_acc % R) * BNp);
+                for (int w = 0; w < nw && !abort; ++w) {
+                    int k0;
+                    const int nsteps = slot_len(p, c, w, k0) / 64;
+                    const int atom0 = (k0 - c * kXChunk) / 64;
+                    for (int s = 0; s < nsteps; ++s, ++ja) {
+                        named_bar_sync(kMmaBar, 64);
+                        if (mma_abort[ja & 1]) {
+                            abort = true;
+                            break;
+                        }
+                        if (lane == 0) {
+                            tc_fence_after_sync();
+                            const uint32_t a =
+                                tmem + kAOff + static_cast<uint32_t>(ja % kAStages) * kAStageCols;
+                            const uint64_t bdesc = xdesc0 + static_cast<uint64_t>(atom0 + s) * atom_desc;
+                            const bool first = w == 0 && s == 0;
 #pragma unroll
-                                for (int kk = 0; kk < 4; ++kk)
-                                    tc_mma_f16kind_ts(d, a + 8 * kk, bdesc + 2 * kk, idesc,
-                                                      (first && kk == 0) ? 0u : 1u);
-                                tc_commit(&a_empty[ja % kAStages]);
-                            }
+                            for (int kk = 0; kk < 4; ++kk)
+                                tc_mma_f16kind_ts(d, a + 8 * kk, bdesc + 2 * kk, idesc,
+                                                  (first && kk == 0) ? 0u : 1u);
+                            tc_commit(&a_empty[ja % kAStages]);
                         }
                     }
-                    if (!abort && lane == 0 && c == it.nchunks - 1) tc_commit(&acc_full[n_acc % R]);
                 }
-                // release the activation chunk once its MMAs complete if the
-                // next item or chunk reads a different one
-                if (!abort && lane == 0) {
-                    int nxt_x = -1, nxt_c = -1;
-                    if (c + 1 < it.nchunks) {
-                        nxt_x = p.xid;
-                        nxt_c = c + 1;
-                    } else if (i + 1 < i_last) {
-                        nxt_x = P.proj[P.items[i + 1].proj].xid;
-                        nxt_c = 0;
-                    }
-                    if (nxt_x >= 0 && !(nxt_x == cur_x && nxt_c == cur_c)) tc_commit(x_empty);
-                }
+                if (!abort && lane == 0) tc_commit(&acc_full[n_acc % R]);
+            }
+            // release the activation chunk once its MMAs complete if the next
+            // item reads a different (activations, chunk)
+            if (!abort && lane == 0 && i + 1 < i_last) {
+                const PlItem &nx = P.items[i + 1];
+                if (!(P.proj[nx.proj].xid == p.xid && nx.chunk == c)) tc_commit(x_empty);
             }
             ntile += it.ntiles;
         }
@@ -486,42 +470,99 @@ __global__ void __launch_bounds__(kPlThreads, 1)
     } else {
         // ======================================================= epilogue
         pdl_wait_prior_grid();         // Y may be read or written by earlier kernels
+        const int et = threadIdx.x - kEpiWarp0 * 32;   // 0..255
         const int q = warp & 3;
         const int half = (warp - kEpiWarp0) >> 2;
         const int cols = BNp / 2;                      // a multiple of 8
         const int c0 = half * cols;
+        const int row = q * 32 + lane;                 // TMEM lane = weight row in the tile
         const uint32_t tq = tmem + (static_cast<uint32_t>(q * 32) << 16);
+        // Thread 0 of the epilogue waits for each accumulator and shares the
+        // outcome through named barrier kEpiBar, so the eight warps always
+        // take the same branch and meet at the same barriers.
+        volatile uint32_t *last_flag = tmem_slot + 3;
+        volatile uint32_t *full_flag = tmem_slot + 4;       // two, by tile parity
         int ntile = 0;
         for (int i = i_first; i < i_last && ok; ++i) {
             const Item it = item_at(P, i);
             const PlProj &p = *it.p;
+            const bool split = it.nchunks > 1;
             for (int tt = 0; tt < it.ntiles && ok; ++tt, ++ntile) {
                 const int slot = ntile % R;
-                ok = mbar_wait(&acc_full[slot], static_cast<uint32_t>(ntile / R) & 1u, lim);
-                ok = __all_sync(0xffffffffu, ok);
+                if (et == 0)
+                    full_flag[ntile & 1] =
+                        mbar_wait(&acc_full[slot], static_cast<uint32_t>(ntile / R) & 1u, lim) ? 1u
+                                                                                                : 0u;
+                named_bar_sync(kEpiBar, kEpiThreads);
+                ok = full_flag[ntile & 1] != 0;
                 if (!ok) break;
                 tc_fence_after_sync();
-                const int o = (it.tile0 + tt) * 128 + q * 32 + lane;
-                float sc = 1.f, b = 0.f;
-                if (p.fmt == 8 && o < p.N) sc = __ldg(static_cast<const float *>(p.S) + o);
-                if (p.bias && o < p.N) b = __ldg(p.bias + o);
+                const int tile = it.tile0 + tt;
+                const int o = tile * 128 + row;
                 const uint32_t tacc = tq + static_cast<uint32_t>(slot * BNp + c0);
-                float *yo = p.Y + o;
-                const size_t rs = static_cast<size_t>(p.N);
+                if (!split) {
+                    float sc = 1.f, b = 0.f;
+                    if (p.fmt == 8 && o < p.N) sc = __ldg(static_cast<const float *>(p.S) + o);
+                    if (p.bias && o < p.N) b = __ldg(p.bias + o);
+                    float *yo = p.Y + o;
+                    const size_t rs = static_cast<size_t>(p.N);
+                    for (int cc = 0; cc < cols; cc += 8) {
+                        uint32_t v[8];
+                        tmem_ld_x8(tacc + static_cast<uint32_t>(cc), v);
+                        tmem_ld_wait();
+                        if (o < p.N) {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                const int m = c0 + cc + e;
+                                if (m < M) yo[static_cast<size_t>(m) * rs] = fmaf(__uint_as_float(v[e]), sc, b);
+                            }
+                        }
+                    }
+                    tc_fence_before_sync();
+                    mbar_arrive(&acc_empty[slot]);
+                    continue;
+                }
+                // Split tile: this chunk's partial goes to its slot of the
+                // partials, column-major ([m][row]) so a warp writes 128
+                // contiguous bytes per column; the accumulator is free then.
+                const int st = p.sbase + tile;
+                float *part = P.partials +
+                              static_cast<size_t>(st * P.max_chunks + it.chunk) * BNp * 128;
                 for (int cc = 0; cc < cols; cc += 8) {
                     uint32_t v[8];
                     tmem_ld_x8(tacc + static_cast<uint32_t>(cc), v);
                     tmem_ld_wait();
-                    if (o < p.N) {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int m = c0 + cc + e;
-                            if (m < M) yo[static_cast<size_t>(m) * rs] = fmaf(__uint_as_float(v[e]), sc, b);
-                        }
-                    }
+                    for (int e = 0; e < 8; ++e)
+                        __stcg(part + static_cast<size_t>(c0 + cc + e) * 128 + row, __uint_as_float(v[e]));
                 }
                 tc_fence_before_sync();
                 mbar_arrive(&acc_empty[slot]);
+                // The last chunk to finish sums the partials in chunk order
+                // (the same order whichever CTA it is) and writes Y.
+                __threadfence();
+                named_bar_sync(kEpiBar, kEpiThreads);
+                if (et == 0) {
+                    const unsigned done = atomicAdd(P.counters + st, 1u);
+                    *last_flag = (done == static_cast<unsigned>(it.nchunks - 1)) ? 1u : 0u;
+                }
+                named_bar_sync(kEpiBar, kEpiThreads);
+                if (*last_flag) {
+                    __threadfence();
+                    if (o < p.N) {
+                        const float sc = p.fmt == 8 ? __ldg(static_cast<const float *>(p.S) + o) : 1.f;
+                        const float b = p.bias ? __ldg(p.bias + o) : 0.f;
+                        const float *p0 = P.partials + static_cast<size_t>(st * P.max_chunks) * BNp * 128;
+                        for (int m = c0; m < c0 + cols && m < M; ++m) {
+                            float acc = __ldcg(p0 + static_cast<size_t>(m) * 128 + row);
+                            for (int ch = 1; ch < it.nchunks; ++ch)
+                                acc += __ldcg(p0 + (static_cast<size_t>(ch) * BNp + m) * 128 + row);
+                            p.Y[static_cast<size_t>(m) * p.N + o] = fmaf(acc, sc, b);
+                        }
+                    }
+                    if (et == 0) P.counters[st] = 0u;      // ready for the next launch
+                }
+                named_bar_sync(kEpiBar, kEpiThreads);      // last_flag is read by all
             }
         }
     }
@@ -544,6 +585,8 @@ __global__ void __launch_bounds__(kPlThreads, 1)
 __global__ void __launch_bounds__(256)
     pl_prep_kernel(const __grid_constant__ PlPrep P, DevCtl *ctl) {
     pdl_wait_prior_grid();
+    if (blockIdx.x == 0 && blockIdx.y == 0)
+        for (int i = threadIdx.x; i < P.n_counters; i += blockDim.x) P.counters[i] = 0u;
     const PlPrepImage &im = P.img[blockIdx.y];
     const int BNp = P.bnp, M = P.M, K = im.K;
     const int64_t pieces = static_cast<int64_t>(K / 8) * BNp;   // 16-byte output pieces
@@ -627,39 +670,66 @@ namespace {
 
 int64_t pl_image_bytes(int M, int K) { return static_cast<int64_t>(pl_bnp(M)) * K * 2; }
 
-// Distinct activation images of a list: (X, K) -> image index, in order of
-// first appearance, with each image's offset in the workspace.
-struct Images {
+// Workspace of a list call: the distinct activation images ((X, K) -> image
+// index, in order of first appearance), then the partial tiles and counters
+// of the projections with K > 512 ("split" tiles, one partial per 512-wide K
+// chunk).
+struct Plan {
     std::vector<int> xid;            // per projection
+    std::vector<int> sbase;          // per projection: first split-tile index, or -1
     std::vector<const float *> X;    // per image
     std::vector<int> K;
     std::vector<size_t> off;
-    size_t bytes = 0;
+    int n_split = 0, max_chunks = 1;
+    size_t partials_off = 0, counters_off = 0, bytes = 0;
 };
 
-Images distinct_images(const PlInput *in, int count, int M) {
-    Images im;
-    im.xid.resize(count);
+constexpr size_t align256(size_t b) { return (b + 255) / 256 * 256; }
+
+Plan plan_list(const PlInput *in, int count, int M) {
+    Plan pl;
+    pl.xid.resize(count);
+    pl.sbase.assign(count, -1);
+    size_t img = 0;
     for (int i = 0; i < count; ++i) {
         int found = -1;
-        for (size_t j = 0; j < im.X.size(); ++j)
-            if (im.X[j] == in[i].X && im.K[j] == in[i].K) found = static_cast<int>(j);
+        for (size_t j = 0; j < pl.X.size(); ++j)
+            if (pl.X[j] == in[i].X && pl.K[j] == in[i].K) found = static_cast<int>(j);
         if (found < 0) {
-            found = static_cast<int>(im.X.size());
-            im.X.push_back(in[i].X);
-            im.K.push_back(in[i].K);
-            im.off.push_back(im.bytes);
-            im.bytes += (pl_image_bytes(M, in[i].K) + 255) / 256 * 256;
+            found = static_cast<int>(pl.X.size());
+            pl.X.push_back(in[i].X);
+            pl.K.push_back(in[i].K);
+            pl.off.push_back(img);
+            img += align256(static_cast<size_t>(pl_image_bytes(M, in[i].K)));
         }
-        im.xid[i] = found;
+        pl.xid[i] = found;
+        const int nchunks = (in[i].K + kXChunk - 1) / kXChunk;
+        if (nchunks > 1) {
+            pl.sbase[i] = pl.n_split;
+            pl.n_split += (in[i].N + 127) / 128;
+            pl.max_chunks = std::max(pl.max_chunks, nchunks);
+        }
     }
-    return im;
+    pl.partials_off = img;
+    const size_t part = static_cast<size_t>(pl.n_split) * pl.max_chunks * pl_bnp(M) * 128 * 4;
+    pl.counters_off = align256(pl.partials_off + part);
+    pl.bytes = align256(pl.counters_off + static_cast<size_t>(pl.n_split) * 4);
+    return pl;
+}
+
+// Tiles per work item: up to about 160 KB of packed weights (four q4 tiles
+// of a 512-wide chunk, two q8 or e4m3 tiles), so that the items assigned to
+// one CTA can be balanced closely.
+int tiles_per_item(const PlInput &q) {
+    const int klen = std::min(q.K, kXChunk);
+    const double tile = 128.0 * klen * (q.fmt == 4 ? 0.625 : 1.0);
+    return std::max(1, std::min(4, static_cast<int>(160.0 * 1024 / tile)));
 }
 
 }  // namespace
 
 size_t pl_workspace_bytes(const PlInput *in, int count, int M) {
-    return distinct_images(in, count, M).bytes;
+    return plan_list(in, count, M).bytes;
 }
 
 cudaError_t launch_pl_batch(const PlInput *in, int count, int M, void *ws, DevCtl *ctl,
@@ -671,19 +741,23 @@ cudaError_t launch_pl_batch(const PlInput *in, int count, int M, void *ws, DevCt
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     sms = std::min(sms, kPlMaxCtas);
     const int bnp = pl_bnp(M), nacc = pl_nacc(bnp), nslots = pl_nslots(bnp);
-    const Images im = distinct_images(in, count, M);
+    const Plan pl = plan_list(in, count, M);
     uint8_t *wsb = static_cast<uint8_t *>(ws);
+    unsigned *counters = reinterpret_cast<unsigned *>(wsb + pl.counters_off);
 
-    // 1. every distinct activation block once into its fp16 image
-    for (size_t i0 = 0; i0 < im.X.size(); i0 += kPlMaxProj) {
+    // 1. every distinct activation block once into its fp16 image; the first
+    // pre-pass launch also zeroes the split tiles' counters
+    for (size_t i0 = 0; i0 < pl.X.size(); i0 += kPlMaxProj) {
         thread_local PlPrep prep;   // large: kept off the stack; a launch copies it
         prep.M = M;
         prep.bnp = bnp;
-        const int n = static_cast<int>(std::min<size_t>(kPlMaxProj, im.X.size() - i0));
+        prep.counters = counters;
+        prep.n_counters = i0 == 0 ? pl.n_split : 0;
+        const int n = static_cast<int>(std::min<size_t>(kPlMaxProj, pl.X.size() - i0));
         int max_k = 0;
         for (int j = 0; j < n; ++j) {
-            prep.img[j] = {im.X[i0 + j], wsb + im.off[i0 + j], im.K[i0 + j], 0};
-            max_k = std::max(max_k, im.K[i0 + j]);
+            prep.img[j] = {pl.X[i0 + j], wsb + pl.off[i0 + j], pl.K[i0 + j], 0};
+            max_k = std::max(max_k, pl.K[i0 + j]);
         }
         if ((e = launch_pl_prep(prep, n, max_k, ctl, s)) != cudaSuccess) return e;
     }
@@ -693,7 +767,7 @@ cudaError_t launch_pl_batch(const PlInput *in, int count, int M, void *ws, DevCt
     std::vector<int> order(count);
     std::iota(order.begin(), order.end(), 0);
     std::stable_sort(order.begin(), order.end(),
-                     [&](int a, int b) { return im.xid[a] < im.xid[b]; });
+                     [&](int a, int b) { return pl.xid[a] < pl.xid[b]; });
     thread_local PlParams P;     // large: kept off the stack; a launch copies it
     size_t pos = 0;
     while (pos < order.size()) {
@@ -701,19 +775,24 @@ cudaError_t launch_pl_batch(const PlInput *in, int count, int M, void *ws, DevCt
         std::vector<double> cost;
         int np = 0;
         for (; pos < order.size() && np < kPlMaxProj; ++np, ++pos) {
-            const PlInput &q = in[order[pos]];
+            const int src = order[pos];
+            const PlInput &q = in[src];
             const int tiles = (q.N + 127) / 128;
-            const int per = q.K > kXChunk ? nacc : 4;    // tiles per item
-            const int n_items = (tiles + per - 1) / per;
+            const int nchunks = (q.K + kXChunk - 1) / kXChunk;
+            const int per = tiles_per_item(q);
+            const int n_items = nchunks * ((tiles + per - 1) / per);
             if (np > 0 && items.size() + n_items > static_cast<size_t>(kPlMaxItems)) break;
-            P.proj[np] = {wsb + im.off[im.xid[order[pos]]], q.Wq, q.S, q.bias, q.Y, q.N, q.K,
-                          q.fmt, im.xid[order[pos]]};
-            for (int t = 0; t < tiles; t += per) {
-                const int nt = std::min(per, tiles - t);
-                items.push_back({static_cast<uint32_t>(t), static_cast<uint16_t>(np),
-                                 static_cast<uint16_t>(nt)});
-                const int rows = std::min(nt * 128, q.N - t * 128);
-                cost.push_back(static_cast<double>(rows) * q.K * (q.fmt == 4 ? 0.625 : 1.0));
+            P.proj[np] = {wsb + pl.off[pl.xid[src]], q.Wq, q.S, q.bias, q.Y, q.N, q.K, q.fmt,
+                          pl.xid[src], pl.sbase[src]};
+            for (int c = 0; c < nchunks; ++c) {
+                const int klen = std::min(kXChunk, q.K - c * kXChunk);
+                for (int t = 0; t < tiles; t += per) {
+                    const int nt = std::min(per, tiles - t);
+                    items.push_back({static_cast<uint32_t>(t), static_cast<uint16_t>(np),
+                                     static_cast<uint8_t>(nt), static_cast<uint8_t>(c)});
+                    const int rows = std::min(nt * 128, q.N - t * 128);
+                    cost.push_back(static_cast<double>(rows) * klen * (q.fmt == 4 ? 0.625 : 1.0));
+                }
             }
         }
         // largest item first onto the least loaded CTA
@@ -730,13 +809,14 @@ cudaError_t launch_pl_batch(const PlInput *in, int count, int M, void *ws, DevCt
             load[b] += cost[it];
             mine[b].push_back(it);
         }
-        // within a CTA: items of one activation image together, in list order
+        // within a CTA: items of one activation chunk together, in list order
         int k = 0;
         for (int b = 0; b < G; ++b) {
             std::sort(mine[b].begin(), mine[b].end(), [&](int a, int c) {
                 const PlItem &x = items[a], &y = items[c];
                 if (P.proj[x.proj].xid != P.proj[y.proj].xid)
                     return P.proj[x.proj].xid < P.proj[y.proj].xid;
+                if (x.chunk != y.chunk) return x.chunk < y.chunk;
                 if (x.proj != y.proj) return x.proj < y.proj;
                 return x.tile0 < y.tile0;
             });
@@ -748,6 +828,10 @@ cudaError_t launch_pl_batch(const PlInput *in, int count, int M, void *ws, DevCt
         P.bnp = bnp;
         P.nslots = nslots;
         P.nacc = nacc;
+        P.partials = reinterpret_cast<float *>(wsb + pl.partials_off);
+        P.counters = counters;
+        P.max_chunks = pl.max_chunks;
+        P.pad = 0;
         if ((e = launch_pl(P, G, ctl, s)) != cudaSuccess) return e;
     }
     return cudaSuccess;
