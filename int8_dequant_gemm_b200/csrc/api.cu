@@ -453,8 +453,9 @@ int batch_route(const rt_qproj *list, int count, int64_t M, int path) {
         const int p = pick_path(M, q.K, path);
         if (p == -1) return -RT_ERR_UNSUPPORTED_SHAPE;
         tc_all = tc_all && p == RT_PATH_TC;
-        // the list kernel copies q4 (scale, min) rows in 16-byte pieces
-        list_ok = list_ok && rtq::pl_supported(q.fmt, static_cast<int>(M), static_cast<int>(q.K)) &&
+        // the list kernel reads q4 (scale, min) rows through a TMA map: 16-byte base
+        list_ok = list_ok &&
+                  rtq::pl_supported(q.fmt, static_cast<int>(M), q.N, static_cast<int>(q.K)) &&
                   (q.fmt != 4 || aligned(q.scales, 16));
         tiles += (q.N + 127) / 128;
     }

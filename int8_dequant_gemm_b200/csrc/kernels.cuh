@@ -114,7 +114,7 @@ struct PlInput {
     float *Y;
     int N, K;
 };
-bool pl_supported(int fmt, int M, int K);
+bool pl_supported(int fmt, int M, int64_t N, int K);
 size_t pl_workspace_bytes(const PlInput *in, int count, int M);
 cudaError_t launch_pl_batch(const PlInput *in, int count, int M, void *ws, DevCtl *ctl,
                             cudaStream_t s);

@@ -18,36 +18,49 @@
 // N dimension; fp16 operands, fp32 accumulation in TMEM.
 //
 // Data movement per CTA:
-//   weights  cp.async (16 bytes per thread) of one slot = 128 rows x 256
-//            bytes of codes (q4: K 512, q8: K 256) plus, for q4, the rows'
-//            (scale, min) words, into a ring of slots in an XOR-swizzled
-//            layout: 16-byte chunk c of row r sits at chunk (c & 8) |
-//            ((c & 7) ^ (r & 7)), so the dequantizers' reads of one chunk
-//            over 8 consecutive rows hit 8 different bank groups.  The slot
-//            completes on an mbarrier through cp.async.mbarrier.arrive.
+//   weights  TMA: one slot = 128 rows x 256 bytes of codes (q4: K 512, q8:
+//            K 256) as two boxes of 128 rows x 128 bytes from the
+//            projection's [N, row bytes] tensor map, plus, for q4, one box of
+//            the rows' 16 (scale, min) words.  The codes land 128-byte
+//            swizzled (16-byte chunk c of row r at chunk c ^ (r & 7)), the
+//            words 64-byte swizzled (chunk c at c ^ ((r >> 1) & 3)), so the
+//            dequantizers' reads of one chunk over 8 consecutive rows hit 8
+//            different bank groups.  The tensor maps travel in the kernel's
+//            parameters, encoded on the host once per weight and thread.
+//            (A slot issued as 16-byte cp.async copies instead costs one
+//            instruction per 16 bytes on the SM's load/store path and paced
+//            the whole pipeline; a TMA box costs one.)
 //   activations  one bulk copy per 512-wide K chunk of the projection's fp16
 //            image (written by pl_prep_kernel below in the 128-byte-swizzled
 //            operand layout) into the resident activation buffer, reloaded
 //            only when the (activations, K chunk) pair changes.
-// Roles (21 warps):
-//   warps 0-7   dequantizers: thread (r, h) converts K values [32h, 32h+32) of
-//               every 64-wide K step of row r into TMEM lane r of the step's A
-//               stage (tcgen05.st), as in the activation-resident kernel.
+// A stages: the MMAs read the dequantized weights from TMEM, one stage = two
+// 64-wide K steps (64 columns) in a ring of four at columns [256, 512).
+// Within every 8 consecutive K values the operands are paired (t, t + 4),
+// t = 0..3, in both A and the activation image: that order lets the q4
+// dequantizer take the 8 nibbles of a 32-bit word apart with one shift and
+// four masks (two nibbles per mask, turned into fp16 by an exponent pattern
+// in the same operation), where the natural pairing needs byte permutes too.
+// Roles (20 warps):
+//   warps 0-7   dequantizers: thread (r, h) converts step h of each stage of
+//               row r (64 K values) into TMEM lane r of the stage: it loads
+//               all its bytes of a weight slot into registers at once,
+//               releases the slot, then converts and stores stage by stage.
 //   warp 8      MMA issuer, fed through named barrier 1 by
 //   warp 9      the MMA waiter, which performs all of the issuer's waits.
 //   warps 10-17 epilogue: TMEM -> registers (q8 row scale) -> fp32 Y.
-//   warps 18-19 weight producers (cp.async).
-//   warp 20     activation loader (one thread, bulk copies).
+//   warp 18     weight producer (one thread, TMA).
+//   warp 19     activation loader (one thread, bulk copies).
 // Work items longer than one 512-wide K chunk (K > 512) run chunk by chunk
 // over all their tiles (each tile in its own accumulator), so one resident
 // activation chunk serves every tile of the item.
 //
-// Work distribution (host, launch_pl): items are cut from the projections
-// (at most 4 tiles, or as many as the accumulator ring holds when K > 512),
-// assigned largest first to the least loaded CTA, and each CTA's items are
-// ordered by their activation buffer so that the resident block is reloaded
-// as rarely as possible.  Every tile is computed by one CTA from start to
-// end, so results do not depend on the assignment.
+// Work distribution (host, launch_pl_batch): items (one 512-wide K chunk of
+// up to four tiles, about 80 KB of packed weights) are sorted by (activation
+// image, K chunk) and the sorted sequence is cut into one contiguous run per
+// CTA with about equal bytes, so a CTA switches its resident activation
+// chunk at most once or twice.  Every tile chunk is computed by one CTA from
+// start to end, so results do not depend on the assignment.
 //
 // Every mbarrier wait is bounded; a wait that gives up latches
 // RT_ERR_DEVICE_TIMEOUT and the CTA winds down: copies it issued complete,
@@ -68,20 +81,19 @@ constexpr int kIssuerWarp = 8;
 constexpr int kWaiterWarp = 9;
 constexpr int kEpiWarp0 = 10;
 constexpr int kEpiWarps = 8;
-constexpr int kProdWarp0 = 18;
-constexpr int kProdWarps = 2;
-constexpr int kXWarp = 20;
-constexpr int kPlThreads = (kXWarp + 1) * 32;        // 672
-constexpr int kProdThreads = kProdWarps * 32;        // 64
+constexpr int kProdWarp = 18;
+constexpr int kXWarp = 19;
+constexpr int kPlThreads = (kXWarp + 1) * 32;        // 640
 constexpr int kEpiThreads = kEpiWarps * 32;          // 256
 constexpr uint32_t kMmaBar = 1;                      // named barrier: waiter <-> issuer
 constexpr uint32_t kEpiBar = 2;                      // named barrier: the epilogue warps
 constexpr int kSlotBytes = 32 * 1024;                // 128 rows x 256 bytes of codes
+constexpr int kBoxBytes = 16 * 1024;                 // one TMA box: 128 rows x 128 bytes
 constexpr int kScaleBytes = 8 * 1024;                // 128 rows x 16 (scale, min) words
 constexpr int kMaxSlots = 4;
 constexpr int kAStages = 4;
-constexpr uint32_t kAStageCols = 32;
-constexpr uint32_t kAOff = 384;                      // A stages at TMEM columns [384, 512)
+constexpr uint32_t kAStageCols = 64;                 // two 64-wide K steps
+constexpr uint32_t kAOff = 256;                      // A stages at TMEM columns [256, 512)
 constexpr int kXChunk = 512;                         // K of one resident activation chunk
 
 // K covered by one weight slot (256 bytes of codes per row).
@@ -103,19 +115,8 @@ __host__ __device__ inline PlLayout pl_layout(int bnp, int nslots) {
     return L;
 }
 
-__device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-
-// Arrives on `bar` once every cp.async this thread issued so far has landed
-// (the barrier's expected count includes this arrival).
-__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar))
-                 : "memory");
-}
-
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.wait_all;" ::: "memory");
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
@@ -127,27 +128,35 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
         : "memory");
 }
 
-// Physical 16-byte chunk of logical chunk c (0..15) of slot row r.
-__device__ __forceinline__ int wswz(int c, int r) { return (c & 8) | ((c & 7) ^ (r & 7)); }
+// Shared address of 16-byte chunk c (0..15) of row r of a weight slot: box
+// c / 8, 128-byte swizzle within it.
+__device__ __forceinline__ uint32_t wchunk(uint32_t slot, int c, int r) {
+    return slot + (static_cast<uint32_t>(c >> 3) << 14) + static_cast<uint32_t>(r * 128) +
+           (static_cast<uint32_t>((c & 7) ^ (r & 7)) << 4);
+}
 // Physical 16-byte chunk of logical scale chunk c (0..3) of row r.
 __device__ __forceinline__ int sswz(int c, int r) { return c ^ ((r >> 1) & 3); }
 
 // The walk every role takes through a CTA's items: item (one K chunk of a
 // few tiles) -> tile -> weight slot -> 64-wide K step.  Each role advances it
-// at its own grain.
+// at its own grain.  The projection's fields are copied into registers once
+// per item: read through a pointer into the parameter space they would be
+// loaded again after every asm statement that clobbers memory (the barrier
+// waits and arrivals), a few hundred cycles each.
 struct Item {
-    const PlProj *p;
-    int tile0, ntiles, chunk, nchunks;
+    PlProj p;
+    int proj, tile0, ntiles, chunk, nchunks;
 };
 
 __device__ __forceinline__ Item item_at(const PlParams &P, int i) {
-    const PlItem &it = P.items[i];
+    const PlItem it = P.items[i];
     Item r;
-    r.p = &P.proj[it.proj];
+    r.p = P.proj[it.proj];
+    r.proj = it.proj;
     r.tile0 = static_cast<int>(it.tile0);
     r.ntiles = it.ntiles;
     r.chunk = it.chunk;
-    r.nchunks = (r.p->K + kXChunk - 1) / kXChunk;
+    r.nchunks = (r.p.K + kXChunk - 1) / kXChunk;
     return r;
 }
 
@@ -162,24 +171,134 @@ __device__ __forceinline__ int slots_in_chunk(const PlProj &p, int c) {
     return (len + slot_k(p.fmt) - 1) / slot_k(p.fmt);
 }
 
+// ------------------------------------------------------------ dequantization
+// Operand pairs (K 8j + t, 8j + t + 4), t = 0..3, of one 8-value chunk j.
+
+// q4: the 8 codes of word v (code i in bits 4i..4i+3) -> 4 fp16 pair words
+// (scale, min applied: w = q * scale + min, one rounding).  A nibble in bits
+// 0-3 of a 16-bit half under exponent pattern 0x6400 is fp16 1024 + q; in
+// bits 4-7 under 0x5400 it is 64 + q (ulp 1/16); both subtractions are exact.
+__device__ __forceinline__ void q4_pairs(uint32_t v, __half2 s, __half2 m, uint32_t *out) {
+    const __half2 k1024 = bits_h2(0x64006400u), k64 = bits_h2(0x54005400u);
+    const uint32_t v8 = v >> 8;
+    out[0] = h2_bits(__hfma2(__hsub2(bits_h2((v & 0x000F000Fu) | 0x64006400u), k1024), s, m));
+    out[1] = h2_bits(__hfma2(__hsub2(bits_h2((v & 0x00F000F0u) | 0x54005400u), k64), s, m));
+    out[2] = h2_bits(__hfma2(__hsub2(bits_h2((v8 & 0x000F000Fu) | 0x64006400u), k1024), s, m));
+    out[3] = h2_bits(__hfma2(__hsub2(bits_h2((v8 & 0x00F000F0u) | 0x54005400u), k64), s, m));
+}
+
+// Byte t of a and byte t of b in the low bytes of the two 16-bit halves.
+__device__ __forceinline__ uint32_t pair_bytes(uint32_t a, uint32_t b, int t) {
+    return __byte_perm(a, b, static_cast<uint32_t>(t | (t << 4) | ((4 + t) << 8) | ((4 + t) << 12)));
+}
+
+// q8: codes 8j..8j+3 in a, 8j+4..8j+7 in b -> 4 fp16 pair words of the
+// integers (the row scale is applied in the epilogue).  The offset-binary
+// byte q + 128 under 0x64 is fp16 1024 + q + 128; subtracting 1152 is exact.
+__device__ __forceinline__ void q8_pairs(uint32_t a, uint32_t b, uint32_t *out) {
+    const __half2 k1152 = bits_h2(0x64806480u);
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+        out[t] = h2_bits(__hsub2(bits_h2((pair_bytes(a, b, t) & 0x00FF00FFu) ^ 0x64806480u), k1152));
+}
+
+__device__ __forceinline__ void e4m3_pairs(uint32_t a, uint32_t b, uint32_t *out) {
+#pragma unroll
+    for (int t = 0; t < 4; ++t) out[t] = e4m3_pair_f16(pair_bytes(a, b, t));
+}
+
+// Half h of 32 K values (h = 0: K 0..31 of the step, 1: K 32..63) of one
+// thread's step -> 16 operand words.  q4: r0 = the 16 bytes of codes, sw =
+// the group's (scale, min) word; q8 / e4m3: r0, r1 = the 32 bytes of codes.
 template <int FMT>
-__device__ __forceinline__ void dequant_slot(uint32_t wslot, uint32_t sslot, int r, int h, int s,
-                                             uint32_t (&w)[16]) {
-    HalfRaw R;
-    if (FMT == 4) {
-        R.p0 = lds_v4(wslot + r * 256 + wswz(2 * s + h, r) * 16);
-        R.p1 = make_uint4(0, 0, 0, 0);
-        // (scale, min) word 2s + h of the row: chunk s >> 1, word (2s + h) & 3
-        const uint4 sc = lds_v4(sslot + r * 64 + sswz(s >> 1, r) * 16);
-        const int wi = (2 * s + h) & 3;
-        R.smw = wi == 0 ? sc.x : wi == 1 ? sc.y : wi == 2 ? sc.z : sc.w;
-        half_words<4>(R, w);
-    } else {   // q8 and e4m3: one byte per weight
-        R.p0 = lds_v4(wslot + r * 256 + wswz(4 * s + 2 * h, r) * 16);
-        R.p1 = lds_v4(wslot + r * 256 + wswz(4 * s + 2 * h + 1, r) * 16);
-        R.smw = 0;
-        half_words<FMT>(R, w);
+__device__ __forceinline__ void convert_half(uint4 r0, uint4 r1, uint32_t sw, uint32_t (&w)[16]) {
+    if (FMT == kFmtQ4) {
+        const __half2 s = bits_h2(__byte_perm(sw, 0u, 0x1010)), m = bits_h2(__byte_perm(sw, 0u, 0x3232));
+        q4_pairs(r0.x, s, m, w + 0);
+        q4_pairs(r0.y, s, m, w + 4);
+        q4_pairs(r0.z, s, m, w + 8);
+        q4_pairs(r0.w, s, m, w + 12);
+    } else if (FMT == kFmtQ8) {
+        q8_pairs(r0.x, r0.y, w + 0);
+        q8_pairs(r0.z, r0.w, w + 4);
+        q8_pairs(r1.x, r1.y, w + 8);
+        q8_pairs(r1.z, r1.w, w + 12);
+    } else {
+        e4m3_pairs(r0.x, r0.y, w + 0);
+        e4m3_pairs(r0.z, r0.w, w + 4);
+        e4m3_pairs(r1.x, r1.y, w + 8);
+        e4m3_pairs(r1.z, r1.w, w + 12);
     }
+}
+
+// Up to kRound stages of one weight slot for thread (r, h) (two for q4, one
+// for the one-byte formats, whose steps hold twice the bytes): its steps
+// s = s0 + 2i + h below nsteps.  Their bytes are loaded first (the slot is
+// released after the slot's last loads); then, per stage, the thread waits
+// for the stage to be free, converts its step and stores it (32 columns at
+// offset 32h), and every thread arrives.  Returns false if a wait ran out.
+template <int FMT>
+__device__ __forceinline__ bool dequant_pair(uint32_t wslot, uint32_t sslot, int r, int h, int s0,
+                                             int nsteps, uint32_t ta, int &ja, uint64_t *slot_empty,
+                                             uint64_t *a_full, uint64_t *a_empty,
+                                             const unsigned long long *lim) {
+    constexpr int kRaw = FMT == kFmtQ4 ? 2 : 4;     // 16-byte pieces per step
+    constexpr int kRound = FMT == kFmtQ4 ? 2 : 1;   // stages per round
+    uint4 raw[kRound][kRaw];
+    uint2 sc[kRound];
+#pragma unroll
+    for (int i = 0; i < kRound; ++i) {
+        const int s = s0 + 2 * i + h;
+        if (s < nsteps) {
+#pragma unroll
+            for (int q = 0; q < kRaw; ++q) raw[i][q] = lds_v4(wchunk(wslot, kRaw * s + q, r));
+            // q4: groups 2s, 2s + 1 = words 4 (s >> 1) + 2h, + 1 of the row
+            if (FMT == kFmtQ4) sc[i] = lds_v2(sslot + r * 64 + sswz(s >> 1, r) * 16 + 8 * h);
+        }
+    }
+    if (s0 + 2 * kRound >= nsteps) mbar_arrive(slot_empty);   // every read of the slot has returned
+#pragma unroll
+    for (int i = 0; i < kRound; ++i) {
+        const int s = s0 + 2 * i + h;
+        if (s0 + 2 * i >= nsteps) break;
+        const int st = ja % kAStages;
+        if (ja >= kAStages &&
+            !mbar_wait(&a_empty[st], static_cast<uint32_t>((ja / kAStages) - 1) & 1u, lim))
+            return false;
+        tc_fence_after_sync();
+        if (s < nsteps) {
+            const uint32_t t = ta + static_cast<uint32_t>(st) * kAStageCols;
+            uint32_t w[16];
+            if (FMT == kFmtQ4) {
+                convert_half<FMT>(raw[i][0], raw[i][0], sc[i].x, w);
+                tmem_st_x16(t, w);
+                convert_half<FMT>(raw[i][1], raw[i][1], sc[i].y, w);
+                tmem_st_x16(t + 16, w);
+            } else {
+                convert_half<FMT>(raw[i][0], raw[i][1], 0u, w);
+                tmem_st_x16(t, w);
+                convert_half<FMT>(raw[i][2], raw[i][3], 0u, w);
+                tmem_st_x16(t + 16, w);
+            }
+            tmem_st_wait();
+        }
+        tc_fence_before_sync();
+        mbar_arrive(&a_full[st]);
+        ++ja;
+    }
+    return true;
+}
+
+// A whole weight slot (nsteps 64-wide steps) for thread (r, h).
+template <int FMT>
+__device__ __forceinline__ bool dequant_slot(uint32_t wslot, uint32_t sslot, int r, int h, int nsteps,
+                                             uint32_t ta, int &ja, uint64_t *slot_empty,
+                                             uint64_t *a_full, uint64_t *a_empty,
+                                             const unsigned long long *lim) {
+    for (int s0 = 0; s0 < nsteps; s0 += FMT == kFmtQ4 ? 4 : 2)
+        if (!dequant_pair<FMT>(wslot, sslot, r, h, s0, nsteps, ta, ja, slot_empty, a_full, a_empty, lim))
+            return false;
+    return true;
 }
 
 __global__ void __launch_bounds__(kPlThreads, 1)
@@ -209,7 +328,7 @@ __global__ void __launch_bounds__(kPlThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kMaxSlots; ++s) {
-            mbar_init(&slot_full[s], kProdThreads);
+            mbar_init(&slot_full[s], 1);
             mbar_init(&slot_empty[s], kDeqWarps * 32);
         }
         for (int s = 0; s < kAStages; ++s) {
@@ -237,60 +356,65 @@ __global__ void __launch_bounds__(kPlThreads, 1)
     pdl_launch_dependents();
     bool ok = true;
 
-    if (warp >= kProdWarp0 && warp < kProdWarp0 + kProdWarps) {
-        // ======================================================= weight producers
+    if (warp == kProdWarp) {
+        // ======================================================= weight producer
         // Packed weights do not depend on the previous kernel in the stream.
-        // (Test hook: with `inject`, thread 0 leaves out its arrival on the
-        // first slot, so the dequantizers' wait for it runs out.)
-        const int t = threadIdx.x - kProdWarp0 * 32;
-        int j = 0;
-        for (int i = i_first; i < i_last && ok; ++i) {
-            const Item it = item_at(P, i);
-            const PlProj &p = *it.p;
-            const int fmt = p.fmt, c = it.chunk;
-            const size_t row_stride = fmt == 4 ? static_cast<size_t>(p.K / 2) : static_cast<size_t>(p.K);
-            const int nw = slots_in_chunk(p, c);
-            for (int tt = 0; tt < it.ntiles && ok; ++tt) {
-                const int o0 = (it.tile0 + tt) * 128;
-                const int rows = min(128, p.N - o0);
-                for (int w = 0; w < nw; ++w, ++j) {
-                    const int slot = j % NS;
-                    if (j >= NS &&
-                        !mbar_wait(&slot_empty[slot], static_cast<uint32_t>((j / NS) - 1) & 1u, lim)) {
-                        ok = false;
-                        break;
-                    }
-                    int k0;
-                    const int klen = slot_len(p, c, w, k0);
-                    const int row_chunks = (fmt == 4 ? klen / 2 : klen) / 16;
-                    const uint8_t *src = static_cast<const uint8_t *>(p.Wq) +
-                                         static_cast<size_t>(o0) * row_stride + (fmt == 4 ? k0 / 2 : k0);
-                    const uint32_t dst = base + L.w_off + slot * kSlotBytes;
-                    for (int e = t; e < 128 * 16; e += kProdThreads) {
-                        const int r = e >> 4, ch = e & 15;
-                        if (r < rows && ch < row_chunks)
-                            cp_async_16(dst + r * 256 + wswz(ch, r) * 16,
-                                        src + static_cast<size_t>(r) * row_stride + ch * 16);
-                    }
-                    if (fmt == 4) {
-                        // (scale, min) words of the slot's groups: klen / 32
-                        // words per row, 16-byte chunks of 4 words
-                        const int schunks = klen / 128;
-                        const uint8_t *ssrc = static_cast<const uint8_t *>(p.S) +
-                                              static_cast<size_t>(o0) * (p.K / 32) * 4 + (k0 / 32) * 4;
-                        const uint32_t sdst = base + L.s_off + slot * kScaleBytes;
-                        for (int e = t; e < 128 * 4; e += kProdThreads) {
-                            const int r = e >> 2, ch = e & 3;
-                            if (r < rows && ch < schunks)
-                                cp_async_16(sdst + r * 64 + sswz(ch, r) * 16,
-                                            ssrc + static_cast<size_t>(r) * (p.K / 32) * 4 + ch * 16);
+        // (Test hook: with `inject`, the first slot is never loaded, so the
+        // dequantizers' wait for it runs out.)
+        if (lane == 0) {
+            for (int i = i_first, last = -1; i < i_last; ++i) {
+                const int pj = P.items[i].proj;
+                if (pj == last) continue;
+                last = pj;
+                prefetch_tensormap(&P.wmap[pj]);
+                if (P.proj[pj].fmt == kFmtQ4) prefetch_tensormap(&P.smap[pj]);
+            }
+            int j = 0;
+            bool skipped0 = false;
+            for (int i = i_first; i < i_last && ok; ++i) {
+                const Item it = item_at(P, i);
+                const PlProj &p = it.p;
+                const CUtensorMap *wm = &P.wmap[it.proj];
+                const CUtensorMap *sm = &P.smap[it.proj];
+                const int fmt = p.fmt, c = it.chunk;
+                const int nw = slots_in_chunk(p, c);
+                for (int tt = 0; tt < it.ntiles && ok; ++tt) {
+                    const int o0 = (it.tile0 + tt) * 128;
+                    for (int w = 0; w < nw; ++w, ++j) {
+                        const int slot = j % NS;
+                        if (j >= NS &&
+                            !mbar_wait(&slot_empty[slot], static_cast<uint32_t>((j / NS) - 1) & 1u, lim)) {
+                            ok = false;
+                            break;
                         }
+                        if (j == 0 && ctl->inject) {
+                            skipped0 = true;
+                            continue;
+                        }
+                        int k0;
+                        const int klen = slot_len(p, c, w, k0);
+                        const int row_bytes = fmt == kFmtQ4 ? klen / 2 : klen;   // 64..256
+                        const int x = fmt == kFmtQ4 ? k0 / 2 : k0;              // multiple of 256
+                        const uint32_t dst = base + L.w_off + slot * kSlotBytes;
+                        // a box's bytes count in full, rows past N and columns
+                        // past the row included (TMA fills them with zeros)
+                        const int boxes = row_bytes > 128 ? 2 : 1;
+                        mbar_expect_tx(&slot_full[slot], static_cast<uint32_t>(
+                                                             boxes * kBoxBytes + (fmt == kFmtQ4 ? kScaleBytes : 0)));
+                        tma_load_2d(dst, wm, x, o0, &slot_full[slot]);
+                        if (boxes == 2) tma_load_2d(dst + kBoxBytes, wm, x + 128, o0, &slot_full[slot]);
+                        if (fmt == kFmtQ4)
+                            tma_load_2d(base + L.s_off + slot * kScaleBytes, sm, k0 / 32, o0, &slot_full[slot]);
                     }
-                    if (!(j == 0 && t == 0 && ctl->inject)) cp_async_arrive(&slot_full[slot]);
                 }
             }
+            // Every load issued has landed before the CTA may exit: slots
+            // before the last NS were reused, so they have been consumed.
+            for (int jj = max(0, j - NS); jj < j; ++jj)
+                if (!(jj == 0 && skipped0))
+                    mbar_wait(&slot_full[jj % NS], static_cast<uint32_t>(jj / NS) & 1u, lim);
         }
-        cp_async_wait_all();   // every copy this thread issued has landed
+        __syncwarp();
     } else if (warp == kXWarp) {
         // ======================================================= activation loader
         if (lane == 0) {
@@ -298,7 +422,7 @@ __global__ void __launch_bounds__(kPlThreads, 1)
             int cur_x = -1, cur_c = -1, nx = 0;
             for (int i = i_first; i < i_last && ok; ++i) {
                 const Item it = item_at(P, i);
-                const PlProj &p = *it.p;
+                const PlProj &p = it.p;
                 const int c = it.chunk;
                 if (p.xid == cur_x && c == cur_c) continue;
                 if (nx > 0 && !mbar_wait(x_empty, static_cast<uint32_t>(nx - 1) & 1u, lim)) {
@@ -321,15 +445,15 @@ __global__ void __launch_bounds__(kPlThreads, 1)
         const int h = warp >> 2;
         const int r = threadIdx.x & 127;
         const uint32_t ta = tmem + kAOff + (static_cast<uint32_t>((warp & 3) * 32) << 16) +
-                            static_cast<uint32_t>(16 * h);
+                            static_cast<uint32_t>(32 * h);
         int j = 0, ja = 0;
         for (int i = i_first; i < i_last && ok; ++i) {
             const Item it = item_at(P, i);
-            const PlProj &p = *it.p;
+            const PlProj &p = it.p;
             const int c = it.chunk;
             const int nw = slots_in_chunk(p, c);
             for (int tt = 0; tt < it.ntiles && ok; ++tt) {
-                for (int w = 0; w < nw; ++w, ++j) {
+                for (int w = 0; w < nw && ok; ++w, ++j) {
                     const int slot = j % NS;
                     if (!mbar_wait(&slot_full[slot], static_cast<uint32_t>(j / NS) & 1u, lim)) {
                         ok = false;
@@ -339,30 +463,15 @@ __global__ void __launch_bounds__(kPlThreads, 1)
                     const int nsteps = slot_len(p, c, w, k0) / 64;
                     const uint32_t wslot = base + L.w_off + slot * kSlotBytes;
                     const uint32_t sslot = base + L.s_off + slot * kScaleBytes;
-                    for (int s = 0; s < nsteps; ++s, ++ja) {
-                        uint32_t wv[16];
-                        if (p.fmt == kFmtQ4)
-                            dequant_slot<kFmtQ4>(wslot, sslot, r, h, s, wv);
-                        else if (p.fmt == kFmtQ8)
-                            dequant_slot<kFmtQ8>(wslot, sslot, r, h, s, wv);
-                        else
-                            dequant_slot<kFmtE4M3>(wslot, sslot, r, h, s, wv);
-                        const int st = ja % kAStages;
-                        if (ja >= kAStages &&
-                            !mbar_wait(&a_empty[st], static_cast<uint32_t>((ja / kAStages) - 1) & 1u,
-                                       lim)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after_sync();
-                        tmem_st_x16(ta + static_cast<uint32_t>(st) * kAStageCols, wv);
-                        tmem_st_wait();
-                        tc_fence_before_sync();
-                        mbar_arrive(&a_full[st]);
-                    }
-                    if (!ok) break;
-                    // every read of the slot has been consumed by a store above
-                    mbar_arrive(&slot_empty[slot]);
+                    if (p.fmt == kFmtQ4)
+                        ok = dequant_slot<kFmtQ4>(wslot, sslot, r, h, nsteps, ta, ja, &slot_empty[slot],
+                                                  a_full, a_empty, lim);
+                    else if (p.fmt == kFmtQ8)
+                        ok = dequant_slot<kFmtQ8>(wslot, sslot, r, h, nsteps, ta, ja, &slot_empty[slot],
+                                                  a_full, a_empty, lim);
+                    else
+                        ok = dequant_slot<kFmtE4M3>(wslot, sslot, r, h, nsteps, ta, ja,
+                                                    &slot_empty[slot], a_full, a_empty, lim);
                 }
             }
         }
@@ -374,7 +483,7 @@ __global__ void __launch_bounds__(kPlThreads, 1)
         int cur_x = -1, cur_c = -1, nx = 0, ja = 0, ntile = 0;
         for (int i = i_first; i < i_last && ok; ++i) {
             const Item it = item_at(P, i);
-            const PlProj &p = *it.p;
+            const PlProj &p = it.p;
             const int c = it.chunk;
             bool good = true;
             const bool fresh = !(p.xid == cur_x && c == cur_c);
@@ -388,8 +497,8 @@ __global__ void __launch_bounds__(kPlThreads, 1)
                 const int n_acc = ntile + tt;                 // accumulator of this tile
                 for (int w = 0; w < nw && ok; ++w) {
                     int k0;
-                    const int nsteps = slot_len(p, c, w, k0) / 64;
-                    for (int s = 0; s < nsteps; ++s, ++ja) {
+                    const int nstages = (slot_len(p, c, w, k0) / 64 + 1) / 2;
+                    for (int s = 0; s < nstages; ++s, ++ja) {
                         if (lane == 0) {
                             if (good && fresh && tt == 0 && w == 0 && s == 0)
                                 good = mbar_wait(x_full, static_cast<uint32_t>(nx - 1) & 1u, lim);
@@ -420,7 +529,7 @@ __global__ void __launch_bounds__(kPlThreads, 1)
         bool abort = false;
         for (int i = i_first; i < i_last && !abort; ++i) {
             const Item it = item_at(P, i);
-            const PlProj &p = *it.p;
+            const PlProj &p = it.p;
             const int c = it.chunk;
             const int nw = slots_in_chunk(p, c);
             for (int tt = 0; tt < it.ntiles && !abort; ++tt) {
@@ -430,7 +539,7 @@ __global__ void __launch_bounds__(kPlThreads, 1)
                     int k0;
                     const int nsteps = slot_len(p, c, w, k0) / 64;
                     const int atom0 = (k0 - c * kXChunk) / 64;
-                    for (int s = 0; s < nsteps; ++s, ++ja) {
+                    for (int s = 0; 2 * s < nsteps; ++s, ++ja) {
                         named_bar_sync(kMmaBar, 64);
                         if (mma_abort[ja & 1]) {
                             abort = true;
@@ -440,12 +549,15 @@ __global__ void __launch_bounds__(kPlThreads, 1)
                             tc_fence_after_sync();
                             const uint32_t a =
                                 tmem + kAOff + static_cast<uint32_t>(ja % kAStages) * kAStageCols;
-                            const uint64_t bdesc = xdesc0 + static_cast<uint64_t>(atom0 + s) * atom_desc;
                             const bool first = w == 0 && s == 0;
+                            for (int u = 0; u < 2 && 2 * s + u < nsteps; ++u) {
+                                const uint64_t bdesc =
+                                    xdesc0 + static_cast<uint64_t>(atom0 + 2 * s + u) * atom_desc;
 #pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                tc_mma_f16kind_ts(d, a + 8 * kk, bdesc + 2 * kk, idesc,
-                                                  (first && kk == 0) ? 0u : 1u);
+                                for (int kk = 0; kk < 4; ++kk)
+                                    tc_mma_f16kind_ts(d, a + 32 * u + 8 * kk, bdesc + 2 * kk, idesc,
+                                                      (first && u == 0 && kk == 0) ? 0u : 1u);
+                            }
                             tc_commit(&a_empty[ja % kAStages]);
                         }
                     }
@@ -485,7 +597,7 @@ __global__ void __launch_bounds__(kPlThreads, 1)
         int ntile = 0;
         for (int i = i_first; i < i_last && ok; ++i) {
             const Item it = item_at(P, i);
-            const PlProj &p = *it.p;
+            const PlProj &p = it.p;
             const bool split = it.nchunks > 1;
             for (int tt = 0; tt < it.ntiles && ok; ++tt, ++ntile) {
                 const int slot = ntile % R;
@@ -552,12 +664,34 @@ __global__ void __launch_bounds__(kPlThreads, 1)
                     if (o < p.N) {
                         const float sc = p.fmt == 8 ? __ldg(static_cast<const float *>(p.S) + o) : 1.f;
                         const float b = p.bias ? __ldg(p.bias + o) : 0.f;
-                        const float *p0 = P.partials + static_cast<size_t>(st * P.max_chunks) * BNp * 128;
-                        for (int m = c0; m < c0 + cols && m < M; ++m) {
-                            float acc = __ldcg(p0 + static_cast<size_t>(m) * 128 + row);
-                            for (int ch = 1; ch < it.nchunks; ++ch)
-                                acc += __ldcg(p0 + (static_cast<size_t>(ch) * BNp + m) * 128 + row);
-                            p.Y[static_cast<size_t>(m) * p.N + o] = fmaf(acc, sc, b);
+                        const float *p0 = P.partials +
+                                          static_cast<size_t>(st * P.max_chunks) * BNp * 128 + row;
+                        const size_t cstride = static_cast<size_t>(BNp) * 128;
+                        for (int mb = c0; mb < c0 + cols && mb < M; mb += 8) {
+                            // up to 4 chunks x 8 columns of loads in flight, then
+                            // the sums in chunk order
+                            float acc[8];
+                            for (int cb = 0; cb < it.nchunks; cb += 4) {
+                                float v[4][8];
+#pragma unroll
+                                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                                    for (int e = 0; e < 8; ++e)
+                                        v[u][e] = cb + u < it.nchunks
+                                                      ? __ldcg(p0 + (cb + u) * cstride +
+                                                               static_cast<size_t>(mb + e) * 128)
+                                                      : 0.f;
+#pragma unroll
+                                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                                    for (int e = 0; e < 8; ++e)
+                                        if (cb + u < it.nchunks)
+                                            acc[e] = (cb + u == 0) ? v[u][e] : acc[e] + v[u][e];
+                            }
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                if (mb + e < M)
+                                    p.Y[static_cast<size_t>(mb + e) * p.N + o] = fmaf(acc[e], sc, b);
                         }
                     }
                     if (et == 0) P.counters[st] = 0u;      // ready for the next launch
@@ -578,12 +712,17 @@ __global__ void __launch_bounds__(kPlThreads, 1)
 // ------------------------------------------------------------ pre-pass
 // Converts each distinct activation block X [M, K] fp32 once into the fp16
 // image the list kernel loads: [K/64 atoms][BNp rows][128 bytes], 16-byte
-// chunk j of row m at chunk j ^ (m & 7) (the 128-byte swizzle), pairs within
-// every chunk in the operand order of dequant.cuh, rows M..BNp-1 zero.  One
+// chunk j of row m at chunk j ^ (m & 7) (the 128-byte swizzle), the 8 values
+// of every chunk as the pairs (t, t + 4) of the dequantizers, rows M..BNp-1
+// zero.  One
 // 512-wide K chunk is then one contiguous range.  An activation that is not
 // a finite fp16 value after rounding latches kStatusRange.
 __global__ void __launch_bounds__(256)
     pl_prep_kernel(const __grid_constant__ PlPrep P, DevCtl *ctl) {
+    // The list launch that follows may start right away: its weight copies
+    // do not depend on this kernel, and it reads the images only after its
+    // own wait for this grid's completion.
+    pdl_launch_dependents();
     pdl_wait_prior_grid();
     if (blockIdx.x == 0 && blockIdx.y == 0)
         for (int i = threadIdx.x; i < P.n_counters; i += blockDim.x) P.counters[i] = 0u;
@@ -601,7 +740,9 @@ __global__ void __launch_bounds__(256)
         if (m < M) {
             const float4 *src =
                 reinterpret_cast<const float4 *>(im.X + static_cast<size_t>(m) * K + a * 64 + j * 8);
-            const uint2 lo = x4_f16(__ldg(src)), hi = x4_f16(__ldg(src + 1));
+            const float4 a = __ldg(src), b = __ldg(src + 1);
+            const uint2 lo = make_uint2(pack_f16x2(a.x, b.x), pack_f16x2(a.y, b.y));
+            const uint2 hi = make_uint2(pack_f16x2(a.z, b.z), pack_f16x2(a.w, b.w));
             bad |= f16x2_nonfinite(lo) | f16x2_nonfinite(hi);
             out = make_uint4(lo.x, lo.y, hi.x, hi.y);
         }
@@ -610,7 +751,6 @@ __global__ void __launch_bounds__(256)
     }
     if (__any_sync(0xffffffffu, bad != 0) && (threadIdx.x & 31) == 0)
         atomicOr(&ctl->status, 1u << kStatusRange);
-    pdl_launch_dependents();
 }
 
 cudaError_t launch_pl_prep(const PlPrep &prep, int n_images, int64_t max_k, DevCtl *ctl,
@@ -661,9 +801,30 @@ int pl_nslots(int bnp) {
     return std::max(2, std::min(kMaxSlots, avail / (kSlotBytes + kScaleBytes)));
 }
 
-bool pl_supported(int fmt, int M, int K) {
-    // q4 (scale, min) rows are 16-byte cp.async copies: K/8 bytes a multiple of 16
-    return M >= 1 && M <= 128 && (fmt == 4 ? K % 128 == 0 : K % 64 == 0);
+namespace {
+
+// Tiles per work item: up to about 80 KB of packed weights (two q4 tiles of
+// a 512-wide chunk, one q8 or e4m3 tile), small against a CTA's share of a
+// list so that the runs cut from the sorted items come out nearly equal.
+int tiles_per_item(int fmt, int K) {
+    const int klen = std::min(K, kXChunk);
+    const double tile = 128.0 * klen * (fmt == 4 ? 0.625 : 1.0);
+    return std::max(1, std::min(4, static_cast<int>(80.0 * 1024 / tile)));
+}
+
+int64_t items_of(int fmt, int64_t N, int K) {
+    const int64_t tiles = (N + 127) / 128;
+    const int per = tiles_per_item(fmt, K);
+    return static_cast<int64_t>((K + kXChunk - 1) / kXChunk) * ((tiles + per - 1) / per);
+}
+
+}  // namespace
+
+bool pl_supported(int fmt, int M, int64_t N, int K) {
+    // TMA boxes: the rows of codes and of q4 (scale, min) words (K/8 bytes)
+    // must be multiples of 16 bytes; one projection's items fit one launch
+    return M >= 1 && M <= 128 && N >= 1 && (fmt == 4 ? K % 128 == 0 : K % 64 == 0) &&
+           items_of(fmt, N, K) <= kPlMaxItems;
 }
 
 namespace {
@@ -717,13 +878,43 @@ Plan plan_list(const PlInput *in, int count, int M) {
     return pl;
 }
 
-// Tiles per work item: up to about 160 KB of packed weights (four q4 tiles
-// of a 512-wide chunk, two q8 or e4m3 tiles), so that the items assigned to
-// one CTA can be balanced closely.
-int tiles_per_item(const PlInput &q) {
-    const int klen = std::min(q.K, kXChunk);
-    const double tile = 128.0 * klen * (q.fmt == 4 ? 0.625 : 1.0);
-    return std::max(1, std::min(4, static_cast<int>(160.0 * 1024 / tile)));
+// Tensor maps of the packed weights, cached per thread by (pointer, shape,
+// kind) in a small direct-mapped table, so that a list call encodes only the
+// weights it has not seen lately.  kind 0: codes, kind 1: q4 (scale, min)
+// words.
+bool weight_map(CUtensorMap *out, int kind, int fmt, const void *ptr, int64_t N, int K) {
+    struct Entry {
+        CUtensorMap map;
+        const void *ptr;
+        int64_t N;
+        int K, key;
+    };
+    constexpr int kEntries = 256;
+    thread_local Entry cache[kEntries] = {};
+    const int key = kind * 16 + fmt;
+    const uintptr_t h = (reinterpret_cast<uintptr_t>(ptr) >> 8) ^ static_cast<uintptr_t>(N * 31 + K) ^
+                        static_cast<uintptr_t>(key);
+    Entry &e = cache[(h ^ (h >> 9)) % kEntries];
+    if (e.ptr == ptr && e.N == N && e.K == K && e.key == key) {
+        *out = e.map;
+        return true;
+    }
+    bool ok;
+    if (kind == 0)
+        ok = encode_tma_2d(out, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ptr,
+                           static_cast<uint64_t>(fmt == 4 ? K / 2 : K), static_cast<uint64_t>(N), 128,
+                           CU_TENSOR_MAP_SWIZZLE_128B, 128);
+    else
+        ok = encode_tma_2d(out, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, ptr, static_cast<uint64_t>(K / 32),
+                           static_cast<uint64_t>(N), 16, CU_TENSOR_MAP_SWIZZLE_64B, 128);
+    if (ok) {
+        e.map = *out;
+        e.ptr = ptr;
+        e.N = N;
+        e.K = K;
+        e.key = key;
+    }
+    return ok;
 }
 
 }  // namespace
@@ -779,9 +970,13 @@ cudaError_t launch_pl_batch(const PlInput *in, int count, int M, void *ws, DevCt
             const PlInput &q = in[src];
             const int tiles = (q.N + 127) / 128;
             const int nchunks = (q.K + kXChunk - 1) / kXChunk;
-            const int per = tiles_per_item(q);
+            const int per = tiles_per_item(q.fmt, q.K);
             const int n_items = nchunks * ((tiles + per - 1) / per);
+            if (n_items > kPlMaxItems) return cudaErrorInvalidValue;   // not pl_supported
             if (np > 0 && items.size() + n_items > static_cast<size_t>(kPlMaxItems)) break;
+            if (!weight_map(&P.wmap[np], 0, q.fmt, q.Wq, q.N, q.K) ||
+                (q.fmt == 4 && !weight_map(&P.smap[np], 1, q.fmt, q.S, q.N, q.K)))
+                return cudaErrorInvalidValue;
             P.proj[np] = {wsb + pl.off[pl.xid[src]], q.Wq, q.S, q.bias, q.Y, q.N, q.K, q.fmt,
                           pl.xid[src], pl.sbase[src]};
             for (int c = 0; c < nchunks; ++c) {
@@ -795,33 +990,34 @@ cudaError_t launch_pl_batch(const PlInput *in, int count, int M, void *ws, DevCt
                 }
             }
         }
-        // largest item first onto the least loaded CTA
+        // items in (activation image, K chunk, projection, tile) order, cut
+        // into G contiguous runs of about equal bytes
         const int n_items = static_cast<int>(items.size());
         const int G = std::min(sms, n_items);
-        std::vector<int> by_cost(n_items);
-        std::iota(by_cost.begin(), by_cost.end(), 0);
-        std::stable_sort(by_cost.begin(), by_cost.end(),
-                         [&](int a, int b) { return cost[a] > cost[b]; });
-        std::vector<double> load(G, 0.0);
-        std::vector<std::vector<int>> mine(G);
-        for (int it : by_cost) {
-            const int b = static_cast<int>(std::min_element(load.begin(), load.end()) - load.begin());
-            load[b] += cost[it];
-            mine[b].push_back(it);
-        }
-        // within a CTA: items of one activation chunk together, in list order
+        std::vector<int> order_it(n_items);
+        std::iota(order_it.begin(), order_it.end(), 0);
+        std::stable_sort(order_it.begin(), order_it.end(), [&](int a, int c) {
+            const PlItem &x = items[a], &y = items[c];
+            if (P.proj[x.proj].xid != P.proj[y.proj].xid) return P.proj[x.proj].xid < P.proj[y.proj].xid;
+            if (x.chunk != y.chunk) return x.chunk < y.chunk;
+            if (x.proj != y.proj) return x.proj < y.proj;
+            return x.tile0 < y.tile0;
+        });
+        double total = 0.0;
+        for (double c : cost) total += c;
         int k = 0;
+        double done = 0.0;
         for (int b = 0; b < G; ++b) {
-            std::sort(mine[b].begin(), mine[b].end(), [&](int a, int c) {
-                const PlItem &x = items[a], &y = items[c];
-                if (P.proj[x.proj].xid != P.proj[y.proj].xid)
-                    return P.proj[x.proj].xid < P.proj[y.proj].xid;
-                if (x.chunk != y.chunk) return x.chunk < y.chunk;
-                if (x.proj != y.proj) return x.proj < y.proj;
-                return x.tile0 < y.tile0;
-            });
             P.cta_items[b] = k;
-            for (int it : mine[b]) P.items[k++] = items[it];
+            const double target = total * (b + 1) / G;
+            // at least one item, and one left for every later CTA; an item
+            // joins this run if its midpoint lies before the target
+            const int last = n_items - (G - 1 - b);
+            do {
+                done += cost[order_it[k]];
+                P.items[k] = items[order_it[k]];
+                ++k;
+            } while (k < last && done + 0.5 * cost[order_it[k]] < target);
         }
         P.cta_items[G] = k;
         P.M = M;

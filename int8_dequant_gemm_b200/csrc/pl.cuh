@@ -1,15 +1,17 @@
-// Parameters of the projection-list kernel (pl.cu): the projections, the work
-// items cut from them and each CTA's share, passed by value as one
-// __grid_constant__ kernel parameter (under the 32 KB parameter limit).
+// Parameters of the projection-list kernel (pl.cu): the projections, their
+// weights' TMA tensor maps, the work items cut from them and each CTA's
+// share, passed by value as one __grid_constant__ kernel parameter (under the
+// 32 KB parameter limit).
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
 
 namespace rtq {
 
-constexpr int kPlMaxProj = 256;     // projections per launch
-constexpr int kPlMaxItems = 1792;   // work items per launch
+constexpr int kPlMaxProj = 64;      // projections per launch
+constexpr int kPlMaxItems = 1440;   // work items per launch
 constexpr int kPlMaxCtas = 160;     // >= the SM count of one B200
 constexpr int kPlMaxAcc = 8;        // accumulators in the TMEM ring
 
@@ -36,6 +38,11 @@ struct PlItem {
 };
 
 struct PlParams {
+    // per projection: its codes as a [N, row bytes] u8 tensor (boxes of 128
+    // rows x 128 bytes, 128-byte swizzle) and, for q4, its (scale, min) words
+    // as a [N, K/32] u32 tensor (boxes of 128 rows x 16 words, 64-byte swizzle)
+    CUtensorMap wmap[kPlMaxProj];
+    CUtensorMap smap[kPlMaxProj];
     int M, bnp, nslots, nacc;
     float *partials;     // split tiles: [tile][chunk][BNp][128] fp32
     unsigned *counters;  // split tiles: chunks finished (reset to 0 by the last)
