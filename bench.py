@@ -615,7 +615,7 @@ def measure_large_m(args, rank, world, local_rank, dev, stream):
 
 # --------------------------------------------------------------- M sweep
 SWEEP_SHAPES = (("q4", 2048, 512), ("q8", 512, 2048))    # ffn.w1 and ffn.w2 shapes
-SWEEP_M = (1, 16, 80, 512, 4096, 65536)
+SWEEP_M = (1, 2, 4, 8, 16, 32, 80, 512, 4096, 65536)
 SWEEP_SIMT_MAX_M = 4096      # the fp32 SIMT path is timed up to here
 
 

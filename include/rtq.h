@@ -96,7 +96,8 @@ typedef enum rt_format {
 } rt_format;
 
 typedef enum rt_path {
-    RT_PATH_AUTO = 0,   /* SIMT for M <= 8 or K % 64 != 0, else TC */
+    RT_PATH_AUTO = 0,   /* SIMT for K % 64 != 0 or M <= 16 (q4) / M <= 1 (q8,
+                           e4m3), else TC: the measured single-call crossover */
     RT_PATH_SIMT = 1,   /* fp32 CUDA-core kernels */
     RT_PATH_TC = 2      /* tcgen05 tensor-core kernels, fp16 operands, fp32 accumulate in TMEM */
 } rt_path;            /* any other value: RT_ERR_INVALID_ARG */

@@ -141,12 +141,12 @@ int pick_kernel(int fmt, int64_t M, int64_t N, int64_t K, int p) {
     return RT_KERNEL_TC_W_STATIONARY;
 }
 
-int pick_path(int64_t M, int64_t K, int path) {
+int pick_path(int fmt, int64_t M, int64_t K, int path) {
     const bool tc_ok = (K % 64) == 0;
     if (path == RT_PATH_TC) return tc_ok ? path : -1;
     if (path == RT_PATH_SIMT) return RT_PATH_SIMT;
     if (path != RT_PATH_AUTO) return -2;
-    return (M <= rtq::kAutoSimtMaxM || !tc_ok) ? RT_PATH_SIMT : RT_PATH_TC;
+    return (M <= rtq::auto_simt_max_m(fmt) || !tc_ok) ? RT_PATH_SIMT : RT_PATH_TC;
 }
 
 inline rt_status from_cuda(cudaError_t e) { return e == cudaSuccess ? RT_OK : RT_ERR_CUDA; }
@@ -155,7 +155,7 @@ inline rt_status from_cuda(cudaError_t e) { return e == cudaSuccess ? RT_OK : RT
 rt_status run_gemm(int fmt, const float *X, const void *Wq, const void *S, const float *bias,
                    float *Y, int64_t M,
                    int64_t N, int64_t K, int path, void *stream) {
-    const int p = pick_path(M, K, path);
+    const int p = pick_path(fmt, M, K, path);
     if (p == -1) return RT_ERR_UNSUPPORTED_SHAPE;
     if (p < 0) return RT_ERR_INVALID_ARG;
     if (M == 0) return RT_OK;
@@ -221,7 +221,7 @@ int rt_version(void) { return 200; }
 int rt_qgemm_auto_path(int fmt, int64_t M, int64_t N, int64_t K) {
     if (!rtq::fmt_valid(fmt) || M < 0 || N < 1 || K < 1) return -1;
     if (K % (fmt == 4 ? 32 : 16) != 0) return -1;
-    return pick_path(M, K, RT_PATH_AUTO);
+    return pick_path(fmt, M, K, RT_PATH_AUTO);
 }
 
 int rt_qgemm_plan(int fmt, int64_t M, int64_t N, int64_t K, int path) {
@@ -229,7 +229,7 @@ int rt_qgemm_plan(int fmt, int64_t M, int64_t N, int64_t K, int path) {
         K > kMaxDim)
         return -1;
     if (K % (fmt == 4 ? 32 : 16) != 0) return -1;
-    const int p = pick_path(M, K, path);
+    const int p = pick_path(fmt, M, K, path);
     if (p < 0) return -1;
     return pick_kernel(fmt, M, N, K, p);
 }
@@ -333,7 +333,7 @@ rt_status block_run(const BlockProj p[4], int64_t M, int64_t d, int64_t f, int p
         if ((st = rtq::check_gemm_args(q.fmt, q.X, q.W, q.S, q.Y, M, q.N, q.K)) != RT_OK ||
             (st = check_bias(q.bias, q.Y, M, q.N)) != RT_OK)
             return st;
-        const int pp = pick_path(M, q.K, path);
+        const int pp = pick_path(q.fmt, M, q.K, path);
         if (pp == -1) return RT_ERR_UNSUPPORTED_SHAPE;
         if (pp < 0) return RT_ERR_INVALID_ARG;
     }
@@ -450,7 +450,7 @@ int batch_route(const rt_qproj *list, int count, int64_t M, int path) {
         rt_status st = rtq::check_gemm_args(q.fmt, q.X, q.Wq, q.scales, q.Y, M, q.N, q.K);
         if (st == RT_OK) st = check_bias(q.bias, q.Y, M, q.N);
         if (st != RT_OK) return -st;
-        const int p = pick_path(M, q.K, path);
+        const int p = pick_path(q.fmt, M, q.K, path);
         if (p == -1) return -RT_ERR_UNSUPPORTED_SHAPE;
         tc_all = tc_all && p == RT_PATH_TC;
         // the list kernel reads q4 (scale, min) rows through a TMA map: 16-byte base

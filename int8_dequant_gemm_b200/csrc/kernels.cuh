@@ -136,7 +136,11 @@ rt_status check_gemm_args(int fmt, const float *X, const void *Wq, const void *S
                           int64_t M, int64_t N, int64_t K);
 rt_status device_ctl(DevCtl **out);
 
-// Largest M the SIMT path takes under RT_PATH_AUTO.
-constexpr int kAutoSimtMaxM = 8;
+// Largest M the SIMT path takes under RT_PATH_AUTO, per format: where a
+// single call of the fp32 SIMT kernel beats the tensor-core kernels in the M
+// sweep of the q4 512->2048 and q8 2048->512 projections (weights rotated
+// beyond L2): q4 up to M = 16 (ahead by 7 % at M = 8, level at 16), q8 and
+// e4m3 only at M = 1 (the tensor-core kernel is ahead from M = 2).
+constexpr int auto_simt_max_m(int fmt) { return fmt == kFmtQ4 ? 16 : 1; }
 
 }  // namespace rtq

@@ -1,6 +1,7 @@
 // fp32 CUDA-core kernels: the exact-rounding path (weights dequantized to
 // fp32 with one rounding -- exactly, for q8 codes and e4m3 values -- fp32 FMA
-// accumulation) and the path for M <= 8.
+// accumulation) and the automatic path at the smallest M (q4: M <= 16, q8 and
+// e4m3: M = 1).
 //
 // Layout of work: each thread owns one output row o of W and MT activation
 // rows, staged per CTA in shared memory.  Inside the K loop every lane of a

@@ -84,6 +84,10 @@ def test_validation_statuses(fn):
 
 
 def test_auto_path_dispatch():
+    # the measured single-call crossover: q4 SIMT up to M = 16, q8 and e4m3 at M = 1
+    assert rtq.auto_path(4, 16, 2048, 512) == 1 and rtq.auto_path(4, 17, 2048, 512) == 2
+    assert rtq.auto_path(8, 1, 512, 2048) == 1 and rtq.auto_path(8, 2, 512, 2048) == 2
+    assert rtq.auto_path(3, 1, 512, 2048) == 1 and rtq.auto_path(3, 2, 512, 2048) == 2
     assert rtq.auto_path(4, 1, 2048, 512) == 1
     assert rtq.auto_path(4, 80, 2048, 512) == 2
     assert rtq.auto_path(8, 65536, 512, 2048) == 2
@@ -145,8 +149,9 @@ def test_block_grouped_launch_plan():
     # one grouped launch exactly where all four projections take the
     # weight-stationary kernel with a single activation tile
     assert rtq.block_fused(80, 512, 2048) == 1
-    assert rtq.block_fused(9, 512, 2048) == 1 and rtq.block_fused(128, 512, 2048) == 1
-    assert rtq.block_fused(8, 512, 2048) == 0             # AUTO takes SIMT at M <= 8
+    assert rtq.block_fused(17, 512, 2048) == 1 and rtq.block_fused(128, 512, 2048) == 1
+    assert rtq.block_fused(16, 512, 2048) == 0            # AUTO takes SIMT for q4 at M <= 16
+    assert rtq.block_fused(8, 512, 2048) == 0
     assert rtq.block_fused(8, 512, 2048, "tc") == 1
     assert rtq.block_fused(1, 512, 2048, "tc") == 1
     assert rtq.block_fused(1, 512, 2048, 3) == -1
@@ -331,7 +336,7 @@ def test_batch_validation_and_routes():
     assert plan(ok, 12, 80, 0) == TC_LIST
     assert plan(ok, 12, 80, 2) == TC_LIST
     assert plan(ok, 12, 80, 1) == 0                           # SIMT: one call per entry
-    assert plan(ok, 12, 4, 0) == 0                            # AUTO takes SIMT at M <= 8
+    assert plan(ok, 12, 4, 0) == 0                            # AUTO takes SIMT for q4 at M <= 16
     assert plan(ok, 12, 200, 2) == 0                          # M > 128: per call
     assert plan(ok, 2, 80, 0) == 0                            # 32 tiles < SMs under AUTO
     assert plan(ok, 2, 80, 2) == TC_LIST                      # forced
@@ -372,7 +377,8 @@ def test_block_fmt_validation_and_routes():
     q8 = blk((8, 8, 8, 8))
     assert fused(C.byref(q8), 80, 0) == 1                  # one grouped launch
     assert fused(C.byref(q8), 2048, 0) == 0                # one call per projection
-    assert fused(C.byref(q8), 4, 0) == 0                   # SIMT under AUTO
+    assert fused(C.byref(q8), 1, 0) == 0                   # SIMT under AUTO (q8: M = 1)
+    assert fused(C.byref(q8), 2, 0) == 1
     mixed = blk((4, 8, 4, 8))
     assert fused(C.byref(mixed), 80, 0) == rtq.block_fused(80, 512, 2048) == 1
     assert fused(C.byref(blk((8, 8, 5, 8))), 80, 0) == -1  # unknown format
@@ -422,7 +428,8 @@ def test_e4m3_gemm_validation_and_plan():
     assert rtq.plan(3, 80, 512, 2048) == "tc_w_stationary"
     assert rtq.plan(3, 4096, 512, 512) == "tc_x_resident"
     assert rtq.plan(3, 4096, 512, 2048) == "tc_w_streamed"
-    assert rtq.plan(3, 4, 512, 2048) == "simt"
+    assert rtq.plan(3, 1, 512, 2048) == "simt"
+    assert rtq.plan(3, 4, 512, 2048) == "tc_w_stationary"
     assert rtq.auto_path(3, 80, 512, 48) == 1                     # K % 64 != 0 -> SIMT
     assert rtq.workspace_bytes(3, 4096, 512, 2048) == 4096 * 2048 * 2
     # a batch entry in e4m3 carries no scales
