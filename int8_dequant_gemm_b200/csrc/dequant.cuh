@@ -36,20 +36,23 @@ __device__ __forceinline__ void q4_word_f32(uint32_t v, float scale, float mn, f
     for (int i = 0; i < 8; ++i) w[i] = fmaf(small_uint_to_f32((v >> (4 * i)) & 0xFu), scale, mn);
 }
 
-// Tensor-core operand chunks hold 8 consecutive K elements in the pair order
-// [0,2 | 1,3 | 4,6 | 5,7] (one 32-bit word per pair).  Weights and
-// activations use the same order, so the MMA's dot products are unchanged;
-// the order lets each pair come from one byte pair of the packed codes and
-// from one float4 of the activations.  Both operands are fp16.
+// Tensor-core operand chunks hold 8 consecutive K elements k .. k+7 as the
+// four fp16 pairs (k + t, k + t + 4), t = 0..3, one 32-bit word per pair.
+// Weights and activations use the same order, so the MMA's dot products are
+// unchanged.  The order lets a q4 payload word (8 codes, code i in bits
+// 4i .. 4i+3) split into its four pairs with one shift and four masks, each
+// mask also setting the fp16 exponent pattern (see q4_word_f16); the two
+// one-byte formats take one byte permute per pair.
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
-// 4 activations (k, k+1, k+2, k+3) -> the two fp16 pair words (k,k+2),
-// (k+1,k+3), rounded to nearest-even.
-__device__ __forceinline__ uint2 x4_f16(float4 a) {
-    return make_uint2(pack_f16x2(a.x, a.z), pack_f16x2(a.y, a.w));
+// 8 activations k .. k+7 (a = k .. k+3, b = k+4 .. k+7) -> one operand chunk,
+// rounded to nearest-even.
+__device__ __forceinline__ uint4 x8_f16(float4 a, float4 b) {
+    return make_uint4(pack_f16x2(a.x, b.x), pack_f16x2(a.y, b.y), pack_f16x2(a.z, b.z),
+                      pack_f16x2(a.w, b.w));
 }
 
 // Non-zero where a half of an fp16 pair word is infinite or NaN (exponent
@@ -62,23 +65,22 @@ __device__ __forceinline__ uint32_t f16x2_nonfinite(uint2 w) {
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
 __device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2 *>(&u); }
 
-// q4, fp16 operands: 8 codes of one payload word -> one chunk.  fp16 0x6400
-// is 1024 with a unit last place, so OR-ing a code into the low mantissa bits
-// gives 1024 + code exactly; subtracting 1024 is exact; fma.rn.f16x2 then
-// rounds code*scale + min once.  s2 / m2 hold the group's scale / min in both
-// halves.
+// q4, fp16 operands: 8 codes of one payload word -> one chunk.  Code i sits
+// in bits 4i .. 4i+3, so codes t and t + 4 are the same nibble of the two
+// 16-bit halves: in bits 0-3 (t = 0, and t = 2 after a shift by 8) under the
+// exponent pattern 0x6400 a nibble reads as fp16 1024 + code, in bits 4-7
+// (t = 1, 3) under 0x5400 as 64 + code (unit last place 1/16).  Both
+// subtractions are exact; fma.rn.f16x2 then rounds code*scale + min once.
+// s2 / m2 hold the group's scale / min in both halves.
 __device__ __forceinline__ uint4 q4_word_f16(uint32_t v, uint32_t s2, uint32_t m2) {
-    const uint32_t x0 = __byte_perm(v, 0u, 0x4140);   // bytes b0, b1 -> half words 0, 1
-    const uint32_t x1 = __byte_perm(v, 0u, 0x4342);   // bytes b2, b3
-    const __half2 k1024 = bits_h2(0x64006400u), s = bits_h2(s2), m = bits_h2(m2);
-    const uint32_t c0 = (x0 & 0x000F000Fu) | 0x64006400u;         // codes 0, 2
-    const uint32_t c1 = ((x0 >> 4) & 0x000F000Fu) | 0x64006400u;  // codes 1, 3
-    const uint32_t c2 = (x1 & 0x000F000Fu) | 0x64006400u;         // codes 4, 6
-    const uint32_t c3 = ((x1 >> 4) & 0x000F000Fu) | 0x64006400u;  // codes 5, 7
-    return make_uint4(h2_bits(__hfma2(__hsub2(bits_h2(c0), k1024), s, m)),
-                      h2_bits(__hfma2(__hsub2(bits_h2(c1), k1024), s, m)),
-                      h2_bits(__hfma2(__hsub2(bits_h2(c2), k1024), s, m)),
-                      h2_bits(__hfma2(__hsub2(bits_h2(c3), k1024), s, m)));
+    const __half2 k1024 = bits_h2(0x64006400u), k64 = bits_h2(0x54005400u);
+    const __half2 s = bits_h2(s2), m = bits_h2(m2);
+    const uint32_t v8 = v >> 8;
+    return make_uint4(
+        h2_bits(__hfma2(__hsub2(bits_h2((v & 0x000F000Fu) | 0x64006400u), k1024), s, m)),
+        h2_bits(__hfma2(__hsub2(bits_h2((v & 0x00F000F0u) | 0x54005400u), k64), s, m)),
+        h2_bits(__hfma2(__hsub2(bits_h2((v8 & 0x000F000Fu) | 0x64006400u), k1024), s, m)),
+        h2_bits(__hfma2(__hsub2(bits_h2((v8 & 0x00F000F0u) | 0x54005400u), k64), s, m)));
 }
 
 // (scale, min) word -> (scale, scale) and (min, min).
@@ -97,13 +99,19 @@ __device__ __forceinline__ float q8_byte_f32(uint32_t v, int i) {
 // q8, fp16 operands: two payload words (codes 0..3, 4..7) -> one chunk.  The
 // offset-binary byte q + 128 under an 0x64 high byte is fp16 1024 + q + 128;
 // subtracting 1152 leaves q exactly.
+// Byte t of a and byte t of b in the low bytes of the two 16-bit halves
+// (the high bytes are bytes of a and b too: callers mask them).
+__device__ __forceinline__ uint32_t pair_bytes(uint32_t a, uint32_t b, int t) {
+    return __byte_perm(a, b, static_cast<uint32_t>(t | (t << 4) | ((4 + t) << 8) | ((4 + t) << 12)));
+}
+
 __device__ __forceinline__ uint4 q8_words_f16(uint32_t a, uint32_t b) {
-    const uint32_t ua = a ^ 0x80808080u, ub = b ^ 0x80808080u;
     const __half2 k1152 = bits_h2(0x64806480u);
-    return make_uint4(h2_bits(__hsub2(bits_h2(__byte_perm(ua, 0x64646464u, 0x4240)), k1152)),
-                      h2_bits(__hsub2(bits_h2(__byte_perm(ua, 0x64646464u, 0x4341)), k1152)),
-                      h2_bits(__hsub2(bits_h2(__byte_perm(ub, 0x64646464u, 0x4240)), k1152)),
-                      h2_bits(__hsub2(bits_h2(__byte_perm(ub, 0x64646464u, 0x4341)), k1152)));
+    uint32_t w[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t)   // mask the bytes, flip bit 7, set the 0x64 high bytes: one op
+        w[t] = h2_bits(__hsub2(bits_h2((pair_bytes(a, b, t) & 0x00FF00FFu) ^ 0x64806480u), k1152));
+    return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 // FP8 E4M3 ("RT-J -- FP8 E4M3 checkpoints", "FP8 Format": weights stored
@@ -121,10 +129,8 @@ __device__ __forceinline__ uint32_t e4m3_pair_f16(uint32_t x) {
 
 // e4m3, fp16 operands: two payload words (codes 0..3, 4..7) -> one chunk.
 __device__ __forceinline__ uint4 e4m3_words_f16(uint32_t a, uint32_t b) {
-    return make_uint4(e4m3_pair_f16(__byte_perm(a, 0u, 0x4240)),
-                      e4m3_pair_f16(__byte_perm(a, 0u, 0x4341)),
-                      e4m3_pair_f16(__byte_perm(b, 0u, 0x4240)),
-                      e4m3_pair_f16(__byte_perm(b, 0u, 0x4341)));
+    return make_uint4(e4m3_pair_f16(pair_bytes(a, b, 0)), e4m3_pair_f16(pair_bytes(a, b, 1)),
+                      e4m3_pair_f16(pair_bytes(a, b, 2)), e4m3_pair_f16(pair_bytes(a, b, 3)));
 }
 
 // e4m3 code (byte i of v) -> fp32, exact: the integer (8 + M) << (E - 1), or
@@ -139,8 +145,8 @@ __device__ __forceinline__ float e4m3_byte_f32(uint32_t v, int i) {
 
 // Chunk in operand order -> natural order (for the dequantization exports).
 __device__ __forceinline__ uint4 chunk_to_natural(uint4 c) {
-    return make_uint4(__byte_perm(c.x, c.y, 0x5410), __byte_perm(c.x, c.y, 0x7632),
-                      __byte_perm(c.z, c.w, 0x5410), __byte_perm(c.z, c.w, 0x7632));
+    return make_uint4(__byte_perm(c.x, c.y, 0x5410), __byte_perm(c.z, c.w, 0x5410),
+                      __byte_perm(c.x, c.y, 0x7632), __byte_perm(c.z, c.w, 0x7632));
 }
 
 }  // namespace rtq

@@ -35,12 +35,9 @@
 //            operand layout) into the resident activation buffer, reloaded
 //            only when the (activations, K chunk) pair changes.
 // A stages: the MMAs read the dequantized weights from TMEM, one stage = two
-// 64-wide K steps (64 columns) in a ring of four at columns [256, 512).
-// Within every 8 consecutive K values the operands are paired (t, t + 4),
-// t = 0..3, in both A and the activation image: that order lets the q4
-// dequantizer take the 8 nibbles of a 32-bit word apart with one shift and
-// four masks (two nibbles per mask, turned into fp16 by an exponent pattern
-// in the same operation), where the natural pairing needs byte permutes too.
+// 64-wide K steps (64 columns) in a ring of four at columns [256, 512), in
+// the operand order of dequant.cuh (pairs (k + t, k + t + 4) in every 8
+// K values), which the activation image follows too.
 // Roles (20 warps):
 //   warps 0-7   dequantizers: thread (r, h) converts step h of each stage of
 //               row r (64 K values) into TMEM lane r of the stage: it loads
@@ -91,7 +88,7 @@ constexpr int kSlotBytes = 32 * 1024;                // 128 rows x 256 bytes of 
 constexpr int kBoxBytes = 16 * 1024;                 // one TMA box: 128 rows x 128 bytes
 constexpr int kScaleBytes = 8 * 1024;                // 128 rows x 16 (scale, min) words
 constexpr int kMaxSlots = 4;
-constexpr int kAStages = 4;
+constexpr int kAStages = 4;                          // a power of two
 constexpr uint32_t kAStageCols = 64;                 // two 64-wide K steps
 constexpr uint32_t kAOff = 256;                      // A stages at TMEM columns [256, 512)
 constexpr int kXChunk = 512;                         // K of one resident activation chunk
@@ -172,39 +169,11 @@ __device__ __forceinline__ int slots_in_chunk(const PlProj &p, int c) {
 }
 
 // ------------------------------------------------------------ dequantization
-// Operand pairs (K 8j + t, 8j + t + 4), t = 0..3, of one 8-value chunk j.
-
-// q4: the 8 codes of word v (code i in bits 4i..4i+3) -> 4 fp16 pair words
-// (scale, min applied: w = q * scale + min, one rounding).  A nibble in bits
-// 0-3 of a 16-bit half under exponent pattern 0x6400 is fp16 1024 + q; in
-// bits 4-7 under 0x5400 it is 64 + q (ulp 1/16); both subtractions are exact.
-__device__ __forceinline__ void q4_pairs(uint32_t v, __half2 s, __half2 m, uint32_t *out) {
-    const __half2 k1024 = bits_h2(0x64006400u), k64 = bits_h2(0x54005400u);
-    const uint32_t v8 = v >> 8;
-    out[0] = h2_bits(__hfma2(__hsub2(bits_h2((v & 0x000F000Fu) | 0x64006400u), k1024), s, m));
-    out[1] = h2_bits(__hfma2(__hsub2(bits_h2((v & 0x00F000F0u) | 0x54005400u), k64), s, m));
-    out[2] = h2_bits(__hfma2(__hsub2(bits_h2((v8 & 0x000F000Fu) | 0x64006400u), k1024), s, m));
-    out[3] = h2_bits(__hfma2(__hsub2(bits_h2((v8 & 0x00F000F0u) | 0x54005400u), k64), s, m));
-}
-
-// Byte t of a and byte t of b in the low bytes of the two 16-bit halves.
-__device__ __forceinline__ uint32_t pair_bytes(uint32_t a, uint32_t b, int t) {
-    return __byte_perm(a, b, static_cast<uint32_t>(t | (t << 4) | ((4 + t) << 8) | ((4 + t) << 12)));
-}
-
-// q8: codes 8j..8j+3 in a, 8j+4..8j+7 in b -> 4 fp16 pair words of the
-// integers (the row scale is applied in the epilogue).  The offset-binary
-// byte q + 128 under 0x64 is fp16 1024 + q + 128; subtracting 1152 is exact.
-__device__ __forceinline__ void q8_pairs(uint32_t a, uint32_t b, uint32_t *out) {
-    const __half2 k1152 = bits_h2(0x64806480u);
-#pragma unroll
-    for (int t = 0; t < 4; ++t)
-        out[t] = h2_bits(__hsub2(bits_h2((pair_bytes(a, b, t) & 0x00FF00FFu) ^ 0x64806480u), k1152));
-}
-
-__device__ __forceinline__ void e4m3_pairs(uint32_t a, uint32_t b, uint32_t *out) {
-#pragma unroll
-    for (int t = 0; t < 4; ++t) out[t] = e4m3_pair_f16(pair_bytes(a, b, t));
+__device__ __forceinline__ void put4(uint32_t (&w)[16], int i, uint4 v) {
+    w[i] = v.x;
+    w[i + 1] = v.y;
+    w[i + 2] = v.z;
+    w[i + 3] = v.w;
 }
 
 // Half h of 32 K values (h = 0: K 0..31 of the step, 1: K 32..63) of one
@@ -213,21 +182,22 @@ __device__ __forceinline__ void e4m3_pairs(uint32_t a, uint32_t b, uint32_t *out
 template <int FMT>
 __device__ __forceinline__ void convert_half(uint4 r0, uint4 r1, uint32_t sw, uint32_t (&w)[16]) {
     if (FMT == kFmtQ4) {
-        const __half2 s = bits_h2(__byte_perm(sw, 0u, 0x1010)), m = bits_h2(__byte_perm(sw, 0u, 0x3232));
-        q4_pairs(r0.x, s, m, w + 0);
-        q4_pairs(r0.y, s, m, w + 4);
-        q4_pairs(r0.z, s, m, w + 8);
-        q4_pairs(r0.w, s, m, w + 12);
+        uint32_t s2, m2;
+        q4_scale_min_f16x2(sw, s2, m2);
+        put4(w, 0, q4_word_f16(r0.x, s2, m2));
+        put4(w, 4, q4_word_f16(r0.y, s2, m2));
+        put4(w, 8, q4_word_f16(r0.z, s2, m2));
+        put4(w, 12, q4_word_f16(r0.w, s2, m2));
     } else if (FMT == kFmtQ8) {
-        q8_pairs(r0.x, r0.y, w + 0);
-        q8_pairs(r0.z, r0.w, w + 4);
-        q8_pairs(r1.x, r1.y, w + 8);
-        q8_pairs(r1.z, r1.w, w + 12);
+        put4(w, 0, q8_words_f16(r0.x, r0.y));
+        put4(w, 4, q8_words_f16(r0.z, r0.w));
+        put4(w, 8, q8_words_f16(r1.x, r1.y));
+        put4(w, 12, q8_words_f16(r1.z, r1.w));
     } else {
-        e4m3_pairs(r0.x, r0.y, w + 0);
-        e4m3_pairs(r0.z, r0.w, w + 4);
-        e4m3_pairs(r1.x, r1.y, w + 8);
-        e4m3_pairs(r1.z, r1.w, w + 12);
+        put4(w, 0, e4m3_words_f16(r0.x, r0.y));
+        put4(w, 4, e4m3_words_f16(r0.z, r0.w));
+        put4(w, 8, e4m3_words_f16(r1.x, r1.y));
+        put4(w, 12, e4m3_words_f16(r1.z, r1.w));
     }
 }
 
@@ -545,30 +515,36 @@ __global__ void __launch_bounds__(kPlThreads, 1)
                             abort = true;
                             break;
                         }
-                        if (lane == 0) {
-                            tc_fence_after_sync();
-                            const uint32_t a =
-                                tmem + kAOff + static_cast<uint32_t>(ja % kAStages) * kAStageCols;
-                            const bool first = w == 0 && s == 0;
-                            for (int u = 0; u < 2 && 2 * s + u < nsteps; ++u) {
-                                const uint64_t bdesc =
-                                    xdesc0 + static_cast<uint64_t>(atom0 + 2 * s + u) * atom_desc;
+                        // the whole warp walks the loop; one elected lane issues
+                        tc_fence_after_sync();
+                        const int st = ja & (kAStages - 1);
+                        const uint32_t a = tmem + kAOff + static_cast<uint32_t>(st) * kAStageCols;
+                        const uint64_t b0 = xdesc0 + static_cast<uint64_t>(atom0 + 2 * s) * atom_desc;
+                        const uint32_t acc0 = (w == 0 && s == 0) ? 0u : 1u;
+                        const bool two = 2 * s + 1 < nsteps;
+                        if (elect_one()) {
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk)
+                                tc_mma_f16kind_ts(d, a + 8 * kk, b0 + 2 * kk, idesc, kk == 0 ? acc0 : 1u);
+                            if (two) {
 #pragma unroll
                                 for (int kk = 0; kk < 4; ++kk)
-                                    tc_mma_f16kind_ts(d, a + 32 * u + 8 * kk, bdesc + 2 * kk, idesc,
-                                                      (first && u == 0 && kk == 0) ? 0u : 1u);
+                                    tc_mma_f16kind_ts(d, a + 32 + 8 * kk, b0 + atom_desc + 2 * kk, idesc, 1u);
                             }
-                            tc_commit(&a_empty[ja % kAStages]);
+                            tc_commit(&a_empty[st]);
                         }
+                        __syncwarp();
                     }
                 }
-                if (!abort && lane == 0) tc_commit(&acc_full[n_acc % R]);
+                if (!abort && elect_one()) tc_commit(&acc_full[n_acc % R]);
+                __syncwarp();
             }
             // release the activation chunk once its MMAs complete if the next
             // item reads a different (activations, chunk)
-            if (!abort && lane == 0 && i + 1 < i_last) {
+            if (!abort && i + 1 < i_last) {
                 const PlItem &nx = P.items[i + 1];
-                if (!(P.proj[nx.proj].xid == p.xid && nx.chunk == c)) tc_commit(x_empty);
+                if (!(P.proj[nx.proj].xid == p.xid && nx.chunk == c) && elect_one()) tc_commit(x_empty);
+                __syncwarp();
             }
             ntile += it.ntiles;
         }
@@ -713,10 +689,9 @@ __global__ void __launch_bounds__(kPlThreads, 1)
 // Converts each distinct activation block X [M, K] fp32 once into the fp16
 // image the list kernel loads: [K/64 atoms][BNp rows][128 bytes], 16-byte
 // chunk j of row m at chunk j ^ (m & 7) (the 128-byte swizzle), the 8 values
-// of every chunk as the pairs (t, t + 4) of the dequantizers, rows M..BNp-1
-// zero.  One
-// 512-wide K chunk is then one contiguous range.  An activation that is not
-// a finite fp16 value after rounding latches kStatusRange.
+// of every chunk in the operand order of dequant.cuh, rows M..BNp-1 zero.
+// One 512-wide K chunk is then one contiguous range.  An activation that is
+// not a finite fp16 value after rounding latches kStatusRange.
 __global__ void __launch_bounds__(256)
     pl_prep_kernel(const __grid_constant__ PlPrep P, DevCtl *ctl) {
     // The list launch that follows may start right away: its weight copies
@@ -740,11 +715,8 @@ __global__ void __launch_bounds__(256)
         if (m < M) {
             const float4 *src =
                 reinterpret_cast<const float4 *>(im.X + static_cast<size_t>(m) * K + a * 64 + j * 8);
-            const float4 a = __ldg(src), b = __ldg(src + 1);
-            const uint2 lo = make_uint2(pack_f16x2(a.x, b.x), pack_f16x2(a.y, b.y));
-            const uint2 hi = make_uint2(pack_f16x2(a.z, b.z), pack_f16x2(a.w, b.w));
-            bad |= f16x2_nonfinite(lo) | f16x2_nonfinite(hi);
-            out = make_uint4(lo.x, lo.y, hi.x, hi.y);
+            out = x8_f16(__ldg(src), __ldg(src + 1));
+            bad |= f16x2_nonfinite(make_uint2(out.x, out.y)) | f16x2_nonfinite(make_uint2(out.z, out.w));
         }
         uint8_t *dst = im.Xh + (static_cast<size_t>(a) * BNp + m) * 128 + ((j ^ (m & 7)) << 4);
         *reinterpret_cast<uint4 *>(dst) = out;

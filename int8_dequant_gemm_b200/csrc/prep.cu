@@ -2,8 +2,8 @@
 // encoder they share.
 //
 // The pre-pass rounds X (fp32 [M, K]) once to fp16 and stores it in the chunk
-// order the MMA operands use (pairs [0,2 | 1,3 | 4,6 | 5,7] within every 8
-// elements, see dequant.cuh).  The GEMM kernels then load activation tiles
+// order the MMA operands use (pairs (k + t, k + t + 4), t = 0..3, within
+// every 8 elements k .. k+7, see dequant.cuh).  The GEMM kernels then load activation tiles
 // with TMA straight into the 128-byte-swizzled operand layout, with no
 // conversion work and at half the bytes of fp32.  It is a pure streaming
 // kernel: 4 bytes read and 2 written per element.  An activation that is not
@@ -26,9 +26,9 @@ __global__ void __launch_bounds__(256)
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_chunks;
          i += stride) {
         const float4 a = __ldcs(X + 2 * i), b = __ldcs(X + 2 * i + 1);
-        const uint2 lo = x4_f16(a), hi = x4_f16(b);
-        bad |= f16x2_nonfinite(lo) | f16x2_nonfinite(hi);
-        Xh[i] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+        const uint4 c = x8_f16(a, b);
+        bad |= f16x2_nonfinite(make_uint2(c.x, c.y)) | f16x2_nonfinite(make_uint2(c.z, c.w));
+        Xh[i] = c;
     }
     if (__any_sync(0xffffffffu, bad != 0) && (threadIdx.x & 31) == 0)
         atomicOr(&ctl->status, 1u << kStatusRange);

@@ -177,6 +177,21 @@ __device__ __forceinline__ void tc_mma_f16kind_ts(uint32_t d_tmem, uint32_t a_tm
         : "memory");
 }
 
+// True in exactly one lane of a converged warp (elect.sync).  A warp that
+// runs a loop in uniform control flow and issues single-thread instructions
+// such as tcgen05.mma from the elected lane keeps its loop and descriptor
+// arithmetic warp-uniform; issuing from a `lane == 0` branch instead costs
+// about a quarter more per MMA, measured.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t.reg .b32 rx;\n\t"
+        "elect.sync rx|P, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, P;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 // Arrives once on `bar` when every previously issued tcgen05.mma of this
 // thread has completed.
 __device__ __forceinline__ void tc_commit(uint64_t *bar) {

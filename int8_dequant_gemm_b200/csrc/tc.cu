@@ -15,8 +15,8 @@
 // finite makes its outputs infinite or NaN, and the epilogue latches
 // kStatusRange in the device control block for any output that is not finite
 // (finite fp16 operands cannot overflow an fp32 sum of K <= 2^20 products).  Within every
-// 8-element K chunk both operands store their pairs in the order
-// [0,2 | 1,3 | 4,6 | 5,7] (see dequant.cuh).
+// 8-element K chunk k .. k+7 both operands store the pairs
+// (k + t, k + t + 4), t = 0..3 (see dequant.cuh).
 //
 // One CTA = 8 converter warps + 1 MMA warp.  Per 64-wide K step the converter
 // warps
@@ -202,9 +202,20 @@ __device__ __forceinline__ void store_stage(const StageRegs<PIECES> &R, const Co
         sts_v4(sA + c.a_off[2], e4m3_words_f16(R.a1.x, R.a1.y));
         sts_v4(sA + c.a_off[3], e4m3_words_f16(R.a1.z, R.a1.w));
     }
+    // A chunk's 8 activations are split between lanes p (even: k .. k+3) and
+    // p + 1 (odd: k+4 .. k+7); each lane takes two values from its partner and
+    // writes its half of the chunk's pairs (k + t, k + t + 4): t = 0, 1 from
+    // the even lane, t = 2, 3 from the odd one.
+    const bool odd = (c.p & 1) != 0;
 #pragma unroll
-    for (int i = 0; i < PIECES; ++i)
-        if (c.rb0 + 16 * i < BN) sts_v2(sB + c.b_off0 + 2048u * i, x4_f16(R.b[i]));
+    for (int i = 0; i < PIECES; ++i) {
+        const float4 a = R.b[i];
+        const float s0 = __shfl_xor_sync(0xffffffffu, odd ? a.x : a.z, 1);
+        const float s1 = __shfl_xor_sync(0xffffffffu, odd ? a.y : a.w, 1);
+        const uint2 v = odd ? make_uint2(pack_f16x2(s0, a.z), pack_f16x2(s1, a.w))
+                            : make_uint2(pack_f16x2(a.x, s0), pack_f16x2(a.y, s1));
+        if (c.rb0 + 16 * i < BN) sts_v2(sB + c.b_off0 + 2048u * i, v);
+    }
 }
 
 // True for an infinite or NaN fp32 value.
@@ -369,12 +380,14 @@ __device__ __forceinline__ void tc_tile(uint8_t *smem_raw, const float *__restri
             }
         }
         if (__any_sync(0xffffffffu, ybad) && lane == 0) atomicOr(&ctl->status, 1u << kStatusRange);
-    } else if (lane == 0) {
+    } else {
         // -------------------------------------------------------- MMA issuer
+        // The whole warp walks the loop and waits; one elected lane issues.
         const uint32_t idesc = idesc_f16_f32acc(kTileO, BN);
         for (int ks = 0; ks < nk; ++ks) {
             const int s = ks % stages;
-            if (!mbar_wait(&full[s], static_cast<uint32_t>(ks / stages) & 1u, lim)) {
+            const bool got = mbar_wait(&full[s], static_cast<uint32_t>(ks / stages) & 1u, lim);
+            if (__shfl_sync(0xffffffffu, got ? 1 : 0, 0) == 0) {
                 ok = false;
                 break;
             }
@@ -383,20 +396,25 @@ __device__ __forceinline__ void tc_tile(uint8_t *smem_raw, const float *__restri
             const uint32_t sB = sA + kAStageBytes;
             const uint64_t adesc = sw128_kmajor_desc(sA);
             const uint64_t bdesc = sw128_kmajor_desc(sB);
+            if (elect_one()) {
 #pragma unroll
-            for (int kk = 0; kk < kTileK / 16; ++kk) {
-                // +32 bytes per 16-element K step -> +2 in the 16-byte address field
-                tc_mma_f16kind(tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc,
-                               (ks > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < kTileK / 16; ++kk) {
+                    // +32 bytes per 16-element K step -> +2 in the 16-byte address field
+                    tc_mma_f16kind(tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc,
+                                   (ks > 0 || kk > 0) ? 1u : 0u);
+                }
+                tc_commit(&empty[s]);
             }
-            tc_commit(&empty[s]);
+            __syncwarp();
         }
         if (ok) {
-            tc_commit(done);
+            if (elect_one()) tc_commit(done);
+            __syncwarp();
         } else {
             // MMAs already issued may still read the stage ring and write
             // TMEM: wait (bounded) for them before the CTA releases either.
-            tc_commit(drain);
+            if (elect_one()) tc_commit(drain);
+            __syncwarp();
             mbar_wait(drain, 0, lim);
         }
     }

@@ -328,11 +328,12 @@ __global__ void __launch_bounds__(kWsThreads, 1)
                     abort = true;
                     break;
                 }
-                if (lane == 0) {
-                    tc_fence_after_sync();
-                    const int s = j % kAStages, sb = j % kStages;
-                    const uint32_t at = tmem + kAccCols + static_cast<uint32_t>(s) * kAStageCols;
-                    const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(sb) * kStageDesc;
+                // the whole warp walks the loop; one elected lane issues
+                tc_fence_after_sync();
+                const int s = j % kAStages, sb = j % kStages;
+                const uint32_t at = tmem + kAccCols + static_cast<uint32_t>(s) * kAStageCols;
+                const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(sb) * kStageDesc;
+                if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < kAtomK / 16; ++kk)
                         tc_mma_f16kind_ts(d, at + 8 * kk, bdesc + 2 * kk, idesc,
@@ -340,9 +341,11 @@ __global__ void __launch_bounds__(kWsThreads, 1)
                     tc_commit(&a_empty[s]);
                     tc_commit(&b_empty[sb]);
                 }
+                __syncwarp();
             }
             if (abort) break;
-            if (lane == 0) tc_commit(&acc_full[b]);
+            if (elect_one()) tc_commit(&acc_full[b]);
+            __syncwarp();
         }
         if (abort && lane == 0) {
             // MMAs already issued may still read shared memory and write

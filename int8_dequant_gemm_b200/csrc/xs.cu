@@ -393,23 +393,26 @@ __global__ void __launch_bounds__(kXsThreads, 1)
                     abort = true;
                     break;
                 }
-                if (lane == 0) {
-                    tc_fence_after_sync();
-                    const uint32_t at = tmem + kAccCols + (j & (kAStages - 1)) * kAStageCols;
+                // the whole warp walks the loop; one elected lane issues
+                tc_fence_after_sync();
+                const uint32_t at = tmem + kAccCols + (j & (kAStages - 1)) * kAStageCols;
+                if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < kAtomK / 16; ++kk)
                         tc_mma_f16kind_ts(d, at + 8 * kk, bdesc + 2 * kk, idesc,
                                           (ks > 0 || kk > 0) ? 1u : 0u);
                     tc_commit(&a_empty[j & (kAStages - 1)]);
                 }
+                __syncwarp();
             }
             if (abort) break;
-            if (lane == 0) {
+            if (elect_one()) {
                 tc_commit(&acc_full[b]);
                 // last item of this activation block with another block to
                 // follow: release the X tile once these MMAs have completed
                 if (it.item + 1 < last && it.o_tile + 1 == n_o_tiles) tc_commit(x_empty);
             }
+            __syncwarp();
         }
         if (abort && lane == 0) {
             // MMAs already issued may still read shared memory and write

@@ -429,14 +429,14 @@ def _guarded_outputs(M, shapes, guard=64):
 FUSED_CASES = [
     (80, 512, 2048, "auto"),      # RT-J block at the small-M config: qkvg, wo, w13 split by 2
                                   # (4 tiles per cluster of 8), w2 by 8; 136 CTAs of 4 K steps
-    (16, 512, 2048, "auto"),      # 16-column activation tile
+    (16, 512, 2048, "tc"),        # 16-column activation tile (AUTO runs q4 on SIMT here)
     (48, 512, 2048, "auto"),
     (128, 512, 2048, "auto"),     # largest single activation tile
     (1, 512, 2048, "tc"),         # one row, tensor cores forced
     (80, 512, 2048, "tc"),
     (100, 256, 1024, "auto"),     # wo's 2 tiles half-fill a cluster: 2 CTA pairs store nothing
     (37, 1024, 4096, "auto"),     # 272 CTAs of 8 K steps
-    (16, 2048, 8192, "auto"),     # clusters of 4: w2 split by 4, the others unsplit
+    (16, 2048, 8192, "tc"),       # clusters of 4: w2 split by 4, the others unsplit
 ]
 
 
