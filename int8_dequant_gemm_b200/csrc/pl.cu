@@ -30,10 +30,13 @@
 //            (A slot issued as 16-byte cp.async copies instead costs one
 //            instruction per 16 bytes on the SM's load/store path and paced
 //            the whole pipeline; a TMA box costs one.)
-//   activations  one bulk copy per 512-wide K chunk of the projection's fp16
-//            image (written by pl_prep_kernel below in the 128-byte-swizzled
-//            operand layout) into the resident activation buffer, reloaded
-//            only when the (activations, K chunk) pair changes.
+//   activations  the projection's fp16 image (written by pl_prep_kernel below
+//            in the 128-byte-swizzled operand layout), one 512-wide K chunk
+//            at a time, into a resident buffer of two halves (K atoms 0-3 and
+//            4-7 of the chunk, one bulk copy each).  A half is reloaded only
+//            when the (activations, K chunk) pair changes, and only once the
+//            MMAs of its previous use have completed: the next chunk's first
+//            half streams in while the current chunk's second half is used.
 // A stages: the MMAs read the dequantized weights from TMEM, one stage = two
 // 64-wide K steps (64 columns) in a ring of four at columns [256, 512), in
 // the operand order of dequant.cuh (pairs (k + t, k + t + 4) in every 8
@@ -48,16 +51,18 @@
 //   warps 10-17 epilogue: TMEM -> registers (q8 row scale) -> fp32 Y.
 //   warp 18     weight producer (one thread, TMA).
 //   warp 19     activation loader (one thread, bulk copies).
-// Work items longer than one 512-wide K chunk (K > 512) run chunk by chunk
-// over all their tiles (each tile in its own accumulator), so one resident
-// activation chunk serves every tile of the item.
+// A tile with K > 512 is one work item that runs chunk by chunk, its
+// accumulator kept in TMEM across the chunks: no partial sums leave the SM.
+// (Splitting K over CTAs, with fp32 partials that the last chunk to finish
+// summed, cost more than half the time of a K = 2048 list: the partial
+// stores, fences and the dependent reduction loads.)
 //
-// Work distribution (host, launch_pl_batch): items (one 512-wide K chunk of
-// up to four tiles, about 80 KB of packed weights) are sorted by (activation
-// image, K chunk) and the sorted sequence is cut into one contiguous run per
-// CTA with about equal bytes, so a CTA switches its resident activation
-// chunk at most once or twice.  Every tile chunk is computed by one CTA from
-// start to end, so results do not depend on the assignment.
+// Work distribution (host, launch_pl_batch): items (up to four tiles of K <=
+// 512, about 80 KB of packed weights; one tile when K > 512) are sorted by
+// (activation image, projection, tile) and the sorted sequence is cut into
+// one contiguous run per CTA with about equal bytes, so a CTA switches its
+// activation image rarely.  Every tile is computed by one CTA from start to
+// end, so results do not depend on the assignment.
 //
 // Every mbarrier wait is bounded; a wait that gives up latches
 // RT_ERR_DEVICE_TIMEOUT and the CTA winds down: copies it issued complete,
@@ -106,9 +111,9 @@ __host__ __device__ inline PlLayout pl_layout(int bnp, int nslots) {
     L.w_off = bnp * kXChunk * 2;
     L.s_off = L.w_off + nslots * kSlotBytes;
     L.bar_off = L.s_off + nslots * kScaleBytes;
-    // slot full/empty, A full/empty, x full/empty, acc full/empty, drain, then
-    // 8 words: TMEM address, 2 issuer abort flags, the epilogue's flags
-    L.total = L.bar_off + (2 * kMaxSlots + 2 * kAStages + 2 + 2 * kPlMaxAcc + 1) * 8 + 32;
+    // slot full/empty, A full/empty, 2 x full/empty, acc full/empty, drain,
+    // then 8 words: TMEM address, 2 issuer abort flags, the epilogue's flags
+    L.total = L.bar_off + (2 * kMaxSlots + 2 * kAStages + 4 + 2 * kPlMaxAcc + 1) * 8 + 32;
     return L;
 }
 
@@ -134,15 +139,14 @@ __device__ __forceinline__ uint32_t wchunk(uint32_t slot, int c, int r) {
 // Physical 16-byte chunk of logical scale chunk c (0..3) of row r.
 __device__ __forceinline__ int sswz(int c, int r) { return c ^ ((r >> 1) & 3); }
 
-// The walk every role takes through a CTA's items: item (one K chunk of a
-// few tiles) -> tile -> weight slot -> 64-wide K step.  Each role advances it
-// at its own grain.  The projection's fields are copied into registers once
+// The walk every role takes through a CTA's items: item -> 512-wide K chunk
+// -> tile -> weight slot -> stage.  Each role advances it at its own grain.  The projection's fields are copied into registers once
 // per item: read through a pointer into the parameter space they would be
 // loaded again after every asm statement that clobbers memory (the barrier
 // waits and arrivals), a few hundred cycles each.
 struct Item {
     PlProj p;
-    int proj, tile0, ntiles, chunk, nchunks;
+    int proj, tile0, ntiles, nchunks;
 };
 
 __device__ __forceinline__ Item item_at(const PlParams &P, int i) {
@@ -152,7 +156,6 @@ __device__ __forceinline__ Item item_at(const PlParams &P, int i) {
     r.proj = it.proj;
     r.tile0 = static_cast<int>(it.tile0);
     r.ntiles = it.ntiles;
-    r.chunk = it.chunk;
     r.nchunks = (r.p.K + kXChunk - 1) / kXChunk;
     return r;
 }
@@ -162,6 +165,9 @@ __device__ __forceinline__ int slot_len(const PlProj &p, int c, int w, int &k0) 
     k0 = c * kXChunk + w * slot_k(p.fmt);
     return max(0, min(slot_k(p.fmt), p.K - k0));
 }
+
+// 64-wide K atoms of chunk c (8 except in a last, shorter chunk).
+__device__ __forceinline__ int chunk_atoms(const PlProj &p, int c) { return min(8, (p.K - c * kXChunk) / 64); }
 
 __device__ __forceinline__ int slots_in_chunk(const PlProj &p, int c) {
     const int len = min(kXChunk, p.K - c * kXChunk);
@@ -284,9 +290,9 @@ __global__ void __launch_bounds__(kPlThreads, 1)
     uint64_t *slot_empty = slot_full + kMaxSlots;
     uint64_t *a_full = slot_empty + kMaxSlots;
     uint64_t *a_empty = a_full + kAStages;
-    uint64_t *x_full = a_empty + kAStages;
-    uint64_t *x_empty = x_full + 1;
-    uint64_t *acc_full = x_empty + 1;
+    uint64_t *x_full = a_empty + kAStages;             // two: the halves of the buffer
+    uint64_t *x_empty = x_full + 2;
+    uint64_t *acc_full = x_empty + 2;
     uint64_t *acc_empty = acc_full + kPlMaxAcc;
     uint64_t *drain = acc_empty + kPlMaxAcc;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
@@ -305,8 +311,10 @@ __global__ void __launch_bounds__(kPlThreads, 1)
             mbar_init(&a_full[s], kDeqWarps * 32);
             mbar_init(&a_empty[s], 1);
         }
-        mbar_init(x_full, 1);
-        mbar_init(x_empty, 1);
+        for (int h = 0; h < 2; ++h) {
+            mbar_init(&x_full[h], 1);
+            mbar_init(&x_empty[h], 1);
+        }
         for (int b = 0; b < kPlMaxAcc; ++b) {
             mbar_init(&acc_full[b], 1);
             mbar_init(&acc_empty[b], kEpiThreads);
@@ -346,35 +354,39 @@ __global__ void __launch_bounds__(kPlThreads, 1)
                 const PlProj &p = it.p;
                 const CUtensorMap *wm = &P.wmap[it.proj];
                 const CUtensorMap *sm = &P.smap[it.proj];
-                const int fmt = p.fmt, c = it.chunk;
-                const int nw = slots_in_chunk(p, c);
-                for (int tt = 0; tt < it.ntiles && ok; ++tt) {
-                    const int o0 = (it.tile0 + tt) * 128;
-                    for (int w = 0; w < nw; ++w, ++j) {
-                        const int slot = j % NS;
-                        if (j >= NS &&
-                            !mbar_wait(&slot_empty[slot], static_cast<uint32_t>((j / NS) - 1) & 1u, lim)) {
-                            ok = false;
-                            break;
+                const int fmt = p.fmt;
+                for (int c = 0; c < it.nchunks && ok; ++c) {
+                    const int nw = slots_in_chunk(p, c);
+                    for (int tt = 0; tt < it.ntiles && ok; ++tt) {
+                        const int o0 = (it.tile0 + tt) * 128;
+                        for (int w = 0; w < nw; ++w, ++j) {
+                            const int slot = j % NS;
+                            if (j >= NS &&
+                                !mbar_wait(&slot_empty[slot], static_cast<uint32_t>((j / NS) - 1) & 1u, lim)) {
+                                ok = false;
+                                break;
+                            }
+                            if (j == 0 && ctl->inject) {
+                                skipped0 = true;
+                                continue;
+                            }
+                            int k0;
+                            const int klen = slot_len(p, c, w, k0);
+                            const int row_bytes = fmt == kFmtQ4 ? klen / 2 : klen;   // 64..256
+                            const int x = fmt == kFmtQ4 ? k0 / 2 : k0;              // multiple of 256
+                            const uint32_t dst = base + L.w_off + slot * kSlotBytes;
+                            // a box's bytes count in full, rows past N and
+                            // columns past the row included (TMA fills zeros)
+                            const int boxes = row_bytes > 128 ? 2 : 1;
+                            mbar_expect_tx(&slot_full[slot],
+                                           static_cast<uint32_t>(boxes * kBoxBytes +
+                                                                 (fmt == kFmtQ4 ? kScaleBytes : 0)));
+                            tma_load_2d(dst, wm, x, o0, &slot_full[slot]);
+                            if (boxes == 2) tma_load_2d(dst + kBoxBytes, wm, x + 128, o0, &slot_full[slot]);
+                            if (fmt == kFmtQ4)
+                                tma_load_2d(base + L.s_off + slot * kScaleBytes, sm, k0 / 32, o0,
+                                            &slot_full[slot]);
                         }
-                        if (j == 0 && ctl->inject) {
-                            skipped0 = true;
-                            continue;
-                        }
-                        int k0;
-                        const int klen = slot_len(p, c, w, k0);
-                        const int row_bytes = fmt == kFmtQ4 ? klen / 2 : klen;   // 64..256
-                        const int x = fmt == kFmtQ4 ? k0 / 2 : k0;              // multiple of 256
-                        const uint32_t dst = base + L.w_off + slot * kSlotBytes;
-                        // a box's bytes count in full, rows past N and columns
-                        // past the row included (TMA fills them with zeros)
-                        const int boxes = row_bytes > 128 ? 2 : 1;
-                        mbar_expect_tx(&slot_full[slot], static_cast<uint32_t>(
-                                                             boxes * kBoxBytes + (fmt == kFmtQ4 ? kScaleBytes : 0)));
-                        tma_load_2d(dst, wm, x, o0, &slot_full[slot]);
-                        if (boxes == 2) tma_load_2d(dst + kBoxBytes, wm, x + 128, o0, &slot_full[slot]);
-                        if (fmt == kFmtQ4)
-                            tma_load_2d(base + L.s_off + slot * kScaleBytes, sm, k0 / 32, o0, &slot_full[slot]);
                     }
                 }
             }
@@ -387,27 +399,39 @@ __global__ void __launch_bounds__(kPlThreads, 1)
         __syncwarp();
     } else if (warp == kXWarp) {
         // ======================================================= activation loader
+        // One use of the resident buffer = one (activation image, K chunk)
+        // over consecutive chunks of the walk.  Each half (atoms 0-3, 4-7 of
+        // the chunk) is refilled once the MMAs of the previous use of that
+        // half have completed, so a chunk's first half loads while the
+        // previous chunk's second half is still being multiplied.
         if (lane == 0) {
             pdl_wait_prior_grid();     // the fp16 images come from the preceding pre-pass
-            int cur_x = -1, cur_c = -1, nx = 0;
+            int cur_x = -1, cur_c = -1, loads0 = 0, loads1 = 0;
             for (int i = i_first; i < i_last && ok; ++i) {
                 const Item it = item_at(P, i);
                 const PlProj &p = it.p;
-                const int c = it.chunk;
-                if (p.xid == cur_x && c == cur_c) continue;
-                if (nx > 0 && !mbar_wait(x_empty, static_cast<uint32_t>(nx - 1) & 1u, lim)) {
-                    ok = false;
-                    break;
+                for (int c = 0; c < it.nchunks && ok; ++c) {
+                    if (p.xid == cur_x && c == cur_c) continue;
+                    cur_x = p.xid;
+                    cur_c = c;
+                    const int atoms = chunk_atoms(p, c);
+                    for (int h = 0; h < (atoms > 4 ? 2 : 1); ++h) {
+                        const int nl = h ? loads1 : loads0;
+                        if (nl > 0 && !mbar_wait(&x_empty[h], static_cast<uint32_t>(nl - 1) & 1u, lim)) {
+                            ok = false;
+                            break;
+                        }
+                        const int na = min(4, atoms - 4 * h);
+                        const uint32_t bytes = static_cast<uint32_t>(na * BNp * 128);
+                        mbar_expect_tx(&x_full[h], bytes);
+                        bulk_load(base + L.x_off + static_cast<uint32_t>(h * 4 * BNp * 128),
+                                  p.Xh + static_cast<size_t>(c * 8 + 4 * h) * BNp * 128, bytes, &x_full[h]);
+                        if (h) ++loads1; else ++loads0;
+                    }
                 }
-                const int atoms = (min(kXChunk, p.K - c * kXChunk)) / 64;
-                const uint32_t bytes = static_cast<uint32_t>(atoms * BNp * 128);
-                mbar_expect_tx(x_full, bytes);
-                bulk_load(base + L.x_off, p.Xh + static_cast<size_t>(c) * BNp * 1024, bytes, x_full);
-                cur_x = p.xid;
-                cur_c = c;
-                ++nx;
             }
-            if (nx > 0) mbar_wait(x_full, static_cast<uint32_t>(nx - 1) & 1u, lim);
+            if (loads0 > 0) mbar_wait(&x_full[0], static_cast<uint32_t>(loads0 - 1) & 1u, lim);
+            if (loads1 > 0) mbar_wait(&x_full[1], static_cast<uint32_t>(loads1 - 1) & 1u, lim);
         }
         __syncwarp();
     } else if (warp < kDeqWarps) {
@@ -420,70 +444,82 @@ __global__ void __launch_bounds__(kPlThreads, 1)
         for (int i = i_first; i < i_last && ok; ++i) {
             const Item it = item_at(P, i);
             const PlProj &p = it.p;
-            const int c = it.chunk;
-            const int nw = slots_in_chunk(p, c);
-            for (int tt = 0; tt < it.ntiles && ok; ++tt) {
-                for (int w = 0; w < nw && ok; ++w, ++j) {
-                    const int slot = j % NS;
-                    if (!mbar_wait(&slot_full[slot], static_cast<uint32_t>(j / NS) & 1u, lim)) {
-                        ok = false;
-                        break;
+            for (int c = 0; c < it.nchunks && ok; ++c) {
+                const int nw = slots_in_chunk(p, c);
+                for (int tt = 0; tt < it.ntiles && ok; ++tt) {
+                    for (int w = 0; w < nw && ok; ++w, ++j) {
+                        const int slot = j % NS;
+                        if (!mbar_wait(&slot_full[slot], static_cast<uint32_t>(j / NS) & 1u, lim)) {
+                            ok = false;
+                            break;
+                        }
+                        int k0;
+                        const int nsteps = slot_len(p, c, w, k0) / 64;
+                        const uint32_t wslot = base + L.w_off + slot * kSlotBytes;
+                        const uint32_t sslot = base + L.s_off + slot * kScaleBytes;
+                        if (p.fmt == kFmtQ4)
+                            ok = dequant_slot<kFmtQ4>(wslot, sslot, r, h, nsteps, ta, ja, &slot_empty[slot],
+                                                      a_full, a_empty, lim);
+                        else if (p.fmt == kFmtQ8)
+                            ok = dequant_slot<kFmtQ8>(wslot, sslot, r, h, nsteps, ta, ja, &slot_empty[slot],
+                                                      a_full, a_empty, lim);
+                        else
+                            ok = dequant_slot<kFmtE4M3>(wslot, sslot, r, h, nsteps, ta, ja,
+                                                        &slot_empty[slot], a_full, a_empty, lim);
                     }
-                    int k0;
-                    const int nsteps = slot_len(p, c, w, k0) / 64;
-                    const uint32_t wslot = base + L.w_off + slot * kSlotBytes;
-                    const uint32_t sslot = base + L.s_off + slot * kScaleBytes;
-                    if (p.fmt == kFmtQ4)
-                        ok = dequant_slot<kFmtQ4>(wslot, sslot, r, h, nsteps, ta, ja, &slot_empty[slot],
-                                                  a_full, a_empty, lim);
-                    else if (p.fmt == kFmtQ8)
-                        ok = dequant_slot<kFmtQ8>(wslot, sslot, r, h, nsteps, ta, ja, &slot_empty[slot],
-                                                  a_full, a_empty, lim);
-                    else
-                        ok = dequant_slot<kFmtE4M3>(wslot, sslot, r, h, nsteps, ta, ja,
-                                                    &slot_empty[slot], a_full, a_empty, lim);
                 }
             }
         }
     } else if (warp == kWaiterWarp) {
         // ======================================================= MMA waiter
-        // All waits of the issuer, handed over per K step through named
+        // All waits of the issuer, handed over per stage through named
         // barrier kMmaBar (a thread that waits on an mbarrier right after a
         // tcgen05.commit stalls until its MMAs drain, so the issuer never waits).
-        int cur_x = -1, cur_c = -1, nx = 0, ja = 0, ntile = 0;
+        // loads of each half so far, and whether this use's stages have
+        // reached each half (scalars: an indexed array would live in memory)
+        int cur_x = -1, cur_c = -1, ja = 0, ntile = 0, loads0 = 0, loads1 = 0;
+        bool seen0 = false, seen1 = false;
+        bool good = true;
         for (int i = i_first; i < i_last && ok; ++i) {
             const Item it = item_at(P, i);
             const PlProj &p = it.p;
-            const int c = it.chunk;
-            bool good = true;
-            const bool fresh = !(p.xid == cur_x && c == cur_c);
-            if (fresh) {
-                cur_x = p.xid;
-                cur_c = c;
-                ++nx;
-            }
-            const int nw = slots_in_chunk(p, c);
-            for (int tt = 0; tt < it.ntiles && ok; ++tt) {
-                const int n_acc = ntile + tt;                 // accumulator of this tile
-                for (int w = 0; w < nw && ok; ++w) {
-                    int k0;
-                    const int nstages = (slot_len(p, c, w, k0) / 64 + 1) / 2;
-                    for (int s = 0; s < nstages; ++s, ++ja) {
-                        if (lane == 0) {
-                            if (good && fresh && tt == 0 && w == 0 && s == 0)
-                                good = mbar_wait(x_full, static_cast<uint32_t>(nx - 1) & 1u, lim);
-                            if (good && w == 0 && s == 0 && n_acc >= R)
-                                good = mbar_wait(&acc_empty[n_acc % R],
-                                                 static_cast<uint32_t>((n_acc / R) - 1) & 1u, lim);
-                            if (good)
-                                good = mbar_wait(&a_full[ja % kAStages],
-                                                 static_cast<uint32_t>(ja / kAStages) & 1u, lim);
-                            mma_abort[ja & 1] = good ? 0u : 1u;
-                        }
-                        named_bar_sync(kMmaBar, 64);
-                        if (__shfl_sync(0xffffffffu, good ? 1 : 0, 0) == 0) {
-                            ok = false;
-                            break;
+            for (int c = 0; c < it.nchunks && ok; ++c) {
+                if (!(p.xid == cur_x && c == cur_c)) {
+                    cur_x = p.xid;
+                    cur_c = c;
+                    ++loads0;
+                    if (chunk_atoms(p, c) > 4) ++loads1;
+                    seen0 = seen1 = false;
+                }
+                const int nw = slots_in_chunk(p, c);
+                for (int tt = 0; tt < it.ntiles && ok; ++tt) {
+                    const int n_acc = ntile + tt;                 // accumulator of this tile
+                    for (int w = 0; w < nw && ok; ++w) {
+                        int k0;
+                        const int nsteps = slot_len(p, c, w, k0) / 64;
+                        const int atom0 = (k0 - c * kXChunk) / 64;
+                        for (int s = 0; 2 * s < nsteps; ++s, ++ja) {
+                            const int hx = atom0 + 2 * s >= 4 ? 1 : 0;
+                            const bool first_touch = hx ? !seen1 : !seen0;
+                            if (lane == 0) {
+                                if (good && first_touch)
+                                    good = mbar_wait(&x_full[hx],
+                                                     static_cast<uint32_t>((hx ? loads1 : loads0) - 1) & 1u, lim);
+                                if (good && c == 0 && w == 0 && s == 0 && n_acc >= R)
+                                    good = mbar_wait(&acc_empty[n_acc % R],
+                                                     static_cast<uint32_t>((n_acc / R) - 1) & 1u, lim);
+                                if (good)
+                                    good = mbar_wait(&a_full[ja % kAStages],
+                                                     static_cast<uint32_t>(ja / kAStages) & 1u, lim);
+                                mma_abort[ja & 1] = good ? 0u : 1u;
+                            }
+                            seen0 = seen0 || hx == 0;
+                            seen1 = seen1 || hx == 1;
+                            named_bar_sync(kMmaBar, 64);
+                            if (__shfl_sync(0xffffffffu, good ? 1 : 0, 0) == 0) {
+                                ok = false;
+                                break;
+                            }
                         }
                     }
                 }
@@ -500,51 +536,62 @@ __global__ void __launch_bounds__(kPlThreads, 1)
         for (int i = i_first; i < i_last && !abort; ++i) {
             const Item it = item_at(P, i);
             const PlProj &p = it.p;
-            const int c = it.chunk;
-            const int nw = slots_in_chunk(p, c);
-            for (int tt = 0; tt < it.ntiles && !abort; ++tt) {
-                const int n_acc = ntile + tt;
-                const uint32_t d = tmem + static_cast<uint32_t>((n_acc % R) * BNp);
-                for (int w = 0; w < nw && !abort; ++w) {
-                    int k0;
-                    const int nsteps = slot_len(p, c, w, k0) / 64;
-                    const int atom0 = (k0 - c * kXChunk) / 64;
-                    for (int s = 0; 2 * s < nsteps; ++s, ++ja) {
-                        named_bar_sync(kMmaBar, 64);
-                        if (mma_abort[ja & 1]) {
-                            abort = true;
-                            break;
-                        }
-                        // the whole warp walks the loop; one elected lane issues
-                        tc_fence_after_sync();
-                        const int st = ja & (kAStages - 1);
-                        const uint32_t a = tmem + kAOff + static_cast<uint32_t>(st) * kAStageCols;
-                        const uint64_t b0 = xdesc0 + static_cast<uint64_t>(atom0 + 2 * s) * atom_desc;
-                        const uint32_t acc0 = (w == 0 && s == 0) ? 0u : 1u;
-                        const bool two = 2 * s + 1 < nsteps;
-                        if (elect_one()) {
-#pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                tc_mma_f16kind_ts(d, a + 8 * kk, b0 + 2 * kk, idesc, kk == 0 ? acc0 : 1u);
-                            if (two) {
+            // does the next item start a different use of the X buffer?
+            bool next_same_x = false;
+            if (i + 1 < i_last) {
+                const PlItem &nx = P.items[i + 1];
+                next_same_x = P.proj[nx.proj].xid == p.xid;
+            }
+            for (int c = 0; c < it.nchunks && !abort; ++c) {
+                const int nw = slots_in_chunk(p, c);
+                // this (item, chunk) ends its use of the X buffer, and another use follows
+                const bool use_ends = c + 1 < it.nchunks || (i + 1 < i_last && !(next_same_x && c == 0));
+                for (int tt = 0; tt < it.ntiles && !abort; ++tt) {
+                    const int n_acc = ntile + tt;
+                    const uint32_t d = tmem + static_cast<uint32_t>((n_acc % R) * BNp);
+                    const bool release = use_ends && tt + 1 == it.ntiles;
+                    for (int w = 0; w < nw && !abort; ++w) {
+                        int k0;
+                        const int nsteps = slot_len(p, c, w, k0) / 64;
+                        const int atom0 = (k0 - c * kXChunk) / 64;
+                        for (int s = 0; 2 * s < nsteps; ++s, ++ja) {
+                            named_bar_sync(kMmaBar, 64);
+                            if (mma_abort[ja & 1]) {
+                                abort = true;
+                                break;
+                            }
+                            // the whole warp walks the loop; one elected lane issues
+                            tc_fence_after_sync();
+                            const int st = ja & (kAStages - 1);
+                            const uint32_t a = tmem + kAOff + static_cast<uint32_t>(st) * kAStageCols;
+                            const int atom = atom0 + 2 * s;
+                            const uint64_t b0 = xdesc0 + static_cast<uint64_t>(atom) * atom_desc;
+                            const uint32_t acc0 = (c == 0 && w == 0 && s == 0) ? 0u : 1u;
+                            const bool two = 2 * s + 1 < nsteps;
+                            // last stage on this half of the buffer in the use: the
+                            // next stage is in the other half, or the tile ends
+                            const int hx = atom >= 4 ? 1 : 0;
+                            const bool tile_end = 2 * s + 2 >= nsteps && w + 1 == nw;
+                            const int next_atom = 2 * s + 2 < nsteps ? atom + 2 : (w + 1) * slot_k(p.fmt) / 64;
+                            const bool half_end = tile_end || (next_atom >= 4 ? 1 : 0) != hx;
+                            if (elect_one()) {
 #pragma unroll
                                 for (int kk = 0; kk < 4; ++kk)
-                                    tc_mma_f16kind_ts(d, a + 32 + 8 * kk, b0 + atom_desc + 2 * kk, idesc, 1u);
+                                    tc_mma_f16kind_ts(d, a + 8 * kk, b0 + 2 * kk, idesc, kk == 0 ? acc0 : 1u);
+                                if (two) {
+#pragma unroll
+                                    for (int kk = 0; kk < 4; ++kk)
+                                        tc_mma_f16kind_ts(d, a + 32 + 8 * kk, b0 + atom_desc + 2 * kk, idesc, 1u);
+                                }
+                                tc_commit(&a_empty[st]);
+                                if (release && half_end) tc_commit(&x_empty[hx]);
                             }
-                            tc_commit(&a_empty[st]);
+                            __syncwarp();
                         }
-                        __syncwarp();
                     }
+                    if (!abort && c + 1 == it.nchunks && elect_one()) tc_commit(&acc_full[n_acc % R]);
+                    __syncwarp();
                 }
-                if (!abort && elect_one()) tc_commit(&acc_full[n_acc % R]);
-                __syncwarp();
-            }
-            // release the activation chunk once its MMAs complete if the next
-            // item reads a different (activations, chunk)
-            if (!abort && i + 1 < i_last) {
-                const PlItem &nx = P.items[i + 1];
-                if (!(P.proj[nx.proj].xid == p.xid && nx.chunk == c) && elect_one()) tc_commit(x_empty);
-                __syncwarp();
             }
             ntile += it.ntiles;
         }
@@ -568,13 +615,11 @@ __global__ void __launch_bounds__(kPlThreads, 1)
         // Thread 0 of the epilogue waits for each accumulator and shares the
         // outcome through named barrier kEpiBar, so the eight warps always
         // take the same branch and meet at the same barriers.
-        volatile uint32_t *last_flag = tmem_slot + 3;
         volatile uint32_t *full_flag = tmem_slot + 4;       // two, by tile parity
         int ntile = 0;
         for (int i = i_first; i < i_last && ok; ++i) {
             const Item it = item_at(P, i);
             const PlProj &p = it.p;
-            const bool split = it.nchunks > 1;
             for (int tt = 0; tt < it.ntiles && ok; ++tt, ++ntile) {
                 const int slot = ntile % R;
                 if (et == 0)
@@ -585,94 +630,27 @@ __global__ void __launch_bounds__(kPlThreads, 1)
                 ok = full_flag[ntile & 1] != 0;
                 if (!ok) break;
                 tc_fence_after_sync();
-                const int tile = it.tile0 + tt;
-                const int o = tile * 128 + row;
+                const int o = (it.tile0 + tt) * 128 + row;
                 const uint32_t tacc = tq + static_cast<uint32_t>(slot * BNp + c0);
-                if (!split) {
-                    float sc = 1.f, b = 0.f;
-                    if (p.fmt == 8 && o < p.N) sc = __ldg(static_cast<const float *>(p.S) + o);
-                    if (p.bias && o < p.N) b = __ldg(p.bias + o);
-                    float *yo = p.Y + o;
-                    const size_t rs = static_cast<size_t>(p.N);
-                    for (int cc = 0; cc < cols; cc += 8) {
-                        uint32_t v[8];
-                        tmem_ld_x8(tacc + static_cast<uint32_t>(cc), v);
-                        tmem_ld_wait();
-                        if (o < p.N) {
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                const int m = c0 + cc + e;
-                                if (m < M) yo[static_cast<size_t>(m) * rs] = fmaf(__uint_as_float(v[e]), sc, b);
-                            }
-                        }
-                    }
-                    tc_fence_before_sync();
-                    mbar_arrive(&acc_empty[slot]);
-                    continue;
-                }
-                // Split tile: this chunk's partial goes to its slot of the
-                // partials, column-major ([m][row]) so a warp writes 128
-                // contiguous bytes per column; the accumulator is free then.
-                const int st = p.sbase + tile;
-                float *part = P.partials +
-                              static_cast<size_t>(st * P.max_chunks + it.chunk) * BNp * 128;
+                float sc = 1.f, b = 0.f;
+                if (p.fmt == kFmtQ8 && o < p.N) sc = __ldg(static_cast<const float *>(p.S) + o);
+                if (p.bias && o < p.N) b = __ldg(p.bias + o);
+                float *yo = p.Y + o;
+                const size_t rs = static_cast<size_t>(p.N);
                 for (int cc = 0; cc < cols; cc += 8) {
                     uint32_t v[8];
                     tmem_ld_x8(tacc + static_cast<uint32_t>(cc), v);
                     tmem_ld_wait();
+                    if (o < p.N) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        __stcg(part + static_cast<size_t>(c0 + cc + e) * 128 + row, __uint_as_float(v[e]));
+                        for (int e = 0; e < 8; ++e) {
+                            const int m = c0 + cc + e;
+                            if (m < M) yo[static_cast<size_t>(m) * rs] = fmaf(__uint_as_float(v[e]), sc, b);
+                        }
+                    }
                 }
                 tc_fence_before_sync();
                 mbar_arrive(&acc_empty[slot]);
-                // The last chunk to finish sums the partials in chunk order
-                // (the same order whichever CTA it is) and writes Y.
-                __threadfence();
-                named_bar_sync(kEpiBar, kEpiThreads);
-                if (et == 0) {
-                    const unsigned done = atomicAdd(P.counters + st, 1u);
-                    *last_flag = (done == static_cast<unsigned>(it.nchunks - 1)) ? 1u : 0u;
-                }
-                named_bar_sync(kEpiBar, kEpiThreads);
-                if (*last_flag) {
-                    __threadfence();
-                    if (o < p.N) {
-                        const float sc = p.fmt == 8 ? __ldg(static_cast<const float *>(p.S) + o) : 1.f;
-                        const float b = p.bias ? __ldg(p.bias + o) : 0.f;
-                        const float *p0 = P.partials +
-                                          static_cast<size_t>(st * P.max_chunks) * BNp * 128 + row;
-                        const size_t cstride = static_cast<size_t>(BNp) * 128;
-                        for (int mb = c0; mb < c0 + cols && mb < M; mb += 8) {
-                            // up to 4 chunks x 8 columns of loads in flight, then
-                            // the sums in chunk order
-                            float acc[8];
-                            for (int cb = 0; cb < it.nchunks; cb += 4) {
-                                float v[4][8];
-#pragma unroll
-                                for (int u = 0; u < 4; ++u)
-#pragma unroll
-                                    for (int e = 0; e < 8; ++e)
-                                        v[u][e] = cb + u < it.nchunks
-                                                      ? __ldcg(p0 + (cb + u) * cstride +
-                                                               static_cast<size_t>(mb + e) * 128)
-                                                      : 0.f;
-#pragma unroll
-                                for (int u = 0; u < 4; ++u)
-#pragma unroll
-                                    for (int e = 0; e < 8; ++e)
-                                        if (cb + u < it.nchunks)
-                                            acc[e] = (cb + u == 0) ? v[u][e] : acc[e] + v[u][e];
-                            }
-#pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                if (mb + e < M)
-                                    p.Y[static_cast<size_t>(mb + e) * p.N + o] = fmaf(acc[e], sc, b);
-                        }
-                    }
-                    if (et == 0) P.counters[st] = 0u;      // ready for the next launch
-                }
-                named_bar_sync(kEpiBar, kEpiThreads);      // last_flag is read by all
             }
         }
     }
@@ -699,8 +677,6 @@ __global__ void __launch_bounds__(256)
     // own wait for this grid's completion.
     pdl_launch_dependents();
     pdl_wait_prior_grid();
-    if (blockIdx.x == 0 && blockIdx.y == 0)
-        for (int i = threadIdx.x; i < P.n_counters; i += blockDim.x) P.counters[i] = 0u;
     const PlPrepImage &im = P.img[blockIdx.y];
     const int BNp = P.bnp, M = P.M, K = im.K;
     const int64_t pieces = static_cast<int64_t>(K / 8) * BNp;   // 16-byte output pieces
@@ -776,18 +752,19 @@ int pl_nslots(int bnp) {
 namespace {
 
 // Tiles per work item: up to about 80 KB of packed weights (two q4 tiles of
-// a 512-wide chunk, one q8 or e4m3 tile), small against a CTA's share of a
-// list so that the runs cut from the sorted items come out nearly equal.
+// K = 512, one q8 or e4m3 tile), small against a CTA's share of a list so
+// that the runs cut from the sorted items come out nearly equal.  With
+// K > 512 an item is one tile: its accumulator stays in TMEM over all chunks.
 int tiles_per_item(int fmt, int K) {
-    const int klen = std::min(K, kXChunk);
-    const double tile = 128.0 * klen * (fmt == 4 ? 0.625 : 1.0);
+    if (K > kXChunk) return 1;
+    const double tile = 128.0 * K * (fmt == 4 ? 0.625 : 1.0);
     return std::max(1, std::min(4, static_cast<int>(80.0 * 1024 / tile)));
 }
 
 int64_t items_of(int fmt, int64_t N, int K) {
     const int64_t tiles = (N + 127) / 128;
     const int per = tiles_per_item(fmt, K);
-    return static_cast<int64_t>((K + kXChunk - 1) / kXChunk) * ((tiles + per - 1) / per);
+    return (tiles + per - 1) / per;
 }
 
 }  // namespace
@@ -804,17 +781,13 @@ namespace {
 int64_t pl_image_bytes(int M, int K) { return static_cast<int64_t>(pl_bnp(M)) * K * 2; }
 
 // Workspace of a list call: the distinct activation images ((X, K) -> image
-// index, in order of first appearance), then the partial tiles and counters
-// of the projections with K > 512 ("split" tiles, one partial per 512-wide K
-// chunk).
+// index, in order of first appearance).
 struct Plan {
     std::vector<int> xid;            // per projection
-    std::vector<int> sbase;          // per projection: first split-tile index, or -1
     std::vector<const float *> X;    // per image
     std::vector<int> K;
     std::vector<size_t> off;
-    int n_split = 0, max_chunks = 1;
-    size_t partials_off = 0, counters_off = 0, bytes = 0;
+    size_t bytes = 0;
 };
 
 constexpr size_t align256(size_t b) { return (b + 255) / 256 * 256; }
@@ -822,7 +795,6 @@ constexpr size_t align256(size_t b) { return (b + 255) / 256 * 256; }
 Plan plan_list(const PlInput *in, int count, int M) {
     Plan pl;
     pl.xid.resize(count);
-    pl.sbase.assign(count, -1);
     size_t img = 0;
     for (int i = 0; i < count; ++i) {
         int found = -1;
@@ -836,17 +808,8 @@ Plan plan_list(const PlInput *in, int count, int M) {
             img += align256(static_cast<size_t>(pl_image_bytes(M, in[i].K)));
         }
         pl.xid[i] = found;
-        const int nchunks = (in[i].K + kXChunk - 1) / kXChunk;
-        if (nchunks > 1) {
-            pl.sbase[i] = pl.n_split;
-            pl.n_split += (in[i].N + 127) / 128;
-            pl.max_chunks = std::max(pl.max_chunks, nchunks);
-        }
     }
-    pl.partials_off = img;
-    const size_t part = static_cast<size_t>(pl.n_split) * pl.max_chunks * pl_bnp(M) * 128 * 4;
-    pl.counters_off = align256(pl.partials_off + part);
-    pl.bytes = align256(pl.counters_off + static_cast<size_t>(pl.n_split) * 4);
+    pl.bytes = img;
     return pl;
 }
 
@@ -906,16 +869,12 @@ cudaError_t launch_pl_batch(const PlInput *in, int count, int M, void *ws, DevCt
     const int bnp = pl_bnp(M), nacc = pl_nacc(bnp), nslots = pl_nslots(bnp);
     const Plan pl = plan_list(in, count, M);
     uint8_t *wsb = static_cast<uint8_t *>(ws);
-    unsigned *counters = reinterpret_cast<unsigned *>(wsb + pl.counters_off);
 
-    // 1. every distinct activation block once into its fp16 image; the first
-    // pre-pass launch also zeroes the split tiles' counters
+    // 1. every distinct activation block once into its fp16 image
     for (size_t i0 = 0; i0 < pl.X.size(); i0 += kPlMaxProj) {
         thread_local PlPrep prep;   // large: kept off the stack; a launch copies it
         prep.M = M;
         prep.bnp = bnp;
-        prep.counters = counters;
-        prep.n_counters = i0 == 0 ? pl.n_split : 0;
         const int n = static_cast<int>(std::min<size_t>(kPlMaxProj, pl.X.size() - i0));
         int max_k = 0;
         for (int j = 0; j < n; ++j) {
@@ -941,29 +900,25 @@ cudaError_t launch_pl_batch(const PlInput *in, int count, int M, void *ws, DevCt
             const int src = order[pos];
             const PlInput &q = in[src];
             const int tiles = (q.N + 127) / 128;
-            const int nchunks = (q.K + kXChunk - 1) / kXChunk;
             const int per = tiles_per_item(q.fmt, q.K);
-            const int n_items = nchunks * ((tiles + per - 1) / per);
+            const int n_items = (tiles + per - 1) / per;
             if (n_items > kPlMaxItems) return cudaErrorInvalidValue;   // not pl_supported
             if (np > 0 && items.size() + n_items > static_cast<size_t>(kPlMaxItems)) break;
             if (!weight_map(&P.wmap[np], 0, q.fmt, q.Wq, q.N, q.K) ||
                 (q.fmt == 4 && !weight_map(&P.smap[np], 1, q.fmt, q.S, q.N, q.K)))
                 return cudaErrorInvalidValue;
             P.proj[np] = {wsb + pl.off[pl.xid[src]], q.Wq, q.S, q.bias, q.Y, q.N, q.K, q.fmt,
-                          pl.xid[src], pl.sbase[src]};
-            for (int c = 0; c < nchunks; ++c) {
-                const int klen = std::min(kXChunk, q.K - c * kXChunk);
-                for (int t = 0; t < tiles; t += per) {
-                    const int nt = std::min(per, tiles - t);
-                    items.push_back({static_cast<uint32_t>(t), static_cast<uint16_t>(np),
-                                     static_cast<uint8_t>(nt), static_cast<uint8_t>(c)});
-                    const int rows = std::min(nt * 128, q.N - t * 128);
-                    cost.push_back(static_cast<double>(rows) * klen * (q.fmt == 4 ? 0.625 : 1.0));
-                }
+                          pl.xid[src], 0};
+            for (int t = 0; t < tiles; t += per) {
+                const int nt = std::min(per, tiles - t);
+                items.push_back({static_cast<uint32_t>(t), static_cast<uint16_t>(np),
+                                 static_cast<uint8_t>(nt), 0});
+                const int rows = std::min(nt * 128, q.N - t * 128);
+                cost.push_back(static_cast<double>(rows) * q.K * (q.fmt == 4 ? 0.625 : 1.0));
             }
         }
-        // items in (activation image, K chunk, projection, tile) order, cut
-        // into G contiguous runs of about equal bytes
+        // items in (activation image, projection, tile) order, cut into G
+        // contiguous runs of about equal bytes
         const int n_items = static_cast<int>(items.size());
         const int G = std::min(sms, n_items);
         std::vector<int> order_it(n_items);
@@ -971,7 +926,6 @@ cudaError_t launch_pl_batch(const PlInput *in, int count, int M, void *ws, DevCt
         std::stable_sort(order_it.begin(), order_it.end(), [&](int a, int c) {
             const PlItem &x = items[a], &y = items[c];
             if (P.proj[x.proj].xid != P.proj[y.proj].xid) return P.proj[x.proj].xid < P.proj[y.proj].xid;
-            if (x.chunk != y.chunk) return x.chunk < y.chunk;
             if (x.proj != y.proj) return x.proj < y.proj;
             return x.tile0 < y.tile0;
         });
@@ -996,10 +950,6 @@ cudaError_t launch_pl_batch(const PlInput *in, int count, int M, void *ws, DevCt
         P.bnp = bnp;
         P.nslots = nslots;
         P.nacc = nacc;
-        P.partials = reinterpret_cast<float *>(wsb + pl.partials_off);
-        P.counters = counters;
-        P.max_chunks = pl.max_chunks;
-        P.pad = 0;
         if ((e = launch_pl(P, G, ctl, s)) != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -22,19 +22,17 @@ struct PlProj {
     const float *bias;   // fp32 [N] or null
     float *Y;            // fp32 [M, N]
     int N, K, fmt, xid;  // xid: index of the distinct activation image
-    int sbase;           // K > 512: index of its first tile among the launch's
-                         // split tiles (partials and counters); else -1
+    int pad;
 };
 
-// One work item: tiles [tile0, tile0 + ntiles) of a projection over one
-// 512-wide K chunk.  A projection with K <= 512 has one chunk and its items
-// write Y; with K > 512 every chunk is a separate item that writes a partial
-// tile, and the last of a tile's chunks to finish sums them into Y.
+// One work item: tiles [tile0, tile0 + ntiles) of a projection over all of
+// K, 512-wide chunk by chunk.  A projection with K > 512 has one tile per
+// item, its accumulator kept in TMEM across the chunks.
 struct PlItem {
     uint32_t tile0;
     uint16_t proj;       // index into PlParams::proj
     uint8_t ntiles;
-    uint8_t chunk;
+    uint8_t pad;
 };
 
 struct PlParams {
@@ -44,10 +42,6 @@ struct PlParams {
     CUtensorMap wmap[kPlMaxProj];
     CUtensorMap smap[kPlMaxProj];
     int M, bnp, nslots, nacc;
-    float *partials;     // split tiles: [tile][chunk][BNp][128] fp32
-    unsigned *counters;  // split tiles: chunks finished (reset to 0 by the last)
-    int max_chunks;      // chunk stride of `partials`
-    int pad;
     int cta_items[kPlMaxCtas + 1];   // CTA b runs items [cta_items[b], cta_items[b + 1])
     PlProj proj[kPlMaxProj];
     PlItem items[kPlMaxItems];
@@ -61,8 +55,6 @@ struct PlPrepImage {
 
 struct PlPrep {
     int M, bnp;
-    unsigned *counters;  // split-tile counters of the call, zeroed by the pre-pass
-    int n_counters, pad;
     PlPrepImage img[kPlMaxProj];
 };
 
