@@ -29,13 +29,20 @@ Other workloads (`--workload`), each printing one line of the same form:
                roofline object then describes that launch) and at M = 2048.
   rot_m80      small M as an aggregate weight stream: the 12 blocks' weights in
                rotating device copies totalling ~4x L2, every copy's projection
-               set at M = 80, replayed from a CUDA graph; value in GB/s of
-               quantized weights.
-  m_sweep      M in {1, 16, 80, 512, 4096, 65536} for the q4 512->2048 and q8
-               2048->512 shapes under the automatic dispatch; value = TFLOP/s
-               of the q4 shape at M = 65536, every point under `sweep`.
+               set at M = 80, 16 copies (64 projections) per rt_qgemm_batch
+               call, the step's calls replayed from a CUDA graph; value in GB/s
+               of quantized weights.
+  m_sweep      M in {1, 2, 4, 8, 16, 32, 80, 512, 4096, 65536} for the q4
+               512->2048 and q8 2048->512 shapes on the SIMT path, the
+               tensor-core path and RT_PATH_AUTO; value = TFLOP/s of the q4
+               shape at M = 65536, every point under `sweep`, the measured
+               crossover under `crossover`.
   w13_m4096, w2_m4096, qkvg_m4096, w13_m16384, w2_m16384
                single projections, sized for profiler captures.
+  blocks12_q8_m4096, block_q8_m80
+               the all-int8 recipe of the int8 card (every projection q8,
+               fused qkvg and w13 included) on the 12 blocks at M = 4096 and
+               on one block at M = 80 (rt_qblock_project_fmt).
 
 Multi-GPU (torchrun): every rank runs the same step on its own batch (replica
 weights, rank-seeded activations, no data-path collective) -> weak scaling.
@@ -82,12 +89,20 @@ WORKLOADS = {
     # outputs larger than L2, for full profiler captures of one launch
     "w13_m16384": (4, 1, 16384, ("w13",)),
     "w2_m16384": (4, 1, 16384, ("w2",)),
+    # the int8 card's all-int8 recipe: every projection q8 (fused qkvg and w13 too)
+    "blocks12_q8_m4096": (4, 12, 4096, ("qkvg", "wo", "w13", "w2")),
+    "block_q8_m80": (3, 1, 80, ("qkvg", "wo", "w13", "w2")),
 }
+
+# Workloads that store every projection in one format instead of the mixed
+# recipe; proj_dims reports the format in force for this process's workload.
+ALL_FORMAT = {"blocks12_q8_m4096": "q8", "block_q8_m80": "q8"}
+FORMAT_OVERRIDE = {}
 
 
 def proj_dims(name):
     spec = wl.BLOCK_PROJECTIONS[name]
-    return spec["fmt"], spec["N"], spec["K"]
+    return FORMAT_OVERRIDE.get(name, spec["fmt"]), spec["N"], spec["K"]
 
 
 def weight_bytes(name):
@@ -215,7 +230,7 @@ def build_host(workload, rank, use_oracle_quantizer=False):
     for b in range(nblocks):
         blk = {}
         for name in projs:
-            fmt = wl.BLOCK_PROJECTIONS[name]["fmt"]
+            fmt = proj_dims(name)[0]
             W = wl.projection_weights(cfg, b, name)
             blk[name] = q4(W) if fmt == "q4" else q8(W)
             # replicas: same weights, rank-specific activations
@@ -750,19 +765,28 @@ def run_gpu(args, rank, world, local_rank):
                                      M, N, K, 0, sptr)))
         dblocks.append(db)
     full_block = tuple(projs) == ("qkvg", "wo", "w13", "w2")
+    # the mixed recipe goes through rt_qblock_project, a one-format workload
+    # through rt_qblock_project_fmt
+    per_fmt = bool(FORMAT_OVERRIDE)
     block_args = []
     if full_block:
         for db in dblocks:
-            c = rtq._QBlockC(*(t.data_ptr() for t in (db["qkvg"][0], db["qkvg"][1], db["wo"][0],
-                                                      db["wo"][1], db["w13"][0], db["w13"][1],
-                                                      db["w2"][0], db["w2"][1])),
-                             wl.D_MODEL, wl.D_FF)
+            if per_fmt:
+                ws = [rtq._QWeightC(4 if proj_dims(n)[0] == "q4" else 8, 0, db[n][0].data_ptr(),
+                                    db[n][1].data_ptr(), None) for n in projs]
+                c = rtq._QBlockFmtC(*ws, wl.D_MODEL, wl.D_FF)
+            else:
+                c = rtq._QBlockC(*(t.data_ptr() for t in (db["qkvg"][0], db["qkvg"][1],
+                                                          db["wo"][0], db["wo"][1], db["w13"][0],
+                                                          db["w13"][1], db["w2"][0], db["w2"][1])),
+                                 wl.D_MODEL, wl.D_FF)
             block_args.append((c, [db[n][2].data_ptr() for n in projs] +
                                [db[n][3].data_ptr() for n in projs]))
+    block_fn = L.rt_qblock_project_fmt if per_fmt else L.rt_qblock_project
 
     def run_block(i):
         c, ptrs = block_args[i]
-        st = L.rt_qblock_project(ctypes.byref(c), M, *ptrs, 0, sptr)
+        st = block_fn(ctypes.byref(c), M, *ptrs, 0, sptr)
         if st:
             raise rtq.RtqError(st, "rt_qblock_project")
 
@@ -778,7 +802,10 @@ def run_gpu(args, rank, world, local_rank):
 
     # the TMA-fed kernels add an activation pre-pass launch; the block driver
     # runs a small-M block as one grouped launch
-    fused_block = full_block and rtq.block_fused(M, wl.D_MODEL, wl.D_FF) == 1
+    if full_block and per_fmt:
+        fused_block = L.rt_qblock_fused_fmt(ctypes.byref(block_args[0][0]), M, 0) == 1
+    else:
+        fused_block = full_block and rtq.block_fused(M, wl.D_MODEL, wl.D_FF) == 1
     if fused_block:
         launches_per_step = nblocks
     else:
@@ -1010,6 +1037,8 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.workload in ALL_FORMAT:
+        FORMAT_OVERRIDE.update({p: ALL_FORMAT[args.workload] for p in wl.BLOCK_PROJECTIONS})
     if args.impl == "reference":
         run_reference(args, rank, world)
         return

@@ -23,8 +23,8 @@
  *         Wq    int8  [N, K], row-major
  *         scale float [N]
  *
- *   e4m3 ("RT-J -- FP8 E4M3 checkpoints", section "FP8 Format"): every weight
- *       stored directly as PyTorch float8_e4m3fn, no scale: sign, 4 exponent
+ *   e4m3 ("RT-J -- FP8 E4M3 checkpoints", section "FP8 Format"): each weight
+ *       matrix holds float8_e4m3fn values as they are, no scale: sign, 4 exponent
  *       bits (bias 7), 3 mantissa bits, subnormals m * 2^-9, largest 448; the
  *       codes S.1111.111 are NaN in the format and are not weights (the GEMM
  *       kernels read them as +-480).
@@ -257,13 +257,13 @@ rt_status rt_qgemm_noalloc(int fmt, const float *X, const void *Wq, const void *
  * multiple of 128 (q4) or 64 (q8 and e4m3) and every q4 scale_min 16-byte
  * aligned, the list runs as RT_KERNEL_TC_LIST: one pre-pass launch rounds
  * each distinct (X, K) once to fp16 into the stream's workspace, then
- * persistent launches of up to 256 entries each stream the entries' weights
- * through every SM.  An entry with K > 512 is computed in 512-wide K chunks
- * whose fp32 partial tiles are summed in chunk order (deterministically) by
- * whichever chunk finishes last.  Workspace (rt_workspace_reserve applies):
- * per distinct (X, K) M16 * K * 2 bytes, plus for the entries with K > 512
- * ceil(N / 128) * ceil(K / 512) * M16 * 512 bytes of partials, with M16 = M
- * rounded up to 16 (a few more bytes for counters and alignment).  Under
+ * persistent launches of up to 64 entries each stream the entries' weights
+ * through every SM.  Each 128-row tile of an entry is computed over all of K
+ * by one CTA (K > 512 in 512-wide chunks into one accumulator), so results
+ * are deterministic.  Workspace (rt_workspace_reserve applies): per distinct
+ * (X, K) M16 * K * 2 bytes (256-byte aligned), with M16 = M rounded up to 16.
+ * The host encodes a TMA tensor map per entry's weights (cached per thread
+ * by pointer and shape); Wq must be 16-byte aligned.  Under
  * RT_PATH_AUTO this happens only when the entries hold at least as many
  * 128-row weight tiles as the GPU has SMs.  Otherwise the entries run one
  * after another as rt_qgemm_q4/q8 calls.  Results are those of the
@@ -403,8 +403,8 @@ rt_status rt_quantize_q4_g32(const float *W, int64_t N, int64_t K, int n_grid,
 rt_status rt_quantize_q8_row(const float *W, int64_t N, int64_t K, int8_t *Wq, float *scale);
 
 /*
- * rt_quantize_e4m3 (FP8 card, "FP8 Format": weights stored directly as
- * float8_e4m3fn): each of the n weights to the nearest E4M3 value, ties to
+ * rt_quantize_e4m3 (FP8 card, "FP8 Format": weight matrices hold
+ * float8_e4m3fn values, no scale): each of the n weights to the nearest E4M3 value, ties to
  * the even code, the same rounding as PyTorch's float8_e4m3fn cast.  W fp32
  * [n] -> codes uint8 [n].  Errors: RT_ERR_INVALID_ARG, RT_ERR_VALUE_RANGE (a
  * weight is NaN or |w| > 464, which would round past 448; out is then
@@ -462,9 +462,9 @@ rt_status rt_device_status(void *stream, int *device_status);
 rt_status rt_debug_inject(int mode, int64_t wait_ns);
 
 /*
- * Quantized checkpoints.  Both quantized cards ship plain safetensors files
- * ("Plain safetensors -- no custom container") that the engine's loader takes
- * directly, "the format is auto-detected from the tensor dtypes"; the FP8 card
+ * Quantized checkpoints.  Both quantized cards ship their checkpoints as
+ * ordinary safetensors files, which the engine's loader reads without
+ * conversion, telling the format from the tensors' dtypes; the FP8 card
  * stores float8_e4m3fn weights the same way.  These calls read such a file
  * on the host (the model cards have no other interface to match):
  *

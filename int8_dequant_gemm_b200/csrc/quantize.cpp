@@ -6,8 +6,8 @@
 //   a min-MSE clip search over the shrink grid 1.0 -> 0.8.
 // q8 per-row: "RT-J -- int8 (Q8_0-style) quantized checkpoints", section
 //   "Quantization format" -- scale[o] = max|W[o,:]|/127, W ~= q*scale[o].
-// e4m3: "RT-J -- FP8 E4M3 checkpoints", section "FP8 Format" -- every weight
-//   stored directly as float8_e4m3fn, no scale.
+// e4m3: "RT-J -- FP8 E4M3 checkpoints", section "FP8 Format" -- weight
+//   matrices hold float8_e4m3fn values, no scale.
 //
 // The grid, rounding and tie rules are spelled out in include/rtq.h.  All
 // weight arithmetic is IEEE double with no contraction (this file is built

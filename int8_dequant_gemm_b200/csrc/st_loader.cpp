@@ -1,8 +1,8 @@
-// Reader of quantized checkpoints in the plain safetensors container, with
-// the weight format auto-detected from the tensor dtypes.
+// Reader of quantized checkpoints in the plain safetensors container; the
+// weight format follows from the tensors' dtypes.
 //
-// Container (the format the checkpoints use, "Plain safetensors -- no custom
-// container" on both quantized cards): an 8-byte little-endian header length
+// Container (the standard safetensors layout, which both quantized cards use
+// with nothing of their own added): an 8-byte little-endian header length
 // n, n bytes of JSON mapping each tensor name to {"dtype", "shape",
 // "data_offsets": [begin, end]} (plus an optional "__metadata__" object of
 // strings), then the tensors' bytes; offsets count from the end of the

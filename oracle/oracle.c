@@ -16,9 +16,8 @@
  *   [Q8]  "RT-J -- int8 (Q8_0-style) quantized checkpoints", section
  *         "Quantization format": int8 codes with one symmetric fp32 scale per
  *         output row, W[o,i] ~= q[o,i] * scale[o], scale[o] = max|W[o,:]|/127.
- *   [F8]  "RT-J -- FP8 E4M3 checkpoints", section "FP8 Format": every
- *         two-dimensional matrix weight is stored directly as PyTorch
- *         float8_e4m3fn (no scale).
+ *   [F8]  "RT-J -- FP8 E4M3 checkpoints", section "FP8 Format": each 2-D
+ *         weight matrix holds float8_e4m3fn values as they are (no scale).
  *   [GEMM] Both cards, opening paragraph: the engine dequantizes inside the
  *         GEMM; the projection computes Y = X * W^T with W indexed [out, in].
  *
@@ -286,7 +285,7 @@ int oracle_e4m3_from_double(double x, uint8_t *out)
     return 0;
 }
 
-/* [F8]: each weight stored directly as its E4M3 rounding.  Returns -1 (and
+/* [F8]: each weight kept as its E4M3 rounding.  Returns -1 (and
  * leaves the rest of `out` unspecified) at the first weight out of range. */
 int oracle_quant_e4m3(const float *W, int64_t n, uint8_t *out)
 {

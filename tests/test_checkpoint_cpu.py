@@ -1,6 +1,6 @@
-"""Quantized checkpoints in plain safetensors (the cards' "Plain safetensors --
-no custom container"), read by the library's rt_st_* calls with the format
-detected from the tensor dtypes.  Files are written here by the independent
+"""Quantized checkpoints in ordinary safetensors files (the int4 and int8
+cards use the standard container, nothing of their own), read by the
+library's rt_st_* calls with the format detected from the tensor dtypes.  Files are written here by the independent
 `safetensors` package from tensors the library's own quantizers produce; the
 reader must return the same bytes and the right format and sizes, and refuse
 malformed files."""

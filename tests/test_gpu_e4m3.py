@@ -1,5 +1,5 @@
-"""FP8 E4M3 weights ("RT-J -- FP8 E4M3 checkpoints", "FP8 Format": every
-matrix weight stored directly as float8_e4m3fn) on a GPU, through the C ABI.
+"""FP8 E4M3 weights ("RT-J -- FP8 E4M3 checkpoints", "FP8 Format": weight
+matrices hold float8_e4m3fn values, no scale) on a GPU, through the C ABI.
 
   - dequantization exports: every finite code to its exact value, in fp32
     and in fp16 (the tensor-core operand), bit for bit against the oracle;
