@@ -168,6 +168,25 @@ __device__ __forceinline__ void load_scale_words(uint32_t row, int r, int h, uin
     }
 }
 
+// The (scale, min) words of row r for 8 K steps when thread (r, h) converts
+// whole steps (step 2i + h of each pair i): it keeps the words of that step's
+// two groups, 4i + 2h and 4i + 2h + 1, as sw[2i], sw[2i + 1].  Same rotated
+// reads as load_scale_words.
+__device__ __forceinline__ void load_scale_pairs(uint32_t row, int r, int h, uint32_t (&sw)[8]) {
+    const int rot = (r >> 1) & 3;
+    uint4 u[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) u[c] = lds_v4(row + ((c + rot) & 3) * 16);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int i0 = (k - 0) & 3, i1 = (k - 1) & 3, i2 = (k - 2) & 3, i3 = (k - 3) & 3;
+        const uint4 v = rot == 0 ? u[i0] : rot == 1 ? u[i1] : rot == 2 ? u[i2] : u[i3];
+        // chunk k = words 4k .. 4k + 3: step 2k (words 4k, 4k + 1), step 2k + 1
+        sw[2 * k] = h ? v.z : v.x;
+        sw[2 * k + 1] = h ? v.w : v.y;
+    }
+}
+
 // ---------------------------------------------------------------- host side
 // Row-major 2-D tensor [rows, cols] of `esize`-byte elements as a TMA map
 // with box {bcols, brows}; swizzle as given.  Returns false if the driver

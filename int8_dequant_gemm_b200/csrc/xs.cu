@@ -25,19 +25,19 @@
 //               128-row slice of packed codes, two K steps per TMA box
 //               (a box costs about the same per row at any width up to 256
 //               bytes), into a ring of kRaw such pairs.
-//   warps 0-7   dequantizers: thread (r, h) converts K values [32h, 32h + 32)
-//               of every K step of weight row r (16 or 32 bytes of codes) and
-//               writes them with tcgen05.st into TMEM lane r of the step's A
-//               stage (16 of its 32 columns).  All 256 threads work on the
-//               same step, so a stage is refilled quickly once the MMAs that
-//               read it complete.  The A operand never touches shared memory,
-//               which leaves its bandwidth to the MMA's activation reads and
-//               the TMA traffic.
-//   warp 8      MMA issuer (one thread): per weight tile, K/64 stages x 4
-//               tcgen05.mma (K = 16, A from TMEM, B from shared memory) into
-//               one of two TMEM accumulators.  It waits on no mbarrier.
+//   warps 0-7   dequantizers: an A stage holds a pair of 64-wide K steps
+//               (64 columns).  Thread (r, h) converts step h of every pair of
+//               weight row r (32 or 64 bytes of codes) and writes it with
+//               tcgen05.st into TMEM lane r of the pair's stage (32 of its 64
+//               columns), so one stage hand-over serves two K steps.  The A
+//               operand never touches shared memory, which leaves its
+//               bandwidth to the MMA's activation reads and the TMA traffic.
+//   warp 8      MMA issuer (the warp walks, an elected lane issues): per
+//               weight tile, K/128 stages x 8 tcgen05.mma (K = 16, A from
+//               TMEM, B from shared memory) into one of two TMEM
+//               accumulators.  It waits on no mbarrier.
 //   warp 19     MMA waiter: waits for each stage (and the activation block
-//               and accumulator) and hands the step to the issuer through a
+//               and accumulator) and hands the pair to the issuer through a
 //               named barrier.
 //   warps 9-16  epilogue, two warps per TMEM lane quadrant: TMEM ->
 //               registers (q8 row scale) -> fp32 Y with 128-byte coalesced
@@ -57,7 +57,7 @@ namespace {
 
 // MMA N.  An M = 128, K = 16 tcgen05.mma costs about the same time for any
 // N up to 192 and only a little more at 256, so the tile is as wide as TMEM
-// allows with two accumulators and the A stages: 2 x 192 + 4 x 32 = 512
+// allows with two accumulators and the A stages: 2 x 192 + 2 x 64 = 512
 // columns.  192 resident rows of K = 512 also just fit in shared memory.
 constexpr int kXsTileM = 192;                 // activation rows per block (MMA N)
 constexpr int kXsMaxK = 512;
@@ -76,10 +76,10 @@ constexpr int kWaitWarp = kXTmaWarp + 1;                 // 19
 constexpr int kXsThreads = (kWaitWarp + 1) * 32;         // 640
 constexpr uint32_t kMmaBar = 1;                          // named barrier: waiter <-> MMA warp
 constexpr int kXAtom = kXsTileM * 128;                   // 24 KB: 192 rows x 64 K
-constexpr int kAStages = 4;                              // A stages in TMEM, 32 columns each
+constexpr int kAStages = 2;                              // A stages in TMEM, two K steps each
 constexpr int kRaw = 2;                                  // packed-code ring depth (step pairs)
 constexpr uint32_t kAccCols = 2 * kXsTileM;              // 2 accumulators x 192 columns
-constexpr uint32_t kAStageCols = kAtomK / 2;             // 64 16-bit values per lane
+constexpr uint32_t kAStageCols = kAtomK;                 // 2 x 64 16-bit values per lane
 constexpr uint32_t kXsTmemCols = 512;                    // accumulators + A stages, pow2
 
 static_assert(kAccCols + kAStages * kAStageCols <= kXsTmemCols, "TMEM budget");
@@ -277,12 +277,13 @@ __global__ void __launch_bounds__(kXsThreads, 1)
         __syncwarp();
     } else if (warp < kDeqWarps) {
         // ============================================================ dequantizers
-        const int h = warp >> 2;                     // K half [32h, 32h + 32) of every step
+        const int h = warp >> 2;                     // step h of every step pair
         const int r = threadIdx.x & (kDeqThreads - 1);
         // this warp's 32 TMEM lanes (warp % 4 selects the lane quadrant) and
-        // its 16 columns of each 32-column A stage
+        // its 32 columns (one K step) of each 64-column A stage
         const uint32_t ta = tmem + kAccCols + (static_cast<uint32_t>((warp & 3) * 32) << 16) +
-                            static_cast<uint32_t>(16 * h);
+                            static_cast<uint32_t>(32 * h);
+        uint32_t jp = 0;                             // step pairs (A stages) so far
         for (ItemCursor it(first, last, n_o_tiles); it.valid() && ok; it.next()) {
             const int n_local = it.item - first;
             const int b = n_local & 1;
@@ -292,48 +293,42 @@ __global__ void __launch_bounds__(kXsThreads, 1)
                     ok = false;
                     break;
                 }
-                load_scale_words(base + L.sc_off + b * kScaleSlot + r * (kScaleWords * 4), r, h,
-                                 sw);
+                load_scale_pairs(base + L.sc_off + b * kScaleSlot + r * (kScaleWords * 4), r, h, sw);
                 // sw depends on every word read, so the reads have completed
                 fence_proxy_async_smem();
                 mbar_arrive(&sc_empty[b]);
             }
 #pragma unroll
-            for (int ks = 0; ks < kXsMaxK / kAtomK; ++ks) {
-                if (ks >= nk) break;
-                const int j = n_local * nk + ks;
-                const int jp = n_local * (nk / 2) + (ks >> 1);   // step pair of the raw ring
-                const int slot = jp % kRaw;
-                if ((ks & 1) == 0 &&
-                    !mbar_wait(&raw_full[slot], static_cast<uint32_t>(jp / kRaw) & 1u, lim)) {
+            for (int kp = 0; kp < kXsMaxK / kAtomK / 2; ++kp, ++jp) {
+                if (2 * kp >= nk) break;
+                const uint32_t jr = n_local * (nk / 2) + kp;          // step pair of the raw ring
+                const int slot = jr % kRaw;
+                if (!mbar_wait(&raw_full[slot], static_cast<uint32_t>(jr / kRaw) & 1u, lim)) {
                     ok = false;
                     break;
                 }
-                const HalfRaw R = load_half_raw2<FMT>(base + L.raw_off + slot * kRawSlot, r, h,
-                                                      ks & 1, sw[ks]);
-                // convert before waiting: only the TMEM store needs the stage
-                // free, which keeps the arithmetic off the stage's round trip
-                uint32_t w[16];
-                half_words<FMT>(R, w);
-                const int s = j % kAStages;
-                if (j >= kAStages &&
-                    !mbar_wait(&a_empty[s], static_cast<uint32_t>((j / kAStages) - 1) & 1u,
-                               lim)) {
+                // step h of the pair, both K halves; convert before waiting for
+                // the stage, so only the TMEM stores sit on its round trip
+                const uint32_t raw = base + L.raw_off + slot * kRawSlot;
+                uint32_t w0[16], w1[16];
+                half_words<FMT>(load_half_raw2<FMT>(raw, r, 0, h, sw[2 * kp]), w0);
+                half_words<FMT>(load_half_raw2<FMT>(raw, r, 1, h, sw[2 * kp + 1]), w1);
+                // the reads are consumed; the proxy fence orders them before
+                // the TMA that refills the slot
+                fence_proxy_async_smem();
+                mbar_arrive(&raw_empty[slot]);
+                const uint32_t st = jp & (kAStages - 1);
+                if (jp >= kAStages &&
+                    !mbar_wait(&a_empty[st], ((jp / kAStages) - 1) & 1u, lim)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after_sync();
-                tmem_st_x16(ta + static_cast<uint32_t>(s) * kAStageCols, w);
+                tmem_st_x16(ta + st * kAStageCols, w0);
+                tmem_st_x16(ta + st * kAStageCols + 16, w1);
                 tmem_st_wait();
                 tc_fence_before_sync();
-                mbar_arrive(&a_full[s]);
-                // the raw slot goes back after the pair's second step has
-                // consumed its reads; the proxy fence orders those generic
-                // reads before the TMA that refills it
-                if (ks & 1) {
-                    fence_proxy_async_smem();
-                    mbar_arrive(&raw_empty[slot]);
-                }
+                mbar_arrive(&a_full[st]);
             }
             if (!ok) break;
         }
@@ -359,9 +354,10 @@ __global__ void __launch_bounds__(kXsThreads, 1)
             if (lane == 0 && n_local >= 2)
                 good = mbar_wait(&acc_empty[b], static_cast<uint32_t>((n_local / 2) - 1) & 1u,
                                  lim);
-            for (int ks = 0; ks < nk; ++ks, ++j) {
+            for (int kp = 0; 2 * kp < nk; ++kp, ++j) {       // j: step pairs so far
                 if (lane == 0) {
-                    if (good && fresh) good = mbar_wait(&x_full[ks], xpar, lim);
+                    if (good && fresh) good = mbar_wait(&x_full[2 * kp], xpar, lim);
+                    if (good && fresh) good = mbar_wait(&x_full[2 * kp + 1], xpar, lim);
                     if (good)
                         good = mbar_wait(&a_full[j & (kAStages - 1)], (j / kAStages) & 1u, lim);
                     mma_abort[j & 1] = good ? 0u : 1u;
@@ -380,27 +376,30 @@ __global__ void __launch_bounds__(kXsThreads, 1)
         static_assert((kAStages & (kAStages - 1)) == 0, "A ring indexed with a mask");
         constexpr uint64_t kXAtomDesc = kXAtom >> 4;   // descriptor step per X atom
         const uint64_t bdesc0 = sw128_kmajor_desc(base + L.x_off);
-        uint32_t j = 0;                                 // K steps issued so far
+        uint32_t j = 0;                                 // step pairs issued so far
         bool abort = false;
         for (ItemCursor it(first, last, n_o_tiles); it.valid() && !abort; it.next()) {
             const int n_local = it.item - first;
             const int b = n_local & 1;
             const uint32_t d = tmem + static_cast<uint32_t>(b * kXsTileM);
             uint64_t bdesc = bdesc0;
-            for (int ks = 0; ks < nk; ++ks, ++j, bdesc += kXAtomDesc) {
-                named_bar_sync(kMmaBar, 64);           // the waiter saw step j's stage full
+            for (int kp = 0; 2 * kp < nk; ++kp, ++j, bdesc += 2 * kXAtomDesc) {
+                named_bar_sync(kMmaBar, 64);           // the waiter saw pair j's stage full
                 if (mma_abort[j & 1]) {
                     abort = true;
                     break;
                 }
-                // the whole warp walks the loop; one elected lane issues
+                // the whole warp walks the loop; one elected lane issues the
+                // pair's 8 MMAs (step u's A in columns 32u .. 32u + 31)
                 tc_fence_after_sync();
                 const uint32_t at = tmem + kAccCols + (j & (kAStages - 1)) * kAStageCols;
                 if (elect_one()) {
 #pragma unroll
-                    for (int kk = 0; kk < kAtomK / 16; ++kk)
-                        tc_mma_f16kind_ts(d, at + 8 * kk, bdesc + 2 * kk, idesc,
-                                          (ks > 0 || kk > 0) ? 1u : 0u);
+                    for (int u = 0; u < 2; ++u)
+#pragma unroll
+                        for (int kk = 0; kk < kAtomK / 16; ++kk)
+                            tc_mma_f16kind_ts(d, at + 32 * u + 8 * kk, bdesc + u * kXAtomDesc + 2 * kk,
+                                              idesc, (kp > 0 || u > 0 || kk > 0) ? 1u : 0u);
                     tc_commit(&a_empty[j & (kAStages - 1)]);
                 }
                 __syncwarp();
