@@ -7,18 +7,18 @@
 // in weight-tile-fastest order, so concurrently running CTAs share activation
 // tiles in L2.
 //
-// Per 64-wide K step one stage holds
-//   A: the 128 x 64 dequantized weights in 32 TMEM columns (written with
-//      tcgen05.st by the dequantizers from TMA-staged packed codes, as in
-//      xs.cu), and
-//   B: the 192 x 64 fp16 activations in shared memory, one TMA box from the
-//      pre-converted activations (prep.cu) in the 128-byte-swizzled operand
-//      layout.
-// The A and B rings are separate: TMEM holds two 192-column accumulators and
-// four 32-column A stages (512 columns); shared memory holds six B stages.
-// Roles (20 warps): warps 0-7 dequantizers (thread (r, h) converts half h of
-// every K step of weight row r, as in xs.cu), warp 8 MMA issuer (fed by the
-// waiter, warp 19, through a named barrier, as in xs.cu), warps 9-16
+// Per pair of 64-wide K steps one A stage holds the 128 x 128 dequantized
+// weights in 64 TMEM columns (written with tcgen05.st by the dequantizers
+// from TMA-staged packed codes, as in xs.cu); per K step one B stage holds the
+// 192 x 64 fp16 activations in shared memory, one TMA box from the
+// pre-converted activations (prep.cu) in the 128-byte-swizzled operand
+// layout.  The A and B rings are separate: TMEM holds two 192-column
+// accumulators and two 64-column A stages (512 columns); shared memory holds
+// six B stages.
+// Roles (20 warps): warps 0-7 dequantizers (thread (r, h) converts step h of
+// every step pair of weight row r, as in xs.cu), warp 8 MMA issuer (fed by
+// the waiter, warp 19, through a named barrier, per step pair, as in xs.cu),
+// warps 9-16
 // epilogue (two per TMEM lane quadrant, double-buffered accumulators), warp 17
 // weight TMA (codes and, for q4, (scale, min) blocks of up to 16 words per
 // row), warp 18 activation TMA.
@@ -51,7 +51,7 @@ constexpr int kWsThreads = (kWaitWarp + 1) * 32;         // 640
 constexpr uint32_t kMmaBar = 1;                          // named barrier: waiter <-> MMA warp
 constexpr int kStages = 6;                               // B stages (shared memory)
 constexpr int kStageBytes = kWsTileM * 128;              // 24 KB: 192 rows x 64 K
-constexpr int kAStages = 4;                              // A stages (TMEM)
+constexpr int kAStages = 2;                              // A stages (TMEM), two K steps each
 constexpr int kRaw = 3;                                  // packed-code ring depth (step pairs)
 // Two K steps of packed codes per TMA box (128 rows x 64 B for q4, x 128 B for
 // q8, swizzled), as in xs.cu: a box costs about the same per row at any width.
@@ -60,7 +60,7 @@ constexpr int kScaleSlot = 8 * 1024;                     // 128 rows x 16 words
 constexpr int kScaleWords = 16;                          // (scale, min) words per chunk row
 constexpr int kChunkSteps = kScaleWords / 2;             // K steps covered by one chunk
 constexpr uint32_t kAccCols = 2 * kWsTileM;              // 2 accumulators x 192 columns
-constexpr uint32_t kAStageCols = kAtomK / 2;
+constexpr uint32_t kAStageCols = kAtomK;                 // 2 x 64 16-bit values per lane
 constexpr uint32_t kWsTmemCols = 512;
 static_assert(kAccCols + kAStages * kAStageCols <= kWsTmemCols, "TMEM budget");
 static_assert(kEpiCols % 32 == 0, "epilogue reads 32 columns at a time");
@@ -229,11 +229,11 @@ __global__ void __launch_bounds__(kWsThreads, 1)
         __syncwarp();
     } else if (warp < kDeqWarps) {
         // ============================================================ dequantizers
-        const int h = warp >> 2;                     // K half [32h, 32h + 32) of every step
+        const int h = warp >> 2;                     // step h of every step pair
         const int r = threadIdx.x & (kDeqThreads - 1);
         const uint32_t ta = tmem + kAccCols + (static_cast<uint32_t>((warp & 3) * 32) << 16) +
-                            static_cast<uint32_t>(16 * h);
-        int tile_local = 0;
+                            static_cast<uint32_t>(32 * h);
+        int tile_local = 0, ja = 0;                  // ja: A stages (step pairs) so far
         for (int t = blockIdx.x; t < n_tiles && ok; t += G, ++tile_local) {
             for (int c = 0; c < n_chunks && ok; ++c) {
                 const int q = tile_local * n_chunks + c;
@@ -244,43 +244,49 @@ __global__ void __launch_bounds__(kWsThreads, 1)
                         ok = false;
                         break;
                     }
-                    load_scale_words(base + L.sc_off + b * kScaleSlot + r * (kScaleWords * 4), r,
+                    load_scale_pairs(base + L.sc_off + b * kScaleSlot + r * (kScaleWords * 4), r,
                                      h, sw);
                     fence_proxy_async_smem();       // sw depends on every word read
                     mbar_arrive(&sc_empty[b]);
                 }
 #pragma unroll
-                for (int i = 0; i < kChunkSteps; ++i) {
-                    const int ks = c * kChunkSteps + i;
-                    if (ks >= nk) break;
-                    const int j = tile_local * nk + ks;
-                    const int jp = tile_local * npairs + (ks >> 1);   // step pair of the raw ring
+                for (int kp = 0; kp < kChunkSteps / 2; ++kp) {
+                    const int ks0 = c * kChunkSteps + 2 * kp;     // first step of the pair
+                    if (ks0 >= nk) break;
+                    const int jp = tile_local * npairs + (ks0 >> 1);   // step pair of the raw ring
                     const int slot = jp % kRaw;
-                    if ((ks & 1) == 0 &&
-                        !mbar_wait(&raw_full[slot], static_cast<uint32_t>(jp / kRaw) & 1u, lim)) {
+                    if (!mbar_wait(&raw_full[slot], static_cast<uint32_t>(jp / kRaw) & 1u, lim)) {
                         ok = false;
                         break;
                     }
-                    const HalfRaw R = load_half_raw2<FMT>(base + L.raw_off + slot * kRawSlot, r, h,
-                                                          ks & 1, sw[i]);
-                    uint32_t w[16];
-                    half_words<FMT>(R, w);          // before the stage wait, as in xs.cu
-                    const int s = j % kAStages;
-                    if (j >= kAStages &&
-                        !mbar_wait(&a_empty[s], static_cast<uint32_t>((j / kAStages) - 1) & 1u,
+                    // step ks0 + h of the pair, both K halves (an odd K leaves
+                    // the last pair's second step to nobody); converted before
+                    // the stage wait, as in xs.cu
+                    const bool mine = ks0 + h < nk;
+                    const uint32_t raw = base + L.raw_off + slot * kRawSlot;
+                    uint32_t w0[16], w1[16];
+                    if (mine) {
+                        half_words<FMT>(load_half_raw2<FMT>(raw, r, 0, h, sw[2 * kp]), w0);
+                        half_words<FMT>(load_half_raw2<FMT>(raw, r, 1, h, sw[2 * kp + 1]), w1);
+                    }
+                    fence_proxy_async_smem();           // the slot's reads are consumed
+                    mbar_arrive(&raw_empty[slot]);
+                    const int st = ja & (kAStages - 1);
+                    if (ja >= kAStages &&
+                        !mbar_wait(&a_empty[st], static_cast<uint32_t>((ja / kAStages) - 1) & 1u,
                                    lim)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after_sync();
-                    tmem_st_x16(ta + static_cast<uint32_t>(s) * kAStageCols, w);
-                    tmem_st_wait();
-                    tc_fence_before_sync();
-                    mbar_arrive(&a_full[s]);
-                    if ((ks & 1) || ks == nk - 1) {   // the pair's last step has consumed it
-                        fence_proxy_async_smem();
-                        mbar_arrive(&raw_empty[slot]);
+                    if (mine) {
+                        tmem_st_x16(ta + static_cast<uint32_t>(st) * kAStageCols, w0);
+                        tmem_st_x16(ta + static_cast<uint32_t>(st) * kAStageCols + 16, w1);
+                        tmem_st_wait();
                     }
+                    tc_fence_before_sync();
+                    mbar_arrive(&a_full[st]);
+                    ++ja;
                 }
             }
         }
@@ -289,21 +295,25 @@ __global__ void __launch_bounds__(kWsThreads, 1)
         // As in xs.cu: the waits of the MMA issuer, handed over per K step
         // through named barrier kMmaBar, so that the issuing thread never
         // waits on an mbarrier after a tcgen05.commit.
-        int j = 0, tile_local = 0;
+        int ja = 0, tile_local = 0;                    // ja: step pairs so far
         for (int t = blockIdx.x; t < n_tiles && ok; t += G, ++tile_local) {
             const int b = tile_local & 1;
             bool good = true;
             if (lane == 0 && tile_local >= 2)
                 good = mbar_wait(&acc_empty[b],
                                  static_cast<uint32_t>((tile_local / 2) - 1) & 1u, lim);
-            for (int ks = 0; ks < nk; ++ks, ++j) {
+            for (int kp = 0; 2 * kp < nk; ++kp, ++ja) {
+                const int j0 = tile_local * nk + 2 * kp;      // the pair's first K step
+                const bool two = 2 * kp + 1 < nk;
                 if (lane == 0) {
                     if (good)
-                        good = mbar_wait(&a_full[j % kAStages],
-                                         static_cast<uint32_t>(j / kAStages) & 1u, lim) &&
-                               mbar_wait(&b_full[j % kStages],
-                                         static_cast<uint32_t>(j / kStages) & 1u, lim);
-                    mma_abort[j & 1] = good ? 0u : 1u;
+                        good = mbar_wait(&a_full[ja % kAStages],
+                                         static_cast<uint32_t>(ja / kAStages) & 1u, lim) &&
+                               mbar_wait(&b_full[j0 % kStages],
+                                         static_cast<uint32_t>(j0 / kStages) & 1u, lim) &&
+                               (!two || mbar_wait(&b_full[(j0 + 1) % kStages],
+                                                  static_cast<uint32_t>((j0 + 1) / kStages) & 1u, lim));
+                    mma_abort[ja & 1] = good ? 0u : 1u;
                 }
                 named_bar_sync(kMmaBar, 64);
                 if (__shfl_sync(0xffffffffu, good ? 1 : 0, 0) == 0) {
@@ -317,29 +327,41 @@ __global__ void __launch_bounds__(kWsThreads, 1)
         const uint32_t idesc = idesc_f16_f32acc(kTileRows, kWsTileM);
         constexpr uint64_t kStageDesc = kStageBytes >> 4;   // descriptor step per B stage
         const uint64_t bdesc0 = sw128_kmajor_desc(base + L.st_off);
-        int j = 0, tile_local = 0;
+        int ja = 0, tile_local = 0;                    // ja: step pairs so far
         bool abort = false;
         for (int t = blockIdx.x; t < n_tiles && !abort; t += G, ++tile_local) {
             const int b = tile_local & 1;
             const uint32_t d = tmem + static_cast<uint32_t>(b * kWsTileM);
-            for (int ks = 0; ks < nk; ++ks, ++j) {
-                named_bar_sync(kMmaBar, 64);           // the waiter saw step j's stages full
-                if (mma_abort[j & 1]) {
+            for (int kp = 0; 2 * kp < nk; ++kp, ++ja) {
+                named_bar_sync(kMmaBar, 64);           // the waiter saw pair ja's stages full
+                if (mma_abort[ja & 1]) {
                     abort = true;
                     break;
                 }
-                // the whole warp walks the loop; one elected lane issues
+                // the whole warp walks the loop; one elected lane issues the
+                // pair's MMAs (step u's A in columns 32u .. 32u + 31)
                 tc_fence_after_sync();
-                const int s = j % kAStages, sb = j % kStages;
+                const int s = ja % kAStages;
+                const int j0 = tile_local * nk + 2 * kp;
+                const bool two = 2 * kp + 1 < nk;
+                const int sb0 = j0 % kStages, sb1 = (j0 + 1) % kStages;
                 const uint32_t at = tmem + kAccCols + static_cast<uint32_t>(s) * kAStageCols;
-                const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(sb) * kStageDesc;
                 if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < kAtomK / 16; ++kk)
-                        tc_mma_f16kind_ts(d, at + 8 * kk, bdesc + 2 * kk, idesc,
-                                          (ks > 0 || kk > 0) ? 1u : 0u);
+                        tc_mma_f16kind_ts(d, at + 8 * kk,
+                                          bdesc0 + static_cast<uint64_t>(sb0) * kStageDesc + 2 * kk,
+                                          idesc, (kp > 0 || kk > 0) ? 1u : 0u);
+                    if (two) {
+#pragma unroll
+                        for (int kk = 0; kk < kAtomK / 16; ++kk)
+                            tc_mma_f16kind_ts(d, at + 32 + 8 * kk,
+                                              bdesc0 + static_cast<uint64_t>(sb1) * kStageDesc + 2 * kk,
+                                              idesc, 1u);
+                    }
                     tc_commit(&a_empty[s]);
-                    tc_commit(&b_empty[sb]);
+                    tc_commit(&b_empty[sb0]);
+                    if (two) tc_commit(&b_empty[sb1]);
                 }
                 __syncwarp();
             }
