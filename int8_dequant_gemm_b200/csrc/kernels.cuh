@@ -96,6 +96,8 @@ cudaError_t launch_xs(int fmt, const void *Xh, const void *Wq, const void *S, co
 // tcgen05, persistent weight-stationary tiles with both operands TMA-staged
 // (more than 128 activation rows, any K of the format's TMA granule); see ws.cu.
 bool ws_supported(int fmt, int M, int N, int K);
+// Activation rows per weight-streamed tile for this shape and SM count.
+int ws_tile_rows(int M, int N, int sms);
 cudaError_t launch_ws(int fmt, const void *Xh, const void *Wq, const void *S, const float *bias,
                       float *Y, int M, int N, int K, DevCtl *ctl, cudaStream_t s);
 

@@ -2,15 +2,19 @@
 // stationary, TMA streams both operands' raw data through a stage ring.
 //
 // Tile product as in tc.cu / xs.cu, D[o, m] = sum_k W_hat[o, k] * X[m, k],
-// 128 weight rows (MMA M) x 192 activation rows (MMA N), full K per tile.
+// 128 weight rows (MMA M) x bn activation rows (MMA N), full K per tile.
 // A persistent CTA (one per SM) walks tiles t = blockIdx.x, + gridDim.x, ...
 // in weight-tile-fastest order, so concurrently running CTAs share activation
-// tiles in L2.
+// tiles in L2.  bn is chosen per launch (a multiple of 32 from 64 to 192,
+// ws_tile_rows): a tile takes about as long as its dequantization plus its
+// MMAs, so the widest tile is the cheapest per output unless the tile count
+// leaves a last wave mostly empty (M = 4096, N = 512: 88 tiles of 192 rows on
+// 148 SMs, against 128 tiles of 128 rows in the same single wave).
 //
 // Per pair of 64-wide K steps one A stage holds the 128 x 128 dequantized
 // weights in 64 TMEM columns (written with tcgen05.st by the dequantizers
 // from TMA-staged packed codes, as in xs.cu); per K step one B stage holds the
-// 192 x 64 fp16 activations in shared memory, one TMA box from the
+// bn x 64 fp16 activations in shared memory, one TMA box from the
 // pre-converted activations (prep.cu) in the 128-byte-swizzled operand
 // layout.  The A and B rings are separate: TMEM holds two 192-column
 // accumulators and two 64-column A stages (512 columns); shared memory holds
@@ -35,7 +39,8 @@
 namespace rtq {
 namespace {
 
-constexpr int kWsTileM = 192;                 // activation rows per tile (MMA N)
+constexpr int kWsTileM = 192;                 // widest activation tile (MMA N)
+constexpr int kWsTileMin = 64;
 constexpr int kDeqGroups = 2;                            // two K halves per step
 constexpr int kDeqThreads = kTileRows;                   // 128 per group
 constexpr int kDeqWarps = kDeqGroups * 4;                // 8
@@ -43,14 +48,13 @@ constexpr int kMmaWarp = kDeqWarps;                      // 8
 constexpr int kEpiWarp0 = kMmaWarp + 1;                  // 9
 constexpr int kEpiWarps = 8;                             // two per TMEM lane quadrant
 constexpr int kEpiThreads = kEpiWarps * 32;
-constexpr int kEpiCols = kWsTileM / 2;
 constexpr int kWTmaWarp = kEpiWarp0 + kEpiWarps;         // 17
 constexpr int kXTmaWarp = kWTmaWarp + 1;                 // 18
 constexpr int kWaitWarp = kXTmaWarp + 1;                 // 19
 constexpr int kWsThreads = (kWaitWarp + 1) * 32;         // 640
 constexpr uint32_t kMmaBar = 1;                          // named barrier: waiter <-> MMA warp
 constexpr int kStages = 6;                               // B stages (shared memory)
-constexpr int kStageBytes = kWsTileM * 128;              // 24 KB: 192 rows x 64 K
+constexpr int kStageBytes = kWsTileM * 128;              // 24 KB: up to 192 rows x 64 K
 constexpr int kAStages = 2;                              // A stages (TMEM), two K steps each
 constexpr int kRaw = 3;                                  // packed-code ring depth (step pairs)
 // Two K steps of packed codes per TMA box (128 rows x 64 B for q4, x 128 B for
@@ -59,11 +63,12 @@ __host__ __device__ constexpr int raw_slot_bytes(int fmt) { return kTileRows * (
 constexpr int kScaleSlot = 8 * 1024;                     // 128 rows x 16 words
 constexpr int kScaleWords = 16;                          // (scale, min) words per chunk row
 constexpr int kChunkSteps = kScaleWords / 2;             // K steps covered by one chunk
-constexpr uint32_t kAccCols = 2 * kWsTileM;              // 2 accumulators x 192 columns
+constexpr uint32_t kAccCols = 2 * kWsTileM;              // 2 accumulators x up to 192 columns
 constexpr uint32_t kAStageCols = kAtomK;                 // 2 x 64 16-bit values per lane
 constexpr uint32_t kWsTmemCols = 512;
 static_assert(kAccCols + kAStages * kAStageCols <= kWsTmemCols, "TMEM budget");
-static_assert(kEpiCols % 32 == 0, "epilogue reads 32 columns at a time");
+static_assert(kWsTileM % 32 == 0 && kWsTileMin % 32 == 0,
+              "an epilogue warp's bn / 2 columns are a multiple of 16");
 
 struct WsLayout {
     int st_off, raw_off, sc_off, bar_off, total;
@@ -81,13 +86,28 @@ __host__ __device__ inline WsLayout ws_layout() {
     return L;
 }
 
+// One output row's values for columns c .. c + W - 1 (Y rows m0 + c + jj, at
+// stride rs), scaled and biased; the first `avail` of them are inside M.
+template <int W>
+__device__ __forceinline__ void store_cols(float *p, size_t rs, const uint32_t (&v)[W], int avail,
+                                           float sc, float bo) {
+    if (avail >= W) {
+#pragma unroll
+        for (int jj = 0; jj < W; ++jj) p[jj * rs] = fmaf(__uint_as_float(v[jj]), sc, bo);
+    } else {
+#pragma unroll
+        for (int jj = 0; jj < W; ++jj)
+            if (jj < avail) p[jj * rs] = fmaf(__uint_as_float(v[jj]), sc, bo);
+    }
+}
+
 template <int FMT>
 __global__ void __launch_bounds__(kWsThreads, 1)
     ws_qgemm_kernel(const __grid_constant__ CUtensorMap w_map,
                     const __grid_constant__ CUtensorMap s_map,
                     const __grid_constant__ CUtensorMap x_map, const float *__restrict__ S8,
                     const float *__restrict__ bias, float *__restrict__ Y, int M, int N, int K,
-                    int n_o_tiles, int n_tiles, DevCtl *ctl) {
+                    int bn, int n_o_tiles, int n_tiles, DevCtl *ctl) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_addr(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;
@@ -206,7 +226,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
             pdl_wait_prior_grid();     // the 16-bit activations come from the pre-pass
             int j = 0;
             for (int t = blockIdx.x; t < n_tiles && ok; t += G) {
-                const int m0 = (t / n_o_tiles) * kWsTileM;
+                const int m0 = (t / n_o_tiles) * bn;
                 for (int ks = 0; ks < nk; ++ks, ++j) {
                     const int s = j % kStages;
                     if (j >= kStages &&
@@ -215,7 +235,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
                         ok = false;
                         break;
                     }
-                    mbar_expect_tx(&b_full[s], kStageBytes);
+                    mbar_expect_tx(&b_full[s], static_cast<uint32_t>(bn * 128));
                     tma_load_2d(base + L.st_off + s * kStageBytes, &x_map,
                                 ks * kAtomK, m0, &b_full[s]);
                 }
@@ -324,7 +344,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
         }
     } else if (warp == kMmaWarp) {
         // ============================================================ MMA issuer
-        const uint32_t idesc = idesc_f16_f32acc(kTileRows, kWsTileM);
+        const uint32_t idesc = idesc_f16_f32acc(kTileRows, bn);
         constexpr uint64_t kStageDesc = kStageBytes >> 4;   // descriptor step per B stage
         const uint64_t bdesc0 = sw128_kmajor_desc(base + L.st_off);
         int ja = 0, tile_local = 0;                    // ja: step pairs so far
@@ -379,7 +399,8 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     } else {
         // ============================================================ epilogue
         const int qd = warp & 3;
-        const int c0 = ((warp - kEpiWarp0) >> 2) * kEpiCols;   // its half of the columns
+        const int ecols = bn / 2;                       // columns per warp: 32 .. 96
+        const int c0 = ((warp - kEpiWarp0) >> 2) * ecols;   // its half of the columns
         const int row = qd * 32 + lane;
         const uint32_t tq = tmem + (static_cast<uint32_t>(qd * 32) << 16);
         int tile_local = 0;
@@ -389,29 +410,27 @@ __global__ void __launch_bounds__(kWsThreads, 1)
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after_sync();
-            const int m0 = (t / n_o_tiles) * kWsTileM;
+            const int m0 = (t / n_o_tiles) * bn;
             const int o = (t % n_o_tiles) * kTileRows + row;
             float sc = 1.f, bo = 0.f;
             if (FMT == 8 && o < N) sc = __ldg(S8 + o);
             if (bias && o < N) bo = __ldg(bias + o);
-            const int mlim = min(kWsTileM, M - m0);
+            const int mlim = min(bn, M - m0);
             float *yo = Y + static_cast<size_t>(m0) * N + o;
             const size_t rs = static_cast<size_t>(N);
-            for (int c = c0; c < c0 + kEpiCols; c += 32) {
+            const uint32_t tb = tq + static_cast<uint32_t>(b * kWsTileM);
+            int c = c0;
+            for (; c + 32 <= c0 + ecols; c += 32) {
                 uint32_t v[32];
-                tmem_ld_x32(tq + static_cast<uint32_t>(b * kWsTileM + c), v);
+                tmem_ld_x32(tb + static_cast<uint32_t>(c), v);
                 tmem_ld_wait();
-                if (o < N) {
-                    float *p = yo + static_cast<size_t>(c) * rs;
-                    if (c + 32 <= mlim) {
-#pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) p[jj * rs] = fmaf(__uint_as_float(v[jj]), sc, bo);
-                    } else {
-#pragma unroll
-                        for (int jj = 0; jj < 32; ++jj)
-                            if (c + jj < mlim) p[jj * rs] = fmaf(__uint_as_float(v[jj]), sc, bo);
-                    }
-                }
+                if (o < N) store_cols(yo + static_cast<size_t>(c) * rs, rs, v, mlim - c, sc, bo);
+            }
+            if (c < c0 + ecols) {                       // bn / 2 an odd multiple of 16
+                uint32_t v[16];
+                tmem_ld_x16(tb + static_cast<uint32_t>(c), v);
+                tmem_ld_wait();
+                if (o < N) store_cols(yo + static_cast<size_t>(c) * rs, rs, v, mlim - c, sc, bo);
             }
             tc_fence_before_sync();
             mbar_arrive(&acc_empty[b]);
@@ -436,9 +455,12 @@ cudaError_t launch_ws_fmt(const void *Xh, const void *Wq, const void *S, const f
     if (e != cudaSuccess) return e;
     if ((e = smem_attr_once(ws_qgemm_kernel<FMT>, 227 * 1024, dev, attr_done)) != cudaSuccess)
         return e;
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int bn = ws_tile_rows(M, N, sms);
     CUtensorMap w_map, s_map, x_map;
     bool enc_ok = encode_tma_2d(&x_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, Xh, K, M, kAtomK,
-                                CU_TENSOR_MAP_SWIZZLE_128B, kWsTileM);
+                                CU_TENSOR_MAP_SWIZZLE_128B, static_cast<uint32_t>(bn));
     if (FMT == 4) {
         enc_ok = enc_ok &&
                  encode_tma_2d(&w_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Wq, K / 2, N, 64,
@@ -451,10 +473,8 @@ cudaError_t launch_ws_fmt(const void *Xh, const void *Wq, const void *S, const f
         s_map = w_map;   // unused by the q8 kernel
     }
     if (!enc_ok) return cudaErrorInvalidValue;
-    int sms = 148;
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int n_o = (N + kTileRows - 1) / kTileRows;
-    const int n_m = (M + kWsTileM - 1) / kWsTileM;
+    const int n_m = (M + bn - 1) / bn;
     const int tiles = n_o * n_m;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(std::min(tiles, sms), 1, 1);
@@ -467,10 +487,34 @@ cudaError_t launch_ws_fmt(const void *Xh, const void *Wq, const void *S, const f
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, ws_qgemm_kernel<FMT>, w_map, s_map, x_map,
-                              static_cast<const float *>(S), bias, Y, M, N, K, n_o, tiles, ctl);
+                              static_cast<const float *>(S), bias, Y, M, N, K, bn, n_o, tiles,
+                              ctl);
 }
 
 }  // namespace
+
+// Activation rows per tile: the multiple of 32 from 64 to 192 with the least
+// waves x (400 + bn), waves = ceil(tiles / SMs).  The per-tile cost, 400 + bn
+// in units of activation columns of MMA, is fitted to the kernel's measured
+// per-wave times (N = 512, K = 2048, M = 4096 and 16384, bn = 128 .. 192): a
+// weight tile's dequantization and hand-overs cost about as much as 400
+// columns.  Measured, this picks the fastest height of the five on each of
+// seven shapes from M = 300 to 65536.  Ties keep the wider tile.
+int ws_tile_rows(int M, int N, int sms) {
+    const long long n_o = (N + kTileRows - 1) / kTileRows;
+    int best = kWsTileM;
+    long long best_cost = -1;
+    for (int bn = kWsTileM; bn >= kWsTileMin; bn -= 32) {
+        const long long tiles = n_o * ((M + bn - 1) / bn);
+        const long long waves = (tiles + sms - 1) / sms;
+        const long long cost = waves * (400 + bn);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = bn;
+        }
+    }
+    return best;
+}
 
 // Shapes the TMA-fed weight-streamed kernel takes: more than 128 activation
 // rows, and K a multiple of 64 (q8) or 128 (q4: the (scale, min) rows are TMA

@@ -220,9 +220,13 @@ def test_x_resident_parity_q8(rtq_lib, M, N, K, path="tc"):
 
 # shapes that the TMA-fed weight-streamed kernel takes: K above the resident
 # limit; ragged M and N; q4 chunks of (scale, min) words that end inside a
-# chunk (K = 640)
+# chunk (K = 640).  The launch picks the activation tile height from the tile
+# count on 148 SMs: the first six shapes take 64 rows, and the
+# four (M, 700, 768) shapes 96, 128, 160 and 192 rows, so every epilogue split
+# (16 + 16 .. 32 + 32 + 32 columns per warp) runs
 WS_SHAPES = [(2048, 512, 2048), (300, 640, 1024), (200, 512, 768), (1000, 700, 2048),
-             (129, 256, 640), (300, 1002, 768)]
+             (129, 256, 640), (300, 1002, 768), (1572, 700, 768), (2312, 700, 768),
+             (3089, 700, 768), (3866, 700, 768)]
 
 
 @pytest.mark.parametrize("M,N,K", WS_SHAPES)
@@ -290,6 +294,31 @@ def test_x_resident_identity_bit_exact(rtq_lib):
     Y = rtq_lib.qgemm_q4(torch.eye(K, device="cuda"), dev(Wq), dev(sm)).cpu().numpy()
     ref = oracle.dequant_q4(Wq, sm).astype(np.float16).astype(np.float32).T
     assert np.array_equal(Y, ref)
+
+
+@pytest.mark.parametrize("fmt", [4, 8])
+def test_x_resident_x_16_byte_aligned(rtq_lib, fmt):
+    """X that starts 16 bytes past a 32-byte boundary (the ABI asks for 16
+    only): the activation-resident route must give the bits it gives for an
+    aligned copy of X."""
+    M, N, K = 700, 640, 384
+    assert rtq_lib.plan(fmt, M, N, K) == "tc_x_resident"
+    X = wl.activations(M, K, 77 + fmt)
+    if fmt == 4:
+        q = q4_weights(N, K, 78, outliers=True)
+        fn, ref = rtq_lib.qgemm_q4, oracle.gemm_q4(X, *q)
+    else:
+        q = q8_weights(N, K, 78, outliers=True)
+        fn, ref = rtq_lib.qgemm_q8, oracle.gemm_q8(X, *q)
+    buf = torch.empty(M * K + 4, device="cuda")
+    Xo = buf[4:].view(M, K)
+    Xo.copy_(dev(X))
+    assert Xo.data_ptr() % 32 == 16
+    Wd, Sd = dev(q[0]), dev(q[1])
+    Ya = fn(dev(X), Wd, Sd, path="tc")
+    Yo = fn(Xo, Wd, Sd, path="tc")
+    assert torch.equal(Ya, Yo)
+    assert rel_err(Yo.cpu().numpy(), ref) <= MAX_REL["tc"]
 
 
 def test_random_format_bytes_both_paths(rtq_lib):
