@@ -168,25 +168,33 @@ int rt_qgemm_auto_path(int fmt, int64_t M, int64_t N, int64_t K);
  *                             operands TMA-staged (M > 128, other K);
  *   RT_KERNEL_TC_LIST         tcgen05, rt_qgemm_batch only: persistent CTAs
  *                             stream the weights of a whole list of
- *                             projections with the same M <= 128.
- * The TMA-fed kernels run an activation pre-pass (X rounded once to fp16)
- * into a per-(device, stream) workspace of M * K * 2 bytes. */
+ *                             projections with the same M <= 128;
+ *   RT_KERNEL_TC_X_RESIDENT_PAIR  the activation-resident product on pairs of
+ *                             CTAs (one tcgen05 MMA over two SMs, 256 weight
+ *                             rows x 192 activation rows), rounding X to fp16
+ *                             inside the kernel (M >= 16384, K a multiple of
+ *                             128 up to 512).
+ * RT_KERNEL_TC_X_RESIDENT and RT_KERNEL_TC_W_STREAMED run an activation
+ * pre-pass (X rounded once to fp16) into a per-(device, stream) workspace of
+ * M * K * 2 bytes; RT_KERNEL_TC_X_RESIDENT_PAIR needs none. */
 typedef enum rt_kernel {
     RT_KERNEL_SIMT = 1,
     RT_KERNEL_TC_W_STATIONARY = 2,
     RT_KERNEL_TC_X_RESIDENT = 3,
     RT_KERNEL_TC_W_STREAMED = 4,
-    RT_KERNEL_TC_LIST = 5
+    RT_KERNEL_TC_LIST = 5,
+    RT_KERNEL_TC_X_RESIDENT_PAIR = 6
 } rt_kernel;
 
 /* The kernel a GEMM of this format, shape and path runs; -1 if rejected. */
 int rt_qgemm_plan(int fmt, int64_t M, int64_t N, int64_t K, int path);
 
 /*
- * Workspace.  The TMA-fed kernels stage the activations, rounded to fp16,
- * in a device buffer the library keeps per (device,
- * stream): rt_workspace_bytes() gives the size a GEMM needs (0 for the other
- * kernels, -1 for a rejected shape).  The buffer grows on first need with
+ * Workspace.  RT_KERNEL_TC_X_RESIDENT and RT_KERNEL_TC_W_STREAMED stage the
+ * activations, rounded to fp16, in a device buffer the library keeps per
+ * (device, stream): rt_workspace_bytes() gives the size a GEMM needs
+ * (M * K * 2 for those two kernels, 0 for the others, -1 for a rejected
+ * shape).  The buffer grows on first need with
  * cudaMalloc; growth synchronizes that stream.  It cannot grow while the
  * stream is being captured into a CUDA graph -- such a call returns
  * RT_ERR_WORKSPACE -- so reserve the largest size first with
@@ -209,11 +217,12 @@ rt_status rt_workspace_release(void);
  * fmt = 4: Wq/scales are the q4 tensors of rt_qgemm_q4; fmt = 8: those of
  * rt_qgemm_q8.  X, Y, M, N, K, path and stream, validation and results are
  * as for rt_qgemm_q4/q8, and the same kernel runs (rt_qgemm_plan).  The
- * TMA-fed kernels stage the fp16 activations in one file-scope device
- * array of RT_NOALLOC_SCRATCH_BYTES (16 MiB) per device instead of the
- * per-stream workspace; a problem whose M * K * 2 exceeds it returns
+ * kernels that stage fp16 activations (RT_KERNEL_TC_X_RESIDENT,
+ * RT_KERNEL_TC_W_STREAMED) use one file-scope device array of
+ * RT_NOALLOC_SCRATCH_BYTES (16 MiB) per device instead of the per-stream
+ * workspace; such a problem whose M * K * 2 exceeds it returns
  * RT_ERR_SCRATCH_LIMIT and launches nothing (for example M * K up to 8M
- * elements, M = 4096 x K = 2048).
+ * elements, M = 4096 x K = 2048).  The other kernels need no scratch.
  *
  * Set-up: the first call on a device that passes validation looks up
  * the array's device address, which may load the library's module; make

@@ -671,7 +671,8 @@ def auto_path(fmt: int, M: int, N: int, K: int) -> int:
     return int(rt_qgemm_auto_path(fmt, M, N, K))
 
 
-KERNELS = {1: "simt", 2: "tc_w_stationary", 3: "tc_x_resident", 4: "tc_w_streamed", 5: "tc_list"}
+KERNELS = {1: "simt", 2: "tc_w_stationary", 3: "tc_x_resident", 4: "tc_w_streamed", 5: "tc_list",
+           6: "tc_x_resident_pair"}
 
 
 def plan(fmt: int, M: int, N: int, K: int, path="auto") -> str:

@@ -19,7 +19,8 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "librtq.so")
 HEADER = os.path.join(ROOT, "include", "rtq.h")
 
-CU_SOURCES = ["api.cu", "simt.cu", "tc.cu", "xs.cu", "ws.cu", "prep.cu", "pl.cu", "noalloc.cu"]
+CU_SOURCES = ["api.cu", "simt.cu", "tc.cu", "xs.cu", "xp.cu", "ws.cu", "prep.cu", "pl.cu",
+              "noalloc.cu"]
 CPP_SOURCES = ["quantize.cpp", "st_loader.cpp"]
 NVCC = os.environ.get("NVCC", "nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -136,7 +136,8 @@ int64_t scale_bytes(int fmt, int64_t N, int64_t K) {
 int pick_kernel(int fmt, int64_t M, int64_t N, int64_t K, int p) {
     if (p == RT_PATH_SIMT) return RT_KERNEL_SIMT;
     const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
-    if (rtq::xs_supported(m, n, k)) return RT_KERNEL_TC_X_RESIDENT;
+    if (rtq::xs_supported(m, n, k))
+        return m >= rtq::kXpMinM ? RT_KERNEL_TC_X_RESIDENT_PAIR : RT_KERNEL_TC_X_RESIDENT;
     if (rtq::ws_supported(fmt, m, n, k)) return RT_KERNEL_TC_W_STREAMED;
     return RT_KERNEL_TC_W_STATIONARY;
 }
@@ -168,6 +169,8 @@ rt_status run_gemm(int fmt, const float *X, const void *Wq, const void *S, const
     if (st != RT_OK) return st;
     if (kern == RT_KERNEL_TC_W_STATIONARY)
         return from_cuda(rtq::launch_tc(fmt, X, Wq, S, bias, Y, m, n, k, ctl, s));
+    if (kern == RT_KERNEL_TC_X_RESIDENT_PAIR)
+        return from_cuda(rtq::launch_xp(fmt, X, Wq, S, bias, Y, m, n, k, ctl, s));
     void *xh = nullptr;
     if ((st = workspace(s, static_cast<size_t>(M) * K * 2, &xh)) != RT_OK) return st;
     cudaError_t e = rtq::launch_cvt_x16(X, xh, M, K, ctl, s);

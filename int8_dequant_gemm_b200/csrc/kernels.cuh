@@ -93,6 +93,17 @@ bool xs_supported(int M, int N, int K);
 cudaError_t launch_xs(int fmt, const void *Xh, const void *Wq, const void *S, const float *bias,
                       float *Y, int M, int N, int K, DevCtl *ctl, cudaStream_t s);
 
+// The same activation-resident product on CTA pairs (cta_group::2, 256 weight
+// rows per MMA), rounding fp32 X to fp16 inside the kernel; see xp.cu.  Same
+// shapes as launch_xs; the plan takes it from kXpMinM activation rows up:
+// measured against the pre-pass + launch_xs, it ties at M = 8192 to 16384
+// and is 4 to 20 % faster at M = 32768 and 65536, while at M = 4096 the
+// rounding of each CTA's first activation block costs more than the
+// pre-pass saves.
+constexpr int kXpMinM = 16384;
+cudaError_t launch_xp(int fmt, const float *X, const void *Wq, const void *S, const float *bias,
+                      float *Y, int M, int N, int K, DevCtl *ctl, cudaStream_t s);
+
 // tcgen05, persistent weight-stationary tiles with both operands TMA-staged
 // (more than 128 activation rows, any K of the format's TMA granule); see ws.cu.
 bool ws_supported(int fmt, int M, int N, int K);

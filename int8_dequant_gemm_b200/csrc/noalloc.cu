@@ -1,7 +1,8 @@
 // rt_qgemm_noalloc: the quantized GEMM without any device allocation.
 //
-// The TMA-fed tensor-core kernels need scratch for the activations rounded
-// to the 16-bit operand type (M * K * 2 bytes).  rt_qgemm_q4/q8 take it from
+// The TMA-fed tensor-core kernels that stage the activations rounded to the
+// 16-bit operand type (activation-resident below 16384 rows, weight-streamed)
+// need scratch for them (M * K * 2 bytes).  rt_qgemm_q4/q8 take it from
 // a per-stream workspace that grows with cudaMalloc and, when it grows,
 // synchronizes the stream and frees the old buffer.  Some callers cannot do
 // that: a serving process whose pool allocator already owns nearly all of
@@ -73,6 +74,8 @@ extern "C" rt_status rt_qgemm_noalloc(int fmt, const float *X, const void *Wq, c
     if ((st = rtq::device_ctl(&ctl)) != RT_OK) return st;
     if (kern == RT_KERNEL_TC_W_STATIONARY)
         return from_cuda(rtq::launch_tc(fmt, X, Wq, scales, nullptr, Y, m, n, k, ctl, s));
+    if (kern == RT_KERNEL_TC_X_RESIDENT_PAIR)
+        return from_cuda(rtq::launch_xp(fmt, X, Wq, scales, nullptr, Y, m, n, k, ctl, s));
     if (rtq::launch_cvt_x16(X, xh, M, K, ctl, s) != cudaSuccess) return RT_ERR_CUDA;
     if (kern == RT_KERNEL_TC_X_RESIDENT)
         return from_cuda(rtq::launch_xs(fmt, xh, Wq, scales, nullptr, Y, m, n, k, ctl, s));

@@ -246,6 +246,103 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32acc(int M, int N) {
            | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
+// ---------------------------------------------- CTA pairs (cta_group::2)
+// A pair of CTAs in a cluster of two (ranks 0 and 1) shares one MMA: the even
+// CTA issues tcgen05.mma.cta_group::2 with M = 256, whose A rows 0..127 and D
+// rows 0..127 live in its own TMEM and rows 128..255 at the same TMEM address
+// of the odd CTA, and whose B columns 0..N/2-1 come from its own shared memory
+// and N/2..N-1 from the same shared-memory offset of the odd CTA.  Every
+// tcgen05 allocation, MMA and commit of such a kernel names cta_group::2.
+
+// Both CTAs: one warp each, the same warp in both, the same slot offset.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t *slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(slot)),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+// Even CTA only: D[tmem] (+)= A[tmem] * B[smem desc]^T over both CTAs of the
+// pair, 16-bit inputs, fp32 accumulate (idesc with M = 256).
+__device__ __forceinline__ void tc_mma_pair_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrives once on the mbarrier at `bar`'s offset in every CTA of `cta_mask`
+// when every earlier cta_group::2 tcgen05 operation of this thread is done.
+__device__ __forceinline__ void tc_commit_pair_mc(uint64_t *bar, uint16_t cta_mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
+        "[%0], %1;" ::"r"(smem_addr(bar)),
+        "h"(cta_mask)
+        : "memory");
+}
+
+// Arrive on an mbarrier of a cluster peer (address from cluster_map), with
+// release semantics at cluster scope: the peer's acquire sees this thread's
+// earlier shared-memory writes.  It costs about as much as a cluster-wide
+// fence (1.5K cycles, measured), so the per-stage signals use the next form.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t caddr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr)
+                 : "memory");
+}
+
+// Arrive on a cluster peer's mbarrier with the default (CTA-scope) release.
+// For signals that order no shared-memory data: TMEM writes that
+// tcgen05.wait::st has completed (followed by tcgen05.fence::before_thread_sync),
+// or reads that are finished.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t caddr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// mbar_wait for a barrier that a cluster peer arrives on: acquire at cluster
+// scope, so the peer's writes before its arrival are visible afterwards.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity,
+                                                  const unsigned long long *limit_ns) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    const uint64_t limit = *limit_ns;
+    uint32_t n = 0;
+    while (true) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if ((++n & 255u) == 0 && global_timer_ns() - t0 > limit) return false;
+    }
+}
+
+// Orders this thread's generic-proxy writes before later async-proxy
+// accesses in every state space (here: a peer's tensor-core reads of this
+// CTA's shared memory).
+__device__ __forceinline__ void fence_proxy_async_all() {
+    asm volatile("fence.proxy.async;" ::: "memory");
+}
+
 // ------------------------------------------------- dependent launch (PDL)
 __device__ __forceinline__ void pdl_wait_prior_grid() {
     asm volatile("griddepcontrol.wait;" ::: "memory");

@@ -100,7 +100,11 @@ def test_kernel_plan():
     assert rtq.plan(4, 4, 2048, 512) == "simt"
     assert rtq.plan(4, 80, 2048, 512) == "tc_w_stationary"
     assert rtq.plan(4, 4096, 4096, 512) == "tc_x_resident"
-    assert rtq.plan(4, 65536, 2048, 512) == "tc_x_resident"
+    assert rtq.plan(4, 65536, 2048, 512) == "tc_x_resident_pair"   # CTA pairs from M = 16384
+    assert rtq.plan(4, 16383, 2048, 512) == "tc_x_resident"
+    assert rtq.plan(8, 16384, 512, 128) == "tc_x_resident_pair"
+    assert rtq.plan(3, 20000, 512, 384) == "tc_x_resident_pair"
+    assert rtq.plan(8, 65536, 512, 2048) == "tc_w_streamed"
     assert rtq.plan(8, 4096, 512, 2048) == "tc_w_streamed"     # K > 512 does not fit resident
     assert rtq.plan(4, 200, 512, 512) == "tc_x_resident"       # one full block and a tail
     assert rtq.plan(4, 129, 512, 512) == "tc_x_resident"
@@ -115,6 +119,7 @@ def test_kernel_plan():
 
 def test_workspace_sizes():
     assert rtq.workspace_bytes(4, 4096, 4096, 512) == 4096 * 512 * 2
+    assert rtq.workspace_bytes(4, 65536, 2048, 512) == 0          # CTA pairs: in-kernel rounding
     assert rtq.workspace_bytes(8, 4096, 512, 2048) == 4096 * 2048 * 2
     assert rtq.workspace_bytes(4, 80, 2048, 512) == 0
     assert rtq.workspace_bytes(4, 4, 2048, 512) == 0
@@ -135,7 +140,9 @@ def test_noalloc_validation_and_scratch_limit():
     limit = rtq.NOALLOC_SCRATCH_BYTES
     assert rtq.plan(8, 4096, 512, 4096) == "tc_w_streamed" and 4096 * 4096 * 2 > limit
     assert f(8, 0x100000000, W, S, 0x300000000, 4096, 512, 4096, 0, None) == 8
-    assert rtq.plan(4, 16384, 4096, 512) == "tc_x_resident" and 16384 * 512 * 2 == limit
+    assert rtq.plan(4, 16383, 4096, 512) == "tc_x_resident" and 16383 * 512 * 2 < limit
+    # the CTA-pair kernel needs no scratch, so its size is not limited
+    assert rtq.plan(4, 65536, 4096, 512) == "tc_x_resident_pair" and 65536 * 512 * 2 > limit
     assert rtq.status_string(8) != "unknown status"
 
 

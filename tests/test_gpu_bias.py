@@ -56,7 +56,8 @@ def problem(fmt, M, N, K, seed):
 CASES = [(4, 5, 640, 512, "simt", "simt"), (8, 3, 300, 256, "simt", "simt"),
          (4, 80, 2048, 512, "tc", "tc_w_stationary"), (8, 80, 512, 2048, "tc", "tc_w_stationary"),
          (3, 48, 1001, 512, "tc", "tc_w_stationary"), (4, 300, 1000, 512, "tc", "tc_x_resident"),
-         (8, 700, 384, 576, "tc", "tc_w_streamed"), (3, 2048, 512, 2048, "tc", "tc_w_streamed")]
+         (8, 700, 384, 576, "tc", "tc_w_streamed"), (3, 2048, 512, 2048, "tc", "tc_w_streamed"),
+         (4, 16400, 640, 128, "tc", "tc_x_resident_pair")]
 
 
 @pytest.mark.parametrize("fmt,M,N,K,path,kernel", CASES)

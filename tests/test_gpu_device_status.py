@@ -66,6 +66,7 @@ CASES = [
     (4, 80, 256, 128, "tc_w_stationary"),     # K split over clusters of 2 CTAs
     (8, 80, 512, 2048, "tc_w_stationary"),    # K split over clusters of 8 CTAs
     (4, 300, 512, 512, "tc_x_resident"),
+    (4, 16500, 384, 256, "tc_x_resident_pair"),
     (8, 300, 512, 1024, "tc_w_streamed"),
     (4, 700, 384, 768, "tc_w_streamed"),
 ]
@@ -121,10 +122,10 @@ def test_injected_timeout_in_grouped_block_launch(rtq_lib):
 
 
 @pytest.mark.parametrize("M,kernel", [(80, "tc_w_stationary"), (80, "tc_w_stationary_split"),
-                                      (300, "tc_x_resident")])
+                                      (300, "tc_x_resident"), (16500, "tc_x_resident_pair")])
 def test_activation_outside_fp16_range_is_reported(rtq_lib, M, kernel):
     N, K = {"tc_w_stationary": (256, 64), "tc_w_stationary_split": (512, 2048),
-            "tc_x_resident": (256, 512)}[kernel]
+            "tc_x_resident": (256, 512), "tc_x_resident_pair": (256, 256)}[kernel]
     X, q, _ = _problem(8, M, N, K, seed=970 + M)
     X[M // 2, 3] = 1.0e5                         # rounds to +inf in fp16
     Xd, Wd, Sd = dev(X), dev(q[0]), dev(q[1])

@@ -85,7 +85,8 @@ def test_identity_input_bit_exact(rtq_lib, path):
 
 SHAPES = [(5, 640, 1024, "simt"), (80, 512, 2048, "tc_w_stationary"),
           (1, 128, 64, "tc_w_stationary"), (300, 1000, 512, "tc_x_resident"),
-          (700, 384, 576, "tc_w_streamed"), (2048, 512, 2048, "tc_w_streamed")]
+          (700, 384, 576, "tc_w_streamed"), (2048, 512, 2048, "tc_w_streamed"),
+          (16400, 256, 128, "tc_x_resident_pair")]
 
 
 @pytest.mark.parametrize("M,N,K,kernel", SHAPES)

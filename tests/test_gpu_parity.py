@@ -277,13 +277,59 @@ def test_x_resident_long_runs_every_tile(rtq_lib):
     X = dev(wl.activations(M, K, 5010))
     Wq, sm = q4_weights(N, K, 5005, outliers=True)
     Wd, Sd = dev(Wq), dev(sm)
-    assert rtq_lib.plan(4, M, N, K) == "tc_x_resident"
+    assert rtq_lib.plan(4, M, N, K) == "tc_x_resident_pair"
     ys = rtq_lib.qgemm_q4(X, Wd, Sd, path="simt")
     scale = ys.abs().max()
     for _ in range(2):
         yt = rtq_lib.qgemm_q4(X, Wd, Sd, path="tc")
         tile_err = ((yt - ys).abs() / scale).view(M // 128, 128, N // 128, 128).amax(dim=(1, 3))
         assert float(tile_err.max()) <= TC_TOL, int((tile_err > TC_TOL).sum())
+
+
+# the CTA-pair activation-resident kernel (from M = 16384): ragged M, an odd
+# number of 128-row weight tiles (the last pair's second CTA holds rows past
+# N), K from 128 to 512
+XP_SHAPES = [(16384, 640, 512), (16500, 700, 384), (17000, 256, 128), (16400, 1000, 256)]
+
+
+@pytest.mark.parametrize("fmt", [4, 8])
+@pytest.mark.parametrize("M,N,K", XP_SHAPES)
+def test_x_resident_pair_parity(rtq_lib, fmt, M, N, K):
+    """Every 128 x 128 output tile against the fp32 SIMT path on the same
+    inputs, and 64 sampled rows (among them the first and last of every
+    192-row activation block's two halves near the ends) against the
+    oracle."""
+    assert rtq_lib.plan(fmt, M, N, K) == "tc_x_resident_pair"
+    Xh = wl.activations(M, K, 7100 + M + fmt)
+    q = q4_weights(N, K, 7101 + N, outliers=True) if fmt == 4 else q8_weights(N, K, 7101 + N, True)
+    fn = rtq_lib.qgemm_q4 if fmt == 4 else rtq_lib.qgemm_q8
+    X, Wd, Sd = dev(Xh), dev(q[0]), dev(q[1])
+    yt = fn(X, Wd, Sd, path="tc")
+    ys = fn(X, Wd, Sd, path="simt")
+    scale = ys.abs().max()
+    mt, nt = (M + 127) // 128, (N + 127) // 128
+    pad = torch.zeros((mt * 128, nt * 128), device="cuda")
+    pad[:M, :N] = (yt - ys).abs() / scale
+    tile_err = pad.view(mt, 128, nt, 128).amax(dim=(1, 3))
+    assert float(tile_err.max()) <= TC_TOL, int((tile_err > TC_TOL).sum())
+    rng = np.random.default_rng(M + N + K)
+    rows = np.unique(np.concatenate([[0, 95, 96, 191, 192, M - 1], rng.integers(0, M, 58)]))
+    gemm = oracle.gemm_q4 if fmt == 4 else oracle.gemm_q8
+    ref = gemm(np.ascontiguousarray(Xh[rows]), *q)
+    assert rel_err(yt[rows].cpu().numpy(), ref) <= MAX_REL["tc"]
+
+
+def test_x_resident_pair_identity_bit_exact(rtq_lib):
+    """X made of 16384 rows of the identity's 256 rows, over and over: every
+    output is one weight rounded to fp16, in both CTAs' rows of every tile."""
+    N, K = 1152, 256
+    Wq, sm = q4_weights(N, K, seed=93, outliers=True)
+    M = 16384
+    assert rtq_lib.plan(4, M, N, K) == "tc_x_resident_pair"
+    X = torch.eye(K, device="cuda").repeat(M // K, 1)
+    Y = rtq_lib.qgemm_q4(X, dev(Wq), dev(sm)).cpu().numpy()
+    ref = oracle.dequant_q4(Wq, sm).astype(np.float16).astype(np.float32).T
+    assert np.array_equal(Y, np.tile(ref, (M // K, 1)))
 
 
 def test_x_resident_identity_bit_exact(rtq_lib):

@@ -9,7 +9,9 @@ the workspace, so the two must agree bit for bit.  Checked here:
     does the same pair run again over the stale array;
   - those later calls change the free device memory by nothing;
   - the other kernels (SIMT, weight-stationary, weight-streamed q4) agree too;
-  - a problem above the scratch limit is rejected and Y is left untouched.
+  - a weight-streamed problem above the scratch limit is rejected and Y is
+    left untouched, while the CTA-pair activation-resident kernel, which
+    rounds the activations inside the kernel, runs at a size above it.
 The file runs alone in a fresh process as well as after the other tests.
 """
 import pytest
@@ -86,6 +88,7 @@ def test_two_calls_in_a_row_match_the_workspace_entry_point():
     (8, 80, 512, 512, "auto"),       # weight-stationary tcgen05
     (4, 300, 640, 1024, "tc"),       # weight-streamed q4
     (8, 4096, 512, 512, "tc"),       # activation-resident
+    (4, 20000, 256, 512, "auto"),    # CTA pairs, no scratch; M * K * 2 above the scratch size
 ])
 def test_other_kernels_match(fmt, M, N, K, path):
     X, Wq, S = _problem(fmt, M, N, K, seed=510 + M)
