@@ -101,6 +101,37 @@ cudaError_t launch_xs(int fmt, const void *Xh, const void *Wq, const void *S, co
 // rounding of each CTA's first activation block costs more than the
 // pre-pass saves.
 constexpr int kXpMinM = 16384;
+
+// Clusters of two CTAs of `kernel` (with this launch's block and shared
+// memory) that the device can hold at once.  Pairs must sit on two SMs of one
+// GPC, so the count can be below SMs / 2; a persistent grid larger than it
+// would run its last clusters as a second wave.  Cached per device.
+template <typename Kernel>
+int resident_pairs(Kernel kernel, const cudaLaunchConfig_t &cfg, int dev,
+                   std::atomic<int> (&cache)[kMaxDevices]) {
+    if (dev < 0 || dev >= kMaxDevices) return 1;
+    int n = cache[dev].load(std::memory_order_acquire);
+    if (n > 0) return n;
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaLaunchConfig_t q = cfg;
+    q.gridDim = dim3(2 * (sms / 2), 1, 1);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    q.attrs = attr;
+    q.numAttrs = 1;
+    int c = 0;
+    if (cudaOccupancyMaxActiveClusters(&c, kernel, &q) != cudaSuccess || c < 1) {
+        cudaGetLastError();
+        c = sms / 2;
+    }
+    cache[dev].store(c, std::memory_order_release);
+    return c;
+}
+
 cudaError_t launch_xp(int fmt, const float *X, const void *Wq, const void *S, const float *bias,
                       float *Y, int M, int N, int K, DevCtl *ctl, cudaStream_t s);
 

@@ -235,8 +235,8 @@ __global__ void __launch_bounds__(kXpThreads, 1)
             mbar_init(&raw_empty[i], kDeqGroups * kDeqThreads);
         }
         // the barriers both CTAs arrive on take one arrival per warp (an
-        // elected lane after __syncwarp): 256 remote arrivals per stage from
-        // the odd CTA cost about 1000 cycles, measured
+        // elected lane after __syncwarp), which keeps the cross-SM arrivals
+        // at 8 per CTA and stage
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sc_full[b], 1);
             mbar_init(&sc_empty[b], kDeqGroups * kDeqThreads);
@@ -586,17 +586,17 @@ cudaError_t launch_xp_fmt(const float *X, const void *Wq, const void *S, const f
         s_map = w_map;   // unused by the q8 kernel
     }
     if (!enc_ok) return cudaErrorInvalidValue;
-    int sms = 148;
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int n_o = (N + kTileRows - 1) / kTileRows;
     const int n_op = (n_o + 1) / 2;
     const int n_m = (M + kXpBlockRows - 1) / kXpBlockRows;
     const int items = n_op * n_m;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * std::min(items, sms / 2), 1, 1);
     cfg.blockDim = dim3(kXpThreads, 1, 1);
     cfg.dynamicSmemBytes = xp_layout(FMT, K).total + 1024;
     cfg.stream = st;
+    static std::atomic<int> pairs_cache[kMaxDevices];
+    const int pairs = resident_pairs(xp_qgemm_kernel<FMT>, cfg, dev, pairs_cache);
+    cfg.gridDim = dim3(2 * std::min(items, pairs), 1, 1);
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
