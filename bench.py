@@ -159,8 +159,71 @@ def recorded_traffic(kernel_key):
     return None
 
 
+class NvmlClockSampler:
+    """NVML sampling (read-only) of SM clock, power and throttle reasons every
+    ~2 ms during a window: the timed regions are milliseconds long, shorter
+    than nvidia-smi's sampling period."""
+    REASONS = (("hw_slowdown", "nvmlClocksThrottleReasonHwSlowdown", 0x8),
+               ("hw_thermal_slowdown", "nvmlClocksThrottleReasonHwThermalSlowdown", 0x40),
+               ("sw_thermal_slowdown", "nvmlClocksThrottleReasonSwThermalSlowdown", 0x20),
+               ("sw_power_cap", "nvmlClocksThrottleReasonSwPowerCap", 0x4))
+
+    def __init__(self, gpu_id):
+        import pynvml
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        if isinstance(gpu_id, str) and gpu_id.startswith("GPU-"):
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(gpu_id)
+        else:
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(int(gpu_id))
+        self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        self.masks = [(n, getattr(pynvml, a, d)) for n, a, d in self.REASONS]
+        self.samples = []
+        self.running = False
+
+    def start(self):
+        self.running = True
+        self.thread = threading.Thread(target=self._loop, daemon=True)
+        self.thread.start()
+
+    def _loop(self):
+        nv = self.nv
+        while self.running:
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                why = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                watts = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                self.samples.append((time.time(), mhz, why, watts))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def stop(self):
+        self.running = False
+        self.thread.join(timeout=2)
+
+    def summary(self, t0, t1):
+        rows = [r for r in self.samples if t0 <= r[0] <= t1] or self.samples[-3:]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        reasons = sorted({n for (_, _, why, _) in rows for n, m in self.masks if why & m})
+        return {"sm_mhz": statistics.median(r[1] for r in rows), "sm_max_mhz": self.max_mhz,
+                "sm_mhz_min": min(r[1] for r in rows), "reasons": reasons,
+                "power_w_median": round(statistics.median(r[3] for r in rows), 1),
+                "samples": len(rows), "source": "nvml, 2 ms"}
+
+
+def clock_sampler(gpu_id):
+    """NVML sampler, else the nvidia-smi one."""
+    try:
+        return NvmlClockSampler(gpu_id)
+    except Exception:
+        return ClockSampler(gpu_id)
+
+
 class ClockSampler:
-    """nvidia-smi sampling of SM clock and throttle reasons during a window."""
+    """nvidia-smi sampling of SM clock and throttle reasons during a window
+    (the fallback when NVML is not importable)."""
     FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -486,7 +549,7 @@ def measure_small_m(args, rank, world, local_rank, dev, stream, blocks=None):
         stream.synchronize()
         if rtq.device_status(stream) != 0:
             raise RuntimeError("device status word reports a fault during the small-M warm-up")
-        sampler = ClockSampler(gpu_uuid(dev, local_rank)) if sample_clocks else None
+        sampler = clock_sampler(gpu_uuid(dev, local_rank)) if sample_clocks else None
         if sampler:
             sampler.start()
             time.sleep(0.3)
@@ -598,7 +661,7 @@ def measure_large_m(args, rank, world, local_rank, dev, stream):
         if st:
             raise rtq.RtqError(st, "rt_qgemm_q4")
 
-    sampler = ClockSampler(gpu_uuid(dev, local_rank))
+    sampler = clock_sampler(gpu_uuid(dev, local_rank))
     sampler.start()
     time.sleep(0.3)
     if world > 1:
@@ -855,7 +918,7 @@ def run_gpu(args, rank, world, local_rank):
             step()
 
     # ---- timed region: K steps through the block driver
-    sampler = ClockSampler(gpu_uuid(dev, local_rank))
+    sampler = clock_sampler(gpu_uuid(dev, local_rank))
     sampler.start()
     time.sleep(0.3)
     e0 = torch.cuda.Event(enable_timing=True)
