@@ -14,7 +14,9 @@ Printed as one JSON line (rank 0):
              are captured once as a CUDA graph and replayed (config.issue;
              --eager issues them call by call);
   e2e        the same metric with the step's inputs copied from pinned host
-             memory and its outputs copied back inside the timed region;
+             memory and its outputs copied back inside the timed region (with
+             whole blocks, block by block on two copy streams beside the
+             compute stream, as a caller of the block driver would);
   roofline   the dominant kernel (the projection with the largest share of the
              step), its algorithmic bytes or flops per launch over its
              CUDA-event duration, against MEASURED_PEAKS.json;
@@ -1002,31 +1004,65 @@ def run_gpu(args, rank, world, local_rank):
         h2d = sum(h.numel() * 4 for h, _ in hx)
         d2h = sum(h.numel() * 4 for h, _ in hy)
         n_e2e = max(1, min(args.steps, args.e2e_steps))
-        with torch.cuda.stream(stream):
-            for h, dv in hx:
-                dv.copy_(h, non_blocking=True)
-            step()
-            for h, dv in hy:
-                h.copy_(dv, non_blocking=True)
+        s_in = torch.cuda.Stream(device=dev)
+        s_out = torch.cuda.Stream(device=dev)
+        nproj = len(projs)
+
+        def e2e_step():
+            """One step end to end.  With whole blocks, block by block on three
+            streams: block i's inputs are copied in on s_in while earlier blocks
+            compute, block i runs on the ABI's stream once they have landed, and
+            its outputs are copied out on s_out while later blocks compute (PCIe
+            carries both directions at once); the streams join at the end of the
+            step.  Otherwise all inputs in, the step, all outputs out."""
+            if not full_block:
+                with torch.cuda.stream(stream):
+                    for h, dv in hx:
+                        dv.copy_(h, non_blocking=True)
+                    step()
+                    for h, dv in hy:
+                        h.copy_(dv, non_blocking=True)
+                return
+            start = torch.cuda.Event()
+            start.record(stream)
+            s_in.wait_event(start)
+            s_out.wait_event(start)
+            for i in range(len(block_args)):
+                landed = torch.cuda.Event()
+                with torch.cuda.stream(s_in):
+                    for h, dv in hx[i * nproj:(i + 1) * nproj]:
+                        dv.copy_(h, non_blocking=True)
+                    landed.record(s_in)
+                stream.wait_event(landed)
+                with torch.cuda.stream(stream):
+                    run_block(i)
+                done = torch.cuda.Event()
+                done.record(stream)
+                s_out.wait_event(done)
+                with torch.cuda.stream(s_out):
+                    for h, dv in hy[i * nproj:(i + 1) * nproj]:
+                        h.copy_(dv, non_blocking=True)
+            out_done = torch.cuda.Event()
+            out_done.record(s_out)
+            stream.wait_event(out_done)
+
+        e2e_step()
         torch.cuda.synchronize(dev)
         barrier()
         f0 = torch.cuda.Event(enable_timing=True)
         f1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            f0.record(stream)
-            for _ in range(n_e2e):
-                for h, dv in hx:
-                    dv.copy_(h, non_blocking=True)
-                step()
-                for h, dv in hy:
-                    h.copy_(dv, non_blocking=True)
-            f1.record(stream)
+        f0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        f1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
         ms_e2e = max_over_ranks(f0.elapsed_time(f1)) / n_e2e
         e2e = {"value": job_value(world, flops, ms_e2e), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
-               "steps": n_e2e}
+               "steps": n_e2e,
+               "copies": ("per block on two copy streams beside the compute stream"
+                          if full_block else "all inputs, the step, all outputs, one stream")}
         del hx, hy
 
     # ---- the two gates of the metric, measured in the same run on the
