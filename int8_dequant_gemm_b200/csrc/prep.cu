@@ -20,6 +20,9 @@ namespace {
 __global__ void __launch_bounds__(256)
     cvt_x16_kernel(const float4 *__restrict__ X, uint4 *__restrict__ Xh, int64_t n_chunks,
                    DevCtl *ctl) {
+    // the next kernel may be scheduled now: it reads this one's output only
+    // after its own wait for this grid's completion
+    pdl_launch_dependents();
     pdl_wait_prior_grid();
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     uint32_t bad = 0;
@@ -32,7 +35,6 @@ __global__ void __launch_bounds__(256)
     }
     if (__any_sync(0xffffffffu, bad != 0) && (threadIdx.x & 31) == 0)
         atomicOr(&ctl->status, 1u << kStatusRange);
-    pdl_launch_dependents();
 }
 
 }  // namespace

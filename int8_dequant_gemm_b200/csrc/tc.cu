@@ -289,6 +289,9 @@ __device__ __forceinline__ void tc_tile(uint8_t *smem_raw, const float *__restri
         }
     }
     pdl_wait_prior_grid();
+    // the next kernel may be scheduled now (it reads this one's output only
+    // after its own wait for this grid's completion)
+    pdl_launch_dependents();
 
     if (warp < kConvWarps) {
         const ConvThread ct = conv_thread(threadIdx.x);
@@ -320,7 +323,6 @@ __device__ __forceinline__ void tc_tile(uint8_t *smem_raw, const float *__restri
                                         BN);
             if (!(ok = consume(r1, ks + 1))) break;
         }
-        pdl_launch_dependents();
         // ---------------------------------------------------------- epilogue
         if (ok) ok = mbar_wait(done, 0, lim);
         // tcgen05.ld is warp-collective: the whole warp takes the epilogue or none of it

@@ -168,6 +168,10 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    // The next kernel in the stream may be scheduled from here on: whatever it
+    // reads of this one's output it reads after its own wait for this grid's
+    // completion, and its CTAs take SMs only as this grid's leave them.
+    pdl_launch_dependents();
     bool ok = true;
 
     if (warp == kWTmaWarp) {
@@ -435,7 +439,6 @@ __global__ void __launch_bounds__(kWsThreads, 1)
             tc_fence_before_sync();
             mbar_arrive(&acc_empty[b]);
         }
-        pdl_launch_dependents();
     }
     if (!ok) atomicOr(&ctl->status, 1u << kStatusTimeout);
     tc_fence_before_sync();
