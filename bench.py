@@ -17,18 +17,22 @@ Printed as one JSON line (rank 0):
              memory and its outputs copied back inside the timed region (with
              whole blocks, block by block on two copy streams beside the
              compute stream, as a caller of the block driver would);
-  roofline   the dominant kernel (the projection with the largest share of the
-             step), its algorithmic bytes or flops per launch over its
-             CUDA-event duration, against MEASURED_PEAKS.json;
+  roofline   the dominant call of the step (the projection, or the block's
+             projections that share one launch of the activation-resident
+             kernel, with the largest share of the step), its algorithmic
+             bytes or flops over its CUDA-event duration, against
+             MEASURED_PEAKS.json;
   cpu_baseline  the CPU oracle on a bounded row sample of the same workload.
 
 `--impl reference` times the CPU oracle itself (rank 0 only) on the same
 workload, metric and unit, one bounded row sample per step.
 
 Other workloads (`--workload`), each printing one line of the same form:
-  block_m80, block_m2048
+  block_m80, block_m2048, block_m4096
                one block's projection set at M = 80 (one grouped launch; the
-               roofline object then describes that launch) and at M = 2048.
+               roofline object then describes that launch), at M = 2048 and at
+               M = 4096 (the default workload's first block, for profiler
+               captures).
   rot_m80      small M as an aggregate weight stream: the 12 blocks' weights in
                rotating device copies totalling ~4x L2, every copy's projection
                set at M = 80, 16 copies (64 projections) per rt_qgemm_batch
@@ -80,6 +84,9 @@ WORKLOADS = {
     "blocks12_m4096": (4, 12, 4096, ("qkvg", "wo", "w13", "w2")),
     "block_m80": (3, 1, 80, ("qkvg", "wo", "w13", "w2")),
     "block_m2048": (3, 1, 2048, ("qkvg", "wo", "w13", "w2")),
+    # one block of the default workload (175 MB of inputs and outputs, more
+    # than L2), sized for profiler captures of the block's grouped launch
+    "block_m4096": (4, 1, 4096, ("qkvg", "wo", "w13", "w2")),
     # single-projection cases sized for profiler captures
     "w13_m4096": (4, 1, 4096, ("w13",)),
     "w2_m4096": (4, 1, 4096, ("w2",)),
@@ -686,7 +693,7 @@ def measure_large_m(args, rank, world, local_rank, dev, stream):
         "unit": "TFLOP/s", "us_per_call": us,
         "frac_of_dense_peak": flops / (us * 1e-6) / 1e12 / peaks["bf16_tflops"],
         "dense_peak_tflops": peaks["bf16_tflops"], "kernel": rtq.plan(4, M, N, K),
-        "launches_per_call": 2,
+        "launches_per_call": 1 if rtq.plan(4, M, N, K) == "tc_x_resident_pair" else 2,
         "config": {"shape": "q4 512->2048", "M": M, "path": "auto", "calls_per_graph": 5,
                    "outliers": "1% of groups x20", "l2": "X 128 MiB + Y 512 MiB > L2"},
         "roofline": r, "clocks": sampler.summary(t0, t1),
@@ -866,18 +873,32 @@ def run_gpu(args, rank, world, local_rank):
                     raise rtq.RtqError(st, "rt_qgemm")
 
     # the TMA-fed kernels add an activation pre-pass launch; the block driver
-    # runs a small-M block as one grouped launch
+    # runs a small-M block as one grouped launch, and above 128 rows the
+    # projections that take the one-CTA activation-resident kernel (if two or
+    # more do) as one pre-pass launch and one launch of that kernel
+    def plan_of(name):
+        fmt, N, K = proj_dims(name)
+        return rtq.plan(4 if fmt == "q4" else 8, M, N, K)
+
+    def call_launches_of(name):
+        return 2 if plan_of(name) in ("tc_x_resident", "tc_w_streamed") else 1
+
     if full_block and per_fmt:
         fused_block = L.rt_qblock_fused_fmt(ctypes.byref(block_args[0][0]), M, 0) == 1
     else:
         fused_block = full_block and rtq.block_fused(M, wl.D_MODEL, wl.D_FF) == 1
+    grouped = []
+    if full_block and not fused_block:
+        grouped = [n for n in projs if plan_of(n) == "tc_x_resident"]
+        if len(grouped) < 2:
+            grouped = []
     if fused_block:
         launches_per_step = nblocks
+    elif full_block:
+        launches_per_step = nblocks * ((2 if grouped else 0) +
+                                       sum(call_launches_of(n) for n in projs if n not in grouped))
     else:
-        launches_per_step = sum(
-            2 if rtq.plan(4 if proj_dims(name)[0] == "q4" else 8, M, *proj_dims(name)[1:])
-            in ("tc_x_resident", "tc_w_streamed") else 1
-            for name, _, _ in calls)
+        launches_per_step = sum(call_launches_of(name) for name, _, _ in calls)
 
     def barrier():
         if world > 1:
@@ -895,7 +916,7 @@ def run_gpu(args, rank, world, local_rank):
         raise RuntimeError("device status word reports a fault during warm-up")
 
     # ---- the step captured once as a CUDA graph, so that the host's cost of
-    # issuing 96 launches stays out of the timed region; if the capture is
+    # issuing the step's launches stays out of the timed region; if the capture is
     # refused, the step is issued call by call instead (named in config.issue)
     graph, issue = None, "eager"
     if not args.eager:
@@ -946,12 +967,31 @@ def run_gpu(args, rank, world, local_rank):
     # 20 back-to-back calls (a block run as one grouped launch is timed as
     # that launch); the sum over the step is checked against ms_per_step
     reps = 20
+    group_key = "+".join(grouped)
     if fused_block:
         kern_us = {"block": graph_time_us(stream, lambda: run_block(0), reps, args.steps,
                                           args.warmup)}
     else:
         kern_us = {}
+        if grouped:
+            # block 0's grouped projections as the block driver runs them: an
+            # rt_qgemm_batch list above 128 rows takes the same grouped launch
+            garr = (rtq._QProjC * len(grouped))()
+            for i, n in enumerate(grouped):
+                fmt, N, K = proj_dims(n)
+                Wq, S, X, Y = dblocks[0][n]
+                garr[i] = rtq._QProjC(4 if fmt == "q4" else 8, 0, X.data_ptr(), Wq.data_ptr(),
+                                      S.data_ptr(), None, Y.data_ptr(), N, K)
+
+            def group_call():
+                st = L.rt_qgemm_batch(garr, len(grouped), M, 0, sptr)
+                if st:
+                    raise rtq.RtqError(st, "rt_qgemm_batch")
+            kern_us[group_key] = graph_time_us(stream, group_call, reps, args.steps, args.warmup)
         for name, fn, a in calls[:len(projs)]:
+            if name in grouped:
+                continue
+
             def one(fn=fn, a=a):
                 st = fn(*a)
                 if st:
@@ -974,19 +1014,29 @@ def run_gpu(args, rank, world, local_rank):
         kernel_key = f"block_grouped_tc_M{M}"
         call_launches = 1
     else:
-        share = {n: kern_us[n] * nblocks for n in projs}
+        share = {n: kern_us[n] * nblocks for n in kern_us}
         dom = max(share, key=share.get)
-        fmt, N, K = proj_dims(dom)
-        fcode = 4 if fmt == "q4" else 8
-        path = "tc" if rtq.auto_path(fcode, M, N, K) == 2 else "simt"
-        b_alg, f_alg = proj_bytes(dom, M), proj_flops(dom, M)
-        kernel_key = f"{dom}_{fmt}_{path}_M{M}"
-        call_launches = 2 if rtq.plan(fcode, M, N, K) in ("tc_x_resident", "tc_w_streamed") else 1
+        if dom == group_key:
+            b_alg = sum(proj_bytes(p, M) for p in grouped)
+            f_alg = sum(proj_flops(p, M) for p in grouped)
+            kernel_key = f"group_{group_key}_M{M}"
+            call_launches = 2
+        else:
+            fmt, N, K = proj_dims(dom)
+            fcode = 4 if fmt == "q4" else 8
+            path = "tc" if rtq.auto_path(fcode, M, N, K) == 2 else "simt"
+            b_alg, f_alg = proj_bytes(dom, M), proj_flops(dom, M)
+            kernel_key = f"{dom}_{fmt}_{path}_M{M}"
+            call_launches = call_launches_of(dom)
+    if dom == "block":
+        dom_plan = "tc_w_stationary (grouped)"
+    elif dom == group_key:
+        dom_plan = "tc_x_resident (one launch for " + ", ".join(grouped) + ")"
+    else:
+        dom_plan = plan_of(dom)
     roof = roofline(f_alg, b_alg, kern_us[dom] * 1e-6, peaks)
     roof.update({"traffic": recorded_traffic(kernel_key), "kernel": kernel_key,
-                 "kernel_plan": (rtq.plan(4 if proj_dims(dom)[0] == "q4" else 8, M,
-                                          *proj_dims(dom)[1:]) if dom != "block"
-                                 else "tc_w_stationary (grouped)"),
+                 "kernel_plan": dom_plan,
                  "launches_per_call": call_launches, "avg_call_us": kern_us[dom],
                  "timed_as": "one call, 20 per CUDA graph, mean over replays",
                  "share_of_step": share[dom] / sum(share.values())})

@@ -44,7 +44,8 @@
  *     enqueued".  Conditions found later on the device (a bounded wait that
  *     gave up, an activation outside the fp16 range) are latched in a device
  *     status word read by rt_device_status().
- *   - Alignment: X, Y and Wq 16-byte aligned; scale_min 4-byte aligned; scale
+ *   - Alignment: X, Y and Wq 16-byte aligned; scale_min 4-byte aligned (16
+ *     for the TMA-fed kernels above 128 rows, see rt_qgemm_plan); scale
  *     4-byte aligned.  Otherwise RT_ERR_ALIGNMENT.
  *   - Shapes: M >= 0 (M == 0 is a no-op), N >= 1, K >= 1; q4 needs K % 32 == 0
  *     (the group size); q8 needs K % 16 == 0.  The tensor-core path also needs
@@ -186,7 +187,11 @@ typedef enum rt_kernel {
     RT_KERNEL_TC_X_RESIDENT_PAIR = 6
 } rt_kernel;
 
-/* The kernel a GEMM of this format, shape and path runs; -1 if rejected. */
+/* The kernel a GEMM of this format, shape and path runs; -1 if rejected.
+ * The plan assumes a 16-byte aligned q4 scale_min: the TMA-fed kernels
+ * (RT_KERNEL_TC_X_RESIDENT, _W_STREAMED, _X_RESIDENT_PAIR) read it through a
+ * tensor map, so a q4 call whose scale_min is only 4-byte aligned runs on
+ * RT_KERNEL_TC_W_STATIONARY instead (same results, any M). */
 int rt_qgemm_plan(int fmt, int64_t M, int64_t N, int64_t K, int path);
 
 /*
@@ -274,9 +279,18 @@ rt_status rt_qgemm_noalloc(int fmt, const float *X, const void *Wq, const void *
  * The host encodes a TMA tensor map per entry's weights (cached per thread
  * by pointer and shape); Wq must be 16-byte aligned.  Under
  * RT_PATH_AUTO this happens only when the entries hold at least as many
- * 128-row weight tiles as the GPU has SMs.  Otherwise the entries run one
- * after another as rt_qgemm_q4/q8 calls.  Results are those of the
- * tensor-core path (<= 4e-3) and do not depend on the entries' order.
+ * 128-row weight tiles as the GPU has SMs.  Otherwise the entries run as
+ * rt_qgemm calls would, except that entries which take
+ * RT_KERNEL_TC_X_RESIDENT (M > 128) share launches: in list order, up to
+ * four of them at a time (q4 scale_min 16-byte aligned) run as one pre-pass
+ * launch that rounds each one's X into its own slice of the stream's
+ * workspace and one launch of the activation-resident kernel that walks all
+ * their tiles, so they share one pipeline fill and drain and one wave tail.
+ * A grouped entry gets the bits a single rt_qgemm call would give.
+ * Workspace of such a list: the sum of M * K * 2 over the largest launch's
+ * entries, or M * K * 2 of the largest other entry that stages X, whichever
+ * is larger.  Results are those of the tensor-core path (<= 4e-3) and do
+ * not depend on the entries' order.
  */
 typedef struct rt_qproj {
     int32_t fmt;
@@ -315,8 +329,13 @@ int rt_qgemm_batch_plan(const rt_qproj *list, int count, int64_t M, int path);
  * the projections and a slice of its K; each projection splits K by its own
  * factor (so w2, with four times the K of the others, splits four times as
  * far) and reduces the slices in distributed shared memory in a fixed order.
- * Otherwise the four run one after another on `stream` in the order qkvg,
- * wo, w13, w2, each as rt_qgemm_q4/q8 would.
+ * Otherwise they run on `stream` as rt_qgemm_batch runs the list (qkvg, wo,
+ * w13, w2) on its per-entry route: the projections that take
+ * RT_KERNEL_TC_X_RESIDENT (128 < M < 16384, K <= 512: qkvg, wo and w13 of
+ * RT-J) share one pre-pass launch and one activation-resident launch, the
+ * others run one call each, as rt_qgemm_q4/q8 would.  Workspace: the sum of
+ * M * K * 2 over the projections that share the launch, or M * K * 2 of a
+ * single call that stages X, whichever is larger (M = 4096 RT-J: 16 MiB).
  *
  * Validation: each product as in rt_qgemm_q4/q8; in addition no output may
  * overlap another projection's output, activations, codes or scales

@@ -142,6 +142,15 @@ int pick_kernel(int fmt, int64_t M, int64_t N, int64_t K, int p) {
     return RT_KERNEL_TC_W_STATIONARY;
 }
 
+// The TMA-fed kernels read q4 (scale, min) rows through a tensor map, whose
+// base must be 16-byte aligned; a q4 call whose scales are only 4-byte
+// aligned runs on the weight-stationary kernel instead (any M).
+int kernel_for_scales(int kern, int fmt, const void *S) {
+    const bool tma = kern == RT_KERNEL_TC_X_RESIDENT || kern == RT_KERNEL_TC_W_STREAMED ||
+                     kern == RT_KERNEL_TC_X_RESIDENT_PAIR;
+    return (tma && fmt == 4 && !aligned(S, 16)) ? RT_KERNEL_TC_W_STATIONARY : kern;
+}
+
 int pick_path(int fmt, int64_t M, int64_t K, int path) {
     const bool tc_ok = (K % 64) == 0;
     if (path == RT_PATH_TC) return tc_ok ? path : -1;
@@ -162,7 +171,7 @@ rt_status run_gemm(int fmt, const float *X, const void *Wq, const void *S, const
     if (M == 0) return RT_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
-    const int kern = pick_kernel(fmt, M, N, K, p);
+    const int kern = kernel_for_scales(pick_kernel(fmt, M, N, K, p), fmt, S);
     if (kern == RT_KERNEL_SIMT) return from_cuda(rtq::launch_simt(fmt, X, Wq, S, bias, Y, m, n, k, s));
     DevCtl *ctl = nullptr;
     rt_status st = ctl_block(&ctl);
@@ -194,6 +203,11 @@ rt_status check_gemm_args(int fmt, const float *X, const void *Wq, const void *S
 }
 
 rt_status device_ctl(DevCtl **out) { return ctl_block(out); }
+
+int plan_with_scales(int fmt, int64_t M, int64_t N, int64_t K, int path, const void *S) {
+    const int kern = rt_qgemm_plan(fmt, M, N, K, path);
+    return kern < 0 ? kern : kernel_for_scales(kern, fmt, S);
+}
 
 }  // namespace rtq
 
@@ -309,6 +323,91 @@ struct BlockProj {
     int64_t N, K;
 };
 
+// Runs validated projections with the same M on `stream`.  Those that take
+// the one-CTA activation-resident kernel run, in list order, in launches of
+// up to kMaxGroup of them (a chunk of one runs as a plain call): one pre-pass
+// launch rounds the chunk's activations into slices of the workspace, then
+// one launch of the kernel walks all of the chunk's tiles, so the chunk
+// shares one pipeline fill and drain and one wave tail.  The others run one
+// call each, reusing the workspace from its start.  The workspace is sized
+// once, before anything is queued, for the largest chunk and every single
+// call.
+rt_status run_list(const BlockProj *p, int count, int64_t M, int path, void *stream) {
+    if (M == 0) return RT_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    std::vector<int> chunk_of(static_cast<size_t>(count), -1);
+    std::vector<std::vector<int>> chunks;
+    std::vector<int> open;
+    int64_t need = 0;
+    auto close = [&]() {
+        if (open.size() >= 2) {
+            std::vector<rtq::XsInput> in;
+            int64_t bytes = 0;
+            for (int i : open) {
+                in.push_back({p[i].fmt, nullptr, p[i].W, p[i].S, p[i].bias, p[i].Y,
+                              static_cast<int>(p[i].N), static_cast<int>(p[i].K)});
+                bytes += M * p[i].K * 2;
+            }
+            if (rtq::xs_group_supported(in.data(), static_cast<int>(in.size()),
+                                        static_cast<int>(M))) {
+                for (int i : open) chunk_of[i] = static_cast<int>(chunks.size());
+                chunks.push_back(open);
+                need = std::max(need, bytes);
+            }
+        }
+        open.clear();
+    };
+    for (int i = 0; i < count; ++i) {
+        const BlockProj &q = p[i];
+        const int kern = kernel_for_scales(
+            pick_kernel(q.fmt, M, q.N, q.K, pick_path(q.fmt, M, q.K, path)), q.fmt, q.S);
+        if (kern == RT_KERNEL_TC_X_RESIDENT) {
+            open.push_back(i);
+            if (static_cast<int>(open.size()) == rtq::kMaxGroup) close();
+        }
+        if (kern == RT_KERNEL_TC_X_RESIDENT || kern == RT_KERNEL_TC_W_STREAMED)
+            need = std::max(need, M * q.K * 2);
+    }
+    close();
+    rt_status st;
+    void *ws = nullptr;
+    DevCtl *ctl = nullptr;
+    if (!chunks.empty() &&
+        ((st = workspace(s, static_cast<size_t>(need), &ws)) != RT_OK ||
+         (st = ctl_block(&ctl)) != RT_OK))
+        return st;
+    for (int i = 0; i < count; ++i) {
+        const BlockProj &q = p[i];
+        if (chunk_of[i] < 0) {
+            if ((st = run_gemm(q.fmt, q.X, q.W, q.S, q.bias, q.Y, M, q.N, q.K, path, stream)) !=
+                RT_OK)
+                return st;
+            continue;
+        }
+        const std::vector<int> &c = chunks[static_cast<size_t>(chunk_of[i])];
+        if (c.front() != i) continue;          // launched at its first member
+        const int n = static_cast<int>(c.size());
+        rtq::XsInput in[rtq::kMaxGroup];
+        const float *xs[rtq::kMaxGroup];
+        void *xh[rtq::kMaxGroup];
+        int64_t ks[rtq::kMaxGroup];
+        int64_t off = 0;                       // M * K * 2: multiples of 256 bytes
+        for (int g = 0; g < n; ++g) {
+            const BlockProj &e = p[c[static_cast<size_t>(g)]];
+            xs[g] = e.X;
+            xh[g] = static_cast<uint8_t *>(ws) + off;
+            ks[g] = e.K;
+            in[g] = {e.fmt, xh[g], e.W, e.S, e.bias, e.Y, static_cast<int>(e.N),
+                     static_cast<int>(e.K)};
+            off += M * e.K * 2;
+        }
+        if (rtq::launch_cvt_x16_group(xs, xh, ks, n, M, ctl, s) != cudaSuccess ||
+            rtq::launch_xs_group(in, n, static_cast<int>(M), ctl, s) != cudaSuccess)
+            return RT_ERR_CUDA;
+    }
+    return RT_OK;
+}
+
 // 1 if the block's four projections run as one grouped launch, 0 if one call
 // each, -1 if a format or size is rejected (shapes only; no pointers).
 int block_route(const int fmt[4], int64_t M, int64_t d, int64_t f, int path) {
@@ -367,12 +466,7 @@ rt_status block_run(const BlockProj p[4], int64_t M, int64_t d, int64_t f, int p
         return from_cuda(rtq::launch_tc_group(g, 4, static_cast<int>(M), ctl,
                                               static_cast<cudaStream_t>(stream)));
     }
-    for (int i = 0; i < 4; ++i) {
-        const BlockProj &q = p[i];
-        if ((st = run_gemm(q.fmt, q.X, q.W, q.S, q.bias, q.Y, M, q.N, q.K, path, stream)) != RT_OK)
-            return st;
-    }
-    return RT_OK;
+    return run_list(p, 4, M, path, stream);
 }
 
 // The int4 card's mixed recipe: qkvg and w13 in q4, wo and w2 in q8.
@@ -569,14 +663,12 @@ rt_status rt_qgemm_batch(const rt_qproj *list, int count, int64_t M, int path, v
     if (M == 0 || count == 0) return RT_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (route != RT_KERNEL_TC_LIST) {
-        rt_status st;
+        std::vector<BlockProj> p(static_cast<size_t>(count));
         for (int i = 0; i < count; ++i) {
             const rt_qproj &q = list[i];
-            if ((st = run_gemm(q.fmt, q.X, q.Wq, q.scales, q.bias, q.Y, M, q.N, q.K, path,
-                               stream)) != RT_OK)
-                return st;
+            p[i] = {q.fmt, q.X, q.Wq, q.scales, q.bias, q.Y, q.N, q.K};
         }
-        return RT_OK;
+        return run_list(p.data(), count, M, path, stream);
     }
     DevCtl *ctl = nullptr;
     rt_status st = ctl_block(&ctl);

@@ -82,16 +82,33 @@ cudaError_t launch_tc_group(const GroupProblem *probs, int count, int M, DevCtl 
 
 // Activation pre-pass of the TMA-fed kernels (prep.cu): X fp32 [M, K] ->
 // fp16 [M, K] in the operand chunk order, into Xh (M * K * 2 bytes); latches
-// kStatusRange for an activation fp16 cannot hold.
+// kStatusRange for an activation fp16 cannot hold.  launch_cvt_x16_group
+// rounds up to kMaxGroup such tensors (each M x K[i], K[i] a multiple of 8)
+// in one launch.
 cudaError_t launch_cvt_x16(const float *X, void *Xh, int64_t M, int64_t K, DevCtl *ctl,
                            cudaStream_t s);
+cudaError_t launch_cvt_x16_group(const float *const *X, void *const *Xh, const int64_t *K,
+                                 int count, int64_t M, DevCtl *ctl, cudaStream_t s);
 
 // tcgen05, activation block resident in shared memory, TMA-streamed weights
 // (K a multiple of 128 up to 512, many activation rows); see xs.cu.  Xh is the
-// pre-pass output.
+// pre-pass output.  launch_xs_group runs up to kMaxGroup such products with
+// the same M in one persistent launch (xs_group_supported: the lists it
+// takes: K a multiple of 128 up to 512, q4 scales 16-byte aligned).
+struct XsInput {
+    int fmt;
+    const void *Xh;
+    const void *Wq;
+    const void *S;
+    const float *bias;
+    float *Y;
+    int N, K;
+};
 bool xs_supported(int M, int N, int K);
+bool xs_group_supported(const XsInput *in, int count, int M);
 cudaError_t launch_xs(int fmt, const void *Xh, const void *Wq, const void *S, const float *bias,
                       float *Y, int M, int N, int K, DevCtl *ctl, cudaStream_t s);
+cudaError_t launch_xs_group(const XsInput *in, int count, int M, DevCtl *ctl, cudaStream_t s);
 
 // The same activation-resident product on CTA pairs (cta_group::2, 256 weight
 // rows per MMA), rounding fp32 X to fp16 inside the kernel; see xp.cu.  Same
@@ -179,6 +196,9 @@ cudaError_t launch_dequant_e4m3(const uint8_t *Wq, void *W, int N, int K, bool f
 rt_status check_gemm_args(int fmt, const float *X, const void *Wq, const void *S, const float *Y,
                           int64_t M, int64_t N, int64_t K);
 rt_status device_ctl(DevCtl **out);
+// rt_qgemm_plan's kernel for this call's scale pointer: q4 scales that are
+// not 16-byte aligned move a TMA-fed plan to the weight-stationary kernel.
+int plan_with_scales(int fmt, int64_t M, int64_t N, int64_t K, int path, const void *S);
 
 // Largest M the SIMT path takes under RT_PATH_AUTO, per format: where a
 // single call of the fp32 SIMT kernel beats the tensor-core kernels in the M

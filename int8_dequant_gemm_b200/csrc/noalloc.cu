@@ -57,7 +57,7 @@ extern "C" rt_status rt_qgemm_noalloc(int fmt, const float *X, const void *Wq, c
     rt_status st = rtq::check_gemm_args(fmt, X, Wq, scales, Y, M, N, K);
     if (st != RT_OK) return st;
     if (path < RT_PATH_AUTO || path > RT_PATH_TC) return RT_ERR_INVALID_ARG;
-    const int kern = rt_qgemm_plan(fmt, M, N, K, path);
+    const int kern = rtq::plan_with_scales(fmt, M, N, K, path, scales);
     if (kern < 0) return RT_ERR_UNSUPPORTED_SHAPE;
     const bool staged = kern == RT_KERNEL_TC_X_RESIDENT || kern == RT_KERNEL_TC_W_STREAMED;
     if (staged && M * K * 2 > static_cast<int64_t>(RT_NOALLOC_SCRATCH_BYTES))

@@ -37,27 +37,82 @@ __global__ void __launch_bounds__(256)
         atomicOr(&ctl->status, 1u << kStatusRange);
 }
 
-}  // namespace
+// The same rounding over up to kMaxGroup tensors, one grid-stride walk over
+// their concatenated 8-element chunks (end[i]: running chunk totals).
+struct CvtGroup {
+    const float4 *X[kMaxGroup];
+    uint4 *Xh[kMaxGroup];
+    int64_t end[kMaxGroup];
+    int count;
+};
 
-cudaError_t launch_cvt_x16(const float *X, void *Xh, int64_t M, int64_t K, DevCtl *ctl,
-                           cudaStream_t s) {
-    const int64_t n_chunks = M * K / 8;
+__global__ void __launch_bounds__(256) cvt_x16_group_kernel(const __grid_constant__ CvtGroup g,
+                                                            DevCtl *ctl) {
+    pdl_launch_dependents();
+    pdl_wait_prior_grid();
+    const int64_t total = g.end[g.count - 1];
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    uint32_t bad = 0;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += stride) {
+        int t = 0;
+        while (i >= g.end[t]) ++t;
+        const int64_t c = i - (t > 0 ? g.end[t - 1] : 0);
+        const float4 a = __ldcs(g.X[t] + 2 * c), b = __ldcs(g.X[t] + 2 * c + 1);
+        const uint4 v = x8_f16(a, b);
+        bad |= f16x2_nonfinite(make_uint2(v.x, v.y)) | f16x2_nonfinite(make_uint2(v.z, v.w));
+        g.Xh[t][c] = v;
+    }
+    if (__any_sync(0xffffffffu, bad != 0) && (threadIdx.x & 31) == 0)
+        atomicOr(&ctl->status, 1u << kStatusRange);
+}
+
+// Launch shape of a pre-pass over n_chunks chunks: 256 threads a block, at
+// most 8 blocks per SM, programmatic dependent launch.
+cudaLaunchConfig_t cvt_config(int64_t n_chunks, cudaStream_t s, cudaLaunchAttribute *attr) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t want = (n_chunks + 255) / 256;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>(want, 8LL * sms)), 1, 1);
+    cfg.gridDim = dim3(static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(want, 8LL * sms))), 1, 1);
     cfg.blockDim = dim3(256, 1, 1);
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    return cfg;
+}
+
+}  // namespace
+
+cudaError_t launch_cvt_x16(const float *X, void *Xh, int64_t M, int64_t K, DevCtl *ctl,
+                           cudaStream_t s) {
+    const int64_t n_chunks = M * K / 8;
+    cudaLaunchAttribute attr[1];
+    const cudaLaunchConfig_t cfg = cvt_config(n_chunks, s, attr);
     const float4 *x4 = reinterpret_cast<const float4 *>(X);
     uint4 *h = static_cast<uint4 *>(Xh);
     return cudaLaunchKernelEx(&cfg, cvt_x16_kernel, x4, h, n_chunks, ctl);
+}
+
+cudaError_t launch_cvt_x16_group(const float *const *X, void *const *Xh, const int64_t *K,
+                                 int count, int64_t M, DevCtl *ctl, cudaStream_t s) {
+    if (count < 1 || count > kMaxGroup) return cudaErrorInvalidValue;
+    CvtGroup g = {};
+    g.count = count;
+    int64_t total = 0;
+    for (int i = 0; i < count; ++i) {
+        g.X[i] = reinterpret_cast<const float4 *>(X[i]);
+        g.Xh[i] = static_cast<uint4 *>(Xh[i]);
+        total += M * K[i] / 8;
+        g.end[i] = total;
+    }
+    if (total == 0) return cudaSuccess;
+    cudaLaunchAttribute attr[1];
+    const cudaLaunchConfig_t cfg = cvt_config(total, s, attr);
+    return cudaLaunchKernelEx(&cfg, cvt_x16_group_kernel, g, ctl);
 }
 
 namespace {

@@ -4,7 +4,9 @@ scale, qkvg a q8 [2048, 512] tensor and w13 a q8 [4096, 512] tensor
 ("RT-J -- int8 (Q8_0-style) quantized checkpoints", "Quantization format").
 
 At M = 80 the four projections run as one grouped launch; at M = 2048 and
-4096 one call each on the TMA-fed kernels (checked on sampled rows).  A block
+4096 qkvg, wo and w13 share one launch of the activation-resident kernel
+(its q8 build) and w2 runs on the weight-streamed kernel (checked on sampled
+rows).  A block
 with the int4 card's mixed formats through the same entry point must give
 the bits of rt_qblock_project.
 """
