@@ -86,6 +86,50 @@ rt_status workspace(cudaStream_t s, size_t need, void **out) {
     return RT_OK;
 }
 
+// A second stream and two events per (device, stream), on which pre-passes
+// run beside the stream's own launches (run_list).  Created on first need
+// outside any stream capture, kept until rt_workspace_release().
+struct SideStream {
+    cudaStream_t stream;
+    cudaEvent_t fork, join;
+};
+struct SideEntry {
+    int dev;
+    cudaStream_t owner;
+    SideStream side;
+};
+std::vector<SideEntry> g_side;   // guarded by g_ws_mu
+
+// The side stream of `s`; false if it does not exist and cannot be created
+// now (inside a capture, or a creation failed).
+bool side_stream(cudaStream_t s, SideStream *out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    std::lock_guard<std::mutex> lk(g_ws_mu);
+    for (const SideEntry &e : g_side)
+        if (e.dev == dev && e.owner == s) {
+            *out = e.side;
+            return true;
+        }
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone)
+        return false;
+    SideStream n = {};
+    if (cudaStreamCreateWithFlags(&n.stream, cudaStreamNonBlocking) != cudaSuccess) return false;
+    if (cudaEventCreateWithFlags(&n.fork, cudaEventDisableTiming) != cudaSuccess) {
+        cudaStreamDestroy(n.stream);
+        return false;
+    }
+    if (cudaEventCreateWithFlags(&n.join, cudaEventDisableTiming) != cudaSuccess) {
+        cudaEventDestroy(n.fork);
+        cudaStreamDestroy(n.stream);
+        return false;
+    }
+    g_side.push_back({dev, s, n});
+    *out = n;
+    return true;
+}
+
 inline bool aligned(const void *p, uintptr_t a) {
     return (reinterpret_cast<uintptr_t>(p) % a) == 0;
 }
@@ -306,6 +350,16 @@ rt_status rt_workspace_release(void) {
             ++it;
         }
     }
+    for (auto it = g_side.begin(); it != g_side.end();) {
+        if (it->dev == dev) {
+            cudaEventDestroy(it->side.fork);
+            cudaEventDestroy(it->side.join);
+            cudaStreamDestroy(it->side.stream);
+            it = g_side.erase(it);
+        } else {
+            ++it;
+        }
+    }
     return RT_OK;
 }
 
@@ -329,16 +383,19 @@ struct BlockProj {
 // launch rounds the chunk's activations into slices of the workspace, then
 // one launch of the kernel walks all of the chunk's tiles, so the chunk
 // shares one pipeline fill and drain and one wave tail.  The others run one
-// call each, reusing the workspace from its start.  The workspace is sized
-// once, before anything is queued, for the largest chunk and every single
-// call.
+// call each.  When a chunk runs beside calls that stage their activations
+// too (the weight-streamed kernel), those calls' pre-passes run on the
+// stream's second stream while the first chunk computes (in blocks that fit
+// beside its CTAs), each into a slice of its own, and the stream waits for
+// them before their GEMM launches, which come after the chunks.  The
+// workspace is sized once, before anything is queued.
 rt_status run_list(const BlockProj *p, int count, int64_t M, int path, void *stream) {
     if (M == 0) return RT_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    std::vector<int> chunk_of(static_cast<size_t>(count), -1);
+    std::vector<int> chunk_of(static_cast<size_t>(count), -1), kern_of(static_cast<size_t>(count));
     std::vector<std::vector<int>> chunks;
     std::vector<int> open;
-    int64_t need = 0;
+    int64_t chunk_need = 0, single_need = 0, staged_sum = 0;
     auto close = [&]() {
         if (open.size() >= 2) {
             std::vector<rtq::XsInput> in;
@@ -352,7 +409,7 @@ rt_status run_list(const BlockProj *p, int count, int64_t M, int path, void *str
                                         static_cast<int>(M))) {
                 for (int i : open) chunk_of[i] = static_cast<int>(chunks.size());
                 chunks.push_back(open);
-                need = std::max(need, bytes);
+                chunk_need = std::max(chunk_need, bytes);
             }
         }
         open.clear();
@@ -361,49 +418,106 @@ rt_status run_list(const BlockProj *p, int count, int64_t M, int path, void *str
         const BlockProj &q = p[i];
         const int kern = kernel_for_scales(
             pick_kernel(q.fmt, M, q.N, q.K, pick_path(q.fmt, M, q.K, path)), q.fmt, q.S);
+        kern_of[i] = kern;
         if (kern == RT_KERNEL_TC_X_RESIDENT) {
             open.push_back(i);
             if (static_cast<int>(open.size()) == rtq::kMaxGroup) close();
         }
-        if (kern == RT_KERNEL_TC_X_RESIDENT || kern == RT_KERNEL_TC_W_STREAMED)
-            need = std::max(need, M * q.K * 2);
     }
     close();
+    // calls outside the chunks that stage their activations
+    std::vector<int> staged;
+    for (int i = 0; i < count; ++i) {
+        if (chunk_of[i] >= 0) continue;
+        if (kern_of[i] == RT_KERNEL_TC_X_RESIDENT || kern_of[i] == RT_KERNEL_TC_W_STREAMED) {
+            staged.push_back(i);
+            single_need = std::max(single_need, M * p[i].K * 2);
+            staged_sum += M * p[i].K * 2;
+        }
+    }
     rt_status st;
+    if (chunks.empty()) {
+        for (int i = 0; i < count; ++i) {
+            const BlockProj &q = p[i];
+            if ((st = run_gemm(q.fmt, q.X, q.W, q.S, q.bias, q.Y, M, q.N, q.K, path, stream)) !=
+                RT_OK)
+                return st;
+        }
+        return RT_OK;
+    }
     void *ws = nullptr;
     DevCtl *ctl = nullptr;
-    if (!chunks.empty() &&
-        ((st = workspace(s, static_cast<size_t>(need), &ws)) != RT_OK ||
-         (st = ctl_block(&ctl)) != RT_OK))
+    SideStream side = {};
+    const bool overlap = !staged.empty() && side_stream(s, &side);
+    const int64_t need = overlap ? chunk_need + staged_sum : std::max(chunk_need, single_need);
+    if ((st = workspace(s, static_cast<size_t>(need), &ws)) != RT_OK ||
+        (st = ctl_block(&ctl)) != RT_OK)
         return st;
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    // slices of the staged calls' activations (overlap only), after the chunks'
+    std::vector<void *> slice(static_cast<size_t>(count), nullptr);
+    if (overlap) {
+        int64_t off = chunk_need;              // M * K * 2: multiples of 256 bytes
+        for (int i : staged) {
+            slice[i] = wsb + off;
+            off += M * p[i].K * 2;
+        }
+    }
+    bool forked = false;
+    cudaError_t e = cudaSuccess;
+    for (size_t c = 0; c < chunks.size() && e == cudaSuccess; ++c) {
+        const int n = static_cast<int>(chunks[c].size());
+        rtq::XsInput in[rtq::kMaxGroup];
+        const float *xs[rtq::kMaxGroup];
+        void *xh[rtq::kMaxGroup];
+        int64_t ks[rtq::kMaxGroup];
+        int64_t off = 0;
+        for (int g = 0; g < n; ++g) {
+            const BlockProj &q = p[chunks[c][static_cast<size_t>(g)]];
+            xs[g] = q.X;
+            xh[g] = wsb + off;
+            ks[g] = q.K;
+            in[g] = {q.fmt, xh[g], q.W, q.S, q.bias, q.Y, static_cast<int>(q.N),
+                     static_cast<int>(q.K)};
+            off += M * q.K * 2;
+        }
+        e = rtq::launch_cvt_x16_group(xs, xh, ks, n, M, ctl, s);
+        if (e == cudaSuccess && overlap && !forked) {
+            // the staged calls' pre-passes start once everything before this
+            // point on the stream has completed, beside the chunk's GEMM
+            forked = true;
+            e = cudaEventRecord(side.fork, s);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(side.stream, side.fork, 0);
+            for (size_t k = 0; k < staged.size() && e == cudaSuccess; ++k) {
+                const BlockProj &q = p[staged[k]];
+                e = rtq::launch_cvt_x16_lean(q.X, slice[staged[k]], M, q.K, ctl, side.stream);
+            }
+            const cudaError_t e2 = cudaEventRecord(side.join, side.stream);
+            if (e == cudaSuccess) e = e2;
+        }
+        if (e == cudaSuccess) e = rtq::launch_xs_group(in, n, static_cast<int>(M), ctl, s);
+    }
+    // the stream waits for the side stream's pre-passes after the chunks'
+    // launches (and always, so that a capture stays whole)
+    if (forked) {
+        const cudaError_t e3 = cudaStreamWaitEvent(s, side.join, 0);
+        if (e == cudaSuccess) e = e3;
+    }
+    if (e != cudaSuccess) return RT_ERR_CUDA;
     for (int i = 0; i < count; ++i) {
         const BlockProj &q = p[i];
-        if (chunk_of[i] < 0) {
+        if (chunk_of[i] >= 0) continue;
+        if (!overlap || slice[i] == nullptr) {
             if ((st = run_gemm(q.fmt, q.X, q.W, q.S, q.bias, q.Y, M, q.N, q.K, path, stream)) !=
                 RT_OK)
                 return st;
             continue;
         }
-        const std::vector<int> &c = chunks[static_cast<size_t>(chunk_of[i])];
-        if (c.front() != i) continue;          // launched at its first member
-        const int n = static_cast<int>(c.size());
-        rtq::XsInput in[rtq::kMaxGroup];
-        const float *xs[rtq::kMaxGroup];
-        void *xh[rtq::kMaxGroup];
-        int64_t ks[rtq::kMaxGroup];
-        int64_t off = 0;                       // M * K * 2: multiples of 256 bytes
-        for (int g = 0; g < n; ++g) {
-            const BlockProj &e = p[c[static_cast<size_t>(g)]];
-            xs[g] = e.X;
-            xh[g] = static_cast<uint8_t *>(ws) + off;
-            ks[g] = e.K;
-            in[g] = {e.fmt, xh[g], e.W, e.S, e.bias, e.Y, static_cast<int>(e.N),
-                     static_cast<int>(e.K)};
-            off += M * e.K * 2;
-        }
-        if (rtq::launch_cvt_x16_group(xs, xh, ks, n, M, ctl, s) != cudaSuccess ||
-            rtq::launch_xs_group(in, n, static_cast<int>(M), ctl, s) != cudaSuccess)
-            return RT_ERR_CUDA;
+        const int m = static_cast<int>(M), n = static_cast<int>(q.N), k = static_cast<int>(q.K);
+        e = kern_of[i] == RT_KERNEL_TC_X_RESIDENT
+                ? rtq::launch_xs(q.fmt, slice[i], q.W, q.S, q.bias, q.Y, m, n, k, ctl, s)
+                : rtq::launch_ws(q.fmt, slice[i], q.W, q.S, q.bias, q.Y, m, n, k, ctl, s);
+        if (e != cudaSuccess) return RT_ERR_CUDA;
     }
     return RT_OK;
 }

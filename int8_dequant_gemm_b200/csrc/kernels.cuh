@@ -84,9 +84,15 @@ cudaError_t launch_tc_group(const GroupProblem *probs, int count, int M, DevCtl 
 // fp16 [M, K] in the operand chunk order, into Xh (M * K * 2 bytes); latches
 // kStatusRange for an activation fp16 cannot hold.  launch_cvt_x16_group
 // rounds up to kMaxGroup such tensors (each M x K[i], K[i] a multiple of 8)
-// in one launch.
+// in one launch.  launch_cvt_x16_lean: the same rounding as one 128-thread
+// block per SM of at most 64 registers a thread (one warp per sub-partition),
+// which fits beside a CTA of the activation-resident kernel, for an input
+// rounded on a second stream while that kernel runs (no programmatic
+// dependent launch).
 cudaError_t launch_cvt_x16(const float *X, void *Xh, int64_t M, int64_t K, DevCtl *ctl,
                            cudaStream_t s);
+cudaError_t launch_cvt_x16_lean(const float *X, void *Xh, int64_t M, int64_t K, DevCtl *ctl,
+                                cudaStream_t s);
 cudaError_t launch_cvt_x16_group(const float *const *X, void *const *Xh, const int64_t *K,
                                  int count, int64_t M, DevCtl *ctl, cudaStream_t s);
 

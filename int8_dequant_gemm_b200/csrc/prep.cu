@@ -37,6 +37,48 @@ __global__ void __launch_bounds__(256)
         atomicOr(&ctl->status, 1u << kStatusRange);
 }
 
+// The same rounding in a shape that fits on each SM beside a persistent GEMM
+// CTA of another launch, for an input rounded on a second stream while that
+// launch computes.  Registers are split between an SM's four sub-partitions
+// (16384 each) and a block's warps are spread over them, so the block is one
+// warp per sub-partition: 128 threads of at most 64 registers (2048 a
+// sub-partition), which fits beside the activation-resident kernel's 5 warps
+// of 88 registers (14080) per sub-partition, with no shared memory; four
+// chunks in flight per thread.
+constexpr int kLeanThreads = 128;
+constexpr int kLeanDepth = 4;
+__global__ void __launch_bounds__(kLeanThreads, 8)
+    cvt_x16_lean_kernel(const float4 *__restrict__ X, uint4 *__restrict__ Xh, int64_t n_chunks,
+                        DevCtl *ctl) {
+    const uint32_t stride = gridDim.x * blockDim.x;       // chunks between a thread's chunks
+    uint32_t bad = 0;
+    int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const float4 *x = X + 2 * i;
+    uint4 *h = Xh + i;
+    for (; i + (kLeanDepth - 1) * static_cast<int64_t>(stride) < n_chunks;
+         i += kLeanDepth * stride, x += 2 * kLeanDepth * stride, h += kLeanDepth * stride) {
+        float4 a[kLeanDepth], b[kLeanDepth];
+#pragma unroll
+        for (int d = 0; d < kLeanDepth; ++d) {
+            a[d] = __ldcs(x + 2 * d * stride);
+            b[d] = __ldcs(x + 2 * d * stride + 1);
+        }
+#pragma unroll
+        for (int d = 0; d < kLeanDepth; ++d) {
+            const uint4 c = x8_f16(a[d], b[d]);
+            h[d * stride] = c;
+            bad |= f16x2_nonfinite(make_uint2(c.x, c.y)) | f16x2_nonfinite(make_uint2(c.z, c.w));
+        }
+    }
+    for (; i < n_chunks; i += stride, x += 2 * stride, h += stride) {
+        const uint4 c = x8_f16(__ldcs(x), __ldcs(x + 1));
+        h[0] = c;
+        bad |= f16x2_nonfinite(make_uint2(c.x, c.y)) | f16x2_nonfinite(make_uint2(c.z, c.w));
+    }
+    if (__any_sync(0xffffffffu, bad != 0) && (threadIdx.x & 31) == 0)
+        atomicOr(&ctl->status, 1u << kStatusRange);
+}
+
 // The same rounding over up to kMaxGroup tensors, one grid-stride walk over
 // their concatenated 8-element chunks (end[i]: running chunk totals).
 struct CvtGroup {
@@ -95,6 +137,19 @@ cudaError_t launch_cvt_x16(const float *X, void *Xh, int64_t M, int64_t K, DevCt
     const float4 *x4 = reinterpret_cast<const float4 *>(X);
     uint4 *h = static_cast<uint4 *>(Xh);
     return cudaLaunchKernelEx(&cfg, cvt_x16_kernel, x4, h, n_chunks, ctl);
+}
+
+cudaError_t launch_cvt_x16_lean(const float *X, void *Xh, int64_t M, int64_t K, DevCtl *ctl,
+                                cudaStream_t s) {
+    const int64_t n_chunks = M * K / 8;
+    if (n_chunks == 0) return cudaSuccess;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t blocks = std::min<int64_t>(sms, (n_chunks + kLeanThreads - 1) / kLeanThreads);
+    cvt_x16_lean_kernel<<<static_cast<unsigned>(blocks), kLeanThreads, 0, s>>>(
+        reinterpret_cast<const float4 *>(X), static_cast<uint4 *>(Xh), n_chunks, ctl);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_cvt_x16_group(const float *const *X, void *const *Xh, const int64_t *K,
