@@ -516,7 +516,7 @@ rt_status run_list(const BlockProj *p, int count, int64_t M, int path, void *str
         const int m = static_cast<int>(M), n = static_cast<int>(q.N), k = static_cast<int>(q.K);
         e = kern_of[i] == RT_KERNEL_TC_X_RESIDENT
                 ? rtq::launch_xs(q.fmt, slice[i], q.W, q.S, q.bias, q.Y, m, n, k, ctl, s)
-                : rtq::launch_ws(q.fmt, slice[i], q.W, q.S, q.bias, q.Y, m, n, k, ctl, s);
+                : rtq::launch_ws(q.fmt, slice[i], q.W, q.S, q.bias, q.Y, m, n, k, ctl, s, true);
         if (e != cudaSuccess) return RT_ERR_CUDA;
     }
     return RT_OK;

@@ -163,8 +163,12 @@ cudaError_t launch_xp(int fmt, const float *X, const void *Wq, const void *S, co
 bool ws_supported(int fmt, int M, int N, int K);
 // Activation rows per weight-streamed tile for this shape and SM count.
 int ws_tile_rows(int M, int N, int sms);
+// x_ready: Xh was complete before this launch (a pre-pass on another stream,
+// joined by an event), so the activation loads need not wait for the previous
+// grid in the stream; the grid still completes only after that grid has.
 cudaError_t launch_ws(int fmt, const void *Xh, const void *Wq, const void *S, const float *bias,
-                      float *Y, int M, int N, int K, DevCtl *ctl, cudaStream_t s);
+                      float *Y, int M, int N, int K, DevCtl *ctl, cudaStream_t s,
+                      bool x_ready = false);
 
 // tcgen05, a list of independent projections with the same M (1..128) in
 // persistent launches that stream every projection's weights back to back;

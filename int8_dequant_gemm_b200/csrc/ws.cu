@@ -107,7 +107,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
                     const __grid_constant__ CUtensorMap s_map,
                     const __grid_constant__ CUtensorMap x_map, const float *__restrict__ S8,
                     const float *__restrict__ bias, float *__restrict__ Y, int M, int N, int K,
-                    int bn, int n_o_tiles, int n_tiles, DevCtl *ctl) {
+                    int bn, int n_o_tiles, int n_tiles, int x_ready, DevCtl *ctl) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_addr(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;
@@ -227,7 +227,10 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     } else if (warp == kXTmaWarp) {
         // ============================================================ activation TMA
         if (lane == 0) {
-            pdl_wait_prior_grid();     // the 16-bit activations come from the pre-pass
+            // the 16-bit activations come from the pre-pass, the previous
+            // grid in the stream -- unless they were complete before this
+            // launch (x_ready), which then starts at once
+            if (!x_ready) pdl_wait_prior_grid();
             int j = 0;
             for (int t = blockIdx.x; t < n_tiles && ok; t += G) {
                 const int m0 = (t / n_o_tiles) * bn;
@@ -441,6 +444,10 @@ __global__ void __launch_bounds__(kWsThreads, 1)
         }
     }
     if (!ok) atomicOr(&ctl->status, 1u << kStatusTimeout);
+    // x_ready: this grid completes only after the previous grid in the stream
+    // has, as it would had it waited before its activation loads, so a later
+    // launch that waits for this grid waits for that one too
+    if (x_ready && threadIdx.x == 0) pdl_wait_prior_grid();
     tc_fence_before_sync();
     __syncthreads();
     if (warp == 0) {
@@ -451,7 +458,8 @@ __global__ void __launch_bounds__(kWsThreads, 1)
 
 template <int FMT>
 cudaError_t launch_ws_fmt(const void *Xh, const void *Wq, const void *S, const float *bias,
-                          float *Y, int M, int N, int K, DevCtl *ctl, cudaStream_t st) {
+                          float *Y, int M, int N, int K, DevCtl *ctl, cudaStream_t st,
+                          bool x_ready) {
     static std::atomic<bool> attr_done[kMaxDevices];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -491,7 +499,7 @@ cudaError_t launch_ws_fmt(const void *Xh, const void *Wq, const void *S, const f
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, ws_qgemm_kernel<FMT>, w_map, s_map, x_map,
                               static_cast<const float *>(S), bias, Y, M, N, K, bn, n_o, tiles,
-                              ctl);
+                              x_ready ? 1 : 0, ctl);
 }
 
 }  // namespace
@@ -529,10 +537,10 @@ bool ws_supported(int fmt, int M, int N, int K) {
 }
 
 cudaError_t launch_ws(int fmt, const void *Xh, const void *Wq, const void *S, const float *bias,
-                      float *Y, int M, int N, int K, DevCtl *ctl, cudaStream_t s) {
-    if (fmt == kFmtQ4) return launch_ws_fmt<kFmtQ4>(Xh, Wq, S, bias, Y, M, N, K, ctl, s);
-    if (fmt == kFmtQ8) return launch_ws_fmt<kFmtQ8>(Xh, Wq, S, bias, Y, M, N, K, ctl, s);
-    return launch_ws_fmt<kFmtE4M3>(Xh, Wq, S, bias, Y, M, N, K, ctl, s);
+                      float *Y, int M, int N, int K, DevCtl *ctl, cudaStream_t s, bool x_ready) {
+    if (fmt == kFmtQ4) return launch_ws_fmt<kFmtQ4>(Xh, Wq, S, bias, Y, M, N, K, ctl, s, x_ready);
+    if (fmt == kFmtQ8) return launch_ws_fmt<kFmtQ8>(Xh, Wq, S, bias, Y, M, N, K, ctl, s, x_ready);
+    return launch_ws_fmt<kFmtE4M3>(Xh, Wq, S, bias, Y, M, N, K, ctl, s, x_ready);
 }
 
 }  // namespace rtq
