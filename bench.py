@@ -887,6 +887,15 @@ def run_gpu(args, rank, world, local_rank):
         fused_block = L.rt_qblock_fused_fmt(ctypes.byref(block_args[0][0]), M, 0) == 1
     else:
         fused_block = full_block and rtq.block_fused(M, wl.D_MODEL, wl.D_FF) == 1
+    # the block driver's route (rt_qblock_route): which launches a block takes
+    route_names = []
+    if full_block:
+        c0 = block_args[0][0]
+        bits = (L.rt_qblock_route_fmt if per_fmt else L.rt_qblock_route)(ctypes.byref(c0), M, 0)
+        route_names = [n for b, n in ((rtq.ROUTE_GROUPED_SMALL_M, "grouped_small_m"),
+                                      (rtq.ROUTE_X_RESIDENT_GROUP, "x_resident_group"),
+                                      (rtq.ROUTE_SIDE_PREPASS, "side_stream_prepass"))
+                       if bits >= 0 and bits & b] or ["one_call_per_projection"]
     grouped = []
     if full_block and not fused_block:
         grouped = [n for n in projs if plan_of(n) == "tc_x_resident"]
@@ -1149,7 +1158,7 @@ def run_gpu(args, rank, world, local_rank):
                        "parallelism": f"replicas{world}" if world > 1 else "single",
                        "l2": f"inputs > L2 ({(bytes_act + wbytes) / 1e9:.2f} GB streamed per "
                              f"step), no flush",
-                       "issue": issue},
+                       "issue": issue, "block_route": route_names},
             "weight_gbs": world * wbytes / (ms_per_step * 1e-3) / 1e9,
             "call_us": kern_us, "calls_sum_ms_per_step": calls_sum_ms,
             "clocks": clocks, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,

@@ -362,6 +362,29 @@ rt_status rt_qblock_project(const rt_qblock *blk, int64_t M,
  * Host-only; touches no device. */
 int rt_qblock_fused(int64_t M, int64_t d_model, int64_t d_ff, int path);
 
+/* How rt_qblock_project (rt_qblock_route) or rt_qblock_project_fmt
+ * (rt_qblock_route_fmt) runs this block at M rows on `path`: the sum of
+ *   RT_ROUTE_GROUPED_SMALL_M   one grouped launch of the weight-stationary
+ *                              kernel (1 <= M <= 128 on the tensor-core path);
+ *   RT_ROUTE_X_RESIDENT_GROUP  the projections that take
+ *                              RT_KERNEL_TC_X_RESIDENT share one pre-pass
+ *                              launch and one launch of that kernel;
+ *   RT_ROUTE_SIDE_PREPASS      the other projections' pre-passes run on a
+ *                              second stream beside that launch (when the
+ *                              pre-pass's blocks fit on the SMs beside its
+ *                              CTAs), and their GEMMs start without waiting
+ *                              for it;
+ * 0 if the projections run one call after another; -1 if the block, M or
+ * path is rejected.  Reads the weights' scale pointers (alignment) and no
+ * device memory; RT_ROUTE_SIDE_PREPASS asks the CUDA runtime for the
+ * kernels' register counts, so it is never set without a device. */
+typedef enum rt_route {
+    RT_ROUTE_GROUPED_SMALL_M = 1,
+    RT_ROUTE_X_RESIDENT_GROUP = 2,
+    RT_ROUTE_SIDE_PREPASS = 4
+} rt_route;
+int rt_qblock_route(const rt_qblock *blk, int64_t M, int path);
+
 /*
  * The same block projection set with each projection's format chosen by the
  * caller, e.g. the int8 card's all-int8 (Q8_0-style) recipe ("RT-J -- int8
@@ -401,6 +424,7 @@ rt_status rt_qblock_project_fmt(const rt_qblock_fmt *blk, int64_t M,
 
 /* As rt_qblock_fused for a block with the formats of `blk` (host-only). */
 int rt_qblock_fused_fmt(const rt_qblock_fmt *blk, int64_t M, int path);
+int rt_qblock_route_fmt(const rt_qblock_fmt *blk, int64_t M, int path);
 
 /*
  * Host-side quantizers (HOST pointers, caller-allocated outputs, synchronous,

@@ -24,7 +24,8 @@ __all__ = [
     "qgemm_noalloc", "plan", "block_fused", "workspace_bytes", "debug_inject",
     "qgemm_batch", "batch_plan", "Proj", "QBlockFmt", "qblock_project_fmt", "block_fused_fmt",
     "gemm_e4m3", "quantize_e4m3", "dequant_e4m3_f32", "dequant_e4m3_f16", "FMT_E4M3",
-    "Checkpoint", "qgemm",
+    "Checkpoint", "qgemm", "block_route", "ROUTE_GROUPED_SMALL_M", "ROUTE_X_RESIDENT_GROUP",
+    "ROUTE_SIDE_PREPASS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -132,6 +133,10 @@ def lib() -> ctypes.CDLL:
                                         _p, _p, _i32, _p]
     L.rt_qblock_fused_fmt.restype = _i32
     L.rt_qblock_fused_fmt.argtypes = [ctypes.POINTER(_QBlockFmtC), _i64, _i32]
+    L.rt_qblock_route.restype = _i32
+    L.rt_qblock_route.argtypes = [ctypes.POINTER(_QBlockC), _i64, _i32]
+    L.rt_qblock_route_fmt.restype = _i32
+    L.rt_qblock_route_fmt.argtypes = [ctypes.POINTER(_QBlockFmtC), _i64, _i32]
     L.rt_quantize_q4_g32.restype = _i32
     L.rt_quantize_q4_g32.argtypes = [_p, _i64, _i64, _i32, _p, _p]
     L.rt_quantize_q8_row.restype = _i32
@@ -212,6 +217,14 @@ def rt_qblock_project_fmt(blk, M, X_qkvg, X_o, X_ffn, X_w2, Y_qkvg, Y_o, Y_13, Y
 
 def rt_qblock_fused_fmt(blk, M, path) -> int:
     return lib().rt_qblock_fused_fmt(ctypes.byref(blk), M, path)
+
+
+def rt_qblock_route(blk, M, path) -> int:
+    return lib().rt_qblock_route(ctypes.byref(blk), M, path)
+
+
+def rt_qblock_route_fmt(blk, M, path) -> int:
+    return lib().rt_qblock_route_fmt(ctypes.byref(blk), M, path)
 
 
 def rt_quantize_q4_g32(W, N, K, n_grid, Wq, scale_min) -> int:
@@ -567,6 +580,18 @@ def qblock_project_fmt(block: QBlockFmt, X_qkvg, X_o, X_ffn, X_w2, Y_qkvg, Y_o, 
 
 def block_fused_fmt(block: QBlockFmt, M: int, path="auto") -> int:
     return int(rt_qblock_fused_fmt(block.as_c(), M, _path(path)))
+
+
+# rt_route bits (see rt_qblock_route in rtq.h)
+ROUTE_GROUPED_SMALL_M, ROUTE_X_RESIDENT_GROUP, ROUTE_SIDE_PREPASS = 1, 2, 4
+
+
+def block_route(block, M: int, path="auto") -> int:
+    """How the block driver runs `block` (a QBlock or QBlockFmt) at M rows: a
+    sum of the ROUTE_* bits, 0 for one call per projection, -1 if rejected."""
+    if isinstance(block, QBlockFmt):
+        return int(rt_qblock_route_fmt(block.as_c(), M, _path(path)))
+    return int(rt_qblock_route(block.as_c(), M, _path(path)))
 
 
 def quantize_q4_g32(W: np.ndarray, n_grid: int = 21):

@@ -389,13 +389,23 @@ struct BlockProj {
 // beside its CTAs), each into a slice of its own, and the stream waits for
 // them before their GEMM launches, which come after the chunks.  The
 // workspace is sized once, before anything is queued.
-rt_status run_list(const BlockProj *p, int count, int64_t M, int path, void *stream) {
-    if (M == 0) return RT_OK;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    std::vector<int> chunk_of(static_cast<size_t>(count), -1), kern_of(static_cast<size_t>(count));
+// How run_list runs a list: its chunks (list indices that share one
+// activation-resident launch), the kernel of every entry, the entries outside
+// the chunks that stage their activations, the workspace they need, and
+// whether the lean pre-pass fits beside the first chunk's CTAs.
+struct ListPlan {
+    std::vector<int> chunk_of, kern_of;
     std::vector<std::vector<int>> chunks;
-    std::vector<int> open;
+    std::vector<int> staged;
     int64_t chunk_need = 0, single_need = 0, staged_sum = 0;
+    bool side_fits = false;
+};
+
+ListPlan plan_list(const BlockProj *p, int count, int64_t M, int path) {
+    ListPlan L;
+    L.chunk_of.assign(static_cast<size_t>(count), -1);
+    L.kern_of.assign(static_cast<size_t>(count), 0);
+    std::vector<int> open;
     auto close = [&]() {
         if (open.size() >= 2) {
             std::vector<rtq::XsInput> in;
@@ -407,9 +417,9 @@ rt_status run_list(const BlockProj *p, int count, int64_t M, int path, void *str
             }
             if (rtq::xs_group_supported(in.data(), static_cast<int>(in.size()),
                                         static_cast<int>(M))) {
-                for (int i : open) chunk_of[i] = static_cast<int>(chunks.size());
-                chunks.push_back(open);
-                chunk_need = std::max(chunk_need, bytes);
+                for (int i : open) L.chunk_of[i] = static_cast<int>(L.chunks.size());
+                L.chunks.push_back(open);
+                L.chunk_need = std::max(L.chunk_need, bytes);
             }
         }
         open.clear();
@@ -418,7 +428,7 @@ rt_status run_list(const BlockProj *p, int count, int64_t M, int path, void *str
         const BlockProj &q = p[i];
         const int kern = kernel_for_scales(
             pick_kernel(q.fmt, M, q.N, q.K, pick_path(q.fmt, M, q.K, path)), q.fmt, q.S);
-        kern_of[i] = kern;
+        L.kern_of[i] = kern;
         if (kern == RT_KERNEL_TC_X_RESIDENT) {
             open.push_back(i);
             if (static_cast<int>(open.size()) == rtq::kMaxGroup) close();
@@ -426,15 +436,40 @@ rt_status run_list(const BlockProj *p, int count, int64_t M, int path, void *str
     }
     close();
     // calls outside the chunks that stage their activations
-    std::vector<int> staged;
     for (int i = 0; i < count; ++i) {
-        if (chunk_of[i] >= 0) continue;
-        if (kern_of[i] == RT_KERNEL_TC_X_RESIDENT || kern_of[i] == RT_KERNEL_TC_W_STREAMED) {
-            staged.push_back(i);
-            single_need = std::max(single_need, M * p[i].K * 2);
-            staged_sum += M * p[i].K * 2;
+        if (L.chunk_of[i] >= 0) continue;
+        if (L.kern_of[i] == RT_KERNEL_TC_X_RESIDENT || L.kern_of[i] == RT_KERNEL_TC_W_STREAMED) {
+            L.staged.push_back(i);
+            L.single_need = std::max(L.single_need, M * p[i].K * 2);
+            L.staged_sum += M * p[i].K * 2;
         }
     }
+    // the side stream's pre-passes must fit beside the first chunk's CTAs,
+    // or they would hold SMs the chunk's persistent CTAs wait for
+    if (!L.staged.empty() && !L.chunks.empty()) {
+        rtq::XsInput in0[rtq::kMaxGroup];
+        const std::vector<int> &c0 = L.chunks.front();
+        for (size_t g = 0; g < c0.size(); ++g) {
+            const BlockProj &q = p[c0[g]];
+            in0[g] = {q.fmt, nullptr, q.W, q.S, q.bias, q.Y, static_cast<int>(q.N),
+                      static_cast<int>(q.K)};
+        }
+        int lt = 0, lr = 0;
+        L.side_fits = rtq::cvt_x16_lean_shape(&lt, &lr) &&
+                      rtq::xs_group_leaves_room(in0, static_cast<int>(c0.size()),
+                                                static_cast<int>(M), lt, lr);
+    }
+    return L;
+}
+
+rt_status run_list(const BlockProj *p, int count, int64_t M, int path, void *stream) {
+    if (M == 0) return RT_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const ListPlan L = plan_list(p, count, M, path);
+    const std::vector<int> &chunk_of = L.chunk_of, &kern_of = L.kern_of, &staged = L.staged;
+    const std::vector<std::vector<int>> &chunks = L.chunks;
+    const int64_t chunk_need = L.chunk_need, single_need = L.single_need;
+    const int64_t staged_sum = L.staged_sum;
     rt_status st;
     if (chunks.empty()) {
         for (int i = 0; i < count; ++i) {
@@ -448,7 +483,7 @@ rt_status run_list(const BlockProj *p, int count, int64_t M, int path, void *str
     void *ws = nullptr;
     DevCtl *ctl = nullptr;
     SideStream side = {};
-    const bool overlap = !staged.empty() && side_stream(s, &side);
+    const bool overlap = L.side_fits && side_stream(s, &side);
     const int64_t need = overlap ? chunk_need + staged_sum : std::max(chunk_need, single_need);
     if ((st = workspace(s, static_cast<size_t>(need), &ws)) != RT_OK ||
         (st = ctl_block(&ctl)) != RT_OK)
@@ -586,6 +621,21 @@ rt_status block_run(const BlockProj p[4], int64_t M, int64_t d, int64_t f, int p
 // The int4 card's mixed recipe: qkvg and w13 in q4, wo and w2 in q8.
 constexpr int kMixedFmt[4] = {4, 8, 4, 8};
 
+// rt_qblock_route / rt_qblock_route_fmt: the route bits of a block.
+int block_route_bits(const BlockProj p[4], int64_t M, int64_t d, int64_t f, int path) {
+    int fmts[4];
+    for (int i = 0; i < 4; ++i) fmts[i] = p[i].fmt;
+    const int r = block_route(fmts, M, d, f, path);
+    if (r < 0) return -1;
+    if (r == 1) return RT_ROUTE_GROUPED_SMALL_M;
+    if (M <= 0) return 0;
+    const ListPlan L = plan_list(p, 4, M, path);
+    int bits = 0;
+    if (!L.chunks.empty()) bits |= RT_ROUTE_X_RESIDENT_GROUP;
+    if (!L.chunks.empty() && L.side_fits) bits |= RT_ROUTE_SIDE_PREPASS;
+    return bits;
+}
+
 }  // namespace
 
 extern "C" {
@@ -605,6 +655,29 @@ rt_status rt_qblock_project(const rt_qblock *blk, int64_t M, const float *X_qkvg
                             {4, X_ffn, blk->w13, blk->w13_sm, nullptr, Y_13, 2 * f, d},
                             {8, X_w2, blk->w2, blk->w2_s, nullptr, Y_2, d, f}};
     return block_run(p, M, d, f, path, stream);
+}
+
+int rt_qblock_route(const rt_qblock *blk, int64_t M, int path) {
+    if (!blk || blk->d_model < 1 || blk->d_ff < 1 || M < 0 || M > kMaxDim) return -1;
+    const int64_t d = blk->d_model, f = blk->d_ff;
+    const BlockProj p[4] = {{4, nullptr, blk->qkvg, blk->qkvg_sm, nullptr, nullptr, 4 * d, d},
+                            {8, nullptr, blk->wo, blk->wo_s, nullptr, nullptr, d, d},
+                            {4, nullptr, blk->w13, blk->w13_sm, nullptr, nullptr, 2 * f, d},
+                            {8, nullptr, blk->w2, blk->w2_s, nullptr, nullptr, d, f}};
+    return block_route_bits(p, M, d, f, path);
+}
+
+int rt_qblock_route_fmt(const rt_qblock_fmt *blk, int64_t M, int path) {
+    if (!blk || blk->d_model < 1 || blk->d_ff < 1 || M < 0 || M > kMaxDim) return -1;
+    const rt_qweight *w[4] = {&blk->qkvg, &blk->wo, &blk->w13, &blk->w2};
+    for (int i = 0; i < 4; ++i)
+        if (w[i]->reserved != 0 || !rtq::fmt_valid(w[i]->fmt)) return -1;
+    const int64_t d = blk->d_model, f = blk->d_ff;
+    const BlockProj p[4] = {{w[0]->fmt, nullptr, w[0]->Wq, w[0]->scales, w[0]->bias, nullptr, 4 * d, d},
+                            {w[1]->fmt, nullptr, w[1]->Wq, w[1]->scales, w[1]->bias, nullptr, d, d},
+                            {w[2]->fmt, nullptr, w[2]->Wq, w[2]->scales, w[2]->bias, nullptr, 2 * f, d},
+                            {w[3]->fmt, nullptr, w[3]->Wq, w[3]->scales, w[3]->bias, nullptr, d, f}};
+    return block_route_bits(p, M, d, f, path);
 }
 
 int rt_qblock_fused_fmt(const rt_qblock_fmt *blk, int64_t M, int path) {

@@ -93,6 +93,9 @@ cudaError_t launch_cvt_x16(const float *X, void *Xh, int64_t M, int64_t K, DevCt
                            cudaStream_t s);
 cudaError_t launch_cvt_x16_lean(const float *X, void *Xh, int64_t M, int64_t K, DevCtl *ctl,
                                 cudaStream_t s);
+// The lean pre-pass's block: threads and registers a thread; false if the
+// runtime cannot report them.
+bool cvt_x16_lean_shape(int *threads, int *regs);
 cudaError_t launch_cvt_x16_group(const float *const *X, void *const *Xh, const int64_t *K,
                                  int count, int64_t M, DevCtl *ctl, cudaStream_t s);
 
@@ -112,6 +115,10 @@ struct XsInput {
 };
 bool xs_supported(int M, int N, int K);
 bool xs_group_supported(const XsInput *in, int count, int M);
+// Whether a block of `threads` threads of `regs` registers and no shared
+// memory fits on an SM beside one CTA of the build launch_xs_group runs for
+// this list (per sub-partition registers, shared memory, threads).
+bool xs_group_leaves_room(const XsInput *in, int count, int M, int threads, int regs);
 cudaError_t launch_xs(int fmt, const void *Xh, const void *Wq, const void *S, const float *bias,
                       float *Y, int M, int N, int K, DevCtl *ctl, cudaStream_t s);
 cudaError_t launch_xs_group(const XsInput *in, int count, int M, DevCtl *ctl, cudaStream_t s);

@@ -152,6 +152,17 @@ cudaError_t launch_cvt_x16_lean(const float *X, void *Xh, int64_t M, int64_t K, 
     return cudaGetLastError();
 }
 
+bool cvt_x16_lean_shape(int *threads, int *regs) {
+    cudaFuncAttributes fa = {};
+    if (cudaFuncGetAttributes(&fa, cvt_x16_lean_kernel) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    *threads = kLeanThreads;
+    *regs = fa.numRegs;
+    return true;
+}
+
 cudaError_t launch_cvt_x16_group(const float *const *X, void *const *Xh, const int64_t *K,
                                  int count, int64_t M, DevCtl *ctl, cudaStream_t s) {
     if (count < 1 || count > kMaxGroup) return cudaErrorInvalidValue;

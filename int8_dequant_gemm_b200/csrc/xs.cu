@@ -661,6 +661,39 @@ bool xs_group_supported(const XsInput *in, int count, int M) {
     return true;
 }
 
+bool xs_group_leaves_room(const XsInput *in, int count, int M, int threads, int regs) {
+    if (!xs_group_supported(in, count, M) || threads < 1 || regs < 1) return false;
+    bool mixed = false;
+    int k_max = 0;
+    for (int i = 0; i < count; ++i) {
+        mixed = mixed || in[i].fmt != in[0].fmt;
+        k_max = std::max(k_max, in[i].K);
+    }
+    const int build = mixed ? kFmtMixed : in[0].fmt;
+    cudaFuncAttributes fa = {};
+    cudaError_t e = build == kFmtQ4    ? cudaFuncGetAttributes(&fa, xs_qgemm_kernel<kFmtQ4>)
+                    : build == kFmtQ8  ? cudaFuncGetAttributes(&fa, xs_qgemm_kernel<kFmtQ8>)
+                    : build == kFmtE4M3 ? cudaFuncGetAttributes(&fa, xs_qgemm_kernel<kFmtE4M3>)
+                                        : cudaFuncGetAttributes(&fa, xs_qgemm_kernel<kFmtMixed>);
+    int dev = 0, sm_regs = 0, sm_smem = 0, sm_threads = 0, reserved = 0;
+    if (e != cudaSuccess || cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sm_regs, cudaDevAttrMaxRegistersPerMultiprocessor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sm_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sm_threads, cudaDevAttrMaxThreadsPerMultiProcessor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    // registers are allocated per warp in units of 8 a thread and split
+    // between the SM's four sub-partitions, over which a block's warps spread
+    auto warp_regs = [](int r) { return (r + 7) / 8 * 8 * 32; };
+    const int own_warps = kXsThreads / 32, other_warps = (threads + 31) / 32;
+    const int per_sub = (own_warps + 3) / 4 * warp_regs(fa.numRegs) +
+                        (other_warps + 3) / 4 * warp_regs(regs);
+    const int smem = xs_layout(build, k_max).total + 1024 + 2 * reserved;
+    return per_sub <= sm_regs / 4 && smem <= sm_smem && kXsThreads + threads <= sm_threads;
+}
+
 cudaError_t launch_xs_group(const XsInput *in, int count, int M, DevCtl *ctl, cudaStream_t s) {
     if (!xs_group_supported(in, count, M)) return cudaErrorInvalidValue;
     bool mixed = false;

@@ -400,6 +400,36 @@ def test_block_fmt_validation_and_routes():
     assert run(C.byref(q8), 0, *X, *Y, 0, None) == RT_OK   # M == 0: no-op
 
 
+def test_block_route_bits():
+    """rt_qblock_route_fmt / rt_qblock_route: which launches a block takes.
+    Without a device the side-stream pre-pass bit is never set."""
+    GB = 1 << 30
+    import ctypes as C
+    route = rtq.lib().rt_qblock_route_fmt
+
+    def blk(fmts, d=512, f=2048, scale_off=0):
+        ws = [rtq._QWeightC(fm, 0, (2 + i) * GB, (6 + i) * GB + scale_off) for i, fm in enumerate(fmts)]
+        return rtq._QBlockFmtC(*ws, d, f)
+    mixed, q8 = blk((4, 8, 4, 8)), blk((8, 8, 8, 8))
+    G, XR = rtq.ROUTE_GROUPED_SMALL_M, rtq.ROUTE_X_RESIDENT_GROUP
+    assert route(C.byref(mixed), 80, 0) == G                 # one grouped launch
+    assert route(C.byref(q8), 4096, 0) == XR                 # qkvg, wo, w13 share a launch
+    assert route(C.byref(mixed), 4096, 0) == XR
+    assert route(C.byref(mixed), 129, 0) == XR
+    assert route(C.byref(mixed), 16384, 0) == 0              # CTA-pair kernels, one call each
+    assert route(C.byref(mixed), 4096, 1) == 0               # SIMT path: one call each
+    assert route(C.byref(mixed), 4096, 2) == XR              # tensor cores forced
+    # q4 scales only 4-byte aligned: qkvg and w13 leave the TMA kernels, wo alone stays
+    assert route(C.byref(blk((4, 8, 4, 8), scale_off=4)), 4096, 0) == 0
+    assert route(C.byref(blk((8, 8, 5, 8))), 4096, 0) == -1  # unknown format
+    assert route(C.byref(mixed), -1, 0) == -1
+    assert route(None, 80, 0) == -1
+    # rt_qblock_route (mixed recipe) agrees with the per-format form
+    mq = rtq._QBlockC(2 * GB, 6 * GB, 3 * GB, 7 * GB, 4 * GB, 8 * GB, 5 * GB, 9 * GB, 512, 2048)
+    for M in (80, 129, 4096, 16384):
+        assert rtq.lib().rt_qblock_route(C.byref(mq), M, 0) == route(C.byref(mixed), M, 0)
+
+
 # --------------------------------------------------------------- FP8 E4M3
 @pytest.mark.parametrize("outliers", [False, True])
 def test_e4m3_quantizer_matches_oracle_bit_for_bit(outliers):

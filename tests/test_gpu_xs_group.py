@@ -202,3 +202,23 @@ def test_block_driver_groups_the_x_resident_projections(rtq_lib, M, d_model, d_f
     assert rtq_lib.block_fused(M, d_model, d_ff, "auto") == 0
     rtq_lib.qblock_project(blk, *(p.X for p in projs), *(p.Y for p in projs))
     check(rtq_lib, entries, projs, flat, mask)
+
+
+def test_default_block_takes_the_side_stream_pre_pass(rtq_lib):
+    """RT-J's block at M = 4096 (the benchmark's configuration), mixed and
+    all-int8 recipes: qkvg, wo and w13 share one launch, and w2's pre-pass
+    runs on the second stream -- its lean blocks fit on the SMs beside the
+    activation-resident CTAs (the check that would turn the overlap off if a
+    kernel's register count grew past the room)."""
+    M, d, f = 4096, 512, 2048
+    both = rtq_lib.ROUTE_X_RESIDENT_GROUP | rtq_lib.ROUTE_SIDE_PREPASS
+    e = _sized_block(d, f, 8, seed=9700)
+    ten = {n: (dev(e[n].q[0]), dev(e[n].q[1])) for n in e}
+    blk = rtq_lib.QBlock(*ten["qkvg"], *ten["wo"], *ten["w13"], *ten["w2"], d_model=d, d_ff=f)
+    assert rtq_lib.block_route(blk, M) == both
+    q8 = {n: oracle.quant_q8_row(wl.weights(N, K, 9800 + i))
+          for i, (n, N, K) in enumerate((("qkvg", 4 * d, d), ("wo", d, d), ("w13", 2 * f, d),
+                                         ("w2", d, f)))}
+    blk8 = rtq_lib.QBlockFmt(*((8, dev(q8[n][0]), dev(q8[n][1])) for n in ("qkvg", "wo", "w13", "w2")),
+                             d_model=d, d_ff=f)
+    assert rtq_lib.block_route(blk8, M) == both
