@@ -94,6 +94,10 @@ constexpr uint32_t kAccCols = 2 * kXsTileM;              // 2 accumulators x 192
 constexpr uint32_t kAStageCols = kAtomK;                 // 2 x 64 16-bit values per lane
 constexpr uint32_t kXsTmemCols = 512;                    // accumulators + A stages, pow2
 constexpr int kFmtMixed = 0;                             // build for launches that mix formats
+// Registers a thread, at most: 20 warps of 88 leave 2304 registers in each of
+// the SM's four sub-partitions, room for one 64-register warp of the side
+// stream's pre-pass (cvt_x16_lean_kernel) beside every CTA.
+constexpr int kXsMaxRegs = 88;
 
 static_assert(kAccCols + kAStages * kAStageCols <= kXsTmemCols, "TMEM budget");
 static_assert(kEpiCols % 32 == 0, "epilogue reads 32 columns at a time");
@@ -215,7 +219,7 @@ __device__ __forceinline__ void convert_half(int fmt, uint32_t raw, int r, int h
 }
 
 template <int FMT>
-__global__ void __launch_bounds__(kXsThreads, 1)
+__global__ void __maxnreg__(kXsMaxRegs)
     xs_qgemm_kernel(const __grid_constant__ XsParams P, int k_max, DevCtl *ctl) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_addr(smem_raw);
