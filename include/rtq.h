@@ -286,10 +286,17 @@ rt_status rt_qgemm_noalloc(int fmt, const float *X, const void *Wq, const void *
  * launch that rounds each one's X into its own slice of the stream's
  * workspace and one launch of the activation-resident kernel that walks all
  * their tiles, so they share one pipeline fill and drain and one wave tail.
- * A grouped entry gets the bits a single rt_qgemm call would give.
+ * A grouped entry gets the bits a single rt_qgemm call would give.  The other
+ * entries that stage X (RT_KERNEL_TC_W_STREAMED, or an activation-resident
+ * entry left alone) then have their pre-passes run on a second stream that the
+ * library keeps per (device, stream), beside the first shared launch, and
+ * their GEMMs follow the shared launches on `stream` (the two streams are
+ * joined with events, so stream order and graph capture hold; the second
+ * stream is created on the first such call outside a capture, and a call
+ * inside a capture before that runs the pre-passes in order on `stream`).
  * Workspace of such a list: the sum of M * K * 2 over the largest launch's
- * entries, or M * K * 2 of the largest other entry that stages X, whichever
- * is larger.  Results are those of the tensor-core path (<= 4e-3) and do
+ * entries plus M * K * 2 of every other entry that stages X (one slice
+ * each); without the second stream, the larger of the two parts.  Results are those of the tensor-core path (<= 4e-3) and do
  * not depend on the entries' order.
  */
 typedef struct rt_qproj {
@@ -333,9 +340,10 @@ int rt_qgemm_batch_plan(const rt_qproj *list, int count, int64_t M, int path);
  * w13, w2) on its per-entry route: the projections that take
  * RT_KERNEL_TC_X_RESIDENT (128 < M < 16384, K <= 512: qkvg, wo and w13 of
  * RT-J) share one pre-pass launch and one activation-resident launch, the
- * others run one call each, as rt_qgemm_q4/q8 would.  Workspace: the sum of
- * M * K * 2 over the projections that share the launch, or M * K * 2 of a
- * single call that stages X, whichever is larger (M = 4096 RT-J: 16 MiB).
+ * others run one call each, as rt_qgemm_q4/q8 would, their pre-passes on the
+ * second stream beside the shared launch (see rt_qgemm_batch).  Workspace:
+ * the sum of M * K * 2 over the projections that share the launch plus
+ * M * K * 2 of each other call that stages X (M = 4096 RT-J: 29.4 MB).
  *
  * Validation: each product as in rt_qgemm_q4/q8; in addition no output may
  * overlap another projection's output, activations, codes or scales
