@@ -289,7 +289,10 @@ def test_x_resident_long_runs_every_tile(rtq_lib):
 # the CTA-pair activation-resident kernel (from M = 16384): ragged M, an odd
 # number of 128-row weight tiles (the last pair's second CTA holds rows past
 # N), K from 128 to 512
-XP_SHAPES = [(16384, 640, 512), (16500, 700, 384), (17000, 256, 128), (16400, 1000, 256)]
+# ragged M (16500, 16390) and N (700, 1000, 130: rows of Y not a multiple of
+# 16 bytes)
+XP_SHAPES = [(16384, 640, 512), (16500, 700, 384), (17000, 256, 128), (16400, 1000, 256),
+             (16390, 130, 256)]
 
 
 @pytest.mark.parametrize("fmt", [4, 8])
