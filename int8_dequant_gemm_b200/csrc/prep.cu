@@ -9,6 +9,7 @@
 // kernel: 4 bytes read and 2 written per element.  An activation that is not
 // a finite fp16 value after rounding latches kStatusRange.
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "kernels.cuh"
@@ -153,13 +154,19 @@ cudaError_t launch_cvt_x16_lean(const float *X, void *Xh, int64_t M, int64_t K, 
 }
 
 bool cvt_x16_lean_shape(int *threads, int *regs) {
-    cudaFuncAttributes fa = {};
-    if (cudaFuncGetAttributes(&fa, cvt_x16_lean_kernel) != cudaSuccess) {
-        cudaGetLastError();
-        return false;
+    static std::atomic<int> regs_cache{0};   // looked up once
+    int r = regs_cache.load(std::memory_order_acquire);
+    if (r == 0) {
+        cudaFuncAttributes fa = {};
+        if (cudaFuncGetAttributes(&fa, cvt_x16_lean_kernel) != cudaSuccess) {
+            cudaGetLastError();
+            return false;
+        }
+        r = fa.numRegs;
+        regs_cache.store(r, std::memory_order_release);
     }
     *threads = kLeanThreads;
-    *regs = fa.numRegs;
+    *regs = r;
     return true;
 }
 

@@ -674,13 +674,27 @@ bool xs_group_leaves_room(const XsInput *in, int count, int M, int threads, int 
         k_max = std::max(k_max, in[i].K);
     }
     const int build = mixed ? kFmtMixed : in[0].fmt;
-    cudaFuncAttributes fa = {};
-    cudaError_t e = build == kFmtQ4    ? cudaFuncGetAttributes(&fa, xs_qgemm_kernel<kFmtQ4>)
-                    : build == kFmtQ8  ? cudaFuncGetAttributes(&fa, xs_qgemm_kernel<kFmtQ8>)
-                    : build == kFmtE4M3 ? cudaFuncGetAttributes(&fa, xs_qgemm_kernel<kFmtE4M3>)
-                                        : cudaFuncGetAttributes(&fa, xs_qgemm_kernel<kFmtMixed>);
+    // registers a thread of each build, looked up once (the same binary on
+    // every device)
+    static std::atomic<int> regs_of[4];
+    const int bi = build == kFmtQ4 ? 0 : build == kFmtQ8 ? 1 : build == kFmtE4M3 ? 2 : 3;
+    int own_regs = regs_of[bi].load(std::memory_order_acquire);
+    if (own_regs == 0) {
+        cudaFuncAttributes fa = {};
+        const cudaError_t e =
+            bi == 0   ? cudaFuncGetAttributes(&fa, xs_qgemm_kernel<kFmtQ4>)
+            : bi == 1 ? cudaFuncGetAttributes(&fa, xs_qgemm_kernel<kFmtQ8>)
+            : bi == 2 ? cudaFuncGetAttributes(&fa, xs_qgemm_kernel<kFmtE4M3>)
+                      : cudaFuncGetAttributes(&fa, xs_qgemm_kernel<kFmtMixed>);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return false;
+        }
+        own_regs = fa.numRegs;
+        regs_of[bi].store(own_regs, std::memory_order_release);
+    }
     int dev = 0, sm_regs = 0, sm_smem = 0, sm_threads = 0, reserved = 0;
-    if (e != cudaSuccess || cudaGetDevice(&dev) != cudaSuccess ||
+    if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sm_regs, cudaDevAttrMaxRegistersPerMultiprocessor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sm_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sm_threads, cudaDevAttrMaxThreadsPerMultiProcessor, dev) != cudaSuccess ||
@@ -692,7 +706,7 @@ bool xs_group_leaves_room(const XsInput *in, int count, int M, int threads, int 
     // between the SM's four sub-partitions, over which a block's warps spread
     auto warp_regs = [](int r) { return (r + 7) / 8 * 8 * 32; };
     const int own_warps = kXsThreads / 32, other_warps = (threads + 31) / 32;
-    const int per_sub = (own_warps + 3) / 4 * warp_regs(fa.numRegs) +
+    const int per_sub = (own_warps + 3) / 4 * warp_regs(own_regs) +
                         (other_warps + 3) / 4 * warp_regs(regs);
     const int smem = xs_layout(build, k_max).total + 1024 + 2 * reserved;
     return per_sub <= sm_regs / 4 && smem <= sm_smem && kXsThreads + threads <= sm_threads;
